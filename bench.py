@@ -1,0 +1,451 @@
+"""Benchmark of the gated delta rule library on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload prefill4k|prefill256k|varlen] [--path auto|tensor|simt]
+                    [--no-decode] [--no-cpu-baseline]
+
+One step = one chunked prefill (gdn_chunk_fwd: L2-norm prologue, gate cumsum,
+intra-chunk products, triangular solve, state carry, RMSNorm x sigmoid(g)
+epilogue) over one batch of the workload (default: B=1, T=4096, 16 QK / 48
+value heads, d=128, bf16).  The JSON line also carries the decode step
+(gdn_decode_step, 256 sequences x 64 steps, in place) as a separate object
+with its own timing, roofline and clocks.
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own
+independent batch (weak scaling; sequences and heads are independent, so the
+data path has no collective).  Timing is on the device with CUDA events, the
+reported time is the max over ranks.
+
+``--impl reference`` times the fp64 CPU oracle (the only other program that
+computes this operation here) on a bounded sample of the same workload, on
+rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "GDN prefill tokens/s (48 heads, d=128) and decode state GB/s; % of roofline"
+H_QK, H_V, D = 16, 48, 128
+CHUNK = 64
+L2_BYTES = 126 * 2 ** 20
+
+
+def flops_per_token(Hqk=H_QK, Hv=H_V, d=D, C=CHUNK):
+    """Counted MMA FLOPs per token at the canonical chunk of 64:
+    per value head 6 d^2 + 6 C d + C^2 / 3, per QK head 4 C d."""
+    return Hv * (6 * d * d + 6 * C * d + C * C / 3.0) + Hqk * 4 * C * d
+
+
+def prefill_bytes(T, n_seq, epilogue=True, init_state=True, in_bytes=2, Hqk=H_QK, Hv=H_V, d=D):
+    """Compulsory HBM bytes of one prefill: every input read once, y and the
+    final state written once."""
+    per_tok = 2 * Hqk * d * in_bytes + Hv * d * in_bytes + Hv * d * in_bytes + Hv * 8
+    if epilogue:
+        per_tok += Hv * d * in_bytes
+    state = n_seq * Hv * d * d * 4
+    return per_tok * T + state * (2 if init_state else 1) + (d * 4 if epilogue else 0)
+
+
+def decode_bytes(N, Hqk=H_QK, Hv=H_V, d=D, in_bytes=2):
+    """Compulsory HBM bytes of one decode step: the state read and written
+    once, plus q/k/v, gates and y."""
+    return N * (2 * Hv * d * d * 4 + 2 * Hqk * d * in_bytes + 2 * Hv * d * in_bytes + Hv * 8)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm_gbs=float(d["hbm_gbs"]), bf16_tflops=float(d["bf16_tflops"]),
+                    bf16_tflops_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0,
+                source="fallback")
+
+
+def kernel_traffic(kernel_key):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel
+    source it was taken on is unchanged; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p)).get(kernel_key)
+        if not d:
+            return None
+        src = os.path.join(ROOT, d["source"])
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        return float(d["bytes_per_launch"]) if sha == d["source_sha"] else None
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during a timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group(
+            "nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+
+
+def timed_steps(fn, steps, warmup, world, flush=None, stream=None):
+    """Warm up, then time exactly `steps` calls with CUDA events on `stream`
+    (flush between steps outside the events).  Returns per-step ms list."""
+    stream = stream or torch.cuda.current_stream()
+    for _ in range(warmup):
+        fn()
+    barrier(world)
+    times = []
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for i in range(steps):
+        if flush is not None:
+            flush()
+        ev[i][0].record(stream)
+        fn()
+        ev[i][1].record(stream)
+    barrier(world)
+    for a, b in ev:
+        times.append(a.elapsed_time(b))
+    return times
+
+
+def cpu_baseline(w, target_s=12.0):
+    """The fp64 oracle, as it stands, on a bounded prefix of the workload's
+    first sequence (all heads), sized for about `target_s` seconds."""
+    import oracle
+    cores = oracle.max_threads()
+
+    def run(T):
+        sub = _prefix(w, T)
+        t0 = time.perf_counter()
+        oracle.recurrence(sub["q"], sub["k"], sub["v"], sub["log_alpha"], sub["beta"],
+                          g=sub["g"], norm_w=sub["norm_w"], initial_state=sub["s0"])
+        return time.perf_counter() - t0
+
+    T_cal = 64
+    dt = run(T_cal)
+    T_s = int(max(64, min(w.total_T, T_cal * target_s / max(dt, 1e-6))))
+    T_s = min(T_s, int(w.cu_seqlens[1].item()))
+    dt = run(T_s)
+    return {"value": T_s / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": "first %d tokens of sequence 0, all %d value heads, fp64, OpenMP over "
+                      "value heads (%.1f s)" % (T_s, w.v.shape[1], dt)}
+
+
+def _prefix(w, T):
+    cpu = lambda x: None if x is None else x[:T].to("cpu", torch.float32)
+    return dict(q=cpu(w.q), k=cpu(w.k), v=cpu(w.v), log_alpha=cpu(w.log_alpha),
+                beta=cpu(w.beta), g=cpu(w.g),
+                norm_w=None if w.norm_w is None else w.norm_w.to("cpu", torch.float32),
+                s0=None if w.initial_state is None else w.initial_state[:1].to("cpu", torch.float32))
+
+
+def make_workload(name, rank):
+    from gated_deltanet_scan_chunked_b200 import inputs
+    w = inputs.workload(name, device="cuda")
+    if rank:
+        # an independent batch per rank: same recipe, another seed
+        seed = inputs.SEEDS[name] + 100 * rank
+        lengths = w.meta["lengths"]
+        w = inputs.make_prefill(lengths, H_QK, H_V, D, D, seed=seed,
+                                s0_std=0.01 if w.initial_state is not None else 0.0,
+                                device="cuda")
+    return w
+
+
+def run_reference(args, world, rank):
+    """The oracle arm: rank 0 only, no process group, no GPU kernels of ours."""
+    if rank != 0:
+        return
+    torch.cuda.set_device(0)
+    w = make_workload(args.workload, 0)
+    times = []
+    base = None
+    per_step = min(args.ref_seconds, 150.0 / (args.steps + args.warmup))
+    for i in range(args.warmup + args.steps):
+        b = cpu_baseline(w, target_s=per_step)
+        if i >= args.warmup:
+            times.append(b)
+        base = b
+    vals = [b["value"] for b in times] or [base["value"]]
+    v = statistics.median(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "global_batch": 1, "seq_len": w.total_T,
+                       "heads": "16 QK / 48 value", "d": D},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": base["cores"],
+                             "kind": "oracle", "sample": base["sample"]},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, world, rank, local):
+    from gated_deltanet_scan_chunked_b200 import gdn, gdn_chunk_fwd, gdn_decode_step, inputs
+    gdn.load()
+    peaks = load_peaks()
+    w = make_workload(args.workload, rank)
+    T, n_seq = w.total_T, w.n_seq
+    has_s0 = w.initial_state is not None
+    stream = torch.cuda.current_stream()
+    y = torch.empty_like(w.v)
+    fs = torch.empty((n_seq, H_V, D, D), dtype=torch.float32, device="cuda")
+    flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
+
+    def step():
+        gdn_chunk_fwd(w.q, w.k, w.v, w.log_alpha, w.beta, g=w.g, norm_w=w.norm_w,
+                      initial_state=w.initial_state, cu_seqlens=w.cu_seqlens, y=y,
+                      final_state=fs, path=args.path)
+
+    def flush():
+        flush_buf.zero_()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    times = timed_steps(step, args.steps, args.warmup, world, flush=flush, stream=stream)
+    clk = clocks.stop()
+    err = gdn.gdn_check_device_error()
+    if err != gdn.GDN_OK:
+        raise RuntimeError("device error: %s" % gdn.status_string(err))
+    ms = statistics.mean(times)
+    ms_max = max_over_ranks(ms, world)
+    value = world * T / (ms_max * 1e-3)
+
+    # roofline of the dominant (only) kernel of the step
+    nbytes = prefill_bytes(T, n_seq, epilogue=w.g is not None, init_state=has_s0)
+    nflops = flops_per_token() * T
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = nflops / (peaks["bf16_tflops"] * 1e12)
+    bound = "hbm" if t_hbm >= t_tc else "tensor"
+    if bound == "hbm":
+        achieved, peak, unit = nbytes / (ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s"
+    else:
+        achieved, peak, unit = nflops / (ms * 1e-3) / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+    kernel_key = "prefill_tc" if args.path in ("auto", "tensor") else "prefill_simt"
+    roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                "frac": achieved / peak, "traffic": kernel_traffic(kernel_key),
+                "peak_source": peaks["source"], "roofline_time_us": max(t_hbm, t_tc) * 1e6,
+                "frac_of_roofline_time": max(t_hbm, t_tc) / (ms * 1e-3),
+                "algorithmic_bytes": nbytes, "counted_flops": nflops,
+                "achieved_tflops": nflops / (ms * 1e-3) / 1e12,
+                "tensor_frac": nflops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"]}
+
+    # end to end through the public call with host buffers
+    e2e = None
+    if not args.no_e2e:
+        host = {}
+        for nm in ("q", "k", "v", "log_alpha", "beta", "g", "norm_w", "initial_state",
+                   "cu_seqlens"):
+            x = getattr(w, nm)
+            host[nm] = None if x is None else x.to("cpu").pin_memory()
+        dev = {nm: (None if x is None else torch.empty_like(x, device="cuda"))
+               for nm, x in host.items()}
+        y_h = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+        fs_h = torch.empty(fs.shape, dtype=fs.dtype).pin_memory()
+        h2d = sum(x.numel() * x.element_size() for x in host.values() if x is not None)
+        d2h = y_h.numel() * y_h.element_size() + fs_h.numel() * fs_h.element_size()
+
+        def e2e_step():
+            for nm, x in host.items():
+                if x is not None:
+                    dev[nm].copy_(x, non_blocking=True)
+            gdn_chunk_fwd(dev["q"], dev["k"], dev["v"], dev["log_alpha"], dev["beta"],
+                          g=dev["g"], norm_w=dev["norm_w"], initial_state=dev["initial_state"],
+                          cu_seqlens=dev["cu_seqlens"], y=y, final_state=fs, path=args.path)
+            y_h.copy_(y, non_blocking=True)
+            fs_h.copy_(fs, non_blocking=True)
+
+        et = timed_steps(e2e_step, max(3, args.steps // 2), 2, world, stream=stream)
+        ems = max_over_ranks(statistics.mean(et), world)
+        e2e = {"value": world * T / (ems * 1e-3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ems}
+        del dev, host
+
+    # the decode step, timed on its own (256 sequences x 64 steps, in place)
+    decode = None
+    launches_decode = 0
+    if not args.no_decode:
+        del flush_buf
+        d = inputs.make_decode(device="cuda", seed=inputs.SEEDS["decode"] + 100 * rank)
+        state0 = d.state.clone()
+        state = d.state
+        yd = torch.empty((d.q.shape[1], H_V, D), dtype=torch.bfloat16, device="cuda")
+        nsteps = d.q.shape[0]
+
+        def dstep():
+            for t in range(nsteps):
+                gdn_decode_step(d.q[t], d.k[t], d.v[t], d.log_alpha[t], d.beta[t], state, y=yd)
+
+        def dreset():
+            state.copy_(state0)
+
+        dclk = ClockSampler(local)
+        dclk.start()
+        dt = timed_steps(dstep, max(3, args.steps // 2), 2, world, flush=dreset, stream=stream)
+        dclk_r = dclk.stop()
+        dms = max_over_ranks(statistics.mean(dt), world) / nsteps
+        N = d.q.shape[1]
+        sbytes = 2 * N * H_V * D * D * 4
+        dbytes = decode_bytes(N)
+        decode = {"workload": "decode: 256 sequences x 64 single-token steps, state 48x128x128 "
+                              "fp32 per sequence, in place",
+                  "us_per_step": dms * 1e3,
+                  "state_GBps": world * sbytes / (dms * 1e-3) / 1e9,
+                  "tokens_per_s": world * N / (dms * 1e-3),
+                  "roofline": {"bound": "hbm",
+                               "achieved": dbytes / (dms * 1e-3) / 1e9,
+                               "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                               "frac": dbytes / (dms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                               "traffic": kernel_traffic("decode"),
+                               "algorithmic_bytes": dbytes},
+                  "state_frac_of_8TBps_nominal": sbytes / (dms * 1e-3) / 8e12,
+                  "clocks": dclk_r}
+        launches_decode = nsteps * max(3, args.steps // 2)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, target_s=args.ref_seconds)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": args.workload, "global_batch": world * n_seq,
+                           "seq_len": T, "heads": "16 QK / 48 value", "d": D,
+                           "path": args.path,
+                           "parallelism": "replicas%d" % world if world > 1 else "single",
+                           "l2": "flushed between steps (256 MB write outside the events)"},
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": args.steps, "clocks": clk, "decode": decode,
+                "gpu_launches_decode_region": launches_decode}
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="prefill4k",
+                    choices=["prefill4k", "prefill256k", "varlen"])
+    ap.add_argument("--path", default="auto", choices=["auto", "tensor", "simt"])
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args, int(os.environ.get("WORLD_SIZE", "1")),
+                      int(os.environ.get("RANK", "0")))
+        return
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,10 @@
+"""Gated DeltaNet chunked scan for NVIDIA B200 (sm_100a).
+
+The computation lives in libgdn.so (CUDA kernels behind the C ABI in
+include/gdn.h).  ``gdn`` is a thin ctypes binding; ``inputs`` holds the
+seeded synthetic workloads; ``build`` compiles the library.
+"""
+from .gdn import (GdnError, gdn_check_device_error, gdn_chunk_fwd,  # noqa: F401
+                  gdn_decode_step, load)
+
+__all__ = ["gdn_chunk_fwd", "gdn_decode_step", "gdn_check_device_error", "GdnError", "load"]

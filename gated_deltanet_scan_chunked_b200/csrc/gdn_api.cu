@@ -1,0 +1,156 @@
+// Host entry points of libgdn: argument validation, kernel selection and the
+// device-side error word.  See include/gdn.h for the contract of each call.
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "gdn_internal.h"
+
+namespace gdn {
+namespace {
+
+// One error word per device.  Kernels OR bits into it (a bounded wait that
+// ran out, a malformed cu_seqlens); gdn_check_device_error reads and clears.
+__device__ int g_error_word = 0;
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+int* g_err_ptr[kMaxDevices] = {nullptr};
+
+int* error_word_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_err_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return nullptr;
+    g_err_ptr[dev] = static_cast<int*>(p);
+  }
+  return g_err_ptr[dev];
+}
+
+bool dim_ok(int32_t d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+gdn_status check_common(int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v, gdn_dtype dt,
+                        float eps_l2, float eps_norm) {
+  if (H_qk <= 0 || H_v <= 0 || H_v % H_qk != 0) return GDN_ERR_INVALID_ARG;
+  if (d_k <= 0 || d_v <= 0) return GDN_ERR_INVALID_ARG;
+  if (!(eps_l2 >= 0.f) || !(eps_norm >= 0.f)) return GDN_ERR_INVALID_ARG;
+  if (dt != GDN_BF16 && dt != GDN_FP32) return GDN_ERR_UNSUPPORTED;
+  if (!dim_ok(d_k) || !dim_ok(d_v)) return GDN_ERR_UNSUPPORTED;
+  return GDN_OK;
+}
+
+}  // namespace
+}  // namespace gdn
+
+using namespace gdn;
+
+extern "C" gdn_status gdn_chunk_fwd_path(
+    const void* q, const void* k, const void* v, const float* log_alpha, const float* beta,
+    const void* g, const float* norm_w, const float* initial_state, const int32_t* cu_seqlens,
+    int32_t n_seq, int64_t total_T, int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v,
+    gdn_dtype in_dtype, int32_t l2norm_qk, float eps_l2, float eps_norm, float scale, void* y,
+    float* final_state, gdn_prefill_path path, gdn_stream_t stream) {
+  gdn_status st = check_common(H_qk, H_v, d_k, d_v, in_dtype, eps_l2, eps_norm);
+  if (st != GDN_OK) return st;
+  if (n_seq < 1 || total_T < 0) return GDN_ERR_INVALID_ARG;
+  if (cu_seqlens == nullptr && n_seq != 1) return GDN_ERR_INVALID_ARG;
+  if ((int64_t)n_seq * H_v > 0x7fffffffLL) return GDN_ERR_INVALID_ARG;
+  if (total_T > 0 && (!q || !k || !v || !log_alpha || !beta || !y)) return GDN_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, log_alpha, beta, g, norm_w, initial_state, y, final_state};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
+  if (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return GDN_ERR_INVALID_ARG;
+  if (initial_state && final_state && initial_state != final_state) {
+    // exact aliasing is allowed; partial overlap is not
+    const char* a0 = reinterpret_cast<const char*>(initial_state);
+    const char* b0 = reinterpret_cast<const char*>(final_state);
+    const size_t bytes = (size_t)n_seq * H_v * d_k * d_v * sizeof(float);
+    if (a0 < b0 + bytes && b0 < a0 + bytes) return GDN_ERR_INVALID_ARG;
+  }
+  if (path != GDN_PATH_AUTO && path != GDN_PATH_TENSOR && path != GDN_PATH_SIMT)
+    return GDN_ERR_INVALID_ARG;
+
+  PrefillArgs a;
+  a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
+  a.g = g; a.norm_w = g ? norm_w : nullptr;
+  a.initial_state = initial_state; a.cu_seqlens = cu_seqlens; a.final_state = final_state;
+  a.y = y; a.n_seq = n_seq; a.total_T = total_T;
+  a.H_qk = H_qk; a.H_v = H_v; a.d_k = d_k; a.d_v = d_v; a.dtype = in_dtype;
+  a.l2norm = l2norm_qk ? 1 : 0; a.eps_l2 = eps_l2; a.eps_norm = eps_norm; a.scale = scale;
+  a.err = error_word_ptr();
+  if (a.err == nullptr) return GDN_ERR_CUDA;
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool tc_ok = prefill_tc_supports(a);
+  if (path == GDN_PATH_TENSOR && !tc_ok) return GDN_ERR_UNSUPPORTED;
+  if (path == GDN_PATH_TENSOR || (path == GDN_PATH_AUTO && tc_ok)) return launch_prefill_tc(a, s);
+  return launch_prefill_simt(a, s);
+}
+
+extern "C" gdn_status gdn_chunk_fwd(
+    const void* q, const void* k, const void* v, const float* log_alpha, const float* beta,
+    const void* g, const float* norm_w, const float* initial_state, const int32_t* cu_seqlens,
+    int32_t n_seq, int64_t total_T, int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v,
+    gdn_dtype in_dtype, int32_t l2norm_qk, float eps_l2, float eps_norm, float scale, void* y,
+    float* final_state, gdn_stream_t stream) {
+  return gdn_chunk_fwd_path(q, k, v, log_alpha, beta, g, norm_w, initial_state, cu_seqlens,
+                            n_seq, total_T, H_qk, H_v, d_k, d_v, in_dtype, l2norm_qk, eps_l2,
+                            eps_norm, scale, y, final_state, GDN_PATH_AUTO, stream);
+}
+
+extern "C" gdn_status gdn_decode_step(const void* q, const void* k, const void* v,
+                                      const float* log_alpha, const float* beta, const void* g,
+                                      const float* norm_w, float* state, int32_t N, int32_t H_qk,
+                                      int32_t H_v, int32_t d_k, int32_t d_v, gdn_dtype in_dtype,
+                                      int32_t l2norm_qk, float eps_l2, float eps_norm,
+                                      float scale, void* y, gdn_stream_t stream) {
+  gdn_status st = check_common(H_qk, H_v, d_k, d_v, in_dtype, eps_l2, eps_norm);
+  if (st != GDN_OK) return st;
+  if (N < 0 || (int64_t)N * H_v > 0x7fffffffLL) return GDN_ERR_INVALID_ARG;
+  if (N == 0) return GDN_OK;
+  if (!q || !k || !v || !log_alpha || !beta || !state || !y) return GDN_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, log_alpha, beta, g, norm_w, state, y};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
+  DecodeArgs a;
+  a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
+  a.g = g; a.norm_w = g ? norm_w : nullptr; a.state = state; a.y = y;
+  a.N = N; a.H_qk = H_qk; a.H_v = H_v; a.d_k = d_k; a.d_v = d_v; a.dtype = in_dtype;
+  a.l2norm = l2norm_qk ? 1 : 0; a.eps_l2 = eps_l2; a.eps_norm = eps_norm; a.scale = scale;
+  return launch_decode(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" gdn_status gdn_check_device_error(gdn_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return GDN_ERR_CUDA;
+  int* p = error_word_ptr();
+  if (p == nullptr) return GDN_ERR_CUDA;
+  int word = 0;
+  if (cudaMemcpy(&word, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return GDN_ERR_CUDA;
+  if (word != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+      return GDN_ERR_CUDA;
+  }
+  if (word & kErrTimeout) return GDN_ERR_TIMEOUT;
+  if (word & kErrBadSeqlens) return GDN_ERR_INVALID_ARG;
+  return GDN_OK;
+}
+
+extern "C" const char* gdn_status_string(gdn_status s) {
+  switch (s) {
+    case GDN_OK: return "ok";
+    case GDN_ERR_INVALID_ARG: return "invalid argument";
+    case GDN_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case GDN_ERR_CUDA: return "CUDA error";
+    case GDN_ERR_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+extern "C" int32_t gdn_version(void) { return 100; }

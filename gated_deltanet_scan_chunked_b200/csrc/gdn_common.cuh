@@ -1,0 +1,88 @@
+// Device helpers shared by the libgdn kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gdn {
+
+template <typename T>
+struct Elem;
+
+template <>
+struct Elem<float> {
+  static __device__ __forceinline__ float load(const float* p) { return __ldg(p); }
+  static __device__ __forceinline__ void store(float* p, float x) { *p = x; }
+  // four consecutive elements (16-byte aligned for float)
+  static __device__ __forceinline__ float4 load4(const float* p) {
+    return __ldg(reinterpret_cast<const float4*>(p));
+  }
+  static __device__ __forceinline__ void store4(float* p, float4 x) {
+    *reinterpret_cast<float4*>(p) = x;
+  }
+};
+
+template <>
+struct Elem<__nv_bfloat16> {
+  static __device__ __forceinline__ float load(const __nv_bfloat16* p) {
+    return __bfloat162float(*p);
+  }
+  static __device__ __forceinline__ void store(__nv_bfloat16* p, float x) {
+    *p = __float2bfloat16_rn(x);
+  }
+  // four consecutive elements (8-byte aligned)
+  static __device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
+    uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+    __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162*>(&u.x);
+    __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162*>(&u.y);
+    float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+    return make_float4(fa.x, fa.y, fb.x, fb.y);
+  }
+  static __device__ __forceinline__ void store4(__nv_bfloat16* p, float4 x) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(x.x, x.y);
+    __nv_bfloat162 b = __floats2bfloat162_rn(x.z, x.w);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t*>(&a);
+    u.y = *reinterpret_cast<uint32_t*>(&b);
+    *reinterpret_cast<uint2*>(p) = u;
+  }
+};
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+// Sum over groups of `width` consecutive lanes (width a power of two <= 32).
+template <int WIDTH>
+__device__ __forceinline__ float group_sum(float x) {
+#pragma unroll
+  for (int o = WIDTH / 2; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+__device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + __expf(-x)); }
+
+// Sequence bounds of sequence s; returns false (and flags the error word)
+// when cu_seqlens is malformed for this sequence.
+__device__ __forceinline__ bool seq_bounds(const int32_t* cu, int s, int64_t total_T,
+                                           int64_t* t0, int64_t* t1, int* err) {
+  if (cu == nullptr) {
+    *t0 = 0;
+    *t1 = total_T;
+    return true;
+  }
+  const int64_t a = cu[s], b = cu[s + 1];
+  const bool ok = (a >= 0) && (b >= a) && (b <= total_T) && (s != 0 || a == 0);
+  if (!ok) {
+    if (err) atomicOr(err, 2);
+    return false;
+  }
+  *t0 = a;
+  *t1 = b;
+  return true;
+}
+
+}  // namespace gdn

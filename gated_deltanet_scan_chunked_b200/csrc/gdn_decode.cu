@@ -1,0 +1,184 @@
+// Single-token decode step of the gated delta rule, one CTA per (sequence,
+// value head).  The step is bound by HBM: the d_k x d_v fp32 state is read
+// once and written once; everything else is a few KB.
+//
+// With S the state before the step, k^ and q^ the L2-normalised key/query,
+// the error form of the rule ("Qwen3.8-Flash-Next: architecture, efficiency
+// and technical lineage", section 03 "Gated DeltaNet", update equations)
+// gives, with a = S^T k^ and b = S^T q^ (one pass over S for both):
+//   e   = v - alpha a
+//   S'  = alpha S + beta k^ e^T
+//   y   = S'^T q^ = alpha b + beta (k^ . q^) e        (times `scale`)
+// so the state is loaded into registers, reduced once over d_k, updated and
+// stored back, with no second read.
+//
+// Thread layout (d_k = d_v = 128, 256 threads): thread (rg, c4) owns columns
+// 4*c4 .. 4*c4+3 (one float4) of rows rg, rg+8, ..., rg+120; a warp reads one
+// whole 512-byte row per load instruction, so every access is a coalesced
+// 128-bit load or store.
+#include "gdn_common.cuh"
+#include "gdn_internal.h"
+
+namespace gdn {
+namespace {
+
+template <int DK, int DV>
+struct DecodeGeom {
+  static constexpr int TPR = DV / 4;  // threads per state row (float4 each)
+  static constexpr int NT_RAW = DK * DV / 16;
+  static constexpr int NT = NT_RAW < 32 ? 32 : (NT_RAW > 256 ? 256 : NT_RAW);
+  static constexpr int ROWG = NT / TPR;  // row groups
+  static constexpr int RPT = DK / ROWG;  // rows per thread
+  static_assert(NT % TPR == 0 && DK % ROWG == 0 && RPT >= 1, "bad decode geometry");
+};
+
+template <int DK, int DV, typename Tin>
+__global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT)
+    gdn_decode_kernel(const DecodeArgs a) {
+  using Geo = DecodeGeom<DK, DV>;
+  constexpr int TPR = Geo::TPR, ROWG = Geo::ROWG, RPT = Geo::RPT;
+  __shared__ float sq[DK], sk[DK];
+  __shared__ float4 red_a[ROWG][TPR], red_b[ROWG][TPR];
+  __shared__ float snorm[3];
+
+  const int n = blockIdx.x / a.H_v;
+  const int h = blockIdx.x % a.H_v;
+  const int hq = h / (a.H_v / a.H_qk);
+  const int tid = threadIdx.x;
+  const int rg = tid / TPR, c4 = tid % TPR;
+
+  float* S = a.state + ((size_t)n * a.H_v + h) * (size_t)(DK * DV);
+  // issue every state load first: they are the whole cost of the step
+  float4 s[RPT];
+#pragma unroll
+  for (int r = 0; r < RPT; ++r) {
+    const int i = rg + ROWG * r;
+    s[r] = __ldcs(reinterpret_cast<const float4*>(S + (size_t)i * DV) + c4);
+  }
+  const Tin* qp = static_cast<const Tin*>(a.q) + ((size_t)n * a.H_qk + hq) * DK;
+  const Tin* kp = static_cast<const Tin*>(a.k) + ((size_t)n * a.H_qk + hq) * DK;
+  for (int i = tid; i < DK; i += Geo::NT) {
+    sq[i] = Elem<Tin>::load(qp + i);
+    sk[i] = Elem<Tin>::load(kp + i);
+  }
+  const float4 v4 =
+      Elem<Tin>::load4(static_cast<const Tin*>(a.v) + ((size_t)n * a.H_v + h) * DV + 4 * c4);
+  const float alpha = __expf(__ldg(a.log_alpha + (size_t)n * a.H_v + h));
+  const float beta = __ldg(a.beta + (size_t)n * a.H_v + h);
+  __syncthreads();
+  if (tid < 32) {
+    float nq = 0.f, nk = 0.f, kq = 0.f;
+    for (int i = tid; i < DK; i += 32) {
+      nq += sq[i] * sq[i];
+      nk += sk[i] * sk[i];
+      kq += sk[i] * sq[i];
+    }
+    nq = warp_sum(nq);
+    nk = warp_sum(nk);
+    kq = warp_sum(kq);
+    if (tid == 0) {
+      const float rq = a.l2norm ? rsqrtf(nq + a.eps_l2) : 1.f;
+      const float rk = a.l2norm ? rsqrtf(nk + a.eps_l2) : 1.f;
+      snorm[0] = rq;
+      snorm[1] = rk;
+      snorm[2] = kq * rq * rk;
+    }
+  }
+  __syncthreads();
+  const float rq = snorm[0], rk = snorm[1], kq = snorm[2];
+
+  // a = S^T k^, b = S^T q^ over this thread's rows, then across row groups
+  float4 pa = make_float4(0.f, 0.f, 0.f, 0.f), pb = pa;
+  float kk[RPT];
+#pragma unroll
+  for (int r = 0; r < RPT; ++r) {
+    const int i = rg + ROWG * r;
+    const float ki = sk[i] * rk, qi = sq[i] * rq;
+    kk[r] = ki;
+    pa.x += s[r].x * ki; pa.y += s[r].y * ki; pa.z += s[r].z * ki; pa.w += s[r].w * ki;
+    pb.x += s[r].x * qi; pb.y += s[r].y * qi; pb.z += s[r].z * qi; pb.w += s[r].w * qi;
+  }
+  red_a[rg][c4] = pa;
+  red_b[rg][c4] = pb;
+  __syncthreads();
+  float4 ta = make_float4(0.f, 0.f, 0.f, 0.f), tb = ta;
+#pragma unroll
+  for (int g2 = 0; g2 < ROWG; ++g2) {
+    const float4 x = red_a[g2][c4], z = red_b[g2][c4];
+    ta.x += x.x; ta.y += x.y; ta.z += x.z; ta.w += x.w;
+    tb.x += z.x; tb.y += z.y; tb.z += z.z; tb.w += z.w;
+  }
+  float4 e;
+  e.x = v4.x - alpha * ta.x; e.y = v4.y - alpha * ta.y;
+  e.z = v4.z - alpha * ta.z; e.w = v4.w - alpha * ta.w;
+
+  // S' = alpha S + beta k^ e^T, stored in place (each thread rewrites
+  // exactly the elements it loaded)
+#pragma unroll
+  for (int r = 0; r < RPT; ++r) {
+    const int i = rg + ROWG * r;
+    const float bk = beta * kk[r];
+    float4 o;
+    o.x = alpha * s[r].x + bk * e.x; o.y = alpha * s[r].y + bk * e.y;
+    o.z = alpha * s[r].z + bk * e.z; o.w = alpha * s[r].w + bk * e.w;
+    __stcs(reinterpret_cast<float4*>(S + (size_t)i * DV) + c4, o);
+  }
+
+  // y = scale (alpha b + beta (k^.q^) e), then the optional epilogue
+  const float bkq = beta * kq;
+  float4 y;
+  y.x = a.scale * (alpha * tb.x + bkq * e.x); y.y = a.scale * (alpha * tb.y + bkq * e.y);
+  y.z = a.scale * (alpha * tb.z + bkq * e.z); y.w = a.scale * (alpha * tb.w + bkq * e.w);
+  const size_t yo = ((size_t)n * a.H_v + h) * DV + 4 * c4;
+  if (a.g != nullptr) {
+    float ss = y.x * y.x + y.y * y.y + y.z * y.z + y.w * y.w;
+    ss = group_sum<TPR>(ss);  // every row group holds the same y
+    const float r = rsqrtf(ss / (float)DV + a.eps_norm);
+    const float4 g4 = Elem<Tin>::load4(static_cast<const Tin*>(a.g) + yo);
+    float4 w4 = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (a.norm_w) w4 = __ldg(reinterpret_cast<const float4*>(a.norm_w + 4 * c4));
+    y.x = y.x * r * (1.f + w4.x) * sigmoidf_(g4.x);
+    y.y = y.y * r * (1.f + w4.y) * sigmoidf_(g4.y);
+    y.z = y.z * r * (1.f + w4.z) * sigmoidf_(g4.z);
+    y.w = y.w * r * (1.f + w4.w) * sigmoidf_(g4.w);
+  }
+  if (rg == 0) Elem<Tin>::store4(static_cast<Tin*>(a.y) + yo, y);
+}
+
+template <int DK, int DV, typename Tin>
+gdn_status launch(const DecodeArgs& a, cudaStream_t stream) {
+  const unsigned grid = (unsigned)a.N * (unsigned)a.H_v;
+  gdn_decode_kernel<DK, DV, Tin><<<grid, DecodeGeom<DK, DV>::NT, 0, stream>>>(a);
+  return cudaPeekAtLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+template <typename Tin>
+gdn_status dispatch_dv(const DecodeArgs& a, cudaStream_t s) {
+#define GDN_DV_CASES(DK)                                     \
+  switch (a.d_v) {                                           \
+    case 16: return launch<DK, 16, Tin>(a, s);               \
+    case 32: return launch<DK, 32, Tin>(a, s);               \
+    case 64: return launch<DK, 64, Tin>(a, s);               \
+    case 128: return launch<DK, 128, Tin>(a, s);             \
+    default: return GDN_ERR_UNSUPPORTED;                     \
+  }
+  switch (a.d_k) {
+    case 16: GDN_DV_CASES(16)
+    case 32: GDN_DV_CASES(32)
+    case 64: GDN_DV_CASES(64)
+    case 128: GDN_DV_CASES(128)
+    default: return GDN_ERR_UNSUPPORTED;
+  }
+#undef GDN_DV_CASES
+}
+
+}  // namespace
+
+gdn_status launch_decode(const DecodeArgs& a, cudaStream_t stream) {
+  if (a.N == 0) return GDN_OK;
+  if (a.dtype == GDN_BF16) return dispatch_dv<__nv_bfloat16>(a, stream);
+  if (a.dtype == GDN_FP32) return dispatch_dv<float>(a, stream);
+  return GDN_ERR_UNSUPPORTED;
+}
+
+}  // namespace gdn

@@ -1,0 +1,62 @@
+// Internal interface between the host entry points (gdn_api.cu) and the
+// kernel translation units.  Not installed; not part of the C ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/gdn.h"
+
+namespace gdn {
+
+// Bits of the device-side error word.
+enum : int {
+  kErrTimeout = 1,      // a bounded wait ran out
+  kErrBadSeqlens = 2,   // cu_seqlens not monotone / out of range
+};
+
+struct PrefillArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* log_alpha;
+  const float* beta;
+  const void* g;           // nullptr: no epilogue
+  const float* norm_w;     // nullptr: zeros
+  const float* initial_state;  // nullptr: zeros
+  const int32_t* cu_seqlens;   // nullptr: one sequence of total_T tokens
+  float* final_state;      // nullptr: not written
+  void* y;
+  int32_t n_seq;
+  int64_t total_T;
+  int32_t H_qk, H_v, d_k, d_v;
+  gdn_dtype dtype;
+  int32_t l2norm;
+  float eps_l2, eps_norm, scale;
+  int* err;                // device error word
+};
+
+struct DecodeArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* log_alpha;
+  const float* beta;
+  const void* g;
+  const float* norm_w;
+  float* state;
+  void* y;
+  int32_t N, H_qk, H_v, d_k, d_v;
+  gdn_dtype dtype;
+  int32_t l2norm;
+  float eps_l2, eps_norm, scale;
+};
+
+// Each launcher returns GDN_OK, GDN_ERR_UNSUPPORTED (shape not compiled) or
+// GDN_ERR_CUDA (launch failed).
+gdn_status launch_decode(const DecodeArgs& a, cudaStream_t stream);
+gdn_status launch_prefill_simt(const PrefillArgs& a, cudaStream_t stream);
+gdn_status launch_prefill_tc(const PrefillArgs& a, cudaStream_t stream);
+bool prefill_tc_supports(const PrefillArgs& a);
+
+}  // namespace gdn

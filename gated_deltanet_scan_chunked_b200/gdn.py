@@ -1,0 +1,181 @@
+"""Thin Python binding of libgdn (see include/gdn.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of libgdn.so.  PyTorch supplies device memory and the current
+stream.  There is no fallback: if the library is missing or the tensors are
+not on a CUDA device, the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgdn.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "gdn.h")
+
+GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_TIMEOUT = range(5)
+GDN_BF16, GDN_FP32 = 0, 1
+PATHS = {"auto": 0, "tensor": 1, "simt": 2}
+
+_lib = None
+_vp = ctypes.c_void_p
+
+
+class GdnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__("%s: %s (status %d)" % (what, status_string(status), status))
+
+
+def load(path: str = LIB_PATH):
+    """Load libgdn.so (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(
+            "libgdn.so not found at %s; build it with "
+            "`python -m gated_deltanet_scan_chunked_b200.build`" % path)
+    lib = ctypes.CDLL(path)
+    f = lib.gdn_chunk_fwd_path
+    f.restype = ctypes.c_int
+    f.argtypes = [_vp] * 9 + [ctypes.c_int32, ctypes.c_int64] + [ctypes.c_int32] * 5 + [
+        ctypes.c_int32, ctypes.c_float, ctypes.c_float, ctypes.c_float, _vp, _vp,
+        ctypes.c_int, _vp]
+    f = lib.gdn_chunk_fwd
+    f.restype = ctypes.c_int
+    f.argtypes = [_vp] * 9 + [ctypes.c_int32, ctypes.c_int64] + [ctypes.c_int32] * 5 + [
+        ctypes.c_int32, ctypes.c_float, ctypes.c_float, ctypes.c_float, _vp, _vp, _vp]
+    f = lib.gdn_decode_step
+    f.restype = ctypes.c_int
+    f.argtypes = [_vp] * 8 + [ctypes.c_int32] * 6 + [
+        ctypes.c_int32, ctypes.c_float, ctypes.c_float, ctypes.c_float, _vp, _vp]
+    lib.gdn_check_device_error.restype = ctypes.c_int
+    lib.gdn_check_device_error.argtypes = [_vp]
+    lib.gdn_status_string.restype = ctypes.c_char_p
+    lib.gdn_status_string.argtypes = [ctypes.c_int]
+    lib.gdn_version.restype = ctypes.c_int32
+    lib.gdn_version.argtypes = []
+    _lib = lib
+    return lib
+
+
+def header_functions(path: str = HEADER_PATH):
+    """Names of the functions declared in include/gdn.h."""
+    text = open(path).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdn_[a-z0-9_]+)\s*\(", text)))
+
+
+def status_string(status: int) -> str:
+    return load().gdn_status_string(int(status)).decode()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return GDN_BF16
+    if t.dtype == torch.float32:
+        return GDN_FP32
+    raise TypeError("q/k/v/g must be bfloat16 or float32, got %s" % t.dtype)
+
+
+def _check(t: Optional[torch.Tensor], name: str, dtype=None, device=None):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor (libgdn has no CPU path)" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if device is not None and t.device != device:
+        raise ValueError("%s is on %s, expected %s" % (name, t.device, device))
+
+
+def gdn_chunk_fwd(q, k, v, log_alpha, beta, g=None, norm_w=None,
+                  initial_state=None, cu_seqlens=None, l2norm_qk=True,
+                  eps_l2=1e-6, eps_norm=1e-6, scale=1.0, y=None,
+                  final_state=None, output_final_state=True, path="auto",
+                  stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Chunked prefill over packed sequences: returns (y, final_state).
+
+    q, k [T, H_qk, d_k]; v [T, H_v, d_v]; log_alpha, beta [T, H_v] fp32;
+    g [T, H_v, d_v] or None; norm_w [d_v] fp32 or None; initial_state
+    [n_seq, H_v, d_k, d_v] fp32 or None; cu_seqlens [n_seq + 1] int32 (device)
+    or None.  y / final_state may be passed in (final_state may be
+    initial_state itself for an in-place update).
+    """
+    lib = load()
+    dev = q.device
+    dt = _dtype_code(q)
+    T, Hqk, dk = q.shape
+    Hv, dv = v.shape[1], v.shape[2]
+    n_seq = 1 if cu_seqlens is None else int(cu_seqlens.shape[0]) - 1
+    for name, t in (("q", q), ("k", k), ("v", v), ("g", g)):
+        _check(t, name, q.dtype, dev)
+    for name, t in (("log_alpha", log_alpha), ("beta", beta), ("norm_w", norm_w),
+                    ("initial_state", initial_state)):
+        _check(t, name, torch.float32, dev)
+    _check(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    if y is None:
+        y = torch.empty((T, Hv, dv), dtype=q.dtype, device=dev)
+    _check(y, "y", q.dtype, dev)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((n_seq, Hv, dk, dv), dtype=torch.float32, device=dev)
+    _check(final_state, "final_state", torch.float32, dev)
+    st = lib.gdn_chunk_fwd_path(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(g), _ptr(norm_w),
+        _ptr(initial_state), _ptr(cu_seqlens), n_seq, T, Hqk, Hv, dk, dv, dt,
+        1 if l2norm_qk else 0, float(eps_l2), float(eps_norm), float(scale), _ptr(y),
+        _ptr(final_state), PATHS[path], _stream_handle(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_chunk_fwd")
+    return y, final_state
+
+
+def gdn_decode_step(q, k, v, log_alpha, beta, state, g=None, norm_w=None,
+                    l2norm_qk=True, eps_l2=1e-6, eps_norm=1e-6, scale=1.0,
+                    y=None, stream=None) -> torch.Tensor:
+    """One token per sequence; ``state`` [N, H_v, d_k, d_v] fp32 is updated
+    in place.  q, k [N, H_qk, d_k]; v [N, H_v, d_v]; gates [N, H_v].
+    Returns y [N, H_v, d_v]."""
+    lib = load()
+    dev = q.device
+    dt = _dtype_code(q)
+    N, Hqk, dk = q.shape
+    Hv, dv = v.shape[1], v.shape[2]
+    for name, t in (("q", q), ("k", k), ("v", v), ("g", g)):
+        _check(t, name, q.dtype, dev)
+    for name, t in (("log_alpha", log_alpha), ("beta", beta), ("norm_w", norm_w),
+                    ("state", state)):
+        _check(t, name, torch.float32, dev)
+    if y is None:
+        y = torch.empty((N, Hv, dv), dtype=q.dtype, device=dev)
+    _check(y, "y", q.dtype, dev)
+    st = lib.gdn_decode_step(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(g), _ptr(norm_w),
+        _ptr(state), N, Hqk, Hv, dk, dv, dt, 1 if l2norm_qk else 0, float(eps_l2),
+        float(eps_norm), float(scale), _ptr(y), _stream_handle(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_decode_step")
+    return y
+
+
+def gdn_check_device_error(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device error status."""
+    return int(load().gdn_check_device_error(_stream_handle(stream)))

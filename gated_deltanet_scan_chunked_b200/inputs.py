@@ -22,6 +22,12 @@ section 02: 48 value heads share 16 QK heads, head dim 128):
 
 q and k are drawn N(0,1) and are L2-normalised by the consumer (the kernel's
 prologue, or the oracle), as the workloads specify.
+
+``device="cpu"`` (default) draws with torch's CPU generator; ``device="cuda"``
+draws the same distributions with torch's CUDA (Philox) generator, which is
+what the full-size workloads use (drawing 2.4 G normals on one CPU core takes
+about a minute).  The two streams differ; a given (workload, device, seed)
+is reproducible.  Oracle comparisons copy the sampled slices to the host.
 """
 from __future__ import annotations
 
@@ -76,13 +82,14 @@ class DecodeInputs:
 def _normal(gen, shape, dtype, std=1.0, mean=0.0):
     """N(mean, std^2) drawn in fp32 in token blocks, rounded to ``dtype``."""
     shape = tuple(int(s) for s in shape)
-    out = torch.empty(shape, dtype=dtype)
+    out = torch.empty(shape, dtype=dtype, device=gen.device)
     if len(shape) == 0 or shape[0] == 0:
         return out
     rest = shape[1:]
     for t0 in range(0, shape[0], _BLOCK_TOKENS):
         t1 = min(shape[0], t0 + _BLOCK_TOKENS)
-        x = torch.randn((t1 - t0,) + rest, generator=gen, dtype=torch.float32)
+        x = torch.randn((t1 - t0,) + rest, generator=gen, dtype=torch.float32,
+                        device=gen.device)
         if std != 1.0:
             x.mul_(std)
         if mean != 0.0:
@@ -94,31 +101,38 @@ def _normal(gen, shape, dtype, std=1.0, mean=0.0):
 def _gates(gen, T, Hv, alpha_kind):
     if alpha_kind == "sigmoid_n2":
         # alpha = sigmoid(N(2,1)); stored as log(alpha)
-        x = torch.randn((T, Hv), generator=gen, dtype=torch.float32) + 2.0
+        x = torch.randn((T, Hv), generator=gen, dtype=torch.float32, device=gen.device) + 2.0
         log_alpha = torch.nn.functional.logsigmoid(x)
     else:
         # log alpha = -softplus(N(0,1)) * 0.1
-        x = torch.randn((T, Hv), generator=gen, dtype=torch.float32)
+        x = torch.randn((T, Hv), generator=gen, dtype=torch.float32, device=gen.device)
         log_alpha = -torch.nn.functional.softplus(x) * 0.1
-    beta = torch.sigmoid(torch.randn((T, Hv), generator=gen, dtype=torch.float32))
+    beta = torch.sigmoid(torch.randn((T, Hv), generator=gen, dtype=torch.float32,
+                                     device=gen.device))
     return log_alpha.contiguous(), beta.contiguous()
 
 
+def _gen(seed, device):
+    return torch.Generator(device=device).manual_seed(int(seed))
+
+
 def make_prefill(lengths, H_qk, H_v, d_k, d_v, dtype=torch.bfloat16, seed=0,
-                 epilogue=True, s0_std=0.0, alpha_kind="softplus01"):
+                 epilogue=True, s0_std=0.0, alpha_kind="softplus01", device="cpu"):
     """Generic seeded prefill inputs over sequences of the given lengths."""
-    gen = torch.Generator().manual_seed(int(seed))
+    gen = _gen(seed, device)
     lengths = [int(x) for x in lengths]
     T = sum(lengths)
     cu = torch.zeros(len(lengths) + 1, dtype=torch.int32)
     if lengths:
         cu[1:] = torch.cumsum(torch.tensor(lengths, dtype=torch.int64), 0).to(torch.int32)
+    cu = cu.to(device)
     q = _normal(gen, (T, H_qk, d_k), dtype)
     k = _normal(gen, (T, H_qk, d_k), dtype)
     v = _normal(gen, (T, H_v, d_v), dtype)
     log_alpha, beta = _gates(gen, T, H_v, alpha_kind)
     g = _normal(gen, (T, H_v, d_v), dtype) if epilogue else None
-    norm_w = (torch.randn((d_v,), generator=gen, dtype=torch.float32) * 0.02) if epilogue else None
+    norm_w = (torch.randn((d_v,), generator=gen, dtype=torch.float32, device=gen.device) * 0.02
+              if epilogue else None)
     s0 = None
     if s0_std > 0.0:
         s0 = _normal(gen, (len(lengths), H_v, d_k, d_v), torch.float32, std=s0_std)
@@ -132,33 +146,36 @@ def varlen_lengths(n_seq=24, lo=512, hi=16384, seed=SEEDS["varlen"]):
     return [int(x) for x in torch.randint(lo, hi + 1, (n_seq,), generator=gen)]
 
 
-def workload(name: str, T: Optional[int] = None):
+def workload(name: str, T: Optional[int] = None, device="cpu"):
     """The named workload's inputs.  ``T`` shortens a prefill workload
     (same recipe, fewer tokens) for oracle-sized parity cases."""
     seed = SEEDS[name]
     if name == "tiny":
         return make_prefill([T or 64], 2, 4, 16, 16, dtype=torch.float32,
                             seed=seed, epilogue=False, s0_std=0.0,
-                            alpha_kind="sigmoid_n2")
+                            alpha_kind="sigmoid_n2", device=device)
     if name == "prefill4k":
-        return make_prefill([T or 4096], 16, 48, 128, 128, seed=seed)
+        return make_prefill([T or 4096], 16, 48, 128, 128, seed=seed, device=device)
     if name == "prefill256k":
-        return make_prefill([T or 262144], 16, 48, 128, 128, seed=seed, s0_std=0.01)
+        return make_prefill([T or 262144], 16, 48, 128, 128, seed=seed, s0_std=0.01,
+                            device=device)
     if name == "varlen":
-        return make_prefill(varlen_lengths(), 16, 48, 128, 128, seed=seed, s0_std=0.01)
+        return make_prefill(varlen_lengths(), 16, 48, 128, 128, seed=seed, s0_std=0.01,
+                            device=device)
     raise KeyError(name)
 
 
 def make_decode(N=256, steps=64, H_qk=16, H_v=48, d_k=128, d_v=128,
                 dtype=torch.bfloat16, seed=SEEDS["decode"], state_std=0.05,
-                epilogue=False):
-    gen = torch.Generator().manual_seed(int(seed))
+                epilogue=False, device="cpu"):
+    gen = _gen(seed, device)
     state = _normal(gen, (N, H_v, d_k, d_v), torch.float32, std=state_std)
     q = _normal(gen, (steps, N, H_qk, d_k), dtype)
     k = _normal(gen, (steps, N, H_qk, d_k), dtype)
     v = _normal(gen, (steps, N, H_v, d_v), dtype)
     la, b = _gates(gen, steps * N, H_v, "softplus01")
     g = _normal(gen, (steps, N, H_v, d_v), dtype) if epilogue else None
-    w = (torch.randn((d_v,), generator=gen, dtype=torch.float32) * 0.02) if epilogue else None
+    w = (torch.randn((d_v,), generator=gen, dtype=torch.float32, device=gen.device) * 0.02
+         if epilogue else None)
     return DecodeInputs(state, q, k, v, la.view(steps, N, H_v), b.view(steps, N, H_v),
                         g, w, meta={"seed": int(seed)})

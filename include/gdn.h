@@ -1,0 +1,164 @@
+/*
+ * gdn.h -- C ABI of libgdn: the Gated DeltaNet (GDN) token mixer's gated
+ * delta rule on NVIDIA B200 (sm_100a).
+ *
+ * The operation ("Qwen3.8-Flash-Next: architecture, efficiency and technical
+ * lineage", section 03 "Gated DeltaNet", update equations; product form in
+ * "On the Design of Qwen3.8-Next Architecture ... close reading", section
+ * 4.1), per sequence and per value head, token by token:
+ *
+ *     S~  = alpha_t S_{t-1}
+ *     e_t = v_t - S~^T k_t
+ *     S_t = S~ + beta_t k_t e_t^T      (= alpha_t (I - beta_t k k^T) S + beta_t k v^T)
+ *     y_t = scale * S_t^T q_t
+ *
+ * with q, k L2-normalised over d_k (the same page, section 03, and the
+ * hyper.ai summary, "Method": queries and keys are L2-normalised), alpha =
+ * exp(log_alpha) in (0,1), beta in (0,1), and an optional output epilogue
+ * (section 03, "what Qwen changed on the original GDN": zero-centred
+ * RMSNorm, sigmoid output gate; normalise first, then gate):
+ *
+ *     out_t = y_t / sqrt(mean_j y_tj^2 + eps_norm) * (1 + w) * sigmoid(g_t)
+ *
+ * Conventions shared by every entry point:
+ *   - All pointers are DEVICE pointers unless stated otherwise, dense and
+ *     row-major, 16-byte aligned.  The caller owns every buffer; the library
+ *     allocates no memory and never synchronises.  Work is enqueued on
+ *     `stream` and runs asynchronously; a CUDA error raised by the kernel
+ *     surfaces on the caller's next synchronisation.
+ *   - Value head h reads QK head h / (H_v / H_qk) (contiguous groups);
+ *     H_v % H_qk != 0 is GDN_ERR_INVALID_ARG.
+ *   - The recurrent state of one head is S[i][j], i over d_k, j over d_v,
+ *     fp32.  Prefill and decode use the same layout, so decode continues from
+ *     a prefill's final state.
+ *   - Supported head dims: d_k, d_v in {16, 32, 64, 128}; anything else is
+ *     GDN_ERR_UNSUPPORTED.
+ *   - Input dtype (q, k, v, g and the output y): GDN_BF16 or GDN_FP32.
+ *     log_alpha, beta, norm_w and all states are always fp32.
+ *   - Arguments are validated on the host before anything is enqueued; a
+ *     rejected call enqueues nothing and leaves every output untouched.
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Opaque CUDA stream handle (same object as cudaStream_t); 0 = legacy
+ * default stream. */
+typedef struct CUstream_st* gdn_stream_t;
+
+typedef enum {
+  GDN_OK = 0,
+  GDN_ERR_INVALID_ARG = 1, /* null pointer, bad shape, bad cu_seqlens ...  */
+  GDN_ERR_UNSUPPORTED = 2, /* a head dim or dtype this build does not have */
+  GDN_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed         */
+  GDN_ERR_TIMEOUT = 4      /* a device-side wait hit its iteration limit   */
+} gdn_status;
+
+typedef enum { GDN_BF16 = 0, GDN_FP32 = 1 } gdn_dtype;
+
+/* Which prefill kernel runs.  AUTO picks the tensor-core kernel when it
+ * supports the shape (bf16, d_k = d_v = 128) and the portable CUDA-core
+ * kernel otherwise.  TENSOR on an unsupported shape is GDN_ERR_UNSUPPORTED. */
+typedef enum {
+  GDN_PATH_AUTO = 0,
+  GDN_PATH_TENSOR = 1, /* tcgen05 MMA + TMA + TMEM chunked kernel */
+  GDN_PATH_SIMT = 2    /* fp32 CUDA-core chunked kernel           */
+} gdn_prefill_path;
+
+/*
+ * gdn_chunk_fwd -- prefill over a packed batch of variable-length sequences,
+ * chunkwise-parallel within each sequence (chunks of 64 tokens), the fp32
+ * state carried from chunk to chunk.  The result equals the token-by-token
+ * recurrence above up to rounding.
+ *
+ *   q, k           [total_T, H_qk, d_k]  in_dtype
+ *   v              [total_T, H_v, d_v]   in_dtype
+ *   log_alpha      [total_T, H_v] fp32, log of the decay gate (finite, <= 0)
+ *   beta           [total_T, H_v] fp32, write gate
+ *   g              [total_T, H_v, d_v] in_dtype, or NULL: no epilogue
+ *   norm_w         [d_v] fp32 (applied as 1 + w), or NULL (= zeros); ignored
+ *                  when g is NULL
+ *   initial_state  [n_seq, H_v, d_k, d_v] fp32, or NULL (= zeros)
+ *   cu_seqlens     [n_seq + 1] int32 DEVICE array of sequence offsets,
+ *                  cu[0] = 0, non-decreasing, cu[n_seq] = total_T; NULL
+ *                  means one sequence (n_seq must be 1).  Empty sequences
+ *                  are allowed (final = initial).  The library cannot read
+ *                  a device array on the host without a synchronisation, so
+ *                  a malformed cu_seqlens is caught by the kernel: offending
+ *                  sequences write nothing and gdn_check_device_error
+ *                  reports GDN_ERR_INVALID_ARG.
+ *   n_seq          number of sequences (>= 1)
+ *   total_T        number of packed tokens (>= 0)
+ *   l2norm_qk      1: normalise q, k in the kernel; 0: used as given
+ *   eps_l2         inside the L2-norm square root (default 1e-6)
+ *   eps_norm       inside the RMSNorm square root (default 1e-6)
+ *   scale          multiplies y before the epilogue (default 1.0)
+ *   y              [total_T, H_v, d_v] in_dtype, written
+ *   final_state    [n_seq, H_v, d_k, d_v] fp32 or NULL; may alias
+ *                  initial_state exactly (in-place update), must not
+ *                  partially overlap it
+ *   path           kernel selection (see gdn_prefill_path)
+ */
+gdn_status gdn_chunk_fwd_path(
+    const void* q, const void* k, const void* v, const float* log_alpha,
+    const float* beta, const void* g, const float* norm_w,
+    const float* initial_state, const int32_t* cu_seqlens, int32_t n_seq,
+    int64_t total_T, int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v,
+    gdn_dtype in_dtype, int32_t l2norm_qk, float eps_l2, float eps_norm,
+    float scale, void* y, float* final_state, gdn_prefill_path path,
+    gdn_stream_t stream);
+
+/* gdn_chunk_fwd -- gdn_chunk_fwd_path with GDN_PATH_AUTO. */
+gdn_status gdn_chunk_fwd(
+    const void* q, const void* k, const void* v, const float* log_alpha,
+    const float* beta, const void* g, const float* norm_w,
+    const float* initial_state, const int32_t* cu_seqlens, int32_t n_seq,
+    int64_t total_T, int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v,
+    gdn_dtype in_dtype, int32_t l2norm_qk, float eps_l2, float eps_norm,
+    float scale, void* y, float* final_state, gdn_stream_t stream);
+
+/*
+ * gdn_decode_step -- one token for each of N independent sequences; the
+ * state is read once and written back once, in place.
+ *
+ *   q, k        [N, H_qk, d_k] in_dtype
+ *   v           [N, H_v, d_v]  in_dtype
+ *   log_alpha   [N, H_v] fp32;  beta [N, H_v] fp32
+ *   g, norm_w   optional epilogue, as for gdn_chunk_fwd
+ *   state       [N, H_v, d_k, d_v] fp32, read and overwritten
+ *   y           [N, H_v, d_v] in_dtype, written
+ * Other arguments as for gdn_chunk_fwd.  N = 0 is a no-op.
+ */
+gdn_status gdn_decode_step(
+    const void* q, const void* k, const void* v, const float* log_alpha,
+    const float* beta, const void* g, const float* norm_w, float* state,
+    int32_t N, int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v,
+    gdn_dtype in_dtype, int32_t l2norm_qk, float eps_l2, float eps_norm,
+    float scale, void* y, gdn_stream_t stream);
+
+/*
+ * gdn_check_device_error -- synchronise `stream`, then read and clear the
+ * library's device-side error word on the current device.  Returns GDN_OK,
+ * GDN_ERR_TIMEOUT (a kernel's bounded wait ran out and the kernel returned
+ * early; its outputs are incomplete), GDN_ERR_INVALID_ARG (a kernel found a
+ * malformed cu_seqlens) or GDN_ERR_CUDA (the synchronisation itself failed).
+ * This call blocks the host; the compute entry points never do.
+ */
+gdn_status gdn_check_device_error(gdn_stream_t stream);
+
+/* Static text for a status code. */
+const char* gdn_status_string(gdn_status status);
+
+/* Library version as an integer (major * 10000 + minor * 100 + patch). */
+int32_t gdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H_ */

@@ -1,0 +1,96 @@
+"""CPU-side checks of the C ABI: the library loads without a GPU, exports
+every function include/gdn.h declares, and rejects bad arguments on the
+host before touching the device."""
+import ctypes
+
+import pytest
+
+from gated_deltanet_scan_chunked_b200 import build as gbuild
+from gated_deltanet_scan_chunked_b200 import gdn
+
+
+@pytest.fixture(scope="module")
+def lib():
+    gbuild.build()
+    return gdn.load()
+
+
+def test_exports_every_declared_function(lib):
+    names = gdn.header_functions()
+    assert set(names) >= {"gdn_chunk_fwd", "gdn_chunk_fwd_path", "gdn_decode_step",
+                          "gdn_check_device_error", "gdn_status_string", "gdn_version"}
+    for n in names:
+        assert hasattr(lib, n), "libgdn.so does not export %s" % n
+
+
+def test_status_strings_and_version(lib):
+    assert gdn.status_string(0) == "ok"
+    assert "timed out" in gdn.status_string(4)
+    assert gdn.status_string(99) == "unknown status"
+    assert lib.gdn_version() >= 100
+
+
+FAKE = 0x1000  # a 16-byte aligned non-null address; never dereferenced
+
+
+def _chunk(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, b=FAKE, g=None, w=None, s0=None, cu=None,
+             n_seq=1, T=64, Hqk=16, Hv=48, dk=128, dv=128, dt=0, l2=1, e1=1e-6, e2=1e-6,
+             sc=1.0, y=FAKE, fs=None, path=0)
+    a.update(kw)
+    return lib.gdn_chunk_fwd_path(a["q"], a["k"], a["v"], a["la"], a["b"], a["g"], a["w"],
+                                  a["s0"], a["cu"], a["n_seq"], a["T"], a["Hqk"], a["Hv"],
+                                  a["dk"], a["dv"], a["dt"], a["l2"], a["e1"], a["e2"],
+                                  a["sc"], a["y"], a["fs"], a["path"], None)
+
+
+def _decode(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, b=FAKE, g=None, w=None, s=FAKE, N=4, Hqk=16,
+             Hv=48, dk=128, dv=128, dt=0, l2=1, e1=1e-6, e2=1e-6, sc=1.0, y=FAKE)
+    a.update(kw)
+    return lib.gdn_decode_step(a["q"], a["k"], a["v"], a["la"], a["b"], a["g"], a["w"],
+                               a["s"], a["N"], a["Hqk"], a["Hv"], a["dk"], a["dv"], a["dt"],
+                               a["l2"], a["e1"], a["e2"], a["sc"], a["y"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(y=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(Hv=40), gdn.GDN_ERR_INVALID_ARG),          # 40 % 16 != 0
+    (dict(Hqk=0), gdn.GDN_ERR_INVALID_ARG),
+    (dict(n_seq=0), gdn.GDN_ERR_INVALID_ARG),
+    (dict(n_seq=2), gdn.GDN_ERR_INVALID_ARG),        # several sequences need cu_seqlens
+    (dict(T=-1), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dk=96), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(dv=256), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(dt=7), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(e1=-1.0), gdn.GDN_ERR_INVALID_ARG),
+    (dict(q=FAKE + 8), gdn.GDN_ERR_INVALID_ARG),     # misaligned
+    (dict(cu=FAKE + 2, n_seq=2), gdn.GDN_ERR_INVALID_ARG),
+    (dict(path=9), gdn.GDN_ERR_INVALID_ARG),
+    (dict(s0=FAKE, fs=FAKE + 4096), gdn.GDN_ERR_INVALID_ARG),  # partial overlap
+])
+def test_chunk_fwd_rejects_bad_arguments_on_host(lib, kw, code):
+    assert _chunk(lib, **kw) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(s=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(N=-1), gdn.GDN_ERR_INVALID_ARG),
+    (dict(Hv=17), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dk=8), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(y=FAKE + 4), gdn.GDN_ERR_INVALID_ARG),
+])
+def test_decode_rejects_bad_arguments_on_host(lib, kw, code):
+    assert _decode(lib, **kw) == code
+
+
+def test_decode_with_no_sequences_is_a_no_op(lib):
+    assert _decode(lib, N=0, q=None, s=None, y=None) == gdn.GDN_OK
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    q = torch.zeros(4, 1, 16)
+    with pytest.raises(ValueError):
+        gdn.gdn_chunk_fwd(q, q, torch.zeros(4, 1, 16), torch.zeros(4, 1), torch.zeros(4, 1))

