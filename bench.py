@@ -163,12 +163,24 @@ def dist_setup(args):
     return world, rank, local
 
 
-def max_over_ranks(x, world):
+def max_over_ranks(x, world, device="cuda"):
+    """Max of a host scalar over all ranks (host plumbing, not data path)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(units_per_rank, world, ms_max):
+    """Units all ranks processed divided by the slowest rank's time."""
+    return world * units_per_rank / (ms_max * 1e-3)
+
+
+def rank_seed(name, rank):
+    """Each rank draws an independent batch of the same recipe."""
+    from gated_deltanet_scan_chunked_b200 import inputs
+    return inputs.SEEDS[name] + 100 * rank
 
 
 def barrier(world):
@@ -235,7 +247,7 @@ def make_workload(name, rank):
     w = inputs.workload(name, device="cuda")
     if rank:
         # an independent batch per rank: same recipe, another seed
-        seed = inputs.SEEDS[name] + 100 * rank
+        seed = rank_seed(name, rank)
         lengths = w.meta["lengths"]
         w = inputs.make_prefill(lengths, H_QK, H_V, D, D, seed=seed,
                                 s0_std=0.01 if w.initial_state is not None else 0.0,
@@ -302,7 +314,7 @@ def run_ours(args, world, rank, local):
         raise RuntimeError("device error: %s" % gdn.status_string(err))
     ms = statistics.mean(times)
     ms_max = max_over_ranks(ms, world)
-    value = world * T / (ms_max * 1e-3)
+    value = whole_job_rate(T, world, ms_max)
 
     # roofline of the dominant (only) kernel of the step
     nbytes = prefill_bytes(T, n_seq, epilogue=w.g is not None, init_state=has_s0)

@@ -45,6 +45,11 @@
 #include "gdn_internal.h"
 #include "gdn_sm100.cuh"
 
+// Section timing hook for tuning builds; compiles to nothing by default.
+#ifndef GDN_TRACE_POINT
+#define GDN_TRACE_POINT(i)
+#endif
+
 namespace gdn {
 namespace {
 
@@ -205,6 +210,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
   for (int64_t c0 = t_begin; c0 < t_end; c0 += kC) {
     const int n = (t_end - c0) < kC ? (int)(t_end - c0) : kC;
 
+    GDN_TRACE_POINT(0);
     // ---- gates: cumsum of log alpha, beta, gamma, exp(G_C - G) --------------
     if (warp == 0) {
       float carry = 0.f;
@@ -236,6 +242,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
     __syncthreads();
     fence_after_sync();
 
+    GDN_TRACE_POINT(1);
     // ---- q, k rows -> operand tiles; v rows kept in registers -----------------
     // warp w owns rows 8w .. 8w+7; lane l owns columns 4l .. 4l+3
     float4 vv[8];
@@ -290,6 +297,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
       }
     }
 
+    GDN_TRACE_POINT(2);
     // ---- S^T from TMEM, block maxima, chunk exponent e ---------------------------
     float sv[64];
     tmem_ld32(tS + half * 64, sv);
@@ -329,6 +337,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
     fence_before_sync();
     __syncthreads();
 
+    GDN_TRACE_POINT(3);
     // ---- MMA0: [K;Q] K^T (bf16, exact);  MMA2: S^T (gamma Q^)^T (fp16) -----------
     if (tid == 0) {
       fence_after_sync();
@@ -350,6 +359,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
     if (!__syncthreads_and(ok)) { ok = false; break; }
     fence_after_sync();
 
+    GDN_TRACE_POINT(4);
     // ---- A (fp32) and P (fp16) from the raw products (warps 0-3) --------------
     if (tid < 128) {
       const int t = tid & 63;
@@ -388,6 +398,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
     fence_before_sync();
     __syncthreads();
 
+    GDN_TRACE_POINT(5);
     // ---- T = (I + A)^{-1}: 16 x 16 diagonal blocks by substitution -------------
     if (tid < 64) {
       const int b = tid >> 4, c = tid & 15;
@@ -423,6 +434,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
       __syncthreads();
     }
 
+    GDN_TRACE_POINT(6);
     // ---- scale exponent of T; T diag(b) 2^-f, T diag(b g) 2^-f -> fp16 ---------
     float tmax = 0.f;
     if (tid < 128) {
@@ -457,6 +469,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
     fence_before_sync();
     __syncthreads();
 
+    GDN_TRACE_POINT(7);
     // ---- MMAW: W^T = K^T (T diag(b g))^T;  MMAU: U^T = V^T (T diag(b))^T -------
     if (tid == 0) {
       fence_after_sync();
@@ -479,6 +492,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
     if (!__syncthreads_and(ok)) { ok = false; break; }
     fence_after_sync();
 
+    GDN_TRACE_POINT(8);
     // ---- W^T 2^-f (fp32) -> fp16 tile, rows d, columns t ------------------------
     {
       float v[32];
@@ -492,6 +506,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
     fence_before_sync();
     __syncthreads();
 
+    GDN_TRACE_POINT(9);
     // ---- MMA1: Delta^T 2^-(e+f) = U^T - S^T W^T ---------------------------------------
     if (tid == 0) {
       fence_after_sync();
@@ -508,6 +523,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
     if (!__syncthreads_and(ok)) { ok = false; break; }
     fence_after_sync();
 
+    GDN_TRACE_POINT(10);
     // ---- Delta^T 2^-e -> fp16 tile, rows j, columns i -------------------------------
     {
       float v[32];
@@ -522,6 +538,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
     fence_before_sync();
     __syncthreads();
 
+    GDN_TRACE_POINT(11);
     // ---- MMA3: S^T += Delta^T (dec K^);  MMA4: Y^T += Delta^T P^T ---------------------
     if (tid == 0) {
       fence_after_sync();
@@ -544,6 +561,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
     if (!__syncthreads_and(ok)) { ok = false; break; }
     fence_after_sync();
 
+    GDN_TRACE_POINT(12);
     // ---- epilogue: Y^T 2^-e -> y (optional RMSNorm x sigmoid(g)) ----------------------
     {
       float v[32];
@@ -584,6 +602,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
     }
     fence_before_sync();
     __syncthreads();
+    GDN_TRACE_POINT(13);
   }
 
   if (ok) {
