@@ -60,26 +60,27 @@ constexpr int kD = 128;   // head dim (d_k = d_v)
 constexpr int kNT = 256;  // threads per CTA
 
 // shared memory map (bytes from a 1024-aligned base)
-constexpr uint32_t OFF_KQ = 0;          // [K; Q] raw bf16 128 x 128, 2 panels x 16 KB
+constexpr uint32_t OFF_KQ = 0;          // [K; Q] raw bf16 128 x 128 (cp.async target), 2 x 16 KB
 constexpr uint32_t OFF_KH = 32768;      // K^ fp16          64 x 128, 2 panels x 8 KB
 constexpr uint32_t OFF_QG = 49152;      // gamma Q^ fp16    64 x 128
 constexpr uint32_t OFF_KT = 65536;      // dec K^ fp16      64 x 128
-constexpr uint32_t OFF_VT = 81920;      // V 2^-e fp16      64 x 128
+constexpr uint32_t OFF_VT = 81920;      // V: raw bf16 (cp.async), then V 2^-e fp16 in place
 constexpr uint32_t OFF_TB = 98304;      // T b 2^-f fp16    64 x 64
 constexpr uint32_t OFF_TBG = 106496;    // T b g 2^-f fp16  64 x 64
 constexpr uint32_t OFF_P = 114688;      // P fp16           64 x 64
-constexpr uint32_t OFF_WT = 122880;     // W^T fp16        128 x 64
-constexpr uint32_t OFF_S0T = 139264;    // S^T 2^-e fp16   128 x 128, 2 panels x 16 KB
+constexpr uint32_t OFF_S0T = 122880;    // S^T 2^-e fp16   128 x 128, 2 panels x 16 KB
+constexpr uint32_t OFF_WT = 155648;     // W^T fp16        128 x 64
 constexpr uint32_t OFF_DT = 172032;     // Delta^T fp16    128 x 64
-// A and T (fp32 64 x 64 each) live in the [K; Q] region, which is dead once
-// MMA0 has completed and is rewritten only after T has been consumed.
-constexpr uint32_t OFF_A = OFF_KQ;
-constexpr uint32_t OFF_T = OFF_KQ + 16384;
-constexpr int kLZ = 52;
-constexpr uint32_t OFF_Z = 188416;                   // Z fp32 [16][52]
-constexpr uint32_t OFF_GATE = OFF_Z + 16 * kLZ * 4;  // G, beta, gamma, dec, rk, rq: 6 x 64
-constexpr uint32_t OFF_RED = OFF_GATE + 6 * 64 * 4;  // red[4][64], rr[64], max[16]
-constexpr uint32_t OFF_BAR = OFF_RED + 5 * 64 * 4 + 64;
+// A and T (fp32 64 x 64) live in the W^T and Delta^T tiles: both are dead
+// between the previous chunk's MMAs and this chunk's W / Delta conversions.
+constexpr uint32_t OFF_A = OFF_WT;
+constexpr uint32_t OFF_T = OFF_DT;
+constexpr uint32_t OFF_GS = 188416;     // g in / y out staging, 2 buffers x [64][128] bf16
+constexpr uint32_t OFF_Z = 221184;      // Z fp32 [1024]
+constexpr uint32_t OFF_GATEBUF = 225280;  // [2 buffers][log alpha, beta][64] fp32
+constexpr uint32_t OFF_GATE = 226304;   // G2, beta, gamma, dec, rk, rq: 6 x 64 fp32
+constexpr uint32_t OFF_RED = 227840;    // red[4][64], rr[64], max[16]
+constexpr uint32_t OFF_BAR = 229248;
 constexpr uint32_t kSmemBytes = OFF_BAR + 64 + 1024;  // + alignment slack
 
 // TMEM columns (fp32, 128 lanes)
@@ -87,6 +88,7 @@ constexpr uint32_t TM_S = 0, TM_KQ = 128, TM_W = 192, TM_D = 256, TM_Y = 320;
 constexpr uint32_t kTmemCols = 512;
 
 constexpr uint32_t kWaitLimit = 1u << 24;
+constexpr float kLog2e = 1.4426950408889634f;
 
 constexpr uint32_t ID_BF_KK = idesc_f16(128, 64, false, false, false, false);  // MMA0
 constexpr uint32_t ID_KK = idesc_f16(128, 64, false, false, false, true);
@@ -135,6 +137,157 @@ __device__ __forceinline__ void st_chunk_f16(uint32_t addr, const float* v, floa
                pack_f16(v[4] * s, v[5] * s), pack_f16(v[6] * s, v[7] * s));
 }
 
+__device__ __forceinline__ float2 bf2_to_f2(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+__device__ __forceinline__ void unpack_bf16x8(const uint4 u, float* f) {
+  float2 p;
+  p = bf2_to_f2(u.x); f[0] = p.x; f[1] = p.y;
+  p = bf2_to_f2(u.y); f[2] = p.x; f[3] = p.y;
+  p = bf2_to_f2(u.z); f[4] = p.x; f[5] = p.y;
+  p = bf2_to_f2(u.w); f[6] = p.x; f[7] = p.y;
+}
+
+
+// One recursive-doubling level of the unit-lower-triangular inverse: for
+// every pair of BS x BS diagonal blocks [[T1, 0], [A21, T2]] of I + A, writes
+// the off-diagonal block X = -T2 (A21 T1) of the inverse.  All 256 threads;
+// each computes an R x 2 (BS >= 16) or 1 x 1 (BS = 8) block of outputs with
+// the sums over m unrolled in steps of 4 (float4 rows of A / T, float2
+// columns of T / Z).  T's strictly upper entries must be zero.
+template <int BS>
+__device__ __forceinline__ void tinv_level(const float* sA, float* sT, float* sZ, int tid) {
+  constexpr int NP = 64 / (2 * BS);                  // pairs
+  constexpr int EPT = NP * BS * BS / kNT;            // outputs per thread
+  constexpr int RC = EPT >= 2 ? 2 : 1;               // columns per thread
+  constexpr int RR = EPT / RC;                       // rows per thread
+  constexpr int CB = BS / RC;                        // column blocks per row
+  constexpr int TPP = (BS / RR) * CB;                // threads per pair
+  const int p = tid / TPP, q = tid % TPP;
+  const int r0 = (q / CB) * RR, c0 = (q % CB) * RC;
+  const int top = 2 * BS * p, bot = top + BS;
+  float acc[RR][RC];
+  // Z = A21 T1
+#pragma unroll
+  for (int i = 0; i < RR; ++i)
+#pragma unroll
+    for (int j = 0; j < RC; ++j) acc[i][j] = 0.f;
+#pragma unroll
+  for (int m = 0; m < BS; m += 4) {
+    float4 ar[RR];
+#pragma unroll
+    for (int i = 0; i < RR; ++i) ar[i] = *reinterpret_cast<const float4*>(sA + fidx(bot + r0 + i, top + m));
+#pragma unroll
+    for (int mm = 0; mm < 4; ++mm) {
+      float tc[RC];
+      if (RC == 2) {
+        const float2 t2 = *reinterpret_cast<const float2*>(sT + fidx(top + m + mm, top + c0));
+        tc[0] = t2.x;
+        tc[RC - 1] = t2.y;
+      } else {
+        tc[0] = sT[fidx(top + m + mm, top + c0)];
+      }
+#pragma unroll
+      for (int i = 0; i < RR; ++i) {
+        const float av = mm == 0 ? ar[i].x : mm == 1 ? ar[i].y : mm == 2 ? ar[i].z : ar[i].w;
+#pragma unroll
+        for (int j = 0; j < RC; ++j) acc[i][j] += av * tc[j];
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < RR; ++i)
+#pragma unroll
+    for (int j = 0; j < RC; ++j) sZ[p * BS * BS + (r0 + i) * BS + c0 + j] = acc[i][j];
+  __syncthreads();
+  // X = -T2 Z
+#pragma unroll
+  for (int i = 0; i < RR; ++i)
+#pragma unroll
+    for (int j = 0; j < RC; ++j) acc[i][j] = 0.f;
+#pragma unroll
+  for (int m = 0; m < BS; m += 4) {
+    float4 tr[RR];
+#pragma unroll
+    for (int i = 0; i < RR; ++i) tr[i] = *reinterpret_cast<const float4*>(sT + fidx(bot + r0 + i, bot + m));
+#pragma unroll
+    for (int mm = 0; mm < 4; ++mm) {
+      float zc[RC];
+      if (RC == 2) {
+        const float2 z2 = *reinterpret_cast<const float2*>(sZ + p * BS * BS + (m + mm) * BS + c0);
+        zc[0] = z2.x;
+        zc[RC - 1] = z2.y;
+      } else {
+        zc[0] = sZ[p * BS * BS + (m + mm) * BS + c0];
+      }
+#pragma unroll
+      for (int i = 0; i < RR; ++i) {
+        const float tv = mm == 0 ? tr[i].x : mm == 1 ? tr[i].y : mm == 2 ? tr[i].z : tr[i].w;
+#pragma unroll
+        for (int j = 0; j < RC; ++j) acc[i][j] -= tv * zc[j];
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < RR; ++i) {
+    if (RC == 2) {
+      *reinterpret_cast<float2*>(sT + fidx(bot + r0 + i, top + c0)) = make_float2(acc[i][0], acc[i][RC - 1]);
+    } else {
+      sT[fidx(bot + r0 + i, top + c0)] = acc[i][0];
+    }
+  }
+  __syncthreads();
+}
+
+struct ChunkLoader {
+  const __nv_bfloat16 *Qg, *Kg, *Vg, *Gg;
+  const float *la, *beta;
+  int H_qk, H_v, h, hq, tid;
+  uint32_t sb;
+  // raw q, k rows of the chunk into the [K; Q] tile (rows >= nn zero filled)
+  __device__ void qk(int64_t c0, int nn) const {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int idx = tid + kNT * k;  // 2048 16-byte pieces
+      const int which = idx >> 10, rr = (idx >> 4) & 63, ch = idx & 15;
+      const bool ok = rr < nn;
+      const __nv_bfloat16* base = which ? Qg : Kg;
+      const __nv_bfloat16* src =
+          base + (ok ? ((size_t)(c0 + rr) * H_qk + hq) * kD + ch * 8 : 0);
+      cp_async16(sb + OFF_KQ + sw128_chunk(which * 64 + rr, ch, 128), src, ok);
+    }
+  }
+  __device__ void v(int64_t c0, int nn) const {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int idx = tid + kNT * k;  // 1024 pieces
+      const int rr = idx >> 4, ch = idx & 15;
+      const bool ok = rr < nn;
+      const __nv_bfloat16* src = Vg + (ok ? ((size_t)(c0 + rr) * H_v + h) * kD + ch * 8 : 0);
+      cp_async16(sb + OFF_VT + sw128_chunk(rr, ch, 64), src, ok);
+    }
+  }
+  __device__ void g(int64_t c0, int nn, int buf) const {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int idx = tid + kNT * k;
+      const int rr = idx >> 4, ch = idx & 15;
+      const bool ok = rr < nn;
+      const __nv_bfloat16* src = Gg + (ok ? ((size_t)(c0 + rr) * H_v + h) * kD + ch * 8 : 0);
+      cp_async16(sb + OFF_GS + buf * 16384 + rr * 256 + ch * 16, src, ok);
+    }
+  }
+  __device__ void gates(int64_t c0, int nn, int buf) const {
+    if (tid < 128) {
+      const int which = tid >> 6, t = tid & 63;
+      const bool ok = t < nn;
+      const float* src = (which ? beta : la) + (ok ? (size_t)(c0 + t) * H_v + h : 0);
+      cp_async4(sb + OFF_GATEBUF + (buf * 2 + which) * 256 + t * 4, src, ok);
+    }
+  }
+};
+
 __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArgs a) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -143,12 +296,13 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
   float* sA = reinterpret_cast<float*>(gb + OFF_A);
   float* sT = reinterpret_cast<float*>(gb + OFF_T);
   float* sZ = reinterpret_cast<float*>(gb + OFF_Z);
-  float* sG = reinterpret_cast<float*>(gb + OFF_GATE);
-  float* sBeta = sG + 64;
-  float* sGam = sG + 128;
-  float* sDec = sG + 192;
-  float* sRk = sG + 256;
-  float* sRq = sG + 320;
+  const float* sGateBuf = reinterpret_cast<const float*>(gb + OFF_GATEBUF);
+  float* sG2 = reinterpret_cast<float*>(gb + OFF_GATE);
+  float* sBeta = sG2 + 64;
+  float* sGam = sG2 + 128;
+  float* sDec = sG2 + 192;
+  float* sRk = sG2 + 256;
+  float* sRq = sG2 + 320;
   float* sRed = reinterpret_cast<float*>(gb + OFF_RED);  // [4][64]
   float* sRr = sRed + 256;                                // [64]
   float* sMax = sRed + 320;                               // [16]
@@ -164,12 +318,33 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
   int64_t t_begin, t_end;
   if (!seq_bounds(a.cu_seqlens, seq, a.total_T, &t_begin, &t_end, a.err)) return;
 
-  const __nv_bfloat16* Qg = static_cast<const __nv_bfloat16*>(a.q);
-  const __nv_bfloat16* Kg = static_cast<const __nv_bfloat16*>(a.k);
-  const __nv_bfloat16* Vg = static_cast<const __nv_bfloat16*>(a.v);
   const __nv_bfloat16* Gg = static_cast<const __nv_bfloat16*>(a.g);
   __nv_bfloat16* Yg = static_cast<__nv_bfloat16*>(a.y);
   const size_t st_off = ((size_t)seq * a.H_v + h) * (size_t)(kD * kD);
+  ChunkLoader ld;
+  ld.Qg = static_cast<const __nv_bfloat16*>(a.q);
+  ld.Kg = static_cast<const __nv_bfloat16*>(a.k);
+  ld.Vg = static_cast<const __nv_bfloat16*>(a.v);
+  ld.Gg = Gg;
+  ld.la = a.log_alpha;
+  ld.beta = a.beta;
+  ld.H_qk = a.H_qk;
+  ld.H_v = a.H_v;
+  ld.h = h;
+  ld.hq = hq;
+  ld.tid = tid;
+  ld.sb = sb;
+  const bool has_g = Gg != nullptr;
+
+  // first chunk's inputs in flight while TMEM and the state are set up
+  if (t_begin < t_end) {
+    const int n0 = (t_end - t_begin) < kC ? (int)(t_end - t_begin) : kC;
+    ld.qk(t_begin, n0);
+    ld.v(t_begin, n0);
+    if (has_g) ld.g(t_begin, n0, 0);
+    ld.gates(t_begin, n0, 0);
+    cp_async_commit();
+  }
 
   if (warp == 0) tmem_alloc(tslot, kTmemCols);
   if (tid == 0) {
@@ -203,23 +378,30 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
 
   uint32_t phase = 0;
   bool ok = true;
-  const bool has_g = Gg != nullptr;
   float wj = 0.f;
   if (has_g && a.norm_w) wj = __ldg(a.norm_w + row);
 
-  for (int64_t c0 = t_begin; c0 < t_end; c0 += kC) {
+  int ci = 0;
+  for (int64_t c0 = t_begin; c0 < t_end; c0 += kC, ++ci) {
     const int n = (t_end - c0) < kC ? (int)(t_end - c0) : kC;
+    const bool has_next = c0 + kC < t_end;
+    const int nn = has_next ? ((t_end - c0 - kC) < kC ? (int)(t_end - c0 - kC) : kC) : 0;
+    const int buf = ci & 1;
 
+    cp_async_wait_all();
+    __syncthreads();
     GDN_TRACE_POINT(0);
-    // ---- gates: cumsum of log alpha, beta, gamma, exp(G_C - G) --------------
+
+    // ---- gates: cumsum of log alpha (log2 units), beta, gamma, exp(G_C - G) ----
     if (warp == 0) {
+      const float* gl = sGateBuf + buf * 128;
       float carry = 0.f;
       float Gv[2], bv[2];
 #pragma unroll
       for (int hb = 0; hb < 2; ++hb) {
         const int t = hb * 32 + lane;
-        float x = t < n ? __ldg(a.log_alpha + (size_t)(c0 + t) * a.H_v + h) : 0.f;
-        bv[hb] = t < n ? __ldg(a.beta + (size_t)(c0 + t) * a.H_v + h) : 0.f;
+        float x = gl[t] * kLog2e;
+        bv[hb] = gl[64 + t];
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
           const float u = __shfl_up_sync(0xffffffffu, x, o);
@@ -228,77 +410,68 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
         Gv[hb] = x + carry;
         carry += __shfl_sync(0xffffffffu, x, 31);
       }
-      const float GC = carry;
 #pragma unroll
       for (int hb = 0; hb < 2; ++hb) {
         const int t = hb * 32 + lane;
-        sG[t] = Gv[hb];
+        sG2[t] = Gv[hb];
         sBeta[t] = bv[hb];
-        sGam[t] = expf(Gv[hb]);
-        sDec[t] = expf(GC - Gv[hb]);
+        sGam[t] = ex2_approx(Gv[hb]);
+        sDec[t] = ex2_approx(carry - Gv[hb]);
       }
     }
-    fence_before_sync();
+    // next chunk's gates and g go into the other buffers now
+    if (has_next) {
+      if (has_g) ld.g(c0 + kC, nn, buf ^ 1);
+      ld.gates(c0 + kC, nn, buf ^ 1);
+    }
+    cp_async_commit();
     __syncthreads();
-    fence_after_sync();
-
     GDN_TRACE_POINT(1);
-    // ---- q, k rows -> operand tiles; v rows kept in registers -----------------
-    // warp w owns rows 8w .. 8w+7; lane l owns columns 4l .. 4l+3
-    float4 vv[8];
+
+    // ---- L2 norms; K^, gamma Q^, dec K^ -> fp16 tiles ---------------------------
+    // warp w owns rows 8w .. 8w+7; 4 lanes per row, 32 columns (4 chunks) each
+    {
+      const int r = warp * 8 + (lane >> 2);
+      const int qc = (lane & 3) * 4;  // first 16-byte chunk of this lane
+      float kf[32], qf[32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        unpack_bf16x8(ld_shared_v4(sb + OFF_KQ + sw128_chunk(r, qc + c, 128)), kf + 8 * c);
+        unpack_bf16x8(ld_shared_v4(sb + OFF_KQ + sw128_chunk(64 + r, qc + c, 128)), qf + 8 * c);
+      }
+      float nk = 0.f, nq = 0.f;
+#pragma unroll
+      for (int x = 0; x < 32; ++x) {
+        nk += kf[x] * kf[x];
+        nq += qf[x] * qf[x];
+      }
+      nk = group_sum<4>(nk);
+      nq = group_sum<4>(nq);
+      const float rk = (a.l2norm && r < n) ? rsqrtf(nk + a.eps_l2) : 1.f;
+      const float rq = (a.l2norm && r < n) ? rsqrtf(nq + a.eps_l2) : 1.f;
+      if ((lane & 3) == 0) {
+        sRk[r] = rk;
+        sRq[r] = rq;
+      }
+      const float gq = sGam[r] * rq, dk = sDec[r] * rk;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        st_chunk_f16(sb + OFF_KH + sw128_chunk(r, qc + c, 64), kf + 8 * c, rk);
+        st_chunk_f16(sb + OFF_QG + sw128_chunk(r, qc + c, 64), qf + 8 * c, gq);
+        st_chunk_f16(sb + OFF_KT + sw128_chunk(r, qc + c, 64), kf + 8 * c, dk);
+      }
+    }
+
+    // ---- block maxima of |V| and |S|, chunk exponent e ---------------------------
+    float vf[32];
     float vmax = 0.f;
 #pragma unroll
-    for (int rp = 0; rp < 2; ++rp) {
-      uint2 kr[4], qr[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int r = warp * 8 + rp * 4 + u;
-        if (r < n) {
-          const size_t qo = ((size_t)(c0 + r) * a.H_qk + hq) * kD + 4 * lane;
-          kr[u] = __ldg(reinterpret_cast<const uint2*>(Kg + qo));
-          qr[u] = __ldg(reinterpret_cast<const uint2*>(Qg + qo));
-          vv[rp * 4 + u] =
-              Elem<__nv_bfloat16>::load4(Vg + ((size_t)(c0 + r) * a.H_v + h) * kD + 4 * lane);
-        } else {
-          kr[u] = qr[u] = make_uint2(0u, 0u);
-          vv[rp * 4 + u] = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int r = warp * 8 + rp * 4 + u;
-        const float2 k01 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&kr[u].x));
-        const float2 k23 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&kr[u].y));
-        const float2 q01 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&qr[u].x));
-        const float2 q23 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&qr[u].y));
-        float nk = k01.x * k01.x + k01.y * k01.y + k23.x * k23.x + k23.y * k23.y;
-        float nq = q01.x * q01.x + q01.y * q01.y + q23.x * q23.x + q23.y * q23.y;
-        nk = warp_sum(nk);
-        nq = warp_sum(nq);
-        const float rk = (a.l2norm && r < n) ? rsqrtf(nk + a.eps_l2) : 1.f;
-        const float rq = (a.l2norm && r < n) ? rsqrtf(nq + a.eps_l2) : 1.f;
-        if (lane == 0) {
-          sRk[r] = rk;
-          sRq[r] = rq;
-        }
-        const int col = 4 * lane;
-        // raw bf16 rows for the exact q.k / k.k products
-        st_shared_v2(sb + OFF_KQ + sw128_off(r, col, 128), kr[u].x, kr[u].y);
-        st_shared_v2(sb + OFF_KQ + sw128_off(64 + r, col, 128), qr[u].x, qr[u].y);
-        const float gq = sGam[r] * rq, dk = sDec[r] * rk;
-        st_shared_v2(sb + OFF_KH + sw128_off(r, col, 64), pack_f16(rk * k01.x, rk * k01.y),
-                     pack_f16(rk * k23.x, rk * k23.y));
-        st_shared_v2(sb + OFF_QG + sw128_off(r, col, 64), pack_f16(gq * q01.x, gq * q01.y),
-                     pack_f16(gq * q23.x, gq * q23.y));
-        st_shared_v2(sb + OFF_KT + sw128_off(r, col, 64), pack_f16(dk * k01.x, dk * k01.y),
-                     pack_f16(dk * k23.x, dk * k23.y));
-        const float4 x = vv[rp * 4 + u];
-        vmax = fmaxf(vmax, fmaxf(fmaxf(fabsf(x.x), fabsf(x.y)), fmaxf(fabsf(x.z), fabsf(x.w))));
-      }
+    for (int k = 0; k < 4; ++k) {
+      const int idx = tid + kNT * k;
+      unpack_bf16x8(ld_shared_v4(sb + OFF_VT + sw128_chunk(idx >> 4, idx & 15, 64)), vf + 8 * k);
     }
-
-    GDN_TRACE_POINT(2);
-    // ---- S^T from TMEM, block maxima, chunk exponent e ---------------------------
+#pragma unroll
+    for (int x = 0; x < 32; ++x) vmax = fmaxf(vmax, fabsf(vf[x]));
     float sv[64];
     tmem_ld32(tS + half * 64, sv);
     tmem_ld32(tS + half * 64 + 32, sv + 32);
@@ -312,15 +485,11 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
     const int e = scale_exp(mV + 12.f * mS, 12);
     {
       const float sv_scale = ldexpf(1.f, -e);
-      // V rows 2^-e -> fp16 tile (rows i, columns j)
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int r = warp * 8 + u;
-        const float4 x = vv[u];
-        st_shared_v2(sb + OFF_VT + sw128_off(r, 4 * lane, 64), pack_f16(x.x * sv_scale, x.y * sv_scale),
-                     pack_f16(x.z * sv_scale, x.w * sv_scale));
+      for (int k = 0; k < 4; ++k) {
+        const int idx = tid + kNT * k;
+        st_chunk_f16(sb + OFF_VT + sw128_chunk(idx >> 4, idx & 15, 64), vf + 8 * k, sv_scale);
       }
-      // S^T 2^-e -> fp16 tile; fp32 state rescaled by gamma_C and to exponent e
       const float to_e = ldexpf(1.f, s_exp - e);
 #pragma unroll
       for (int q = 0; q < 8; ++q)
@@ -336,8 +505,8 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
     fence_proxy_async();
     fence_before_sync();
     __syncthreads();
+    GDN_TRACE_POINT(2);
 
-    GDN_TRACE_POINT(3);
     // ---- MMA0: [K;Q] K^T (bf16, exact);  MMA2: S^T (gamma Q^)^T (fp16) -----------
     if (tid == 0) {
       fence_after_sync();
@@ -358,118 +527,122 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
     phase ^= 1;
     if (!__syncthreads_and(ok)) { ok = false; break; }
     fence_after_sync();
+    // the raw [K; Q] tile is free: next chunk's q, k
+    if (has_next) ld.qk(c0 + kC, nn);
+    cp_async_commit();
+    GDN_TRACE_POINT(3);
 
-    GDN_TRACE_POINT(4);
-    // ---- A (fp32) and P (fp16) from the raw products (warps 0-3) --------------
-    if (tid < 128) {
-      const int t = tid & 63;
-      float v[64];
-      tmem_ld32(tKQ, v);
-      tmem_ld32(tKQ + 32, v + 32);
+    // ---- A (fp32) and P (fp16) from the raw products: all 256 threads -----------
+    {
+      const int t = row & 63;
+      const int i0 = half * 32;
+      float v[32];
+      tmem_ld32(tKQ + i0, v);
       tmem_wait_ld();
-      const float Gt = sG[t];
-      if (tid < 64) {
+      const float Gt = sG2[t];
+      if (row < 64) {
         const float bt = sBeta[t] * sRk[t];
 #pragma unroll
-        for (int i = 0; i < 64; i += 4) {
+        for (int i = 0; i < 32; i += 4) {
           float4 o;
-          o.x = (i + 0 < t) ? bt * sRk[i + 0] * expf(Gt - sG[i + 0]) * v[i + 0] : 0.f;
-          o.y = (i + 1 < t) ? bt * sRk[i + 1] * expf(Gt - sG[i + 1]) * v[i + 1] : 0.f;
-          o.z = (i + 2 < t) ? bt * sRk[i + 2] * expf(Gt - sG[i + 2]) * v[i + 2] : 0.f;
-          o.w = (i + 3 < t) ? bt * sRk[i + 3] * expf(Gt - sG[i + 3]) * v[i + 3] : 0.f;
-          *reinterpret_cast<float4*>(sA + fidx(t, i)) = o;
+          o.x = (i0 + i + 0 < t) ? bt * sRk[i0 + i + 0] * ex2_approx(Gt - sG2[i0 + i + 0]) * v[i + 0] : 0.f;
+          o.y = (i0 + i + 1 < t) ? bt * sRk[i0 + i + 1] * ex2_approx(Gt - sG2[i0 + i + 1]) * v[i + 1] : 0.f;
+          o.z = (i0 + i + 2 < t) ? bt * sRk[i0 + i + 2] * ex2_approx(Gt - sG2[i0 + i + 2]) * v[i + 2] : 0.f;
+          o.w = (i0 + i + 3 < t) ? bt * sRk[i0 + i + 3] * ex2_approx(Gt - sG2[i0 + i + 3]) * v[i + 3] : 0.f;
+          *reinterpret_cast<float4*>(sA + fidx(t, i0 + i)) = o;
         }
       } else {
         const float qt = sRq[t];
 #pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {
+        for (int c8 = 0; c8 < 4; ++c8) {
           uint32_t pk[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const int i0 = 8 * c8 + 2 * u, i1 = i0 + 1;
-            const float p0 = (i0 <= t) ? qt * sRk[i0] * expf(Gt - sG[i0]) * v[i0] : 0.f;
-            const float p1 = (i1 <= t) ? qt * sRk[i1] * expf(Gt - sG[i1]) * v[i1] : 0.f;
+            const int ia = i0 + 8 * c8 + 2 * u, ib = ia + 1;
+            const float p0 = (ia <= t) ? qt * sRk[ia] * ex2_approx(Gt - sG2[ia]) * v[8 * c8 + 2 * u] : 0.f;
+            const float p1 = (ib <= t) ? qt * sRk[ib] * ex2_approx(Gt - sG2[ib]) * v[8 * c8 + 2 * u + 1] : 0.f;
             pk[u] = pack_f16(p0, p1);
           }
-          st_shared_v4(sb + OFF_P + sw128_chunk(t, c8, 64), pk[0], pk[1], pk[2], pk[3]);
+          st_shared_v4(sb + OFF_P + sw128_chunk(t, half * 4 + c8, 64), pk[0], pk[1], pk[2], pk[3]);
         }
       }
     }
+    // T starts from zero (its strictly upper blocks are never computed)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) reinterpret_cast<float4*>(sT)[tid + kNT * k] = make_float4(0.f, 0.f, 0.f, 0.f);
     fence_before_sync();
     __syncthreads();
+    GDN_TRACE_POINT(4);
 
-    GDN_TRACE_POINT(5);
-    // ---- T = (I + A)^{-1}: 16 x 16 diagonal blocks by substitution -------------
+    // ---- T = (I + A)^{-1} by recursive doubling ---------------------------------
+    // 8 x 8 diagonal blocks by substitution, then for block sizes b = 8, 16, 32:
+    //   [[T1, 0], [A21, T2]] -> off-diagonal block X = -T2 (A21 T1)
     if (tid < 64) {
-      const int b = tid >> 4, c = tid & 15;
-      float x[16];
+      const int b = tid >> 3, c = tid & 7;
+      float ab[8][8];
 #pragma unroll
-      for (int r = 0; r < 16; ++r) {
+      for (int r = 1; r < 8; ++r) {
+        const float4 lo = *reinterpret_cast<const float4*>(sA + fidx(8 * b + r, 8 * b));
+        const float4 hi = *reinterpret_cast<const float4*>(sA + fidx(8 * b + r, 8 * b + 4));
+        ab[r][0] = lo.x; ab[r][1] = lo.y; ab[r][2] = lo.z; ab[r][3] = lo.w;
+        ab[r][4] = hi.x; ab[r][5] = hi.y; ab[r][6] = hi.z; ab[r][7] = hi.w;
+      }
+      float x[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
         float s = (r == c) ? 1.f : 0.f;
 #pragma unroll
-        for (int m = 0; m < r; ++m) s -= sA[fidx(16 * b + r, 16 * b + m)] * x[m];
+        for (int m = 0; m < r; ++m) s -= ab[r][m] * x[m];
         x[r] = s;
       }
 #pragma unroll
-      for (int r = 0; r < 16; ++r) sT[fidx(16 * b + r, 16 * b + c)] = x[r];
+      for (int r = 0; r < 8; ++r) sT[fidx(8 * b + r, 8 * b + c)] = x[r];
     }
     __syncthreads();
-    // off-diagonal blocks: T_rc = -T_rr sum_{m=c}^{r-1} A_rm T_mc, block row by row
-#pragma unroll 1
-    for (int rb = 1; rb < 4; ++rb) {
-      const int ncols = 16 * rb, total = 16 * ncols;
-      for (int e2 = tid; e2 < total; e2 += kNT) {
-        const int p = e2 / ncols, q = e2 % ncols;
-        float s = 0.f;
-        for (int m = 16 * (q >> 4); m < 16 * rb; ++m) s += sA[fidx(16 * rb + p, m)] * sT[fidx(m, q)];
-        sZ[p * kLZ + q] = s;
-      }
-      __syncthreads();
-      for (int e2 = tid; e2 < total; e2 += kNT) {
-        const int p = e2 / ncols, q = e2 % ncols;
-        float s = 0.f;
-        for (int u = 0; u <= p; ++u) s += sT[fidx(16 * rb + p, 16 * rb + u)] * sZ[u * kLZ + q];
-        sT[fidx(16 * rb + p, q)] = -s;
-      }
-      __syncthreads();
-    }
+    tinv_level<8>(sA, sT, sZ, tid);
+    tinv_level<16>(sA, sT, sZ, tid);
+    tinv_level<32>(sA, sT, sZ, tid);
+    GDN_TRACE_POINT(5);
 
-    GDN_TRACE_POINT(6);
     // ---- scale exponent of T; T diag(b) 2^-f, T diag(b g) 2^-f -> fp16 ---------
-    float tmax = 0.f;
-    if (tid < 128) {
-      const int t = tid & 63;
-      for (int i = (tid >> 6) * 32; i < (tid >> 6) * 32 + 32; ++i)
-        if (i <= t) tmax = fmaxf(tmax, fabsf(sT[fidx(t, i)]));
-    }
-    const int f = max(0, scale_exp(block_max(tmax, sMax, warp, lane), 8));
-    if (tid < 128) {
-      const int t = tid & 63;
-      const bool withg = tid >= 64;
+    {
+      const int t = row & 63;
+      const bool withg = row >= 64;
+      float tv[32];
+      float tmax = 0.f;
+#pragma unroll
+      for (int i = 0; i < 32; i += 4) {
+        const float4 x = *reinterpret_cast<const float4*>(sT + fidx(t, half * 32 + i));
+        tv[i] = x.x; tv[i + 1] = x.y; tv[i + 2] = x.z; tv[i + 3] = x.w;
+        tmax = fmaxf(tmax, fmaxf(fmaxf(fabsf(x.x), fabsf(x.y)), fmaxf(fabsf(x.z), fabsf(x.w))));
+      }
+      const int f = max(0, scale_exp(block_max(tmax, sMax, warp, lane), 8));
       const float sf = ldexpf(1.f, -f);
 #pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) {
+      for (int c8 = 0; c8 < 4; ++c8) {
         uint32_t pk[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const int i0 = 8 * c8 + 2 * u, i1 = i0 + 1;
-          float x0 = (i0 <= t) ? sT[fidx(t, i0)] * sBeta[i0] * sf : 0.f;
-          float x1 = (i1 <= t) ? sT[fidx(t, i1)] * sBeta[i1] * sf : 0.f;
+          const int ia = half * 32 + 8 * c8 + 2 * u;
+          float x0 = tv[8 * c8 + 2 * u] * sBeta[ia] * sf;
+          float x1 = tv[8 * c8 + 2 * u + 1] * sBeta[ia + 1] * sf;
           if (withg) {
-            x0 *= sGam[i0];
-            x1 *= sGam[i1];
+            x0 *= sGam[ia];
+            x1 *= sGam[ia + 1];
           }
           pk[u] = pack_f16(x0, x1);
         }
-        st_shared_v4(sb + (withg ? OFF_TBG : OFF_TB) + sw128_chunk(t, c8, 64), pk[0], pk[1],
-                     pk[2], pk[3]);
+        st_shared_v4(sb + (withg ? OFF_TBG : OFF_TB) + sw128_chunk(t, half * 4 + c8, 64), pk[0],
+                     pk[1], pk[2], pk[3]);
       }
+      if (tid == 0) sMax[8] = (float)f;
     }
     fence_proxy_async();
     fence_before_sync();
     __syncthreads();
+    const int f = (int)sMax[8];
+    GDN_TRACE_POINT(6);
 
-    GDN_TRACE_POINT(7);
     // ---- MMAW: W^T = K^T (T diag(b g))^T;  MMAU: U^T = V^T (T diag(b))^T -------
     if (tid == 0) {
       fence_after_sync();
@@ -491,8 +664,11 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
     phase ^= 1;
     if (!__syncthreads_and(ok)) { ok = false; break; }
     fence_after_sync();
+    // the V tile is free: next chunk's v
+    if (has_next) ld.v(c0 + kC, nn);
+    cp_async_commit();
+    GDN_TRACE_POINT(7);
 
-    GDN_TRACE_POINT(8);
     // ---- W^T 2^-f (fp32) -> fp16 tile, rows d, columns t ------------------------
     {
       float v[32];
@@ -505,8 +681,8 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
     fence_proxy_async();
     fence_before_sync();
     __syncthreads();
+    GDN_TRACE_POINT(8);
 
-    GDN_TRACE_POINT(9);
     // ---- MMA1: Delta^T 2^-(e+f) = U^T - S^T W^T ---------------------------------------
     if (tid == 0) {
       fence_after_sync();
@@ -522,8 +698,8 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
     phase ^= 1;
     if (!__syncthreads_and(ok)) { ok = false; break; }
     fence_after_sync();
+    GDN_TRACE_POINT(9);
 
-    GDN_TRACE_POINT(10);
     // ---- Delta^T 2^-e -> fp16 tile, rows j, columns i -------------------------------
     {
       float v[32];
@@ -537,8 +713,8 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
     fence_proxy_async();
     fence_before_sync();
     __syncthreads();
+    GDN_TRACE_POINT(10);
 
-    GDN_TRACE_POINT(11);
     // ---- MMA3: S^T += Delta^T (dec K^);  MMA4: Y^T += Delta^T P^T ---------------------
     if (tid == 0) {
       fence_after_sync();
@@ -560,9 +736,9 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
     phase ^= 1;
     if (!__syncthreads_and(ok)) { ok = false; break; }
     fence_after_sync();
+    GDN_TRACE_POINT(11);
 
-    GDN_TRACE_POINT(12);
-    // ---- epilogue: Y^T 2^-e -> y (optional RMSNorm x sigmoid(g)) ----------------------
+    // ---- epilogue: Y^T 2^-e -> y through the staging buffer ----------------------------
     {
       float v[32];
       tmem_ld32(tY + half * 32, v);
@@ -586,24 +762,33 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
                                 (float)kD + a.eps_norm);
         __syncthreads();
       }
-#pragma unroll 4
+      __nv_bfloat16* gs = reinterpret_cast<__nv_bfloat16*>(gb + OFF_GS + buf * 16384);
+      const float w1 = 1.f + wj;
+#pragma unroll
       for (int x = 0; x < 32; ++x) {
         const int t = half * 32 + x;
-        if (t < n) {
-          const size_t yo = ((size_t)(c0 + t) * a.H_v + h) * kD + row;
-          float o = v[x];
-          if (has_g) {
-            const float gg = __bfloat162float(Gg[yo]);
-            o = o * sRr[t] * (1.f + wj) / (1.f + __expf(-gg));
-          }
-          Yg[yo] = __float2bfloat16_rn(o);
+        float o = v[x];
+        if (has_g) {
+          const float gg = __bfloat162float(gs[t * kD + row]);
+          o = __fdividef(o * sRr[t] * w1, 1.f + __expf(-gg));
+        }
+        gs[t * kD + row] = __float2bfloat16_rn(o);
+      }
+      __syncthreads();
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int idx = tid + kNT * k;
+        const int rr = idx >> 4, ch = idx & 15;
+        if (rr < n) {
+          const uint4 val = ld_shared_v4(sb + OFF_GS + buf * 16384 + rr * 256 + ch * 16);
+          *reinterpret_cast<uint4*>(Yg + ((size_t)(c0 + rr) * a.H_v + h) * kD + ch * 8) = val;
         }
       }
     }
     fence_before_sync();
-    __syncthreads();
-    GDN_TRACE_POINT(13);
+    GDN_TRACE_POINT(12);
   }
+  cp_async_wait_all();
 
   if (ok) {
     // final state from TMEM, undoing the state exponent
