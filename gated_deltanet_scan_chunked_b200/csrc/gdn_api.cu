@@ -71,7 +71,8 @@ extern "C" gdn_status gdn_chunk_fwd_path(
     const size_t bytes = (size_t)n_seq * H_v * d_k * d_v * sizeof(float);
     if (a0 < b0 + bytes && b0 < a0 + bytes) return GDN_ERR_INVALID_ARG;
   }
-  if (path != GDN_PATH_AUTO && path != GDN_PATH_TENSOR && path != GDN_PATH_SIMT)
+  if (path != GDN_PATH_AUTO && path != GDN_PATH_TENSOR && path != GDN_PATH_SIMT &&
+      path != GDN_PATH_TENSOR_PAIR && path != GDN_PATH_TENSOR_SINGLE)
     return GDN_ERR_INVALID_ARG;
 
   PrefillArgs a;
@@ -81,13 +82,16 @@ extern "C" gdn_status gdn_chunk_fwd_path(
   a.y = y; a.n_seq = n_seq; a.total_T = total_T;
   a.H_qk = H_qk; a.H_v = H_v; a.d_k = d_k; a.d_v = d_v; a.dtype = in_dtype;
   a.l2norm = l2norm_qk ? 1 : 0; a.eps_l2 = eps_l2; a.eps_norm = eps_norm; a.scale = scale;
-  a.err = error_word_ptr();
-  if (a.err == nullptr) return GDN_ERR_CUDA;
+  a.tc_variant = path == GDN_PATH_TENSOR_PAIR ? 1 : (path == GDN_PATH_TENSOR_SINGLE ? 2 : 0);
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool tc_ok = prefill_tc_supports(a);
-  if (path == GDN_PATH_TENSOR && !tc_ok) return GDN_ERR_UNSUPPORTED;
-  if (path == GDN_PATH_TENSOR || (path == GDN_PATH_AUTO && tc_ok)) return launch_prefill_tc(a, s);
+  const bool want_tc = path == GDN_PATH_TENSOR || path == GDN_PATH_TENSOR_PAIR ||
+                       path == GDN_PATH_TENSOR_SINGLE;
+  if (want_tc && !tc_ok) return GDN_ERR_UNSUPPORTED;
+  a.err = error_word_ptr();
+  if (a.err == nullptr) return GDN_ERR_CUDA;
+  if (want_tc || (path == GDN_PATH_AUTO && tc_ok)) return launch_prefill_tc(a, s);
   return launch_prefill_simt(a, s);
 }
 

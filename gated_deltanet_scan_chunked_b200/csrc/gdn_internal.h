@@ -34,6 +34,7 @@ struct PrefillArgs {
   int32_t l2norm;
   float eps_l2, eps_norm, scale;
   int* err;                // device error word
+  int tc_variant;          // tensor kernel: 0 auto, 1 CTA pairs, 2 one CTA per head
 };
 
 struct DecodeArgs {

@@ -245,6 +245,7 @@ struct ChunkLoader {
   const float *la, *beta;
   int H_qk, H_v, h, hq, tid;
   uint32_t sb;
+  uint32_t off_kq = OFF_KQ, off_vt = OFF_VT, off_gs = OFF_GS, off_gate = OFF_GATEBUF;
   // raw q, k rows of the chunk into the [K; Q] tile (rows >= nn zero filled)
   __device__ void qk(int64_t c0, int nn) const {
 #pragma unroll
@@ -255,7 +256,7 @@ struct ChunkLoader {
       const __nv_bfloat16* base = which ? Qg : Kg;
       const __nv_bfloat16* src =
           base + (ok ? ((size_t)(c0 + rr) * H_qk + hq) * kD + ch * 8 : 0);
-      cp_async16(sb + OFF_KQ + sw128_chunk(which * 64 + rr, ch, 128), src, ok);
+      cp_async16(sb + off_kq + sw128_chunk(which * 64 + rr, ch, 128), src, ok);
     }
   }
   __device__ void v(int64_t c0, int nn) const {
@@ -265,7 +266,7 @@ struct ChunkLoader {
       const int rr = idx >> 4, ch = idx & 15;
       const bool ok = rr < nn;
       const __nv_bfloat16* src = Vg + (ok ? ((size_t)(c0 + rr) * H_v + h) * kD + ch * 8 : 0);
-      cp_async16(sb + OFF_VT + sw128_chunk(rr, ch, 64), src, ok);
+      cp_async16(sb + off_vt + sw128_chunk(rr, ch, 64), src, ok);
     }
   }
   __device__ void g(int64_t c0, int nn, int buf) const {
@@ -275,7 +276,7 @@ struct ChunkLoader {
       const int rr = idx >> 4, ch = idx & 15;
       const bool ok = rr < nn;
       const __nv_bfloat16* src = Gg + (ok ? ((size_t)(c0 + rr) * H_v + h) * kD + ch * 8 : 0);
-      cp_async16(sb + OFF_GS + buf * 16384 + rr * 256 + ch * 16, src, ok);
+      cp_async16(sb + off_gs + buf * 16384 + rr * 256 + ch * 16, src, ok);
     }
   }
   __device__ void gates(int64_t c0, int nn, int buf) const {
@@ -283,7 +284,7 @@ struct ChunkLoader {
       const int which = tid >> 6, t = tid & 63;
       const bool ok = t < nn;
       const float* src = (which ? beta : la) + (ok ? (size_t)(c0 + t) * H_v + h : 0);
-      cp_async4(sb + OFF_GATEBUF + (buf * 2 + which) * 256 + t * 4, src, ok);
+      cp_async4(sb + off_gate + (buf * 2 + which) * 256 + t * 4, src, ok);
     }
   }
 };
@@ -815,6 +816,636 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
   if (warp == 0) tmem_dealloc(tbase, kTmemCols);
 }
 
+// ============================================================================
+// CTA-pair variant: one 2-CTA cluster per (sequence, value head).  CTA 1
+// ("prep") does everything that does not depend on the state -- L2 norms,
+// [K; Q] K^T, A and P, the triangular inverse, W -- and ships the chain's
+// operand tiles (dec K^, gamma Q^, W^T, P, T diag(beta): 64 KB per chunk,
+// double-buffered) into CTA 0's shared memory with bulk copies
+// (shared::cta -> shared::cluster, no multicast).  CTA 0 ("chain") keeps the
+// state in TMEM and runs U, Delta, Y, the state update and the epilogue.
+// Buffer hand-off: "full" barriers in CTA 0 (arrive + expected bytes from
+// CTA 1, completed by the copies), "empty" barriers in CTA 1 (arrived by
+// CTA 0 once its MMAs have read the buffer).  Every wait is bounded.
+// ============================================================================
+
+// chain CTA (rank 0) shared memory
+constexpr uint32_t SH_KT = 0, SH_QG = 16384, SH_WT = 32768, SH_P = 49152, SH_TB = 57344;
+constexpr uint32_t kShipBytes = 65536;
+constexpr uint32_t C_SHIP = 0;            // 2 x 64 KB
+constexpr uint32_t C_VT = 131072;         // V raw -> fp16
+constexpr uint32_t C_S0T = 147456;        // S^T fp16
+constexpr uint32_t C_DT = 180224;         // Delta^T fp16
+constexpr uint32_t C_GS = 196608;         // g in / y out staging
+constexpr uint32_t C_SCAL = 212992;       // shipped scalars [2][4]
+constexpr uint32_t C_RED = 213248;        // red[4][64], rr[64], max[16]
+constexpr uint32_t C_BAR = 214656;        // full[2], mma, tmem slot
+// prep CTA (rank 1) shared memory
+constexpr uint32_t P_KQ = 0;              // raw [K; Q] bf16
+constexpr uint32_t P_KH = 32768;          // K^ fp16
+constexpr uint32_t P_TBG = 49152;         // T diag(b g) 2^-f fp16
+constexpr uint32_t P_A = 57344;           // A fp32
+constexpr uint32_t P_T = 73728;           // T fp32
+constexpr uint32_t P_STG = 90112;         // ship staging, 2 x 64 KB
+constexpr uint32_t P_Z = 221184;          // Z fp32 [1024]
+constexpr uint32_t P_GATEBUF = 225280;    // [2][la, beta][64]
+constexpr uint32_t P_GATE = 226304;       // G2, beta, gamma, dec, rk, rq
+constexpr uint32_t P_SCAL = 227840;       // scalar staging [2][4]
+constexpr uint32_t P_MAX = 227872;        // block-max scratch [16]
+constexpr uint32_t P_BAR = 227936;        // empty[2], mma, tmem slot
+constexpr uint32_t kPairSmemBytes = 228000 + 1024;
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNT, 1)
+    gdn_prefill_tc_pair_kernel(const PrefillArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sb = (raw + 1023u) & ~1023u;
+  uint8_t* gb = smem_raw + (sb - raw);
+  const uint32_t rank = cluster_ctarank();
+  const int item = blockIdx.x >> 1;
+  const int seq = item / a.H_v;
+  const int h = item % a.H_v;
+  const int hq = h / (a.H_v / a.H_qk);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int row = tid & 127;
+  const int half = tid >> 7;
+  int64_t t_begin, t_end;
+  // both CTAs see the same bounds, so both leave before touching the other
+  if (!seq_bounds(a.cu_seqlens, seq, a.total_T, &t_begin, &t_end, rank == 0 ? a.err : nullptr))
+    return;
+  const bool has_g = a.g != nullptr;
+  ChunkLoader ld;
+  ld.Qg = static_cast<const __nv_bfloat16*>(a.q);
+  ld.Kg = static_cast<const __nv_bfloat16*>(a.k);
+  ld.Vg = static_cast<const __nv_bfloat16*>(a.v);
+  ld.Gg = static_cast<const __nv_bfloat16*>(a.g);
+  ld.la = a.log_alpha;
+  ld.beta = a.beta;
+  ld.H_qk = a.H_qk;
+  ld.H_v = a.H_v;
+  ld.h = h;
+  ld.hq = hq;
+  ld.tid = tid;
+  ld.sb = sb;
+  ld.off_kq = P_KQ;
+  ld.off_vt = C_VT;
+  ld.off_gs = C_GS;
+  ld.off_gate = P_GATEBUF;
+  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+  uint32_t phase = 0;
+  bool ok = true;
+
+  if (rank == 0) {
+    // =========================== chain CTA ===========================
+    uint64_t* full = reinterpret_cast<uint64_t*>(gb + C_BAR);
+    uint64_t* mbar = reinterpret_cast<uint64_t*>(gb + C_BAR + 16);
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(gb + C_BAR + 24);
+    float* sRed = reinterpret_cast<float*>(gb + C_RED);
+    float* sRr = sRed + 256;
+    float* sMax = sRed + 320;
+    const float* sScal = reinterpret_cast<const float*>(gb + C_SCAL);
+    __nv_bfloat16* Yg = static_cast<__nv_bfloat16*>(a.y);
+    const size_t st_off = ((size_t)seq * a.H_v + h) * (size_t)(kD * kD);
+    if (t_begin < t_end) {
+      const int n0 = (t_end - t_begin) < kC ? (int)(t_end - t_begin) : kC;
+      ld.v(t_begin, n0);
+      if (has_g) ld.g(t_begin, n0, 0);
+      cp_async_commit();
+    }
+    if (warp == 0) tmem_alloc(tslot, 256);
+    if (tid == 0) {
+      mbar_init(&full[0], 1);
+      mbar_init(&full[1], 1);
+      mbar_init(mbar, 1);
+      fence_mbar_init();
+    }
+    fence_before_sync();
+    __syncthreads();
+    cluster_sync();
+    fence_after_sync();
+    const uint32_t tbase = *tslot;
+    const uint32_t tS = tbase + lane_off, tD = tbase + lane_off + 128, tY = tbase + lane_off + 192;
+    {
+      float v[32];
+#pragma unroll
+      for (int cb = 0; cb < 2; ++cb) {
+        const int d0 = half * 64 + cb * 32;
+#pragma unroll
+        for (int x = 0; x < 32; ++x)
+          v[x] = a.initial_state ? __ldg(a.initial_state + st_off + (size_t)(d0 + x) * kD + row)
+                                 : 0.f;
+        tmem_st32(tS + d0, v);
+      }
+      tmem_wait_st();
+    }
+    int s_exp = 0;
+    const float w1 = 1.f + ((has_g && a.norm_w) ? __ldg(a.norm_w + row) : 0.f);
+
+    int ci = 0;
+    for (int64_t c0 = t_begin; c0 < t_end; c0 += kC, ++ci) {
+      const int n = (t_end - c0) < kC ? (int)(t_end - c0) : kC;
+      const bool has_next = c0 + kC < t_end;
+      const int nn = has_next ? ((t_end - c0 - kC) < kC ? (int)(t_end - c0 - kC) : kC) : 0;
+      const int b = ci & 1;
+      const uint32_t ship = sb + C_SHIP + b * kShipBytes;
+      cp_async_wait_all();
+      __syncthreads();
+      GDN_TRACE_POINT(0);
+      bool okw = mbar_wait_cluster(&full[b], (ci >> 1) & 1, kWaitLimit);
+      if (!__syncthreads_and(okw)) { ok = false; break; }
+      GDN_TRACE_POINT(1);
+      const float gC = sScal[b * 4 + 0];
+      const int f = (int)sScal[b * 4 + 1];
+
+      // V, S maxima -> e; V 2^-e and S^T 2^-e to fp16; state rescaled
+      float vf[32];
+      float vmax = 0.f;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int idx = tid + kNT * k;
+        unpack_bf16x8(ld_shared_v4(sb + C_VT + sw128_chunk(idx >> 4, idx & 15, 64)), vf + 8 * k);
+      }
+#pragma unroll
+      for (int x = 0; x < 32; ++x) vmax = fmaxf(vmax, fabsf(vf[x]));
+      float sv[64];
+      tmem_ld32(tS + half * 64, sv);
+      tmem_ld32(tS + half * 64 + 32, sv + 32);
+      tmem_wait_ld();
+      float smax = 0.f;
+#pragma unroll
+      for (int x = 0; x < 64; ++x) smax = fmaxf(smax, fabsf(sv[x]));
+      const float mV = block_max(vmax, sMax, warp, lane);
+      const float mS = ldexpf(block_max(smax, sMax, warp, lane), s_exp);
+      const int e = scale_exp(mV + 12.f * mS, 12);
+      {
+        const float sv_scale = ldexpf(1.f, -e);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int idx = tid + kNT * k;
+          st_chunk_f16(sb + C_VT + sw128_chunk(idx >> 4, idx & 15, 64), vf + 8 * k, sv_scale);
+        }
+        const float to_e = ldexpf(1.f, s_exp - e);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          st_chunk_f16(sb + C_S0T + sw128_chunk(row, half * 8 + q, 128), sv + 8 * q, to_e);
+        const float upd = gC * to_e;
+#pragma unroll
+        for (int x = 0; x < 64; ++x) sv[x] *= upd;
+        tmem_st32(tS + half * 64, sv);
+        tmem_st32(tS + half * 64 + 32, sv + 32);
+        tmem_wait_st();
+        s_exp = e;
+      }
+      fence_proxy_async();
+      fence_before_sync();
+      __syncthreads();
+      GDN_TRACE_POINT(2);
+
+      // U^T = V^T (T diag b)^T;  Y^T = S^T (gamma Q^)^T;  Delta^T = U^T - S^T W^T
+      if (tid == 0) {
+        fence_after_sync();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t da = sdesc(sb + C_VT + kk * 2048, 8192, 1024);
+          const uint64_t db = sdesc(ship + SH_TB + kk * 32, 16, 1024);
+          mma_f16(tbase + 128, da, db, ID_MK, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t da = sdesc(sb + C_S0T + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+          const uint64_t db = sdesc(ship + SH_QG + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+          mma_f16(tbase + 192, da, db, ID_KK, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t da = sdesc(sb + C_S0T + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+          const uint64_t db = sdesc(ship + SH_WT + kk * 2048, 16384, 1024);
+          mma_f16(tbase + 128, da, db, ID_KM_NEG, 1);
+        }
+        mma_commit(mbar);
+      }
+      okw = mbar_wait(mbar, phase, kWaitLimit);
+      phase ^= 1;
+      if (!__syncthreads_and(okw)) { ok = false; break; }
+      fence_after_sync();
+      if (has_next) ld.v(c0 + kC, nn);
+      cp_async_commit();
+      GDN_TRACE_POINT(3);
+
+      // Delta^T 2^-e -> fp16 tile
+      {
+        float v[32];
+        tmem_ld32(tD + half * 32, v);
+        tmem_wait_ld();
+        const float sf = ldexpf(1.f, f);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          st_chunk_f16(sb + C_DT + sw128_chunk(row, half * 4 + q, 128), v + 8 * q, sf);
+      }
+      fence_proxy_async();
+      fence_before_sync();
+      __syncthreads();
+      GDN_TRACE_POINT(4);
+
+      // S^T += Delta^T (dec K^);  Y^T += Delta^T P^T
+      if (tid == 0) {
+        fence_after_sync();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t da = sdesc(sb + C_DT + kk * 32, 16, 1024);
+          const uint64_t db = sdesc(ship + SH_KT + kk * 2048, 8192, 1024);
+          mma_f16(tbase, da, db, ID_KM128, 1);
+        }
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t da = sdesc(sb + C_DT + kk * 32, 16, 1024);
+          const uint64_t db = sdesc(ship + SH_P + kk * 32, 16, 1024);
+          mma_f16(tbase + 192, da, db, ID_KK, 1);
+        }
+        mma_commit(mbar);
+      }
+      okw = mbar_wait(mbar, phase, kWaitLimit);
+      phase ^= 1;
+      if (!__syncthreads_and(okw)) { ok = false; break; }
+      fence_after_sync();
+      // this chunk's shipped tiles are no longer read: hand the buffer back
+      if (tid == 0) mbar_remote_arrive(mapa_shared(sb + P_BAR + 8 * b, 1));
+      GDN_TRACE_POINT(5);
+
+      // epilogue
+      {
+        float v[32];
+        tmem_ld32(tY + half * 32, v);
+        tmem_wait_ld();
+        const float ys = ldexpf(a.scale, e);
+#pragma unroll
+        for (int x = 0; x < 32; ++x) v[x] *= ys;
+        if (has_g) {
+          float s2[32];
+#pragma unroll
+          for (int x = 0; x < 32; ++x) s2[x] = v[x] * v[x];
+          rs_stage(s2, 16, lane);
+          rs_stage(s2, 8, lane);
+          rs_stage(s2, 4, lane);
+          rs_stage(s2, 2, lane);
+          rs_stage(s2, 1, lane);
+          sRed[(warp & 3) * 64 + half * 32 + lane] = s2[0];
+          __syncthreads();
+          if (tid < 64)
+            sRr[tid] = rsqrtf((sRed[tid] + sRed[64 + tid] + sRed[128 + tid] + sRed[192 + tid]) /
+                                  (float)kD + a.eps_norm);
+          __syncthreads();
+        }
+        __nv_bfloat16* gs = reinterpret_cast<__nv_bfloat16*>(gb + C_GS);
+#pragma unroll
+        for (int x = 0; x < 32; ++x) {
+          const int t = half * 32 + x;
+          float o = v[x];
+          if (has_g) {
+            const float gg = __bfloat162float(gs[t * kD + row]);
+            o = __fdividef(o * sRr[t] * w1, 1.f + __expf(-gg));
+          }
+          gs[t * kD + row] = __float2bfloat16_rn(o);
+        }
+        __syncthreads();
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int idx = tid + kNT * k;
+          const int rr = idx >> 4, ch = idx & 15;
+          if (rr < n) {
+            const uint4 val = ld_shared_v4(sb + C_GS + rr * 256 + ch * 16);
+            *reinterpret_cast<uint4*>(Yg + ((size_t)(c0 + rr) * a.H_v + h) * kD + ch * 8) = val;
+          }
+        }
+        __syncthreads();
+        if (has_next && has_g) ld.g(c0 + kC, nn, 0);
+        cp_async_commit();
+      }
+      fence_before_sync();
+      GDN_TRACE_POINT(6);
+    }
+    cp_async_wait_all();
+    if (ok) {
+      if (a.final_state) {
+        const float sc = ldexpf(1.f, s_exp);
+        float v[32];
+#pragma unroll 1
+        for (int cb = 0; cb < 2; ++cb) {
+          const int d0 = half * 64 + cb * 32;
+          tmem_ld32(tS + d0, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int x = 0; x < 32; ++x)
+            a.final_state[st_off + (size_t)(d0 + x) * kD + row] = v[x] * sc;
+        }
+      }
+    } else {
+      if (tid == 0) atomicOr(a.err, kErrTimeout);
+      mbar_wait(mbar, phase ^ 1, kWaitLimit);
+    }
+    fence_before_sync();
+    __syncthreads();
+    cluster_sync();
+    if (warp == 0) tmem_dealloc(tbase, 256);
+  } else {
+    // =========================== prep CTA ============================
+    uint64_t* empty = reinterpret_cast<uint64_t*>(gb + P_BAR);
+    uint64_t* mbar = reinterpret_cast<uint64_t*>(gb + P_BAR + 16);
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(gb + P_BAR + 24);
+    float* sA = reinterpret_cast<float*>(gb + P_A);
+    float* sT = reinterpret_cast<float*>(gb + P_T);
+    float* sZ = reinterpret_cast<float*>(gb + P_Z);
+    const float* sGateBuf = reinterpret_cast<const float*>(gb + P_GATEBUF);
+    float* sG2 = reinterpret_cast<float*>(gb + P_GATE);
+    float* sBeta = sG2 + 64;
+    float* sGam = sG2 + 128;
+    float* sDec = sG2 + 192;
+    float* sRk = sG2 + 256;
+    float* sRq = sG2 + 320;
+    float* sScal = reinterpret_cast<float*>(gb + P_SCAL);
+    float* sMax = reinterpret_cast<float*>(gb + P_MAX);
+    if (t_begin < t_end) {
+      const int n0 = (t_end - t_begin) < kC ? (int)(t_end - t_begin) : kC;
+      ld.qk(t_begin, n0);
+      ld.gates(t_begin, n0, 0);
+      cp_async_commit();
+    }
+    if (warp == 0) tmem_alloc(tslot, 128);
+    if (tid == 0) {
+      mbar_init(&empty[0], 1);
+      mbar_init(&empty[1], 1);
+      mbar_init(mbar, 1);
+      fence_mbar_init();
+    }
+    fence_before_sync();
+    __syncthreads();
+    cluster_sync();
+    fence_after_sync();
+    const uint32_t tbase = *tslot;
+    const uint32_t tKQ = tbase + lane_off, tW = tbase + lane_off + 64;
+    const uint32_t full_cl0 = mapa_shared(sb + C_BAR, 0);
+    const uint32_t ship_cl0 = mapa_shared(sb + C_SHIP, 0);
+    const uint32_t scal_cl0 = mapa_shared(sb + C_SCAL, 0);
+
+    int ci = 0;
+    for (int64_t c0 = t_begin; c0 < t_end; c0 += kC, ++ci) {
+      const int n = (t_end - c0) < kC ? (int)(t_end - c0) : kC;
+      const bool has_next = c0 + kC < t_end;
+      const int nn = has_next ? ((t_end - c0 - kC) < kC ? (int)(t_end - c0 - kC) : kC) : 0;
+      const int b = ci & 1;
+      const uint32_t stg = sb + P_STG + b * kShipBytes;
+      cp_async_wait_all();
+      if (tid == 0) bulk_wait_read_le1();  // staging buffer b is no longer being copied
+      __syncthreads();
+
+      // gates
+      if (warp == 0) {
+        const float* gl = sGateBuf + b * 128;
+        float carry = 0.f;
+        float Gv[2], bv[2];
+#pragma unroll
+        for (int hb = 0; hb < 2; ++hb) {
+          const int t = hb * 32 + lane;
+          float x = gl[t] * kLog2e;
+          bv[hb] = gl[64 + t];
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const float u = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += u;
+          }
+          Gv[hb] = x + carry;
+          carry += __shfl_sync(0xffffffffu, x, 31);
+        }
+#pragma unroll
+        for (int hb = 0; hb < 2; ++hb) {
+          const int t = hb * 32 + lane;
+          sG2[t] = Gv[hb];
+          sBeta[t] = bv[hb];
+          sGam[t] = ex2_approx(Gv[hb]);
+          sDec[t] = ex2_approx(carry - Gv[hb]);
+        }
+        if (lane == 0) sScal[b * 4 + 0] = ex2_approx(carry);
+      }
+      if (has_next) ld.gates(c0 + kC, nn, b ^ 1);
+      cp_async_commit();
+      __syncthreads();
+
+      // norms -> K^ (local), gamma Q^ and dec K^ (shipped)
+      {
+        const int r = warp * 8 + (lane >> 2);
+        const int qc = (lane & 3) * 4;
+        float kf[32], qf[32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          unpack_bf16x8(ld_shared_v4(sb + P_KQ + sw128_chunk(r, qc + c, 128)), kf + 8 * c);
+          unpack_bf16x8(ld_shared_v4(sb + P_KQ + sw128_chunk(64 + r, qc + c, 128)), qf + 8 * c);
+        }
+        float nk = 0.f, nq = 0.f;
+#pragma unroll
+        for (int x = 0; x < 32; ++x) {
+          nk += kf[x] * kf[x];
+          nq += qf[x] * qf[x];
+        }
+        nk = group_sum<4>(nk);
+        nq = group_sum<4>(nq);
+        const float rk = (a.l2norm && r < n) ? rsqrtf(nk + a.eps_l2) : 1.f;
+        const float rq = (a.l2norm && r < n) ? rsqrtf(nq + a.eps_l2) : 1.f;
+        if ((lane & 3) == 0) {
+          sRk[r] = rk;
+          sRq[r] = rq;
+        }
+        const float gq = sGam[r] * rq, dk = sDec[r] * rk;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          st_chunk_f16(sb + P_KH + sw128_chunk(r, qc + c, 64), kf + 8 * c, rk);
+          st_chunk_f16(stg + SH_QG + sw128_chunk(r, qc + c, 64), qf + 8 * c, gq);
+          st_chunk_f16(stg + SH_KT + sw128_chunk(r, qc + c, 64), kf + 8 * c, dk);
+        }
+      }
+      fence_proxy_async();
+      fence_before_sync();
+      __syncthreads();
+
+      // [K; Q] K^T on the raw inputs
+      if (tid == 0) {
+        fence_after_sync();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t d = sdesc(sb + P_KQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+          mma_f16(tbase, d, d, ID_BF_KK, kk > 0);
+        }
+        mma_commit(mbar);
+      }
+      bool okw = mbar_wait(mbar, phase, kWaitLimit);
+      phase ^= 1;
+      if (!__syncthreads_and(okw)) { ok = false; break; }
+      fence_after_sync();
+      if (has_next) ld.qk(c0 + kC, nn);
+      cp_async_commit();
+
+      // A (fp32) and P (fp16, shipped)
+      {
+        const int t = row & 63;
+        const int i0 = half * 32;
+        float v[32];
+        tmem_ld32(tKQ + i0, v);
+        tmem_wait_ld();
+        const float Gt = sG2[t];
+        if (row < 64) {
+          const float bt = sBeta[t] * sRk[t];
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            float4 o;
+            o.x = (i0 + i + 0 < t) ? bt * sRk[i0 + i + 0] * ex2_approx(Gt - sG2[i0 + i + 0]) * v[i + 0] : 0.f;
+            o.y = (i0 + i + 1 < t) ? bt * sRk[i0 + i + 1] * ex2_approx(Gt - sG2[i0 + i + 1]) * v[i + 1] : 0.f;
+            o.z = (i0 + i + 2 < t) ? bt * sRk[i0 + i + 2] * ex2_approx(Gt - sG2[i0 + i + 2]) * v[i + 2] : 0.f;
+            o.w = (i0 + i + 3 < t) ? bt * sRk[i0 + i + 3] * ex2_approx(Gt - sG2[i0 + i + 3]) * v[i + 3] : 0.f;
+            *reinterpret_cast<float4*>(sA + fidx(t, i0 + i)) = o;
+          }
+        } else {
+          const float qt = sRq[t];
+#pragma unroll
+          for (int c8 = 0; c8 < 4; ++c8) {
+            uint32_t pk[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int ia = i0 + 8 * c8 + 2 * u, ib = ia + 1;
+              const float p0 = (ia <= t) ? qt * sRk[ia] * ex2_approx(Gt - sG2[ia]) * v[8 * c8 + 2 * u] : 0.f;
+              const float p1 = (ib <= t) ? qt * sRk[ib] * ex2_approx(Gt - sG2[ib]) * v[8 * c8 + 2 * u + 1] : 0.f;
+              pk[u] = pack_f16(p0, p1);
+            }
+            st_shared_v4(stg + SH_P + sw128_chunk(t, half * 4 + c8, 64), pk[0], pk[1], pk[2], pk[3]);
+          }
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        reinterpret_cast<float4*>(sT)[tid + kNT * k] = make_float4(0.f, 0.f, 0.f, 0.f);
+      fence_before_sync();
+      __syncthreads();
+
+      // T = (I + A)^{-1}
+      if (tid < 64) {
+        const int bq = tid >> 3, c = tid & 7;
+        float ab[8][8];
+#pragma unroll
+        for (int r = 1; r < 8; ++r) {
+          const float4 lo = *reinterpret_cast<const float4*>(sA + fidx(8 * bq + r, 8 * bq));
+          const float4 hi = *reinterpret_cast<const float4*>(sA + fidx(8 * bq + r, 8 * bq + 4));
+          ab[r][0] = lo.x; ab[r][1] = lo.y; ab[r][2] = lo.z; ab[r][3] = lo.w;
+          ab[r][4] = hi.x; ab[r][5] = hi.y; ab[r][6] = hi.z; ab[r][7] = hi.w;
+        }
+        float x[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          float s = (r == c) ? 1.f : 0.f;
+#pragma unroll
+          for (int m = 0; m < r; ++m) s -= ab[r][m] * x[m];
+          x[r] = s;
+        }
+#pragma unroll
+        for (int r = 0; r < 8; ++r) sT[fidx(8 * bq + r, 8 * bq + c)] = x[r];
+      }
+      __syncthreads();
+      tinv_level<8>(sA, sT, sZ, tid);
+      tinv_level<16>(sA, sT, sZ, tid);
+      tinv_level<32>(sA, sT, sZ, tid);
+
+      // f; T diag(b) 2^-f (shipped), T diag(b g) 2^-f (local)
+      {
+        const int t = row & 63;
+        const bool withg = row >= 64;
+        float tv[32];
+        float tmax = 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) {
+          const float4 x = *reinterpret_cast<const float4*>(sT + fidx(t, half * 32 + i));
+          tv[i] = x.x; tv[i + 1] = x.y; tv[i + 2] = x.z; tv[i + 3] = x.w;
+          tmax = fmaxf(tmax, fmaxf(fmaxf(fabsf(x.x), fabsf(x.y)), fmaxf(fabsf(x.z), fabsf(x.w))));
+        }
+        const int f = max(0, scale_exp(block_max(tmax, sMax, warp, lane), 8));
+        const float sf = ldexpf(1.f, -f);
+#pragma unroll
+        for (int c8 = 0; c8 < 4; ++c8) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int ia = half * 32 + 8 * c8 + 2 * u;
+            float x0 = tv[8 * c8 + 2 * u] * sBeta[ia] * sf;
+            float x1 = tv[8 * c8 + 2 * u + 1] * sBeta[ia + 1] * sf;
+            if (withg) {
+              x0 *= sGam[ia];
+              x1 *= sGam[ia + 1];
+            }
+            pk[u] = pack_f16(x0, x1);
+          }
+          st_shared_v4((withg ? sb + P_TBG : stg + SH_TB) + sw128_chunk(t, half * 4 + c8, 64),
+                       pk[0], pk[1], pk[2], pk[3]);
+        }
+        if (tid == 0) sScal[b * 4 + 1] = (float)f;
+      }
+      fence_proxy_async();
+      fence_before_sync();
+      __syncthreads();
+
+      // W^T = K^T (T diag(b g))^T
+      if (tid == 0) {
+        fence_after_sync();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t da = sdesc(sb + P_KH + kk * 2048, 8192, 1024);
+          const uint64_t db = sdesc(sb + P_TBG + kk * 32, 16, 1024);
+          mma_f16(tbase + 64, da, db, ID_MK, kk > 0);
+        }
+        mma_commit(mbar);
+      }
+      okw = mbar_wait(mbar, phase, kWaitLimit);
+      phase ^= 1;
+      if (!__syncthreads_and(okw)) { ok = false; break; }
+      fence_after_sync();
+      {
+        float v[32];
+        tmem_ld32(tW + half * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          st_chunk_f16(stg + SH_WT + sw128_chunk(row, half * 4 + q, 128), v + 8 * q, 1.f);
+      }
+      fence_proxy_async();
+      fence_before_sync();
+      __syncthreads();
+
+      // ship this chunk's tiles once the chain CTA has released buffer b
+      okw = true;
+      if (tid == 0) {
+        okw = mbar_wait_cluster(&empty[b], ((ci >> 1) & 1) ^ 1, kWaitLimit);
+        if (okw) {
+          // the cluster window keeps the peer's layout: offsets carry over
+          const uint32_t full_cl = full_cl0 + 8 * b;
+          const uint32_t ship_cl = ship_cl0 + b * kShipBytes;
+          mbar_remote_arrive_expect_tx(full_cl, kShipBytes + 16);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            bulk_copy_to_peer(ship_cl + 16384 * k, stg + 16384 * k, 16384, full_cl);
+          bulk_copy_to_peer(scal_cl0 + 16 * b, sb + P_SCAL + 16 * b, 16, full_cl);
+          bulk_commit();
+        }
+      }
+      if (!__syncthreads_and(okw)) { ok = false; break; }
+    }
+    cp_async_wait_all();
+    if (tid == 0) bulk_wait_all();
+    if (!ok) {
+      if (tid == 0) atomicOr(a.err, kErrTimeout);
+      mbar_wait(mbar, phase ^ 1, kWaitLimit);
+    }
+    fence_before_sync();
+    __syncthreads();
+    cluster_sync();
+    if (warp == 0) tmem_dealloc(tbase, 128);
+  }
+}
+
 }  // namespace
 
 bool prefill_tc_supports(const PrefillArgs& a) {
@@ -833,8 +1464,30 @@ gdn_status launch_prefill_tc(const PrefillArgs& a, cudaStream_t stream) {
       return GDN_ERR_CUDA;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
-  const unsigned grid = (unsigned)a.n_seq * (unsigned)a.H_v;
-  gdn_prefill_tc_kernel<<<grid, kNT, kSmemBytes, stream>>>(a);
+  static bool pair_attr_set[64] = {false};
+  static int sm_count[64] = {0};
+  if (dev >= 0 && dev < 64 && sm_count[dev] == 0) {
+    int c = 0;
+    if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return GDN_ERR_CUDA;
+    sm_count[dev] = c;
+  }
+  const int sms = (dev >= 0 && dev < 64) ? sm_count[dev] : 148;
+  const long long items = (long long)a.n_seq * a.H_v;
+  // CTA pairs while there are too few (sequence, head) items to fill the GPU
+  const bool pair = a.tc_variant == 1 || (a.tc_variant == 0 && 2 * items <= sms);
+  if (pair) {
+    if (dev < 0 || dev >= 64 || !pair_attr_set[dev]) {
+      if (cudaFuncSetAttribute(gdn_prefill_tc_pair_kernel,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)kPairSmemBytes) != cudaSuccess)
+        return GDN_ERR_CUDA;
+      if (dev >= 0 && dev < 64) pair_attr_set[dev] = true;
+    }
+    gdn_prefill_tc_pair_kernel<<<(unsigned)(2 * items), kNT, kPairSmemBytes, stream>>>(a);
+  } else {
+    gdn_prefill_tc_kernel<<<(unsigned)items, kNT, kSmemBytes, stream>>>(a);
+  }
   return cudaPeekAtLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 

@@ -20,7 +20,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "gdn.h")
 
 GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_TIMEOUT = range(5)
 GDN_BF16, GDN_FP32 = 0, 1
-PATHS = {"auto": 0, "tensor": 1, "simt": 2}
+PATHS = {"auto": 0, "tensor": 1, "simt": 2, "tensor_pair": 3, "tensor_single": 4}
 
 _lib = None
 _vp = ctypes.c_void_p

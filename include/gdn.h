@@ -63,11 +63,17 @@ typedef enum { GDN_BF16 = 0, GDN_FP32 = 1 } gdn_dtype;
 
 /* Which prefill kernel runs.  AUTO picks the tensor-core kernel when it
  * supports the shape (bf16, d_k = d_v = 128) and the portable CUDA-core
- * kernel otherwise.  TENSOR on an unsupported shape is GDN_ERR_UNSUPPORTED. */
+ * kernel otherwise.  The tensor kernel runs either one CTA per (sequence,
+ * value head) or, when there are too few of those to fill the GPU, a pair of
+ * CTAs per item that split the per-chunk work; PAIR / SINGLE force one
+ * layout (same results up to rounding).  A tensor path on an unsupported
+ * shape is GDN_ERR_UNSUPPORTED. */
 typedef enum {
   GDN_PATH_AUTO = 0,
-  GDN_PATH_TENSOR = 1, /* tcgen05 MMA + TMA + TMEM chunked kernel */
-  GDN_PATH_SIMT = 2    /* fp32 CUDA-core chunked kernel           */
+  GDN_PATH_TENSOR = 1,        /* tcgen05 MMA + TMEM chunked kernel, layout chosen by size */
+  GDN_PATH_SIMT = 2,          /* fp32 CUDA-core chunked kernel                           */
+  GDN_PATH_TENSOR_PAIR = 3,   /* tensor kernel, two CTAs (a cluster) per sequence x head */
+  GDN_PATH_TENSOR_SINGLE = 4  /* tensor kernel, one CTA per sequence x head              */
 } gdn_prefill_path;
 
 /*

@@ -1,7 +1,9 @@
 """Chunked prefill on the GPU against the fp64 oracle.
 
-Covers both kernels (``simt``: fp32 CUDA cores, every shape and dtype;
-``tensor``: tcgen05 kernel for bf16, d_k = d_v = 128) on the workload recipes
+Covers every kernel (``simt``: fp32 CUDA cores, every shape and dtype;
+``tensor_single`` / ``tensor_pair``: the tcgen05 kernel for bf16, d_k = d_v =
+128, with one CTA or a two-CTA cluster per (sequence, head)) on the workload
+recipes
 (shortened where the oracle must see every output), ragged chunk tails,
 empty and one-token sequences, packed batches, in-place state update,
 split-and-carry, and sampled outputs at the full workload sizes.
@@ -15,7 +17,7 @@ from tests._parity import assert_close, oracle_prefill, to_device
 
 pytestmark = pytest.mark.gpu
 
-BF16_PATHS = ["simt", "tensor"]
+BF16_PATHS = ["simt", "tensor_single", "tensor_pair"]
 
 
 def _run(w, path="auto", **kw):
