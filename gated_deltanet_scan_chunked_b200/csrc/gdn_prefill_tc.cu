@@ -855,14 +855,14 @@ constexpr uint32_t P_MAX = 227872;        // block-max scratch [16]
 constexpr uint32_t P_BAR = 227936;        // empty[2], mma, tmem slot
 constexpr uint32_t kPairSmemBytes = 228000 + 1024;
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNT, 1)
-    gdn_prefill_tc_pair_kernel(const PrefillArgs a) {
+template <int NPREP>
+__global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const PrefillArgs a) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sb = (raw + 1023u) & ~1023u;
   uint8_t* gb = smem_raw + (sb - raw);
   const uint32_t rank = cluster_ctarank();
-  const int item = blockIdx.x >> 1;
+  const int item = blockIdx.x / (1 + NPREP);
   const int seq = item / a.H_v;
   const int h = item % a.H_v;
   const int hq = h / (a.H_v / a.H_qk);
@@ -1069,7 +1069,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNT, 1)
       if (!__syncthreads_and(okw)) { ok = false; break; }
       fence_after_sync();
       // this chunk's shipped tiles are no longer read: hand the buffer back
-      if (tid == 0) mbar_remote_arrive(mapa_shared(sb + P_BAR + 8 * b, 1));
+      if (tid == 0) mbar_remote_arrive(mapa_shared(sb + P_BAR + 8 * b, 1 + ci % NPREP));
       GDN_TRACE_POINT(5);
 
       // epilogue
@@ -1164,10 +1164,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNT, 1)
     float* sRq = sG2 + 320;
     float* sScal = reinterpret_cast<float*>(gb + P_SCAL);
     float* sMax = reinterpret_cast<float*>(gb + P_MAX);
-    if (t_begin < t_end) {
-      const int n0 = (t_end - t_begin) < kC ? (int)(t_end - t_begin) : kC;
-      ld.qk(t_begin, n0);
-      ld.gates(t_begin, n0, 0);
+    // prep CTA r handles chunks r-1, r-1+NPREP, ...
+    const int first = (int)rank - 1;
+    const int64_t c_first = t_begin + (int64_t)kC * first;
+    if (c_first < t_end) {
+      const int n0 = (t_end - c_first) < kC ? (int)(t_end - c_first) : kC;
+      ld.qk(c_first, n0);
+      ld.gates(c_first, n0, 0);
       cp_async_commit();
     }
     if (warp == 0) tmem_alloc(tslot, 128);
@@ -1187,20 +1190,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNT, 1)
     const uint32_t ship_cl0 = mapa_shared(sb + C_SHIP, 0);
     const uint32_t scal_cl0 = mapa_shared(sb + C_SCAL, 0);
 
-    int ci = 0;
-    for (int64_t c0 = t_begin; c0 < t_end; c0 += kC, ++ci) {
+    int ci = first, lc = 0;  // chunk index, local count
+    for (int64_t c0 = c_first; c0 < t_end; c0 += (int64_t)kC * NPREP, ci += NPREP, ++lc) {
       const int n = (t_end - c0) < kC ? (int)(t_end - c0) : kC;
-      const bool has_next = c0 + kC < t_end;
-      const int nn = has_next ? ((t_end - c0 - kC) < kC ? (int)(t_end - c0 - kC) : kC) : 0;
-      const int b = ci & 1;
-      const uint32_t stg = sb + P_STG + b * kShipBytes;
+      const int64_t cnext = c0 + (int64_t)kC * NPREP;
+      const bool has_next = cnext < t_end;
+      const int nn = has_next ? ((t_end - cnext) < kC ? (int)(t_end - cnext) : kC) : 0;
+      const int b = ci & 1;       // buffer in the chain CTA
+      const int lb = lc & 1;      // local staging / prefetch buffer
+      const uint32_t stg = sb + P_STG + lb * kShipBytes;
       cp_async_wait_all();
-      if (tid == 0) bulk_wait_read_le1();  // staging buffer b is no longer being copied
+      if (tid == 0) bulk_wait_read_le1();  // staging buffer lb is no longer being copied
       __syncthreads();
 
       // gates
       if (warp == 0) {
-        const float* gl = sGateBuf + b * 128;
+        const float* gl = sGateBuf + lb * 128;
         float carry = 0.f;
         float Gv[2], bv[2];
 #pragma unroll
@@ -1224,9 +1229,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNT, 1)
           sGam[t] = ex2_approx(Gv[hb]);
           sDec[t] = ex2_approx(carry - Gv[hb]);
         }
-        if (lane == 0) sScal[b * 4 + 0] = ex2_approx(carry);
+        if (lane == 0) sScal[lb * 4 + 0] = ex2_approx(carry);
       }
-      if (has_next) ld.gates(c0 + kC, nn, b ^ 1);
+      if (has_next) ld.gates(cnext, nn, lb ^ 1);
       cp_async_commit();
       __syncthreads();
 
@@ -1280,7 +1285,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNT, 1)
       phase ^= 1;
       if (!__syncthreads_and(okw)) { ok = false; break; }
       fence_after_sync();
-      if (has_next) ld.qk(c0 + kC, nn);
+      if (has_next) ld.qk(cnext, nn);
       cp_async_commit();
 
       // A (fp32) and P (fp16, shipped)
@@ -1382,7 +1387,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNT, 1)
           st_shared_v4((withg ? sb + P_TBG : stg + SH_TB) + sw128_chunk(t, half * 4 + c8, 64),
                        pk[0], pk[1], pk[2], pk[3]);
         }
-        if (tid == 0) sScal[b * 4 + 1] = (float)f;
+        if (tid == 0) sScal[lb * 4 + 1] = (float)f;
       }
       fence_proxy_async();
       fence_before_sync();
@@ -1427,7 +1432,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNT, 1)
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             bulk_copy_to_peer(ship_cl + 16384 * k, stg + 16384 * k, 16384, full_cl);
-          bulk_copy_to_peer(scal_cl0 + 16 * b, sb + P_SCAL + 16 * b, 16, full_cl);
+          bulk_copy_to_peer(scal_cl0 + 16 * b, sb + P_SCAL + 16 * lb, 16, full_cl);
           bulk_commit();
         }
       }
@@ -1464,7 +1469,7 @@ gdn_status launch_prefill_tc(const PrefillArgs& a, cudaStream_t stream) {
       return GDN_ERR_CUDA;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
-  static bool pair_attr_set[64] = {false};
+  static bool pair_attr_set[64][2] = {{false}};
   static int sm_count[64] = {0};
   if (dev >= 0 && dev < 64 && sm_count[dev] == 0) {
     int c = 0;
@@ -1474,17 +1479,64 @@ gdn_status launch_prefill_tc(const PrefillArgs& a, cudaStream_t stream) {
   }
   const int sms = (dev >= 0 && dev < 64) ? sm_count[dev] : 148;
   const long long items = (long long)a.n_seq * a.H_v;
-  // CTA pairs while there are too few (sequence, head) items to fill the GPU
-  const bool pair = a.tc_variant == 1 || (a.tc_variant == 0 && 2 * items <= sms);
-  if (pair) {
-    if (dev < 0 || dev >= 64 || !pair_attr_set[dev]) {
-      if (cudaFuncSetAttribute(gdn_prefill_tc_pair_kernel,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+  // While there are too few (sequence, head) items to fill the GPU, give each
+  // a cluster: one chain CTA plus one or two preparation CTAs -- but only a
+  // cluster size whose clusters all fit on the GPU at once (a second wave
+  // would double the time).
+  static int max_clusters[64][2] = {{0}};
+  auto fits = [&](int np) -> bool {
+    if (dev < 0 || dev >= 64) return false;
+    if (max_clusters[dev][np - 1] == 0) {
+      const void* fn = np == 2 ? (const void*)gdn_prefill_tc_pair_kernel<2>
+                               : (const void*)gdn_prefill_tc_pair_kernel<1>;
+      if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)kPairSmemBytes) != cudaSuccess)
+        return false;
+      pair_attr_set[dev][np - 1] = true;
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((unsigned)(1 + np), 1, 1);
+      cfg.blockDim = dim3(kNT, 1, 1);
+      cfg.dynamicSmemBytes = kPairSmemBytes;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 1 + np;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int mc = 0;
+      if (cudaOccupancyMaxActiveClusters(&mc, fn, &cfg) != cudaSuccess) mc = -1;
+      max_clusters[dev][np - 1] = mc;
+    }
+    return max_clusters[dev][np - 1] >= items;
+  };
+  int nprep = 0;
+  if (a.tc_variant == 1) nprep = fits(2) ? 2 : 1;
+  else if (a.tc_variant == 0) nprep = fits(2) ? 2 : (fits(1) ? 1 : 0);
+  if (nprep > 0) {
+    const void* fn = nprep == 2 ? (const void*)gdn_prefill_tc_pair_kernel<2>
+                                : (const void*)gdn_prefill_tc_pair_kernel<1>;
+    if (dev < 0 || dev >= 64 || !pair_attr_set[dev][nprep - 1]) {
+      if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)kPairSmemBytes) != cudaSuccess)
         return GDN_ERR_CUDA;
-      if (dev >= 0 && dev < 64) pair_attr_set[dev] = true;
+      if (dev >= 0 && dev < 64) pair_attr_set[dev][nprep - 1] = true;
     }
-    gdn_prefill_tc_pair_kernel<<<(unsigned)(2 * items), kNT, kPairSmemBytes, stream>>>(a);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((1 + nprep) * items), 1, 1);
+    cfg.blockDim = dim3(kNT, 1, 1);
+    cfg.dynamicSmemBytes = kPairSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1 + nprep;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t err = nprep == 2 ? cudaLaunchKernelEx(&cfg, gdn_prefill_tc_pair_kernel<2>, a)
+                                 : cudaLaunchKernelEx(&cfg, gdn_prefill_tc_pair_kernel<1>, a);
+    if (err != cudaSuccess) return GDN_ERR_CUDA;
   } else {
     gdn_prefill_tc_kernel<<<(unsigned)items, kNT, kSmemBytes, stream>>>(a);
   }
