@@ -1,7 +1,8 @@
 """Benchmark of the gated delta rule library on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload prefill4k|prefill256k|varlen] [--path auto|tensor|simt]
+                    [--workload prefill4k|prefill256k|varlen]
+                    [--path auto|tensor|tensor_pair|tensor_single|simt]
                     [--no-decode] [--no-cpu-baseline]
 
 One step = one chunked prefill (gdn_chunk_fwd: L2-norm prologue, gate cumsum,
@@ -326,7 +327,7 @@ def run_ours(args, world, rank, local):
         achieved, peak, unit = nbytes / (ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s"
     else:
         achieved, peak, unit = nflops / (ms * 1e-3) / 1e12, peaks["bf16_tflops"], "TFLOP/s"
-    kernel_key = "prefill_tc" if args.path in ("auto", "tensor") else "prefill_simt"
+    kernel_key = "prefill_simt" if args.path == "simt" else "prefill_tc"
     roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                 "frac": achieved / peak, "traffic": kernel_traffic(kernel_key),
                 "peak_source": peaks["source"], "roofline_time_us": max(t_hbm, t_tc) * 1e6,
@@ -435,7 +436,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="prefill4k",
                     choices=["prefill4k", "prefill256k", "varlen"])
-    ap.add_argument("--path", default="auto", choices=["auto", "tensor", "simt"])
+    ap.add_argument("--path", default="auto",
+                    choices=["auto", "tensor", "simt", "tensor_pair", "tensor_single"])
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
