@@ -75,6 +75,7 @@ constexpr uint32_t OFF_DT = 172032;     // Delta^T fp16    128 x 64
 // between the previous chunk's MMAs and this chunk's W / Delta conversions.
 constexpr uint32_t OFF_A = OFF_WT;
 constexpr uint32_t OFF_T = OFF_DT;
+constexpr uint32_t OFF_TBG_LO = OFF_A;  // rounding remainder of T diag(b g), after A is dead
 constexpr uint32_t OFF_GS = 188416;     // g in / y out staging, 2 buffers x [64][128] bf16
 constexpr uint32_t OFF_Z = 221184;      // Z fp32 [1024]
 constexpr uint32_t OFF_GATEBUF = 225280;  // [2 buffers][log alpha, beta][64] fp32
@@ -130,6 +131,15 @@ __device__ __forceinline__ int scale_exp(float x, int target) {
   int ex;
   frexpf(x, &ex);  // x = m 2^ex, m in [0.5, 1)
   return ex - target;
+}
+
+// fp16 pair split into a rounded part and the rounding remainder:
+// hi + lo carries the fp32 value to ~2^-22 relative.
+__device__ __forceinline__ void split_pack_f16(float x0, float x1, uint32_t* hi, uint32_t* lo) {
+  const __half2 h = __floats2half2_rn(x0, x1);
+  const float2 hf = __half22float2(h);
+  *hi = *reinterpret_cast<const uint32_t*>(&h);
+  *lo = pack_f16(x0 - hf.x, x1 - hf.y);
 }
 
 __device__ __forceinline__ void st_chunk_f16(uint32_t addr, const float* v, float s) {
@@ -238,6 +248,57 @@ __device__ __forceinline__ void tinv_level(const float* sA, float* sT, float* sZ
     }
   }
   __syncthreads();
+}
+
+
+// A (fp32, strictly lower) and P (fp16 tile, lower incl. diagonal) for one
+// row t of the chunk from 32 raw products v of this thread's TMEM lane:
+//   A_ti = beta_t rk_t rk_i 2^(G2_t - G2_i) (k.k)_ti      (i < t)
+//   P_ti = rq_t rk_i 2^(G2_t - G2_i) (q.k)_ti             (i <= t)
+// columns i0 .. i0+31.  Blocks of columns entirely above the diagonal are
+// skipped (whole warps skip them together, rows are warp-contiguous).
+__device__ __forceinline__ void chunk_ap(const float* v, int t, int i0, bool is_a,
+                                         const float* sG2, const float* sBeta, const float* sRk,
+                                         const float* sRq, float* sA, uint32_t p_tile) {
+  const float Gt = sG2[t];
+  if (is_a) {
+    const float bt = sBeta[t] * sRk[t];
+#pragma unroll
+    for (int i = 0; i < 32; i += 4) {
+      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (i0 + i < t) {
+        const float4 g4 = *reinterpret_cast<const float4*>(sG2 + i0 + i);
+        const float4 k4 = *reinterpret_cast<const float4*>(sRk + i0 + i);
+        o.x = bt * k4.x * ex2_approx(Gt - g4.x) * v[i + 0];
+        o.y = (i0 + i + 1 < t) ? bt * k4.y * ex2_approx(Gt - g4.y) * v[i + 1] : 0.f;
+        o.z = (i0 + i + 2 < t) ? bt * k4.z * ex2_approx(Gt - g4.z) * v[i + 2] : 0.f;
+        o.w = (i0 + i + 3 < t) ? bt * k4.w * ex2_approx(Gt - g4.w) * v[i + 3] : 0.f;
+      }
+      *reinterpret_cast<float4*>(sA + fidx(t, i0 + i)) = o;
+    }
+  } else {
+    const float qt = sRq[t];
+#pragma unroll
+    for (int c8 = 0; c8 < 4; ++c8) {
+      uint32_t pk[4] = {0u, 0u, 0u, 0u};
+      if (i0 + 8 * c8 <= t) {
+#pragma unroll
+        for (int hq = 0; hq < 2; ++hq) {
+          const int ib = i0 + 8 * c8 + 4 * hq;
+          const float4 g4 = *reinterpret_cast<const float4*>(sG2 + ib);
+          const float4 k4 = *reinterpret_cast<const float4*>(sRk + ib);
+          const float* vv = v + 8 * c8 + 4 * hq;
+          const float p0 = (ib + 0 <= t) ? qt * k4.x * ex2_approx(Gt - g4.x) * vv[0] : 0.f;
+          const float p1 = (ib + 1 <= t) ? qt * k4.y * ex2_approx(Gt - g4.y) * vv[1] : 0.f;
+          const float p2 = (ib + 2 <= t) ? qt * k4.z * ex2_approx(Gt - g4.z) * vv[2] : 0.f;
+          const float p3 = (ib + 3 <= t) ? qt * k4.w * ex2_approx(Gt - g4.w) * vv[3] : 0.f;
+          pk[2 * hq] = pack_f16(p0, p1);
+          pk[2 * hq + 1] = pack_f16(p2, p3);
+        }
+      }
+      st_shared_v4(p_tile + sw128_chunk(t, i0 / 8 + c8, 64), pk[0], pk[1], pk[2], pk[3]);
+    }
+  }
 }
 
 struct ChunkLoader {
@@ -535,38 +596,10 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
 
     // ---- A (fp32) and P (fp16) from the raw products: all 256 threads -----------
     {
-      const int t = row & 63;
-      const int i0 = half * 32;
       float v[32];
-      tmem_ld32(tKQ + i0, v);
+      tmem_ld32(tKQ + half * 32, v);
       tmem_wait_ld();
-      const float Gt = sG2[t];
-      if (row < 64) {
-        const float bt = sBeta[t] * sRk[t];
-#pragma unroll
-        for (int i = 0; i < 32; i += 4) {
-          float4 o;
-          o.x = (i0 + i + 0 < t) ? bt * sRk[i0 + i + 0] * ex2_approx(Gt - sG2[i0 + i + 0]) * v[i + 0] : 0.f;
-          o.y = (i0 + i + 1 < t) ? bt * sRk[i0 + i + 1] * ex2_approx(Gt - sG2[i0 + i + 1]) * v[i + 1] : 0.f;
-          o.z = (i0 + i + 2 < t) ? bt * sRk[i0 + i + 2] * ex2_approx(Gt - sG2[i0 + i + 2]) * v[i + 2] : 0.f;
-          o.w = (i0 + i + 3 < t) ? bt * sRk[i0 + i + 3] * ex2_approx(Gt - sG2[i0 + i + 3]) * v[i + 3] : 0.f;
-          *reinterpret_cast<float4*>(sA + fidx(t, i0 + i)) = o;
-        }
-      } else {
-        const float qt = sRq[t];
-#pragma unroll
-        for (int c8 = 0; c8 < 4; ++c8) {
-          uint32_t pk[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int ia = i0 + 8 * c8 + 2 * u, ib = ia + 1;
-            const float p0 = (ia <= t) ? qt * sRk[ia] * ex2_approx(Gt - sG2[ia]) * v[8 * c8 + 2 * u] : 0.f;
-            const float p1 = (ib <= t) ? qt * sRk[ib] * ex2_approx(Gt - sG2[ib]) * v[8 * c8 + 2 * u + 1] : 0.f;
-            pk[u] = pack_f16(p0, p1);
-          }
-          st_shared_v4(sb + OFF_P + sw128_chunk(t, half * 4 + c8, 64), pk[0], pk[1], pk[2], pk[3]);
-        }
-      }
+      chunk_ap(v, row & 63, half * 32, row < 64, sG2, sBeta, sRk, sRq, sA, sb + OFF_P);
     }
     // T starts from zero (its strictly upper blocks are never computed)
 #pragma unroll
@@ -619,9 +652,11 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
       }
       const int f = max(0, scale_exp(block_max(tmax, sMax, warp, lane), 8));
       const float sf = ldexpf(1.f, -f);
+      // T diag(b g) feeds W, a cancellation when keys repeat: it goes in as
+      // fp16 hi + lo (the lo tile reuses the dead A scratch)
 #pragma unroll
       for (int c8 = 0; c8 < 4; ++c8) {
-        uint32_t pk[4];
+        uint32_t pk[4], pl[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const int ia = half * 32 + 8 * c8 + 2 * u;
@@ -631,10 +666,11 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
             x0 *= sGam[ia];
             x1 *= sGam[ia + 1];
           }
-          pk[u] = pack_f16(x0, x1);
+          split_pack_f16(x0, x1, &pk[u], &pl[u]);
         }
-        st_shared_v4(sb + (withg ? OFF_TBG : OFF_TB) + sw128_chunk(t, half * 4 + c8, 64), pk[0],
-                     pk[1], pk[2], pk[3]);
+        const uint32_t off = sw128_chunk(t, half * 4 + c8, 64);
+        st_shared_v4(sb + (withg ? OFF_TBG : OFF_TB) + off, pk[0], pk[1], pk[2], pk[3]);
+        if (withg) st_shared_v4(sb + OFF_TBG_LO + off, pl[0], pl[1], pl[2], pl[3]);
       }
       if (tid == 0) sMax[8] = (float)f;
     }
@@ -652,6 +688,12 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
         const uint64_t da = sdesc(sb + OFF_KH + kk * 2048, 8192, 1024);
         const uint64_t db = sdesc(sb + OFF_TBG + kk * 32, 16, 1024);
         mma_f16(tbase + TM_W, da, db, ID_MK, kk > 0);
+      }
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t da = sdesc(sb + OFF_KH + kk * 2048, 8192, 1024);
+        const uint64_t db = sdesc(sb + OFF_TBG_LO + kk * 32, 16, 1024);
+        mma_f16(tbase + TM_W, da, db, ID_MK, 1);
       }
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
@@ -846,6 +888,7 @@ constexpr uint32_t P_KH = 32768;          // K^ fp16
 constexpr uint32_t P_TBG = 49152;         // T diag(b g) 2^-f fp16
 constexpr uint32_t P_A = 57344;           // A fp32
 constexpr uint32_t P_T = 73728;           // T fp32
+constexpr uint32_t P_TBG_LO = P_A;        // remainder of T diag(b g), after A is dead
 constexpr uint32_t P_STG = 90112;         // ship staging, 2 x 64 KB
 constexpr uint32_t P_Z = 221184;          // Z fp32 [1024]
 constexpr uint32_t P_GATEBUF = 225280;    // [2][la, beta][64]
@@ -1290,38 +1333,10 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
 
       // A (fp32) and P (fp16, shipped)
       {
-        const int t = row & 63;
-        const int i0 = half * 32;
         float v[32];
-        tmem_ld32(tKQ + i0, v);
+        tmem_ld32(tKQ + half * 32, v);
         tmem_wait_ld();
-        const float Gt = sG2[t];
-        if (row < 64) {
-          const float bt = sBeta[t] * sRk[t];
-#pragma unroll
-          for (int i = 0; i < 32; i += 4) {
-            float4 o;
-            o.x = (i0 + i + 0 < t) ? bt * sRk[i0 + i + 0] * ex2_approx(Gt - sG2[i0 + i + 0]) * v[i + 0] : 0.f;
-            o.y = (i0 + i + 1 < t) ? bt * sRk[i0 + i + 1] * ex2_approx(Gt - sG2[i0 + i + 1]) * v[i + 1] : 0.f;
-            o.z = (i0 + i + 2 < t) ? bt * sRk[i0 + i + 2] * ex2_approx(Gt - sG2[i0 + i + 2]) * v[i + 2] : 0.f;
-            o.w = (i0 + i + 3 < t) ? bt * sRk[i0 + i + 3] * ex2_approx(Gt - sG2[i0 + i + 3]) * v[i + 3] : 0.f;
-            *reinterpret_cast<float4*>(sA + fidx(t, i0 + i)) = o;
-          }
-        } else {
-          const float qt = sRq[t];
-#pragma unroll
-          for (int c8 = 0; c8 < 4; ++c8) {
-            uint32_t pk[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int ia = i0 + 8 * c8 + 2 * u, ib = ia + 1;
-              const float p0 = (ia <= t) ? qt * sRk[ia] * ex2_approx(Gt - sG2[ia]) * v[8 * c8 + 2 * u] : 0.f;
-              const float p1 = (ib <= t) ? qt * sRk[ib] * ex2_approx(Gt - sG2[ib]) * v[8 * c8 + 2 * u + 1] : 0.f;
-              pk[u] = pack_f16(p0, p1);
-            }
-            st_shared_v4(stg + SH_P + sw128_chunk(t, half * 4 + c8, 64), pk[0], pk[1], pk[2], pk[3]);
-          }
-        }
+        chunk_ap(v, row & 63, half * 32, row < 64, sG2, sBeta, sRk, sRq, sA, stg + SH_P);
       }
 #pragma unroll
       for (int k = 0; k < 4; ++k)
@@ -1372,7 +1387,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
         const float sf = ldexpf(1.f, -f);
 #pragma unroll
         for (int c8 = 0; c8 < 4; ++c8) {
-          uint32_t pk[4];
+          uint32_t pk[4], pl[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const int ia = half * 32 + 8 * c8 + 2 * u;
@@ -1382,10 +1397,11 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
               x0 *= sGam[ia];
               x1 *= sGam[ia + 1];
             }
-            pk[u] = pack_f16(x0, x1);
+            split_pack_f16(x0, x1, &pk[u], &pl[u]);
           }
-          st_shared_v4((withg ? sb + P_TBG : stg + SH_TB) + sw128_chunk(t, half * 4 + c8, 64),
-                       pk[0], pk[1], pk[2], pk[3]);
+          const uint32_t off = sw128_chunk(t, half * 4 + c8, 64);
+          st_shared_v4((withg ? sb + P_TBG : stg + SH_TB) + off, pk[0], pk[1], pk[2], pk[3]);
+          if (withg) st_shared_v4(sb + P_TBG_LO + off, pl[0], pl[1], pl[2], pl[3]);
         }
         if (tid == 0) sScal[lb * 4 + 1] = (float)f;
       }
@@ -1401,6 +1417,12 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
           const uint64_t da = sdesc(sb + P_KH + kk * 2048, 8192, 1024);
           const uint64_t db = sdesc(sb + P_TBG + kk * 32, 16, 1024);
           mma_f16(tbase + 64, da, db, ID_MK, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t da = sdesc(sb + P_KH + kk * 2048, 8192, 1024);
+          const uint64_t db = sdesc(sb + P_TBG_LO + kk * 32, 16, 1024);
+          mma_f16(tbase + 64, da, db, ID_MK, 1);
         }
         mma_commit(mbar);
       }
@@ -1470,14 +1492,6 @@ gdn_status launch_prefill_tc(const PrefillArgs& a, cudaStream_t stream) {
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
   static bool pair_attr_set[64][2] = {{false}};
-  static int sm_count[64] = {0};
-  if (dev >= 0 && dev < 64 && sm_count[dev] == 0) {
-    int c = 0;
-    if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      return GDN_ERR_CUDA;
-    sm_count[dev] = c;
-  }
-  const int sms = (dev >= 0 && dev < 64) ? sm_count[dev] : 148;
   const long long items = (long long)a.n_seq * a.H_v;
   // While there are too few (sequence, head) items to fill the GPU, give each
   // a cluster: one chain CTA plus one or two preparation CTAs -- but only a
