@@ -2,13 +2,15 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload prefill4k|prefill256k|varlen]
-                    [--path auto|tensor|tensor_pair|tensor_single|simt]
+                    [--path auto|tensor|tensor_pair|tensor_single|tensor_split|simt]
                     [--no-decode] [--no-cpu-baseline]
 
 One step = one chunked prefill (gdn_chunk_fwd: L2-norm prologue, gate cumsum,
 intra-chunk products, triangular solve, state carry, RMSNorm x sigmoid(g)
 epilogue) over one batch of the workload (default: B=1, T=4096, 16 QK / 48
-value heads, d=128, bf16).  The JSON line also carries the decode step
+value heads, d=128, bf16).  The call gets a preallocated workspace, so small
+batches may take the split layout (one kernel, after an asynchronous memset of
+the workspace flags).  The JSON line also carries the decode step
 (gdn_decode_step, 256 sequences x 64 steps, in place) as a separate object
 with its own timing, roofline and clocks.
 
@@ -297,11 +299,16 @@ def run_ours(args, world, rank, local):
     y = torch.empty_like(w.v)
     fs = torch.empty((n_seq, H_V, D, D), dtype=torch.float32, device="cuda")
     flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
+    # caller-owned workspace for the small-batch split layout (allocated once)
+    ws = None
+    ws_bytes = gdn.workspace_size(n_seq, H_V, D, D) if args.path in gdn._WS_PATHS else 0
+    if ws_bytes > 0:
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
 
     def step():
         gdn_chunk_fwd(w.q, w.k, w.v, w.log_alpha, w.beta, g=w.g, norm_w=w.norm_w,
                       initial_state=w.initial_state, cu_seqlens=w.cu_seqlens, y=y,
-                      final_state=fs, path=args.path)
+                      final_state=fs, path=args.path, workspace=ws)
 
     def flush():
         flush_buf.zero_()
@@ -357,7 +364,8 @@ def run_ours(args, world, rank, local):
                     dev[nm].copy_(x, non_blocking=True)
             gdn_chunk_fwd(dev["q"], dev["k"], dev["v"], dev["log_alpha"], dev["beta"],
                           g=dev["g"], norm_w=dev["norm_w"], initial_state=dev["initial_state"],
-                          cu_seqlens=dev["cu_seqlens"], y=y, final_state=fs, path=args.path)
+                          cu_seqlens=dev["cu_seqlens"], y=y, final_state=fs, path=args.path,
+                          workspace=ws)
             y_h.copy_(y, non_blocking=True)
             fs_h.copy_(fs, non_blocking=True)
 
@@ -419,7 +427,7 @@ def run_ours(args, world, rank, local):
                 "dtype": "bf16", "data": "synthetic",
                 "config": {"workload": args.workload, "global_batch": world * n_seq,
                            "seq_len": T, "heads": "16 QK / 48 value", "d": D,
-                           "path": args.path,
+                           "path": args.path, "workspace_bytes": ws_bytes,
                            "parallelism": "replicas%d" % world if world > 1 else "single",
                            "l2": "flushed between steps (256 MB write outside the events)"},
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
@@ -437,7 +445,8 @@ def main():
     ap.add_argument("--workload", default="prefill4k",
                     choices=["prefill4k", "prefill256k", "varlen"])
     ap.add_argument("--path", default="auto",
-                    choices=["auto", "tensor", "simt", "tensor_pair", "tensor_single"])
+                    choices=["auto", "tensor", "simt", "tensor_pair", "tensor_single",
+                             "tensor_split"])
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

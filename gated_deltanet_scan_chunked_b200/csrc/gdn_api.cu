@@ -48,12 +48,13 @@ gdn_status check_common(int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v, gdn
 
 using namespace gdn;
 
-extern "C" gdn_status gdn_chunk_fwd_path(
+extern "C" gdn_status gdn_chunk_fwd_ws(
     const void* q, const void* k, const void* v, const float* log_alpha, const float* beta,
     const void* g, const float* norm_w, const float* initial_state, const int32_t* cu_seqlens,
     int32_t n_seq, int64_t total_T, int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v,
     gdn_dtype in_dtype, int32_t l2norm_qk, float eps_l2, float eps_norm, float scale, void* y,
-    float* final_state, gdn_prefill_path path, gdn_stream_t stream) {
+    float* final_state, gdn_prefill_path path, void* workspace, size_t workspace_bytes,
+    gdn_stream_t stream) {
   gdn_status st = check_common(H_qk, H_v, d_k, d_v, in_dtype, eps_l2, eps_norm);
   if (st != GDN_OK) return st;
   if (n_seq < 1 || total_T < 0) return GDN_ERR_INVALID_ARG;
@@ -72,8 +73,16 @@ extern "C" gdn_status gdn_chunk_fwd_path(
     if (a0 < b0 + bytes && b0 < a0 + bytes) return GDN_ERR_INVALID_ARG;
   }
   if (path != GDN_PATH_AUTO && path != GDN_PATH_TENSOR && path != GDN_PATH_SIMT &&
-      path != GDN_PATH_TENSOR_PAIR && path != GDN_PATH_TENSOR_SINGLE)
+      path != GDN_PATH_TENSOR_PAIR && path != GDN_PATH_TENSOR_SINGLE &&
+      path != GDN_PATH_TENSOR_SPLIT)
     return GDN_ERR_INVALID_ARG;
+  const size_t ws_need = prefill_tc_workspace_bytes(n_seq, H_v, d_k, d_v, in_dtype);
+  if (workspace != nullptr) {
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return GDN_ERR_INVALID_ARG;
+    if (workspace_bytes < ws_need) return GDN_ERR_INVALID_ARG;
+  }
+  if (path == GDN_PATH_TENSOR_SPLIT && (workspace == nullptr || ws_need == 0))
+    return workspace == nullptr && ws_need != 0 ? GDN_ERR_INVALID_ARG : GDN_ERR_UNSUPPORTED;
 
   PrefillArgs a;
   a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
@@ -82,17 +91,38 @@ extern "C" gdn_status gdn_chunk_fwd_path(
   a.y = y; a.n_seq = n_seq; a.total_T = total_T;
   a.H_qk = H_qk; a.H_v = H_v; a.d_k = d_k; a.d_v = d_v; a.dtype = in_dtype;
   a.l2norm = l2norm_qk ? 1 : 0; a.eps_l2 = eps_l2; a.eps_norm = eps_norm; a.scale = scale;
-  a.tc_variant = path == GDN_PATH_TENSOR_PAIR ? 1 : (path == GDN_PATH_TENSOR_SINGLE ? 2 : 0);
+  a.tc_variant = path == GDN_PATH_TENSOR_PAIR     ? 1
+                 : path == GDN_PATH_TENSOR_SINGLE ? 2
+                 : path == GDN_PATH_TENSOR_SPLIT  ? 3
+                                                  : 0;
+  if (workspace != nullptr && ws_need != 0) prefill_tc_workspace_layout(workspace, n_seq, H_v, &a);
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool tc_ok = prefill_tc_supports(a);
   const bool want_tc = path == GDN_PATH_TENSOR || path == GDN_PATH_TENSOR_PAIR ||
-                       path == GDN_PATH_TENSOR_SINGLE;
+                       path == GDN_PATH_TENSOR_SINGLE || path == GDN_PATH_TENSOR_SPLIT;
   if (want_tc && !tc_ok) return GDN_ERR_UNSUPPORTED;
   a.err = error_word_ptr();
   if (a.err == nullptr) return GDN_ERR_CUDA;
   if (want_tc || (path == GDN_PATH_AUTO && tc_ok)) return launch_prefill_tc(a, s);
   return launch_prefill_simt(a, s);
+}
+
+extern "C" gdn_status gdn_chunk_fwd_path(
+    const void* q, const void* k, const void* v, const float* log_alpha, const float* beta,
+    const void* g, const float* norm_w, const float* initial_state, const int32_t* cu_seqlens,
+    int32_t n_seq, int64_t total_T, int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v,
+    gdn_dtype in_dtype, int32_t l2norm_qk, float eps_l2, float eps_norm, float scale, void* y,
+    float* final_state, gdn_prefill_path path, gdn_stream_t stream) {
+  return gdn_chunk_fwd_ws(q, k, v, log_alpha, beta, g, norm_w, initial_state, cu_seqlens, n_seq,
+                          total_T, H_qk, H_v, d_k, d_v, in_dtype, l2norm_qk, eps_l2, eps_norm,
+                          scale, y, final_state, path, nullptr, 0, stream);
+}
+
+extern "C" size_t gdn_chunk_fwd_workspace_size(int32_t n_seq, int32_t H_v, int32_t d_k,
+                                               int32_t d_v, gdn_dtype in_dtype) {
+  if (n_seq < 1 || H_v < 1) return 0;
+  return prefill_tc_workspace_bytes(n_seq, H_v, d_k, d_v, in_dtype);
 }
 
 extern "C" gdn_status gdn_chunk_fwd(

@@ -34,7 +34,11 @@ struct PrefillArgs {
   int32_t l2norm;
   float eps_l2, eps_norm, scale;
   int* err;                // device error word
-  int tc_variant;          // tensor kernel: 0 auto, 1 CTA pairs, 2 one CTA per head
+  int tc_variant;          // tensor kernel: 0 auto, 1 CTA pairs, 2 one CTA per head, 3 split
+  // Split-launch workspace (nullptr: none): hand-off ring slots and their
+  // flags, laid out by prefill_tc_workspace_bytes.
+  void* ring = nullptr;
+  unsigned long long* ring_flags = nullptr;
 };
 
 struct DecodeArgs {
@@ -59,5 +63,11 @@ gdn_status launch_decode(const DecodeArgs& a, cudaStream_t stream);
 gdn_status launch_prefill_simt(const PrefillArgs& a, cudaStream_t stream);
 gdn_status launch_prefill_tc(const PrefillArgs& a, cudaStream_t stream);
 bool prefill_tc_supports(const PrefillArgs& a);
+// Workspace bytes the split launch of the tensor kernel needs for n_seq x H_v
+// items (0 when it can never apply), and the placement of its parts within a
+// 256-byte aligned workspace.
+size_t prefill_tc_workspace_bytes(int32_t n_seq, int32_t H_v, int32_t d_k, int32_t d_v,
+                                  gdn_dtype dtype);
+void prefill_tc_workspace_layout(void* ws, int32_t n_seq, int32_t H_v, PrefillArgs* a);
 
 }  // namespace gdn

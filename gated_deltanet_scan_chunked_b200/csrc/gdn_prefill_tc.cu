@@ -125,6 +125,29 @@ __device__ __forceinline__ float block_max(float x, float* sMax, int warp, int l
   return m;
 }
 
+// Block-wide maxima of two non-negative values with one exchange (sMax
+// holds 2 x 8 floats).
+__device__ __forceinline__ float2 block_max2(float x, float y, float* sMax, int warp, int lane) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+    y = fmaxf(y, __shfl_xor_sync(0xffffffffu, y, o));
+  }
+  if (lane == 0) {
+    sMax[warp] = x;
+    sMax[8 + warp] = y;
+  }
+  __syncthreads();
+  float mx = sMax[0], my = sMax[8];
+#pragma unroll
+  for (int w = 1; w < kNT / 32; ++w) {
+    mx = fmaxf(mx, sMax[w]);
+    my = fmaxf(my, sMax[8 + w]);
+  }
+  __syncthreads();  // sMax reusable afterwards
+  return make_float2(mx, my);
+}
+
 // Exponent e with x * 2^-e <= 2^target (x >= 0); 0 for x == 0 or non-finite.
 __device__ __forceinline__ int scale_exp(float x, int target) {
   if (!(x > 0.f) || !(x < 3.0e38f)) return 0;
@@ -157,6 +180,20 @@ __device__ __forceinline__ void unpack_bf16x8(const uint4 u, float* f) {
   p = bf2_to_f2(u.y); f[2] = p.x; f[3] = p.y;
   p = bf2_to_f2(u.z); f[4] = p.x; f[5] = p.y;
   p = bf2_to_f2(u.w); f[6] = p.x; f[7] = p.y;
+}
+
+__device__ __forceinline__ float2 h2_to_f2(uint32_t w) {
+  __half2 h;
+  memcpy(&h, &w, 4);
+  return __half22float2(h);
+}
+
+__device__ __forceinline__ void unpack_f16x8(const uint4 u, float* f) {
+  float2 p;
+  p = h2_to_f2(u.x); f[0] = p.x; f[1] = p.y;
+  p = h2_to_f2(u.y); f[2] = p.x; f[3] = p.y;
+  p = h2_to_f2(u.z); f[4] = p.x; f[5] = p.y;
+  p = h2_to_f2(u.w); f[6] = p.x; f[7] = p.y;
 }
 
 
@@ -868,7 +905,20 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
 // state in TMEM and runs U, Delta, Y, the state update and the epilogue.
 // Buffer hand-off: "full" barriers in CTA 0 (arrive + expected bytes from
 // CTA 1, completed by the copies), "empty" barriers in CTA 1 (arrived by
-// CTA 0 once its MMAs have read the buffer).  Every wait is bounded.
+// CTA 0 once its MMAs have read the buffer), "staging free" barriers in
+// CTA 1 (arrived by CTA 0 once a copy has landed, so CTA 1 may overwrite the
+// copy's source).  Every wait is bounded.
+//
+// Split launch (kGlobal): the same two roles without a cluster.  One
+// cooperative launch holds items chain CTAs followed by NPREP preparation
+// CTAs per item, placed anywhere on the GPU (clusters of 3 cannot all be
+// placed at once on 148 SMs; single CTAs can).  The tiles travel through a
+// ring of kRing slots per item in a caller-provided global workspace, which
+// stays in L2: the preparation CTA bulk-stores its staging buffer into slot
+// (chunk % kRing) and publishes it with a release flag; the chain CTA
+// acquires the flag and bulk-loads the slot into its buffer, then returns
+// the slot with a second release flag.  Flags hold chunk index + 1 and start
+// at zero.
 // ============================================================================
 
 // chain CTA (rank 0) shared memory
@@ -878,10 +928,10 @@ constexpr uint32_t C_SHIP = 0;            // 2 x 64 KB
 constexpr uint32_t C_VT = 131072;         // V raw -> fp16
 constexpr uint32_t C_S0T = 147456;        // S^T fp16
 constexpr uint32_t C_DT = 180224;         // Delta^T fp16
-constexpr uint32_t C_GS = 196608;         // g in / y out staging
-constexpr uint32_t C_SCAL = 212992;       // shipped scalars [2][4]
-constexpr uint32_t C_RED = 213248;        // red[4][64], rr[64], max[16]
-constexpr uint32_t C_BAR = 214656;        // full[2], mma, tmem slot
+constexpr uint32_t C_GS = 196608;         // g (-> gate factors) per chunk parity, 2 x 16 KB
+constexpr uint32_t C_SCAL = 229376;       // shipped scalars [2][4]
+constexpr uint32_t C_RED = 229632;        // red[4][64], rr[64], max[16]
+constexpr uint32_t C_BAR = 231040;        // full[2], mma, tmem slot
 // prep CTA (rank 1) shared memory
 constexpr uint32_t P_KQ = 0;              // raw [K; Q] bf16
 constexpr uint32_t P_KH = 32768;          // K^ fp16
@@ -895,17 +945,30 @@ constexpr uint32_t P_GATEBUF = 225280;    // [2][la, beta][64]
 constexpr uint32_t P_GATE = 226304;       // G2, beta, gamma, dec, rk, rq
 constexpr uint32_t P_SCAL = 227840;       // scalar staging [2][4]
 constexpr uint32_t P_MAX = 227872;        // block-max scratch [16]
-constexpr uint32_t P_BAR = 227936;        // empty[2], mma, tmem slot
-constexpr uint32_t kPairSmemBytes = 228000 + 1024;
+constexpr uint32_t P_BAR = 227936;        // empty[2], mma, tmem slot, staging free[2]
+constexpr uint32_t kPairSmemBytes = 231072 + 1024;  // the chain CTA's map is the larger
+// split launch: global ring per item
+constexpr int kRing = 4;
+constexpr size_t kSlotBytes = kShipBytes + 256;   // tiles, then scalars [4] fp32
 
-template <int NPREP>
+template <int NPREP, bool kGlobal>
 __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const PrefillArgs a) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sb = (raw + 1023u) & ~1023u;
   uint8_t* gb = smem_raw + (sb - raw);
-  const uint32_t rank = cluster_ctarank();
-  const int item = blockIdx.x / (1 + NPREP);
+  uint32_t rank;
+  int item;
+  if constexpr (kGlobal) {
+    // [0, items): chain CTAs; then NPREP preparation CTAs per item
+    const int items = a.n_seq * a.H_v;
+    const int bx = (int)blockIdx.x;
+    rank = bx < items ? 0u : 1u + (uint32_t)((bx - items) % NPREP);
+    item = bx < items ? bx : (bx - items) / NPREP;
+  } else {
+    rank = cluster_ctarank();
+    item = blockIdx.x / (1 + NPREP);
+  }
   const int seq = item / a.H_v;
   const int h = item % a.H_v;
   const int hq = h / (a.H_v / a.H_qk);
@@ -937,6 +1000,15 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
   const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
   uint32_t phase = 0;
   bool ok = true;
+  // this item's ring of slots and its flags (split launch only)
+  uint8_t* ring = nullptr;
+  unsigned long long* ready = nullptr;
+  unsigned long long* consumed = nullptr;
+  if constexpr (kGlobal) {
+    ring = static_cast<uint8_t*>(a.ring) + (size_t)item * kRing * kSlotBytes;
+    ready = a.ring_flags + (size_t)item * 2 * kRing;
+    consumed = ready + kRing;
+  }
 
   if (rank == 0) {
     // =========================== chain CTA ===========================
@@ -949,12 +1021,14 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
     const float* sScal = reinterpret_cast<const float*>(gb + C_SCAL);
     __nv_bfloat16* Yg = static_cast<__nv_bfloat16*>(a.y);
     const size_t st_off = ((size_t)seq * a.H_v + h) * (size_t)(kD * kD);
+    // Copies: V_c+1 is issued after chunk c's first MMA batch, g_c+1 (into
+    // buffer (c+1) & 1) at the top of chunk c; the loop top waits for all.
     if (t_begin < t_end) {
       const int n0 = (t_end - t_begin) < kC ? (int)(t_end - t_begin) : kC;
       ld.v(t_begin, n0);
       if (has_g) ld.g(t_begin, n0, 0);
-      cp_async_commit();
     }
+    cp_async_commit();
     if (warp == 0) tmem_alloc(tslot, 256);
     if (tid == 0) {
       mbar_init(&full[0], 1);
@@ -964,10 +1038,39 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
     }
     fence_before_sync();
     __syncthreads();
-    cluster_sync();
+    if constexpr (!kGlobal) cluster_sync();
     fence_after_sync();
     const uint32_t tbase = *tslot;
     const uint32_t tS = tbase + lane_off, tD = tbase + lane_off + 128, tY = tbase + lane_off + 192;
+    // Split launch, thread kFetcher only (not the MMA issuer: its proxy
+    // fence would wait for the MMAs in flight): issue the bulk load of chunk
+    // c from its slot into buffer c & 1 (free: it held chunk c - 2, whose
+    // MMAs are complete).  `block` waits (bounded) for the slot's flag;
+    // otherwise a slot not yet published is left for a later call.  Loads
+    // are issued in chunk order; `fetched` counts them.
+    constexpr int kFetcher = 32;
+    int fetched = 0;
+    auto fetch = [&](int c, bool block) -> bool {
+      if (fetched > c) return true;
+      const int s = c % kRing;
+      const unsigned long long want = (unsigned long long)c + 1;
+      if (block) {
+        if (!wait_flag_ge(&ready[s], want, kWaitLimit)) return false;
+      } else if (ld_acquire_u64(&ready[s]) < want) {
+        return true;
+      }
+      fence_proxy_async_global();
+      const int bb = c & 1;
+      const uint8_t* src = ring + (size_t)s * kSlotBytes;
+      mbar_arrive_expect_tx(&full[bb], kShipBytes + 16);
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        bulk_load_g2s(sb + C_SHIP + bb * kShipBytes + 16384 * k, src + 16384 * k, 16384,
+                      &full[bb]);
+      bulk_load_g2s(sb + C_SCAL + 16 * bb, src + kShipBytes, 16, &full[bb]);
+      ++fetched;
+      return true;
+    };
     {
       float v[32];
 #pragma unroll
@@ -982,7 +1085,12 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
       tmem_wait_st();
     }
     int s_exp = 0;
-    const float w1 = 1.f + ((has_g && a.norm_w) ? __ldg(a.norm_w + row) : 0.f);
+    // 1 + w for the 8 output columns this thread stores (the same in every
+    // chunk: piece index tid + 256 k has column block tid % 16)
+    float wv[8];
+#pragma unroll
+    for (int j2 = 0; j2 < 8; ++j2)
+      wv[j2] = 1.f + ((has_g && a.norm_w) ? __ldg(a.norm_w + (tid & 15) * 8 + j2) : 0.f);
 
     int ci = 0;
     for (int64_t c0 = t_begin; c0 < t_end; c0 += kC, ++ci) {
@@ -991,11 +1099,35 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
       const int nn = has_next ? ((t_end - c0 - kC) < kC ? (int)(t_end - c0 - kC) : kC) : 0;
       const int b = ci & 1;
       const uint32_t ship = sb + C_SHIP + b * kShipBytes;
+      const uint32_t gsb = sb + C_GS + b * 16384;  // this chunk's g buffer
       cp_async_wait_all();
-      __syncthreads();
+      // the other g buffer was last read by the previous chunk's epilogue
+      if (has_next && has_g) ld.g(c0 + kC, nn, b ^ 1);
+      cp_async_commit();
+      bool okw = true;
+      if constexpr (kGlobal) {
+        if (tid == kFetcher) okw = fetch(ci, true);
+        if (!__syncthreads_and(okw)) { ok = false; break; }
+      } else {
+        __syncthreads();
+      }
       GDN_TRACE_POINT(0);
-      bool okw = mbar_wait_cluster(&full[b], (ci >> 1) & 1, kWaitLimit);
+      if constexpr (kGlobal) okw = mbar_wait(&full[b], (ci >> 1) & 1, kWaitLimit);
+      else okw = mbar_wait_cluster(&full[b], (ci >> 1) & 1, kWaitLimit);
       if (!__syncthreads_and(okw)) { ok = false; break; }
+      if constexpr (kGlobal) {
+        // Chunk ci's bytes are in shared memory: hand its slot back.  The
+        // bulk reads of the slot are complete (the barrier phase above), so
+        // a relaxed store suffices: nothing this thread did afterwards needs
+        // to be visible to the preparation CTA, and a release here would
+        // first drain this thread's outstanding y stores.
+        if (tid == 0) st_relaxed_u64(&consumed[ci % kRing], (unsigned long long)ci + 1);
+      } else {
+        // the copy has landed: its source staging buffer may be reused
+        if (tid == 0)
+          mbar_remote_arrive(
+              mapa_shared(sb + P_BAR + 32 + 8 * ((ci / NPREP) & 1), 1 + ci % NPREP));
+      }
       GDN_TRACE_POINT(1);
       const float gC = sScal[b * 4 + 0];
       const int f = (int)sScal[b * 4 + 1];
@@ -1017,8 +1149,9 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
       float smax = 0.f;
 #pragma unroll
       for (int x = 0; x < 64; ++x) smax = fmaxf(smax, fabsf(sv[x]));
-      const float mV = block_max(vmax, sMax, warp, lane);
-      const float mS = ldexpf(block_max(smax, sMax, warp, lane), s_exp);
+      const float2 mx = block_max2(vmax, smax, sMax, warp, lane);
+      const float mV = mx.x;
+      const float mS = ldexpf(mx.y, s_exp);
       const int e = scale_exp(mV + 12.f * mS, 12);
       {
         const float sv_scale = ldexpf(1.f, -e);
@@ -1067,6 +1200,28 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
         }
         mma_commit(mbar);
       }
+      if constexpr (kGlobal) {
+        // the next chunk's tiles, while the MMAs run
+        if (tid == kFetcher && has_next) fetch(ci + 1, false);
+      }
+      if (has_g) {
+        // Also while the MMAs run: this chunk's gate factors (1 + w)
+        // sigmoid(g), in place as fp16.  Each thread converts the pieces it
+        // loaded itself (waited for at the loop top), so no barrier is needed.
+        const int ch = tid & 15;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t addr = gsb + ((tid >> 4) + 16 * k) * 256 + ch * 16;
+          float gf[8];
+          unpack_bf16x8(ld_shared_v4(addr), gf);
+          uint32_t o[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            o[q] = pack_f16(__fdividef(wv[2 * q], 1.f + __expf(-gf[2 * q])),
+                            __fdividef(wv[2 * q + 1], 1.f + __expf(-gf[2 * q + 1])));
+          st_shared_v4(addr, o[0], o[1], o[2], o[3]);
+        }
+      }
       okw = mbar_wait(mbar, phase, kWaitLimit);
       phase ^= 1;
       if (!__syncthreads_and(okw)) { ok = false; break; }
@@ -1112,14 +1267,19 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
       if (!__syncthreads_and(okw)) { ok = false; break; }
       fence_after_sync();
       // this chunk's shipped tiles are no longer read: hand the buffer back
-      if (tid == 0) mbar_remote_arrive(mapa_shared(sb + P_BAR + 8 * b, 1 + ci % NPREP));
+      if constexpr (kGlobal) {
+        if (tid == kFetcher && has_next) fetch(ci + 1, false);
+      } else {
+        if (tid == 0) mbar_remote_arrive(mapa_shared(sb + P_BAR + 8 * b, 1 + ci % NPREP));
+      }
       GDN_TRACE_POINT(5);
 
-      // epilogue
+      // epilogue: y = scale 2^e Y^T; with the gate, out = y rr (1 + w) sigmoid(g)
       {
         float v[32];
         tmem_ld32(tY + half * 32, v);
         tmem_wait_ld();
+        GDN_TRACE_POINT(50);
         const float ys = ldexpf(a.scale, e);
 #pragma unroll
         for (int x = 0; x < 32; ++x) v[x] *= ys;
@@ -1138,31 +1298,57 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
             sRr[tid] = rsqrtf((sRed[tid] + sRed[64 + tid] + sRed[128 + tid] + sRed[192 + tid]) /
                                   (float)kD + a.eps_norm);
           __syncthreads();
-        }
-        __nv_bfloat16* gs = reinterpret_cast<__nv_bfloat16*>(gb + C_GS);
+          GDN_TRACE_POINT(51);
+          // y rr (|y rr| <= sqrt(d_v)) as fp16, token-major, into the Delta^T
+          // tile (its MMAs are complete; it is rewritten next chunk)
+          __half* yst = reinterpret_cast<__half*>(gb + C_DT) + half * 32 * kD + row;
+          const float4* rr4 = reinterpret_cast<const float4*>(sRr + half * 32);
 #pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          const int t = half * 32 + x;
-          float o = v[x];
-          if (has_g) {
-            const float gg = __bfloat162float(gs[t * kD + row]);
-            o = __fdividef(o * sRr[t] * w1, 1.f + __expf(-gg));
+          for (int x4 = 0; x4 < 8; ++x4) {
+            const float4 r = rr4[x4];
+            yst[(4 * x4 + 0) * kD] = __float2half_rn(v[4 * x4 + 0] * r.x);
+            yst[(4 * x4 + 1) * kD] = __float2half_rn(v[4 * x4 + 1] * r.y);
+            yst[(4 * x4 + 2) * kD] = __float2half_rn(v[4 * x4 + 2] * r.z);
+            yst[(4 * x4 + 3) * kD] = __float2half_rn(v[4 * x4 + 3] * r.w);
           }
-          gs[t * kD + row] = __float2bfloat16_rn(o);
-        }
-        __syncthreads();
+          __syncthreads();
+          GDN_TRACE_POINT(52);
+          // 8 consecutive outputs of one token per piece: times the gate
+          // factors (this thread's own pieces), pack, store
+          const int ch = tid & 15;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int idx = tid + kNT * k;
-          const int rr = idx >> 4, ch = idx & 15;
-          if (rr < n) {
-            const uint4 val = ld_shared_v4(sb + C_GS + rr * 256 + ch * 16);
-            *reinterpret_cast<uint4*>(Yg + ((size_t)(c0 + rr) * a.H_v + h) * kD + ch * 8) = val;
+          for (int k = 0; k < 4; ++k) {
+            const int rr = (tid >> 4) + 16 * k;
+            if (rr < n) {
+              float yf[8], gf[8];
+              unpack_f16x8(ld_shared_v4(sb + C_DT + rr * 256 + ch * 16), yf);
+              unpack_f16x8(ld_shared_v4(gsb + rr * 256 + ch * 16), gf);
+              uint32_t o[4];
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                o[q] = pack_bf16(yf[2 * q] * gf[2 * q], yf[2 * q + 1] * gf[2 * q + 1]);
+              *reinterpret_cast<uint4*>(Yg + ((size_t)(c0 + rr) * a.H_v + h) * kD + ch * 8) =
+                  make_uint4(o[0], o[1], o[2], o[3]);
+            }
+          }
+        } else {
+          // no gate: y as bf16 through the staging buffer, coalesced stores
+          __nv_bfloat16* gs = reinterpret_cast<__nv_bfloat16*>(gb + C_GS);
+#pragma unroll
+          for (int x = 0; x < 32; ++x) gs[(half * 32 + x) * kD + row] = __float2bfloat16_rn(v[x]);
+          __syncthreads();
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int idx = tid + kNT * k;
+            const int rr = idx >> 4, ch = idx & 15;
+            if (rr < n) {
+              const uint4 val = ld_shared_v4(sb + C_GS + rr * 256 + ch * 16);
+              *reinterpret_cast<uint4*>(Yg + ((size_t)(c0 + rr) * a.H_v + h) * kD + ch * 8) = val;
+            }
           }
         }
-        __syncthreads();
-        if (has_next && has_g) ld.g(c0 + kC, nn, 0);
-        cp_async_commit();
+        __syncthreads();  // staging reads done: g buffer and Delta^T tile reusable
+        GDN_TRACE_POINT(53);
       }
       fence_before_sync();
       GDN_TRACE_POINT(6);
@@ -1185,16 +1371,25 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
     } else {
       if (tid == 0) atomicOr(a.err, kErrTimeout);
       mbar_wait(mbar, phase ^ 1, kWaitLimit);
+      // copies into this CTA's buffers that may still be landing
+      if constexpr (kGlobal) {
+        if (tid == 0)
+          for (int c = ci; c < fetched; ++c) mbar_wait(&full[c & 1], (c >> 1) & 1, kWaitLimit);
+      } else {
+        if (t_begin + (int64_t)(ci + 1) * kC < t_end)
+          mbar_wait_cluster(&full[(ci + 1) & 1], ((ci + 1) >> 1) & 1, kWaitLimit >> 6);
+      }
     }
     fence_before_sync();
     __syncthreads();
-    cluster_sync();
+    if constexpr (!kGlobal) cluster_sync();
     if (warp == 0) tmem_dealloc(tbase, 256);
   } else {
     // =========================== prep CTA ============================
     uint64_t* empty = reinterpret_cast<uint64_t*>(gb + P_BAR);
     uint64_t* mbar = reinterpret_cast<uint64_t*>(gb + P_BAR + 16);
     uint32_t* tslot = reinterpret_cast<uint32_t*>(gb + P_BAR + 24);
+    uint64_t* stg_free = reinterpret_cast<uint64_t*>(gb + P_BAR + 32);
     float* sA = reinterpret_cast<float*>(gb + P_A);
     float* sT = reinterpret_cast<float*>(gb + P_T);
     float* sZ = reinterpret_cast<float*>(gb + P_Z);
@@ -1221,18 +1416,36 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
       mbar_init(&empty[0], 1);
       mbar_init(&empty[1], 1);
       mbar_init(mbar, 1);
+      mbar_init(&stg_free[0], 1);
+      mbar_init(&stg_free[1], 1);
       fence_mbar_init();
     }
     fence_before_sync();
     __syncthreads();
-    cluster_sync();
+    if constexpr (!kGlobal) cluster_sync();
     fence_after_sync();
     const uint32_t tbase = *tslot;
     const uint32_t tKQ = tbase + lane_off, tW = tbase + lane_off + 64;
-    const uint32_t full_cl0 = mapa_shared(sb + C_BAR, 0);
-    const uint32_t ship_cl0 = mapa_shared(sb + C_SHIP, 0);
-    const uint32_t scal_cl0 = mapa_shared(sb + C_SCAL, 0);
+    uint32_t full_cl0 = 0, ship_cl0 = 0, scal_cl0 = 0;
+    if constexpr (!kGlobal) {
+      full_cl0 = mapa_shared(sb + C_BAR, 0);
+      ship_cl0 = mapa_shared(sb + C_SHIP, 0);
+      scal_cl0 = mapa_shared(sb + C_SCAL, 0);
+    }
 
+    // Split launch, thread 0: the slot whose bulk stores are in flight and
+    // not yet published (published once complete, during the next chunk).
+    int pend_slot = -1;
+    unsigned long long pend_val = 0;
+    auto publish = [&]() {
+      if (pend_slot >= 0) {
+        bulk_wait_all();
+        // the stores are complete; publish them to the chain CTA
+        fence_proxy_async_global();
+        st_release_u64(&ready[pend_slot], pend_val);
+        pend_slot = -1;
+      }
+    };
     int ci = first, lc = 0;  // chunk index, local count
     for (int64_t c0 = c_first; c0 < t_end; c0 += (int64_t)kC * NPREP, ci += NPREP, ++lc) {
       const int n = (t_end - c0) < kC ? (int)(t_end - c0) : kC;
@@ -1243,8 +1456,16 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
       const int lb = lc & 1;      // local staging / prefetch buffer
       const uint32_t stg = sb + P_STG + lb * kShipBytes;
       cp_async_wait_all();
-      if (tid == 0) bulk_wait_read_le1();  // staging buffer lb is no longer being copied
-      __syncthreads();
+      bool okw = true;
+      if constexpr (!kGlobal) {
+        // staging buffer lb was the source of the copy two local chunks ago;
+        // the chain CTA reports when that copy has landed.  (The split
+        // launch waits for its stores to complete when it issues them.)
+        if (tid == 0 && lc >= 2)
+          okw = mbar_wait_cluster(&stg_free[lb], ((lc - 2) >> 1) & 1, kWaitLimit);
+      }
+      if (!__syncthreads_and(okw)) { ok = false; break; }
+      GDN_TRACE_POINT(20);
 
       // gates
       if (warp == 0) {
@@ -1276,6 +1497,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
       }
       if (has_next) ld.gates(cnext, nn, lb ^ 1);
       cp_async_commit();
+      GDN_TRACE_POINT(21);
       __syncthreads();
 
       // norms -> K^ (local), gamma Q^ and dec K^ (shipped)
@@ -1323,13 +1545,15 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
           mma_f16(tbase, d, d, ID_BF_KK, kk > 0);
         }
         mma_commit(mbar);
+        if constexpr (kGlobal) publish();
       }
-      bool okw = mbar_wait(mbar, phase, kWaitLimit);
+      okw = mbar_wait(mbar, phase, kWaitLimit);
       phase ^= 1;
       if (!__syncthreads_and(okw)) { ok = false; break; }
       fence_after_sync();
       if (has_next) ld.qk(cnext, nn);
       cp_async_commit();
+      GDN_TRACE_POINT(22);
 
       // A (fp32) and P (fp16, shipped)
       {
@@ -1343,6 +1567,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
         reinterpret_cast<float4*>(sT)[tid + kNT * k] = make_float4(0.f, 0.f, 0.f, 0.f);
       fence_before_sync();
       __syncthreads();
+      GDN_TRACE_POINT(23);
 
       // T = (I + A)^{-1}
       if (tid < 64) {
@@ -1370,6 +1595,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
       tinv_level<8>(sA, sT, sZ, tid);
       tinv_level<16>(sA, sT, sZ, tid);
       tinv_level<32>(sA, sT, sZ, tid);
+      GDN_TRACE_POINT(24);
 
       // f; T diag(b) 2^-f (shipped), T diag(b g) 2^-f (local)
       {
@@ -1408,6 +1634,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
       fence_proxy_async();
       fence_before_sync();
       __syncthreads();
+      GDN_TRACE_POINT(25);
 
       // W^T = K^T (T diag(b g))^T
       if (tid == 0) {
@@ -1441,10 +1668,31 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
       fence_proxy_async();
       fence_before_sync();
       __syncthreads();
+      GDN_TRACE_POINT(26);
 
       // ship this chunk's tiles once the chain CTA has released buffer b
       okw = true;
-      if (tid == 0) {
+      if constexpr (kGlobal) {
+        if (tid == 0) {
+          // slot ci % kRing last held chunk ci - kRing: the chain CTA must
+          // have loaded it
+          const int s = ci % kRing;
+          if (ci >= kRing)
+            okw = wait_flag_ge(&consumed[s], (unsigned long long)(ci - kRing) + 1, kWaitLimit);
+          GDN_TRACE_POINT(30);
+          if (okw) {
+            uint8_t* dst = ring + (size_t)s * kSlotBytes;
+            fence_proxy_async_global();
+#pragma unroll
+            for (int k = 0; k < 4; ++k) bulk_store_s2g(dst + 16384 * k, stg + 16384 * k, 16384);
+            bulk_store_s2g(dst + kShipBytes, sb + P_SCAL + 16 * lb, 16);
+            bulk_commit();
+            pend_slot = s;
+            pend_val = (unsigned long long)ci + 1;
+            GDN_TRACE_POINT(31);
+          }
+        }
+      } else if (tid == 0) {
         okw = mbar_wait_cluster(&empty[b], ((ci >> 1) & 1) ^ 1, kWaitLimit);
         if (okw) {
           // the cluster window keeps the peer's layout: offsets carry over
@@ -1455,12 +1703,15 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
           for (int k = 0; k < 4; ++k)
             bulk_copy_to_peer(ship_cl + 16384 * k, stg + 16384 * k, 16384, full_cl);
           bulk_copy_to_peer(scal_cl0 + 16 * b, sb + P_SCAL + 16 * lb, 16, full_cl);
-          bulk_commit();
         }
       }
       if (!__syncthreads_and(okw)) { ok = false; break; }
+      GDN_TRACE_POINT(27);
     }
     cp_async_wait_all();
+    if constexpr (kGlobal) {
+      if (tid == 0 && ok) publish();
+    }
     if (tid == 0) bulk_wait_all();
     if (!ok) {
       if (tid == 0) atomicOr(a.err, kErrTimeout);
@@ -1468,7 +1719,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
     }
     fence_before_sync();
     __syncthreads();
-    cluster_sync();
+    if constexpr (!kGlobal) cluster_sync();
     if (warp == 0) tmem_dealloc(tbase, 128);
   }
 }
@@ -1477,6 +1728,29 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
 
 bool prefill_tc_supports(const PrefillArgs& a) {
   return a.dtype == GDN_BF16 && a.d_k == kD && a.d_v == kD;
+}
+
+// Split-launch workspace: flags (ready[kRing], consumed[kRing] per item,
+// 64-bit), padded to 256 bytes, then the ring slots (kSlotBytes each, a
+// multiple of 256).  Only batches of at most kSplitMaxItems items can use it.
+constexpr long long kSplitMaxItems = 64;
+
+static size_t split_flag_bytes(long long items) {
+  return ((size_t)items * 2 * kRing * sizeof(unsigned long long) + 255) & ~(size_t)255;
+}
+
+size_t prefill_tc_workspace_bytes(int32_t n_seq, int32_t H_v, int32_t d_k, int32_t d_v,
+                                  gdn_dtype dtype) {
+  const long long items = (long long)n_seq * H_v;
+  if (dtype != GDN_BF16 || d_k != kD || d_v != kD || items < 1 || items > kSplitMaxItems)
+    return 0;
+  return split_flag_bytes(items) + (size_t)items * kRing * kSlotBytes;
+}
+
+void prefill_tc_workspace_layout(void* ws, int32_t n_seq, int32_t H_v, PrefillArgs* a) {
+  const long long items = (long long)n_seq * H_v;
+  a->ring_flags = static_cast<unsigned long long*>(ws);
+  a->ring = static_cast<uint8_t*>(ws) + split_flag_bytes(items);
 }
 
 gdn_status launch_prefill_tc(const PrefillArgs& a, cudaStream_t stream) {
@@ -1493,6 +1767,48 @@ gdn_status launch_prefill_tc(const PrefillArgs& a, cudaStream_t stream) {
   }
   static bool pair_attr_set[64][2] = {{false}};
   const long long items = (long long)a.n_seq * a.H_v;
+  // Split launch (needs the workspace): chain + two preparation CTAs per
+  // item as one cooperative grid, used when every CTA can be resident at
+  // once.  Capacity = co-resident CTAs of that kernel on this device.
+  static int split_capacity[64] = {0};
+  auto split_fits = [&]() -> bool {
+    if (a.ring == nullptr || a.ring_flags == nullptr || items > kSplitMaxItems) return false;
+    if (dev < 0 || dev >= 64) return false;
+    if (split_capacity[dev] == 0) {
+      int cap = -1;
+      const void* fn = (const void*)gdn_prefill_tc_pair_kernel<2, true>;
+      int coop = 0, sms = 0, per_sm = 0;
+      if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)kPairSmemBytes) == cudaSuccess &&
+          cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) == cudaSuccess &&
+          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+          cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kNT, kPairSmemBytes) ==
+              cudaSuccess &&
+          coop)
+        cap = per_sm * sms;
+      split_capacity[dev] = cap;
+    }
+    return split_capacity[dev] >= 3 * items;
+  };
+  if (a.tc_variant == 3 || (a.tc_variant == 0 && split_fits())) {
+    if (!split_fits()) return GDN_ERR_UNSUPPORTED;
+    // flags count chunks from zero in every call
+    if (cudaMemsetAsync(a.ring_flags, 0, split_flag_bytes(items), stream) != cudaSuccess)
+      return GDN_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(3 * items), 1, 1);
+    cfg.blockDim = dim3(kNT, 1, 1);
+    cfg.dynamicSmemBytes = kPairSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, gdn_prefill_tc_pair_kernel<2, true>, a) != cudaSuccess)
+      return GDN_ERR_CUDA;
+    return cudaPeekAtLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+  }
   // While there are too few (sequence, head) items to fill the GPU, give each
   // a cluster: one chain CTA plus one or two preparation CTAs -- but only a
   // cluster size whose clusters all fit on the GPU at once (a second wave
@@ -1501,8 +1817,8 @@ gdn_status launch_prefill_tc(const PrefillArgs& a, cudaStream_t stream) {
   auto fits = [&](int np) -> bool {
     if (dev < 0 || dev >= 64) return false;
     if (max_clusters[dev][np - 1] == 0) {
-      const void* fn = np == 2 ? (const void*)gdn_prefill_tc_pair_kernel<2>
-                               : (const void*)gdn_prefill_tc_pair_kernel<1>;
+      const void* fn = np == 2 ? (const void*)gdn_prefill_tc_pair_kernel<2, false>
+                               : (const void*)gdn_prefill_tc_pair_kernel<1, false>;
       if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)kPairSmemBytes) != cudaSuccess)
         return false;
@@ -1528,8 +1844,8 @@ gdn_status launch_prefill_tc(const PrefillArgs& a, cudaStream_t stream) {
   if (a.tc_variant == 1) nprep = fits(2) ? 2 : 1;
   else if (a.tc_variant == 0) nprep = fits(2) ? 2 : (fits(1) ? 1 : 0);
   if (nprep > 0) {
-    const void* fn = nprep == 2 ? (const void*)gdn_prefill_tc_pair_kernel<2>
-                                : (const void*)gdn_prefill_tc_pair_kernel<1>;
+    const void* fn = nprep == 2 ? (const void*)gdn_prefill_tc_pair_kernel<2, false>
+                                : (const void*)gdn_prefill_tc_pair_kernel<1, false>;
     if (dev < 0 || dev >= 64 || !pair_attr_set[dev][nprep - 1]) {
       if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)kPairSmemBytes) != cudaSuccess)
@@ -1548,8 +1864,8 @@ gdn_status launch_prefill_tc(const PrefillArgs& a, cudaStream_t stream) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t err = nprep == 2 ? cudaLaunchKernelEx(&cfg, gdn_prefill_tc_pair_kernel<2>, a)
-                                 : cudaLaunchKernelEx(&cfg, gdn_prefill_tc_pair_kernel<1>, a);
+    cudaError_t err = nprep == 2 ? cudaLaunchKernelEx(&cfg, gdn_prefill_tc_pair_kernel<2, false>, a)
+                                 : cudaLaunchKernelEx(&cfg, gdn_prefill_tc_pair_kernel<1, false>, a);
     if (err != cudaSuccess) return GDN_ERR_CUDA;
   } else {
     gdn_prefill_tc_kernel<<<(unsigned)items, kNT, kSmemBytes, stream>>>(a);

@@ -20,7 +20,10 @@ HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "gdn.h")
 
 GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_TIMEOUT = range(5)
 GDN_BF16, GDN_FP32 = 0, 1
-PATHS = {"auto": 0, "tensor": 1, "simt": 2, "tensor_pair": 3, "tensor_single": 4}
+PATHS = {"auto": 0, "tensor": 1, "simt": 2, "tensor_pair": 3, "tensor_single": 4,
+         "tensor_split": 5}
+# paths that may run the split layout, which needs a workspace
+_WS_PATHS = ("auto", "tensor", "tensor_split")
 
 _lib = None
 _vp = ctypes.c_void_p
@@ -47,6 +50,14 @@ def load(path: str = LIB_PATH):
     f.argtypes = [_vp] * 9 + [ctypes.c_int32, ctypes.c_int64] + [ctypes.c_int32] * 5 + [
         ctypes.c_int32, ctypes.c_float, ctypes.c_float, ctypes.c_float, _vp, _vp,
         ctypes.c_int, _vp]
+    f = lib.gdn_chunk_fwd_ws
+    f.restype = ctypes.c_int
+    f.argtypes = [_vp] * 9 + [ctypes.c_int32, ctypes.c_int64] + [ctypes.c_int32] * 5 + [
+        ctypes.c_int32, ctypes.c_float, ctypes.c_float, ctypes.c_float, _vp, _vp,
+        ctypes.c_int, _vp, ctypes.c_size_t, _vp]
+    f = lib.gdn_chunk_fwd_workspace_size
+    f.restype = ctypes.c_size_t
+    f.argtypes = [ctypes.c_int32] * 4 + [ctypes.c_int]
     f = lib.gdn_chunk_fwd
     f.restype = ctypes.c_int
     f.argtypes = [_vp] * 9 + [ctypes.c_int32, ctypes.c_int64] + [ctypes.c_int32] * 5 + [
@@ -86,12 +97,16 @@ def _stream_handle(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def _dtype_code(t: torch.Tensor) -> int:
-    if t.dtype == torch.bfloat16:
+def _dtype_code_of(dtype) -> int:
+    if dtype == torch.bfloat16:
         return GDN_BF16
-    if t.dtype == torch.float32:
+    if dtype == torch.float32:
         return GDN_FP32
-    raise TypeError("q/k/v/g must be bfloat16 or float32, got %s" % t.dtype)
+    raise TypeError("q/k/v/g must be bfloat16 or float32, got %s" % dtype)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    return _dtype_code_of(t.dtype)
 
 
 def _check(t: Optional[torch.Tensor], name: str, dtype=None, device=None):
@@ -107,18 +122,27 @@ def _check(t: Optional[torch.Tensor], name: str, dtype=None, device=None):
         raise ValueError("%s is on %s, expected %s" % (name, t.device, device))
 
 
+def workspace_size(n_seq: int, H_v: int, d_k: int, d_v: int, dtype=torch.bfloat16) -> int:
+    """Bytes of workspace the split prefill layout uses (0: not applicable)."""
+    return int(load().gdn_chunk_fwd_workspace_size(n_seq, H_v, d_k, d_v, _dtype_code_of(dtype)))
+
+
 def gdn_chunk_fwd(q, k, v, log_alpha, beta, g=None, norm_w=None,
                   initial_state=None, cu_seqlens=None, l2norm_qk=True,
                   eps_l2=1e-6, eps_norm=1e-6, scale=1.0, y=None,
                   final_state=None, output_final_state=True, path="auto",
-                  stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+                  workspace="auto", stream=None
+                  ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Chunked prefill over packed sequences: returns (y, final_state).
 
     q, k [T, H_qk, d_k]; v [T, H_v, d_v]; log_alpha, beta [T, H_v] fp32;
     g [T, H_v, d_v] or None; norm_w [d_v] fp32 or None; initial_state
     [n_seq, H_v, d_k, d_v] fp32 or None; cu_seqlens [n_seq + 1] int32 (device)
     or None.  y / final_state may be passed in (final_state may be
-    initial_state itself for an in-place update).
+    initial_state itself for an in-place update).  ``workspace``: a uint8
+    CUDA tensor of at least ``workspace_size(...)`` bytes, None (no split
+    layout), or "auto" (allocated here through torch when the path may use
+    it).  A workspace must not be shared by calls that can overlap.
     """
     lib = load()
     dev = q.device
@@ -138,11 +162,21 @@ def gdn_chunk_fwd(q, k, v, log_alpha, beta, g=None, norm_w=None,
     if final_state is None and output_final_state:
         final_state = torch.empty((n_seq, Hv, dk, dv), dtype=torch.float32, device=dev)
     _check(final_state, "final_state", torch.float32, dev)
-    st = lib.gdn_chunk_fwd_path(
+    if isinstance(workspace, str):
+        if workspace != "auto":
+            raise ValueError("workspace must be a tensor, None or 'auto'")
+        workspace = None
+        if path in _WS_PATHS:
+            nbytes = int(lib.gdn_chunk_fwd_workspace_size(n_seq, Hv, dk, dv, dt))
+            if nbytes > 0:
+                workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    _check(workspace, "workspace", torch.uint8, dev)
+    ws_bytes = 0 if workspace is None else workspace.numel()
+    st = lib.gdn_chunk_fwd_ws(
         _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(g), _ptr(norm_w),
         _ptr(initial_state), _ptr(cu_seqlens), n_seq, T, Hqk, Hv, dk, dv, dt,
         1 if l2norm_qk else 0, float(eps_l2), float(eps_norm), float(scale), _ptr(y),
-        _ptr(final_state), PATHS[path], _stream_handle(stream))
+        _ptr(final_state), PATHS[path], _ptr(workspace), ws_bytes, _stream_handle(stream))
     if st != GDN_OK:
         raise GdnError(st, "gdn_chunk_fwd")
     return y, final_state

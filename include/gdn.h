@@ -41,6 +41,7 @@
 #ifndef GDN_H_
 #define GDN_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -64,16 +65,19 @@ typedef enum { GDN_BF16 = 0, GDN_FP32 = 1 } gdn_dtype;
 /* Which prefill kernel runs.  AUTO picks the tensor-core kernel when it
  * supports the shape (bf16, d_k = d_v = 128) and the portable CUDA-core
  * kernel otherwise.  The tensor kernel runs either one CTA per (sequence,
- * value head) or, when there are too few of those to fill the GPU, a pair of
- * CTAs per item that split the per-chunk work; PAIR / SINGLE force one
- * layout (same results up to rounding).  A tensor path on an unsupported
- * shape is GDN_ERR_UNSUPPORTED. */
+ * value head) or, when there are too few of those to fill the GPU, several
+ * CTAs per item that split the per-chunk work: a cluster (PAIR) or, given a
+ * workspace (gdn_chunk_fwd_ws), one chain CTA and two preparation CTAs per
+ * item exchanging tiles through the workspace (SPLIT).  PAIR / SINGLE /
+ * SPLIT force one layout (same results up to rounding).  A tensor path on an
+ * unsupported shape is GDN_ERR_UNSUPPORTED. */
 typedef enum {
   GDN_PATH_AUTO = 0,
   GDN_PATH_TENSOR = 1,        /* tcgen05 MMA + TMEM chunked kernel, layout chosen by size */
   GDN_PATH_SIMT = 2,          /* fp32 CUDA-core chunked kernel                           */
   GDN_PATH_TENSOR_PAIR = 3,   /* tensor kernel, two CTAs (a cluster) per sequence x head */
-  GDN_PATH_TENSOR_SINGLE = 4  /* tensor kernel, one CTA per sequence x head              */
+  GDN_PATH_TENSOR_SINGLE = 4, /* tensor kernel, one CTA per sequence x head             */
+  GDN_PATH_TENSOR_SPLIT = 5   /* tensor kernel, chain + 2 prep CTAs per item; workspace  */
 } gdn_prefill_path;
 
 /*
@@ -118,6 +122,45 @@ gdn_status gdn_chunk_fwd_path(
     gdn_dtype in_dtype, int32_t l2norm_qk, float eps_l2, float eps_norm,
     float scale, void* y, float* final_state, gdn_prefill_path path,
     gdn_stream_t stream);
+
+/*
+ * gdn_chunk_fwd_workspace_size -- bytes of device workspace that
+ * gdn_chunk_fwd_ws can use for a batch of n_seq sequences x H_v value heads
+ * (the split layout: a ring of four 64.25 KB hand-off slots plus 64 bytes of
+ * flags per item).  Returns 0 when that layout cannot apply to the shape:
+ * not bf16 with d_k = d_v = 128, or more than 64 items.  Host only; no CUDA
+ * call.
+ */
+size_t gdn_chunk_fwd_workspace_size(int32_t n_seq, int32_t H_v, int32_t d_k, int32_t d_v,
+                                    gdn_dtype in_dtype);
+
+/*
+ * gdn_chunk_fwd_ws -- gdn_chunk_fwd_path with a caller-owned device
+ * workspace that enables the split layout for small batches.
+ *
+ *   workspace        DEVICE pointer, 256-byte aligned, or NULL (then this is
+ *                    gdn_chunk_fwd_path)
+ *   workspace_bytes  its size; must be >= gdn_chunk_fwd_workspace_size(...)
+ *                    when workspace is not NULL (else GDN_ERR_INVALID_ARG)
+ *
+ * With AUTO / TENSOR, the split layout runs when the workspace is given and
+ * all 3 x n_seq x H_v CTAs fit on the device at once (one cooperative
+ * launch); otherwise the call behaves as gdn_chunk_fwd_path and the
+ * workspace is not touched.  SPLIT without a workspace is
+ * GDN_ERR_INVALID_ARG; SPLIT on a batch that does not fit is
+ * GDN_ERR_UNSUPPORTED.  The library clears the workspace's flags on `stream`
+ * at the start of every call (an asynchronous memset), so no initialisation
+ * is needed; its contents are meaningless between calls.  Two calls that
+ * may run at the same time (different streams) must not share a workspace.
+ */
+gdn_status gdn_chunk_fwd_ws(
+    const void* q, const void* k, const void* v, const float* log_alpha,
+    const float* beta, const void* g, const float* norm_w,
+    const float* initial_state, const int32_t* cu_seqlens, int32_t n_seq,
+    int64_t total_T, int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v,
+    gdn_dtype in_dtype, int32_t l2norm_qk, float eps_l2, float eps_norm,
+    float scale, void* y, float* final_state, gdn_prefill_path path,
+    void* workspace, size_t workspace_bytes, gdn_stream_t stream);
 
 /* gdn_chunk_fwd -- gdn_chunk_fwd_path with GDN_PATH_AUTO. */
 gdn_status gdn_chunk_fwd(

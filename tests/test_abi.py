@@ -17,7 +17,8 @@ def lib():
 
 def test_exports_every_declared_function(lib):
     names = gdn.header_functions()
-    assert set(names) >= {"gdn_chunk_fwd", "gdn_chunk_fwd_path", "gdn_decode_step",
+    assert set(names) >= {"gdn_chunk_fwd", "gdn_chunk_fwd_path", "gdn_chunk_fwd_ws",
+                          "gdn_chunk_fwd_workspace_size", "gdn_decode_step",
                           "gdn_check_device_error", "gdn_status_string", "gdn_version"}
     for n in names:
         assert hasattr(lib, n), "libgdn.so does not export %s" % n
@@ -83,6 +84,42 @@ def test_chunk_fwd_rejects_bad_arguments_on_host(lib, kw, code):
 ])
 def test_decode_rejects_bad_arguments_on_host(lib, kw, code):
     assert _decode(lib, **kw) == code
+
+
+def _chunk_ws(lib, ws=None, ws_bytes=0, path=0, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, b=FAKE, g=None, w=None, s0=None, cu=None,
+             n_seq=1, T=64, Hqk=16, Hv=48, dk=128, dv=128, dt=0, l2=1, e1=1e-6, e2=1e-6,
+             sc=1.0, y=FAKE, fs=None)
+    a.update(kw)
+    return lib.gdn_chunk_fwd_ws(a["q"], a["k"], a["v"], a["la"], a["b"], a["g"], a["w"],
+                                a["s0"], a["cu"], a["n_seq"], a["T"], a["Hqk"], a["Hv"],
+                                a["dk"], a["dv"], a["dt"], a["l2"], a["e1"], a["e2"],
+                                a["sc"], a["y"], a["fs"], path, ws, ws_bytes, None)
+
+
+def test_workspace_size(lib):
+    """Split layout: 64 bytes of flags per item (padded to 256), then four
+    64 KB + 256 B slots per item; nothing for shapes it cannot serve."""
+    one = 4 * (65536 + 256)
+    assert gdn.workspace_size(1, 48, 128, 128) == 48 * 64 + 48 * one
+    assert gdn.workspace_size(1, 1, 128, 128) == 256 + one
+    assert gdn.workspace_size(2, 32, 128, 128) == 64 * 64 + 64 * one
+    assert gdn.workspace_size(3, 32, 128, 128) == 0          # more than 64 items
+    assert gdn.workspace_size(1, 48, 64, 128) == 0
+    assert gdn.workspace_size(1, 48, 128, 128, dtype=__import__("torch").float32) == 0
+    assert lib.gdn_chunk_fwd_workspace_size(0, 48, 128, 128, 0) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(ws=FAKE + 16, ws_bytes=1 << 30), gdn.GDN_ERR_INVALID_ARG),   # not 256-aligned
+    (dict(ws=FAKE, ws_bytes=1000), gdn.GDN_ERR_INVALID_ARG),           # too small
+    (dict(path=5), gdn.GDN_ERR_INVALID_ARG),                           # split, no workspace
+    (dict(path=5, ws=FAKE, ws_bytes=1 << 30, dk=64), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(path=5, ws=FAKE, ws_bytes=1 << 30, dt=1), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(path=6), gdn.GDN_ERR_INVALID_ARG),
+])
+def test_chunk_fwd_ws_rejects_bad_workspace_on_host(lib, kw, code):
+    assert _chunk_ws(lib, **kw) == code
 
 
 def test_decode_with_no_sequences_is_a_no_op(lib):

@@ -17,7 +17,7 @@ from tests._parity import errors, oracle_prefill, to_device
 
 pytestmark = pytest.mark.gpu
 
-PATHS = ["simt", "tensor_single", "tensor_pair"]
+PATHS = ["simt", "tensor_single", "tensor_pair", "tensor_split"]
 
 
 def _run(w, path, **kw):
@@ -112,7 +112,7 @@ def test_caller_normalised_keys_and_scale(path):
     _check(fs, s_ref, 1.0, "state")
 
 
-@pytest.mark.parametrize("path", ["auto", "simt"])
+@pytest.mark.parametrize("path", ["auto", "simt", "tensor_split", "tensor_pair"])
 def test_empty_batch(path):
     """total_T = 0: nothing to scan, the final state is the initial state."""
     w = to_device(_case(T=0))

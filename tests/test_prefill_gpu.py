@@ -1,9 +1,10 @@
 """Chunked prefill on the GPU against the fp64 oracle.
 
 Covers every kernel (``simt``: fp32 CUDA cores, every shape and dtype;
-``tensor_single`` / ``tensor_pair``: the tcgen05 kernel for bf16, d_k = d_v =
-128, with one CTA or a two-CTA cluster per (sequence, head)) on the workload
-recipes
+``tensor_single`` / ``tensor_pair`` / ``tensor_split``: the tcgen05 kernel for
+bf16, d_k = d_v = 128, with one CTA, a cluster, or a chain CTA and two
+preparation CTAs exchanging tiles through a global workspace per (sequence,
+head)) on the workload recipes
 (shortened where the oracle must see every output), ragged chunk tails,
 empty and one-token sequences, packed batches, in-place state update,
 split-and-carry, and sampled outputs at the full workload sizes.
@@ -17,7 +18,9 @@ from tests._parity import assert_close, oracle_prefill, to_device
 
 pytestmark = pytest.mark.gpu
 
-BF16_PATHS = ["simt", "tensor_single", "tensor_pair"]
+BF16_PATHS = ["simt", "tensor_single", "tensor_pair", "tensor_split"]
+# the split layout needs all 3 x items CTAs resident: batches of <= 49 items
+MANY_ITEM_PATHS = ["simt", "tensor_single", "tensor_pair"]
 
 
 def _run(w, path="auto", **kw):
@@ -50,7 +53,7 @@ def test_model_shape_ragged_lengths(path, T):
     _check_all(w, y, fs, torch.bfloat16, "T=%d %s" % (T, path))
 
 
-@pytest.mark.parametrize("path", BF16_PATHS)
+@pytest.mark.parametrize("path", MANY_ITEM_PATHS)
 @pytest.mark.parametrize("epilogue", [True, False])
 def test_packed_varlen_small(path, epilogue):
     lengths = [0, 5, 64, 130, 1, 77, 0, 128]
@@ -60,6 +63,43 @@ def test_packed_varlen_small(path, epilogue):
     _check_all(w, y, fs, torch.bfloat16, "varlen %s" % path)
     # empty sequences: final state is the initial state
     np.testing.assert_array_equal(fs[0].cpu().numpy(), w.initial_state[0].cpu().numpy())
+
+
+@pytest.mark.parametrize("path", ["tensor_split", "tensor_pair"])
+@pytest.mark.parametrize("epilogue", [True, False])
+def test_packed_varlen_few_heads(path, epilogue):
+    """Packed sequences with 1 QK / 4 value heads (32 items): ragged, empty
+    and one-token sequences through the small-batch layouts."""
+    lengths = [0, 5, 64, 130, 1, 77, 0, 128]
+    w = to_device(inputs.make_prefill(lengths, 1, 4, 128, 128, seed=8, epilogue=epilogue,
+                                      s0_std=0.01))
+    y, fs = _run(w, path)
+    _check_all(w, y, fs, torch.bfloat16, "varlen few heads %s" % path)
+    np.testing.assert_array_equal(fs[0].cpu().numpy(), w.initial_state[0].cpu().numpy())
+
+
+def test_split_workspace_reuse_and_fallback():
+    """One workspace serves consecutive calls (its flags are cleared by each
+    call); without a workspace AUTO takes another layout, with the same
+    results up to rounding."""
+    w = to_device(inputs.make_prefill([333], 16, 48, 128, 128, seed=13, s0_std=0.01))
+    ws = torch.empty(gdn.workspace_size(1, 48, 128, 128), dtype=torch.uint8, device="cuda")
+    outs = []
+    for _ in range(2):
+        outs.append(_run(w, "tensor_split", workspace=ws))
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+    y_nows, s_nows = _run(w, "auto", workspace=None)
+    y_ref, s_ref, _ = oracle_prefill(w)
+    assert_close(outs[0][0], y_ref, torch.bfloat16, "split y")
+    assert_close(y_nows, y_ref, torch.bfloat16, "no-workspace y")
+    assert_close(s_nows, s_ref, torch.bfloat16, "no-workspace state")
+
+
+def test_split_rejects_batches_that_do_not_fit():
+    w = to_device(inputs.make_prefill([10, 10], 16, 48, 128, 128, seed=1))  # 96 items
+    with pytest.raises(gdn.GdnError) as e:
+        _run(w, "tensor_split")
+    assert e.value.status in (gdn.GDN_ERR_UNSUPPORTED, gdn.GDN_ERR_INVALID_ARG)
 
 
 @pytest.mark.parametrize("dk,dv", [(16, 16), (16, 128), (128, 16), (32, 64), (64, 32),
@@ -81,7 +121,8 @@ def test_fp32_model_shape():
 
 @pytest.mark.parametrize("path", BF16_PATHS)
 def test_in_place_state_update(path):
-    w = to_device(inputs.make_prefill([90, 40], 16, 48, 128, 128, seed=11, s0_std=0.01))
+    # 2 sequences x 16 value heads: few enough items for every layout
+    w = to_device(inputs.make_prefill([90, 40], 4, 16, 128, 128, seed=11, s0_std=0.01))
     y_ref, s_ref, _ = oracle_prefill(w)
     st = w.initial_state.clone()
     y, fs = gdn_chunk_fwd(w.q, w.k, w.v, w.log_alpha, w.beta, g=w.g, norm_w=w.norm_w,
@@ -126,7 +167,7 @@ def test_native_context_T262144_sampled_heads(path):
     assert_close(fs[:, heads], s_ref, torch.bfloat16, "final state")
 
 
-@pytest.mark.parametrize("path", BF16_PATHS)
+@pytest.mark.parametrize("path", MANY_ITEM_PATHS)
 def test_packed_varlen_full_sampled(path):
     """24 sequences (~200k tokens) with their own states; sampled
     (sequence, head) pairs against the oracle, plus no leakage: every final
