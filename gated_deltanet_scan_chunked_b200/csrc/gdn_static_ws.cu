@@ -1,0 +1,59 @@
+// gdn_chunk_fwd_static_ws: the split-layout prefill with its hand-off
+// workspace in a fixed device array of this library, for callers that cannot
+// hand the library any memory.  Nothing here allocates: the array is part of
+// the module image, its address comes from cudaGetSymbolAddress (looked up
+// once per device), and the call forwards to gdn_chunk_fwd_ws.
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "gdn_internal.h"
+
+namespace gdn {
+namespace {
+
+// Capacity: 48 (sequence, value head) items -- one sequence of a 48-value-head
+// layer.  Per item the split layout needs 64 bytes of flags and four 64.25 KB
+// hand-off slots, 263,232 bytes; 48 items need 12,635,136 bytes.
+constexpr int kStaticItems = 48;
+constexpr size_t kStaticBytes = (size_t)kStaticItems * 64 + (size_t)kStaticItems * 4 * 65792;
+
+static __device__ __align__(256) unsigned char g_static_ws[kStaticBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_ws_mu;
+void* g_ws_ptr[kMaxDevices] = {nullptr};
+
+void* static_ws_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_ws_mu);
+  if (g_ws_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_ws) != cudaSuccess) return nullptr;
+    g_ws_ptr[dev] = p;
+  }
+  return g_ws_ptr[dev];
+}
+
+}  // namespace
+}  // namespace gdn
+
+extern "C" gdn_status gdn_chunk_fwd_static_ws(
+    const void* q, const void* k, const void* v, const float* log_alpha, const float* beta,
+    const void* g, const float* norm_w, const float* initial_state, const int32_t* cu_seqlens,
+    int32_t n_seq, int64_t total_T, int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v,
+    gdn_dtype in_dtype, int32_t l2norm_qk, float eps_l2, float eps_norm, float scale, void* y,
+    float* final_state, gdn_stream_t stream) {
+  if (n_seq < 1 || H_v < 1) return GDN_ERR_INVALID_ARG;
+  const size_t need = gdn_chunk_fwd_workspace_size(n_seq, H_v, d_k, d_v, in_dtype);
+  // a shape the split layout does not serve, or more items than the array holds
+  if (need == 0 || need > gdn::kStaticBytes) return GDN_ERR_UNSUPPORTED;
+  void* ws = gdn::static_ws_ptr();
+  if (ws == nullptr) return GDN_ERR_CUDA;
+  // the split launch clears the array's flags on `stream` before its kernel
+  return gdn_chunk_fwd_ws(q, k, v, log_alpha, beta, g, norm_w, initial_state, cu_seqlens, n_seq,
+                          total_T, H_qk, H_v, d_k, d_v, in_dtype, l2norm_qk, eps_l2, eps_norm,
+                          scale, y, final_state, GDN_PATH_TENSOR_SPLIT, ws, gdn::kStaticBytes,
+                          stream);
+}

@@ -55,6 +55,10 @@ def load(path: str = LIB_PATH):
     f.argtypes = [_vp] * 9 + [ctypes.c_int32, ctypes.c_int64] + [ctypes.c_int32] * 5 + [
         ctypes.c_int32, ctypes.c_float, ctypes.c_float, ctypes.c_float, _vp, _vp,
         ctypes.c_int, _vp, ctypes.c_size_t, _vp]
+    f = lib.gdn_chunk_fwd_static_ws
+    f.restype = ctypes.c_int
+    f.argtypes = [_vp] * 9 + [ctypes.c_int32, ctypes.c_int64] + [ctypes.c_int32] * 5 + [
+        ctypes.c_int32, ctypes.c_float, ctypes.c_float, ctypes.c_float, _vp, _vp, _vp]
     f = lib.gdn_chunk_fwd_workspace_size
     f.restype = ctypes.c_size_t
     f.argtypes = [ctypes.c_int32] * 4 + [ctypes.c_int]
@@ -179,6 +183,42 @@ def gdn_chunk_fwd(q, k, v, log_alpha, beta, g=None, norm_w=None,
         _ptr(final_state), PATHS[path], _ptr(workspace), ws_bytes, _stream_handle(stream))
     if st != GDN_OK:
         raise GdnError(st, "gdn_chunk_fwd")
+    return y, final_state
+
+
+def gdn_chunk_fwd_static_ws(q, k, v, log_alpha, beta, g=None, norm_w=None,
+                            initial_state=None, cu_seqlens=None, l2norm_qk=True,
+                            eps_l2=1e-6, eps_norm=1e-6, scale=1.0, y=None,
+                            final_state=None, output_final_state=True, stream=None
+                            ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """The split-layout prefill with the library's own fixed workspace (at
+    most 48 sequence x head items); arguments and results as gdn_chunk_fwd.
+    Calls that can overlap must not be made (they share that workspace)."""
+    lib = load()
+    dev = q.device
+    dt = _dtype_code(q)
+    T, Hqk, dk = q.shape
+    Hv, dv = v.shape[1], v.shape[2]
+    n_seq = 1 if cu_seqlens is None else int(cu_seqlens.shape[0]) - 1
+    for name, t in (("q", q), ("k", k), ("v", v), ("g", g)):
+        _check(t, name, q.dtype, dev)
+    for name, t in (("log_alpha", log_alpha), ("beta", beta), ("norm_w", norm_w),
+                    ("initial_state", initial_state)):
+        _check(t, name, torch.float32, dev)
+    _check(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    if y is None:
+        y = torch.empty((T, Hv, dv), dtype=q.dtype, device=dev)
+    _check(y, "y", q.dtype, dev)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((n_seq, Hv, dk, dv), dtype=torch.float32, device=dev)
+    _check(final_state, "final_state", torch.float32, dev)
+    st = lib.gdn_chunk_fwd_static_ws(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(g), _ptr(norm_w),
+        _ptr(initial_state), _ptr(cu_seqlens), n_seq, T, Hqk, Hv, dk, dv, dt,
+        1 if l2norm_qk else 0, float(eps_l2), float(eps_norm), float(scale), _ptr(y),
+        _ptr(final_state), _stream_handle(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_chunk_fwd_static_ws")
     return y, final_state
 
 

@@ -162,6 +162,35 @@ gdn_status gdn_chunk_fwd_ws(
     float scale, void* y, float* final_state, gdn_prefill_path path,
     void* workspace, size_t workspace_bytes, gdn_stream_t stream);
 
+/*
+ * gdn_chunk_fwd_static_ws -- gdn_chunk_fwd_ws with GDN_PATH_TENSOR_SPLIT and
+ * a workspace that is a fixed array inside the library (12,635,136 bytes of
+ * device memory per device, part of the module image) instead of caller
+ * memory: for callers that cannot give the library any memory.  The method's
+ * description has no counterpart to this call; it is a deployment variant of
+ * the split layout.  Nothing is allocated.
+ *
+ *   Arguments as for gdn_chunk_fwd.
+ *   Capacity: n_seq * H_v <= 48 items.  A larger batch, or a shape the split
+ *   layout does not serve (not bf16 with d_k = d_v = 128), returns
+ *   GDN_ERR_UNSUPPORTED before anything is enqueued; so does a batch whose
+ *   3 x n_seq x H_v CTAs cannot all be resident on the device.
+ *   The first call on each device looks the array's address up
+ *   (cudaGetSymbolAddress, which may load the module); make that first call
+ *   outside stream capture.  Each call clears the array's flags on `stream`
+ *   before its kernel runs, so nothing needs initialising.
+ *   All calls on a device share the one array: calls that can overlap (other
+ *   streams, other host threads) race on it and must be serialised by the
+ *   caller.  Calls on one stream are ordered and safe.
+ */
+gdn_status gdn_chunk_fwd_static_ws(
+    const void* q, const void* k, const void* v, const float* log_alpha,
+    const float* beta, const void* g, const float* norm_w,
+    const float* initial_state, const int32_t* cu_seqlens, int32_t n_seq,
+    int64_t total_T, int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v,
+    gdn_dtype in_dtype, int32_t l2norm_qk, float eps_l2, float eps_norm,
+    float scale, void* y, float* final_state, gdn_stream_t stream);
+
 /* gdn_chunk_fwd -- gdn_chunk_fwd_path with GDN_PATH_AUTO. */
 gdn_status gdn_chunk_fwd(
     const void* q, const void* k, const void* v, const float* log_alpha,

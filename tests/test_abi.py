@@ -131,3 +131,18 @@ def test_binding_refuses_cpu_tensors(lib):
     q = torch.zeros(4, 1, 16)
     with pytest.raises(ValueError):
         gdn.gdn_chunk_fwd(q, q, torch.zeros(4, 1, 16), torch.zeros(4, 1), torch.zeros(4, 1))
+
+
+def test_static_workspace_call_rejects_on_host(lib):
+    """gdn_chunk_fwd_static_ws: over-capacity batches (96 items) and shapes
+    the split layout does not serve are refused before any CUDA call."""
+    def call(**kw):
+        a = dict(cu=FAKE, n_seq=2, Hv=48, dk=128, dt=0)
+        a.update(kw)
+        return lib.gdn_chunk_fwd_static_ws(FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None,
+                                           a["cu"], a["n_seq"], 64, 16, a["Hv"], a["dk"], 128,
+                                           a["dt"], 1, 1e-6, 1e-6, 1.0, FAKE, None, None)
+    assert call() == gdn.GDN_ERR_UNSUPPORTED
+    assert call(n_seq=1, cu=None, dk=64) == gdn.GDN_ERR_UNSUPPORTED
+    assert call(n_seq=1, cu=None, dt=1) == gdn.GDN_ERR_UNSUPPORTED
+    assert call(n_seq=0) == gdn.GDN_ERR_INVALID_ARG
