@@ -96,6 +96,8 @@ constexpr uint32_t ID_KK = idesc_f16(128, 64, false, false, false, true);
 constexpr uint32_t ID_MK = idesc_f16(128, 64, true, false, false, true);
 constexpr uint32_t ID_KM_NEG = idesc_f16(128, 64, false, true, true, true);
 constexpr uint32_t ID_KM128 = idesc_f16(128, 128, false, true, false, true);
+constexpr uint32_t ID_KK128 = idesc_f16(128, 128, false, false, false, true);
+constexpr uint32_t ID_W64 = idesc_f16(64, 128, false, true, false, true);
 
 // fp32 64 x 64 scratch with an XOR swizzle on float4 groups (no padding)
 __device__ __forceinline__ int fidx(int r, int c) { return r * 64 + (c ^ ((r & 7) << 2)); }
@@ -922,13 +924,12 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
 // ============================================================================
 
 // chain CTA (rank 0) shared memory
-constexpr uint32_t SH_KT = 0, SH_QG = 16384, SH_WT = 32768, SH_P = 49152, SH_TB = 57344;
+// shipped tiles: dec K^ [t][d_k]; [-W; gamma Q^] [128][d_k] (K-major, rows 0-63
+// -W, rows 64-127 gamma Q^: one N = 128 MMA gives [Delta^T | Y^T]); P; T diag(b)
+constexpr uint32_t SH_KT = 0, SH_WQ = 16384, SH_P = 49152, SH_TB = 57344;
 constexpr uint32_t kShipBytes = 65536;
-constexpr uint32_t C_SHIP = 0;            // 2 x 64 KB
-constexpr uint32_t C_VT = 131072;         // V raw -> fp16
-constexpr uint32_t C_S0T = 147456;        // S^T fp16
-constexpr uint32_t C_DT = 180224;         // Delta^T fp16
-constexpr uint32_t C_GS = 196608;         // g (-> gate factors) per chunk parity, 2 x 16 KB
+constexpr uint32_t C_SHIP = 0;            // 2 ship buffers; then V raw -> fp16, S^T fp16,
+                                          // Delta^T fp16, g (cluster launch): see the kernel
 constexpr uint32_t C_SCAL = 229376;       // shipped scalars [2][4]
 constexpr uint32_t C_RED = 229632;        // red[4][64], rr[64], max[16]
 constexpr uint32_t C_BAR = 231040;        // full[2], mma, tmem slot
@@ -949,10 +950,23 @@ constexpr uint32_t P_BAR = 227936;        // empty[2], mma, tmem slot, staging f
 constexpr uint32_t kPairSmemBytes = 231072 + 1024;  // the chain CTA's map is the larger
 // split launch: global ring per item
 constexpr int kRing = 4;
-constexpr size_t kSlotBytes = kShipBytes + 256;   // tiles, then scalars [4] fp32
+// slot: tiles (64 KB), gate factors (1 + w) sigmoid(g) fp16 [64][128] (16 KB),
+// scalars [4] fp32 (16 B), padding to a multiple of 256
+constexpr uint32_t kSlotGF = kShipBytes;
+constexpr uint32_t kSlotLoad = kShipBytes + 16384;  // bytes of tiles + gate factors
+constexpr size_t kSlotBytes = kSlotLoad + 256;
 
 template <int NPREP, bool kGlobal>
 __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const PrefillArgs a) {
+  // chain CTA map: 2 ship buffers (the split launch also ships the gate
+  // factors: 80 KB each), V, S^T, Delta^T, and (cluster launch only) two g
+  // buffers; then C_SCAL / C_RED / C_BAR at fixed offsets.
+  constexpr uint32_t kShipStride = kGlobal ? kSlotLoad : kShipBytes;
+  constexpr uint32_t X_VT = C_SHIP + 2 * kShipStride;
+  constexpr uint32_t X_S0T = X_VT + 16384;
+  constexpr uint32_t X_DT = X_S0T + 32768;
+  constexpr uint32_t X_GS = X_DT + 16384;
+  static_assert((kGlobal ? X_GS : X_GS + 32768) <= C_SCAL, "chain shared-memory map overlaps");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sb = (raw + 1023u) & ~1023u;
@@ -994,8 +1008,8 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
   ld.tid = tid;
   ld.sb = sb;
   ld.off_kq = P_KQ;
-  ld.off_vt = C_VT;
-  ld.off_gs = C_GS;
+  ld.off_vt = X_VT;
+  ld.off_gs = X_GS;
   ld.off_gate = P_GATEBUF;
   const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
   uint32_t phase = 0;
@@ -1026,7 +1040,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
     if (t_begin < t_end) {
       const int n0 = (t_end - t_begin) < kC ? (int)(t_end - t_begin) : kC;
       ld.v(t_begin, n0);
-      if (has_g) ld.g(t_begin, n0, 0);
+      if (!kGlobal && has_g) ld.g(t_begin, n0, 0);
     }
     cp_async_commit();
     if (warp == 0) tmem_alloc(tslot, 256);
@@ -1062,12 +1076,12 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
       fence_proxy_async_global();
       const int bb = c & 1;
       const uint8_t* src = ring + (size_t)s * kSlotBytes;
-      mbar_arrive_expect_tx(&full[bb], kShipBytes + 16);
+      mbar_arrive_expect_tx(&full[bb], kSlotLoad + 16);
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
-        bulk_load_g2s(sb + C_SHIP + bb * kShipBytes + 16384 * k, src + 16384 * k, 16384,
+      for (int k = 0; k < 5; ++k)
+        bulk_load_g2s(sb + C_SHIP + bb * kShipStride + 16384 * k, src + 16384 * k, 16384,
                       &full[bb]);
-      bulk_load_g2s(sb + C_SCAL + 16 * bb, src + kShipBytes, 16, &full[bb]);
+      bulk_load_g2s(sb + C_SCAL + 16 * bb, src + kSlotLoad, 16, &full[bb]);
       ++fetched;
       return true;
     };
@@ -1098,11 +1112,13 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
       const bool has_next = c0 + kC < t_end;
       const int nn = has_next ? ((t_end - c0 - kC) < kC ? (int)(t_end - c0 - kC) : kC) : 0;
       const int b = ci & 1;
-      const uint32_t ship = sb + C_SHIP + b * kShipBytes;
-      const uint32_t gsb = sb + C_GS + b * 16384;  // this chunk's g buffer
+      const uint32_t ship = sb + C_SHIP + b * kShipStride;
+      // this chunk's gate factors: shipped (split launch) or computed here
+      // from g in place (cluster launch)
+      const uint32_t gsb = kGlobal ? ship + kSlotGF : sb + X_GS + b * 16384;
       cp_async_wait_all();
       // the other g buffer was last read by the previous chunk's epilogue
-      if (has_next && has_g) ld.g(c0 + kC, nn, b ^ 1);
+      if (!kGlobal && has_next && has_g) ld.g(c0 + kC, nn, b ^ 1);
       cp_async_commit();
       bool okw = true;
       if constexpr (kGlobal) {
@@ -1138,7 +1154,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const int idx = tid + kNT * k;
-        unpack_bf16x8(ld_shared_v4(sb + C_VT + sw128_chunk(idx >> 4, idx & 15, 64)), vf + 8 * k);
+        unpack_bf16x8(ld_shared_v4(sb + X_VT + sw128_chunk(idx >> 4, idx & 15, 64)), vf + 8 * k);
       }
 #pragma unroll
       for (int x = 0; x < 32; ++x) vmax = fmaxf(vmax, fabsf(vf[x]));
@@ -1158,12 +1174,12 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const int idx = tid + kNT * k;
-          st_chunk_f16(sb + C_VT + sw128_chunk(idx >> 4, idx & 15, 64), vf + 8 * k, sv_scale);
+          st_chunk_f16(sb + X_VT + sw128_chunk(idx >> 4, idx & 15, 64), vf + 8 * k, sv_scale);
         }
         const float to_e = ldexpf(1.f, s_exp - e);
 #pragma unroll
         for (int q = 0; q < 8; ++q)
-          st_chunk_f16(sb + C_S0T + sw128_chunk(row, half * 8 + q, 128), sv + 8 * q, to_e);
+          st_chunk_f16(sb + X_S0T + sw128_chunk(row, half * 8 + q, 128), sv + 8 * q, to_e);
         const float upd = gC * to_e;
 #pragma unroll
         for (int x = 0; x < 64; ++x) sv[x] *= upd;
@@ -1177,41 +1193,40 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
       __syncthreads();
       GDN_TRACE_POINT(2);
 
-      // U^T = V^T (T diag b)^T;  Y^T = S^T (gamma Q^)^T;  Delta^T = U^T - S^T W^T
+      // [Delta^T | Y^T] = S^T [-W; gamma Q^]^T (one N = 128 product), then
+      // Delta^T += U^T = V^T (T diag b)^T
       if (tid == 0) {
         fence_after_sync();
 #pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t da = sdesc(sb + X_S0T + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+          const uint64_t db = sdesc(ship + SH_WQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+          mma_f16(tbase + 128, da, db, ID_KK128, kk > 0);
+        }
+#pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t da = sdesc(sb + C_VT + kk * 2048, 8192, 1024);
+          const uint64_t da = sdesc(sb + X_VT + kk * 2048, 8192, 1024);
           const uint64_t db = sdesc(ship + SH_TB + kk * 32, 16, 1024);
-          mma_f16(tbase + 128, da, db, ID_MK, kk > 0);
-        }
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t da = sdesc(sb + C_S0T + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-          const uint64_t db = sdesc(ship + SH_QG + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
-          mma_f16(tbase + 192, da, db, ID_KK, kk > 0);
-        }
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t da = sdesc(sb + C_S0T + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-          const uint64_t db = sdesc(ship + SH_WT + kk * 2048, 16384, 1024);
-          mma_f16(tbase + 128, da, db, ID_KM_NEG, 1);
+          mma_f16(tbase + 128, da, db, ID_MK, 1);
         }
         mma_commit(mbar);
+        GDN_TRACE_POINT(43);
       }
+      GDN_TRACE_POINT(60);
       if constexpr (kGlobal) {
         // the next chunk's tiles, while the MMAs run
         if (tid == kFetcher && has_next) fetch(ci + 1, false);
       }
-      if (has_g) {
+      GDN_TRACE_POINT(61);
+      GDN_TRACE_POINT(70);
+      if (!kGlobal && has_g && tid >= 64) {
         // Also while the MMAs run: this chunk's gate factors (1 + w)
-        // sigmoid(g), in place as fp16.  Each thread converts the pieces it
-        // loaded itself (waited for at the loop top), so no barrier is needed.
-        const int ch = tid & 15;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint32_t addr = gsb + ((tid >> 4) + 16 * k) * 256 + ch * 16;
+        // sigmoid(g), in place as fp16 (g landed before the loop-top
+        // barrier).  Warps 2-7 only: warp 0 issues the MMAs, warp 1 fetches.
+        // Piece p = tid - 64 + 192 k has column block p % 16 = tid % 16.
+#pragma unroll 1
+        for (int pc = tid - 64; pc < 1024; pc += 192) {
+          const uint32_t addr = gsb + (pc >> 4) * 256 + (pc & 15) * 16;
           float gf[8];
           unpack_bf16x8(ld_shared_v4(addr), gf);
           uint32_t o[4];
@@ -1222,6 +1237,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
           st_shared_v4(addr, o[0], o[1], o[2], o[3]);
         }
       }
+      GDN_TRACE_POINT(71);
       okw = mbar_wait(mbar, phase, kWaitLimit);
       phase ^= 1;
       if (!__syncthreads_and(okw)) { ok = false; break; }
@@ -1238,7 +1254,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
         const float sf = ldexpf(1.f, f);
 #pragma unroll
         for (int q = 0; q < 4; ++q)
-          st_chunk_f16(sb + C_DT + sw128_chunk(row, half * 4 + q, 128), v + 8 * q, sf);
+          st_chunk_f16(sb + X_DT + sw128_chunk(row, half * 4 + q, 128), v + 8 * q, sf);
       }
       fence_proxy_async();
       fence_before_sync();
@@ -1250,13 +1266,13 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
         fence_after_sync();
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t da = sdesc(sb + C_DT + kk * 32, 16, 1024);
+          const uint64_t da = sdesc(sb + X_DT + kk * 32, 16, 1024);
           const uint64_t db = sdesc(ship + SH_KT + kk * 2048, 8192, 1024);
           mma_f16(tbase, da, db, ID_KM128, 1);
         }
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t da = sdesc(sb + C_DT + kk * 32, 16, 1024);
+          const uint64_t da = sdesc(sb + X_DT + kk * 32, 16, 1024);
           const uint64_t db = sdesc(ship + SH_P + kk * 32, 16, 1024);
           mma_f16(tbase + 192, da, db, ID_KK, 1);
         }
@@ -1301,7 +1317,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
           GDN_TRACE_POINT(51);
           // y rr (|y rr| <= sqrt(d_v)) as fp16, token-major, into the Delta^T
           // tile (its MMAs are complete; it is rewritten next chunk)
-          __half* yst = reinterpret_cast<__half*>(gb + C_DT) + half * 32 * kD + row;
+          __half* yst = reinterpret_cast<__half*>(gb + X_DT) + half * 32 * kD + row;
           const float4* rr4 = reinterpret_cast<const float4*>(sRr + half * 32);
 #pragma unroll
           for (int x4 = 0; x4 < 8; ++x4) {
@@ -1321,7 +1337,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
             const int rr = (tid >> 4) + 16 * k;
             if (rr < n) {
               float yf[8], gf[8];
-              unpack_f16x8(ld_shared_v4(sb + C_DT + rr * 256 + ch * 16), yf);
+              unpack_f16x8(ld_shared_v4(sb + X_DT + rr * 256 + ch * 16), yf);
               unpack_f16x8(ld_shared_v4(gsb + rr * 256 + ch * 16), gf);
               uint32_t o[4];
 #pragma unroll
@@ -1332,8 +1348,8 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
             }
           }
         } else {
-          // no gate: y as bf16 through the staging buffer, coalesced stores
-          __nv_bfloat16* gs = reinterpret_cast<__nv_bfloat16*>(gb + C_GS);
+          // no gate: y as bf16 through the Delta^T tile, coalesced stores
+          __nv_bfloat16* gs = reinterpret_cast<__nv_bfloat16*>(gb + X_DT);
 #pragma unroll
           for (int x = 0; x < 32; ++x) gs[(half * 32 + x) * kD + row] = __float2bfloat16_rn(v[x]);
           __syncthreads();
@@ -1342,7 +1358,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
             const int idx = tid + kNT * k;
             const int rr = idx >> 4, ch = idx & 15;
             if (rr < n) {
-              const uint4 val = ld_shared_v4(sb + C_GS + rr * 256 + ch * 16);
+              const uint4 val = ld_shared_v4(sb + X_DT + rr * 256 + ch * 16);
               *reinterpret_cast<uint4*>(Yg + ((size_t)(c0 + rr) * a.H_v + h) * kD + ch * 8) = val;
             }
           }
@@ -1425,7 +1441,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
     if constexpr (!kGlobal) cluster_sync();
     fence_after_sync();
     const uint32_t tbase = *tslot;
-    const uint32_t tKQ = tbase + lane_off, tW = tbase + lane_off + 64;
+    const uint32_t tKQ = tbase + lane_off, tW = tbase + lane_off;
     uint32_t full_cl0 = 0, ship_cl0 = 0, scal_cl0 = 0;
     if constexpr (!kGlobal) {
       full_cl0 = mapa_shared(sb + C_BAR, 0);
@@ -1433,6 +1449,16 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
       scal_cl0 = mapa_shared(sb + C_SCAL, 0);
     }
 
+    // Split launch: this CTA also computes the chunk's gate factors
+    // (1 + w) sigmoid(g) and stores them into the slot; thread (r, c) of
+    // piece index tid + 256 k handles token row (tid / 16) + 16 k, columns
+    // 8 (tid % 16) .. + 7.
+    float wv[8];
+#pragma unroll
+    for (int j2 = 0; j2 < 8; ++j2)
+      wv[j2] = 1.f + ((has_g && a.norm_w) ? __ldg(a.norm_w + (tid & 15) * 8 + j2) : 0.f);
+    const __nv_bfloat16* Gh = static_cast<const __nv_bfloat16*>(a.g);
+    uint4 gfac[4];  // this thread's gate factors (fp16 x 8 per piece)
     // Split launch, thread 0: the slot whose bulk stores are in flight and
     // not yet published (published once complete, during the next chunk).
     int pend_slot = -1;
@@ -1456,6 +1482,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
       const int lb = lc & 1;      // local staging / prefetch buffer
       const uint32_t stg = sb + P_STG + lb * kShipBytes;
       cp_async_wait_all();
+      fence_proxy_async();  // the raw [K; Q] tile is read by MMA0 below
       bool okw = true;
       if constexpr (!kGlobal) {
         // staging buffer lb was the source of the copy two local chunks ago;
@@ -1467,8 +1494,30 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
       if (!__syncthreads_and(okw)) { ok = false; break; }
       GDN_TRACE_POINT(20);
 
-      // gates
-      if (warp == 0) {
+      if constexpr (kGlobal) {
+        // g of this chunk into L2 now; it is read after the W product
+        if (has_g) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int rr = (tid >> 4) + 16 * k;
+            if (rr < n) prefetch_l2(Gh + ((size_t)(c0 + rr) * a.H_v + h) * kD + (tid & 15) * 8);
+          }
+        }
+      }
+
+      // [K; Q] K^T on the raw inputs, overlapped with the gates and norms
+      if (tid == 0) {
+        fence_after_sync();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t d = sdesc(sb + P_KQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+          mma_f16(tbase, d, d, ID_BF_KK, kk > 0);
+        }
+        mma_commit(mbar);
+      }
+
+      // gates (warp 1: thread 0 of warp 0 has just issued the MMAs)
+      if (warp == 1) {
         const float* gl = sGateBuf + lb * 128;
         float carry = 0.f;
         float Gv[2], bv[2];
@@ -1528,25 +1577,12 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           st_chunk_f16(sb + P_KH + sw128_chunk(r, qc + c, 64), kf + 8 * c, rk);
-          st_chunk_f16(stg + SH_QG + sw128_chunk(r, qc + c, 64), qf + 8 * c, gq);
+          st_chunk_f16(stg + SH_WQ + sw128_chunk(64 + r, qc + c, 128), qf + 8 * c, gq);
           st_chunk_f16(stg + SH_KT + sw128_chunk(r, qc + c, 64), kf + 8 * c, dk);
         }
       }
       fence_proxy_async();
       fence_before_sync();
-      __syncthreads();
-
-      // [K; Q] K^T on the raw inputs
-      if (tid == 0) {
-        fence_after_sync();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t d = sdesc(sb + P_KQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-          mma_f16(tbase, d, d, ID_BF_KK, kk > 0);
-        }
-        mma_commit(mbar);
-        if constexpr (kGlobal) publish();
-      }
       okw = mbar_wait(mbar, phase, kWaitLimit);
       phase ^= 1;
       if (!__syncthreads_and(okw)) { ok = false; break; }
@@ -1636,34 +1672,69 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
       __syncthreads();
       GDN_TRACE_POINT(25);
 
-      // W^T = K^T (T diag(b g))^T
+      // W = (T diag(b g)) K^ (M = 64 tokens, N = 128 = d_k; hi + lo parts
+      // of T diag(b g)), into TMEM columns 0-127 ([K; Q] K^T is consumed)
       if (tid == 0) {
         fence_after_sync();
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t da = sdesc(sb + P_KH + kk * 2048, 8192, 1024);
-          const uint64_t db = sdesc(sb + P_TBG + kk * 32, 16, 1024);
-          mma_f16(tbase + 64, da, db, ID_MK, kk > 0);
+          const uint64_t da = sdesc(sb + P_TBG + kk * 32, 16, 1024);
+          const uint64_t db = sdesc(sb + P_KH + kk * 2048, 8192, 1024);
+          mma_f16(tbase, da, db, ID_W64, kk > 0);
         }
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t da = sdesc(sb + P_KH + kk * 2048, 8192, 1024);
-          const uint64_t db = sdesc(sb + P_TBG_LO + kk * 32, 16, 1024);
-          mma_f16(tbase + 64, da, db, ID_MK, 1);
+          const uint64_t da = sdesc(sb + P_TBG_LO + kk * 32, 16, 1024);
+          const uint64_t db = sdesc(sb + P_KH + kk * 2048, 8192, 1024);
+          mma_f16(tbase, da, db, ID_W64, 1);
         }
         mma_commit(mbar);
+        // the previous chunk's slot (its stores are long complete), while
+        // the MMAs run; a first chunk is published as soon as it is stored
+        if constexpr (kGlobal) publish();
+      }
+      if constexpr (kGlobal) {
+        // this chunk's gate factors from g (in L2) while the MMAs run; they
+        // are stored once the slot is free
+        if (has_g) {
+          uint4 graw[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int rr = (tid >> 4) + 16 * k;
+            graw[k] = rr < n ? ld_nc_v4(Gh + ((size_t)(c0 + rr) * a.H_v + h) * kD + (tid & 15) * 8)
+                             : make_uint4(0u, 0u, 0u, 0u);
+          }
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            float gf[8];
+            unpack_bf16x8(graw[k], gf);
+            uint32_t o[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              o[q] = pack_f16(__fdividef(wv[2 * q], 1.f + __expf(-gf[2 * q])),
+                              __fdividef(wv[2 * q + 1], 1.f + __expf(-gf[2 * q + 1])));
+            gfac[k] = make_uint4(o[0], o[1], o[2], o[3]);
+          }
+        }
       }
       okw = mbar_wait(mbar, phase, kWaitLimit);
       phase ^= 1;
       if (!__syncthreads_and(okw)) { ok = false; break; }
       fence_after_sync();
       {
-        float v[32];
-        tmem_ld32(tW + half * 32, v);
+        // M = 64 accumulator: row t sits in TMEM lane (t % 16) + 32 (t / 16),
+        // i.e. lanes 0-15 of warp quarter t / 16; warps w and w + 4 take the
+        // two halves of d_k.  -W goes to rows 0-63 of the merged tile.
+        float v[64];
+        tmem_ld32(tW + half * 64, v);
+        tmem_ld32(tW + half * 64 + 32, v + 32);
         tmem_wait_ld();
+        if (lane < 16) {
+          const int t = 16 * (warp & 3) + lane;
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          st_chunk_f16(stg + SH_WT + sw128_chunk(row, half * 4 + q, 128), v + 8 * q, 1.f);
+          for (int q = 0; q < 8; ++q)
+            st_chunk_f16(stg + SH_WQ + sw128_chunk(t, half * 8 + q, 128), v + 8 * q, -1.f);
+        }
       }
       fence_proxy_async();
       fence_before_sync();
@@ -1673,25 +1744,37 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
       // ship this chunk's tiles once the chain CTA has released buffer b
       okw = true;
       if constexpr (kGlobal) {
+        // slot ci % kRing last held chunk ci - kRing: the chain CTA must
+        // have loaded it
+        const int s = ci % kRing;
+        uint8_t* dst = ring + (size_t)s * kSlotBytes;
+        if (tid == 0 && ci >= kRing)
+          okw = wait_flag_ge(&consumed[s], (unsigned long long)(ci - kRing) + 1, kWaitLimit);
+        if (!__syncthreads_and(okw)) { ok = false; break; }
+        GDN_TRACE_POINT(30);
         if (tid == 0) {
-          // slot ci % kRing last held chunk ci - kRing: the chain CTA must
-          // have loaded it
-          const int s = ci % kRing;
-          if (ci >= kRing)
-            okw = wait_flag_ge(&consumed[s], (unsigned long long)(ci - kRing) + 1, kWaitLimit);
-          GDN_TRACE_POINT(30);
-          if (okw) {
-            uint8_t* dst = ring + (size_t)s * kSlotBytes;
-            fence_proxy_async_global();
+          fence_proxy_async_global();
 #pragma unroll
-            for (int k = 0; k < 4; ++k) bulk_store_s2g(dst + 16384 * k, stg + 16384 * k, 16384);
-            bulk_store_s2g(dst + kShipBytes, sb + P_SCAL + 16 * lb, 16);
-            bulk_commit();
-            pend_slot = s;
-            pend_val = (unsigned long long)ci + 1;
-            GDN_TRACE_POINT(31);
+          for (int k = 0; k < 4; ++k) bulk_store_s2g(dst + 16384 * k, stg + 16384 * k, 16384);
+          bulk_store_s2g(dst + kSlotLoad, sb + P_SCAL + 16 * lb, 16);
+          bulk_commit();
+          pend_slot = s;
+          pend_val = (unsigned long long)ci + 1;
+        }
+        if (has_g) {
+          // gate factors, token-major [64][128] fp16, beside the tiles.  The
+          // barrier below orders these stores before thread 0's release of
+          // the slot (release is cumulative over what the barrier ordered).
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int rr = (tid >> 4) + 16 * k;
+            if (rr < n)
+              *reinterpret_cast<uint4*>(dst + kSlotGF + rr * 256 + (tid & 15) * 16) = gfac[k];
           }
         }
+        __syncthreads();
+        if (tid == 0 && lc == 0) publish();
+        GDN_TRACE_POINT(31);
       } else if (tid == 0) {
         okw = mbar_wait_cluster(&empty[b], ((ci >> 1) & 1) ^ 1, kWaitLimit);
         if (okw) {

@@ -334,6 +334,21 @@ __device__ __forceinline__ void bulk_store_s2g(void* dst, uint32_t src_smem, uin
                : "memory");
 }
 
+// 16-byte read-only global load, issued where it stands (volatile: not
+// sunk towards its first use by the compiler).
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// Prefetch the 128-byte line holding `p` into L2.
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // ---- cp.async (Ampere-style asynchronous global -> shared copies) -------------
 // 16 bytes; when `pred` is false nothing is read and the destination is zero
 // filled (src must still be a valid address).

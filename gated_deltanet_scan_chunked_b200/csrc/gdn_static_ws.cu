@@ -13,10 +13,10 @@ namespace gdn {
 namespace {
 
 // Capacity: 48 (sequence, value head) items -- one sequence of a 48-value-head
-// layer.  Per item the split layout needs 64 bytes of flags and four 64.25 KB
-// hand-off slots, 263,232 bytes; 48 items need 12,635,136 bytes.
+// layer.  Per item the split layout needs 64 bytes of flags and four 80.25 KB
+// hand-off slots, 328,768 bytes; 48 items need 15,780,864 bytes.
 constexpr int kStaticItems = 48;
-constexpr size_t kStaticBytes = (size_t)kStaticItems * 64 + (size_t)kStaticItems * 4 * 65792;
+constexpr size_t kStaticBytes = (size_t)kStaticItems * 64 + (size_t)kStaticItems * 4 * 82176;
 
 static __device__ __align__(256) unsigned char g_static_ws[kStaticBytes];
 

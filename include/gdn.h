@@ -126,7 +126,7 @@ gdn_status gdn_chunk_fwd_path(
 /*
  * gdn_chunk_fwd_workspace_size -- bytes of device workspace that
  * gdn_chunk_fwd_ws can use for a batch of n_seq sequences x H_v value heads
- * (the split layout: a ring of four 64.25 KB hand-off slots plus 64 bytes of
+ * (the split layout: a ring of four 80.25 KB hand-off slots plus 64 bytes of
  * flags per item).  Returns 0 when that layout cannot apply to the shape:
  * not bf16 with d_k = d_v = 128, or more than 64 items.  Host only; no CUDA
  * call.
@@ -164,7 +164,7 @@ gdn_status gdn_chunk_fwd_ws(
 
 /*
  * gdn_chunk_fwd_static_ws -- gdn_chunk_fwd_ws with GDN_PATH_TENSOR_SPLIT and
- * a workspace that is a fixed array inside the library (12,635,136 bytes of
+ * a workspace that is a fixed array inside the library (15,780,864 bytes of
  * device memory per device, part of the module image) instead of caller
  * memory: for callers that cannot give the library any memory.  The method's
  * description has no counterpart to this call; it is a deployment variant of

@@ -99,8 +99,8 @@ def _chunk_ws(lib, ws=None, ws_bytes=0, path=0, **kw):
 
 def test_workspace_size(lib):
     """Split layout: 64 bytes of flags per item (padded to 256), then four
-    64 KB + 256 B slots per item; nothing for shapes it cannot serve."""
-    one = 4 * (65536 + 256)
+    80 KB + 256 B slots per item; nothing for shapes it cannot serve."""
+    one = 4 * (81920 + 256)
     assert gdn.workspace_size(1, 48, 128, 128) == 48 * 64 + 48 * one
     assert gdn.workspace_size(1, 1, 128, 128) == 256 + one
     assert gdn.workspace_size(2, 32, 128, 128) == 64 * 64 + 64 * one
