@@ -959,12 +959,13 @@ constexpr size_t kSlotBytes = kSlotLoad + 256;
 template <int NPREP, bool kGlobal>
 __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const PrefillArgs a) {
   // chain CTA map: 2 ship buffers (the split launch also ships the gate
-  // factors: 80 KB each), V, S^T, Delta^T, and (cluster launch only) two g
-  // buffers; then C_SCAL / C_RED / C_BAR at fixed offsets.
+  // factors: 80 KB each), V, the output staging tile, and (cluster launch
+  // only) two g buffers; then C_SCAL / C_RED / C_BAR at fixed offsets.
+  // TMEM (512 columns): S^T fp32 0-127, Delta^T 128-191, Y^T 192-255, and the
+  // fp16 MMA A operands S^T 2^-e (256-319) and Delta^T 2^-e (320-351).
   constexpr uint32_t kShipStride = kGlobal ? kSlotLoad : kShipBytes;
   constexpr uint32_t X_VT = C_SHIP + 2 * kShipStride;
-  constexpr uint32_t X_S0T = X_VT + 16384;
-  constexpr uint32_t X_DT = X_S0T + 32768;
+  constexpr uint32_t X_DT = X_VT + 16384;  // output staging (16 KB)
   constexpr uint32_t X_GS = X_DT + 16384;
   static_assert((kGlobal ? X_GS : X_GS + 32768) <= C_SCAL, "chain shared-memory map overlaps");
   extern __shared__ uint8_t smem_raw[];
@@ -1043,7 +1044,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
       if (!kGlobal && has_g) ld.g(t_begin, n0, 0);
     }
     cp_async_commit();
-    if (warp == 0) tmem_alloc(tslot, 256);
+    if (warp == 0) tmem_alloc(tslot, 512);
     if (tid == 0) {
       mbar_init(&full[0], 1);
       mbar_init(&full[1], 1);
@@ -1056,6 +1057,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
     fence_after_sync();
     const uint32_t tbase = *tslot;
     const uint32_t tS = tbase + lane_off, tD = tbase + lane_off + 128, tY = tbase + lane_off + 192;
+    const uint32_t tSA = tbase + lane_off + 256, tDA = tbase + lane_off + 320;
     // Split launch, thread kFetcher only (not the MMA issuer: its proxy
     // fence would wait for the MMAs in flight): issue the bulk load of chunk
     // c from its slot into buffer c & 1 (free: it held chunk c - 2, whose
@@ -1177,9 +1179,13 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
           st_chunk_f16(sb + X_VT + sw128_chunk(idx >> 4, idx & 15, 64), vf + 8 * k, sv_scale);
         }
         const float to_e = ldexpf(1.f, s_exp - e);
+        {
+          // S^T 2^-e as the fp16 A operand, in TMEM (d_k pairs per column)
+          uint32_t pk[32];
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-          st_chunk_f16(sb + X_S0T + sw128_chunk(row, half * 8 + q, 128), sv + 8 * q, to_e);
+          for (int x = 0; x < 32; ++x) pk[x] = pack_f16(sv[2 * x] * to_e, sv[2 * x + 1] * to_e);
+          tmem_st32(tSA + half * 32, reinterpret_cast<const float*>(pk));
+        }
         const float upd = gC * to_e;
 #pragma unroll
         for (int x = 0; x < 64; ++x) sv[x] *= upd;
@@ -1199,9 +1205,8 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
         fence_after_sync();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t da = sdesc(sb + X_S0T + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
           const uint64_t db = sdesc(ship + SH_WQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-          mma_f16(tbase + 128, da, db, ID_KK128, kk > 0);
+          mma_f16_ta(tbase + 128, tbase + 256 + kk * 8, db, ID_KK128, kk > 0);
         }
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
@@ -1246,17 +1251,18 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
       cp_async_commit();
       GDN_TRACE_POINT(3);
 
-      // Delta^T 2^-e -> fp16 tile
+      // Delta^T 2^-e -> fp16 A operand in TMEM (token pairs per column)
       {
         float v[32];
         tmem_ld32(tD + half * 32, v);
         tmem_wait_ld();
         const float sf = ldexpf(1.f, f);
+        uint32_t pk[16];
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          st_chunk_f16(sb + X_DT + sw128_chunk(row, half * 4 + q, 128), v + 8 * q, sf);
+        for (int x = 0; x < 16; ++x) pk[x] = pack_f16(v[2 * x] * sf, v[2 * x + 1] * sf);
+        tmem_st16(tDA + half * 16, pk);
+        tmem_wait_st();
       }
-      fence_proxy_async();
       fence_before_sync();
       __syncthreads();
       GDN_TRACE_POINT(4);
@@ -1266,15 +1272,13 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
         fence_after_sync();
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t da = sdesc(sb + X_DT + kk * 32, 16, 1024);
           const uint64_t db = sdesc(ship + SH_KT + kk * 2048, 8192, 1024);
-          mma_f16(tbase, da, db, ID_KM128, 1);
+          mma_f16_ta(tbase, tbase + 320 + kk * 8, db, ID_KM128, 1);
         }
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t da = sdesc(sb + X_DT + kk * 32, 16, 1024);
           const uint64_t db = sdesc(ship + SH_P + kk * 32, 16, 1024);
-          mma_f16(tbase + 192, da, db, ID_KK, 1);
+          mma_f16_ta(tbase + 192, tbase + 320 + kk * 8, db, ID_KK, 1);
         }
         mma_commit(mbar);
       }
@@ -1315,8 +1319,8 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
                                   (float)kD + a.eps_norm);
           __syncthreads();
           GDN_TRACE_POINT(51);
-          // y rr (|y rr| <= sqrt(d_v)) as fp16, token-major, into the Delta^T
-          // tile (its MMAs are complete; it is rewritten next chunk)
+          // y rr (|y rr| <= sqrt(d_v)) as fp16, token-major, into the staging
+          // tile
           __half* yst = reinterpret_cast<__half*>(gb + X_DT) + half * 32 * kD + row;
           const float4* rr4 = reinterpret_cast<const float4*>(sRr + half * 32);
 #pragma unroll
@@ -1348,7 +1352,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
             }
           }
         } else {
-          // no gate: y as bf16 through the Delta^T tile, coalesced stores
+          // no gate: y as bf16 through the staging tile, coalesced stores
           __nv_bfloat16* gs = reinterpret_cast<__nv_bfloat16*>(gb + X_DT);
 #pragma unroll
           for (int x = 0; x < 32; ++x) gs[(half * 32 + x) * kD + row] = __float2bfloat16_rn(v[x]);
@@ -1363,7 +1367,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
             }
           }
         }
-        __syncthreads();  // staging reads done: g buffer and Delta^T tile reusable
+        __syncthreads();  // staging reads done: g buffer and staging tile reusable
         GDN_TRACE_POINT(53);
       }
       fence_before_sync();
@@ -1399,7 +1403,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
     fence_before_sync();
     __syncthreads();
     if constexpr (!kGlobal) cluster_sync();
-    if (warp == 0) tmem_dealloc(tbase, 256);
+    if (warp == 0) tmem_dealloc(tbase, 512);
   } else {
     // =========================== prep CTA ============================
     uint64_t* empty = reinterpret_cast<uint64_t*>(gb + P_BAR);
