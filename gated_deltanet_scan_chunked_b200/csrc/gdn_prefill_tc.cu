@@ -59,24 +59,20 @@ constexpr int kC = 64;    // chunk length
 constexpr int kD = 128;   // head dim (d_k = d_v)
 constexpr int kNT = 256;  // threads per CTA
 
-// shared memory map (bytes from a 1024-aligned base)
+// shared memory map of the one-CTA kernel (bytes from a 1024-aligned base)
 constexpr uint32_t OFF_KQ = 0;          // [K; Q] raw bf16 128 x 128 (cp.async target), 2 x 16 KB
 constexpr uint32_t OFF_KH = 32768;      // K^ fp16          64 x 128, 2 panels x 8 KB
-constexpr uint32_t OFF_QG = 49152;      // gamma Q^ fp16    64 x 128
-constexpr uint32_t OFF_KT = 65536;      // dec K^ fp16      64 x 128
-constexpr uint32_t OFF_VT = 81920;      // V: raw bf16 (cp.async), then V 2^-e fp16 in place
-constexpr uint32_t OFF_TB = 98304;      // T b 2^-f fp16    64 x 64
-constexpr uint32_t OFF_TBG = 106496;    // T b g 2^-f fp16  64 x 64
-constexpr uint32_t OFF_P = 114688;      // P fp16           64 x 64
-constexpr uint32_t OFF_S0T = 122880;    // S^T 2^-e fp16   128 x 128, 2 panels x 16 KB
-constexpr uint32_t OFF_WT = 155648;     // W^T fp16        128 x 64
-constexpr uint32_t OFF_DT = 172032;     // Delta^T fp16    128 x 64
-// A and T (fp32 64 x 64) live in the W^T and Delta^T tiles: both are dead
-// between the previous chunk's MMAs and this chunk's W / Delta conversions.
-constexpr uint32_t OFF_A = OFF_WT;
-constexpr uint32_t OFF_T = OFF_DT;
+constexpr uint32_t OFF_KT = 49152;      // dec K^ fp16      64 x 128
+constexpr uint32_t OFF_VT = 65536;      // V: raw bf16 (cp.async), then V 2^-e fp16 in place
+constexpr uint32_t OFF_TB = 81920;      // T b 2^-f fp16    64 x 64
+constexpr uint32_t OFF_TBG = 90112;     // T b g 2^-f fp16  64 x 64 (rounded part)
+constexpr uint32_t OFF_P = 98304;       // P fp16           64 x 64
+constexpr uint32_t OFF_WQ = 106496;     // [-W; gamma Q^] fp16 128 x 128 K-major, 2 panels x 16 KB
+constexpr uint32_t OFF_A = 139264;      // A fp32 64 x 64
+constexpr uint32_t OFF_T = 155648;      // T fp32 64 x 64
 constexpr uint32_t OFF_TBG_LO = OFF_A;  // rounding remainder of T diag(b g), after A is dead
-constexpr uint32_t OFF_GS = 188416;     // g in / y out staging, 2 buffers x [64][128] bf16
+constexpr uint32_t OFF_STG = 172032;    // output staging [64][128] 16-bit
+constexpr uint32_t OFF_GS = 188416;     // g (-> gate factors in place), 2 buffers x [64][128]
 constexpr uint32_t OFF_Z = 221184;      // Z fp32 [1024]
 constexpr uint32_t OFF_GATEBUF = 225280;  // [2 buffers][log alpha, beta][64] fp32
 constexpr uint32_t OFF_GATE = 226304;   // G2, beta, gamma, dec, rk, rq: 6 x 64 fp32
@@ -84,8 +80,11 @@ constexpr uint32_t OFF_RED = 227840;    // red[4][64], rr[64], max[16]
 constexpr uint32_t OFF_BAR = 229248;
 constexpr uint32_t kSmemBytes = OFF_BAR + 64 + 1024;  // + alignment slack
 
-// TMEM columns (fp32, 128 lanes)
-constexpr uint32_t TM_S = 0, TM_KQ = 128, TM_W = 192, TM_D = 256, TM_Y = 320;
+// TMEM columns (fp32, 128 lanes): S^T, [K;Q]K^T (then W, M = 64 x N = 128),
+// Delta^T | Y^T (adjacent: one N = 128 product writes both), and the fp16
+// MMA A operands S^T 2^-e and Delta^T 2^-e
+constexpr uint32_t TM_S = 0, TM_KQ = 128, TM_W = 128, TM_D = 256, TM_Y = 320, TM_SA = 384,
+                   TM_DA = 448;
 constexpr uint32_t kTmemCols = 512;
 
 constexpr uint32_t kWaitLimit = 1u << 24;
@@ -94,7 +93,6 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t ID_BF_KK = idesc_f16(128, 64, false, false, false, false);  // MMA0
 constexpr uint32_t ID_KK = idesc_f16(128, 64, false, false, false, true);
 constexpr uint32_t ID_MK = idesc_f16(128, 64, true, false, false, true);
-constexpr uint32_t ID_KM_NEG = idesc_f16(128, 64, false, true, true, true);
 constexpr uint32_t ID_KM128 = idesc_f16(128, 128, false, true, false, true);
 constexpr uint32_t ID_KK128 = idesc_f16(128, 128, false, false, false, true);
 constexpr uint32_t ID_W64 = idesc_f16(64, 128, false, true, false, true);
@@ -460,6 +458,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
   const uint32_t tS = tbase + lane_off + TM_S, tKQ = tbase + lane_off + TM_KQ;
   const uint32_t tW = tbase + lane_off + TM_W, tD = tbase + lane_off + TM_D;
   const uint32_t tY = tbase + lane_off + TM_Y;
+  const uint32_t tSA = tbase + lane_off + TM_SA, tDA = tbase + lane_off + TM_DA;
 
   // initial state -> TMEM S^T (lane j = column j of S, columns d), exponent 0
   {
@@ -477,10 +476,15 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
   }
   int s_exp = 0;  // S_true = S_tmem * 2^s_exp
 
+  // 1 + w for the 8 output columns this thread gates and stores (the same
+  // in every chunk: piece index p has column block p % 16 = tid % 16)
+  float wv[8];
+#pragma unroll
+  for (int j2 = 0; j2 < 8; ++j2)
+    wv[j2] = 1.f + ((has_g && a.norm_w) ? __ldg(a.norm_w + (tid & 15) * 8 + j2) : 0.f);
+
   uint32_t phase = 0;
   bool ok = true;
-  float wj = 0.f;
-  if (has_g && a.norm_w) wj = __ldg(a.norm_w + row);
 
   int ci = 0;
   for (int64_t c0 = t_begin; c0 < t_end; c0 += kC, ++ci) {
@@ -488,13 +492,27 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
     const bool has_next = c0 + kC < t_end;
     const int nn = has_next ? ((t_end - c0 - kC) < kC ? (int)(t_end - c0 - kC) : kC) : 0;
     const int buf = ci & 1;
+    const uint32_t gsb = sb + OFF_GS + buf * 16384;  // this chunk's g -> gate factors
 
     cp_async_wait_all();
+    fence_proxy_async();  // the raw [K; Q] tile is read by MMA0 below
     __syncthreads();
     GDN_TRACE_POINT(0);
 
+    // ---- MMA0: [K;Q] K^T on the raw bf16 inputs (exact), while the gates,
+    // norms and conversions run --------------------------------------------------
+    if (tid == 0) {
+      fence_after_sync();
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint64_t d = sdesc(sb + OFF_KQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+        mma_f16(tbase + TM_KQ, d, d, ID_BF_KK, kk > 0);
+      }
+      mma_commit(bar);
+    }
+
     // ---- gates: cumsum of log alpha (log2 units), beta, gamma, exp(G_C - G) ----
-    if (warp == 0) {
+    if (warp == 1) {
       const float* gl = sGateBuf + buf * 128;
       float carry = 0.f;
       float Gv[2], bv[2];
@@ -529,7 +547,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
     __syncthreads();
     GDN_TRACE_POINT(1);
 
-    // ---- L2 norms; K^, gamma Q^, dec K^ -> fp16 tiles ---------------------------
+    // ---- L2 norms; K^, dec K^ and gamma Q^ (rows 64-127 of [-W; gamma Q^]) -----
     // warp w owns rows 8w .. 8w+7; 4 lanes per row, 32 columns (4 chunks) each
     {
       const int r = warp * 8 + (lane >> 2);
@@ -558,7 +576,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         st_chunk_f16(sb + OFF_KH + sw128_chunk(r, qc + c, 64), kf + 8 * c, rk);
-        st_chunk_f16(sb + OFF_QG + sw128_chunk(r, qc + c, 64), qf + 8 * c, gq);
+        st_chunk_f16(sb + OFF_WQ + sw128_chunk(64 + r, qc + c, 128), qf + 8 * c, gq);
         st_chunk_f16(sb + OFF_KT + sw128_chunk(r, qc + c, 64), kf + 8 * c, dk);
       }
     }
@@ -580,8 +598,9 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
     float smax = 0.f;
 #pragma unroll
     for (int x = 0; x < 64; ++x) smax = fmaxf(smax, fabsf(sv[x]));
-    const float mV = block_max(vmax, sMax, warp, lane);
-    const float mS = ldexpf(block_max(smax, sMax, warp, lane), s_exp);
+    const float2 mx = block_max2(vmax, smax, sMax, warp, lane);
+    const float mV = mx.x;
+    const float mS = ldexpf(mx.y, s_exp);
     // |Delta| <= |v| + |S| ||k^||_1 <= max|V| + 12 max|S|; keep that <= 2^12
     const int e = scale_exp(mV + 12.f * mS, 12);
     {
@@ -592,9 +611,13 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
         st_chunk_f16(sb + OFF_VT + sw128_chunk(idx >> 4, idx & 15, 64), vf + 8 * k, sv_scale);
       }
       const float to_e = ldexpf(1.f, s_exp - e);
+      {
+        // S^T 2^-e as the fp16 A operand, in TMEM (d_k pairs per column)
+        uint32_t pk[32];
 #pragma unroll
-      for (int q = 0; q < 8; ++q)
-        st_chunk_f16(sb + OFF_S0T + sw128_chunk(row, half * 8 + q, 128), sv + 8 * q, to_e);
+        for (int x = 0; x < 32; ++x) pk[x] = pack_f16(sv[2 * x] * to_e, sv[2 * x + 1] * to_e);
+        tmem_st32(tSA + half * 32, reinterpret_cast<const float*>(pk));
+      }
       const float upd = sGam[63] * to_e;
 #pragma unroll
       for (int x = 0; x < 64; ++x) sv[x] *= upd;
@@ -605,33 +628,14 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
     }
     fence_proxy_async();
     fence_before_sync();
-    __syncthreads();
-    GDN_TRACE_POINT(2);
-
-    // ---- MMA0: [K;Q] K^T (bf16, exact);  MMA2: S^T (gamma Q^)^T (fp16) -----------
-    if (tid == 0) {
-      fence_after_sync();
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint64_t d = sdesc(sb + OFF_KQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-        mma_f16(tbase + TM_KQ, d, d, ID_BF_KK, kk > 0);
-      }
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint64_t da = sdesc(sb + OFF_S0T + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-        const uint64_t db = sdesc(sb + OFF_QG + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
-        mma_f16(tbase + TM_Y, da, db, ID_KK, kk > 0);
-      }
-      mma_commit(bar);
-    }
-    ok = mbar_wait(bar, phase, kWaitLimit);
+    ok = mbar_wait(bar, phase, kWaitLimit);  // MMA0
     phase ^= 1;
     if (!__syncthreads_and(ok)) { ok = false; break; }
     fence_after_sync();
-    // the raw [K; Q] tile is free: next chunk's q, k
+    // the raw [K; Q] tile is free (MMA0 done, norms read it): next chunk's q, k
     if (has_next) ld.qk(c0 + kC, nn);
     cp_async_commit();
-    GDN_TRACE_POINT(3);
+    GDN_TRACE_POINT(2);
 
     // ---- A (fp32) and P (fp16) from the raw products: all 256 threads -----------
     {
@@ -645,7 +649,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
     for (int k = 0; k < 4; ++k) reinterpret_cast<float4*>(sT)[tid + kNT * k] = make_float4(0.f, 0.f, 0.f, 0.f);
     fence_before_sync();
     __syncthreads();
-    GDN_TRACE_POINT(4);
+    GDN_TRACE_POINT(3);
 
     // ---- T = (I + A)^{-1} by recursive doubling ---------------------------------
     // 8 x 8 diagonal blocks by substitution, then for block sizes b = 8, 16, 32:
@@ -675,7 +679,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
     tinv_level<8>(sA, sT, sZ, tid);
     tinv_level<16>(sA, sT, sZ, tid);
     tinv_level<32>(sA, sT, sZ, tid);
-    GDN_TRACE_POINT(5);
+    GDN_TRACE_POINT(4);
 
     // ---- scale exponent of T; T diag(b) 2^-f, T diag(b g) 2^-f -> fp16 ---------
     {
@@ -717,28 +721,82 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
     fence_before_sync();
     __syncthreads();
     const int f = (int)sMax[8];
-    GDN_TRACE_POINT(6);
+    GDN_TRACE_POINT(5);
 
-    // ---- MMAW: W^T = K^T (T diag(b g))^T;  MMAU: U^T = V^T (T diag(b))^T -------
+    // ---- W = (T diag(b g)) K^ (M = 64 tokens, N = 128; hi + lo parts), into
+    // TMEM columns TM_W .. +127 ([K; Q] K^T is consumed) ---------------------------
     if (tid == 0) {
       fence_after_sync();
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t da = sdesc(sb + OFF_KH + kk * 2048, 8192, 1024);
-        const uint64_t db = sdesc(sb + OFF_TBG + kk * 32, 16, 1024);
-        mma_f16(tbase + TM_W, da, db, ID_MK, kk > 0);
+        const uint64_t da = sdesc(sb + OFF_TBG + kk * 32, 16, 1024);
+        const uint64_t db = sdesc(sb + OFF_KH + kk * 2048, 8192, 1024);
+        mma_f16(tbase + TM_W, da, db, ID_W64, kk > 0);
       }
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t da = sdesc(sb + OFF_KH + kk * 2048, 8192, 1024);
-        const uint64_t db = sdesc(sb + OFF_TBG_LO + kk * 32, 16, 1024);
-        mma_f16(tbase + TM_W, da, db, ID_MK, 1);
+        const uint64_t da = sdesc(sb + OFF_TBG_LO + kk * 32, 16, 1024);
+        const uint64_t db = sdesc(sb + OFF_KH + kk * 2048, 8192, 1024);
+        mma_f16(tbase + TM_W, da, db, ID_W64, 1);
+      }
+      mma_commit(bar);
+    }
+    if (has_g && tid >= 32) {
+      // meanwhile, warps 1-7: this chunk's gate factors (1 + w) sigmoid(g),
+      // in place as fp16 (g landed before the loop-top barrier).  Piece
+      // p = tid - 32 + 224 k has column block p % 16 = tid % 16.
+#pragma unroll 1
+      for (int pc = tid - 32; pc < 1024; pc += 224) {
+        const uint32_t addr = gsb + (pc >> 4) * 256 + (pc & 15) * 16;
+        float gf[8];
+        unpack_bf16x8(ld_shared_v4(addr), gf);
+        uint32_t o[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          o[q] = pack_f16(__fdividef(wv[2 * q], 1.f + __expf(-gf[2 * q])),
+                          __fdividef(wv[2 * q + 1], 1.f + __expf(-gf[2 * q + 1])));
+        st_shared_v4(addr, o[0], o[1], o[2], o[3]);
+      }
+    }
+    ok = mbar_wait(bar, phase, kWaitLimit);
+    phase ^= 1;
+    if (!__syncthreads_and(ok)) { ok = false; break; }
+    fence_after_sync();
+    GDN_TRACE_POINT(6);
+
+    // ---- -W -> rows 0-63 of [-W; gamma Q^] (M = 64 accumulator: row t sits in
+    // TMEM lane (t % 16) + 32 (t / 16); warps w and w + 4 take the d_k halves) ---
+    {
+      float v[64];
+      tmem_ld32(tW + half * 64, v);
+      tmem_ld32(tW + half * 64 + 32, v + 32);
+      tmem_wait_ld();
+      if (lane < 16) {
+        const int t = 16 * (warp & 3) + lane;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          st_chunk_f16(sb + OFF_WQ + sw128_chunk(t, half * 8 + q, 128), v + 8 * q, -1.f);
+      }
+    }
+    fence_proxy_async();
+    fence_before_sync();
+    __syncthreads();
+    GDN_TRACE_POINT(7);
+
+    // ---- [Delta^T | Y^T] = S^T [-W; gamma Q^]^T (one N = 128 product per K step),
+    // then Delta^T += U^T = V^T (T diag b)^T ---------------------------------------
+    if (tid == 0) {
+      fence_after_sync();
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint64_t db = sdesc(sb + OFF_WQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+        mma_f16_ta(tbase + TM_D, tbase + TM_SA + kk * 8, db, ID_KK128, kk > 0);
       }
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
         const uint64_t da = sdesc(sb + OFF_VT + kk * 2048, 8192, 1024);
         const uint64_t db = sdesc(sb + OFF_TB + kk * 32, 16, 1024);
-        mma_f16(tbase + TM_D, da, db, ID_MK, kk > 0);
+        mma_f16(tbase + TM_D, da, db, ID_MK, 1);
       }
       mma_commit(bar);
     }
@@ -749,68 +807,36 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
     // the V tile is free: next chunk's v
     if (has_next) ld.v(c0 + kC, nn);
     cp_async_commit();
-    GDN_TRACE_POINT(7);
-
-    // ---- W^T 2^-f (fp32) -> fp16 tile, rows d, columns t ------------------------
-    {
-      float v[32];
-      tmem_ld32(tW + half * 32, v);
-      tmem_wait_ld();
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        st_chunk_f16(sb + OFF_WT + sw128_chunk(row, half * 4 + q, 128), v + 8 * q, 1.f);
-    }
-    fence_proxy_async();
-    fence_before_sync();
-    __syncthreads();
     GDN_TRACE_POINT(8);
 
-    // ---- MMA1: Delta^T 2^-(e+f) = U^T - S^T W^T ---------------------------------------
-    if (tid == 0) {
-      fence_after_sync();
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint64_t da = sdesc(sb + OFF_S0T + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-        const uint64_t db = sdesc(sb + OFF_WT + kk * 2048, 16384, 1024);
-        mma_f16(tbase + TM_D, da, db, ID_KM_NEG, 1);
-      }
-      mma_commit(bar);
-    }
-    ok = mbar_wait(bar, phase, kWaitLimit);
-    phase ^= 1;
-    if (!__syncthreads_and(ok)) { ok = false; break; }
-    fence_after_sync();
-    GDN_TRACE_POINT(9);
-
-    // ---- Delta^T 2^-e -> fp16 tile, rows j, columns i -------------------------------
+    // ---- Delta^T 2^-e -> fp16 A operand in TMEM (token pairs per column) -------
     {
       float v[32];
       tmem_ld32(tD + half * 32, v);
       tmem_wait_ld();
       const float sf = ldexpf(1.f, f);
+      uint32_t pk[16];
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
-        st_chunk_f16(sb + OFF_DT + sw128_chunk(row, half * 4 + q, 128), v + 8 * q, sf);
+      for (int x = 0; x < 16; ++x) pk[x] = pack_f16(v[2 * x] * sf, v[2 * x + 1] * sf);
+      tmem_st16(tDA + half * 16, pk);
+      tmem_wait_st();
     }
-    fence_proxy_async();
     fence_before_sync();
     __syncthreads();
-    GDN_TRACE_POINT(10);
+    GDN_TRACE_POINT(9);
 
-    // ---- MMA3: S^T += Delta^T (dec K^);  MMA4: Y^T += Delta^T P^T ---------------------
+    // ---- S^T += Delta^T (dec K^);  Y^T += Delta^T P^T ------------------------------
     if (tid == 0) {
       fence_after_sync();
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t da = sdesc(sb + OFF_DT + kk * 32, 16, 1024);
         const uint64_t db = sdesc(sb + OFF_KT + kk * 2048, 8192, 1024);
-        mma_f16(tbase + TM_S, da, db, ID_KM128, 1);
+        mma_f16_ta(tbase + TM_S, tbase + TM_DA + kk * 8, db, ID_KM128, 1);
       }
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t da = sdesc(sb + OFF_DT + kk * 32, 16, 1024);
         const uint64_t db = sdesc(sb + OFF_P + kk * 32, 16, 1024);
-        mma_f16(tbase + TM_Y, da, db, ID_KK, 1);
+        mma_f16_ta(tbase + TM_Y, tbase + TM_DA + kk * 8, db, ID_KK, 1);
       }
       mma_commit(bar);
     }
@@ -818,9 +844,9 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
     phase ^= 1;
     if (!__syncthreads_and(ok)) { ok = false; break; }
     fence_after_sync();
-    GDN_TRACE_POINT(11);
+    GDN_TRACE_POINT(10);
 
-    // ---- epilogue: Y^T 2^-e -> y through the staging buffer ----------------------------
+    // ---- epilogue: y = scale 2^e Y^T; with the gate, out = y rr (1 + w) sigmoid(g)
     {
       float v[32];
       tmem_ld32(tY + half * 32, v);
@@ -843,32 +869,54 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
           sRr[tid] = rsqrtf((sRed[tid] + sRed[64 + tid] + sRed[128 + tid] + sRed[192 + tid]) /
                                 (float)kD + a.eps_norm);
         __syncthreads();
-      }
-      __nv_bfloat16* gs = reinterpret_cast<__nv_bfloat16*>(gb + OFF_GS + buf * 16384);
-      const float w1 = 1.f + wj;
+        // y rr (|y rr| <= sqrt(d_v)) as fp16, token-major, into the staging tile
+        __half* yst = reinterpret_cast<__half*>(gb + OFF_STG) + half * 32 * kD + row;
+        const float4* rr4 = reinterpret_cast<const float4*>(sRr + half * 32);
 #pragma unroll
-      for (int x = 0; x < 32; ++x) {
-        const int t = half * 32 + x;
-        float o = v[x];
-        if (has_g) {
-          const float gg = __bfloat162float(gs[t * kD + row]);
-          o = __fdividef(o * sRr[t] * w1, 1.f + __expf(-gg));
+        for (int x4 = 0; x4 < 8; ++x4) {
+          const float4 r = rr4[x4];
+          yst[(4 * x4 + 0) * kD] = __float2half_rn(v[4 * x4 + 0] * r.x);
+          yst[(4 * x4 + 1) * kD] = __float2half_rn(v[4 * x4 + 1] * r.y);
+          yst[(4 * x4 + 2) * kD] = __float2half_rn(v[4 * x4 + 2] * r.z);
+          yst[(4 * x4 + 3) * kD] = __float2half_rn(v[4 * x4 + 3] * r.w);
         }
-        gs[t * kD + row] = __float2bfloat16_rn(o);
-      }
-      __syncthreads();
+        __syncthreads();
+        // 8 consecutive outputs of one token per piece, times the gate factors
+        const int ch = tid & 15;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int idx = tid + kNT * k;
-        const int rr = idx >> 4, ch = idx & 15;
-        if (rr < n) {
-          const uint4 val = ld_shared_v4(sb + OFF_GS + buf * 16384 + rr * 256 + ch * 16);
-          *reinterpret_cast<uint4*>(Yg + ((size_t)(c0 + rr) * a.H_v + h) * kD + ch * 8) = val;
+        for (int k = 0; k < 4; ++k) {
+          const int rr = (tid >> 4) + 16 * k;
+          if (rr < n) {
+            float yf[8], gf[8];
+            unpack_f16x8(ld_shared_v4(sb + OFF_STG + rr * 256 + ch * 16), yf);
+            unpack_f16x8(ld_shared_v4(gsb + rr * 256 + ch * 16), gf);
+            uint32_t o[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              o[q] = pack_bf16(yf[2 * q] * gf[2 * q], yf[2 * q + 1] * gf[2 * q + 1]);
+            *reinterpret_cast<uint4*>(Yg + ((size_t)(c0 + rr) * a.H_v + h) * kD + ch * 8) =
+                make_uint4(o[0], o[1], o[2], o[3]);
+          }
+        }
+      } else {
+        // no gate: y as bf16 through the staging tile, coalesced stores
+        __nv_bfloat16* gs = reinterpret_cast<__nv_bfloat16*>(gb + OFF_STG);
+#pragma unroll
+        for (int x = 0; x < 32; ++x) gs[(half * 32 + x) * kD + row] = __float2bfloat16_rn(v[x]);
+        __syncthreads();
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int idx = tid + kNT * k;
+          const int rr = idx >> 4, ch = idx & 15;
+          if (rr < n) {
+            const uint4 val = ld_shared_v4(sb + OFF_STG + rr * 256 + ch * 16);
+            *reinterpret_cast<uint4*>(Yg + ((size_t)(c0 + rr) * a.H_v + h) * kD + ch * 8) = val;
+          }
         }
       }
     }
     fence_before_sync();
-    GDN_TRACE_POINT(12);
+    GDN_TRACE_POINT(11);
   }
   cp_async_wait_all();
 
