@@ -458,6 +458,40 @@ def run_ours(args, world, rank, local):
                   "clocks": dclk_r}
         launches_decode = nsteps * max(3, args.steps // 2)
 
+        # multi-token decode: the same 64 tokens as 16 launches of 4 tokens
+        # per sequence (speculative verification), state read/written once
+        # per launch, in place
+        from gated_deltanet_scan_chunked_b200 import gdn_decode_multi
+        TS = 4
+        tr = lambda x: x.transpose(0, 1).contiguous()
+        groups = [dict(q=tr(d.q[c:c + TS]), k=tr(d.k[c:c + TS]), v=tr(d.v[c:c + TS]),
+                       la=tr(d.log_alpha[c:c + TS]), b=tr(d.beta[c:c + TS]))
+                  for c in range(0, nsteps, TS)]
+        ym = torch.empty((N, TS, H_V, D), dtype=torch.bfloat16, device="cuda")
+
+        def mstep():
+            for gr in groups:
+                gdn_decode_multi(gr["q"], gr["k"], gr["v"], gr["la"], gr["b"], state, y=ym)
+
+        mclk = ClockSampler(local)
+        mclk.start()
+        mt = timed_steps(mstep, max(3, args.steps // 2), 2, world, flush=dreset, stream=stream)
+        mclk_r = mclk.stop()
+        mms = max_over_ranks(statistics.mean(mt), world) / len(groups)  # per launch
+        mbytes = N * 2 * H_V * D * D * 4 + TS * (decode_bytes(N) - N * 2 * H_V * D * D * 4)
+        decode["multi_token"] = {
+            "workload": "256 sequences x 4 tokens per launch (16 launches = the same 64 tokens), "
+                        "in place",
+            "us_per_launch": mms * 1e3,
+            "tokens_per_s": world * N * TS / (mms * 1e-3),
+            "state_GBps": world * sbytes / (mms * 1e-3) / 1e9,
+            "roofline": {"bound": "hbm", "achieved": mbytes / (mms * 1e-3) / 1e9,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": mbytes / (mms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                         "algorithmic_bytes": mbytes},
+            "clocks": mclk_r}
+        launches_decode += len(groups) * max(3, args.steps // 2)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, target_s=args.ref_seconds)

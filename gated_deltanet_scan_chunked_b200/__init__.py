@@ -5,7 +5,7 @@ include/gdn.h).  ``gdn`` is a thin ctypes binding; ``inputs`` holds the
 seeded synthetic workloads; ``build`` compiles the library.
 """
 from .gdn import (GdnError, gdn_check_device_error, gdn_chunk_fwd,  # noqa: F401
-                  gdn_decode_step, load, workspace_size)
+                  gdn_decode_multi, gdn_decode_step, load, workspace_size)
 
-__all__ = ["gdn_chunk_fwd", "gdn_decode_step", "gdn_check_device_error", "GdnError", "load",
-           "workspace_size"]
+__all__ = ["gdn_chunk_fwd", "gdn_decode_step", "gdn_decode_multi", "gdn_check_device_error",
+           "GdnError", "load", "workspace_size"]

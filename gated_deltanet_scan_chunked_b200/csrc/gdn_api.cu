@@ -136,26 +136,57 @@ extern "C" gdn_status gdn_chunk_fwd(
                             eps_norm, scale, y, final_state, GDN_PATH_AUTO, stream);
 }
 
+extern "C" gdn_status gdn_decode_multi(
+    const void* q, const void* k, const void* v, const float* log_alpha, const float* beta,
+    const void* g, const float* norm_w, const float* state_in, float* state_out,
+    float* snapshots, int32_t N, int32_t T_s, int32_t H_qk, int32_t H_v, int32_t d_k,
+    int32_t d_v, gdn_dtype in_dtype, int32_t l2norm_qk, float eps_l2, float eps_norm,
+    float scale, void* y, gdn_stream_t stream) {
+  gdn_status st = check_common(H_qk, H_v, d_k, d_v, in_dtype, eps_l2, eps_norm);
+  if (st != GDN_OK) return st;
+  if (N < 0 || T_s < 0 || (int64_t)N * H_v > 0x7fffffffLL) return GDN_ERR_INVALID_ARG;
+  if (N == 0 || T_s == 0) return GDN_OK;
+  if (!q || !k || !v || !log_alpha || !beta || !state_in || !y) return GDN_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, log_alpha, beta, g, norm_w, state_in, state_out, snapshots, y};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
+  const size_t sbytes = (size_t)N * H_v * d_k * d_v * sizeof(float);
+  if (state_out && state_out != state_in) {
+    // exact aliasing is allowed; partial overlap is not
+    const char* a0 = reinterpret_cast<const char*>(state_in);
+    const char* b0 = reinterpret_cast<const char*>(state_out);
+    if (a0 < b0 + sbytes && b0 < a0 + sbytes) return GDN_ERR_INVALID_ARG;
+  }
+  if (snapshots) {
+    // snapshots may not overlap either state
+    const char* s0 = reinterpret_cast<const char*>(snapshots);
+    const size_t nb = sbytes * (size_t)T_s;
+    const float* states[] = {state_in, state_out};
+    for (const float* x : states) {
+      const char* x0 = reinterpret_cast<const char*>(x);
+      if (x && x0 < s0 + nb && s0 < x0 + sbytes) return GDN_ERR_INVALID_ARG;
+    }
+  }
+  DecodeArgs a;
+  a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
+  a.g = g; a.norm_w = g ? norm_w : nullptr;
+  a.state_in = state_in; a.state_out = state_out; a.snapshots = snapshots; a.y = y;
+  a.N = N; a.T_s = T_s; a.H_qk = H_qk; a.H_v = H_v; a.d_k = d_k; a.d_v = d_v;
+  a.dtype = in_dtype;
+  a.l2norm = l2norm_qk ? 1 : 0; a.eps_l2 = eps_l2; a.eps_norm = eps_norm; a.scale = scale;
+  return launch_decode(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
 extern "C" gdn_status gdn_decode_step(const void* q, const void* k, const void* v,
                                       const float* log_alpha, const float* beta, const void* g,
                                       const float* norm_w, float* state, int32_t N, int32_t H_qk,
                                       int32_t H_v, int32_t d_k, int32_t d_v, gdn_dtype in_dtype,
                                       int32_t l2norm_qk, float eps_l2, float eps_norm,
                                       float scale, void* y, gdn_stream_t stream) {
-  gdn_status st = check_common(H_qk, H_v, d_k, d_v, in_dtype, eps_l2, eps_norm);
-  if (st != GDN_OK) return st;
-  if (N < 0 || (int64_t)N * H_v > 0x7fffffffLL) return GDN_ERR_INVALID_ARG;
-  if (N == 0) return GDN_OK;
-  if (!q || !k || !v || !log_alpha || !beta || !state || !y) return GDN_ERR_INVALID_ARG;
-  const void* ptrs[] = {q, k, v, log_alpha, beta, g, norm_w, state, y};
-  for (const void* p : ptrs)
-    if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
-  DecodeArgs a;
-  a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
-  a.g = g; a.norm_w = g ? norm_w : nullptr; a.state = state; a.y = y;
-  a.N = N; a.H_qk = H_qk; a.H_v = H_v; a.d_k = d_k; a.d_v = d_v; a.dtype = in_dtype;
-  a.l2norm = l2norm_qk ? 1 : 0; a.eps_l2 = eps_l2; a.eps_norm = eps_norm; a.scale = scale;
-  return launch_decode(a, reinterpret_cast<cudaStream_t>(stream));
+  if (N > 0 && !state) return GDN_ERR_INVALID_ARG;
+  return gdn_decode_multi(q, k, v, log_alpha, beta, g, norm_w, state, state, nullptr, N, 1,
+                          H_qk, H_v, d_k, d_v, in_dtype, l2norm_qk, eps_l2, eps_norm, scale, y,
+                          stream);
 }
 
 extern "C" gdn_status gdn_check_device_error(gdn_stream_t stream) {

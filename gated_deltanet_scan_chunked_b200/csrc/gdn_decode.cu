@@ -10,7 +10,10 @@
 //   S'  = alpha S + beta k^ e^T
 //   y   = S'^T q^ = alpha b + beta (k^ . q^) e        (times `scale`)
 // so the state is loaded into registers, reduced once over d_k, updated and
-// stored back, with no second read.
+// stored back, with no second read.  Several tokens of one sequence (for
+// speculative verification) run in one launch: the state stays in registers
+// from token to token, is read once and written once, and may be
+// snapshotted after every token.
 //
 // Thread layout (d_k = d_v = 128, 256 threads): thread (rg, c4) owns columns
 // 4*c4 .. 4*c4+3 (one float4) of rows rg, rg+8, ..., rg+120; a warp reads one
@@ -47,7 +50,8 @@ __global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT)
   const int tid = threadIdx.x;
   const int rg = tid / TPR, c4 = tid % TPR;
 
-  float* S = a.state + ((size_t)n * a.H_v + h) * (size_t)(DK * DV);
+  // one token, state updated in place (state_out == state_in)
+  float* S = a.state_out + ((size_t)n * a.H_v + h) * (size_t)(DK * DV);
   // issue every state load first: they are the whole cost of the step
   float4 s[RPT];
 #pragma unroll
@@ -145,10 +149,159 @@ __global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT)
   if (rg == 0) Elem<Tin>::store4(static_cast<Tin*>(a.y) + yo, y);
 }
 
+// a.T_s tokens per sequence, the state in registers from token to token,
+// stored to state_out after the last token and optionally snapshotted after
+// every token.
+template <int DK, int DV, typename Tin>
+__global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT)
+    gdn_decode_multi_kernel(const DecodeArgs a) {
+  using Geo = DecodeGeom<DK, DV>;
+  constexpr int TPR = Geo::TPR, ROWG = Geo::ROWG, RPT = Geo::RPT;
+  __shared__ float sq[DK], sk[DK];
+  __shared__ float4 red_a[ROWG][TPR], red_b[ROWG][TPR];
+  __shared__ float snorm[3];
+
+  const int n = blockIdx.x / a.H_v;
+  const int h = blockIdx.x % a.H_v;
+  const int hq = h / (a.H_v / a.H_qk);
+  const int tid = threadIdx.x;
+  const int rg = tid / TPR, c4 = tid % TPR;
+  const bool has_g = a.g != nullptr;
+  const int T_s = a.T_s;
+
+  const size_t so = ((size_t)n * a.H_v + h) * (size_t)(DK * DV);
+  const float* Sin = a.state_in + so;
+  // issue every state load first: they are the whole cost of the step
+  float4 s[RPT];
+#pragma unroll
+  for (int r = 0; r < RPT; ++r) {
+    const int i = rg + ROWG * r;
+    s[r] = __ldcs(reinterpret_cast<const float4*>(Sin + (size_t)i * DV) + c4);
+  }
+
+  // The per-token inputs go through registers one token ahead (token t + 1's
+  // q, k, v, gates and g are in flight while token t is computed).  Every
+  // thread holds at most one element of q and k.
+  static_assert(Geo::NT >= DK, "one q/k element per thread");
+  float qn = 0.f, kn = 0.f, lan = 0.f, bn = 0.f;
+  float4 vn = make_float4(0.f, 0.f, 0.f, 0.f), gn = vn;
+  auto fetch_token = [&](int t) {
+    const size_t tok = (size_t)n * T_s + t;  // token row in the [N, T_s, ...] inputs
+    const size_t vo = (tok * a.H_v + h) * DV + 4 * c4;
+    if (tid < DK) {
+      qn = Elem<Tin>::load(static_cast<const Tin*>(a.q) + (tok * a.H_qk + hq) * DK + tid);
+      kn = Elem<Tin>::load(static_cast<const Tin*>(a.k) + (tok * a.H_qk + hq) * DK + tid);
+    }
+    vn = Elem<Tin>::load4(static_cast<const Tin*>(a.v) + vo);
+    if (has_g) gn = Elem<Tin>::load4(static_cast<const Tin*>(a.g) + vo);
+    lan = __ldg(a.log_alpha + tok * a.H_v + h);
+    bn = __ldg(a.beta + tok * a.H_v + h);
+  };
+  fetch_token(0);
+
+  for (int t = 0; t < T_s; ++t) {
+    const size_t tok = (size_t)n * T_s + t;
+    if (tid < DK) {
+      sq[tid] = qn;
+      sk[tid] = kn;
+    }
+    const float4 v4 = vn, g4 = gn;
+    const float alpha = __expf(lan), beta = bn;
+    if (t + 1 < T_s) fetch_token(t + 1);
+    __syncthreads();
+    if (tid < 32) {
+      float nq = 0.f, nk = 0.f, kq = 0.f;
+      for (int i = tid; i < DK; i += 32) {
+        nq += sq[i] * sq[i];
+        nk += sk[i] * sk[i];
+        kq += sk[i] * sq[i];
+      }
+      nq = warp_sum(nq);
+      nk = warp_sum(nk);
+      kq = warp_sum(kq);
+      if (tid == 0) {
+        const float rq = a.l2norm ? rsqrtf(nq + a.eps_l2) : 1.f;
+        const float rk = a.l2norm ? rsqrtf(nk + a.eps_l2) : 1.f;
+        snorm[0] = rq;
+        snorm[1] = rk;
+        snorm[2] = kq * rq * rk;
+      }
+    }
+    __syncthreads();
+    const float rq = snorm[0], rk = snorm[1], kq = snorm[2];
+
+    // a = S^T k^, b = S^T q^ over this thread's rows, then across row groups
+    float4 pa = make_float4(0.f, 0.f, 0.f, 0.f), pb = pa;
+    float kk[RPT];
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) {
+      const int i = rg + ROWG * r;
+      const float ki = sk[i] * rk, qi = sq[i] * rq;
+      kk[r] = ki;
+      pa.x += s[r].x * ki; pa.y += s[r].y * ki; pa.z += s[r].z * ki; pa.w += s[r].w * ki;
+      pb.x += s[r].x * qi; pb.y += s[r].y * qi; pb.z += s[r].z * qi; pb.w += s[r].w * qi;
+    }
+    red_a[rg][c4] = pa;
+    red_b[rg][c4] = pb;
+    __syncthreads();
+    float4 ta = make_float4(0.f, 0.f, 0.f, 0.f), tb = ta;
+#pragma unroll
+    for (int g2 = 0; g2 < ROWG; ++g2) {
+      const float4 x = red_a[g2][c4], z = red_b[g2][c4];
+      ta.x += x.x; ta.y += x.y; ta.z += x.z; ta.w += x.w;
+      tb.x += z.x; tb.y += z.y; tb.z += z.z; tb.w += z.w;
+    }
+    float4 e;
+    e.x = v4.x - alpha * ta.x; e.y = v4.y - alpha * ta.y;
+    e.z = v4.z - alpha * ta.z; e.w = v4.w - alpha * ta.w;
+
+    // S' = alpha S + beta k^ e^T (each thread updates exactly the elements it
+    // loaded), kept in registers, optionally snapshotted, stored to
+    // state_out after the last token
+    float* snap = a.snapshots ? a.snapshots + ((size_t)t * a.N * a.H_v) * (size_t)(DK * DV) + so
+                              : nullptr;
+    float* sout = (t + 1 == T_s && a.state_out) ? a.state_out + so : nullptr;
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) {
+      const int i = rg + ROWG * r;
+      const float bk = beta * kk[r];
+      float4 o;
+      o.x = alpha * s[r].x + bk * e.x; o.y = alpha * s[r].y + bk * e.y;
+      o.z = alpha * s[r].z + bk * e.z; o.w = alpha * s[r].w + bk * e.w;
+      s[r] = o;
+      if (snap) __stcs(reinterpret_cast<float4*>(snap + (size_t)i * DV) + c4, o);
+      if (sout) __stcs(reinterpret_cast<float4*>(sout + (size_t)i * DV) + c4, o);
+    }
+
+    // y = scale (alpha b + beta (k^.q^) e), then the optional epilogue
+    const float bkq = beta * kq;
+    float4 y;
+    y.x = a.scale * (alpha * tb.x + bkq * e.x); y.y = a.scale * (alpha * tb.y + bkq * e.y);
+    y.z = a.scale * (alpha * tb.z + bkq * e.z); y.w = a.scale * (alpha * tb.w + bkq * e.w);
+    const size_t yo = (tok * a.H_v + h) * DV + 4 * c4;
+    if (has_g) {
+      float ss = y.x * y.x + y.y * y.y + y.z * y.z + y.w * y.w;
+      ss = group_sum<TPR>(ss);  // every row group holds the same y
+      const float r = rsqrtf(ss / (float)DV + a.eps_norm);
+      float4 w4 = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (a.norm_w) w4 = __ldg(reinterpret_cast<const float4*>(a.norm_w + 4 * c4));
+      y.x = y.x * r * (1.f + w4.x) * sigmoidf_(g4.x);
+      y.y = y.y * r * (1.f + w4.y) * sigmoidf_(g4.y);
+      y.z = y.z * r * (1.f + w4.z) * sigmoidf_(g4.z);
+      y.w = y.w * r * (1.f + w4.w) * sigmoidf_(g4.w);
+    }
+    if (rg == 0) Elem<Tin>::store4(static_cast<Tin*>(a.y) + yo, y);
+  }  // tokens
+}
+
 template <int DK, int DV, typename Tin>
 gdn_status launch(const DecodeArgs& a, cudaStream_t stream) {
   const unsigned grid = (unsigned)a.N * (unsigned)a.H_v;
-  gdn_decode_kernel<DK, DV, Tin><<<grid, DecodeGeom<DK, DV>::NT, 0, stream>>>(a);
+  const bool single = a.T_s == 1 && a.snapshots == nullptr && a.state_out == a.state_in;
+  if (single)
+    gdn_decode_kernel<DK, DV, Tin><<<grid, DecodeGeom<DK, DV>::NT, 0, stream>>>(a);
+  else
+    gdn_decode_multi_kernel<DK, DV, Tin><<<grid, DecodeGeom<DK, DV>::NT, 0, stream>>>(a);
   return cudaPeekAtLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
@@ -175,7 +328,7 @@ gdn_status dispatch_dv(const DecodeArgs& a, cudaStream_t s) {
 }  // namespace
 
 gdn_status launch_decode(const DecodeArgs& a, cudaStream_t stream) {
-  if (a.N == 0) return GDN_OK;
+  if (a.N == 0 || a.T_s == 0) return GDN_OK;
   if (a.dtype == GDN_BF16) return dispatch_dv<__nv_bfloat16>(a, stream);
   if (a.dtype == GDN_FP32) return dispatch_dv<float>(a, stream);
   return GDN_ERR_UNSUPPORTED;

@@ -42,16 +42,18 @@ struct PrefillArgs {
 };
 
 struct DecodeArgs {
-  const void* q;
+  const void* q;           // [N, T_s, H_qk, d_k]
   const void* k;
-  const void* v;
-  const float* log_alpha;
+  const void* v;           // [N, T_s, H_v, d_v]
+  const float* log_alpha;  // [N, T_s, H_v]
   const float* beta;
-  const void* g;
+  const void* g;           // [N, T_s, H_v, d_v] or nullptr
   const float* norm_w;
-  float* state;
-  void* y;
-  int32_t N, H_qk, H_v, d_k, d_v;
+  const float* state_in;   // [N, H_v, d_k, d_v]
+  float* state_out;        // same shape, may be state_in; nullptr: not written
+  float* snapshots;        // [T_s, N, H_v, d_k, d_v] or nullptr: state after each token
+  void* y;                 // [N, T_s, H_v, d_v]
+  int32_t N, T_s, H_qk, H_v, d_k, d_v;
   gdn_dtype dtype;
   int32_t l2norm;
   float eps_l2, eps_norm, scale;

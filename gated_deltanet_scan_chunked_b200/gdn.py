@@ -70,6 +70,10 @@ def load(path: str = LIB_PATH):
     f.restype = ctypes.c_int
     f.argtypes = [_vp] * 8 + [ctypes.c_int32] * 6 + [
         ctypes.c_int32, ctypes.c_float, ctypes.c_float, ctypes.c_float, _vp, _vp]
+    f = lib.gdn_decode_multi
+    f.restype = ctypes.c_int
+    f.argtypes = [_vp] * 10 + [ctypes.c_int32] * 7 + [
+        ctypes.c_int32, ctypes.c_float, ctypes.c_float, ctypes.c_float, _vp, _vp]
     lib.gdn_check_device_error.restype = ctypes.c_int
     lib.gdn_check_device_error.argtypes = [_vp]
     lib.gdn_status_string.restype = ctypes.c_char_p
@@ -248,6 +252,45 @@ def gdn_decode_step(q, k, v, log_alpha, beta, state, g=None, norm_w=None,
     if st != GDN_OK:
         raise GdnError(st, "gdn_decode_step")
     return y
+
+
+def gdn_decode_multi(q, k, v, log_alpha, beta, state_in, state_out="in_place",
+                     snapshots=None, g=None, norm_w=None, l2norm_qk=True, eps_l2=1e-6,
+                     eps_norm=1e-6, scale=1.0, y=None, stream=None) -> torch.Tensor:
+    """T_s tokens per sequence in one launch.  q, k [N, T_s, H_qk, d_k];
+    v [N, T_s, H_v, d_v]; gates [N, T_s, H_v]; state_in [N, H_v, d_k, d_v]
+    fp32.  state_out: "in_place" (default: state_in is updated), a tensor, or
+    None (not written).  snapshots: None, True (allocated here), or a
+    [T_s, N, H_v, d_k, d_v] fp32 tensor receiving the state after each
+    token.  Returns (y, snapshots)."""
+    lib = load()
+    dev = q.device
+    dt = _dtype_code(q)
+    N, T_s, Hqk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    for name, t in (("q", q), ("k", k), ("v", v), ("g", g)):
+        _check(t, name, q.dtype, dev)
+    if isinstance(state_out, str):
+        if state_out != "in_place":
+            raise ValueError("state_out must be a tensor, None or 'in_place'")
+        state_out = state_in
+    if snapshots is True:
+        snapshots = torch.empty((T_s, N, Hv, dk, dv), dtype=torch.float32, device=dev)
+    for name, t in (("log_alpha", log_alpha), ("beta", beta), ("norm_w", norm_w),
+                    ("state_in", state_in), ("state_out", state_out),
+                    ("snapshots", snapshots)):
+        _check(t, name, torch.float32, dev)
+    if y is None:
+        y = torch.empty((N, T_s, Hv, dv), dtype=q.dtype, device=dev)
+    _check(y, "y", q.dtype, dev)
+    st = lib.gdn_decode_multi(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(g), _ptr(norm_w),
+        _ptr(state_in), _ptr(state_out), _ptr(snapshots), N, T_s, Hqk, Hv, dk, dv, dt,
+        1 if l2norm_qk else 0, float(eps_l2), float(eps_norm), float(scale), _ptr(y),
+        _stream_handle(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_decode_multi")
+    return y, snapshots
 
 
 def gdn_check_device_error(stream=None) -> int:

@@ -220,6 +220,36 @@ gdn_status gdn_decode_step(
     float scale, void* y, gdn_stream_t stream);
 
 /*
+ * gdn_decode_multi -- T_s consecutive tokens for each of N independent
+ * sequences in one launch (e.g. verifying T_s speculative tokens).  The
+ * result equals T_s calls of gdn_decode_step; the state is read once and
+ * written once, and may be snapshotted after every token so that a caller
+ * can roll back to any accepted prefix.  (A deployment variant of the decode
+ * step; the update per token is the one described for gdn_decode_step.)
+ *
+ *   q, k        [N, T_s, H_qk, d_k] in_dtype
+ *   v           [N, T_s, H_v, d_v]  in_dtype
+ *   log_alpha   [N, T_s, H_v] fp32;  beta [N, T_s, H_v] fp32
+ *   g, norm_w   optional epilogue: g [N, T_s, H_v, d_v], as for gdn_chunk_fwd
+ *   state_in    [N, H_v, d_k, d_v] fp32, the state before the first token
+ *   state_out   [N, H_v, d_k, d_v] fp32, the state after the last token; may
+ *               be state_in exactly (in place), must not partially overlap
+ *               it; NULL: not written (state_in is left as it was)
+ *   snapshots   [T_s, N, H_v, d_k, d_v] fp32 or NULL: snapshot t holds the
+ *               state after token t of every sequence (each one a valid
+ *               state tensor); must not overlap state_in or state_out
+ *   y           [N, T_s, H_v, d_v] in_dtype, written
+ * Other arguments as for gdn_chunk_fwd.  N = 0 or T_s = 0 is a no-op.
+ */
+gdn_status gdn_decode_multi(
+    const void* q, const void* k, const void* v, const float* log_alpha,
+    const float* beta, const void* g, const float* norm_w,
+    const float* state_in, float* state_out, float* snapshots, int32_t N,
+    int32_t T_s, int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v,
+    gdn_dtype in_dtype, int32_t l2norm_qk, float eps_l2, float eps_norm,
+    float scale, void* y, gdn_stream_t stream);
+
+/*
  * gdn_check_device_error -- synchronise `stream`, then read and clear the
  * library's device-side error word on the current device.  Returns GDN_OK,
  * GDN_ERR_TIMEOUT (a kernel's bounded wait ran out and the kernel returned

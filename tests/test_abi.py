@@ -146,3 +146,29 @@ def test_static_workspace_call_rejects_on_host(lib):
     assert call(n_seq=1, cu=None, dk=64) == gdn.GDN_ERR_UNSUPPORTED
     assert call(n_seq=1, cu=None, dt=1) == gdn.GDN_ERR_UNSUPPORTED
     assert call(n_seq=0) == gdn.GDN_ERR_INVALID_ARG
+
+
+def _multi(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, b=FAKE, g=None, w=None, si=FAKE, so=FAKE,
+             sn=None, N=4, T=4, Hqk=16, Hv=48, dk=128, dv=128, dt=0, y=FAKE)
+    a.update(kw)
+    return lib.gdn_decode_multi(a["q"], a["k"], a["v"], a["la"], a["b"], a["g"], a["w"],
+                                a["si"], a["so"], a["sn"], a["N"], a["T"], a["Hqk"], a["Hv"],
+                                a["dk"], a["dv"], a["dt"], 1, 1e-6, 1e-6, 1.0, a["y"], None)
+
+
+STATE_BYTES = 4 * 48 * 128 * 128 * 4
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(T=-1), gdn.GDN_ERR_INVALID_ARG),
+    (dict(si=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(so=FAKE + 4096), gdn.GDN_ERR_INVALID_ARG),                   # partial overlap
+    (dict(so=FAKE + STATE_BYTES, sn=FAKE + 4096), gdn.GDN_ERR_INVALID_ARG),  # snapshots overlap
+    (dict(sn=FAKE + 8), gdn.GDN_ERR_INVALID_ARG),                      # misaligned
+    (dict(dk=48), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(T=0, q=None), gdn.GDN_OK),                                   # no-op
+    (dict(N=0, y=None), gdn.GDN_OK),
+])
+def test_decode_multi_rejects_bad_arguments_on_host(lib, kw, code):
+    assert _multi(lib, **kw) == code
