@@ -1510,7 +1510,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
     for (int j2 = 0; j2 < 8; ++j2)
       wv[j2] = 1.f + ((has_g && a.norm_w) ? __ldg(a.norm_w + (tid & 15) * 8 + j2) : 0.f);
     const __nv_bfloat16* Gh = static_cast<const __nv_bfloat16*>(a.g);
-    uint4 gfac[4];  // this thread's gate factors (fp16 x 8 per piece)
+    uint4 graw[4];  // this thread's g pieces of the chunk (bf16 x 8)
     // Split launch, thread 0: the slot whose bulk stores are in flight and
     // not yet published (published once complete, during the next chunk).
     int pend_slot = -1;
@@ -1522,6 +1522,26 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
         fence_proxy_async_global();
         st_release_u64(&ready[pend_slot], pend_val);
         pend_slot = -1;
+      }
+    };
+    // Split launch, thread 0: a slot whose bulk stores are staged but not
+    // yet issued.  They are issued right after the next loop-top barrier:
+    // issued earlier, the loop-top proxy fence would wait for their reads.
+    int iss_slot = -1, iss_lb = 0;
+    unsigned long long iss_val = 0;
+    auto issue = [&]() {
+      if (iss_slot >= 0) {
+        uint8_t* dst = ring + (size_t)iss_slot * kSlotBytes;
+        const uint32_t src = sb + P_STG + iss_lb * kShipBytes;
+        fence_proxy_async_global();
+#pragma unroll
+        for (int k = 0; k < 4; ++k) bulk_store_s2g(dst + 16384 * k, src + 16384 * k, 16384);
+        if (has_g) bulk_store_s2g(dst + kSlotGF, sb + P_A, 16384);
+        bulk_store_s2g(dst + kSlotLoad, sb + P_SCAL + 16 * iss_lb, 16);
+        bulk_commit();
+        pend_slot = iss_slot;
+        pend_val = iss_val;
+        iss_slot = -1;
       }
     };
     int ci = first, lc = 0;  // chunk index, local count
@@ -1544,6 +1564,9 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
           okw = mbar_wait_cluster(&stg_free[lb], ((lc - 2) >> 1) & 1, kWaitLimit);
       }
       if (!__syncthreads_and(okw)) { ok = false; break; }
+      if constexpr (kGlobal) {
+        if (tid == 0) issue();  // the previous chunk's slot
+      }
       GDN_TRACE_POINT(20);
 
       if constexpr (kGlobal) {
@@ -1635,6 +1658,11 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
       }
       fence_proxy_async();
       fence_before_sync();
+      // split launch: the last bulk store has finished reading its sources
+      // before the A scratch (its gate-factor staging) is rewritten below
+      if constexpr (kGlobal) {
+        if (tid == 0) bulk_wait_read_all();
+      }
       okw = mbar_wait(mbar, phase, kWaitLimit);
       phase ^= 1;
       if (!__syncthreads_and(okw)) { ok = false; break; }
@@ -1746,26 +1774,13 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
         if constexpr (kGlobal) publish();
       }
       if constexpr (kGlobal) {
-        // this chunk's gate factors from g (in L2) while the MMAs run; they
-        // are stored once the slot is free
+        // this chunk's g rows (from L2) while the MMAs run
         if (has_g) {
-          uint4 graw[4];
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             const int rr = (tid >> 4) + 16 * k;
             graw[k] = rr < n ? ld_nc_v4(Gh + ((size_t)(c0 + rr) * a.H_v + h) * kD + (tid & 15) * 8)
                              : make_uint4(0u, 0u, 0u, 0u);
-          }
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            float gf[8];
-            unpack_bf16x8(graw[k], gf);
-            uint32_t o[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              o[q] = pack_f16(__fdividef(wv[2 * q], 1.f + __expf(-gf[2 * q])),
-                              __fdividef(wv[2 * q + 1], 1.f + __expf(-gf[2 * q + 1])));
-            gfac[k] = make_uint4(o[0], o[1], o[2], o[3]);
           }
         }
       }
@@ -1799,33 +1814,38 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
         // slot ci % kRing last held chunk ci - kRing: the chain CTA must
         // have loaded it
         const int s = ci % kRing;
-        uint8_t* dst = ring + (size_t)s * kSlotBytes;
         if (tid == 0 && ci >= kRing)
           okw = wait_flag_ge(&consumed[s], (unsigned long long)(ci - kRing) + 1, kWaitLimit);
-        if (!__syncthreads_and(okw)) { ok = false; break; }
-        GDN_TRACE_POINT(30);
-        if (tid == 0) {
-          fence_proxy_async_global();
-#pragma unroll
-          for (int k = 0; k < 4; ++k) bulk_store_s2g(dst + 16384 * k, stg + 16384 * k, 16384);
-          bulk_store_s2g(dst + kSlotLoad, sb + P_SCAL + 16 * lb, 16);
-          bulk_commit();
-          pend_slot = s;
-          pend_val = (unsigned long long)ci + 1;
-        }
         if (has_g) {
-          // gate factors, token-major [64][128] fp16, beside the tiles.  The
-          // barrier below orders these stores before thread 0's release of
-          // the slot (release is cumulative over what the barrier ordered).
+          // meanwhile (the other threads), the gate factors (1 + w) sigmoid(g),
+          // token-major [64][128] fp16, staged in the A scratch (dead since
+          // the W product) and shipped with the tiles
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             const int rr = (tid >> 4) + 16 * k;
-            if (rr < n)
-              *reinterpret_cast<uint4*>(dst + kSlotGF + rr * 256 + (tid & 15) * 16) = gfac[k];
+            float gf[8];
+            unpack_bf16x8(graw[k], gf);
+            uint32_t o[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              o[q] = pack_f16(__fdividef(wv[2 * q], 1.f + __expf(-gf[2 * q])),
+                              __fdividef(wv[2 * q + 1], 1.f + __expf(-gf[2 * q + 1])));
+            st_shared_v4(sb + P_A + rr * 256 + (tid & 15) * 16, o[0], o[1], o[2], o[3]);
+          }
+          fence_proxy_async();
+        }
+        if (!__syncthreads_and(okw)) { ok = false; break; }
+        GDN_TRACE_POINT(30);
+        if (tid == 0) {
+          iss_slot = s;
+          iss_lb = lb;
+          iss_val = (unsigned long long)ci + 1;
+          if (lc == 0) {
+            // the first chunk is shipped and published at once
+            issue();
+            publish();
           }
         }
-        __syncthreads();
-        if (tid == 0 && lc == 0) publish();
         GDN_TRACE_POINT(31);
       } else if (tid == 0) {
         okw = mbar_wait_cluster(&empty[b], ((ci >> 1) & 1) ^ 1, kWaitLimit);
@@ -1845,7 +1865,11 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
     }
     cp_async_wait_all();
     if constexpr (kGlobal) {
-      if (tid == 0 && ok) publish();
+      if (tid == 0 && ok) {
+        publish();
+        issue();
+        publish();
+      }
     }
     if (tid == 0) bulk_wait_all();
     if (!ok) {

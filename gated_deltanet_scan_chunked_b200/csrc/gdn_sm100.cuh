@@ -256,6 +256,10 @@ __device__ __forceinline__ void bulk_commit() {
 }
 // Bulk groups track only copies issued with bulk-group completion (shared ->
 // global); copies completed on an mbarrier are not part of any group.
+// Wait until no committed bulk group of this thread still reads its source.
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
 // Wait until every committed bulk group of this thread is complete.
 __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
