@@ -145,6 +145,7 @@ extern "C" gdn_status gdn_decode_multi(
   gdn_status st = check_common(H_qk, H_v, d_k, d_v, in_dtype, eps_l2, eps_norm);
   if (st != GDN_OK) return st;
   if (N < 0 || T_s < 0 || (int64_t)N * H_v > 0x7fffffffLL) return GDN_ERR_INVALID_ARG;
+  if (T_s > kMaxDecodeTokens) return GDN_ERR_UNSUPPORTED;
   if (N == 0 || T_s == 0) return GDN_OK;
   if (!q || !k || !v || !log_alpha || !beta || !state_in || !y) return GDN_ERR_INVALID_ARG;
   const void* ptrs[] = {q, k, v, log_alpha, beta, g, norm_w, state_in, state_out, snapshots, y};

@@ -151,84 +151,86 @@ __global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT)
 
 // a.T_s tokens per sequence, the state in registers from token to token,
 // stored to state_out after the last token and optionally snapshotted after
-// every token.
+// every token.  All tokens' inputs (q, k, v, g, gates) are staged in shared
+// memory at the start, in flight together with the state loads; per token
+// there is then a single block barrier (the cross-warp reduction, double
+// buffered by token parity), the q/k norms being computed by every warp.
 template <int DK, int DV, typename Tin>
 __global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT)
     gdn_decode_multi_kernel(const DecodeArgs a) {
   using Geo = DecodeGeom<DK, DV>;
-  constexpr int TPR = Geo::TPR, ROWG = Geo::ROWG, RPT = Geo::RPT;
-  __shared__ float sq[DK], sk[DK];
-  __shared__ float4 red_a[ROWG][TPR], red_b[ROWG][TPR];
-  __shared__ float snorm[3];
+  constexpr int TPR = Geo::TPR, ROWG = Geo::ROWG, RPT = Geo::RPT, NT = Geo::NT;
+  extern __shared__ float4 dsm4[];
+  __shared__ float4 red_a[2][ROWG][TPR], red_b[2][ROWG][TPR];
 
   const int n = blockIdx.x / a.H_v;
   const int h = blockIdx.x % a.H_v;
   const int hq = h / (a.H_v / a.H_qk);
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31;
   const int rg = tid / TPR, c4 = tid % TPR;
   const bool has_g = a.g != nullptr;
   const int T_s = a.T_s;
+  // staged inputs, fp32: q, k [T_s][DK]; v, g [T_s][DV]; log alpha, beta [T_s]
+  float* tq = reinterpret_cast<float*>(dsm4);
+  float* tk = tq + T_s * DK;
+  float* tv = tk + T_s * DK;
+  float* tg = tv + T_s * DV;
+  float* tla = tg + (has_g ? T_s * DV : 0);
+  float* tb = tla + T_s;
 
   const size_t so = ((size_t)n * a.H_v + h) * (size_t)(DK * DV);
   const float* Sin = a.state_in + so;
-  // issue every state load first: they are the whole cost of the step
+  // issue every state load first: they are the bulk of the traffic
   float4 s[RPT];
 #pragma unroll
   for (int r = 0; r < RPT; ++r) {
     const int i = rg + ROWG * r;
     s[r] = __ldcs(reinterpret_cast<const float4*>(Sin + (size_t)i * DV) + c4);
   }
-
-  // The per-token inputs go through registers one token ahead (token t + 1's
-  // q, k, v, gates and g are in flight while token t is computed).  Every
-  // thread holds at most one element of q and k.
-  static_assert(Geo::NT >= DK, "one q/k element per thread");
-  float qn = 0.f, kn = 0.f, lan = 0.f, bn = 0.f;
-  float4 vn = make_float4(0.f, 0.f, 0.f, 0.f), gn = vn;
-  auto fetch_token = [&](int t) {
-    const size_t tok = (size_t)n * T_s + t;  // token row in the [N, T_s, ...] inputs
-    const size_t vo = (tok * a.H_v + h) * DV + 4 * c4;
-    if (tid < DK) {
-      qn = Elem<Tin>::load(static_cast<const Tin*>(a.q) + (tok * a.H_qk + hq) * DK + tid);
-      kn = Elem<Tin>::load(static_cast<const Tin*>(a.k) + (tok * a.H_qk + hq) * DK + tid);
+  {
+    const Tin* Q = static_cast<const Tin*>(a.q);
+    const Tin* K = static_cast<const Tin*>(a.k);
+    const Tin* V = static_cast<const Tin*>(a.v);
+    const Tin* G = static_cast<const Tin*>(a.g);
+    for (int i = tid; i < T_s * DK; i += NT) {
+      const size_t tok = (size_t)n * T_s + i / DK;
+      tq[i] = Elem<Tin>::load(Q + (tok * a.H_qk + hq) * DK + i % DK);
+      tk[i] = Elem<Tin>::load(K + (tok * a.H_qk + hq) * DK + i % DK);
     }
-    vn = Elem<Tin>::load4(static_cast<const Tin*>(a.v) + vo);
-    if (has_g) gn = Elem<Tin>::load4(static_cast<const Tin*>(a.g) + vo);
-    lan = __ldg(a.log_alpha + tok * a.H_v + h);
-    bn = __ldg(a.beta + tok * a.H_v + h);
-  };
-  fetch_token(0);
+    for (int i = tid; i < T_s * DV; i += NT) {
+      const size_t tok = (size_t)n * T_s + i / DV;
+      tv[i] = Elem<Tin>::load(V + (tok * a.H_v + h) * DV + i % DV);
+      if (has_g) tg[i] = Elem<Tin>::load(G + (tok * a.H_v + h) * DV + i % DV);
+    }
+    for (int i = tid; i < T_s; i += NT) {
+      const size_t tok = (size_t)n * T_s + i;
+      tla[i] = __ldg(a.log_alpha + tok * a.H_v + h);
+      tb[i] = __ldg(a.beta + tok * a.H_v + h);
+    }
+  }
+  float4 w4 = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (has_g && a.norm_w) w4 = __ldg(reinterpret_cast<const float4*>(a.norm_w + 4 * c4));
+  __syncthreads();
 
   for (int t = 0; t < T_s; ++t) {
-    const size_t tok = (size_t)n * T_s + t;
-    if (tid < DK) {
-      sq[tid] = qn;
-      sk[tid] = kn;
+    const int par = t & 1;
+    const float* sq = tq + t * DK;
+    const float* sk = tk + t * DK;
+    const float alpha = __expf(tla[t]);
+    const float beta = tb[t];
+    // norms and k.q, computed by every warp (no barrier)
+    float nq = 0.f, nk = 0.f, kq = 0.f;
+    for (int i = lane; i < DK; i += 32) {
+      nq += sq[i] * sq[i];
+      nk += sk[i] * sk[i];
+      kq += sk[i] * sq[i];
     }
-    const float4 v4 = vn, g4 = gn;
-    const float alpha = __expf(lan), beta = bn;
-    if (t + 1 < T_s) fetch_token(t + 1);
-    __syncthreads();
-    if (tid < 32) {
-      float nq = 0.f, nk = 0.f, kq = 0.f;
-      for (int i = tid; i < DK; i += 32) {
-        nq += sq[i] * sq[i];
-        nk += sk[i] * sk[i];
-        kq += sk[i] * sq[i];
-      }
-      nq = warp_sum(nq);
-      nk = warp_sum(nk);
-      kq = warp_sum(kq);
-      if (tid == 0) {
-        const float rq = a.l2norm ? rsqrtf(nq + a.eps_l2) : 1.f;
-        const float rk = a.l2norm ? rsqrtf(nk + a.eps_l2) : 1.f;
-        snorm[0] = rq;
-        snorm[1] = rk;
-        snorm[2] = kq * rq * rk;
-      }
-    }
-    __syncthreads();
-    const float rq = snorm[0], rk = snorm[1], kq = snorm[2];
+    nq = warp_sum(nq);
+    nk = warp_sum(nk);
+    kq = warp_sum(kq);
+    const float rq = a.l2norm ? rsqrtf(nq + a.eps_l2) : 1.f;
+    const float rk = a.l2norm ? rsqrtf(nk + a.eps_l2) : 1.f;
+    kq = kq * rq * rk;  // the same association as the single-token kernel
 
     // a = S^T k^, b = S^T q^ over this thread's rows, then across row groups
     float4 pa = make_float4(0.f, 0.f, 0.f, 0.f), pb = pa;
@@ -241,16 +243,17 @@ __global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT)
       pa.x += s[r].x * ki; pa.y += s[r].y * ki; pa.z += s[r].z * ki; pa.w += s[r].w * ki;
       pb.x += s[r].x * qi; pb.y += s[r].y * qi; pb.z += s[r].z * qi; pb.w += s[r].w * qi;
     }
-    red_a[rg][c4] = pa;
-    red_b[rg][c4] = pb;
-    __syncthreads();
-    float4 ta = make_float4(0.f, 0.f, 0.f, 0.f), tb = ta;
+    red_a[par][rg][c4] = pa;
+    red_b[par][rg][c4] = pb;
+    __syncthreads();  // (the other parity's buffers were read before this barrier)
+    float4 ta = make_float4(0.f, 0.f, 0.f, 0.f), tbv = ta;
 #pragma unroll
     for (int g2 = 0; g2 < ROWG; ++g2) {
-      const float4 x = red_a[g2][c4], z = red_b[g2][c4];
+      const float4 x = red_a[par][g2][c4], z = red_b[par][g2][c4];
       ta.x += x.x; ta.y += x.y; ta.z += x.z; ta.w += x.w;
-      tb.x += z.x; tb.y += z.y; tb.z += z.z; tb.w += z.w;
+      tbv.x += z.x; tbv.y += z.y; tbv.z += z.z; tbv.w += z.w;
     }
+    const float4 v4 = *reinterpret_cast<const float4*>(tv + t * DV + 4 * c4);
     float4 e;
     e.x = v4.x - alpha * ta.x; e.y = v4.y - alpha * ta.y;
     e.z = v4.z - alpha * ta.z; e.w = v4.w - alpha * ta.w;
@@ -274,17 +277,17 @@ __global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT)
     }
 
     // y = scale (alpha b + beta (k^.q^) e), then the optional epilogue
+    const size_t tok = (size_t)n * T_s + t;
     const float bkq = beta * kq;
     float4 y;
-    y.x = a.scale * (alpha * tb.x + bkq * e.x); y.y = a.scale * (alpha * tb.y + bkq * e.y);
-    y.z = a.scale * (alpha * tb.z + bkq * e.z); y.w = a.scale * (alpha * tb.w + bkq * e.w);
+    y.x = a.scale * (alpha * tbv.x + bkq * e.x); y.y = a.scale * (alpha * tbv.y + bkq * e.y);
+    y.z = a.scale * (alpha * tbv.z + bkq * e.z); y.w = a.scale * (alpha * tbv.w + bkq * e.w);
     const size_t yo = (tok * a.H_v + h) * DV + 4 * c4;
     if (has_g) {
       float ss = y.x * y.x + y.y * y.y + y.z * y.z + y.w * y.w;
       ss = group_sum<TPR>(ss);  // every row group holds the same y
       const float r = rsqrtf(ss / (float)DV + a.eps_norm);
-      float4 w4 = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (a.norm_w) w4 = __ldg(reinterpret_cast<const float4*>(a.norm_w + 4 * c4));
+      const float4 g4 = *reinterpret_cast<const float4*>(tg + t * DV + 4 * c4);
       y.x = y.x * r * (1.f + w4.x) * sigmoidf_(g4.x);
       y.y = y.y * r * (1.f + w4.y) * sigmoidf_(g4.y);
       y.z = y.z * r * (1.f + w4.z) * sigmoidf_(g4.z);
@@ -294,14 +297,36 @@ __global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT)
   }  // tokens
 }
 
+// Dynamic shared memory of the multi-token kernel for T_s tokens.
+template <int DK, int DV>
+size_t multi_smem_bytes(int T_s, bool has_g) {
+  return sizeof(float) * (size_t)T_s * (2 * DK + (has_g ? 2 : 1) * DV + 2);
+}
+
 template <int DK, int DV, typename Tin>
 gdn_status launch(const DecodeArgs& a, cudaStream_t stream) {
   const unsigned grid = (unsigned)a.N * (unsigned)a.H_v;
   const bool single = a.T_s == 1 && a.snapshots == nullptr && a.state_out == a.state_in;
   if (single)
     gdn_decode_kernel<DK, DV, Tin><<<grid, DecodeGeom<DK, DV>::NT, 0, stream>>>(a);
-  else
-    gdn_decode_multi_kernel<DK, DV, Tin><<<grid, DecodeGeom<DK, DV>::NT, 0, stream>>>(a);
+  else {
+    const size_t smem = multi_smem_bytes<DK, DV>(a.T_s, a.g != nullptr);
+    if (smem > 48 * 1024) {
+      // more than the default allowance: opt in (per device, once)
+      static bool opted[64] = {false};
+      int dev = 0;
+      if (cudaGetDevice(&dev) != cudaSuccess) return GDN_ERR_CUDA;
+      if (dev < 0 || dev >= 64 || !opted[dev]) {
+        if (cudaFuncSetAttribute(gdn_decode_multi_kernel<DK, DV, Tin>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)multi_smem_bytes<DK, DV>(kMaxDecodeTokens, true)) !=
+            cudaSuccess)
+          return GDN_ERR_CUDA;
+        if (dev >= 0 && dev < 64) opted[dev] = true;
+      }
+    }
+    gdn_decode_multi_kernel<DK, DV, Tin><<<grid, DecodeGeom<DK, DV>::NT, smem, stream>>>(a);
+  }
   return cudaPeekAtLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 

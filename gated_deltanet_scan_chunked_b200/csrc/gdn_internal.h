@@ -41,6 +41,10 @@ struct PrefillArgs {
   unsigned long long* ring_flags = nullptr;
 };
 
+// Tokens per launch of the multi-token decode (its inputs are staged in
+// shared memory: ~4.1 KB per token at d_k = d_v = 128).
+constexpr int kMaxDecodeTokens = 32;
+
 struct DecodeArgs {
   const void* q;           // [N, T_s, H_qk, d_k]
   const void* k;

@@ -239,7 +239,8 @@ gdn_status gdn_decode_step(
  *               state after token t of every sequence (each one a valid
  *               state tensor); must not overlap state_in or state_out
  *   y           [N, T_s, H_v, d_v] in_dtype, written
- * Other arguments as for gdn_chunk_fwd.  N = 0 or T_s = 0 is a no-op.
+ * Other arguments as for gdn_chunk_fwd.  N = 0 or T_s = 0 is a no-op;
+ * T_s > 32 is GDN_ERR_UNSUPPORTED (the tokens' inputs are staged on chip).
  */
 gdn_status gdn_decode_multi(
     const void* q, const void* k, const void* v, const float* log_alpha,

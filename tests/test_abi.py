@@ -167,6 +167,7 @@ STATE_BYTES = 4 * 48 * 128 * 128 * 4
     (dict(so=FAKE + STATE_BYTES, sn=FAKE + 4096), gdn.GDN_ERR_INVALID_ARG),  # snapshots overlap
     (dict(sn=FAKE + 8), gdn.GDN_ERR_INVALID_ARG),                      # misaligned
     (dict(dk=48), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(T=33), gdn.GDN_ERR_UNSUPPORTED),                             # over 32 tokens
     (dict(T=0, q=None), gdn.GDN_OK),                                   # no-op
     (dict(N=0, y=None), gdn.GDN_OK),
 ])

@@ -128,3 +128,32 @@ def test_multi_full_batch_sampled():
         y_ref, s_ref = _oracle(d, int(n), heads, 4)
         assert_close(y[n][:, heads], y_ref, torch.bfloat16, "y seq %d" % n)
         assert_close(state[n][heads], s_ref[0], torch.bfloat16, "state seq %d" % n)
+
+
+@pytest.mark.parametrize("T_s", [1, 7, 32])
+def test_multi_token_counts(T_s):
+    """1 token (the loop kernel with a separate output state), an odd count,
+    and the maximum of 32 tokens, against single steps."""
+    d = inputs.make_decode(N=3, steps=T_s, epilogue=True, seed=46 + T_s)
+    ys1, states1 = _single_steps(d, T_s)
+    m = _multi_inputs(d)
+    s_in = d.state.clone().cuda()
+    s_out = torch.empty_like(s_in)
+    y, _ = gdn_decode_multi(m["q"], m["k"], m["v"], m["log_alpha"], m["beta"], s_in,
+                            state_out=s_out, g=m["g"], norm_w=m["norm_w"])
+    torch.cuda.synchronize()
+    assert gdn.gdn_check_device_error() == gdn.GDN_OK
+    assert torch.equal(y, ys1) and torch.equal(s_out, states1[-1])
+
+
+@pytest.mark.parametrize("dk,dv", [(16, 16), (128, 16), (16, 128), (64, 32)])
+def test_multi_other_head_dims_fp32(dk, dv):
+    d = inputs.make_decode(N=3, steps=5, H_qk=2, H_v=4, d_k=dk, d_v=dv, dtype=torch.float32,
+                           epilogue=True, seed=dk + dv)
+    ys1, states1 = _single_steps(d, 5)
+    m = _multi_inputs(d)
+    state = d.state.clone().cuda()
+    y, _ = gdn_decode_multi(m["q"], m["k"], m["v"], m["log_alpha"], m["beta"], state,
+                            g=m["g"], norm_w=m["norm_w"])
+    torch.cuda.synchronize()
+    assert torch.equal(y, ys1) and torch.equal(state, states1[-1])
