@@ -1,5 +1,5 @@
 // Chunked prefill of the gated delta rule on the sm_100a tensor cores
-// (tcgen05 MMA from shared-memory operands into TMEM accumulators), for bf16
+// (tcgen05 MMA from shared-memory and TMEM operands into TMEM accumulators), for bf16
 // inputs with d_k = d_v = 128.
 //
 // The recurrence ("Qwen3.8-Flash-Next: architecture, efficiency and technical
@@ -16,15 +16,17 @@
 //   S  <- gamma_C S + (diag(exp(G_C - G)) K^)^T Delta
 //
 // Every product is computed transposed so that the 128 TMEM lanes index d_v
-// (or d_k) and all MMAs are M = 128:
-//   MMA0  [K; Q] K^T   raw bf16 inputs, exact products; the L2-norm factors
-//                      are applied afterwards in fp32
-//   MMAW  W^T  = K^T (T diag(beta gamma))^T      (128 x 64)
-//   MMAU  U^T  = V^T (T diag(beta))^T            (128 x 64)
-//   MMA1  D^T  = U^T - S^T W^T                   (128 x 64, A negated)
-//   MMA2  Y^T  = S^T (diag(gamma) Q^)^T          (128 x 64)
-//   MMA3  S^T += D^T diag(exp(G_C - G)) K^       (128 x 128)
-//   MMA4  Y^T += D^T P^T                         (128 x 64)
+// (or d_k) and the state-side MMAs are M = 128:
+//   MMA0  [K; Q] K^T     raw bf16 inputs, exact products; the L2-norm factors
+//                        are applied afterwards in fp32
+//   MMAW  W = (T diag(beta gamma)) K^        (M = 64 tokens x N = 128), stored
+//                        negated and K-major beside gamma Q^
+//   MMA1  [Delta^T | Y^T] = S^T [-W; gamma Q^]^T   (one N = 128 product)
+//   MMAU  Delta^T += V^T (T diag(beta))^T  (= U^T)
+//   MMA3  S^T += Delta^T diag(exp(G_C - G)) K^     (128 x 128)
+//   MMA4  Y^T += Delta^T P^T
+// The fp16 copies of S^T and Delta^T that MMA1 / MMA3 / MMA4 read are written
+// straight into TMEM (tcgen05.st) and used as TMEM A operands.
 //
 // Precision.  The state S^T stays in TMEM in fp32 for the whole sequence.
 // MMA0 multiplies the raw bf16 q, k (exact, so q.k for near-orthogonal pairs
@@ -32,13 +34,16 @@
 // significand, 8x finer than bf16), with exact power-of-two scaling to stay
 // inside fp16 range: per chunk, an exponent e is chosen from the block maxima
 // of |V| and |S| and every value-like quantity (V, S, Delta, Y) enters the
-// tensor core multiplied by 2^-e; T enters as T 2^-f, f chosen from max |T|.
-// The fp32 TMEM state carries its own exponent; the scales are undone in the
-// fp32 epilogue and in the final state.
+// tensor core multiplied by 2^-e; T enters as T 2^-f, f chosen from max |T|,
+// and T diag(beta gamma) as an fp16 hi + lo pair (W is a cancellation when
+// keys repeat).  The fp32 TMEM state carries its own exponent; the scales are
+// undone in the fp32 epilogue and in the final state.
 //
-// One CTA (8 warps) per (sequence, value head).  Warps 0-3 and 4-7 reach the
-// same TMEM lanes (lane quarter = warp % 4) and split the columns.  Thread 0
-// issues the MMAs; completion is tracked with one mbarrier whose waits are
+// Layouts: one CTA (8 warps) per (sequence, value head) for large batches
+// (gdn_prefill_tc_kernel); for small batches a chain CTA plus preparation
+// CTAs per item (gdn_prefill_tc_pair_kernel, below).  Warps 0-3 and 4-7 reach
+// the same TMEM lanes (lane quarter = warp % 4) and split the columns.  One
+// thread issues the MMAs; completion is tracked with mbarriers whose waits are
 // bounded: a wait that runs out flags the device error word and the CTA
 // stops (after a second bounded wait for its own MMAs) without faulting.
 #include "gdn_common.cuh"
@@ -946,29 +951,36 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
 }
 
 // ============================================================================
-// CTA-pair variant: one 2-CTA cluster per (sequence, value head).  CTA 1
-// ("prep") does everything that does not depend on the state -- L2 norms,
-// [K; Q] K^T, A and P, the triangular inverse, W -- and ships the chain's
-// operand tiles (dec K^, gamma Q^, W^T, P, T diag(beta): 64 KB per chunk,
-// double-buffered) into CTA 0's shared memory with bulk copies
-// (shared::cta -> shared::cluster, no multicast).  CTA 0 ("chain") keeps the
-// state in TMEM and runs U, Delta, Y, the state update and the epilogue.
-// Buffer hand-off: "full" barriers in CTA 0 (arrive + expected bytes from
-// CTA 1, completed by the copies), "empty" barriers in CTA 1 (arrived by
-// CTA 0 once its MMAs have read the buffer), "staging free" barriers in
-// CTA 1 (arrived by CTA 0 once a copy has landed, so CTA 1 may overwrite the
-// copy's source).  Every wait is bounded.
+// Small-batch layouts: per (sequence, value head) item, a "chain" CTA and
+// NPREP "preparation" CTAs.  A preparation CTA does everything that does not
+// depend on the state -- L2 norms, [K; Q] K^T, A and P, the triangular
+// inverse, T diag(beta), and W (an M = 64 x N = 128 product, stored negated
+// and K-major beside gamma Q^) -- and ships the chain's operand tiles per
+// chunk: dec K^, [-W; gamma Q^], P and T diag(beta), 64 KB.  The chain CTA
+// keeps the state in TMEM, converts S^T and Delta^T to fp16 straight into
+// TMEM (MMA A operands), and runs [Delta | Y] = S^T [-W; gamma Q^]^T,
+// Delta += U, the state update, Y += Delta P^T and the epilogue.
 //
-// Split launch (kGlobal): the same two roles without a cluster.  One
-// cooperative launch holds items chain CTAs followed by NPREP preparation
-// CTAs per item, placed anywhere on the GPU (clusters of 3 cannot all be
-// placed at once on 148 SMs; single CTAs can).  The tiles travel through a
-// ring of kRing slots per item in a caller-provided global workspace, which
-// stays in L2: the preparation CTA bulk-stores its staging buffer into slot
-// (chunk % kRing) and publishes it with a release flag; the chain CTA
-// acquires the flag and bulk-loads the slot into its buffer, then returns
-// the slot with a second release flag.  Flags hold chunk index + 1 and start
-// at zero.
+// Cluster launch (kGlobal = false): one 2- or 3-CTA cluster per item; the
+// tiles go over distributed shared memory with bulk copies (shared::cta ->
+// shared::cluster, no multicast), double-buffered.  "full" barriers in the
+// chain CTA (arrive + expected bytes, completed by the copies), "empty"
+// barriers in the preparation CTA (arrived by the chain CTA once its MMAs
+// have read a buffer), "staging free" barriers in the preparation CTA
+// (arrived once a copy has landed, so its source may be overwritten).
+//
+// Split launch (kGlobal = true, needs a caller workspace): the same roles
+// without a cluster, in one cooperative launch of items chain CTAs followed
+// by NPREP preparation CTAs per item, placed anywhere (clusters of 3 cannot
+// all be placed at once on 148 SMs; single CTAs can).  Per item a ring of
+// kRing slots in the workspace (L2-resident) carries the tiles plus the
+// chunk's gate factors (1 + w) sigmoid(g), 80 KB: the preparation CTA
+// bulk-stores them (shared::cta -> global) and, once the stores are
+// complete, publishes the slot with a release flag; a non-MMA thread of the
+// chain CTA acquires the flag and bulk-loads the slot into shared memory a
+// chunk ahead, then returns the slot with a relaxed flag store once its bytes
+// have landed.  Flags hold chunk index + 1 and start at zero.  Every wait is
+// bounded.
 // ============================================================================
 
 // chain CTA (rank 0) shared memory
@@ -1263,15 +1275,11 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
           mma_f16(tbase + 128, da, db, ID_MK, 1);
         }
         mma_commit(mbar);
-        GDN_TRACE_POINT(43);
       }
-      GDN_TRACE_POINT(60);
       if constexpr (kGlobal) {
         // the next chunk's tiles, while the MMAs run
         if (tid == kFetcher && has_next) fetch(ci + 1, false);
       }
-      GDN_TRACE_POINT(61);
-      GDN_TRACE_POINT(70);
       if (!kGlobal && has_g && tid >= 64) {
         // Also while the MMAs run: this chunk's gate factors (1 + w)
         // sigmoid(g), in place as fp16 (g landed before the loop-top
@@ -1290,7 +1298,6 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
           st_shared_v4(addr, o[0], o[1], o[2], o[3]);
         }
       }
-      GDN_TRACE_POINT(71);
       okw = mbar_wait(mbar, phase, kWaitLimit);
       phase ^= 1;
       if (!__syncthreads_and(okw)) { ok = false; break; }

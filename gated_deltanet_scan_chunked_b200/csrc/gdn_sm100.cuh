@@ -27,12 +27,6 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-// Byte offset of element (row, col) of a swizzled bf16 tile whose panels hold
-// `rows` rows each.
-__device__ __forceinline__ uint32_t sw128_off(int row, int col, int rows) {
-  return (uint32_t)((col >> 6) * rows * 128 + row * 128 +
-                    ((((col & 63) >> 3) ^ (row & 7)) << 4) + ((col & 7) << 1));
-}
 
 // Byte offset of the 16-byte chunk holding columns [8c, 8c+8) of `row`.
 __device__ __forceinline__ uint32_t sw128_chunk(int row, int chunk, int rows) {
@@ -225,22 +219,6 @@ __device__ __forceinline__ void mbar_remote_arrive(uint32_t cl_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cl_addr)
                : "memory");
 }
-// 16-byte store into another CTA's shared memory (cluster address).
-__device__ __forceinline__ void st_cluster_v4(uint32_t cl_addr, uint32_t a, uint32_t b, uint32_t c,
-                                              uint32_t d) {
-  asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(cl_addr), "r"(a), "r"(b),
-               "r"(c), "r"(d)
-               : "memory");
-}
-__device__ __forceinline__ void st_cluster_f32(uint32_t cl_addr, float x) {
-  asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(cl_addr), "r"(__float_as_uint(x))
-               : "memory");
-}
-// Order this thread's generic writes to cluster shared memory before later
-// tensor-core (async proxy) reads of it.
-__device__ __forceinline__ void fence_proxy_async_cluster() {
-  asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
-}
 // Bulk copy of `bytes` (multiple of 16) from this CTA's shared memory into
 // another CTA's shared memory; completion is counted on that CTA's barrier.
 __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cl, uint32_t src_cta,
@@ -283,31 +261,6 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
   return false;
 }
 
-// Named barrier over `nthreads` threads (a multiple of 32), id 1..15.
-__device__ __forceinline__ void named_sync(uint32_t id, uint32_t nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-// Named barrier that also ANDs a predicate over the participating threads.
-__device__ __forceinline__ bool named_sync_and(uint32_t id, uint32_t nthreads, bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, %2, %3, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}\n"
-      : "=r"(r)
-      : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
-      : "memory");
-  return r != 0;
-}
-__device__ __forceinline__ void cp_async_wait_le1() {
-  asm volatile("cp.async.wait_group 1;" ::: "memory");
-}
-// Local (this CTA) mbarrier arrive with release semantics.
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
 
 // ---- global <-> shared bulk copies and flags ----------------------------------
 // Bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned) from
@@ -428,9 +381,6 @@ __device__ __forceinline__ void st_shared_v4(uint32_t saddr, uint32_t a, uint32_
                : "memory");
 }
 
-__device__ __forceinline__ void st_shared_v2(uint32_t saddr, uint32_t a, uint32_t b) {
-  asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(saddr), "r"(a), "r"(b) : "memory");
-}
 
 }  // namespace sm100
 }  // namespace gdn
