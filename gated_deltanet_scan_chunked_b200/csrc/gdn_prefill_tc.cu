@@ -1018,16 +1018,19 @@ constexpr size_t kSlotBytes = kSlotLoad + 256;
 
 template <int NPREP, bool kGlobal>
 __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const PrefillArgs a) {
-  // chain CTA map: 2 ship buffers (the split launch also ships the gate
-  // factors: 80 KB each), V, the output staging tile, and (cluster launch
-  // only) two g buffers; then C_SCAL / C_RED / C_BAR at fixed offsets.
-  // TMEM (512 columns): S^T fp32 0-127, Delta^T 128-191, Y^T 192-255, and the
-  // fp16 MMA A operands S^T 2^-e (256-319) and Delta^T 2^-e (320-351).
-  constexpr uint32_t kShipStride = kGlobal ? kSlotLoad : kShipBytes;
+  // chain CTA map: 2 ship buffers (64 KB of tiles each), V, the output
+  // staging tile, and gate-factor buffers (cluster launch: 2 for g,
+  // converted in place; split launch: a ring of 3 that the slot loads fill
+  // directly); then C_SCAL / C_RED / C_BAR at fixed offsets.
+  // TMEM (512 columns): S^T fp32 0-127, [Delta^T | Y^T] 128-255, the fp16 MMA
+  // A operands S^T 2^-e (256-319) and Delta^T 2^-e (320-351), and (split
+  // launch) a second [Delta^T | Y^T] 384-511 for odd chunks: the split launch
+  // runs chunk c's epilogue during chunk c+1's MMAs.
+  constexpr uint32_t kShipStride = kShipBytes;
   constexpr uint32_t X_VT = C_SHIP + 2 * kShipStride;
   constexpr uint32_t X_DT = X_VT + 16384;  // output staging (16 KB)
   constexpr uint32_t X_GS = X_DT + 16384;
-  static_assert((kGlobal ? X_GS : X_GS + 32768) <= C_SCAL, "chain shared-memory map overlaps");
+  static_assert(X_GS + 3 * 16384 <= C_SCAL, "chain shared-memory map overlaps");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sb = (raw + 1023u) & ~1023u;
@@ -1116,8 +1119,10 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
     if constexpr (!kGlobal) cluster_sync();
     fence_after_sync();
     const uint32_t tbase = *tslot;
-    const uint32_t tS = tbase + lane_off, tD = tbase + lane_off + 128, tY = tbase + lane_off + 192;
+    const uint32_t tS = tbase + lane_off;
     const uint32_t tSA = tbase + lane_off + 256, tDA = tbase + lane_off + 320;
+    // TMEM column of chunk c's [Delta^T | Y^T]
+    auto dy_col = [](int c) -> uint32_t { return (kGlobal && (c & 1)) ? 384u : 128u; };
     // Split launch, thread kFetcher only (not the MMA issuer: its proxy
     // fence would wait for the MMAs in flight): issue the bulk load of chunk
     // c from its slot into buffer c & 1 (free: it held chunk c - 2, whose
@@ -1140,9 +1145,12 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
       const uint8_t* src = ring + (size_t)s * kSlotBytes;
       mbar_arrive_expect_tx(&full[bb], kSlotLoad + 16);
 #pragma unroll
-      for (int k = 0; k < 5; ++k)
+      for (int k = 0; k < 4; ++k)
         bulk_load_g2s(sb + C_SHIP + bb * kShipStride + 16384 * k, src + 16384 * k, 16384,
                       &full[bb]);
+      // gate factors into ring entry c % 3 (last read by the epilogue of
+      // chunk c - 3, which ran during chunk c - 2)
+      bulk_load_g2s(sb + X_GS + (c % 3) * 16384, src + kSlotGF, 16384, &full[bb]);
       bulk_load_g2s(sb + C_SCAL + 16 * bb, src + kSlotLoad, 16, &full[bb]);
       ++fetched;
       return true;
@@ -1168,6 +1176,76 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
     for (int j2 = 0; j2 < 8; ++j2)
       wv[j2] = 1.f + ((has_g && a.norm_w) ? __ldg(a.norm_w + (tid & 15) * 8 + j2) : 0.f);
 
+    // Epilogue of one chunk in two parts.  (A) Y^T from TMEM, scaled back,
+    // with the gate: per-token RMS over d_v and y rr staged as fp16, token-
+    // major; without: y staged as bf16.  (B) with the gate: 8 consecutive
+    // outputs of one token per piece times the gate factors (gfa), packed to
+    // bf16 and stored; without: the staged rows copied out.  Between (A) and
+    // (B), and after (B) before the next (A), the caller provides a barrier.
+    auto epi_a = [&](uint32_t ty, int ee) {
+      float v[32];
+      tmem_ld32(ty + half * 32, v);
+      tmem_wait_ld();
+      const float ys = ldexpf(a.scale, ee);
+#pragma unroll
+      for (int x = 0; x < 32; ++x) v[x] *= ys;
+      if (has_g) {
+        float s2[32];
+#pragma unroll
+        for (int x = 0; x < 32; ++x) s2[x] = v[x] * v[x];
+        rs_stage(s2, 16, lane);
+        rs_stage(s2, 8, lane);
+        rs_stage(s2, 4, lane);
+        rs_stage(s2, 2, lane);
+        rs_stage(s2, 1, lane);
+        sRed[(warp & 3) * 64 + half * 32 + lane] = s2[0];
+        __syncthreads();
+        if (tid < 64)
+          sRr[tid] = rsqrtf((sRed[tid] + sRed[64 + tid] + sRed[128 + tid] + sRed[192 + tid]) /
+                                (float)kD + a.eps_norm);
+        __syncthreads();
+        // y rr (|y rr| <= sqrt(d_v)) as fp16, token-major, into the staging tile
+        __half* yst = reinterpret_cast<__half*>(gb + X_DT) + half * 32 * kD + row;
+        const float4* rr4 = reinterpret_cast<const float4*>(sRr + half * 32);
+#pragma unroll
+        for (int x4 = 0; x4 < 8; ++x4) {
+          const float4 r = rr4[x4];
+          yst[(4 * x4 + 0) * kD] = __float2half_rn(v[4 * x4 + 0] * r.x);
+          yst[(4 * x4 + 1) * kD] = __float2half_rn(v[4 * x4 + 1] * r.y);
+          yst[(4 * x4 + 2) * kD] = __float2half_rn(v[4 * x4 + 2] * r.z);
+          yst[(4 * x4 + 3) * kD] = __float2half_rn(v[4 * x4 + 3] * r.w);
+        }
+      } else {
+        __nv_bfloat16* gs = reinterpret_cast<__nv_bfloat16*>(gb + X_DT);
+#pragma unroll
+        for (int x = 0; x < 32; ++x) gs[(half * 32 + x) * kD + row] = __float2bfloat16_rn(v[x]);
+      }
+    };
+    auto epi_b = [&](int64_t cc0, int nc, uint32_t gfa) {
+      const int ch = tid & 15;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int rr = (tid >> 4) + 16 * k;
+        if (rr < nc) {
+          uint4 val = ld_shared_v4(sb + X_DT + rr * 256 + ch * 16);
+          if (has_g) {
+            float yf[8], gf[8];
+            unpack_f16x8(val, yf);
+            unpack_f16x8(ld_shared_v4(gfa + rr * 256 + ch * 16), gf);
+            val = make_uint4(pack_bf16(yf[0] * gf[0], yf[1] * gf[1]),
+                             pack_bf16(yf[2] * gf[2], yf[3] * gf[3]),
+                             pack_bf16(yf[4] * gf[4], yf[5] * gf[5]),
+                             pack_bf16(yf[6] * gf[6], yf[7] * gf[7]));
+          }
+          *reinterpret_cast<uint4*>(Yg + ((size_t)(cc0 + rr) * a.H_v + h) * kD + ch * 8) = val;
+        }
+      }
+    };
+    // split launch: the previous chunk, whose epilogue runs in this chunk's
+    // MMA windows
+    int64_t p_c0 = 0;
+    int p_n = 0, p_e = 0;
+
     int ci = 0;
     for (int64_t c0 = t_begin; c0 < t_end; c0 += kC, ++ci) {
       const int n = (t_end - c0) < kC ? (int)(t_end - c0) : kC;
@@ -1175,9 +1253,9 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
       const int nn = has_next ? ((t_end - c0 - kC) < kC ? (int)(t_end - c0 - kC) : kC) : 0;
       const int b = ci & 1;
       const uint32_t ship = sb + C_SHIP + b * kShipStride;
-      // this chunk's gate factors: shipped (split launch) or computed here
-      // from g in place (cluster launch)
-      const uint32_t gsb = kGlobal ? ship + kSlotGF : sb + X_GS + b * 16384;
+      // this chunk's gate factors: shipped (split launch: ring entry ci % 3)
+      // or computed here from g in place (cluster launch: buffer b)
+      const uint32_t gsb = kGlobal ? sb + X_GS + (ci % 3) * 16384 : sb + X_GS + b * 16384;
       cp_async_wait_all();
       // the other g buffer was last read by the previous chunk's epilogue
       if (!kGlobal && has_next && has_g) ld.g(c0 + kC, nn, b ^ 1);
@@ -1266,19 +1344,21 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t db = sdesc(ship + SH_WQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-          mma_f16_ta(tbase + 128, tbase + 256 + kk * 8, db, ID_KK128, kk > 0);
+          mma_f16_ta(tbase + dy_col(ci), tbase + 256 + kk * 8, db, ID_KK128, kk > 0);
         }
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint64_t da = sdesc(sb + X_VT + kk * 2048, 8192, 1024);
           const uint64_t db = sdesc(ship + SH_TB + kk * 32, 16, 1024);
-          mma_f16(tbase + 128, da, db, ID_MK, 1);
+          mma_f16(tbase + dy_col(ci), da, db, ID_MK, 1);
         }
         mma_commit(mbar);
       }
       if constexpr (kGlobal) {
         // the next chunk's tiles, while the MMAs run
         if (tid == kFetcher && has_next) fetch(ci + 1, false);
+        // and part (A) of the previous chunk's epilogue
+        if (ci > 0) epi_a(tbase + lane_off + dy_col(ci - 1) + 64, p_e);
       }
       if (!kGlobal && has_g && tid >= 64) {
         // Also while the MMAs run: this chunk's gate factors (1 + w)
@@ -1309,7 +1389,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
       // Delta^T 2^-e -> fp16 A operand in TMEM (token pairs per column)
       {
         float v[32];
-        tmem_ld32(tD + half * 32, v);
+        tmem_ld32(tbase + lane_off + dy_col(ci) + half * 32, v);
         tmem_wait_ld();
         const float sf = ldexpf(1.f, f);
         uint32_t pk[16];
@@ -1333,9 +1413,13 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint64_t db = sdesc(ship + SH_P + kk * 32, 16, 1024);
-          mma_f16_ta(tbase + 192, tbase + 320 + kk * 8, db, ID_KK, 1);
+          mma_f16_ta(tbase + dy_col(ci) + 64, tbase + 320 + kk * 8, db, ID_KK, 1);
         }
         mma_commit(mbar);
+      }
+      if constexpr (kGlobal) {
+        // part (B) of the previous chunk's epilogue, while the MMAs run
+        if (ci > 0) epi_b(p_c0, p_n, sb + X_GS + ((ci - 1) % 3) * 16384);
       }
       okw = mbar_wait(mbar, phase, kWaitLimit);
       phase ^= 1;
@@ -1349,86 +1433,29 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
       }
       GDN_TRACE_POINT(5);
 
-      // epilogue: y = scale 2^e Y^T; with the gate, out = y rr (1 + w) sigmoid(g)
-      {
-        float v[32];
-        tmem_ld32(tY + half * 32, v);
-        tmem_wait_ld();
-        GDN_TRACE_POINT(50);
-        const float ys = ldexpf(a.scale, e);
-#pragma unroll
-        for (int x = 0; x < 32; ++x) v[x] *= ys;
-        if (has_g) {
-          float s2[32];
-#pragma unroll
-          for (int x = 0; x < 32; ++x) s2[x] = v[x] * v[x];
-          rs_stage(s2, 16, lane);
-          rs_stage(s2, 8, lane);
-          rs_stage(s2, 4, lane);
-          rs_stage(s2, 2, lane);
-          rs_stage(s2, 1, lane);
-          sRed[(warp & 3) * 64 + half * 32 + lane] = s2[0];
-          __syncthreads();
-          if (tid < 64)
-            sRr[tid] = rsqrtf((sRed[tid] + sRed[64 + tid] + sRed[128 + tid] + sRed[192 + tid]) /
-                                  (float)kD + a.eps_norm);
-          __syncthreads();
-          GDN_TRACE_POINT(51);
-          // y rr (|y rr| <= sqrt(d_v)) as fp16, token-major, into the staging
-          // tile
-          __half* yst = reinterpret_cast<__half*>(gb + X_DT) + half * 32 * kD + row;
-          const float4* rr4 = reinterpret_cast<const float4*>(sRr + half * 32);
-#pragma unroll
-          for (int x4 = 0; x4 < 8; ++x4) {
-            const float4 r = rr4[x4];
-            yst[(4 * x4 + 0) * kD] = __float2half_rn(v[4 * x4 + 0] * r.x);
-            yst[(4 * x4 + 1) * kD] = __float2half_rn(v[4 * x4 + 1] * r.y);
-            yst[(4 * x4 + 2) * kD] = __float2half_rn(v[4 * x4 + 2] * r.z);
-            yst[(4 * x4 + 3) * kD] = __float2half_rn(v[4 * x4 + 3] * r.w);
-          }
-          __syncthreads();
-          GDN_TRACE_POINT(52);
-          // 8 consecutive outputs of one token per piece: times the gate
-          // factors (this thread's own pieces), pack, store
-          const int ch = tid & 15;
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int rr = (tid >> 4) + 16 * k;
-            if (rr < n) {
-              float yf[8], gf[8];
-              unpack_f16x8(ld_shared_v4(sb + X_DT + rr * 256 + ch * 16), yf);
-              unpack_f16x8(ld_shared_v4(gsb + rr * 256 + ch * 16), gf);
-              uint32_t o[4];
-#pragma unroll
-              for (int q = 0; q < 4; ++q)
-                o[q] = pack_bf16(yf[2 * q] * gf[2 * q], yf[2 * q + 1] * gf[2 * q + 1]);
-              *reinterpret_cast<uint4*>(Yg + ((size_t)(c0 + rr) * a.H_v + h) * kD + ch * 8) =
-                  make_uint4(o[0], o[1], o[2], o[3]);
-            }
-          }
-        } else {
-          // no gate: y as bf16 through the staging tile, coalesced stores
-          __nv_bfloat16* gs = reinterpret_cast<__nv_bfloat16*>(gb + X_DT);
-#pragma unroll
-          for (int x = 0; x < 32; ++x) gs[(half * 32 + x) * kD + row] = __float2bfloat16_rn(v[x]);
-          __syncthreads();
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int idx = tid + kNT * k;
-            const int rr = idx >> 4, ch = idx & 15;
-            if (rr < n) {
-              const uint4 val = ld_shared_v4(sb + X_DT + rr * 256 + ch * 16);
-              *reinterpret_cast<uint4*>(Yg + ((size_t)(c0 + rr) * a.H_v + h) * kD + ch * 8) = val;
-            }
-          }
-        }
+      if constexpr (kGlobal) {
+        p_c0 = c0;
+        p_n = n;
+        p_e = e;
+      } else {
+        // epilogue now (its gate factors were converted in place, buffer b)
+        epi_a(tbase + lane_off + 128 + 64, e);
+        __syncthreads();
+        epi_b(c0, n, gsb);
         __syncthreads();  // staging reads done: g buffer and staging tile reusable
-        GDN_TRACE_POINT(53);
       }
       fence_before_sync();
       GDN_TRACE_POINT(6);
     }
     cp_async_wait_all();
+    if constexpr (kGlobal) {
+      // the last chunk's epilogue
+      if (ok && ci > 0) {
+        epi_a(tbase + lane_off + dy_col(ci - 1) + 64, p_e);
+        __syncthreads();
+        epi_b(p_c0, p_n, sb + X_GS + ((ci - 1) % 3) * 16384);
+      }
+    }
     if (ok) {
       if (a.final_state) {
         const float sc = ldexpf(1.f, s_exp);
