@@ -1545,7 +1545,12 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
       wv[j2] = 1.f + ((has_g && a.norm_w) ? __ldg(a.norm_w + (tid & 15) * 8 + j2) : 0.f);
     const __nv_bfloat16* Gh = static_cast<const __nv_bfloat16*>(a.g);
     uint4 graw[4];  // this thread's g pieces of the chunk (bf16 x 8)
-    // Split launch, thread 0: the slot whose bulk stores are in flight and
+    // Split launch: thread kShip (warp 2: it issues no MMAs -- a release or
+    // proxy fence on the MMA issuer waits for its MMAs -- and is idle in the
+    // windows used) does all the slot traffic: it issues the bulk stores,
+    // waits for them and publishes the slot.
+    constexpr int kShip = 64;
+    // Split launch, thread kShip: the slot whose bulk stores are in flight and
     // not yet published (published once complete, during the next chunk).
     int pend_slot = -1;
     unsigned long long pend_val = 0;
@@ -1558,7 +1563,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
         pend_slot = -1;
       }
     };
-    // Split launch, thread 0: a slot whose bulk stores are staged but not
+    // Split launch, thread kShip: a slot whose bulk stores are staged but not
     // yet issued.  They are issued right after the next loop-top barrier:
     // issued earlier, the loop-top proxy fence would wait for their reads.
     int iss_slot = -1, iss_lb = 0;
@@ -1599,7 +1604,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
       }
       if (!__syncthreads_and(okw)) { ok = false; break; }
       if constexpr (kGlobal) {
-        if (tid == 0) issue();  // the previous chunk's slot
+        if (tid == kShip) issue();  // the previous chunk's slot
       }
       GDN_TRACE_POINT(20);
 
@@ -1695,7 +1700,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
       // split launch: the last bulk store has finished reading its sources
       // before the A scratch (its gate-factor staging) is rewritten below
       if constexpr (kGlobal) {
-        if (tid == 0) bulk_wait_read_all();
+        if (tid == kShip) bulk_wait_read_all();
       }
       okw = mbar_wait(mbar, phase, kWaitLimit);
       phase ^= 1;
@@ -1803,9 +1808,11 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
           mma_f16(tbase, da, db, ID_W64, 1);
         }
         mma_commit(mbar);
+      }
+      if constexpr (kGlobal) {
         // the previous chunk's slot (its stores are long complete), while
         // the MMAs run; a first chunk is published as soon as it is stored
-        if constexpr (kGlobal) publish();
+        if (tid == kShip) publish();
       }
       if constexpr (kGlobal) {
         // this chunk's g rows (from L2) while the MMAs run
@@ -1870,7 +1877,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
         }
         if (!__syncthreads_and(okw)) { ok = false; break; }
         GDN_TRACE_POINT(30);
-        if (tid == 0) {
+        if (tid == kShip) {
           iss_slot = s;
           iss_lb = lb;
           iss_val = (unsigned long long)ci + 1;
@@ -1899,13 +1906,13 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
     }
     cp_async_wait_all();
     if constexpr (kGlobal) {
-      if (tid == 0 && ok) {
+      if (tid == kShip && ok) {
         publish();
         issue();
         publish();
       }
+      if (tid == kShip) bulk_wait_all();
     }
-    if (tid == 0) bulk_wait_all();
     if (!ok) {
       if (tid == 0) atomicOr(a.err, kErrTimeout);
       mbar_wait(mbar, phase ^ 1, kWaitLimit);
