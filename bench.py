@@ -231,10 +231,15 @@ def cpu_baseline(w, target_s=12.0):
     dt = run(T_cal)
     T_s = int(max(64, min(w.total_T, T_cal * target_s / max(dt, 1e-6))))
     T_s = min(T_s, int(w.cu_seqlens[1].item()))
-    dt = run(T_s)
-    return {"value": T_s / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+    # a sequence shorter than the target is run repeatedly (the oracle as it
+    # stands; each run is the same work) until about target_s has passed
+    reps, total = 0, 0.0
+    while reps == 0 or total < 0.5 * target_s:
+        total += run(T_s)
+        reps += 1
+    return {"value": reps * T_s / total, "unit": "tokens/s", "cores": cores, "kind": "oracle",
             "sample": "first %d tokens of sequence 0, all %d value heads, fp64, OpenMP over "
-                      "value heads (%.1f s)" % (T_s, w.v.shape[1], dt)}
+                      "value heads, %d run(s) (%.1f s)" % (T_s, w.v.shape[1], reps, total)}
 
 
 def _prefix(w, T):
