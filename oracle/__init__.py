@@ -17,7 +17,9 @@ stated at the top of ``gdn_oracle.c``:
   ("On the Design of Qwen3.8-Next Architecture ... close reading",
   section 4.1), used only to pin the error form;
 * the optional zero-centred RMSNorm x sigmoid(g) epilogue (section 03,
-  "what Qwen changed on the original GDN"; hyper.ai summary, "Method").
+  "what Qwen changed on the original GDN"; hyper.ai summary, "Method");
+* the backward of all of the above (the adjoint of the error-form recurrence,
+  differentiated by hand token by token in reverse order), for training.
 
 Parity pins for every function here are in ``tests/test_oracle_pins.py``.
 """
@@ -66,6 +68,13 @@ def _load():
         lib.gdn_oracle_product_form.argtypes = [
             _f64p, _f64p, _f64p, _f64p, _f64p, _f64p, ctypes.c_int64,
             ctypes.c_int, ctypes.c_int, _f64p, _f64p]
+        lib.gdn_oracle_backward.restype = ctypes.c_int
+        lib.gdn_oracle_backward.argtypes = [
+            _f32p, _f32p, _f32p, _f32p, _f32p, _f32p, _f32p, _f32p, _i64p,
+            ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+            ctypes.c_double, ctypes.c_double, _f32p, _f32p, _f64p, _f64p,
+            _f64p, _f64p, _f64p, _f64p, _f64p, _f64p, ctypes.c_int]
         lib.gdn_oracle_max_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -154,3 +163,53 @@ def product_form(q, k, v, alpha, beta, s0=None):
     if rc != 0:
         raise ValueError("oracle rejected its arguments")
     return y, s
+
+
+def backward(q, k, v, log_alpha, beta, dy, g=None, norm_w=None,
+             initial_state=None, d_final_state=None, cu_seqlens=None,
+             l2norm=True, eps_l2=1e-6, eps_norm=1e-6, scale=1.0, n_threads=0):
+    """Gradients of sum(dy * y) + sum(d_final_state * final_state) with
+    respect to every input of ``recurrence``, in fp64.
+
+    dy has the shape of y ([T, H_v, d_v]; the gradient after the epilogue when
+    g is given); d_final_state [n_seq, H_v, d_k, d_v] or None (zeros).  Inputs
+    are widened exactly to fp32 then fp64.  Returns a dict with dq, dk
+    [T, H_qk, d_k]; dv [T, H_v, d_v]; dlog_alpha, dbeta [T, H_v];
+    d_initial_state [n_seq, H_v, d_k, d_v]; and, when g is given, dg
+    [T, H_v, d_v] and dnorm_w [d_v].
+    """
+    lib = _load()
+    q = _as_np(q, np.float32)
+    k = _as_np(k, np.float32)
+    v = _as_np(v, np.float32)
+    la = _as_np(log_alpha, np.float32)
+    b = _as_np(beta, np.float32)
+    g = _as_np(g, np.float32)
+    w = _as_np(norm_w, np.float32)
+    s0 = _as_np(initial_state, np.float32)
+    dyy = _as_np(dy, np.float32)
+    dsT = _as_np(d_final_state, np.float32)
+    T, Hqk, dk = q.shape
+    Hv, dv = v.shape[1], v.shape[2]
+    cu = (np.array([0, T], dtype=np.int64) if cu_seqlens is None
+          else _as_np(cu_seqlens, np.int64))
+    n_seq = cu.shape[0] - 1
+    out = dict(dq=np.zeros((T, Hqk, dk)), dk=np.zeros((T, Hqk, dk)),
+               dv=np.zeros((T, Hv, dv)), dlog_alpha=np.zeros((T, Hv)),
+               dbeta=np.zeros((T, Hv)), d_initial_state=np.zeros((n_seq, Hv, dk, dv)))
+    if g is not None:
+        out["dg"] = np.zeros((T, Hv, dv))
+        out["dnorm_w"] = np.zeros(dv)
+    rc = lib.gdn_oracle_backward(
+        _ptr(q, _f32p), _ptr(k, _f32p), _ptr(v, _f32p), _ptr(la, _f32p),
+        _ptr(b, _f32p), _ptr(g, _f32p), _ptr(w, _f32p), _ptr(s0, _f32p),
+        _ptr(cu, _i64p), n_seq, T, Hqk, Hv, dk, dv, int(bool(l2norm)),
+        float(eps_l2), float(eps_norm), float(scale), _ptr(dyy, _f32p),
+        _ptr(dsT, _f32p), _ptr(out["dq"], _f64p), _ptr(out["dk"], _f64p),
+        _ptr(out["dv"], _f64p), _ptr(out["dlog_alpha"], _f64p),
+        _ptr(out["dbeta"], _f64p), _ptr(out.get("dg"), _f64p),
+        _ptr(out.get("dnorm_w"), _f64p), _ptr(out["d_initial_state"], _f64p),
+        int(n_threads))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    return out

@@ -242,6 +242,321 @@ int gdn_oracle_product_form(const double* q, const double* k, const double* v,
   return 0;
 }
 
+/*
+ * Backward of the error-form recurrence (the adjoint of run_pair), for one
+ * (sequence, value head) pair.  The forward result is differentiated by
+ * hand, step by step in reverse token order; for each token, with S' =
+ * alpha S_{t-1}, e = v - S'^T k, S_t = S' + beta k e^T, o = scale S_t^T q:
+ *
+ *     dS     += scale q do^T             dq   = scale S_t do
+ *     de      = beta dS^T k              dv   = de
+ *     dbeta   = k^T dS e                 dk   = beta dS e - S' de
+ *     dS'     = dS - k de^T              dlog alpha = <dS', S'>
+ *     dS_{t-1} = alpha dS'
+ *
+ * where dS is the gradient with respect to S_t.  With the epilogue
+ * y = n (1 + w) sigmoid(g), n = o / sqrt(mean o^2 + eps_norm), the gradient
+ * do comes from dy by the chain rule through the gate and the RMS norm.  The
+ * L2 norm of q and k is differentiated afterwards (by the caller), once the
+ * gradients of the value heads sharing a QK head are summed.
+ *
+ * States are recomputed from checkpoints taken every kCk tokens of the
+ * forward pass; the recomputation repeats the forward arithmetic exactly.
+ * dqh/dkh receive the gradients with respect to the normalised q and k of
+ * this value head, [total_T, H_v, d_k]; dw (may be NULL) receives this
+ * pair's share of the norm-weight gradient, [d_v].
+ */
+enum { kCk = 64 };
+
+static void l2_unit(const float* x, int n, int l2norm, double eps, double* xh) {
+  double s = 0.0;
+  for (int i = 0; i < n; ++i) {
+    xh[i] = (double)x[i];
+    s += xh[i] * xh[i];
+  }
+  if (l2norm) {
+    const double r = 1.0 / sqrt(s + eps);
+    for (int i = 0; i < n; ++i) xh[i] *= r;
+  }
+}
+
+static void step_state(const double* Sp, const double* kh, const float* vt,
+                       double alpha, double b, int dk, int dv, double* Sn,
+                       double* e) {
+  /* Sn = S' + b k e^T with S' = alpha Sp and e = v - S'^T k */
+  for (int i = 0; i < dk * dv; ++i) Sn[i] = alpha * Sp[i];
+  for (int j = 0; j < dv; ++j) e[j] = (double)vt[j];
+  for (int i = 0; i < dk; ++i)
+    for (int j = 0; j < dv; ++j) e[j] -= Sn[(size_t)i * dv + j] * kh[i];
+  for (int i = 0; i < dk; ++i)
+    for (int j = 0; j < dv; ++j) Sn[(size_t)i * dv + j] += b * kh[i] * e[j];
+}
+
+static int backward_pair(const float* q, const float* k, const float* v,
+                         const float* log_alpha, const float* beta,
+                         const float* g, const float* norm_w, const float* s0,
+                         const float* dy, const float* dsT, int64_t t0,
+                         int64_t t1, int h, int Hqk, int Hv, int dk, int dv,
+                         int l2norm, double eps_l2, double eps_norm,
+                         double scale, double* dqh, double* dkh, double* dv_out,
+                         double* dla, double* dbeta, double* dg, double* dw,
+                         double* ds0) {
+  const int group = Hv / Hqk;
+  const int hq = h / group;
+  const size_t SS = (size_t)dk * dv;
+  const int64_t T = t1 - t0;
+  const int64_t nck = (T + kCk - 1) / kCk;
+  double* ck = (double*)malloc(sizeof(double) * SS * (size_t)(nck > 0 ? nck : 1));
+  double* St = (double*)malloc(sizeof(double) * SS * (kCk + 1));
+  double* dS = (double*)malloc(sizeof(double) * SS);
+  double* Sp = (double*)malloc(sizeof(double) * SS);
+  double* kh = (double*)malloc(sizeof(double) * dk);
+  double* qh = (double*)malloc(sizeof(double) * dk);
+  double* e = (double*)malloc(sizeof(double) * dv);
+  double* o = (double*)malloc(sizeof(double) * dv);
+  double* dO = (double*)malloc(sizeof(double) * dv);
+  double* de = (double*)malloc(sizeof(double) * dv);
+  double* tmp = (double*)malloc(sizeof(double) * (dk > dv ? dk : dv));
+  int ok = ck && St && dS && Sp && kh && qh && e && o && dO && de && tmp;
+  if (ok) {
+    /* forward pass: the state entering every kCk-token block */
+    double* S = St;
+    if (s0) {
+      for (size_t i = 0; i < SS; ++i) S[i] = (double)s0[i];
+    } else {
+      memset(S, 0, sizeof(double) * SS);
+    }
+    for (int64_t t = t0; t < t1; ++t) {
+      if ((t - t0) % kCk == 0) memcpy(ck + SS * (size_t)((t - t0) / kCk), S, sizeof(double) * SS);
+      l2_unit(k + ((size_t)t * Hqk + hq) * dk, dk, l2norm, eps_l2, kh);
+      const double alpha = exp((double)log_alpha[(size_t)t * Hv + h]);
+      const double b = (double)beta[(size_t)t * Hv + h];
+      step_state(S, kh, v + ((size_t)t * Hv + h) * dv, alpha, b, dk, dv, Sp, e);
+      memcpy(S, Sp, sizeof(double) * SS);
+    }
+    /* reverse pass, one block at a time */
+    if (dsT) {
+      for (size_t i = 0; i < SS; ++i) dS[i] = (double)dsT[i];
+    } else {
+      memset(dS, 0, sizeof(double) * SS);
+    }
+    for (int64_t blk = nck - 1; blk >= 0; --blk) {
+      const int64_t b0 = t0 + blk * kCk;
+      const int64_t b1 = (b0 + kCk < t1) ? b0 + kCk : t1;
+      /* St[m] = state entering token b0 + m; St[b1 - b0] = state after the block */
+      memcpy(St, ck + SS * (size_t)blk, sizeof(double) * SS);
+      for (int64_t t = b0; t < b1; ++t) {
+        l2_unit(k + ((size_t)t * Hqk + hq) * dk, dk, l2norm, eps_l2, kh);
+        const double alpha = exp((double)log_alpha[(size_t)t * Hv + h]);
+        const double b = (double)beta[(size_t)t * Hv + h];
+        step_state(St + SS * (size_t)(t - b0), kh, v + ((size_t)t * Hv + h) * dv, alpha, b,
+                   dk, dv, St + SS * (size_t)(t - b0 + 1), e);
+      }
+      for (int64_t t = b1 - 1; t >= b0; --t) {
+        const double* Sprev = St + SS * (size_t)(t - b0);
+        const double* Snew = St + SS * (size_t)(t - b0 + 1);
+        l2_unit(k + ((size_t)t * Hqk + hq) * dk, dk, l2norm, eps_l2, kh);
+        l2_unit(q + ((size_t)t * Hqk + hq) * dk, dk, l2norm, eps_l2, qh);
+        const double alpha = exp((double)log_alpha[(size_t)t * Hv + h]);
+        const double b = (double)beta[(size_t)t * Hv + h];
+        const size_t row = (size_t)t * Hv + h;
+        /* S' and e of this token */
+        for (size_t i = 0; i < SS; ++i) Sp[i] = alpha * Sprev[i];
+        for (int j = 0; j < dv; ++j) e[j] = (double)v[row * dv + j];
+        for (int i = 0; i < dk; ++i)
+          for (int j = 0; j < dv; ++j) e[j] -= Sp[(size_t)i * dv + j] * kh[i];
+        /* o = scale S_t^T q, then do from dy */
+        for (int j = 0; j < dv; ++j) {
+          double acc = 0.0;
+          for (int i = 0; i < dk; ++i) acc += Snew[(size_t)i * dv + j] * qh[i];
+          o[j] = scale * acc;
+        }
+        const float* dyt = dy + row * dv;
+        if (g) {
+          const float* gt = g + row * dv;
+          double ms = 0.0;
+          for (int j = 0; j < dv; ++j) ms += o[j] * o[j];
+          const double r = 1.0 / sqrt(ms / (double)dv + eps_norm);
+          double dot = 0.0;
+          for (int j = 0; j < dv; ++j) {
+            const double w = norm_w ? (double)norm_w[j] : 0.0;
+            const double sg = 1.0 / (1.0 + exp(-(double)gt[j]));
+            const double n = o[j] * r;
+            const double dyj = (double)dyt[j];
+            dg[row * dv + j] = dyj * n * (1.0 + w) * sg * (1.0 - sg);
+            if (dw) dw[j] += dyj * n * sg;
+            dO[j] = dyj * (1.0 + w) * sg; /* gradient w.r.t. n */
+            dot += dO[j] * n;
+          }
+          dot /= (double)dv;
+          for (int j = 0; j < dv; ++j) dO[j] = r * (dO[j] - o[j] * r * dot);
+        } else {
+          for (int j = 0; j < dv; ++j) dO[j] = (double)dyt[j];
+        }
+        /* read-out: dq = scale S_t do, dS += scale q do^T */
+        for (int i = 0; i < dk; ++i) {
+          double acc = 0.0;
+          for (int j = 0; j < dv; ++j) acc += Snew[(size_t)i * dv + j] * dO[j];
+          dqh[row * dk + i] = scale * acc;
+        }
+        for (int i = 0; i < dk; ++i)
+          for (int j = 0; j < dv; ++j) dS[(size_t)i * dv + j] += scale * qh[i] * dO[j];
+        /* write: de = beta dS^T k, dbeta = k^T dS e, dk = beta dS e - S' de */
+        for (int j = 0; j < dv; ++j) {
+          double acc = 0.0;
+          for (int i = 0; i < dk; ++i) acc += dS[(size_t)i * dv + j] * kh[i];
+          de[j] = b * acc;
+          dv_out[row * dv + j] = de[j];
+        }
+        double db = 0.0;
+        for (int i = 0; i < dk; ++i) {
+          double dse = 0.0, spde = 0.0;
+          for (int j = 0; j < dv; ++j) {
+            dse += dS[(size_t)i * dv + j] * e[j];
+            spde += Sp[(size_t)i * dv + j] * de[j];
+          }
+          db += kh[i] * dse;
+          tmp[i] = b * dse - spde;
+        }
+        dbeta[row] = db;
+        for (int i = 0; i < dk; ++i) dkh[row * dk + i] = tmp[i];
+        /* dS' = dS - k de^T; dlog alpha = <dS', S'>; dS_{t-1} = alpha dS' */
+        double dl = 0.0;
+        for (int i = 0; i < dk; ++i)
+          for (int j = 0; j < dv; ++j) {
+            const size_t x = (size_t)i * dv + j;
+            dS[x] -= kh[i] * de[j];
+            dl += dS[x] * Sp[x];
+            dS[x] *= alpha;
+          }
+        dla[row] = dl;
+      }
+    }
+    memcpy(ds0, dS, sizeof(double) * SS);
+  }
+  free(ck);
+  free(St);
+  free(dS);
+  free(Sp);
+  free(kh);
+  free(qh);
+  free(e);
+  free(o);
+  free(dO);
+  free(de);
+  free(tmp);
+  return ok ? 0 : -1;
+}
+
+/*
+ * Backward over a packed batch.  Inputs as gdn_oracle_recurrence plus
+ * dy [total_T, H_v, d_v] (the gradient of the loss with respect to y, after
+ * the epilogue when g is given) and d_final_state [n_seq, H_v, d_k, d_v] (may
+ * be NULL = zeros).  Outputs, all fp64 and written in full:
+ *   dq, dk          [total_T, H_qk, d_k]  (through the L2 norm when l2norm)
+ *   dv              [total_T, H_v, d_v]
+ *   dlog_alpha, dbeta [total_T, H_v]
+ *   dg              [total_T, H_v, d_v]  (only when g is given; may be NULL)
+ *   dnorm_w         [d_v]                (only when g is given; may be NULL)
+ *   d_initial_state [n_seq, H_v, d_k, d_v]
+ * Returns 0 on success, -1 on a bad argument or an allocation failure.
+ */
+int gdn_oracle_backward(const float* q, const float* k, const float* v,
+                        const float* log_alpha, const float* beta,
+                        const float* g, const float* norm_w,
+                        const float* initial_state, const int64_t* cu_seqlens,
+                        int64_t n_seq, int64_t total_T, int Hqk, int Hv,
+                        int dk, int dv, int l2norm, double eps_l2,
+                        double eps_norm, double scale, const float* dy,
+                        const float* d_final_state, double* dq, double* dk_out,
+                        double* dv_out, double* dlog_alpha, double* dbeta,
+                        double* dg, double* dnorm_w, double* d_initial_state,
+                        int n_threads) {
+  if (!q || !k || !v || !log_alpha || !beta || !dy || !cu_seqlens) return -1;
+  if (!dq || !dk_out || !dv_out || !dlog_alpha || !dbeta || !d_initial_state) return -1;
+  if (g && !dg) return -1;
+  if (Hqk <= 0 || Hv <= 0 || Hv % Hqk != 0 || dk <= 0 || dv <= 0) return -1;
+  if (n_seq < 0 || cu_seqlens[0] != 0 || cu_seqlens[n_seq] != total_T) return -1;
+  for (int64_t s = 0; s < n_seq; ++s)
+    if (cu_seqlens[s + 1] < cu_seqlens[s]) return -1;
+  const int64_t pairs = n_seq * (int64_t)Hv;
+  const size_t nq = (size_t)total_T * Hv * dk;
+  double* dqh = (double*)calloc(nq ? nq : 1, sizeof(double));
+  double* dkh = (double*)calloc(nq ? nq : 1, sizeof(double));
+  double* dwp = (double*)calloc((size_t)(pairs ? pairs : 1) * dv, sizeof(double));
+  if (!dqh || !dkh || !dwp) {
+    free(dqh);
+    free(dkh);
+    free(dwp);
+    return -1;
+  }
+#ifdef _OPENMP
+  if (n_threads > 0) omp_set_num_threads(n_threads);
+#else
+  (void)n_threads;
+#endif
+  int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t p = 0; p < pairs; ++p) {
+    const int64_t s = p / Hv;
+    const int h = (int)(p % Hv);
+    const size_t st = ((size_t)s * Hv + h) * (size_t)dk * dv;
+    if (backward_pair(q, k, v, log_alpha, beta, g, norm_w,
+                      initial_state ? initial_state + st : NULL, dy,
+                      d_final_state ? d_final_state + st : NULL, cu_seqlens[s],
+                      cu_seqlens[s + 1], h, Hqk, Hv, dk, dv, l2norm, eps_l2,
+                      eps_norm, scale, dqh, dkh, dv_out, dlog_alpha, dbeta, dg,
+                      g ? dwp + (size_t)p * dv : NULL, d_initial_state + st) != 0) {
+#pragma omp atomic write
+      bad = 1;
+    }
+  }
+  if (!bad) {
+    /* sum the value heads of each QK group, then differentiate the L2 norm:
+       for x^ = x r, r = 1/sqrt(|x|^2 + eps): dx = r (dx^ - x^ (x^ . dx^)) */
+    const int group = Hv / Hqk;
+    double* xh = (double*)malloc(sizeof(double) * dk);
+    double* gq = (double*)malloc(sizeof(double) * dk);
+    if (!xh || !gq) bad = 1;
+    for (int64_t t = 0; t < total_T && !bad; ++t)
+      for (int hq = 0; hq < Hqk; ++hq)
+        for (int which = 0; which < 2; ++which) {
+          const float* x = (which ? k : q) + ((size_t)t * Hqk + hq) * dk;
+          const double* part = which ? dkh : dqh;
+          double* out = (which ? dk_out : dq) + ((size_t)t * Hqk + hq) * dk;
+          for (int i = 0; i < dk; ++i) gq[i] = 0.0;
+          for (int m = 0; m < group; ++m) {
+            const double* pr = part + ((size_t)t * Hv + (size_t)hq * group + m) * dk;
+            for (int i = 0; i < dk; ++i) gq[i] += pr[i];
+          }
+          if (l2norm) {
+            double ss = 0.0;
+            for (int i = 0; i < dk; ++i) ss += (double)x[i] * (double)x[i];
+            const double r = 1.0 / sqrt(ss + eps_l2);
+            double dot = 0.0;
+            for (int i = 0; i < dk; ++i) {
+              xh[i] = (double)x[i] * r;
+              dot += xh[i] * gq[i];
+            }
+            for (int i = 0; i < dk; ++i) out[i] = r * (gq[i] - xh[i] * dot);
+          } else {
+            for (int i = 0; i < dk; ++i) out[i] = gq[i];
+          }
+        }
+    free(xh);
+    free(gq);
+    if (g && dnorm_w) {
+      for (int j = 0; j < dv; ++j) dnorm_w[j] = 0.0;
+      for (int64_t p = 0; p < pairs; ++p)
+        for (int j = 0; j < dv; ++j) dnorm_w[j] += dwp[(size_t)p * dv + j];
+    }
+  }
+  free(dqh);
+  free(dkh);
+  free(dwp);
+  return bad ? -1 : 0;
+}
+
 /* Number of threads an OpenMP parallel region would use. */
 int gdn_oracle_max_threads(void) {
 #ifdef _OPENMP
