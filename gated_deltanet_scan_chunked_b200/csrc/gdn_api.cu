@@ -190,6 +190,56 @@ extern "C" gdn_status gdn_decode_step(const void* q, const void* k, const void* 
                           stream);
 }
 
+extern "C" size_t gdn_chunk_bwd_workspace_size(int32_t n_seq, int64_t total_T, int32_t H_qk,
+                                               int32_t H_v, int32_t d_k, int32_t d_v) {
+  if (!dim_ok(d_k) || !dim_ok(d_v) || H_qk < 1 || H_v % H_qk != 0) return 0;
+  return chunk_bwd_workspace_bytes(n_seq, total_T, H_qk, H_v, d_k, d_v);
+}
+
+extern "C" gdn_status gdn_chunk_bwd(
+    const void* q, const void* k, const void* v, const float* log_alpha, const float* beta,
+    const void* g, const float* norm_w, const float* initial_state, const int32_t* cu_seqlens,
+    int32_t n_seq, int64_t total_T, int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v,
+    gdn_dtype in_dtype, int32_t l2norm_qk, float eps_l2, float eps_norm, float scale,
+    const void* dy, const float* d_final_state, float* dq, float* dk, float* dv,
+    float* dlog_alpha, float* dbeta, float* dg, float* dnorm_w, float* d_initial_state,
+    void* workspace, size_t workspace_bytes, gdn_stream_t stream) {
+  gdn_status st = check_common(H_qk, H_v, d_k, d_v, in_dtype, eps_l2, eps_norm);
+  if (st != GDN_OK) return st;
+  if (n_seq < 1 || total_T < 0) return GDN_ERR_INVALID_ARG;
+  if (cu_seqlens == nullptr && n_seq != 1) return GDN_ERR_INVALID_ARG;
+  if ((int64_t)n_seq * H_v > 0x7fffffffLL) return GDN_ERR_INVALID_ARG;
+  if (total_T > 0 && (!q || !k || !v || !log_alpha || !beta || !dy || !dq || !dk || !dv ||
+                      !dlog_alpha || !dbeta))
+    return GDN_ERR_INVALID_ARG;
+  if ((g != nullptr) != (dg != nullptr) || (g == nullptr && dnorm_w != nullptr))
+    return GDN_ERR_INVALID_ARG;
+  const void* ptrs[] = {q,  k,  v,  log_alpha, beta,  g,  norm_w,  initial_state,  dy,
+                        d_final_state, dq, dk, dv, dlog_alpha, dbeta, dg, dnorm_w,
+                        d_initial_state};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
+  if (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return GDN_ERR_INVALID_ARG;
+  const size_t need = chunk_bwd_workspace_bytes(n_seq, total_T, H_qk, H_v, d_k, d_v);
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+      workspace_bytes < need)
+    return GDN_ERR_INVALID_ARG;
+  BwdArgs a;
+  a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
+  a.g = g; a.norm_w = g ? norm_w : nullptr;
+  a.initial_state = initial_state; a.cu_seqlens = cu_seqlens;
+  a.dy = dy; a.d_final_state = d_final_state;
+  a.dq = dq; a.dk = dk; a.dv = dv; a.dlog_alpha = dlog_alpha; a.dbeta = dbeta;
+  a.dg = dg; a.dnorm_w = dnorm_w; a.d_initial_state = d_initial_state;
+  a.n_seq = n_seq; a.total_T = total_T;
+  a.H_qk = H_qk; a.H_v = H_v; a.d_k = d_k; a.d_v = d_v; a.dtype = in_dtype;
+  a.l2norm = l2norm_qk ? 1 : 0; a.eps_l2 = eps_l2; a.eps_norm = eps_norm; a.scale = scale;
+  a.err = error_word_ptr();
+  if (a.err == nullptr) return GDN_ERR_CUDA;
+  chunk_bwd_workspace_layout(workspace, &a);
+  return launch_chunk_bwd(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
 extern "C" gdn_status gdn_check_device_error(gdn_stream_t stream) {
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return GDN_ERR_CUDA;

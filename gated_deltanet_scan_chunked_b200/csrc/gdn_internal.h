@@ -63,6 +63,45 @@ struct DecodeArgs {
   float eps_l2, eps_norm, scale;
 };
 
+struct BwdArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* log_alpha;
+  const float* beta;
+  const void* g;               // nullptr: no epilogue
+  const float* norm_w;         // nullptr: zeros
+  const float* initial_state;  // nullptr: zeros
+  const int32_t* cu_seqlens;   // nullptr: one sequence
+  const void* dy;              // [total_T, H_v, d_v], input dtype
+  const float* d_final_state;  // nullptr: zeros
+  float* dq;                   // [total_T, H_qk, d_k]
+  float* dk;
+  float* dv;                   // [total_T, H_v, d_v]
+  float* dlog_alpha;           // [total_T, H_v]
+  float* dbeta;
+  float* dg;                   // [total_T, H_v, d_v] (with g)
+  float* dnorm_w;              // [d_v] (with g) or nullptr
+  float* d_initial_state;      // [n_seq, H_v, d_k, d_v] or nullptr
+  int32_t n_seq;
+  int64_t total_T;
+  int32_t H_qk, H_v, d_k, d_v;
+  gdn_dtype dtype;
+  int32_t l2norm;
+  float eps_l2, eps_norm, scale;
+  int* err;
+  // workspace parts, placed by chunk_bwd_workspace_layout
+  void* chunks;
+  int32_t* seq_first;
+  float *S, *dS, *W, *UT, *D, *dD, *T, *KKE, *P, *dPE, *Bm, *G, *row, *dw, *dO, *dqh, *dkh,
+      *qh, *kh;
+};
+
+size_t chunk_bwd_workspace_bytes(int32_t n_seq, int64_t total_T, int32_t H_qk, int32_t H_v,
+                                 int32_t d_k, int32_t d_v);
+void chunk_bwd_workspace_layout(void* ws, BwdArgs* a);
+gdn_status launch_chunk_bwd(const BwdArgs& a, cudaStream_t stream);
+
 // Each launcher returns GDN_OK, GDN_ERR_UNSUPPORTED (shape not compiled) or
 // GDN_ERR_CUDA (launch failed).
 gdn_status launch_decode(const DecodeArgs& a, cudaStream_t stream);

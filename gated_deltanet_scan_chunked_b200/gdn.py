@@ -74,6 +74,14 @@ def load(path: str = LIB_PATH):
     f.restype = ctypes.c_int
     f.argtypes = [_vp] * 10 + [ctypes.c_int32] * 7 + [
         ctypes.c_int32, ctypes.c_float, ctypes.c_float, ctypes.c_float, _vp, _vp]
+    f = lib.gdn_chunk_bwd_workspace_size
+    f.restype = ctypes.c_size_t
+    f.argtypes = [ctypes.c_int32, ctypes.c_int64] + [ctypes.c_int32] * 4
+    f = lib.gdn_chunk_bwd
+    f.restype = ctypes.c_int
+    f.argtypes = [_vp] * 9 + [ctypes.c_int32, ctypes.c_int64] + [ctypes.c_int32] * 5 + [
+        ctypes.c_int32, ctypes.c_float, ctypes.c_float, ctypes.c_float] + [_vp] * 10 + [
+        _vp, ctypes.c_size_t, _vp]
     lib.gdn_check_device_error.restype = ctypes.c_int
     lib.gdn_check_device_error.argtypes = [_vp]
     lib.gdn_status_string.restype = ctypes.c_char_p
@@ -224,6 +232,66 @@ def gdn_chunk_fwd_static_ws(q, k, v, log_alpha, beta, g=None, norm_w=None,
     if st != GDN_OK:
         raise GdnError(st, "gdn_chunk_fwd_static_ws")
     return y, final_state
+
+
+def bwd_workspace_size(n_seq: int, total_T: int, H_qk: int, H_v: int, d_k: int,
+                       d_v: int) -> int:
+    """Bytes of workspace gdn_chunk_bwd needs (0: arguments it never accepts)."""
+    return int(load().gdn_chunk_bwd_workspace_size(n_seq, total_T, H_qk, H_v, d_k, d_v))
+
+
+def gdn_chunk_bwd(q, k, v, log_alpha, beta, dy, g=None, norm_w=None,
+                  initial_state=None, d_final_state=None, cu_seqlens=None,
+                  l2norm_qk=True, eps_l2=1e-6, eps_norm=1e-6, scale=1.0,
+                  want_d_initial_state=True, want_dnorm_w=True, workspace=None,
+                  stream=None) -> dict:
+    """Gradients of a gdn_chunk_fwd call with the same inputs.
+
+    dy [T, H_v, d_v] (dtype of q): gradient with respect to y; d_final_state
+    [n_seq, H_v, d_k, d_v] fp32 or None.  Returns a dict of fp32 tensors: dq,
+    dk [T, H_qk, d_k]; dv [T, H_v, d_v]; dlog_alpha, dbeta [T, H_v]; and
+    d_initial_state [n_seq, H_v, d_k, d_v], dg [T, H_v, d_v], dnorm_w [d_v]
+    when asked for / when g is given.  ``workspace``: a uint8 CUDA tensor of
+    at least ``bwd_workspace_size(...)`` bytes, or None (allocated here
+    through torch).
+    """
+    lib = load()
+    dev = q.device
+    dt = _dtype_code(q)
+    T, Hqk, dk = q.shape
+    Hv, dv = v.shape[1], v.shape[2]
+    n_seq = 1 if cu_seqlens is None else int(cu_seqlens.shape[0]) - 1
+    for name, t in (("q", q), ("k", k), ("v", v), ("g", g), ("dy", dy)):
+        _check(t, name, q.dtype, dev)
+    for name, t in (("log_alpha", log_alpha), ("beta", beta), ("norm_w", norm_w),
+                    ("initial_state", initial_state), ("d_final_state", d_final_state)):
+        _check(t, name, torch.float32, dev)
+    _check(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    out = dict(dq=torch.empty((T, Hqk, dk), **f32), dk=torch.empty((T, Hqk, dk), **f32),
+               dv=torch.empty((T, Hv, dv), **f32), dlog_alpha=torch.empty((T, Hv), **f32),
+               dbeta=torch.empty((T, Hv), **f32))
+    if want_d_initial_state:
+        out["d_initial_state"] = torch.empty((n_seq, Hv, dk, dv), **f32)
+    if g is not None:
+        out["dg"] = torch.empty((T, Hv, dv), **f32)
+        if want_dnorm_w:
+            out["dnorm_w"] = torch.empty((dv,), **f32)
+    nbytes = int(lib.gdn_chunk_bwd_workspace_size(n_seq, T, Hqk, Hv, dk, dv))
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
+    _check(workspace, "workspace", torch.uint8, dev)
+    st = lib.gdn_chunk_bwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(g), _ptr(norm_w),
+        _ptr(initial_state), _ptr(cu_seqlens), n_seq, T, Hqk, Hv, dk, dv, dt,
+        1 if l2norm_qk else 0, float(eps_l2), float(eps_norm), float(scale), _ptr(dy),
+        _ptr(d_final_state), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
+        _ptr(out["dlog_alpha"]), _ptr(out["dbeta"]), _ptr(out.get("dg")),
+        _ptr(out.get("dnorm_w")), _ptr(out.get("d_initial_state")), _ptr(workspace),
+        workspace.numel(), _stream_handle(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_chunk_bwd")
+    return out
 
 
 def gdn_decode_step(q, k, v, log_alpha, beta, state, g=None, norm_w=None,

@@ -140,6 +140,20 @@ def make_prefill(lengths, H_qk, H_v, d_k, d_v, dtype=torch.bfloat16, seed=0,
                          meta={"lengths": lengths, "seed": int(seed)})
 
 
+def make_cotangents(w: PrefillInputs, seed=0, ds_std=0.5, final_grad=True):
+    """Seeded gradients for a backward pass over the prefill inputs ``w``:
+    dy ~ N(0, 1) in the dtype of q (shape of y) and, if ``final_grad``,
+    d_final_state ~ N(0, ds_std^2) fp32 [n_seq, H_v, d_k, d_v]."""
+    gen = _gen(int(seed) + 99, w.q.device)
+    T, Hv, dv = w.v.shape
+    dk = w.q.shape[2]
+    dy = _normal(gen, (T, Hv, dv), w.q.dtype)
+    dsT = None
+    if final_grad:
+        dsT = _normal(gen, (w.cu_seqlens.shape[0] - 1, Hv, dk, dv), torch.float32, std=ds_std)
+    return dy, dsT
+
+
 def varlen_lengths(n_seq=24, lo=512, hi=16384, seed=SEEDS["varlen"]):
     """Sequence lengths drawn uniformly from the integers [lo, hi]."""
     gen = torch.Generator().manual_seed(int(seed) + 7)

@@ -251,6 +251,63 @@ gdn_status gdn_decode_multi(
     float scale, void* y, gdn_stream_t stream);
 
 /*
+ * gdn_chunk_bwd_workspace_size -- bytes of device workspace gdn_chunk_bwd
+ * needs for a packed batch (0 for arguments it can never accept).  About
+ * 460 KB per 64-token chunk per value head at d_k = d_v = 128 (chunk states
+ * and their gradients, per-chunk matrices) plus 1.1 KB per token per value
+ * head; e.g. 1.45 GB for one 4,096-token sequence with 48 value heads.
+ */
+size_t gdn_chunk_bwd_workspace_size(int32_t n_seq, int64_t total_T, int32_t H_qk,
+                                    int32_t H_v, int32_t d_k, int32_t d_v);
+
+/*
+ * gdn_chunk_bwd -- gradients of a gdn_chunk_fwd call, for training.
+ *
+ * Differentiates the forward of gdn_chunk_fwd (the recurrence of
+ * "Qwen3.8-Flash-Next: architecture, efficiency and technical lineage",
+ * section 03 "Gated DeltaNet", update equations, with the optional RMSNorm x
+ * sigmoid(g) epilogue of the same section) given the gradient of the loss
+ * with respect to its outputs.  The pages describe no backward; this is the
+ * exact derivative of the forward, evaluated chunkwise (C = 64) on CUDA
+ * cores in fp32.  Nothing of the forward call is needed: the chunk states
+ * are recomputed from the inputs.
+ *
+ * Inputs: every forward input, with the same meaning, shapes, dtypes and
+ * defaults as for gdn_chunk_fwd (g and norm_w select the epilogue), plus
+ *   dy              [total_T, H_v, d_v] in_dtype: dLoss/dy (y after the
+ *                   epilogue when g is given)
+ *   d_final_state   [n_seq, H_v, d_k, d_v] fp32 or NULL (zeros)
+ * Outputs (fp32, caller-owned, fully overwritten):
+ *   dq, dk          [total_T, H_qk, d_k]  (through the in-kernel L2 norm
+ *                   when l2norm_qk; summed over the value heads of a group)
+ *   dv              [total_T, H_v, d_v]
+ *   dlog_alpha      [total_T, H_v]
+ *   dbeta           [total_T, H_v]
+ *   dg              [total_T, H_v, d_v]; required when g is given, else
+ *                   must be NULL
+ *   dnorm_w         [d_v] or NULL (only with g; not written when NULL)
+ *   d_initial_state [n_seq, H_v, d_k, d_v] or NULL (not written)
+ *   workspace       device memory, 256-byte aligned, at least
+ *                   gdn_chunk_bwd_workspace_size(...) bytes; owned by the
+ *                   caller and not retained; calls that may overlap must not
+ *                   share one
+ * Every pointer 16-byte aligned; outputs must not overlap inputs or each
+ * other.  Errors as for gdn_chunk_fwd; a workspace that is missing, too
+ * small or misaligned is GDN_ERR_INVALID_ARG.  Asynchronous on `stream`;
+ * allocates nothing.
+ */
+gdn_status gdn_chunk_bwd(
+    const void* q, const void* k, const void* v, const float* log_alpha,
+    const float* beta, const void* g, const float* norm_w,
+    const float* initial_state, const int32_t* cu_seqlens, int32_t n_seq,
+    int64_t total_T, int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v,
+    gdn_dtype in_dtype, int32_t l2norm_qk, float eps_l2, float eps_norm,
+    float scale, const void* dy, const float* d_final_state, float* dq, float* dk,
+    float* dv, float* dlog_alpha, float* dbeta, float* dg, float* dnorm_w,
+    float* d_initial_state, void* workspace, size_t workspace_bytes,
+    gdn_stream_t stream);
+
+/*
  * gdn_check_device_error -- synchronise `stream`, then read and clear the
  * library's device-side error word on the current device.  Returns GDN_OK,
  * GDN_ERR_TIMEOUT (a kernel's bounded wait ran out and the kernel returned

@@ -17,7 +17,8 @@ def lib():
 
 def test_exports_every_declared_function(lib):
     names = gdn.header_functions()
-    assert set(names) >= {"gdn_chunk_fwd", "gdn_chunk_fwd_path", "gdn_chunk_fwd_ws",
+    assert set(names) >= {"gdn_chunk_fwd", "gdn_chunk_fwd_path", "gdn_chunk_fwd_ws", "gdn_chunk_bwd",
+                          "gdn_chunk_bwd_workspace_size",
                           "gdn_chunk_fwd_workspace_size", "gdn_decode_step",
                           "gdn_check_device_error", "gdn_status_string", "gdn_version"}
     for n in names:
@@ -173,3 +174,45 @@ STATE_BYTES = 4 * 48 * 128 * 128 * 4
 ])
 def test_decode_multi_rejects_bad_arguments_on_host(lib, kw, code):
     assert _multi(lib, **kw) == code
+
+
+def _bwd(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, b=FAKE, g=None, w=None, s0=None, cu=None,
+             n_seq=1, T=64, Hqk=16, Hv=48, dk=128, dv=128, dt=0, dy=FAKE, dsT=None,
+             dq=FAKE, dkk=FAKE, dvv=FAKE, dla=FAKE, db=FAKE, dg=None, dw=None, ds0=None,
+             ws=FAKE, wsb=1 << 40)
+    a.update(kw)
+    return lib.gdn_chunk_bwd(a["q"], a["k"], a["v"], a["la"], a["b"], a["g"], a["w"], a["s0"],
+                             a["cu"], a["n_seq"], a["T"], a["Hqk"], a["Hv"], a["dk"], a["dv"],
+                             a["dt"], 1, 1e-6, 1e-6, 1.0, a["dy"], a["dsT"], a["dq"], a["dkk"],
+                             a["dvv"], a["dla"], a["db"], a["dg"], a["dw"], a["ds0"], a["ws"],
+                             a["wsb"], None)
+
+
+def test_bwd_workspace_size(lib):
+    """Backward workspace: grows with chunks x heads; 0 for unsupported dims."""
+    n1 = gdn.bwd_workspace_size(1, 4096, 16, 48, 128, 128)
+    assert 1.3e9 < n1 < 1.6e9
+    assert gdn.bwd_workspace_size(1, 8192, 16, 48, 128, 128) > 1.9 * n1
+    assert gdn.bwd_workspace_size(1, 64, 16, 48, 96, 128) == 0
+    assert gdn.bwd_workspace_size(1, 64, 16, 40, 128, 128) == 0
+    assert gdn.bwd_workspace_size(0, 64, 16, 48, 128, 128) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(ws=None), gdn.GDN_ERR_INVALID_ARG),                       # no workspace
+    (dict(ws=FAKE + 16), gdn.GDN_ERR_INVALID_ARG),                  # not 256-aligned
+    (dict(wsb=1000), gdn.GDN_ERR_INVALID_ARG),                      # too small
+    (dict(dy=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dq=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(g=FAKE), gdn.GDN_ERR_INVALID_ARG),                        # g without dg
+    (dict(dg=FAKE), gdn.GDN_ERR_INVALID_ARG),                       # dg without g
+    (dict(dw=FAKE), gdn.GDN_ERR_INVALID_ARG),                       # dnorm_w without g
+    (dict(dvv=FAKE + 4), gdn.GDN_ERR_INVALID_ARG),                  # misaligned
+    (dict(dk=48), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(dt=3), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(n_seq=2), gdn.GDN_ERR_INVALID_ARG),                       # needs cu_seqlens
+    (dict(Hv=40), gdn.GDN_ERR_INVALID_ARG),
+])
+def test_chunk_bwd_rejects_bad_arguments_on_host(lib, kw, code):
+    assert _bwd(lib, **kw) == code
