@@ -42,13 +42,19 @@
 //   dw_reduce    the norm weight's gradient, summed over chunks
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
+#include "gdn_sm100.cuh"
 
 namespace gdn {
 namespace {
 
+using sm100::cp_async16;
+using sm100::cp_async_commit;
+using sm100::cp_async_wait_all;
+using sm100::smem_u32;
+
 constexpr int kC = 64;    // chunk length
 constexpr int kNT = 256;  // threads per CTA; (ty, tx) = (tid / 16, tid % 16)
-constexpr int kLC = kC + 1;
+constexpr int kLC = kC + 4;  // padded row length of C x C tiles (16-byte rows)
 
 struct ChunkEnt {
   long long t0;  // first token
@@ -61,23 +67,31 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 int64_t max_chunks_of(int32_t n_seq, int64_t total_T) { return (total_T + kC - 1) / kC + n_seq; }
 
 // ---------------------------------------------------------------------------
-// Shared-memory tiles are row-major with one float of padding per row.
+// Shared-memory tiles are row-major, rows padded by 4 floats (16-byte rows).
 
-__device__ __forceinline__ void ld_rows(float* s, int ld, const float* g, size_t gstride, int rows,
+// rows x cols fp32 (cols % 4 == 0) from global rows of stride gstride floats
+// (16-byte aligned) into shared memory, asynchronously; rows >= valid are
+// zero-filled.  Completes at cp_async_wait_all() + __syncthreads().
+__device__ __forceinline__ void cp_tile(float* s, int ld, const float* g, size_t gstride, int rows,
                                         int valid, int cols) {
-  // rows x cols from global rows of stride gstride; rows >= valid are zero
-  for (int e = threadIdx.x; e < rows * cols; e += kNT) {
-    const int r = e / cols, c = e % cols;
-    s[r * ld + c] = r < valid ? g[(size_t)r * gstride + c] : 0.f;
+  const int c4 = cols / 4;
+  for (int e = threadIdx.x; e < rows * c4; e += kNT) {
+    const int r = e / c4, c = (e % c4) * 4;
+    const bool ok = r < valid;
+    cp_async16(smem_u32(s + r * ld + c), ok ? g + (size_t)r * gstride + c : g, ok);
   }
 }
 
+// The same for input-dtype rows (bf16 or fp32), converted to fp32; synchronous.
 template <typename Tin>
 __device__ __forceinline__ void ld_rows_in(float* s, int ld, const Tin* g, size_t gstride, int rows,
                                            int valid, int cols) {
-  for (int e = threadIdx.x; e < rows * cols; e += kNT) {
-    const int r = e / cols, c = e % cols;
-    s[r * ld + c] = r < valid ? Elem<Tin>::load(g + (size_t)r * gstride + c) : 0.f;
+  const int c4 = cols / 4;
+  for (int e = threadIdx.x; e < rows * c4; e += kNT) {
+    const int r = e / c4, c = (e % c4) * 4;
+    const float4 x = r < valid ? Elem<Tin>::load4(g + (size_t)r * gstride + c)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+    *reinterpret_cast<float4*>(s + r * ld + c) = x;
   }
 }
 
@@ -172,17 +186,18 @@ __global__ void __launch_bounds__(kNT) bwd_normalise_kernel(const BwdArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// prep: per (chunk, value head).
+// prep: per (chunk, value head).  Two CTAs per SM.
 
 template <int DK, int DV>
 struct PrepSmem {
-  static constexpr int LK = DK + 1, LV = DV + 1;
-  static constexpr int oK = 0, oQ = oK + kC * LK, oV = oQ + kC * LK, oA = oV + kC * LV,
-                       oT = oA + kC * kLC, oG = oT + kC * kLC, oB = oG + kC, total = oB + kC;
+  static constexpr int LK = DK + 4, LQV = (DK > DV ? DK : DV) + 4;
+  static constexpr int oK = 0, oQV = oK + kC * LK, oA = oQV + kC * LQV, oT = oA + kC * kLC,
+                       oG = oT + kC * kLC, oB = oG + kC, total = oB + kC;
   static constexpr size_t bytes = sizeof(float) * total;
 };
 
-// Inclusive cumsum of log alpha and beta over one chunk into sG / sB (warp 0).
+// Inclusive cumsum of log alpha over one chunk into sG, beta into sB (warp 0;
+// rows >= n get log alpha = 0, beta = 0).
 __device__ __forceinline__ void load_gates(const BwdArgs& a, const ChunkEnt& e, int h, float* sG,
                                            float* sB) {
   const int lane = threadIdx.x & 31;
@@ -198,28 +213,30 @@ __device__ __forceinline__ void load_gates(const BwdArgs& a, const ChunkEnt& e, 
       if (lane >= o) x += u;
     }
     sG[r] = x + carry;
-    if (sB) sB[r] = b;
+    sB[r] = b;
     carry += __shfl_sync(0xffffffffu, x, 31);
   }
 }
 
 template <int DK, int DV, typename Tin>
-__global__ void __launch_bounds__(kNT, 1) bwd_prep_kernel(const BwdArgs a) {
+__global__ void __launch_bounds__(kNT, 2) bwd_prep_kernel(const BwdArgs a) {
   using L = PrepSmem<DK, DV>;
-  extern __shared__ float smem[];
+  constexpr int NK = DK / 16, NV = DV / 16;
+  extern __shared__ __align__(16) float smem[];
   const ChunkEnt* e;
   if (!chunk_of(a, &e)) return;
   const int h = blockIdx.y, hq = h / (a.H_v / a.H_qk);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, ty = tid / 16, tx = tid % 16;
-  float *sK = smem + L::oK, *sQ = smem + L::oQ, *sV = smem + L::oV, *sA = smem + L::oA,
-        *sT = smem + L::oT, *sG = smem + L::oG, *sB = smem + L::oB;
+  float *sK = smem + L::oK, *sQV = smem + L::oQV, *sA = smem + L::oA, *sT = smem + L::oT,
+        *sG = smem + L::oG, *sB = smem + L::oB;
   const size_t ch = (size_t)blockIdx.x * a.H_v + h;
   const int n = e->n;
-  ld_rows(sK, L::LK, a.kh + ((size_t)e->t0 * a.H_qk + hq) * DK, (size_t)a.H_qk * DK, kC, n, DK);
-  ld_rows(sQ, L::LK, a.qh + ((size_t)e->t0 * a.H_qk + hq) * DK, (size_t)a.H_qk * DK, kC, n, DK);
-  ld_rows_in(sV, L::LV, static_cast<const Tin*>(a.v) + ((size_t)e->t0 * a.H_v + h) * DV,
-             (size_t)a.H_v * DV, kC, n, DV);
+  const size_t krow = (size_t)a.H_qk * DK;
+  cp_tile(sK, L::LK, a.kh + ((size_t)e->t0 * a.H_qk + hq) * DK, krow, kC, n, DK);
+  cp_tile(sQV, L::LQV, a.qh + ((size_t)e->t0 * a.H_qk + hq) * DK, krow, kC, n, DK);
+  cp_async_commit();
   load_gates(a, *e, h, sG, sB);
+  cp_async_wait_all();
   __syncthreads();
 
   // K K^T o E (strictly lower) -> global and A = beta_t (.) into sA; P -> global
@@ -234,7 +251,7 @@ __global__ void __launch_bounds__(kNT, 1) bwd_prep_kernel(const BwdArgs a) {
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         kt[u] = sK[(ty + 16 * u) * L::LK + d];
-        qt[u] = sQ[(ty + 16 * u) * L::LK + d];
+        qt[u] = sQV[(ty + 16 * u) * L::LQV + d];
         ki[u] = sK[(tx + 16 * u) * L::LK + d];
       }
 #pragma unroll
@@ -259,7 +276,22 @@ __global__ void __launch_bounds__(kNT, 1) bwd_prep_kernel(const BwdArgs a) {
         gP[t * kC + i] = i <= t ? a.scale * qk[u][w] * E : 0.f;
       }
   }
-  __syncthreads();
+  // this thread's share of V, fetched while T is being formed
+  float vr[kC * DV / kNT];
+  {
+    const Tin* V = static_cast<const Tin*>(a.v) + ((size_t)e->t0 * a.H_v + h) * DV;
+#pragma unroll
+    for (int m = 0; m < kC * DV / (4 * kNT); ++m) {
+      const int x = (tid + m * kNT) * 4, r = x / DV, c = x % DV;
+      const float4 f = r < n ? Elem<Tin>::load4(V + (size_t)r * a.H_v * DV + c)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+      vr[4 * m] = f.x;
+      vr[4 * m + 1] = f.y;
+      vr[4 * m + 2] = f.z;
+      vr[4 * m + 3] = f.w;
+    }
+  }
+  __syncthreads();  // sA complete; Q^ no longer read
 
   // T = (I + A)^-1, row by row: T_t = e_t - sum_{i<t} A_ti T_i.  Each warp
   // owns 8 columns, 4 lanes per column split the sum.
@@ -274,11 +306,16 @@ __global__ void __launch_bounds__(kNT, 1) bwd_prep_kernel(const BwdArgs a) {
       __syncwarp();
     }
   }
+#pragma unroll
+  for (int m = 0; m < kC * DV / (4 * kNT); ++m) {
+    const int x = (tid + m * kNT) * 4, r = x / DV, c = x % DV;
+    *reinterpret_cast<float4*>(sQV + r * L::LQV + c) =
+        make_float4(vr[4 * m], vr[4 * m + 1], vr[4 * m + 2], vr[4 * m + 3]);
+  }
   __syncthreads();
 
   // W = T diag(beta gamma) K, U = T diag(beta) V
   {
-    constexpr int NK = DK / 16, NV = DV / 16;
     float wacc[4][NK], uacc[4][NV];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
@@ -300,7 +337,7 @@ __global__ void __launch_bounds__(kNT, 1) bwd_prep_kernel(const BwdArgs a) {
       }
 #pragma unroll
       for (int w = 0; w < NV; ++w) {
-        const float vv = bi * sV[i * L::LV + tx + 16 * w];
+        const float vv = bi * sQV[i * L::LQV + tx + 16 * w];
 #pragma unroll
         for (int u = 0; u < 4; ++u) uacc[u][w] += tr[u] * vv;
       }
@@ -321,7 +358,9 @@ __global__ void __launch_bounds__(kNT, 1) bwd_prep_kernel(const BwdArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// fwd_chain: per (sequence, value head, slice of SW state columns).
+// Chains: per (sequence, value head, slice of SW state columns).  The state
+// columns evolve independently, so each slice is its own recurrence.  Two
+// CTAs per SM: one's loads overlap the other's arithmetic.
 
 template <int DV>
 struct Slice {
@@ -331,153 +370,163 @@ struct Slice {
 };
 
 template <int DK, int DV>
-struct FwdChainSmem {
-  static constexpr int LK = DK + 1, LS = Slice<DV>::SW + 1;
+struct ChainSmem {
+  static constexpr int LK = DK + 4, LS = Slice<DV>::SW + 4;
   static constexpr int oW = 0, oK = oW + kC * LK, oS = oK + kC * LK, oD = oS + DK * LS,
                        oG = oD + kC * LS, total = oG + kC;
   static constexpr size_t bytes = sizeof(float) * total;
 };
 
+// fwd_chain: S entering each chunk -> ws S; Delta = U - W S -> ws D.
 template <int DK, int DV>
-__global__ void __launch_bounds__(kNT, 1) bwd_fwd_chain_kernel(const BwdArgs a) {
-  using L = FwdChainSmem<DK, DV>;
+__global__ void __launch_bounds__(kNT, 2) bwd_fwd_chain_kernel(const BwdArgs a) {
+  using L = ChainSmem<DK, DV>;
   using SL = Slice<DV>;
   constexpr int SW = SL::SW, NW = SL::NW, NK = DK / 16;
-  extern __shared__ float smem[];
+  extern __shared__ __align__(16) float smem[];
   float *sW = smem + L::oW, *sK = smem + L::oK, *sS = smem + L::oS, *sD = smem + L::oD,
         *sG = smem + L::oG;
   const int seq = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * SW;
   const int hq = h / (a.H_v / a.H_qk);
   const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
   const size_t st = ((size_t)seq * a.H_v + h) * DK * DV;
-  for (int x = tid; x < DK * SW; x += kNT) {
-    const int i = x / SW, j = x % SW;
-    sS[i * L::LS + j] = a.initial_state ? __ldg(a.initial_state + st + (size_t)i * DV + j0 + j) : 0.f;
-  }
+  float sr[NK][NW];  // this thread's state elements: rows ty + 16u, columns j0 + tx + 16w
+#pragma unroll
+  for (int u = 0; u < NK; ++u)
+#pragma unroll
+    for (int w = 0; w < NW; ++w)
+      sr[u][w] = a.initial_state
+                     ? __ldg(a.initial_state + st + (size_t)(ty + 16 * u) * DV + j0 + tx + 16 * w)
+                     : 0.f;
   const int c_begin = a.seq_first[seq], c_end = a.seq_first[seq + 1];
   const ChunkEnt* ents = reinterpret_cast<const ChunkEnt*>(a.chunks);
   for (int c = c_begin; c < c_end; ++c) {
     const ChunkEnt e = ents[c];
     const size_t ch = (size_t)c * a.H_v + h;
-    __syncthreads();  // previous chunk done with sW, sK, sD, sG; sS final
-    float* gS = a.S + ch * DK * DV;
-    for (int x = tid; x < DK * SW; x += kNT) {
-      const int i = x / SW, j = x % SW;
-      gS[(size_t)i * DV + j0 + j] = sS[i * L::LS + j];
-    }
-    ld_rows(sW, L::LK, a.W + ch * kC * DK, DK, kC, kC, DK);
-    ld_rows(sK, L::LK, a.kh + ((size_t)e.t0 * a.H_qk + hq) * DK, (size_t)a.H_qk * DK, kC, e.n, DK);
-    ld_rows(sD, L::LS, a.UT + ch * kC * DV + j0, DV, kC, kC, SW);
-    if (tid < kC) sG[tid] = a.G[ch * kC + tid];
+    __syncthreads();  // the previous chunk is done with every buffer
+    cp_tile(sW, L::LK, a.W + ch * kC * DK, DK, kC, kC, DK);
+    cp_tile(sK, L::LK, a.kh + ((size_t)e.t0 * a.H_qk + hq) * DK, (size_t)a.H_qk * DK, kC, e.n, DK);
+    cp_tile(sG, kC, a.G + ch * kC, kC, 1, 1, kC);
+    cp_async_commit();
+    float* gS = a.S + ch * DK * DV + j0;
+    float acc[4][NW];
+#pragma unroll
+    for (int u = 0; u < NK; ++u)
+#pragma unroll
+      for (int w = 0; w < NW; ++w) {
+        const int i = ty + 16 * u, j = tx + 16 * w;
+        sS[i * L::LS + j] = sr[u][w];
+        gS[(size_t)i * DV + j] = sr[u][w];
+      }
+    const float* gU = a.UT + ch * kC * DV + j0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int w = 0; w < NW; ++w) acc[u][w] = __ldg(gU + (size_t)(ty + 16 * u) * DV + tx + 16 * w);
+    cp_async_wait_all();
     __syncthreads();
     // Delta = U - W S
-    {
-      float acc[4][NW];
+    for (int i = 0; i < DK; ++i) {
+      float sv[NW];
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
+      for (int w = 0; w < NW; ++w) sv[w] = sS[i * L::LS + tx + 16 * w];
 #pragma unroll
-        for (int w = 0; w < NW; ++w) acc[u][w] = sD[(ty + 16 * u) * L::LS + tx + 16 * w];
-      for (int i = 0; i < DK; ++i) {
-        float sv[NW];
+      for (int u = 0; u < 4; ++u) {
+        const float wv = sW[(ty + 16 * u) * L::LK + i];
 #pragma unroll
-        for (int w = 0; w < NW; ++w) sv[w] = sS[i * L::LS + tx + 16 * w];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float wv = sW[(ty + 16 * u) * L::LK + i];
-#pragma unroll
-          for (int w = 0; w < NW; ++w) acc[u][w] -= wv * sv[w];
-        }
+        for (int w = 0; w < NW; ++w) acc[u][w] -= wv * sv[w];
       }
-      __syncthreads();  // all reads of U done
-      float* gD = a.D + ch * kC * DV + j0;
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-#pragma unroll
-        for (int w = 0; w < NW; ++w) {
-          const int t = ty + 16 * u, j = tx + 16 * w;
-          sD[t * L::LS + j] = acc[u][w];
-          gD[(size_t)t * DV + j] = acc[u][w];
-        }
     }
+    float* gD = a.D + ch * kC * DV + j0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int w = 0; w < NW; ++w) {
+        const int t = ty + 16 * u, j = tx + 16 * w;
+        sD[t * L::LS + j] = acc[u][w];
+        gD[(size_t)t * DV + j] = acc[u][w];
+      }
     __syncthreads();
     // S <- gamma_C S + (diag(b) K)^T Delta
-    {
-      const float GC = sG[kC - 1], gC = expf(GC);
-      float acc[NK][NW];
+    const float GC = sG[kC - 1], gC = expf(GC);
 #pragma unroll
-      for (int u = 0; u < NK; ++u)
+    for (int u = 0; u < NK; ++u)
 #pragma unroll
-        for (int w = 0; w < NW; ++w) acc[u][w] = 0.f;
-      for (int t = 0; t < kC; ++t) {
-        const float bt = expf(GC - sG[t]);
-        float dv[NW];
+      for (int w = 0; w < NW; ++w) sr[u][w] *= gC;
+    for (int t = 0; t < kC; ++t) {
+      const float bt = expf(GC - sG[t]);
+      float dv[NW];
 #pragma unroll
-        for (int w = 0; w < NW; ++w) dv[w] = sD[t * L::LS + tx + 16 * w];
+      for (int w = 0; w < NW; ++w) dv[w] = sD[t * L::LS + tx + 16 * w];
 #pragma unroll
-        for (int u = 0; u < NK; ++u) {
-          const float kv = bt * sK[t * L::LK + ty + 16 * u];
+      for (int u = 0; u < NK; ++u) {
+        const float kv = bt * sK[t * L::LK + ty + 16 * u];
 #pragma unroll
-          for (int w = 0; w < NW; ++w) acc[u][w] += kv * dv[w];
-        }
+        for (int w = 0; w < NW; ++w) sr[u][w] += kv * dv[w];
       }
-#pragma unroll
-      for (int u = 0; u < NK; ++u)
-#pragma unroll
-        for (int w = 0; w < NW; ++w) {
-          float* p = sS + (ty + 16 * u) * L::LS + tx + 16 * w;
-          *p = gC * *p + acc[u][w];  // each element owned by one thread
-        }
     }
   }
 }
 
 // ---------------------------------------------------------------------------
-// epilogue: per (chunk, value head).  dO = dy without the epilogue; with it,
-// O is recomputed and dy is taken back through sigmoid(g), (1 + w) and the
-// RMS norm.  Also writes dg and this chunk's share of dw.
+// dout: per (chunk, value head).  dO = dy without the epilogue; with it, O is
+// recomputed and dy is taken back through sigmoid(g), (1 + w) and the RMS
+// norm (also writing dg and this chunk's share of dw).  Then the two
+// products the state-gradient chain needs from dO alone:
+//   X1 = P^T dO -> ws dD (the chain turns it into dDelta in place)
+//   X2 = scale (diag(gamma) Q^)^T dO -> ws dS (read by the chain before it
+//        stores dS1 there)
 
-template <int DK, int DV>
-struct EpiSmem {
-  static constexpr int LK = DK + 1, LV = DV + 1;
-  static constexpr int oQ = 0, oS = oQ + kC * LK, oP = oS + DK * LV, oD = oP + kC * kLC,
-                       oO = oD + kC * LV, oW = oO + kC * LV, oG = oW + (kNT / 32) * DV,
-                       total = oG + kC;
+template <int DK, int DV, bool EPI>
+struct DoutSmem {
+  static constexpr int LK = DK + 4, LV = DV + 4;
+  static constexpr int oQ = 0, oP = oQ + kC * LK, oO = oP + kC * kLC, oS = oO + kC * LV,
+                       oD = oS + (EPI ? DK * LV : 0), oW = oD + (EPI ? kC * LV : 0),
+                       oG = oW + (EPI ? 16 * DV : 0), total = oG + kC;
   static constexpr size_t bytes = sizeof(float) * total;
 };
 
-template <int DK, int DV, typename Tin>
-__global__ void __launch_bounds__(kNT, 1) bwd_epilogue_kernel(const BwdArgs a) {
-  using L = EpiSmem<DK, DV>;
-  constexpr int NV = DV / 16;
-  extern __shared__ float smem[];
+template <int DK, int DV, typename Tin, bool EPI>
+__global__ void __launch_bounds__(kNT, EPI ? 1 : 2) bwd_dout_kernel(const BwdArgs a) {
+  using L = DoutSmem<DK, DV, EPI>;
+  constexpr int NK = DK / 16, NV = DV / 16;
+  extern __shared__ __align__(16) float smem[];
   const ChunkEnt* e;
   if (!chunk_of(a, &e)) return;
   const int h = blockIdx.y, hq = h / (a.H_v / a.H_qk);
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, ty = tid / 16, tx = tid % 16;
+  const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
   const size_t ch = (size_t)blockIdx.x * a.H_v + h;
   const int n = e->n;
-  const Tin* dY = static_cast<const Tin*>(a.dy);
-  if (a.g == nullptr) {
-    for (int x = tid; x < n * DV; x += kNT) {
-      const size_t off = ((size_t)(e->t0 + x / DV) * a.H_v + h) * DV + x % DV;
-      a.dO[off] = Elem<Tin>::load(dY + off);
-    }
-    return;
+  float *sQ = smem + L::oQ, *sP = smem + L::oP, *sO = smem + L::oO, *sS = smem + L::oS,
+        *sD = smem + L::oD, *sWr = smem + L::oW, *sG = smem + L::oG;
+  cp_tile(sQ, L::LK, a.qh + ((size_t)e->t0 * a.H_qk + hq) * DK, (size_t)a.H_qk * DK, kC, n, DK);
+  cp_tile(sP, kLC, a.P + ch * kC * kC, kC, kC, kC, kC);
+  cp_tile(sG, kC, a.G + ch * kC, kC, 1, 1, kC);
+  if (EPI) {
+    cp_tile(sS, L::LV, a.S + ch * DK * DV, DV, DK, DK, DV);
+    cp_tile(sD, L::LV, a.D + ch * kC * DV, DV, kC, kC, DV);
   }
-  float *sQ = smem + L::oQ, *sS = smem + L::oS, *sP = smem + L::oP, *sD = smem + L::oD,
-        *sO = smem + L::oO, *sWp = smem + L::oW, *sG = smem + L::oG;
-  ld_rows(sQ, L::LK, a.qh + ((size_t)e->t0 * a.H_qk + hq) * DK, (size_t)a.H_qk * DK, kC, n, DK);
-  ld_rows(sS, L::LV, a.S + ch * DK * DV, DV, DK, DK, DV);
-  ld_rows(sP, kLC, a.P + ch * kC * kC, kC, kC, kC, kC);
-  ld_rows(sD, L::LV, a.D + ch * kC * DV, DV, kC, kC, DV);
-  if (tid < kC) sG[tid] = a.G[ch * kC + tid];
+  cp_async_commit();
+  const Tin* dY = static_cast<const Tin*>(a.dy);
+  const size_t row0 = (size_t)e->t0 * a.H_v + h;  // row of token t0, this head
+  // this thread's tile of dy: rows ty + 16u, columns tx + 16w
+  float dyr[4][NV];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int t = ty + 16 * u;
+#pragma unroll
+    for (int w = 0; w < NV; ++w)
+      dyr[u][w] = t < n ? Elem<Tin>::load(dY + (row0 + (size_t)t * a.H_v) * DV + tx + 16 * w) : 0.f;
+  }
+  cp_async_wait_all();
   __syncthreads();
-  {
-    float acc[4][NV], pacc[4][NV];
+  if (EPI) {
+    // O = scale diag(gamma) Q^ S0 + P Delta, in registers
+    float o[4][NV], pacc[4][NV];
 #pragma unroll
     for (int u = 0; u < 4; ++u)
 #pragma unroll
-      for (int w = 0; w < NV; ++w) acc[u][w] = pacc[u][w] = 0.f;
+      for (int w = 0; w < NV; ++w) o[u][w] = pacc[u][w] = 0.f;
     for (int i = 0; i < DK; ++i) {
       float sv[NV];
 #pragma unroll
@@ -486,7 +535,7 @@ __global__ void __launch_bounds__(kNT, 1) bwd_epilogue_kernel(const BwdArgs a) {
       for (int u = 0; u < 4; ++u) {
         const float qv = sQ[(ty + 16 * u) * L::LK + i];
 #pragma unroll
-        for (int w = 0; w < NV; ++w) acc[u][w] += qv * sv[w];
+        for (int w = 0; w < NV; ++w) o[u][w] += qv * sv[w];
       }
     }
     for (int i = 0; i < kC; ++i) {
@@ -500,124 +549,174 @@ __global__ void __launch_bounds__(kNT, 1) bwd_epilogue_kernel(const BwdArgs a) {
         for (int w = 0; w < NV; ++w) pacc[u][w] += pv * dv[w];
       }
     }
+    const Tin* Gg = static_cast<const Tin*>(a.g);
+    float wsum[NV];
+#pragma unroll
+    for (int w = 0; w < NV; ++w) wsum[w] = 0.f;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int t = ty + 16 * u;
-      const float sg = a.scale * expf(sG[t]);
+      const float sg0 = a.scale * expf(sG[t]);
+      float ss = 0.f;
 #pragma unroll
-      for (int w = 0; w < NV; ++w) sO[t * L::LV + tx + 16 * w] = sg * acc[u][w] + pacc[u][w];
+      for (int w = 0; w < NV; ++w) {
+        o[u][w] = sg0 * o[u][w] + pacc[u][w];
+        ss += o[u][w] * o[u][w];
+      }
+      ss = group_sum<16>(ss);
+      const float rs = rsqrtf(ss / (float)DV + a.eps_norm);
+      float dot = 0.f;
+#pragma unroll
+      for (int w = 0; w < NV; ++w) {
+        const int j = tx + 16 * w;
+        const float wj = a.norm_w ? __ldg(a.norm_w + j) : 0.f;
+        const float gv = t < n ? Elem<Tin>::load(Gg + (row0 + (size_t)t * a.H_v) * DV + j) : 0.f;
+        const float sgm = sigmoidf_(gv);
+        const float nv = o[u][w] * rs;
+        const float dyj = dyr[u][w];
+        if (t < n) a.dg[(row0 + (size_t)t * a.H_v) * DV + j] = dyj * nv * (1.f + wj) * sgm * (1.f - sgm);
+        wsum[w] += dyj * nv * sgm;
+        const float dn = dyj * (1.f + wj) * sgm;
+        pacc[u][w] = nv;   // keep n
+        dyr[u][w] = dn;    // dn in place of dy
+        dot += dn * nv;
+      }
+      dot = group_sum<16>(dot) / (float)DV;
+#pragma unroll
+      for (int w = 0; w < NV; ++w) dyr[u][w] = rs * (dyr[u][w] - pacc[u][w] * dot);
+    }
+#pragma unroll
+    for (int w = 0; w < NV; ++w) sWr[ty * DV + tx + 16 * w] = wsum[w];
+  }
+  // dO -> ws (valid rows) and shared memory (all rows; padded rows are 0)
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int t = ty + 16 * u;
+#pragma unroll
+    for (int w = 0; w < NV; ++w) {
+      const int j = tx + 16 * w;
+      sO[t * L::LV + j] = dyr[u][w];
+      if (t < n) a.dO[(row0 + (size_t)t * a.H_v) * DV + j] = dyr[u][w];
     }
   }
-  for (int x = tid; x < (kNT / 32) * DV; x += kNT) sWp[x] = 0.f;
   __syncthreads();
-  const Tin* Gg = static_cast<const Tin*>(a.g);
-  for (int r = warp; r < n; r += kNT / 32) {
-    const size_t off = ((size_t)(e->t0 + r) * a.H_v + h) * DV;
-    float ss = 0.f;
-    for (int j = lane; j < DV; j += 32) ss += sO[r * L::LV + j] * sO[r * L::LV + j];
-    ss = warp_sum(ss);
-    const float rs = rsqrtf(ss / (float)DV + a.eps_norm);
-    float dn[(DV + 31) / 32], nr[(DV + 31) / 32];
-    float dot = 0.f;
+  if (EPI) {
+    for (int j = tid; j < DV; j += kNT) {
+      float s = 0.f;
+      for (int r = 0; r < 16; ++r) s += sWr[r * DV + j];
+      a.dw[ch * DV + j] = s;
+    }
+  }
+  // X1 = P^T dO: X1_tj = sum_{s >= t} P_st dO_sj
+  {
+    float acc[4][NV];
 #pragma unroll
-    for (int m = 0; m < (DV + 31) / 32; ++m) {
-      const int j = lane + 32 * m;
-      dn[m] = nr[m] = 0.f;
-      if (j < DV) {
-        const float w = a.norm_w ? __ldg(a.norm_w + j) : 0.f;
-        const float sg = sigmoidf_(Elem<Tin>::load(Gg + off + j));
-        const float nv = sO[r * L::LV + j] * rs;
-        const float dyj = Elem<Tin>::load(dY + off + j);
-        a.dg[off + j] = dyj * nv * (1.f + w) * sg * (1.f - sg);
-        sWp[warp * DV + j] += dyj * nv * sg;
-        dn[m] = dyj * (1.f + w) * sg;
-        nr[m] = nv;
-        dot += dn[m] * nv;
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int w = 0; w < NV; ++w) acc[u][w] = 0.f;
+    for (int s = 0; s < kC; ++s) {
+      float yv[NV];
+#pragma unroll
+      for (int w = 0; w < NV; ++w) yv[w] = sO[s * L::LV + tx + 16 * w];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float pv = sP[s * kLC + ty + 16 * u];
+#pragma unroll
+        for (int w = 0; w < NV; ++w) acc[u][w] += pv * yv[w];
       }
     }
-    dot = warp_sum(dot) / (float)DV;
+    float* gX1 = a.dD + ch * kC * DV;
 #pragma unroll
-    for (int m = 0; m < (DV + 31) / 32; ++m) {
-      const int j = lane + 32 * m;
-      if (j < DV) a.dO[off + j] = rs * (dn[m] - nr[m] * dot);
-    }
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int w = 0; w < NV; ++w) gX1[(size_t)(ty + 16 * u) * DV + tx + 16 * w] = acc[u][w];
   }
-  __syncthreads();
-  for (int j = tid; j < DV; j += kNT) {
-    float s = 0.f;
-    for (int w = 0; w < kNT / 32; ++w) s += sWp[w * DV + j];
-    a.dw[ch * DV + j] = s;
+  // X2 = scale sum_t gamma_t q^_t dO_t^T (d_k x d_v)
+  {
+    float acc[NK][NV];
+#pragma unroll
+    for (int u = 0; u < NK; ++u)
+#pragma unroll
+      for (int w = 0; w < NV; ++w) acc[u][w] = 0.f;
+    for (int t = 0; t < kC; ++t) {
+      const float sg0 = a.scale * expf(sG[t]);
+      float yv[NV];
+#pragma unroll
+      for (int w = 0; w < NV; ++w) yv[w] = sO[t * L::LV + tx + 16 * w];
+#pragma unroll
+      for (int u = 0; u < NK; ++u) {
+        const float qv = sg0 * sQ[t * L::LK + ty + 16 * u];
+#pragma unroll
+        for (int w = 0; w < NV; ++w) acc[u][w] += qv * yv[w];
+      }
+    }
+    float* gX2 = a.dS + ch * DK * DV;
+#pragma unroll
+    for (int u = 0; u < NK; ++u)
+#pragma unroll
+      for (int w = 0; w < NV; ++w) gX2[(size_t)(ty + 16 * u) * DV + tx + 16 * w] = acc[u][w];
   }
 }
 
-// ---------------------------------------------------------------------------
-// bwd_chain: per (sequence, value head, slice of SW state columns), chunks in
-// reverse order.
-
+// bwd_chain: chunks in reverse; dS1 of each chunk -> ws dS (after taking X2
+// from there); dDelta = X1 + diag(b) K dS1 -> ws dD (in place of X1).
 template <int DK, int DV>
-struct BwdChainSmem {
-  static constexpr int LK = DK + 1, LS = Slice<DV>::SW + 1;
-  static constexpr int oP = 0, oK = oP + kC * kLC, oW = oK + kC * LK, oQ = oW + kC * LK,
-                       odS = oQ + kC * LK, odY = odS + DK * LS, odD = odY + kC * LS,
-                       oG = odD + kC * LS, total = oG + kC;
-  static constexpr size_t bytes = sizeof(float) * total;
-};
-
-template <int DK, int DV>
-__global__ void __launch_bounds__(kNT, 1) bwd_bwd_chain_kernel(const BwdArgs a) {
-  using L = BwdChainSmem<DK, DV>;
+__global__ void __launch_bounds__(kNT, 2) bwd_bwd_chain_kernel(const BwdArgs a) {
+  using L = ChainSmem<DK, DV>;
   using SL = Slice<DV>;
   constexpr int SW = SL::SW, NW = SL::NW, NK = DK / 16;
-  extern __shared__ float smem[];
-  float *sP = smem + L::oP, *sK = smem + L::oK, *sW = smem + L::oW, *sQ = smem + L::oQ,
-        *sdS = smem + L::odS, *sdY = smem + L::odY, *sdD = smem + L::odD, *sG = smem + L::oG;
+  extern __shared__ __align__(16) float smem[];
+  float *sW = smem + L::oW, *sK = smem + L::oK, *sdS = smem + L::oS, *sdD = smem + L::oD,
+        *sG = smem + L::oG;
   const int seq = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * SW;
   const int hq = h / (a.H_v / a.H_qk);
   const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
   const size_t st = ((size_t)seq * a.H_v + h) * DK * DV;
-  for (int x = tid; x < DK * SW; x += kNT) {
-    const int i = x / SW, j = x % SW;
-    sdS[i * L::LS + j] =
-        a.d_final_state ? __ldg(a.d_final_state + st + (size_t)i * DV + j0 + j) : 0.f;
-  }
+  float dr[NK][NW];  // this thread's dS elements: rows ty + 16u, columns j0 + tx + 16w
+#pragma unroll
+  for (int u = 0; u < NK; ++u)
+#pragma unroll
+    for (int w = 0; w < NW; ++w)
+      dr[u][w] = a.d_final_state
+                     ? __ldg(a.d_final_state + st + (size_t)(ty + 16 * u) * DV + j0 + tx + 16 * w)
+                     : 0.f;
   const int c_begin = a.seq_first[seq], c_end = a.seq_first[seq + 1];
   const ChunkEnt* ents = reinterpret_cast<const ChunkEnt*>(a.chunks);
   for (int c = c_end - 1; c >= c_begin; --c) {
     const ChunkEnt e = ents[c];
     const size_t ch = (size_t)c * a.H_v + h;
     __syncthreads();
-    float* gdS = a.dS + ch * DK * DV;
-    for (int x = tid; x < DK * SW; x += kNT) {
-      const int i = x / SW, j = x % SW;
-      gdS[(size_t)i * DV + j0 + j] = sdS[i * L::LS + j];
-    }
-    ld_rows(sP, kLC, a.P + ch * kC * kC, kC, kC, kC, kC);
-    ld_rows(sK, L::LK, a.kh + ((size_t)e.t0 * a.H_qk + hq) * DK, (size_t)a.H_qk * DK, kC, e.n, DK);
-    ld_rows(sW, L::LK, a.W + ch * kC * DK, DK, kC, kC, DK);
-    ld_rows(sQ, L::LK, a.qh + ((size_t)e.t0 * a.H_qk + hq) * DK, (size_t)a.H_qk * DK, kC, e.n, DK);
-    ld_rows(sdY, L::LS, a.dO + ((size_t)e.t0 * a.H_v + h) * DV + j0, (size_t)a.H_v * DV, kC, e.n,
-            SW);
-    if (tid < kC) sG[tid] = a.G[ch * kC + tid];
+    cp_tile(sW, L::LK, a.W + ch * kC * DK, DK, kC, kC, DK);
+    cp_tile(sK, L::LK, a.kh + ((size_t)e.t0 * a.H_qk + hq) * DK, (size_t)a.H_qk * DK, kC, e.n, DK);
+    cp_tile(sG, kC, a.G + ch * kC, kC, 1, 1, kC);
+    cp_async_commit();
+    float* gdS = a.dS + ch * DK * DV + j0;
+    float x2[NK][NW];
+#pragma unroll
+    for (int u = 0; u < NK; ++u)
+#pragma unroll
+      for (int w = 0; w < NW; ++w) {
+        const int i = ty + 16 * u, j = tx + 16 * w;
+        x2[u][w] = gdS[(size_t)i * DV + j];  // X2, then the same element gets dS1
+        gdS[(size_t)i * DV + j] = dr[u][w];
+        sdS[i * L::LS + j] = dr[u][w];
+      }
+    float* gdD = a.dD + ch * kC * DV + j0;
+    float acc[4][NW];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int w = 0; w < NW; ++w) acc[u][w] = gdD[(size_t)(ty + 16 * u) * DV + tx + 16 * w];
+    cp_async_wait_all();
     __syncthreads();
     const float GC = sG[kC - 1];
-    // dDelta = P^T dO + diag(b) K dS
+    // dDelta = X1 + diag(b) K dS1  (zero on rows past the chunk's end)
     {
-      float acc[4][NW], kacc[4][NW];
+      float kacc[4][NW];
 #pragma unroll
       for (int u = 0; u < 4; ++u)
 #pragma unroll
-        for (int w = 0; w < NW; ++w) acc[u][w] = kacc[u][w] = 0.f;
-      for (int s = 0; s < kC; ++s) {
-        float yv[NW];
-#pragma unroll
-        for (int w = 0; w < NW; ++w) yv[w] = sdY[s * L::LS + tx + 16 * w];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float pv = sP[s * kLC + ty + 16 * u];  // P_{s,t}
-#pragma unroll
-          for (int w = 0; w < NW; ++w) acc[u][w] += pv * yv[w];
-        }
-      }
+        for (int w = 0; w < NW; ++w) kacc[u][w] = 0.f;
       for (int i = 0; i < DK; ++i) {
         float sv[NW];
 #pragma unroll
@@ -629,7 +728,6 @@ __global__ void __launch_bounds__(kNT, 1) bwd_bwd_chain_kernel(const BwdArgs a) 
           for (int w = 0; w < NW; ++w) kacc[u][w] += kv * sv[w];
         }
       }
-      float* gdD = a.dD + ch * kC * DV + j0;
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int t = ty + 16 * u;
@@ -637,49 +735,39 @@ __global__ void __launch_bounds__(kNT, 1) bwd_bwd_chain_kernel(const BwdArgs a) 
 #pragma unroll
         for (int w = 0; w < NW; ++w) {
           const int j = tx + 16 * w;
-          const float v = acc[u][w] + bt * kacc[u][w];
+          const float v = t < e.n ? acc[u][w] + bt * kacc[u][w] : 0.f;
           sdD[t * L::LS + j] = v;
           gdD[(size_t)t * DV + j] = v;
         }
       }
     }
     __syncthreads();
-    // dS <- gamma_C dS + (diag(gamma) Qs)^T dO - W^T dDelta
+    // dS <- gamma_C dS + X2 - W^T dDelta
     {
       const float gC = expf(GC);
-      float acc[NK][NW];
 #pragma unroll
       for (int u = 0; u < NK; ++u)
 #pragma unroll
-        for (int w = 0; w < NW; ++w) acc[u][w] = gC * sdS[(ty + 16 * u) * L::LS + tx + 16 * w];
+        for (int w = 0; w < NW; ++w) dr[u][w] = gC * dr[u][w] + x2[u][w];
       for (int t = 0; t < kC; ++t) {
-        const float sg = a.scale * expf(sG[t]);
-        float yv[NW], dv[NW];
+        float dv[NW];
 #pragma unroll
-        for (int w = 0; w < NW; ++w) {
-          yv[w] = sdY[t * L::LS + tx + 16 * w];
-          dv[w] = sdD[t * L::LS + tx + 16 * w];
-        }
+        for (int w = 0; w < NW; ++w) dv[w] = sdD[t * L::LS + tx + 16 * w];
 #pragma unroll
         for (int u = 0; u < NK; ++u) {
-          const float qv = sg * sQ[t * L::LK + ty + 16 * u];
           const float wv = sW[t * L::LK + ty + 16 * u];
 #pragma unroll
-          for (int w = 0; w < NW; ++w) acc[u][w] += qv * yv[w] - wv * dv[w];
+          for (int w = 0; w < NW; ++w) dr[u][w] -= wv * dv[w];
         }
       }
-#pragma unroll
-      for (int u = 0; u < NK; ++u)
-#pragma unroll
-        for (int w = 0; w < NW; ++w) sdS[(ty + 16 * u) * L::LS + tx + 16 * w] = acc[u][w];
     }
   }
-  __syncthreads();
   if (a.d_initial_state) {
-    for (int x = tid; x < DK * SW; x += kNT) {
-      const int i = x / SW, j = x % SW;
-      a.d_initial_state[st + (size_t)i * DV + j0 + j] = sdS[i * L::LS + j];
-    }
+#pragma unroll
+    for (int u = 0; u < NK; ++u)
+#pragma unroll
+      for (int w = 0; w < NW; ++w)
+        a.d_initial_state[st + (size_t)(ty + 16 * u) * DV + j0 + tx + 16 * w] = dr[u][w];
   }
 }
 
@@ -688,7 +776,7 @@ __global__ void __launch_bounds__(kNT, 1) bwd_bwd_chain_kernel(const BwdArgs a) 
 
 template <int DV>
 struct ChunkASmem {
-  static constexpr int LV = DV + 1;
+  static constexpr int LV = DV + 4;
   static constexpr int oD = 0, odD = oD + kC * LV, odY = odD + kC * LV, oX = odY + kC * LV,
                        oT = oX + kC * LV, oKKE = oT + kC * kLC, oP = oKKE + kC * kLC,
                        oM1 = oP + kC * kLC, oM2 = oM1 + kC * kLC, oG = oM2 + kC * kLC,
@@ -700,7 +788,7 @@ template <int DK, int DV, typename Tin>
 __global__ void __launch_bounds__(kNT, 1) bwd_chunk_a_kernel(const BwdArgs a) {
   using L = ChunkASmem<DV>;
   constexpr int NV = DV / 16;
-  extern __shared__ float smem[];
+  extern __shared__ __align__(16) float smem[];
   const ChunkEnt* e;
   if (!chunk_of(a, &e)) return;
   const int h = blockIdx.y;
@@ -711,18 +799,18 @@ __global__ void __launch_bounds__(kNT, 1) bwd_chunk_a_kernel(const BwdArgs a) {
         *sT = smem + L::oT, *sKKE = smem + L::oKKE, *sP = smem + L::oP, *sM1 = smem + L::oM1,
         *sM2 = smem + L::oM2, *sG = smem + L::oG, *sB = smem + L::oB, *sR0 = smem + L::oR0,
         *sR1 = smem + L::oR1;
-  ld_rows(sD, L::LV, a.D + ch * kC * DV, DV, kC, kC, DV);
-  ld_rows(sdD, L::LV, a.dD + ch * kC * DV, DV, kC, kC, DV);
-  ld_rows(sdY, L::LV, a.dO + ((size_t)e->t0 * a.H_v + h) * DV, (size_t)a.H_v * DV, kC, n, DV);
+  cp_tile(sD, L::LV, a.D + ch * kC * DV, DV, kC, kC, DV);
+  cp_tile(sdD, L::LV, a.dD + ch * kC * DV, DV, kC, kC, DV);
+  cp_tile(sdY, L::LV, a.dO + ((size_t)e->t0 * a.H_v + h) * DV, (size_t)a.H_v * DV, kC, n, DV);
+  cp_tile(sT, kLC, a.T + ch * kC * kC, kC, kC, kC, kC);
+  cp_tile(sKKE, kLC, a.KKE + ch * kC * kC, kC, kC, kC, kC);
+  cp_tile(sP, kLC, a.P + ch * kC * kC, kC, kC, kC, kC);
+  cp_tile(sG, kC, a.G + ch * kC, kC, 1, 1, kC);
+  cp_async_commit();
   ld_rows_in(sX, L::LV, static_cast<const Tin*>(a.v) + ((size_t)e->t0 * a.H_v + h) * DV,
              (size_t)a.H_v * DV, kC, n, DV);
-  ld_rows(sT, kLC, a.T + ch * kC * kC, kC, kC, kC, kC);
-  ld_rows(sKKE, kLC, a.KKE + ch * kC * kC, kC, kC, kC, kC);
-  ld_rows(sP, kLC, a.P + ch * kC * kC, kC, kC, kC, kC);
-  if (tid < kC) {
-    sG[tid] = a.G[ch * kC + tid];
-    sB[tid] = tid < n ? __ldg(a.beta + (size_t)(e->t0 + tid) * a.H_v + h) : 0.f;
-  }
+  if (tid < kC) sB[tid] = tid < n ? __ldg(a.beta + (size_t)(e->t0 + tid) * a.H_v + h) : 0.f;
+  cp_async_wait_all();
   __syncthreads();
 
   // TdD = T^T dDelta -> global (reusing U's place); dV = diag(beta) TdD;
@@ -910,7 +998,7 @@ __global__ void __launch_bounds__(kNT, 1) bwd_chunk_a_kernel(const BwdArgs a) {
 
 template <int DK, int DV>
 struct ChunkBSmem {
-  static constexpr int LK = DK + 1, LV = DV + 1;
+  static constexpr int LK = DK + 4, LV = DV + 4;
   static constexpr int r1a = DK * LV, r1b = 2 * kC * LK;
   static constexpr int r2a = 2 * kC * LV, r2b = 2 * kC * kLC;
   static constexpr int oR1 = 0, oR2 = oR1 + (r1a > r1b ? r1a : r1b),
@@ -923,7 +1011,7 @@ template <int DK, int DV>
 __global__ void __launch_bounds__(kNT, 1) bwd_chunk_b_kernel(const BwdArgs a) {
   using L = ChunkBSmem<DK, DV>;
   constexpr int NK = DK / 16;
-  extern __shared__ float smem[];
+  extern __shared__ __align__(16) float smem[];
   const ChunkEnt* e;
   if (!chunk_of(a, &e)) return;
   const int h = blockIdx.y, hq = h / (a.H_v / a.H_qk);
@@ -938,9 +1026,11 @@ __global__ void __launch_bounds__(kNT, 1) bwd_chunk_b_kernel(const BwdArgs a) {
     float* sS = sR1;
     float* sY = sR2;
     float* sTd = sR2 + kC * L::LV;
-    ld_rows(sS, L::LV, a.S + ch * DK * DV, DV, DK, DK, DV);
-    ld_rows(sY, L::LV, a.dO + ((size_t)e->t0 * a.H_v + h) * DV, (size_t)a.H_v * DV, kC, n, DV);
-    ld_rows(sTd, L::LV, a.UT + ch * kC * DV, DV, kC, kC, DV);
+    cp_tile(sS, L::LV, a.S + ch * DK * DV, DV, DK, DK, DV);
+    cp_tile(sY, L::LV, a.dO + ((size_t)e->t0 * a.H_v + h) * DV, (size_t)a.H_v * DV, kC, n, DV);
+    cp_tile(sTd, L::LV, a.UT + ch * kC * DV, DV, kC, kC, DV);
+    cp_async_commit();
+    cp_async_wait_all();
     __syncthreads();
 #pragma unroll
     for (int u = 0; u < 4; ++u)
@@ -970,8 +1060,10 @@ __global__ void __launch_bounds__(kNT, 1) bwd_chunk_b_kernel(const BwdArgs a) {
   {
     float* sdS = sR1;
     float* sDl = sR2;
-    ld_rows(sdS, L::LV, a.dS + ch * DK * DV, DV, DK, DK, DV);
-    ld_rows(sDl, L::LV, a.D + ch * kC * DV, DV, kC, kC, DV);
+    cp_tile(sdS, L::LV, a.dS + ch * DK * DV, DV, DK, DK, DV);
+    cp_tile(sDl, L::LV, a.D + ch * kC * DV, DV, kC, kC, DV);
+    cp_async_commit();
+    cp_async_wait_all();
     __syncthreads();
     const float* gS = a.S + ch * DK * DV;
     for (int x = tid; x < DK * DV; x += kNT) sdot += gS[x] * sdS[(x / DV) * L::LV + x % DV];
@@ -1001,14 +1093,14 @@ __global__ void __launch_bounds__(kNT, 1) bwd_chunk_b_kernel(const BwdArgs a) {
   float* sBm = sR2 + kC * kLC;
   float sd_total = 0.f;
   for (int w = 0; w < kNT / 32; ++w) sd_total += sRed[w];
-  ld_rows(sK, L::LK, a.kh + ((size_t)e->t0 * a.H_qk + hq) * DK, (size_t)a.H_qk * DK, kC, n, DK);
-  ld_rows(sQ, L::LK, a.qh + ((size_t)e->t0 * a.H_qk + hq) * DK, (size_t)a.H_qk * DK, kC, n, DK);
-  ld_rows(sdPE, kLC, a.dPE + ch * kC * kC, kC, kC, kC, kC);
-  ld_rows(sBm, kLC, a.Bm + ch * kC * kC, kC, kC, kC, kC);
-  if (tid < kC) {
-    sG[tid] = a.G[ch * kC + tid];
-    sB[tid] = tid < n ? __ldg(a.beta + (size_t)(e->t0 + tid) * a.H_v + h) : 0.f;
-  }
+  cp_tile(sK, L::LK, a.kh + ((size_t)e->t0 * a.H_qk + hq) * DK, (size_t)a.H_qk * DK, kC, n, DK);
+  cp_tile(sQ, L::LK, a.qh + ((size_t)e->t0 * a.H_qk + hq) * DK, (size_t)a.H_qk * DK, kC, n, DK);
+  cp_tile(sdPE, kLC, a.dPE + ch * kC * kC, kC, kC, kC, kC);
+  cp_tile(sBm, kLC, a.Bm + ch * kC * kC, kC, kC, kC, kC);
+  cp_tile(sG, kC, a.G + ch * kC, kC, 1, 1, kC);
+  cp_async_commit();
+  if (tid < kC) sB[tid] = tid < n ? __ldg(a.beta + (size_t)(e->t0 + tid) * a.H_v + h) : 0.f;
+  cp_async_wait_all();
   __syncthreads();
   const float GC = sG[kC - 1];
   float dG6[4], db6[4], bk3[4];
@@ -1190,30 +1282,37 @@ template <int DK, int DV, typename Tin>
 gdn_status launch(const BwdArgs& a, cudaStream_t s) {
   const int64_t maxc = max_chunks_of(a.n_seq, a.total_T);
   const unsigned H = (unsigned)a.H_v;
+  const dim3 per_chunk((unsigned)maxc, H), per_slice((unsigned)a.n_seq, H, Slice<DV>::NS);
   bwd_chunk_table_kernel<<<1, kNT, 0, s>>>(a);
   if (a.total_T > 0) {
     const unsigned rows = (unsigned)((a.total_T * a.H_qk + 7) / 8);
     bwd_normalise_kernel<DK, Tin><<<rows, kNT, 0, s>>>(a);
     auto k1 = bwd_prep_kernel<DK, DV, Tin>;
     if (!set_smem(k1, PrepSmem<DK, DV>::bytes)) return GDN_ERR_CUDA;
-    k1<<<dim3((unsigned)maxc, H), kNT, PrepSmem<DK, DV>::bytes, s>>>(a);
+    k1<<<per_chunk, kNT, PrepSmem<DK, DV>::bytes, s>>>(a);
     auto k2 = bwd_fwd_chain_kernel<DK, DV>;
-    if (!set_smem(k2, FwdChainSmem<DK, DV>::bytes)) return GDN_ERR_CUDA;
-    k2<<<dim3((unsigned)a.n_seq, H, Slice<DV>::NS), kNT, FwdChainSmem<DK, DV>::bytes, s>>>(a);
-    auto k3 = bwd_epilogue_kernel<DK, DV, Tin>;
-    if (!set_smem(k3, EpiSmem<DK, DV>::bytes)) return GDN_ERR_CUDA;
-    k3<<<dim3((unsigned)maxc, H), kNT, EpiSmem<DK, DV>::bytes, s>>>(a);
+    if (!set_smem(k2, ChainSmem<DK, DV>::bytes)) return GDN_ERR_CUDA;
+    k2<<<per_slice, kNT, ChainSmem<DK, DV>::bytes, s>>>(a);
+    if (a.g != nullptr) {
+      auto k3 = bwd_dout_kernel<DK, DV, Tin, true>;
+      if (!set_smem(k3, DoutSmem<DK, DV, true>::bytes)) return GDN_ERR_CUDA;
+      k3<<<per_chunk, kNT, DoutSmem<DK, DV, true>::bytes, s>>>(a);
+    } else {
+      auto k3 = bwd_dout_kernel<DK, DV, Tin, false>;
+      if (!set_smem(k3, DoutSmem<DK, DV, false>::bytes)) return GDN_ERR_CUDA;
+      k3<<<per_chunk, kNT, DoutSmem<DK, DV, false>::bytes, s>>>(a);
+    }
   }
   auto k4 = bwd_bwd_chain_kernel<DK, DV>;
-  if (!set_smem(k4, BwdChainSmem<DK, DV>::bytes)) return GDN_ERR_CUDA;
-  k4<<<dim3((unsigned)a.n_seq, H, Slice<DV>::NS), kNT, BwdChainSmem<DK, DV>::bytes, s>>>(a);
+  if (!set_smem(k4, ChainSmem<DK, DV>::bytes)) return GDN_ERR_CUDA;
+  k4<<<per_slice, kNT, ChainSmem<DK, DV>::bytes, s>>>(a);
   if (a.total_T > 0) {
     auto k5 = bwd_chunk_a_kernel<DK, DV, Tin>;
     if (!set_smem(k5, ChunkASmem<DV>::bytes)) return GDN_ERR_CUDA;
-    k5<<<dim3((unsigned)maxc, H), kNT, ChunkASmem<DV>::bytes, s>>>(a);
+    k5<<<per_chunk, kNT, ChunkASmem<DV>::bytes, s>>>(a);
     auto k6 = bwd_chunk_b_kernel<DK, DV>;
     if (!set_smem(k6, ChunkBSmem<DK, DV>::bytes)) return GDN_ERR_CUDA;
-    k6<<<dim3((unsigned)maxc, H), kNT, ChunkBSmem<DK, DV>::bytes, s>>>(a);
+    k6<<<per_chunk, kNT, ChunkBSmem<DK, DV>::bytes, s>>>(a);
     const unsigned rows = (unsigned)((a.total_T * a.H_qk + 7) / 8);
     bwd_qk_final_kernel<DK, Tin><<<rows, kNT, 0, s>>>(a);
   }
