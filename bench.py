@@ -3,7 +3,7 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload prefill4k|prefill256k|varlen]
                     [--path auto|tensor|tensor_pair|tensor_single|tensor_split|simt]
-                    [--no-decode] [--no-cpu-baseline]
+                    [--no-decode] [--no-backward] [--no-cpu-baseline]
 
 One step = one chunked prefill (gdn_chunk_fwd: L2-norm prologue, gate cumsum,
 intra-chunk products, triangular solve, state carry, RMSNorm x sigmoid(g)
@@ -11,8 +11,9 @@ epilogue) over one batch of the workload (default: B=1, T=4096, 16 QK / 48
 value heads, d=128, bf16).  The call gets a preallocated workspace, so small
 batches may take the split layout (one kernel, after an asynchronous memset of
 the workspace flags).  The JSON line also carries the decode step
-(gdn_decode_step, 256 sequences x 64 steps, in place) as a separate object
-with its own timing, roofline and clocks.
+(gdn_decode_step, 256 sequences x 64 steps, in place) and the backward of the
+model-shape prefill (gdn_chunk_bwd, T=4096) as separate objects with their
+own timing, roofline and clocks.
 
 Multi-GPU (torchrun, one process per GPU): every rank runs its own
 independent batch (weak scaling; sequences and heads are independent, so the
@@ -61,6 +62,22 @@ def prefill_bytes(T, n_seq, epilogue=True, init_state=True, in_bytes=2, Hqk=H_QK
         per_tok += Hv * d * in_bytes
     state = n_seq * Hv * d * d * 4
     return per_tok * T + state * (2 if init_state else 1) + (d * 4 if epilogue else 0)
+
+
+def bwd_flops_per_token(Hqk=H_QK, Hv=H_V, d=D, C=CHUNK, epilogue=True):
+    """Counted contraction FLOPs per token of the chunkwise backward at the
+    canonical chunk of 64 (forward recomputation included): per value head
+    (18 or 16) d^2 + 24 C d + 13 C^2 / 3, per QK head 4 C d."""
+    dd = 18 if epilogue else 16
+    return Hv * (dd * d * d + 24 * C * d + 13.0 * C * C / 3.0) + Hqk * 4 * C * d
+
+
+def bwd_bytes(T, n_seq, epilogue=True, in_bytes=2, Hqk=H_QK, Hv=H_V, d=D):
+    """Compulsory HBM bytes of one backward: inputs and dy read once (the
+    input dtype), fp32 gradients written once, dS_T read and dS0 written."""
+    per_tok_in = 2 * Hqk * d * in_bytes + (3 if epilogue else 2) * Hv * d * in_bytes + Hv * 8
+    per_tok_out = 2 * Hqk * d * 4 + (2 if epilogue else 1) * Hv * d * 4 + Hv * 8
+    return (per_tok_in + per_tok_out) * T + 2 * n_seq * Hv * d * d * 4 + (d * 4 if epilogue else 0)
 
 
 def decode_bytes(N, Hqk=H_QK, Hv=H_V, d=D, in_bytes=2):
@@ -497,6 +514,54 @@ def run_ours(args, world, rank, local):
             "clocks": mclk_r}
         launches_decode += len(groups) * max(3, args.steps // 2)
 
+    # the backward (gdn_chunk_bwd) on the model-shape sequence, timed on its own
+    backward = None
+    launches_bwd = 0
+    if not args.no_backward:
+        from gated_deltanet_scan_chunked_b200 import gdn_chunk_bwd
+        wb = inputs.workload("prefill4k", device="cuda")
+        dy, dsT = inputs.make_cotangents(wb, seed=inputs.SEEDS["prefill4k"] + 100 * rank)
+        Tb = wb.q.shape[0]
+        bws = torch.empty(gdn.bwd_workspace_size(1, Tb, H_QK, H_V, D, D), dtype=torch.uint8,
+                          device="cuda")
+        bflush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
+
+        def bstep():
+            gdn_chunk_bwd(wb.q, wb.k, wb.v, wb.log_alpha, wb.beta, dy, g=wb.g, norm_w=wb.norm_w,
+                          d_final_state=dsT, workspace=bws)
+
+        bclk = ClockSampler(local)
+        bclk.start()
+        bsteps = max(3, args.steps // 4)
+        bt = timed_steps(bstep, bsteps, 3, world, flush=lambda: bflush.zero_(), stream=stream)
+        bclk_r = bclk.stop()
+        err = gdn.gdn_check_device_error()
+        if err != gdn.GDN_OK:
+            raise RuntimeError("device error in the backward: %s" % gdn.status_string(err))
+        bms = max_over_ranks(statistics.mean(bt), world)
+        bb = bwd_bytes(Tb, 1)
+        bfl = bwd_flops_per_token() * Tb
+        alu_peak = 148 * 128 * 2 * 1.965  # fp32 FMA lanes x 2 FLOP x max SM GHz, in GFLOP/s
+        backward = {
+            "workload": "backward of prefill4k: T=4096, 16 QK / 48 value heads, d=128, bf16 "
+                        "inputs and dy, epilogue, dS_T given; fp32 gradients",
+            "ms_per_step": bms, "tokens_per_s": world * Tb / (bms * 1e-3),
+            "workspace_bytes": bws.numel(),
+            "roofline": {"bound": "hbm", "achieved": bb / (bms * 1e-3) / 1e9,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": bb / (bms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                         "algorithmic_bytes": bb, "traffic": None},
+            "tensor": {"achieved_tflops": bfl / (bms * 1e-3) / 1e12,
+                       "peak_tflops": peaks["bf16_tflops"],
+                       "frac": bfl / (bms * 1e-3) / 1e12 / (peaks["bf16_tflops"])},
+            "alu_roofline": {"bound": "alu", "achieved": bfl / (bms * 1e-3) / 1e9,
+                             "peak": alu_peak, "unit": "GFLOP/s",
+                             "frac": bfl / (bms * 1e-3) / 1e9 / alu_peak,
+                             "note": "fp32 CUDA-core arithmetic, the limiter of this kernel set"},
+            "clocks": bclk_r}
+        launches_bwd = bsteps * (10 if wb.g is not None else 9)
+        del bws, bflush
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, target_s=args.ref_seconds)
@@ -513,7 +578,8 @@ def run_ours(args, world, rank, local):
                            "l2": "flushed between steps (256 MB write outside the events)"},
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": args.steps, "clocks": clk, "decode": decode,
-                "gpu_launches_decode_region": launches_decode}
+                "gpu_launches_decode_region": launches_decode, "backward": backward,
+                "gpu_launches_backward_region": launches_bwd}
         print(json.dumps(line), flush=True)
 
 
@@ -529,6 +595,7 @@ def main():
                     choices=["auto", "tensor", "simt", "tensor_pair", "tensor_single",
                              "tensor_split"])
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-seconds", type=float, default=12.0)
