@@ -18,6 +18,8 @@ stated at the top of ``gdn_oracle.c``:
   section 4.1), used only to pin the error form;
 * the optional zero-centred RMSNorm x sigmoid(g) epilogue (section 03,
   "what Qwen changed on the original GDN"; hyper.ai summary, "Method");
+* the front end: short depthwise causal convolution (kernel 4) and SiLU
+  (section 02 module table, GDN row; hyper.ai "Method"; close reading 4.1);
 * the backward of all of the above (the adjoint of the error-form recurrence,
   differentiated by hand token by token in reverse order), for training.
 
@@ -75,6 +77,10 @@ def _load():
             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
             ctypes.c_double, ctypes.c_double, _f32p, _f32p, _f64p, _f64p,
             _f64p, _f64p, _f64p, _f64p, _f64p, _f64p, ctypes.c_int]
+        lib.gdn_oracle_conv.restype = ctypes.c_int
+        lib.gdn_oracle_conv.argtypes = [
+            _f32p, ctypes.c_int64, ctypes.c_int, _f32p, _f32p, _i64p, ctypes.c_int64,
+            ctypes.c_int, _f64p, _f64p]
         lib.gdn_oracle_max_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -213,3 +219,29 @@ def backward(q, k, v, log_alpha, beta, dy, g=None, norm_w=None,
     if rc != 0:
         raise ValueError("oracle rejected its arguments")
     return out
+
+
+def conv(x, w, state_in=None, cu_seqlens=None, silu=True):
+    """Depthwise causal convolution of kernel 4 over time, then SiLU, in fp64.
+
+    x [T, C]; w [C, 4] (w[:, 3] weighs the current token); state_in
+    [n_seq, 3, C] or None (zeros): the three inputs before each sequence's
+    first token, oldest first.  Returns (y [T, C], state_out [n_seq, 3, C]),
+    state_out holding the last three inputs of each sequence, oldest first.
+    """
+    lib = _load()
+    xx = _as_np(x, np.float32)
+    ww = _as_np(w, np.float32)
+    st = _as_np(state_in, np.float32)
+    T, C = xx.shape
+    cu = (np.array([0, T], dtype=np.int64) if cu_seqlens is None
+          else _as_np(cu_seqlens, np.int64))
+    n_seq = cu.shape[0] - 1
+    y = np.zeros((T, C), dtype=np.float64)
+    so = np.zeros((n_seq, 3, C), dtype=np.float64)
+    rc = lib.gdn_oracle_conv(_ptr(xx, _f32p), T, C, _ptr(ww, _f32p), _ptr(st, _f32p),
+                             _ptr(cu, _i64p), n_seq, int(bool(silu)), _ptr(y, _f64p),
+                             _ptr(so, _f64p))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    return y, so

@@ -557,6 +557,57 @@ int gdn_oracle_backward(const float* q, const float* k, const float* v,
   return bad ? -1 : 0;
 }
 
+/*
+ * Front end of the mixer: short depthwise causal convolution of kernel 4
+ * over time, then SiLU ("Qwen3.8-Flash-Next: architecture, efficiency and
+ * technical lineage", section 02 module table, GDN row: Q/K/V pass a short
+ * causal conv of kernel 4; hyper.ai summary, "Method": projections followed
+ * by short depthwise causal convolutions; "On the Design of Qwen3.8-Next
+ * Architecture ... close reading", section 4.1: short conv + SiLU + L2 norm).
+ *
+ * x [total_T, C] (C channels of one token side by side), w [C, 4] with w[c][3]
+ * the weight of the current token and w[c][3 - j] that of the token j steps
+ * back; no bias.  For each sequence s and channel c:
+ *     u_t = sum_{j=0..3} w[c][3 - j] * x_{t - j}
+ * where x_{t - j} before the sequence's first token comes from state_in[s]
+ * ([3, C]; row m holds the input m - 3 tokens before the start, row 2 the
+ * last one) or is 0 when state_in is NULL.  y_t = silu ? u_t / (1 + e^-u_t)
+ * : u_t.  state_out[s] (may be NULL) receives the three inputs the next
+ * segment of the sequence would need: rows 0..2 = the inputs 3, 2, 1 tokens
+ * before the end (taken from state_in, or 0, for short sequences).
+ * Returns 0, or -1 on a bad argument.
+ */
+int gdn_oracle_conv(const float* x, int64_t total_T, int C, const float* w,
+                    const float* state_in, const int64_t* cu_seqlens,
+                    int64_t n_seq, int silu, double* y, double* state_out) {
+  if (!x && total_T > 0) return -1;
+  if (!w || !y || !cu_seqlens || C <= 0 || n_seq < 0) return -1;
+  if (cu_seqlens[0] != 0 || cu_seqlens[n_seq] != total_T) return -1;
+  for (int64_t s = 0; s < n_seq; ++s)
+    if (cu_seqlens[s + 1] < cu_seqlens[s]) return -1;
+  for (int64_t s = 0; s < n_seq; ++s) {
+    const int64_t t0 = cu_seqlens[s], t1 = cu_seqlens[s + 1];
+    const float* st = state_in ? state_in + (size_t)s * 3 * C : NULL;
+    for (int c = 0; c < C; ++c) {
+      /* the input `back` tokens before token t of this sequence */
+#define XIN(t, back)                                                        \
+  (((t) - (back) >= t0) ? (double)x[(size_t)((t) - (back)) * C + c]         \
+   : (st ? (double)st[(size_t)(3 - ((back) - ((t) - t0))) * C + c] : 0.0))
+      for (int64_t t = t0; t < t1; ++t) {
+        double u = 0.0;
+        for (int j = 0; j < 4; ++j) u += (double)w[(size_t)c * 4 + 3 - j] * XIN(t, j);
+        y[(size_t)t * C + c] = silu ? u / (1.0 + exp(-u)) : u;
+      }
+      if (state_out) {
+        for (int m = 0; m < 3; ++m)
+          state_out[((size_t)s * 3 + m) * C + c] = XIN(t1, 3 - m);
+      }
+#undef XIN
+    }
+  }
+  return 0;
+}
+
 /* Number of threads an OpenMP parallel region would use. */
 int gdn_oracle_max_threads(void) {
 #ifdef _OPENMP
