@@ -4,9 +4,11 @@ The computation lives in libgdn.so (CUDA kernels behind the C ABI in
 include/gdn.h).  ``gdn`` is a thin ctypes binding; ``inputs`` holds the
 seeded synthetic workloads; ``build`` compiles the library.
 """
-from .gdn import (GdnError, bwd_workspace_size, gdn_check_device_error,  # noqa: F401
-                  gdn_chunk_bwd, gdn_chunk_fwd, gdn_decode_multi, gdn_decode_step, load,
+from .gdn import (GdnError, bwd_workspace_size, conv_workspace_size,  # noqa: F401
+                  gdn_check_device_error, gdn_chunk_bwd, gdn_chunk_fwd, gdn_chunk_fwd_conv,
+                  gdn_conv_frontend, gdn_decode_conv, gdn_decode_multi, gdn_decode_step, load,
                   workspace_size)
 
 __all__ = ["gdn_chunk_fwd", "gdn_chunk_bwd", "gdn_decode_step", "gdn_decode_multi",
-           "gdn_check_device_error", "GdnError", "load", "workspace_size", "bwd_workspace_size"]
+           "gdn_check_device_error", "gdn_conv_frontend", "gdn_chunk_fwd_conv", "gdn_decode_conv", "GdnError", "load",
+           "workspace_size", "bwd_workspace_size", "conv_workspace_size"]

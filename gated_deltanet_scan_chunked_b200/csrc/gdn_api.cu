@@ -136,12 +136,22 @@ extern "C" gdn_status gdn_chunk_fwd(
                             eps_norm, scale, y, final_state, GDN_PATH_AUTO, stream);
 }
 
-extern "C" gdn_status gdn_decode_multi(
-    const void* q, const void* k, const void* v, const float* log_alpha, const float* beta,
-    const void* g, const float* norm_w, const float* state_in, float* state_out,
-    float* snapshots, int32_t N, int32_t T_s, int32_t H_qk, int32_t H_v, int32_t d_k,
-    int32_t d_v, gdn_dtype in_dtype, int32_t l2norm_qk, float eps_l2, float eps_norm,
-    float scale, void* y, gdn_stream_t stream) {
+namespace {
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  if (!a || !b) return false;
+  const char* x = static_cast<const char*>(a);
+  const char* y = static_cast<const char*>(b);
+  return x < y + nb && y < x + na;
+}
+
+gdn_status decode_impl(const void* q, const void* k, const void* v, const float* log_alpha,
+                       const float* beta, const void* g, const float* norm_w,
+                       const float* conv_w, float* conv_state, const float* state_in,
+                       float* state_out, float* snapshots, int32_t N, int32_t T_s, int32_t H_qk,
+                       int32_t H_v, int32_t d_k, int32_t d_v, gdn_dtype in_dtype,
+                       int32_t l2norm_qk, float eps_l2, float eps_norm, float scale, void* y,
+                       gdn_stream_t stream) {
   gdn_status st = check_common(H_qk, H_v, d_k, d_v, in_dtype, eps_l2, eps_norm);
   if (st != GDN_OK) return st;
   if (N < 0 || T_s < 0 || (int64_t)N * H_v > 0x7fffffffLL) return GDN_ERR_INVALID_ARG;
@@ -175,7 +185,143 @@ extern "C" gdn_status gdn_decode_multi(
   a.N = N; a.T_s = T_s; a.H_qk = H_qk; a.H_v = H_v; a.d_k = d_k; a.d_v = d_v;
   a.dtype = in_dtype;
   a.l2norm = l2norm_qk ? 1 : 0; a.eps_l2 = eps_l2; a.eps_norm = eps_norm; a.scale = scale;
+  a.conv_w = conv_w; a.conv_state = conv_state;
   return launch_decode(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+
+extern "C" gdn_status gdn_decode_multi(
+    const void* q, const void* k, const void* v, const float* log_alpha, const float* beta,
+    const void* g, const float* norm_w, const float* state_in, float* state_out,
+    float* snapshots, int32_t N, int32_t T_s, int32_t H_qk, int32_t H_v, int32_t d_k,
+    int32_t d_v, gdn_dtype in_dtype, int32_t l2norm_qk, float eps_l2, float eps_norm,
+    float scale, void* y, gdn_stream_t stream) {
+  return decode_impl(q, k, v, log_alpha, beta, g, norm_w, nullptr, nullptr, state_in, state_out,
+                     snapshots, N, T_s, H_qk, H_v, d_k, d_v, in_dtype, l2norm_qk, eps_l2,
+                     eps_norm, scale, y, stream);
+}
+
+extern "C" gdn_status gdn_decode_conv(
+    const void* q, const void* k, const void* v, const float* conv_w, float* conv_state,
+    const float* log_alpha, const float* beta, const void* g, const float* norm_w,
+    const float* state_in, float* state_out, float* snapshots, int32_t N, int32_t T_s,
+    int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v, gdn_dtype in_dtype, int32_t l2norm_qk,
+    float eps_l2, float eps_norm, float scale, void* y, gdn_stream_t stream) {
+  if (N > 0 && T_s > 0 && conv_w == nullptr) return GDN_ERR_INVALID_ARG;
+  if ((conv_w && !aligned16(conv_w)) || (conv_state && !aligned16(conv_state)))
+    return GDN_ERR_INVALID_ARG;
+  if (conv_state) {
+    // the conv state may not overlap the recurrent states or the snapshots
+    const size_t cb = (size_t)N * H_v * 3 * (2 * d_k + d_v) * sizeof(float);
+    const size_t sb = (size_t)N * H_v * d_k * d_v * sizeof(float);
+    if (overlaps(conv_state, cb, state_in, sb) || overlaps(conv_state, cb, state_out, sb) ||
+        overlaps(conv_state, cb, snapshots, sb * (size_t)(T_s > 0 ? T_s : 0)))
+      return GDN_ERR_INVALID_ARG;
+  }
+  return decode_impl(q, k, v, log_alpha, beta, g, norm_w, conv_w, conv_state, state_in,
+                     state_out, snapshots, N, T_s, H_qk, H_v, d_k, d_v, in_dtype, l2norm_qk,
+                     eps_l2, eps_norm, scale, y, stream);
+}
+
+namespace {
+
+size_t conv_buffers_bytes(int64_t total_T, int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v,
+                          gdn_dtype dt) {
+  const size_t e = dt == GDN_BF16 ? 2 : 4;
+  auto a256 = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  return 2 * a256((size_t)total_T * H_qk * d_k * e) + a256((size_t)total_T * H_v * d_v * e);
+}
+
+gdn_status conv_impl(const void* q, const void* k, const void* v, const float* conv_w,
+                     const float* conv_state_in, float* conv_state_out,
+                     const int32_t* cu_seqlens, int32_t n_seq, int64_t total_T, int32_t H_qk,
+                     int32_t H_v, int32_t d_k, int32_t d_v, gdn_dtype in_dtype, void* q_out,
+                     void* k_out, void* v_out, gdn_stream_t stream) {
+  gdn_status st = check_common(H_qk, H_v, d_k, d_v, in_dtype, 0.f, 0.f);
+  if (st != GDN_OK) return st;
+  if (n_seq < 1 || total_T < 0) return GDN_ERR_INVALID_ARG;
+  if (cu_seqlens == nullptr && n_seq != 1) return GDN_ERR_INVALID_ARG;
+  if ((int64_t)n_seq * H_v > 0x7fffffffLL) return GDN_ERR_INVALID_ARG;
+  if (!conv_w) return GDN_ERR_INVALID_ARG;
+  if (total_T > 0 && (!q || !k || !v || !q_out || !k_out || !v_out)) return GDN_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, conv_w, conv_state_in, conv_state_out, q_out, k_out, v_out};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
+  if (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return GDN_ERR_INVALID_ARG;
+  const size_t e = in_dtype == GDN_BF16 ? 2 : 4;
+  const size_t nqk = (size_t)total_T * H_qk * d_k * e, nv = (size_t)total_T * H_v * d_v * e;
+  const size_t ns = (size_t)n_seq * H_v * 3 * (2 * d_k + d_v) * sizeof(float);
+  if (overlaps(conv_state_in, ns, conv_state_out, ns)) return GDN_ERR_INVALID_ARG;
+  const void* ins[] = {q, k, v};
+  const size_t in_n[] = {nqk, nqk, nv};
+  void* outs[] = {q_out, k_out, v_out};
+  for (int i = 0; i < 3; ++i)
+    for (int j = 0; j < 3; ++j)
+      if (overlaps(outs[i], in_n[i], ins[j], in_n[j])) return GDN_ERR_INVALID_ARG;
+  ConvArgs a;
+  a.q = q; a.k = k; a.v = v; a.conv_w = conv_w; a.state_in = conv_state_in;
+  a.state_out = conv_state_out; a.cu_seqlens = cu_seqlens; a.n_seq = n_seq; a.total_T = total_T;
+  a.H_qk = H_qk; a.H_v = H_v; a.d_k = d_k; a.d_v = d_v; a.dtype = in_dtype;
+  a.q_out = q_out; a.k_out = k_out; a.v_out = v_out;
+  a.err = error_word_ptr();
+  if (a.err == nullptr) return GDN_ERR_CUDA;
+  return launch_conv(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+
+extern "C" gdn_status gdn_conv_frontend(
+    const void* q, const void* k, const void* v, const float* conv_w,
+    const float* conv_state_in, float* conv_state_out, const int32_t* cu_seqlens, int32_t n_seq,
+    int64_t total_T, int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v, gdn_dtype in_dtype,
+    void* q_out, void* k_out, void* v_out, gdn_stream_t stream) {
+  return conv_impl(q, k, v, conv_w, conv_state_in, conv_state_out, cu_seqlens, n_seq, total_T,
+                   H_qk, H_v, d_k, d_v, in_dtype, q_out, k_out, v_out, stream);
+}
+
+extern "C" size_t gdn_chunk_fwd_conv_workspace_size(int32_t n_seq, int64_t total_T,
+                                                    int32_t H_qk, int32_t H_v, int32_t d_k,
+                                                    int32_t d_v, gdn_dtype in_dtype) {
+  if (n_seq < 1 || total_T < 0 || H_qk < 1 || H_v < 1 || H_v % H_qk != 0) return 0;
+  if (!dim_ok(d_k) || !dim_ok(d_v) || (in_dtype != GDN_BF16 && in_dtype != GDN_FP32)) return 0;
+  return conv_buffers_bytes(total_T, H_qk, H_v, d_k, d_v, in_dtype) +
+         prefill_tc_workspace_bytes(n_seq, H_v, d_k, d_v, in_dtype);
+}
+
+extern "C" gdn_status gdn_chunk_fwd_conv(
+    const void* q, const void* k, const void* v, const float* conv_w,
+    const float* conv_state_in, float* conv_state_out, const float* log_alpha,
+    const float* beta, const void* g, const float* norm_w, const float* initial_state,
+    const int32_t* cu_seqlens, int32_t n_seq, int64_t total_T, int32_t H_qk, int32_t H_v,
+    int32_t d_k, int32_t d_v, gdn_dtype in_dtype, int32_t l2norm_qk, float eps_l2,
+    float eps_norm, float scale, void* y, float* final_state, gdn_prefill_path path,
+    void* workspace, size_t workspace_bytes, gdn_stream_t stream) {
+  gdn_status st = check_common(H_qk, H_v, d_k, d_v, in_dtype, eps_l2, eps_norm);
+  if (st != GDN_OK) return st;
+  if (n_seq < 1 || total_T < 0) return GDN_ERR_INVALID_ARG;
+  const size_t need = gdn_chunk_fwd_conv_workspace_size(n_seq, total_T, H_qk, H_v, d_k, d_v,
+                                                        in_dtype);
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+      workspace_bytes < need)
+    return GDN_ERR_INVALID_ARG;
+  // the front end's outputs first in the workspace, the prefill's part after
+  const size_t e = in_dtype == GDN_BF16 ? 2 : 4;
+  auto a256 = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  char* p = static_cast<char*>(workspace);
+  void* qc = p;
+  void* kc = p + a256((size_t)total_T * H_qk * d_k * e);
+  void* vc = p + 2 * a256((size_t)total_T * H_qk * d_k * e);
+  const size_t cbytes = conv_buffers_bytes(total_T, H_qk, H_v, d_k, d_v, in_dtype);
+  const size_t pbytes = prefill_tc_workspace_bytes(n_seq, H_v, d_k, d_v, in_dtype);
+  st = conv_impl(q, k, v, conv_w, conv_state_in, conv_state_out, cu_seqlens, n_seq, total_T,
+                 H_qk, H_v, d_k, d_v, in_dtype, total_T > 0 ? qc : nullptr,
+                 total_T > 0 ? kc : nullptr, total_T > 0 ? vc : nullptr, stream);
+  if (st != GDN_OK) return st;
+  return gdn_chunk_fwd_ws(qc, kc, vc, log_alpha, beta, g, norm_w, initial_state, cu_seqlens,
+                          n_seq, total_T, H_qk, H_v, d_k, d_v, in_dtype, l2norm_qk, eps_l2,
+                          eps_norm, scale, y, final_state, path,
+                          pbytes > 0 ? p + cbytes : nullptr, pbytes, stream);
 }
 
 extern "C" gdn_status gdn_decode_step(const void* q, const void* k, const void* v,

@@ -210,6 +210,42 @@ __global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT)
   }
   float4 w4 = make_float4(0.f, 0.f, 0.f, 0.f);
   if (has_g && a.norm_w) w4 = __ldg(reinterpret_cast<const float4*>(a.norm_w + 4 * c4));
+  if (a.conv_w != nullptr) {
+    // front end: causal depthwise conv of kernel 4, then SiLU, over each
+    // q / k / v channel of this (sequence, value head), in place on the
+    // staged inputs; the three inputs before the first token come from this
+    // value head's conv state, which is then rewritten with the last three
+    __syncthreads();  // raw inputs staged
+    constexpr int SROW = 2 * DK + DV;
+    float* cst = a.conv_state ? a.conv_state + ((size_t)n * a.H_v + h) * 3 * SROW : nullptr;
+    for (int c = tid; c < SROW; c += NT) {
+      float* col;
+      int stride, wrow;
+      if (c < DK) {
+        col = tq + c; stride = DK; wrow = hq * DK + c;
+      } else if (c < 2 * DK) {
+        col = tk + (c - DK); stride = DK; wrow = (a.H_qk + hq) * DK + (c - DK);
+      } else {
+        col = tv + (c - 2 * DK); stride = DV; wrow = 2 * a.H_qk * DK + h * DV + (c - 2 * DK);
+      }
+      const float4 cw = __ldg(reinterpret_cast<const float4*>(a.conv_w) + wrow);
+      float x3 = cst ? cst[c] : 0.f, x2 = cst ? cst[SROW + c] : 0.f,
+            x1 = cst ? cst[2 * SROW + c] : 0.f;  // inputs 3, 2, 1 tokens back
+      for (int t = 0; t < T_s; ++t) {
+        const float x = col[t * stride];
+        const float u = cw.w * x + cw.z * x1 + cw.y * x2 + cw.x * x3;
+        col[t * stride] = u / (1.f + __expf(-u));
+        x3 = x2;
+        x2 = x1;
+        x1 = x;
+      }
+      if (cst) {
+        cst[c] = x3;
+        cst[SROW + c] = x2;
+        cst[2 * SROW + c] = x1;
+      }
+    }
+  }
   __syncthreads();
 
   for (int t = 0; t < T_s; ++t) {
@@ -306,7 +342,8 @@ size_t multi_smem_bytes(int T_s, bool has_g) {
 template <int DK, int DV, typename Tin>
 gdn_status launch(const DecodeArgs& a, cudaStream_t stream) {
   const unsigned grid = (unsigned)a.N * (unsigned)a.H_v;
-  const bool single = a.T_s == 1 && a.snapshots == nullptr && a.state_out == a.state_in;
+  const bool single = a.T_s == 1 && a.snapshots == nullptr && a.state_out == a.state_in &&
+                      a.conv_w == nullptr;
   if (single)
     gdn_decode_kernel<DK, DV, Tin><<<grid, DecodeGeom<DK, DV>::NT, 0, stream>>>(a);
   else {

@@ -57,6 +57,8 @@ struct DecodeArgs {
   float* state_out;        // same shape, may be state_in; nullptr: not written
   float* snapshots;        // [T_s, N, H_v, d_k, d_v] or nullptr: state after each token
   void* y;                 // [N, T_s, H_v, d_v]
+  const float* conv_w = nullptr;  // [2 H_qk d_k + H_v d_v, 4]: q, k, v pass the front end
+  float* conv_state = nullptr;    // [N, H_v, 3, 2 d_k + d_v], read and rewritten; nullptr: zeros
   int32_t N, T_s, H_qk, H_v, d_k, d_v;
   gdn_dtype dtype;
   int32_t l2norm;
@@ -96,6 +98,26 @@ struct BwdArgs {
   float *S, *dS, *W, *UT, *D, *dD, *T, *KKE, *P, *dPE, *Bm, *G, *row, *dw, *dO, *dqh, *dkh,
       *qh, *kh;
 };
+
+struct ConvArgs {
+  const void* q;               // [total_T, H_qk, d_k] input dtype (before the front end)
+  const void* k;
+  const void* v;               // [total_T, H_v, d_v]
+  const float* conv_w;         // [2 H_qk d_k + H_v d_v, 4]
+  const float* state_in;       // [n_seq, H_v, 3, 2 d_k + d_v] or nullptr (zeros)
+  float* state_out;            // same shape or nullptr; must not overlap state_in
+  const int32_t* cu_seqlens;   // nullptr: one sequence
+  int32_t n_seq;
+  int64_t total_T;
+  int32_t H_qk, H_v, d_k, d_v;
+  gdn_dtype dtype;
+  void* q_out;                 // outputs, input dtype, shapes of q, k, v
+  void* k_out;
+  void* v_out;
+  int* err;
+};
+
+gdn_status launch_conv(const ConvArgs& a, cudaStream_t stream);
 
 size_t chunk_bwd_workspace_bytes(int32_t n_seq, int64_t total_T, int32_t H_qk, int32_t H_v,
                                  int32_t d_k, int32_t d_v);

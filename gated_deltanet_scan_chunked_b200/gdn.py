@@ -82,6 +82,22 @@ def load(path: str = LIB_PATH):
     f.argtypes = [_vp] * 9 + [ctypes.c_int32, ctypes.c_int64] + [ctypes.c_int32] * 5 + [
         ctypes.c_int32, ctypes.c_float, ctypes.c_float, ctypes.c_float] + [_vp] * 10 + [
         _vp, ctypes.c_size_t, _vp]
+    f = lib.gdn_conv_frontend
+    f.restype = ctypes.c_int
+    f.argtypes = [_vp] * 7 + [ctypes.c_int32, ctypes.c_int64] + [ctypes.c_int32] * 5 + [
+        _vp, _vp, _vp, _vp]
+    f = lib.gdn_chunk_fwd_conv_workspace_size
+    f.restype = ctypes.c_size_t
+    f.argtypes = [ctypes.c_int32, ctypes.c_int64] + [ctypes.c_int32] * 4 + [ctypes.c_int]
+    f = lib.gdn_chunk_fwd_conv
+    f.restype = ctypes.c_int
+    f.argtypes = [_vp] * 12 + [ctypes.c_int32, ctypes.c_int64] + [ctypes.c_int32] * 5 + [
+        ctypes.c_int32, ctypes.c_float, ctypes.c_float, ctypes.c_float, _vp, _vp,
+        ctypes.c_int, _vp, ctypes.c_size_t, _vp]
+    f = lib.gdn_decode_conv
+    f.restype = ctypes.c_int
+    f.argtypes = [_vp] * 12 + [ctypes.c_int32] * 7 + [
+        ctypes.c_int32, ctypes.c_float, ctypes.c_float, ctypes.c_float, _vp, _vp]
     lib.gdn_check_device_error.restype = ctypes.c_int
     lib.gdn_check_device_error.argtypes = [_vp]
     lib.gdn_status_string.restype = ctypes.c_char_p
@@ -358,6 +374,134 @@ def gdn_decode_multi(q, k, v, log_alpha, beta, state_in, state_out="in_place",
         _stream_handle(stream))
     if st != GDN_OK:
         raise GdnError(st, "gdn_decode_multi")
+    return y, snapshots
+
+
+def conv_state_shape(n_seq: int, H_v: int, d_k: int, d_v: int):
+    """Shape of the carried conv state: [n_seq, H_v, 3, 2 d_k + d_v]."""
+    return (n_seq, H_v, 3, 2 * d_k + d_v)
+
+
+def gdn_conv_frontend(q, k, v, conv_w, conv_state_in=None, cu_seqlens=None,
+                      conv_state_out=True, out=None, stream=None):
+    """Causal depthwise conv (kernel 4) + SiLU over q, k, v (pre-conv, shapes
+    as gdn_chunk_fwd).  conv_w [2 H_qk d_k + H_v d_v, 4] fp32 (channels q |
+    k | v); conv_state_in [n_seq, H_v, 3, 2 d_k + d_v] fp32 or None;
+    conv_state_out: True (allocated here), a tensor, or None (not written).
+    Returns (q', k', v', conv_state_out)."""
+    lib = load()
+    dev = q.device
+    dt = _dtype_code(q)
+    T, Hqk, dk = q.shape
+    Hv, dv = v.shape[1], v.shape[2]
+    n_seq = 1 if cu_seqlens is None else int(cu_seqlens.shape[0]) - 1
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check(t, name, q.dtype, dev)
+    if conv_state_out is True:
+        conv_state_out = torch.empty(conv_state_shape(n_seq, Hv, dk, dv), dtype=torch.float32,
+                                     device=dev)
+    for name, t in (("conv_w", conv_w), ("conv_state_in", conv_state_in),
+                    ("conv_state_out", conv_state_out)):
+        _check(t, name, torch.float32, dev)
+    _check(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    qo, ko, vo = out if out is not None else (torch.empty_like(q), torch.empty_like(k),
+                                              torch.empty_like(v))
+    st = lib.gdn_conv_frontend(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(conv_w), _ptr(conv_state_in), _ptr(conv_state_out),
+        _ptr(cu_seqlens), n_seq, T, Hqk, Hv, dk, dv, dt, _ptr(qo), _ptr(ko), _ptr(vo),
+        _stream_handle(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_conv_frontend")
+    return qo, ko, vo, conv_state_out
+
+
+def conv_workspace_size(n_seq: int, total_T: int, H_qk: int, H_v: int, d_k: int, d_v: int,
+                        dtype=torch.bfloat16) -> int:
+    """Bytes of workspace gdn_chunk_fwd_conv needs (0: never accepted)."""
+    return int(load().gdn_chunk_fwd_conv_workspace_size(n_seq, total_T, H_qk, H_v, d_k, d_v,
+                                                        _dtype_code_of(dtype)))
+
+
+def gdn_chunk_fwd_conv(q, k, v, conv_w, log_alpha, beta, conv_state_in=None,
+                       conv_state_out=True, g=None, norm_w=None, initial_state=None,
+                       cu_seqlens=None, l2norm_qk=True, eps_l2=1e-6, eps_norm=1e-6,
+                       scale=1.0, y=None, final_state=None, output_final_state=True,
+                       path="auto", workspace=None, stream=None):
+    """Prefill on pre-conv q, k, v: the front end, then gdn_chunk_fwd.
+    Returns (y, final_state, conv_state_out).  ``workspace``: a uint8 CUDA
+    tensor of at least conv_workspace_size(...) bytes, or None (allocated)."""
+    lib = load()
+    dev = q.device
+    dt = _dtype_code(q)
+    T, Hqk, dk = q.shape
+    Hv, dv = v.shape[1], v.shape[2]
+    n_seq = 1 if cu_seqlens is None else int(cu_seqlens.shape[0]) - 1
+    for name, t in (("q", q), ("k", k), ("v", v), ("g", g)):
+        _check(t, name, q.dtype, dev)
+    if conv_state_out is True:
+        conv_state_out = torch.empty(conv_state_shape(n_seq, Hv, dk, dv), dtype=torch.float32,
+                                     device=dev)
+    for name, t in (("conv_w", conv_w), ("conv_state_in", conv_state_in),
+                    ("conv_state_out", conv_state_out), ("log_alpha", log_alpha),
+                    ("beta", beta), ("norm_w", norm_w), ("initial_state", initial_state)):
+        _check(t, name, torch.float32, dev)
+    _check(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    if y is None:
+        y = torch.empty((T, Hv, dv), dtype=q.dtype, device=dev)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((n_seq, Hv, dk, dv), dtype=torch.float32, device=dev)
+    _check(y, "y", q.dtype, dev)
+    _check(final_state, "final_state", torch.float32, dev)
+    nbytes = int(lib.gdn_chunk_fwd_conv_workspace_size(n_seq, T, Hqk, Hv, dk, dv, dt))
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
+    _check(workspace, "workspace", torch.uint8, dev)
+    st = lib.gdn_chunk_fwd_conv(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(conv_w), _ptr(conv_state_in), _ptr(conv_state_out),
+        _ptr(log_alpha), _ptr(beta), _ptr(g), _ptr(norm_w), _ptr(initial_state),
+        _ptr(cu_seqlens), n_seq, T, Hqk, Hv, dk, dv, dt, 1 if l2norm_qk else 0,
+        float(eps_l2), float(eps_norm), float(scale), _ptr(y), _ptr(final_state), PATHS[path],
+        _ptr(workspace), workspace.numel(), _stream_handle(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_chunk_fwd_conv")
+    return y, final_state, conv_state_out
+
+
+def gdn_decode_conv(q, k, v, conv_w, log_alpha, beta, state_in, conv_state,
+                    state_out="in_place", snapshots=None, g=None, norm_w=None,
+                    l2norm_qk=True, eps_l2=1e-6, eps_norm=1e-6, scale=1.0, y=None,
+                    stream=None):
+    """gdn_decode_multi on pre-conv q, k, v with the front end fused: q, k
+    [N, T_s, H_qk, d_k]; v [N, T_s, H_v, d_v]; conv_state [N, H_v, 3,
+    2 d_k + d_v] fp32, updated in place (None: zeros, not written).  Returns
+    (y, snapshots)."""
+    lib = load()
+    dev = q.device
+    dt = _dtype_code(q)
+    N, T_s, Hqk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    for name, t in (("q", q), ("k", k), ("v", v), ("g", g)):
+        _check(t, name, q.dtype, dev)
+    if isinstance(state_out, str):
+        if state_out != "in_place":
+            raise ValueError("state_out must be a tensor, None or 'in_place'")
+        state_out = state_in
+    if snapshots is True:
+        snapshots = torch.empty((T_s, N, Hv, dk, dv), dtype=torch.float32, device=dev)
+    for name, t in (("conv_w", conv_w), ("conv_state", conv_state), ("log_alpha", log_alpha),
+                    ("beta", beta), ("norm_w", norm_w), ("state_in", state_in),
+                    ("state_out", state_out), ("snapshots", snapshots)):
+        _check(t, name, torch.float32, dev)
+    if y is None:
+        y = torch.empty((N, T_s, Hv, dv), dtype=q.dtype, device=dev)
+    _check(y, "y", q.dtype, dev)
+    st = lib.gdn_decode_conv(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(conv_w), _ptr(conv_state), _ptr(log_alpha),
+        _ptr(beta), _ptr(g), _ptr(norm_w), _ptr(state_in), _ptr(state_out), _ptr(snapshots),
+        N, T_s, Hqk, Hv, dk, dv, dt, 1 if l2norm_qk else 0, float(eps_l2), float(eps_norm),
+        float(scale), _ptr(y), _stream_handle(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_decode_conv")
     return y, snapshots
 
 

@@ -154,6 +154,26 @@ def make_cotangents(w: PrefillInputs, seed=0, ds_std=0.5, final_grad=True):
     return dy, dsT
 
 
+def make_conv_params(n_seq, H_qk, H_v, d_k, d_v, seed=0, w_std=0.5, state=True,
+                     device="cpu"):
+    """Seeded front-end parameters: conv_w ~ N(0, w_std^2) fp32
+    [2 H_qk d_k + H_v d_v, 4] and, if ``state``, a carried conv state
+    ~ N(0, 1) fp32 [n_seq, H_v, 3, 2 d_k + d_v] whose q/k part is the same
+    in every value head of a group (as the library keeps it)."""
+    gen = _gen(int(seed) + 77, device)
+    C = 2 * H_qk * d_k + H_v * d_v
+    w = torch.randn((C, 4), generator=gen, dtype=torch.float32, device=device) * w_std
+    st = None
+    if state:
+        G = H_v // H_qk
+        qk = torch.randn((n_seq, H_qk, 3, 2 * d_k), generator=gen, dtype=torch.float32,
+                         device=device)
+        vv = torch.randn((n_seq, H_v, 3, d_v), generator=gen, dtype=torch.float32,
+                         device=device)
+        st = torch.cat([qk.repeat_interleave(G, dim=1), vv], dim=3).contiguous()
+    return w, st
+
+
 def varlen_lengths(n_seq=24, lo=512, hi=16384, seed=SEEDS["varlen"]):
     """Sequence lengths drawn uniformly from the integers [lo, hi]."""
     gen = torch.Generator().manual_seed(int(seed) + 7)

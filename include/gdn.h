@@ -251,6 +251,90 @@ gdn_status gdn_decode_multi(
     float scale, void* y, gdn_stream_t stream);
 
 /*
+ * Front end of the mixer: a short depthwise causal convolution over time
+ * (kernel 4) followed by SiLU, applied channel by channel to q, k and v
+ * before the gated delta rule ("Qwen3.8-Flash-Next: architecture, efficiency
+ * and technical lineage", section 02 module table, GDN row: Q/K/V pass a
+ * short causal conv of kernel 4; hyper.ai summary, "Method": projections
+ * followed by short depthwise causal convolutions; "On the Design of
+ * Qwen3.8-Next Architecture ... close reading", section 4.1: short conv +
+ * SiLU + L2 norm).  Per channel, with w[c][3] the weight of the current
+ * token: u_t = w3 x_t + w2 x_{t-1} + w1 x_{t-2} + w0 x_{t-3} (no bias), and
+ * the output is u_t * sigmoid(u_t).  SiLU on v as well as on q and k is a
+ * reading: the pages name the activation for q and k only.
+ *
+ * Shared conventions of the calls below:
+ *   conv_w      [2 H_qk d_k + H_v d_v, 4] fp32; channels numbered q (head
+ *               major, H_qk d_k of them), then k, then v (H_v d_v)
+ *   conv state  [n_seq (or N), H_v, 3, 2 d_k + d_v] fp32: for value head h,
+ *               the three inputs before the next token (oldest first) of its
+ *               QK head's q channels, k channels, then its own v channels.
+ *               The q/k part is repeated in each value head of a group (all
+ *               copies equal), so one value head's slice can be rewritten in
+ *               place by the kernel that owns it.  NULL input = zeros.
+ */
+
+/*
+ * gdn_conv_frontend -- the front end alone over a packed batch.
+ *   q, k, v            pre-conv inputs, shapes and dtype as gdn_chunk_fwd's
+ *   conv_state_in      the state before each sequence, or NULL (zeros)
+ *   conv_state_out     the state after each sequence (its last three inputs,
+ *                      earlier ones from conv_state_in for sequences shorter
+ *                      than three), or NULL; must not overlap conv_state_in
+ *   q_out, k_out, v_out  outputs, same shapes and dtype; must not overlap
+ *                      the inputs
+ * HBM-bound: every element read once and written once.
+ */
+gdn_status gdn_conv_frontend(
+    const void* q, const void* k, const void* v, const float* conv_w,
+    const float* conv_state_in, float* conv_state_out, const int32_t* cu_seqlens,
+    int32_t n_seq, int64_t total_T, int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v,
+    gdn_dtype in_dtype, void* q_out, void* k_out, void* v_out, gdn_stream_t stream);
+
+/* Workspace bytes gdn_chunk_fwd_conv needs (0 for arguments it never accepts):
+ * the front end's outputs plus gdn_chunk_fwd_workspace_size(...). */
+size_t gdn_chunk_fwd_conv_workspace_size(int32_t n_seq, int64_t total_T, int32_t H_qk,
+                                         int32_t H_v, int32_t d_k, int32_t d_v,
+                                         gdn_dtype in_dtype);
+
+/*
+ * gdn_chunk_fwd_conv -- gdn_chunk_fwd_ws on pre-conv q, k, v: the front end
+ * (gdn_conv_frontend, written into the workspace in the input dtype), then
+ * the chunked prefill on its outputs (the L2 norm of q and k, when
+ * l2norm_qk, follows the SiLU).  conv_state_in / conv_state_out as for
+ * gdn_conv_frontend; everything else as for gdn_chunk_fwd_ws.  The workspace
+ * (256-byte aligned, at least gdn_chunk_fwd_conv_workspace_size bytes) is
+ * required.
+ */
+gdn_status gdn_chunk_fwd_conv(
+    const void* q, const void* k, const void* v, const float* conv_w,
+    const float* conv_state_in, float* conv_state_out, const float* log_alpha,
+    const float* beta, const void* g, const float* norm_w, const float* initial_state,
+    const int32_t* cu_seqlens, int32_t n_seq, int64_t total_T, int32_t H_qk, int32_t H_v,
+    int32_t d_k, int32_t d_v, gdn_dtype in_dtype, int32_t l2norm_qk, float eps_l2,
+    float eps_norm, float scale, void* y, float* final_state, gdn_prefill_path path,
+    void* workspace, size_t workspace_bytes, gdn_stream_t stream);
+
+/*
+ * gdn_decode_conv -- gdn_decode_multi on pre-conv q, k, v with the front end
+ * fused into the decode kernel: each (sequence, value head) convolves its
+ * staged q/k/v channels with its slice of conv_state ([N, H_v, 3,
+ * 2 d_k + d_v], read, then rewritten in place with the last three inputs;
+ * NULL = zeros, not written), applies SiLU, then runs the T_s decode steps.
+ * conv_w is required and is laid out as for gdn_conv_frontend; conv_state
+ * must not overlap state_in, state_out or snapshots.  Other arguments as for
+ * gdn_decode_multi.  Continues a gdn_chunk_fwd_conv prefill exactly (same
+ * state layouts).
+ */
+gdn_status gdn_decode_conv(
+    const void* q, const void* k, const void* v, const float* conv_w, float* conv_state,
+    const float* log_alpha, const float* beta, const void* g, const float* norm_w,
+    const float* state_in, float* state_out, float* snapshots, int32_t N, int32_t T_s,
+    int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v, gdn_dtype in_dtype,
+    int32_t l2norm_qk, float eps_l2, float eps_norm, float scale, void* y,
+    gdn_stream_t stream);
+
+/*
  * gdn_chunk_bwd_workspace_size -- bytes of device workspace gdn_chunk_bwd
  * needs for a packed batch (0 for arguments it can never accept).  About
  * 460 KB per 64-token chunk per value head at d_k = d_v = 128 (chunk states

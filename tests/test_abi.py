@@ -216,3 +216,49 @@ def test_bwd_workspace_size(lib):
 ])
 def test_chunk_bwd_rejects_bad_arguments_on_host(lib, kw, code):
     assert _bwd(lib, **kw) == code
+
+
+def test_conv_entry_points_reject_on_host(lib):
+    """Front-end calls: overlapping conv states, missing weights, outputs on
+    top of inputs, a missing or short workspace are refused on the host."""
+    C4 = (2 * 16 * 128 + 48 * 128) * 16  # bytes of conv_w
+    ns = 2 * 48 * 3 * 384 * 4            # bytes of a 2-sequence conv state
+
+    def fe(**kw):
+        a = dict(q=FAKE, k=FAKE + (1 << 24), v=FAKE + (2 << 24), w=FAKE + (3 << 24), si=None,
+                 so=None, cu=FAKE + (4 << 24), n_seq=2, T=64, dk=128, qo=FAKE + (5 << 24),
+                 ko=FAKE + (6 << 24), vo=FAKE + (7 << 24))
+        a.update(kw)
+        return lib.gdn_conv_frontend(a["q"], a["k"], a["v"], a["w"], a["si"], a["so"], a["cu"],
+                                     a["n_seq"], a["T"], 16, 48, a["dk"], 128, 0, a["qo"],
+                                     a["ko"], a["vo"], None)
+    S = FAKE + (8 << 24)
+    assert fe(w=None) == gdn.GDN_ERR_INVALID_ARG
+    assert fe(si=S, so=S) == gdn.GDN_ERR_INVALID_ARG              # in place is refused
+    assert fe(si=S, so=S + ns - 256) == gdn.GDN_ERR_INVALID_ARG   # partial overlap
+    assert fe(qo=FAKE) == gdn.GDN_ERR_INVALID_ARG                 # output on its input
+    assert fe(vo=FAKE + (1 << 24) + 64) == gdn.GDN_ERR_INVALID_ARG  # output inside k
+    assert fe(dk=96) == gdn.GDN_ERR_UNSUPPORTED
+    assert C4 > 0
+
+    n = gdn.conv_workspace_size(2, 64, 16, 48, 128, 128)
+    assert n >= 64 * (2 * 16 * 128 + 48 * 128) * 2
+    assert gdn.conv_workspace_size(2, 64, 16, 48, 96, 128) == 0
+
+    def cf(ws, wsb):
+        return lib.gdn_chunk_fwd_conv(FAKE, FAKE, FAKE, FAKE, None, None, FAKE, FAKE, None, None,
+                                      None, FAKE, 2, 64, 16, 48, 128, 128, 0, 1, 1e-6, 1e-6,
+                                      1.0, FAKE, None, 0, ws, wsb, None)
+    assert cf(None, 0) == gdn.GDN_ERR_INVALID_ARG
+    assert cf(S, n - 256) == gdn.GDN_ERR_INVALID_ARG
+    assert cf(S + 16, n) == gdn.GDN_ERR_INVALID_ARG
+
+    def dc(**kw):
+        a = dict(w=FAKE, cs=S, si=FAKE + (9 << 24), so=FAKE + (9 << 24), sn=None)
+        a.update(kw)
+        return lib.gdn_decode_conv(FAKE, FAKE, FAKE, a["w"], a["cs"], FAKE, FAKE, None, None,
+                                   a["si"], a["so"], a["sn"], 4, 2, 16, 48, 128, 128, 0, 1,
+                                   1e-6, 1e-6, 1.0, FAKE, None)
+    assert dc(w=None) == gdn.GDN_ERR_INVALID_ARG
+    assert dc(cs=FAKE + (9 << 24) + 4096) == gdn.GDN_ERR_INVALID_ARG  # inside the state
+    assert dc(cs=S + 8) == gdn.GDN_ERR_INVALID_ARG                     # misaligned
