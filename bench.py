@@ -3,7 +3,8 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload prefill4k|prefill256k|varlen]
                     [--path auto|tensor|tensor_pair|tensor_single|tensor_split|simt]
-                    [--no-decode] [--no-backward] [--no-cpu-baseline]
+                    [--no-decode] [--no-backward] [--no-front-end]
+                    [--no-cpu-baseline]
 
 One step = one chunked prefill (gdn_chunk_fwd: L2-norm prologue, gate cumsum,
 intra-chunk products, triangular solve, state carry, RMSNorm x sigmoid(g)
@@ -12,8 +13,9 @@ value heads, d=128, bf16).  The call gets a preallocated workspace, so small
 batches may take the split layout (one kernel, after an asynchronous memset of
 the workspace flags).  The JSON line also carries the decode step
 (gdn_decode_step, 256 sequences x 64 steps, in place) and the backward of the
-model-shape prefill (gdn_chunk_bwd, T=4096) as separate objects with their
-own timing, roofline and clocks.
+model-shape prefill (gdn_chunk_bwd, T=4096) and the conv + SiLU front end
+(alone, ahead of the prefill, and fused into a 4-token decode) as separate
+objects with their own timing, roofline and clocks.
 
 Multi-GPU (torchrun, one process per GPU): every rank runs its own
 independent batch (weak scaling; sequences and heads are independent, so the
@@ -562,6 +564,85 @@ def run_ours(args, world, rank, local):
         launches_bwd = bsteps * (10 if wb.g is not None else 9)
         del bws, bflush
 
+    # the front end (causal conv of kernel 4 + SiLU): alone, in front of the
+    # model-shape prefill, and fused into the multi-token decode
+    front = None
+    launches_front = 0
+    if not args.no_front_end:
+        from gated_deltanet_scan_chunked_b200 import (gdn_chunk_fwd_conv, gdn_conv_frontend,
+                                                      gdn_decode_conv)
+        wf = inputs.workload("prefill4k", device="cuda")
+        Tf = wf.q.shape[0]
+        cw, cst = inputs.make_conv_params(1, H_QK, H_V, D, D, seed=inputs.SEEDS["prefill4k"],
+                                          device="cuda")
+        cso = torch.empty_like(cst)
+        outs = (torch.empty_like(wf.q), torch.empty_like(wf.k), torch.empty_like(wf.v))
+        fflush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
+        fclk = ClockSampler(local)
+        fclk.start()
+        fsteps = max(3, args.steps // 2)
+        # the conv kernel takes less time than the Python call that launches
+        # it: time it as a CUDA graph replay so that host overhead stays out
+        conv_call = lambda: gdn_conv_frontend(wf.q, wf.k, wf.v, cw, cst, conv_state_out=cso,
+                                              out=outs)
+        for _ in range(3):
+            conv_call()
+        torch.cuda.synchronize()
+        cgraph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(cgraph):
+            conv_call()
+        ct = timed_steps(cgraph.replay, fsteps, 3, world, flush=lambda: fflush.zero_(),
+                         stream=stream)
+        cms = max_over_ranks(statistics.mean(ct), world)
+        cbytes = 2 * Tf * (2 * H_QK * D + H_V * D) * 2 + 2 * H_V * 3 * (3 * D) * 4
+        cws = torch.empty(gdn.conv_workspace_size(1, Tf, H_QK, H_V, D, D), dtype=torch.uint8,
+                          device="cuda")
+        yf = torch.empty_like(wf.v)
+        fsf = torch.empty((1, H_V, D, D), dtype=torch.float32, device="cuda")
+        pt = timed_steps(lambda: gdn_chunk_fwd_conv(wf.q, wf.k, wf.v, cw, wf.log_alpha, wf.beta,
+                                                    conv_state_in=cst, conv_state_out=cso,
+                                                    g=wf.g, norm_w=wf.norm_w, y=yf,
+                                                    final_state=fsf, workspace=cws),
+                         fsteps, 3, world, flush=lambda: fflush.zero_(), stream=stream)
+        pms = max_over_ranks(statistics.mean(pt), world)
+        del cws, fflush, cgraph
+        # decode with the front end fused: 256 sequences x 4 tokens per launch, in place
+        dd = inputs.make_decode(steps=4, device="cuda", seed=inputs.SEEDS["decode"] + 7)
+        Nd = dd.q.shape[1]
+        tr = lambda x: x.transpose(0, 1).contiguous()
+        dq, dk_, dv_, dla, db = tr(dd.q), tr(dd.k), tr(dd.v), tr(dd.log_alpha), tr(dd.beta)
+        dcw, dcst = inputs.make_conv_params(Nd, H_QK, H_V, D, D, seed=3, device="cuda")
+        dstate0 = dd.state.clone()
+        ydc = torch.empty((Nd, 4, H_V, D), dtype=torch.bfloat16, device="cuda")
+        dct = timed_steps(lambda: gdn_decode_conv(dq, dk_, dv_, dcw, dla, db, dd.state, dcst,
+                                                  y=ydc),
+                          fsteps, 3, world, flush=lambda: dd.state.copy_(dstate0), stream=stream)
+        fclk_r = fclk.stop()
+        err = gdn.gdn_check_device_error()
+        if err != gdn.GDN_OK:
+            raise RuntimeError("device error in the front end: %s" % gdn.status_string(err))
+        dcms = max_over_ranks(statistics.mean(dct), world)
+        dcbytes = (Nd * 2 * H_V * D * D * 4 + 4 * (decode_bytes(Nd) - Nd * 2 * H_V * D * D * 4)
+                   + 2 * Nd * H_V * 3 * 3 * D * 4)
+        front = {
+            "workload": "front end at the model shape: q, k, v of T=4096 (16 QK / 48 value "
+                        "heads, d=128, bf16), conv state carried; decode: 256 sequences x 4 "
+                        "tokens per launch with the front end fused, in place",
+            "conv_us": cms * 1e3, "conv_timing": "CUDA graph replay of one call",
+            "conv_roofline": {"bound": "hbm", "achieved": cbytes / (cms * 1e-3) / 1e9,
+                              "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                              "frac": cbytes / (cms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                              "algorithmic_bytes": cbytes, "traffic": None},
+            "prefill_with_front_end_ms": pms,
+            "prefill_with_front_end_tokens_per_s": world * Tf / (pms * 1e-3),
+            "decode_conv_us_per_launch": dcms * 1e3,
+            "decode_conv_roofline": {"bound": "hbm", "achieved": dcbytes / (dcms * 1e-3) / 1e9,
+                                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                     "frac": dcbytes / (dcms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                     "algorithmic_bytes": dcbytes},
+            "clocks": fclk_r}
+        launches_front = fsteps * (1 + 2 + 1)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, target_s=args.ref_seconds)
@@ -579,7 +660,8 @@ def run_ours(args, world, rank, local):
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": args.steps, "clocks": clk, "decode": decode,
                 "gpu_launches_decode_region": launches_decode, "backward": backward,
-                "gpu_launches_backward_region": launches_bwd}
+                "gpu_launches_backward_region": launches_bwd, "front_end": front,
+                "gpu_launches_front_end_region": launches_front}
         print(json.dumps(line), flush=True)
 
 
@@ -596,6 +678,7 @@ def main():
                              "tensor_split"])
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--no-front-end", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-seconds", type=float, default=12.0)

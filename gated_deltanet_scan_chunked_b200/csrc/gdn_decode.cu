@@ -187,6 +187,28 @@ __global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT)
     const int i = rg + ROWG * r;
     s[r] = __ldcs(reinterpret_cast<const float4*>(Sin + (size_t)i * DV) + c4);
   }
+  // front end: this thread's channels' conv weights and carried inputs,
+  // fetched together with the state
+  constexpr int SROW = 2 * DK + DV;
+  constexpr int CPT = (SROW + NT - 1) / NT;  // channels per thread
+  float4 cwr[CPT];
+  float cxr[CPT][3];
+  float* cst = (a.conv_w && a.conv_state) ? a.conv_state + ((size_t)n * a.H_v + h) * 3 * SROW
+                                          : nullptr;
+  if (a.conv_w != nullptr) {
+#pragma unroll
+    for (int u = 0; u < CPT; ++u) {
+      const int c = tid + u * NT;
+      if (c < SROW) {
+        const int wrow = c < DK ? hq * DK + c
+                         : c < 2 * DK ? (a.H_qk + hq) * DK + (c - DK)
+                                      : 2 * a.H_qk * DK + h * DV + (c - 2 * DK);
+        cwr[u] = __ldg(reinterpret_cast<const float4*>(a.conv_w) + wrow);
+#pragma unroll
+        for (int r = 0; r < 3; ++r) cxr[u][r] = cst ? cst[r * SROW + c] : 0.f;
+      }
+    }
+  }
   {
     const Tin* Q = static_cast<const Tin*>(a.q);
     const Tin* K = static_cast<const Tin*>(a.k);
@@ -216,25 +238,18 @@ __global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT)
     // staged inputs; the three inputs before the first token come from this
     // value head's conv state, which is then rewritten with the last three
     __syncthreads();  // raw inputs staged
-    constexpr int SROW = 2 * DK + DV;
-    float* cst = a.conv_state ? a.conv_state + ((size_t)n * a.H_v + h) * 3 * SROW : nullptr;
-    for (int c = tid; c < SROW; c += NT) {
-      float* col;
-      int stride, wrow;
-      if (c < DK) {
-        col = tq + c; stride = DK; wrow = hq * DK + c;
-      } else if (c < 2 * DK) {
-        col = tk + (c - DK); stride = DK; wrow = (a.H_qk + hq) * DK + (c - DK);
-      } else {
-        col = tv + (c - 2 * DK); stride = DV; wrow = 2 * a.H_qk * DK + h * DV + (c - 2 * DK);
-      }
-      const float4 cw = __ldg(reinterpret_cast<const float4*>(a.conv_w) + wrow);
-      float x3 = cst ? cst[c] : 0.f, x2 = cst ? cst[SROW + c] : 0.f,
-            x1 = cst ? cst[2 * SROW + c] : 0.f;  // inputs 3, 2, 1 tokens back
+#pragma unroll
+    for (int u = 0; u < CPT; ++u) {
+      const int c = tid + u * NT;
+      if (c >= SROW) break;
+      float* col = c < DK ? tq + c : c < 2 * DK ? tk + (c - DK) : tv + (c - 2 * DK);
+      const int stride = c < 2 * DK ? DK : DV;
+      const float4 cw = cwr[u];
+      float x3 = cxr[u][0], x2 = cxr[u][1], x1 = cxr[u][2];  // inputs 3, 2, 1 tokens back
       for (int t = 0; t < T_s; ++t) {
         const float x = col[t * stride];
-        const float u = cw.w * x + cw.z * x1 + cw.y * x2 + cw.x * x3;
-        col[t * stride] = u / (1.f + __expf(-u));
+        const float uu = cw.w * x + cw.z * x1 + cw.y * x2 + cw.x * x3;
+        col[t * stride] = uu / (1.f + __expf(-uu));
         x3 = x2;
         x2 = x1;
         x1 = x;
