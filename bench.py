@@ -632,7 +632,7 @@ def run_ours(args, world, rank, local):
             "conv_roofline": {"bound": "hbm", "achieved": cbytes / (cms * 1e-3) / 1e9,
                               "peak": peaks["hbm_gbs"], "unit": "GB/s",
                               "frac": cbytes / (cms * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                              "algorithmic_bytes": cbytes, "traffic": None},
+                              "algorithmic_bytes": cbytes, "traffic": kernel_traffic("conv")},
             "prefill_with_front_end_ms": pms,
             "prefill_with_front_end_tokens_per_s": world * Tf / (pms * 1e-3),
             "decode_conv_us_per_launch": dcms * 1e3,
