@@ -6,9 +6,10 @@ seeded synthetic workloads; ``build`` compiles the library.
 """
 from .gdn import (GdnError, bwd_workspace_size, conv_workspace_size,  # noqa: F401
                   gdn_check_device_error, gdn_chunk_bwd, gdn_chunk_fwd, gdn_chunk_fwd_conv,
-                  gdn_conv_frontend, gdn_decode_conv, gdn_decode_multi, gdn_decode_step, load,
-                  workspace_size)
+                  gdn_conv_frontend, gdn_decode_conv, gdn_decode_multi, gdn_decode_step,
+                  gdn_gr_read, gdn_gr_write, load, workspace_size)
 
 __all__ = ["gdn_chunk_fwd", "gdn_chunk_bwd", "gdn_decode_step", "gdn_decode_multi",
-           "gdn_check_device_error", "gdn_conv_frontend", "gdn_chunk_fwd_conv", "gdn_decode_conv", "GdnError", "load",
+           "gdn_check_device_error", "gdn_conv_frontend", "gdn_chunk_fwd_conv", "gdn_decode_conv", "gdn_gr_read",
+           "gdn_gr_write", "GdnError", "load",
            "workspace_size", "bwd_workspace_size", "conv_workspace_size"]

@@ -386,6 +386,56 @@ extern "C" gdn_status gdn_chunk_bwd(
   return launch_chunk_bwd(a, reinterpret_cast<cudaStream_t>(stream));
 }
 
+namespace {
+
+gdn_status gr_check(int64_t T, int32_t n_r, int32_t d) {
+  if (T < 0 || n_r < 1 || n_r > kMaxGrBranches || d < 8 || d % 8 != 0) return GDN_ERR_INVALID_ARG;
+  if ((int64_t)n_r * d > (1 << 24)) return GDN_ERR_UNSUPPORTED;
+  return GDN_OK;
+}
+
+}  // namespace
+
+extern "C" size_t gdn_gr_read_workspace_size(int64_t T, int32_t n_r, int32_t d, int32_t rank) {
+  if (gr_check(T, n_r, d) != GDN_OK || rank < 8 || rank % 8 != 0) return 0;
+  return gr_read_workspace_bytes(T, n_r, d, rank);
+}
+
+extern "C" gdn_status gdn_gr_read(const uint8_t* codes, const float* scales, const float* gamma,
+                                  const void* W_d, const void* W_u, const void* W_w, int64_t T,
+                                  int32_t n_r, int32_t d, int32_t rank, float eps, void* x,
+                                  float* s, void* workspace, size_t workspace_bytes,
+                                  gdn_stream_t stream) {
+  gdn_status st = gr_check(T, n_r, d);
+  if (st != GDN_OK) return st;
+  if (rank < 8 || rank % 8 != 0 || !(eps >= 0.f)) return GDN_ERR_INVALID_ARG;
+  if (T > 0 && (!codes || !scales || !gamma || !W_d || !W_u || !W_w || !x || !s))
+    return GDN_ERR_INVALID_ARG;
+  const void* ptrs[] = {codes, scales, gamma, W_d, W_u, W_w, x, s};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+      workspace_bytes < gr_read_workspace_bytes(T, n_r, d, rank))
+    return GDN_ERR_INVALID_ARG;
+  GrArgs a;
+  a.codes = codes; a.scales = scales; a.gamma = gamma; a.W_d = W_d; a.W_u = W_u; a.W_w = W_w;
+  a.T = T; a.n_r = n_r; a.d = d; a.rank = rank; a.eps = eps; a.x = x; a.s = s;
+  return launch_gr_read(a, workspace, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" gdn_status gdn_gr_write(uint8_t* codes, float* scales, const void* y, const float* s,
+                                   int64_t T, int32_t n_r, int32_t d, gdn_stream_t stream) {
+  gdn_status st = gr_check(T, n_r, d);
+  if (st != GDN_OK) return st;
+  if (T > 0 && (!codes || !scales || !y || !s)) return GDN_ERR_INVALID_ARG;
+  const void* ptrs[] = {codes, scales, y, s};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
+  GrWriteArgs a;
+  a.codes = codes; a.scales = scales; a.y = y; a.s = s; a.T = T; a.n_r = n_r; a.d = d;
+  return launch_gr_write(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
 extern "C" gdn_status gdn_check_device_error(gdn_stream_t stream) {
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return GDN_ERR_CUDA;

@@ -2,6 +2,7 @@
 // kernel translation units.  Not installed; not part of the C ABI.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -118,6 +119,38 @@ struct ConvArgs {
 };
 
 gdn_status launch_conv(const ConvArgs& a, cudaStream_t stream);
+
+// Gated Residual read / write over an E4M3 residual state.
+constexpr int kMaxGrBranches = 8;
+
+struct GrArgs {
+  const uint8_t* codes;   // [T, n_r, d] E4M3
+  const float* scales;    // [T, n_r]
+  const float* gamma;     // [n_r, d]
+  const void* W_d;        // [rank, n_r d] bf16
+  const void* W_u;        // [n_r d, rank] bf16
+  const void* W_w;        // [n_r, n_r d] bf16
+  int64_t T;
+  int32_t n_r, d, rank;
+  float eps;
+  void* x;                // [T, d] bf16
+  float* s;               // [T, n_r]
+  __nv_bfloat16* rhat = nullptr;    // workspace: [T, n_r d]
+  __nv_bfloat16* logits = nullptr;  // workspace: [T, n_r d]
+};
+
+struct GrWriteArgs {
+  uint8_t* codes;         // [T, n_r, d], rewritten
+  float* scales;          // [T, n_r], rewritten
+  const void* y;          // [T, d] bf16
+  const float* s;         // [T, n_r]
+  int64_t T;
+  int32_t n_r, d;
+};
+
+size_t gr_read_workspace_bytes(int64_t T, int32_t n_r, int32_t d, int32_t rank);
+gdn_status launch_gr_read(GrArgs a, void* ws, cudaStream_t stream);
+gdn_status launch_gr_write(const GrWriteArgs& a, cudaStream_t stream);
 
 size_t chunk_bwd_workspace_bytes(int32_t n_seq, int64_t total_T, int32_t H_qk, int32_t H_v,
                                  int32_t d_k, int32_t d_v);

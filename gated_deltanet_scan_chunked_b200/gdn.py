@@ -98,6 +98,16 @@ def load(path: str = LIB_PATH):
     f.restype = ctypes.c_int
     f.argtypes = [_vp] * 12 + [ctypes.c_int32] * 7 + [
         ctypes.c_int32, ctypes.c_float, ctypes.c_float, ctypes.c_float, _vp, _vp]
+    f = lib.gdn_gr_read_workspace_size
+    f.restype = ctypes.c_size_t
+    f.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32]
+    f = lib.gdn_gr_read
+    f.restype = ctypes.c_int
+    f.argtypes = [_vp] * 6 + [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                              ctypes.c_float, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+    f = lib.gdn_gr_write
+    f.restype = ctypes.c_int
+    f.argtypes = [_vp] * 4 + [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, _vp]
     lib.gdn_check_device_error.restype = ctypes.c_int
     lib.gdn_check_device_error.argtypes = [_vp]
     lib.gdn_status_string.restype = ctypes.c_char_p
@@ -503,6 +513,55 @@ def gdn_decode_conv(q, k, v, conv_w, log_alpha, beta, state_in, conv_state,
     if st != GDN_OK:
         raise GdnError(st, "gdn_decode_conv")
     return y, snapshots
+
+
+def gr_read_workspace_size(T: int, n_r: int, d: int, rank: int) -> int:
+    return int(load().gdn_gr_read_workspace_size(T, n_r, d, rank))
+
+
+def gdn_gr_read(codes, scales, gamma, W_d, W_u, W_w, eps=1e-6, x=None, s=None,
+                workspace=None, stream=None):
+    """Gated Residual read: codes [T, n_r, d] uint8 (E4M3), scales [T, n_r]
+    fp32, gamma [n_r, d] fp32, W_d [rank, n_r d], W_u [n_r d, rank], W_w
+    [n_r, n_r d] bf16.  Returns (x [T, d] bf16, s [T, n_r] fp32)."""
+    lib = load()
+    dev = codes.device
+    T, n_r, d = codes.shape
+    rank = W_d.shape[0]
+    _check(codes, "codes", torch.uint8, dev)
+    for name, t in (("scales", scales), ("gamma", gamma)):
+        _check(t, name, torch.float32, dev)
+    for name, t in (("W_d", W_d), ("W_u", W_u), ("W_w", W_w)):
+        _check(t, name, torch.bfloat16, dev)
+    if x is None:
+        x = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
+    if s is None:
+        s = torch.empty((T, n_r), dtype=torch.float32, device=dev)
+    nbytes = int(lib.gdn_gr_read_workspace_size(T, n_r, d, rank))
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
+    st = lib.gdn_gr_read(_ptr(codes), _ptr(scales), _ptr(gamma), _ptr(W_d), _ptr(W_u),
+                         _ptr(W_w), T, n_r, d, rank, float(eps), _ptr(x), _ptr(s),
+                         _ptr(workspace), workspace.numel(), _stream_handle(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_gr_read")
+    return x, s
+
+
+def gdn_gr_write(codes, scales, y, s, stream=None):
+    """Gated Residual write, in place: R'_i = R_i + s_i y, requantised."""
+    lib = load()
+    dev = codes.device
+    T, n_r, d = codes.shape
+    _check(codes, "codes", torch.uint8, dev)
+    _check(scales, "scales", torch.float32, dev)
+    _check(y, "y", torch.bfloat16, dev)
+    _check(s, "s", torch.float32, dev)
+    st = lib.gdn_gr_write(_ptr(codes), _ptr(scales), _ptr(y), _ptr(s), T, n_r, d,
+                          _stream_handle(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_gr_write")
+    return codes, scales
 
 
 def gdn_check_device_error(stream=None) -> int:

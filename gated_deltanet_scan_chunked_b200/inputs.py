@@ -174,6 +174,29 @@ def make_conv_params(n_seq, H_qk, H_v, d_k, d_v, seed=0, w_std=0.5, state=True,
     return w, st
 
 
+def make_gr(T, n_r=4, d=2560, rank=320, seed=0, device="cpu"):
+    """Seeded Gated Residual inputs: an E4M3 state given directly as codes
+    (random sign, exponent field 4..14, mantissa; no NaN codes) with fp32
+    scales ~ U(0.01, 0.1), gains ~ 1 + N(0, 0.1^2), router and write weights
+    ~ N(0, 1/fan_in) in bf16, a block output y ~ N(0, 1) bf16 and write
+    scalars s ~ U(0.1, 1.9)."""
+    gen = _gen(int(seed) + 500, device)
+    sign = torch.randint(0, 2, (T, n_r, d), generator=gen, device=device)
+    expo = torch.randint(4, 15, (T, n_r, d), generator=gen, device=device)
+    mant = torch.randint(0, 8, (T, n_r, d), generator=gen, device=device)
+    codes = (sign * 128 + expo * 8 + mant).to(torch.uint8)
+    scales = torch.rand((T, n_r), generator=gen, device=device) * 0.09 + 0.01
+    gamma = 1.0 + 0.1 * torch.randn((n_r, d), generator=gen, device=device)
+    nd = n_r * d
+    W_d = (torch.randn((rank, nd), generator=gen, device=device) / nd ** 0.5).to(torch.bfloat16)
+    W_u = (torch.randn((nd, rank), generator=gen, device=device) / rank ** 0.5).to(torch.bfloat16)
+    W_w = (torch.randn((n_r, nd), generator=gen, device=device) / nd ** 0.5).to(torch.bfloat16)
+    y = torch.randn((T, d), generator=gen, device=device).to(torch.bfloat16)
+    s = torch.rand((T, n_r), generator=gen, device=device) * 1.8 + 0.1
+    return dict(codes=codes, scales=scales.float(), gamma=gamma.float(), W_d=W_d, W_u=W_u,
+                W_w=W_w, y=y, s=s.float())
+
+
 def varlen_lengths(n_seq=24, lo=512, hi=16384, seed=SEEDS["varlen"]):
     """Sequence lengths drawn uniformly from the integers [lo, hi]."""
     gen = torch.Generator().manual_seed(int(seed) + 7)

@@ -335,6 +335,59 @@ gdn_status gdn_decode_conv(
     gdn_stream_t stream);
 
 /*
+ * Gated Residual (GR) with an FP8 residual state, around each block of the
+ * layer ("Qwen3.8-Flash-Next: architecture, efficiency and technical
+ * lineage", section 05 "Residual design", part 4 "GR", its "Group RMSNorm"
+ * and "Low-rank router" boxes, and the inference paragraph of the same
+ * section on the FP8 state and the fused read and write).  The residual
+ * stream of a token is n_r branches of d channels (the model: n_r = 4,
+ * d = 2560, router rank d / 8 = 320):
+ *
+ *   read:  R^_i = R_i / sqrt(mean(R_i^2) + eps) * gamma_i
+ *          G    = sigmoid(W_u SiLU((1/n_r) W_d vec(R^)))      (n_r x d gates)
+ *          x    = (1/n_r) sum_i G_i o R^_i                     (block input)
+ *          s    = 2 sigmoid((1/n_r) W_w vec(R^))               (n_r write scalars)
+ *   write: R'_i = R_i + s_i y                                  (block output y)
+ *
+ * State: codes [T, n_r, d] uint8, OCP E4M3 (finite, saturating), and one
+ * fp32 scale per (token, branch) row: value = E4M3(code) * scale.  A written
+ * row is requantised with scale max|R'| / 448 (1 for an all-zero row), codes
+ * rounded to nearest even.  Format, scaling and eps are readings: the pages
+ * say only that the state is FP8.
+ */
+
+/* Workspace bytes gdn_gr_read needs (0 for arguments it never accepts). */
+size_t gdn_gr_read_workspace_size(int64_t T, int32_t n_r, int32_t d, int32_t rank);
+
+/*
+ * gdn_gr_read -- the block input x and the write scalars s from the state.
+ *   codes, scales   the state, as above (read only)
+ *   gamma           [n_r, d] fp32 branch gains
+ *   W_d             [rank, n_r d] bf16;  W_u [n_r d, rank] bf16;
+ *   W_w             [n_r, n_r d] bf16
+ *   T, n_r (1..8), d (multiple of 8), rank (multiple of 8), eps (>= 0)
+ *   x               [T, d] bf16, written
+ *   s               [T, n_r] fp32, written (pass to gdn_gr_write)
+ *   workspace       256-byte aligned, gdn_gr_read_workspace_size bytes
+ * The two router products run as bf16 GEMMs with fp32 accumulation through
+ * cuBLASLt; the normalisation and the gated branch mean are this library's
+ * kernels.
+ */
+gdn_status gdn_gr_read(const uint8_t* codes, const float* scales, const float* gamma,
+                       const void* W_d, const void* W_u, const void* W_w, int64_t T,
+                       int32_t n_r, int32_t d, int32_t rank, float eps, void* x, float* s,
+                       void* workspace, size_t workspace_bytes, gdn_stream_t stream);
+
+/*
+ * gdn_gr_write -- R'_i = R_i + s_i y, requantised in place (codes and scales
+ * are rewritten).  y [T, d] bf16; s [T, n_r] fp32 from gdn_gr_read.  One
+ * kernel; each row is read twice (its maximum, then its codes) and written
+ * once.
+ */
+gdn_status gdn_gr_write(uint8_t* codes, float* scales, const void* y, const float* s,
+                        int64_t T, int32_t n_r, int32_t d, gdn_stream_t stream);
+
+/*
  * gdn_chunk_bwd_workspace_size -- bytes of device workspace gdn_chunk_bwd
  * needs for a packed batch (0 for arguments it can never accept).  About
  * 460 KB per 64-token chunk per value head at d_k = d_v = 128 (chunk states

@@ -262,3 +262,27 @@ def test_conv_entry_points_reject_on_host(lib):
     assert dc(w=None) == gdn.GDN_ERR_INVALID_ARG
     assert dc(cs=FAKE + (9 << 24) + 4096) == gdn.GDN_ERR_INVALID_ARG  # inside the state
     assert dc(cs=S + 8) == gdn.GDN_ERR_INVALID_ARG                     # misaligned
+
+
+def test_gr_entry_points_reject_on_host(lib):
+    n = gdn.gr_read_workspace_size(64, 4, 2560, 320)
+    assert n > 64 * 4 * 2560 * 2 * 2
+    assert gdn.gr_read_workspace_size(64, 9, 2560, 320) == 0      # more than 8 branches
+    assert gdn.gr_read_workspace_size(64, 4, 2561, 320) == 0      # d not a multiple of 8
+    assert gdn.gr_read_workspace_size(64, 4, 2560, 12) == 0       # rank not a multiple of 8
+
+    def rd(**kw):
+        a = dict(c=FAKE, ws=FAKE, wsb=n, T=64, nr=4, d=2560, r=320, x=FAKE, s=FAKE)
+        a.update(kw)
+        return lib.gdn_gr_read(a["c"], FAKE, FAKE, FAKE, FAKE, FAKE, a["T"], a["nr"], a["d"],
+                               a["r"], 1e-6, a["x"], a["s"], a["ws"], a["wsb"], None)
+    assert rd(ws=None) == gdn.GDN_ERR_INVALID_ARG
+    assert rd(wsb=n - 256) == gdn.GDN_ERR_INVALID_ARG
+    assert rd(c=None) == gdn.GDN_ERR_INVALID_ARG
+    assert rd(nr=0) == gdn.GDN_ERR_INVALID_ARG
+    assert rd(x=FAKE + 8) == gdn.GDN_ERR_INVALID_ARG
+    assert rd(T=0, c=None, x=None, s=None, wsb=gdn.gr_read_workspace_size(0, 4, 2560, 320)) \
+        == gdn.GDN_OK
+    assert lib.gdn_gr_write(FAKE, FAKE, FAKE, FAKE, 64, 4, 12, None) == gdn.GDN_ERR_INVALID_ARG
+    assert lib.gdn_gr_write(None, FAKE, FAKE, FAKE, 64, 4, 16, None) == gdn.GDN_ERR_INVALID_ARG
+    assert lib.gdn_gr_write(None, None, None, None, 0, 4, 16, None) == gdn.GDN_OK
