@@ -25,7 +25,7 @@ Read: fp64 arithmetic from the exact fp32 dequantised state.  Write: the
 codes are integers decided by floating point, so the write takes them in the
 precision the kernel uses, fp32, one rounding per operation in this order:
 r = deq + s * y (product rounded, then the sum), amax, scale = amax / 448,
-code = E4M3(r / scale).
+inv = 1 / scale, code = E4M3(r * inv).
 """
 from __future__ import annotations
 
@@ -78,12 +78,14 @@ def dequant(codes, scales):
 
 def quantize_rows(r):
     """fp32 rows [..., d] -> (codes uint8, scales fp32) with the row's own
-    scale amax / 448 (1 for an all-zero row); divisions in fp32."""
+    scale amax / 448 (1 for an all-zero row): inv = 1 / scale, code =
+    E4M3(r * inv), each operation rounded in fp32."""
     r = np.asarray(r, dtype=np.float32)
     amax = np.abs(r).max(axis=-1).astype(np.float32)
     scale = np.where(amax > 0, (amax / np.float32(E4M3_MAX)).astype(np.float32),
                      np.float32(1.0)).astype(np.float32)
-    q = (r / scale[..., None]).astype(np.float32)
+    inv = (np.float32(1.0) / scale).astype(np.float32)
+    q = (r * inv[..., None]).astype(np.float32)
     return e4m3_encode(q), scale
 
 
