@@ -3,7 +3,7 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload prefill4k|prefill256k|varlen]
                     [--path auto|tensor|tensor_pair|tensor_single|tensor_split|simt]
-                    [--no-decode] [--no-backward] [--no-front-end]
+                    [--no-decode] [--no-backward] [--no-front-end] [--no-gr]
                     [--no-cpu-baseline]
 
 One step = one chunked prefill (gdn_chunk_fwd: L2-norm prologue, gate cumsum,
@@ -14,8 +14,9 @@ batches may take the split layout (one kernel, after an asynchronous memset of
 the workspace flags).  The JSON line also carries the decode step
 (gdn_decode_step, 256 sequences x 64 steps, in place) and the backward of the
 model-shape prefill (gdn_chunk_bwd, T=4096) and the conv + SiLU front end
-(alone, ahead of the prefill, and fused into a 4-token decode) as separate
-objects with their own timing, roofline and clocks.
+(alone, ahead of the prefill, and fused into a 4-token decode) and the
+Gated Residual read / write over an FP8 state as separate objects with their
+own timing, roofline and clocks.
 
 Multi-GPU (torchrun, one process per GPU): every rank runs its own
 independent batch (weak scaling; sequences and heads are independent, so the
@@ -643,6 +644,77 @@ def run_ours(args, world, rank, local):
             "clocks": fclk_r}
         launches_front = fsteps * (1 + 2 + 1)
 
+    # Gated Residual read / write around a block, FP8 state, model shape
+    # (n_r = 4 branches of d = 2560, router rank 320), 4096 tokens
+    grd = None
+    launches_gr = 0
+    if not args.no_gr:
+        from gated_deltanet_scan_chunked_b200 import gdn_gr_read, gdn_gr_write
+        Tg, NR, DG, RK = 4096, 4, 2560, 320
+        g = inputs.make_gr(Tg, NR, DG, RK, seed=inputs.SEEDS["prefill4k"] + 100 * rank,
+                           device="cuda")
+        gws = torch.empty(gdn.gr_read_workspace_size(Tg, NR, DG, RK), dtype=torch.uint8,
+                          device="cuda")
+        xg = torch.empty((Tg, DG), dtype=torch.bfloat16, device="cuda")
+        sg = torch.empty((Tg, NR), dtype=torch.float32, device="cuda")
+        codes0, scales0 = g["codes"].clone(), g["scales"].clone()
+        gflush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
+        gclk = ClockSampler(local)
+        gclk.start()
+        gsteps = max(3, args.steps // 2)
+        # both calls are shorter than the Python that launches them: time them
+        # as CUDA graph replays so that host overhead stays out
+
+        def graph_of(fn):
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize()
+            gg = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gg):
+                fn()
+            return gg
+
+        rgraph = graph_of(lambda: gdn_gr_read(g["codes"], g["scales"], g["gamma"], g["W_d"],
+                                              g["W_u"], g["W_w"], x=xg, s=sg, workspace=gws))
+        rt = timed_steps(rgraph.replay, gsteps, 3, world, flush=lambda: gflush.zero_(),
+                         stream=stream)
+
+        def wreset():
+            g["codes"].copy_(codes0)
+            g["scales"].copy_(scales0)
+            gflush.zero_()
+
+        wgraph = graph_of(lambda: gdn_gr_write(g["codes"], g["scales"], g["y"], g["s"]))
+        wt = timed_steps(wgraph.replay, gsteps, 3, world, flush=wreset, stream=stream)
+        gclk_r = gclk.stop()
+        err = gdn.gdn_check_device_error()
+        if err != gdn.GDN_OK:
+            raise RuntimeError("device error in the gated residual: %s" % gdn.status_string(err))
+        rms_ = max_over_ranks(statistics.mean(rt), world)
+        wms_ = max_over_ranks(statistics.mean(wt), world)
+        nd = NR * DG
+        rbytes = Tg * (nd + NR * 4 + DG * 2 + NR * 4) + (2 * RK * nd + NR * nd) * 2 + nd * 4
+        rflops = 2.0 * 2 * RK * nd * Tg + 2.0 * NR * nd * Tg
+        wbytes = Tg * (2 * nd + 2 * NR * 4 + DG * 2 + NR * 4)
+        grd = {
+            "workload": "Gated Residual, 4096 tokens x 4 branches x d=2560, E4M3 state with a "
+                        "scale per row, router rank 320 (bf16 weights)",
+            "timing": "CUDA graph replay of one call",
+            "read_us": rms_ * 1e3,
+            "read_roofline": {"bound": "tensor", "achieved": rflops / (rms_ * 1e-3) / 1e12,
+                              "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                              "frac": rflops / (rms_ * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                              "algorithmic_flops": rflops, "algorithmic_bytes": rbytes,
+                              "hbm_frac": rbytes / (rms_ * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+            "write_us": wms_ * 1e3,
+            "write_roofline": {"bound": "hbm", "achieved": wbytes / (wms_ * 1e-3) / 1e9,
+                               "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                               "frac": wbytes / (wms_ * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                               "algorithmic_bytes": wbytes},
+            "clocks": gclk_r}
+        launches_gr = gsteps * (3 + 1)  # our kernels: norm, silu, gate; write (plus 2 cuBLASLt GEMMs)
+        del gws, gflush, rgraph, wgraph
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, target_s=args.ref_seconds)
@@ -661,7 +733,8 @@ def run_ours(args, world, rank, local):
                 "gpu_launches": args.steps, "clocks": clk, "decode": decode,
                 "gpu_launches_decode_region": launches_decode, "backward": backward,
                 "gpu_launches_backward_region": launches_bwd, "front_end": front,
-                "gpu_launches_front_end_region": launches_front}
+                "gpu_launches_front_end_region": launches_front, "gated_residual": grd,
+                "gpu_launches_gated_residual_region": launches_gr}
         print(json.dumps(line), flush=True)
 
 
@@ -679,6 +752,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--no-front-end", action="store_true")
+    ap.add_argument("--no-gr", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-seconds", type=float, default=12.0)
