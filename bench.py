@@ -117,6 +117,64 @@ def kernel_traffic(kernel_key):
         return None
 
 
+class NvmlClockSampler:
+    """SM clocks and clock-event reasons read through NVML every ~1 ms from
+    start() to stop() (the timed region and its warm-up), for the GPU that
+    cuda:`index` is (matched by PCI bus id).  Reads only; changes nothing."""
+    NAMES = [("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+             ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+             ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+             ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap")]
+
+    def __init__(self, index):
+        import pynvml
+        self.nv = pynvml
+        pynvml.nvmlInit()
+        pr = torch.cuda.get_device_properties(index)
+        bus = "%08x:%02x:%02x.0" % (pr.pci_domain_id, pr.pci_bus_id, pr.pci_device_id)
+        self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        self.samples = []
+        self.stop_flag = threading.Event()
+
+    def _poll(self):
+        nv = self.nv
+        while not self.stop_flag.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((sm, rs))
+            except Exception:
+                pass
+            time.sleep(0.001)
+
+    def start(self):
+        self.t = threading.Thread(target=self._poll, daemon=True)
+        self.t.start()
+
+    def stop(self):
+        self.stop_flag.set()
+        self.t.join(timeout=2)
+        nv = self.nv
+        if not self.samples:
+            return None
+        mx = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+        reasons = set()
+        for _, rs in self.samples:
+            for nm, const in self.NAMES:
+                if rs & getattr(nv, const):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median([sm for sm, _ in self.samples]), "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(self.samples), "source": "nvml"}
+
+
+def clock_sampler(index):
+    """NVML sampler (fine-grained), else nvidia-smi."""
+    try:
+        return NvmlClockSampler(index)
+    except Exception:
+        return ClockSampler(index)
+
+
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons sampled during a timed region."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -338,7 +396,7 @@ def run_ours(args, world, rank, local):
     def flush():
         flush_buf.zero_()
 
-    clocks = ClockSampler(local)
+    clocks = clock_sampler(local)
     clocks.start()
     times = timed_steps(step, args.steps, args.warmup, world, flush=flush, stream=stream)
     clk = clocks.stop()
@@ -460,7 +518,7 @@ def run_ours(args, world, rank, local):
         def dreset():
             state.copy_(state0)
 
-        dclk = ClockSampler(local)
+        dclk = clock_sampler(local)
         dclk.start()
         dt = timed_steps(dstep, max(3, args.steps // 2), 2, world, flush=dreset, stream=stream)
         dclk_r = dclk.stop()
@@ -498,7 +556,7 @@ def run_ours(args, world, rank, local):
             for gr in groups:
                 gdn_decode_multi(gr["q"], gr["k"], gr["v"], gr["la"], gr["b"], state, y=ym)
 
-        mclk = ClockSampler(local)
+        mclk = clock_sampler(local)
         mclk.start()
         mt = timed_steps(mstep, max(3, args.steps // 2), 2, world, flush=dreset, stream=stream)
         mclk_r = mclk.stop()
@@ -533,7 +591,7 @@ def run_ours(args, world, rank, local):
             gdn_chunk_bwd(wb.q, wb.k, wb.v, wb.log_alpha, wb.beta, dy, g=wb.g, norm_w=wb.norm_w,
                           d_final_state=dsT, workspace=bws)
 
-        bclk = ClockSampler(local)
+        bclk = clock_sampler(local)
         bclk.start()
         bsteps = max(3, args.steps // 4)
         bt = timed_steps(bstep, bsteps, 3, world, flush=lambda: bflush.zero_(), stream=stream)
@@ -579,7 +637,7 @@ def run_ours(args, world, rank, local):
         cso = torch.empty_like(cst)
         outs = (torch.empty_like(wf.q), torch.empty_like(wf.k), torch.empty_like(wf.v))
         fflush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
-        fclk = ClockSampler(local)
+        fclk = clock_sampler(local)
         fclk.start()
         fsteps = max(3, args.steps // 2)
         # the conv kernel takes less time than the Python call that launches
@@ -659,7 +717,7 @@ def run_ours(args, world, rank, local):
         sg = torch.empty((Tg, NR), dtype=torch.float32, device="cuda")
         codes0, scales0 = g["codes"].clone(), g["scales"].clone()
         gflush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
-        gclk = ClockSampler(local)
+        gclk = clock_sampler(local)
         gclk.start()
         gsteps = max(3, args.steps // 2)
         # both calls are shorter than the Python that launches them: time them
