@@ -343,12 +343,16 @@ __global__ void __launch_bounds__(kNT, 2) bwd_prep_kernel(const BwdArgs a) {
       }
     }
     float* gW = a.W + ch * kC * DK;
+    float* gWT = a.WT + ch * kC * DK;
     float* gU = a.UT + ch * kC * DV;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int t = ty + 16 * u;
 #pragma unroll
-      for (int w = 0; w < NK; ++w) gW[t * DK + tx + 16 * w] = wacc[u][w];
+      for (int w = 0; w < NK; ++w) {
+        gW[t * DK + tx + 16 * w] = wacc[u][w];
+        gWT[(tx + 16 * w) * kC + t] = wacc[u][w];
+      }
 #pragma unroll
       for (int w = 0; w < NV; ++w) gU[t * DV + tx + 16 * w] = uacc[u][w];
     }
@@ -371,32 +375,60 @@ struct Slice {
 
 template <int DK, int DV>
 struct ChainSmem {
-  static constexpr int LK = DK + 4, LS = Slice<DV>::SW + 4;
-  static constexpr int oW = 0, oK = oW + kC * LK, oS = oK + kC * LK, oD = oS + DK * LS,
-                       oG = oD + kC * LS, total = oG + kC;
+  static constexpr int LK = DK + 4, LS = Slice<DV>::SW + 4, LT = kC + 4;
+  // fwd_chain: W^T [DK][LT]; bwd_chain: W [C][LK] (the larger of the two)
+  static constexpr int WSZ = (DK * LT > kC * LK) ? DK * LT : kC * LK;
+  static constexpr int oW = 0, oK = oW + WSZ, oS = oK + kC * LK, oD = oS + DK * LS,
+                       oB = oD + kC * LS, oG = oB + kC, total = oG + kC;
   static constexpr size_t bytes = sizeof(float) * total;
 };
 
-// fwd_chain: S entering each chunk -> ws S; Delta = U - W S -> ws D.
+// N consecutive floats from shared memory (N = 1, 2, 4 or 8; 4N-byte aligned)
+template <int N>
+__device__ __forceinline__ void lds_row(const float* p, float* x) {
+  if constexpr (N == 8) {
+    const float4 a = reinterpret_cast<const float4*>(p)[0];
+    const float4 b = reinterpret_cast<const float4*>(p)[1];
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+  } else if constexpr (N == 4) {
+    const float4 a = *reinterpret_cast<const float4*>(p);
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+  } else if constexpr (N == 2) {
+    const float2 a = *reinterpret_cast<const float2*>(p);
+    x[0] = a.x; x[1] = a.y;
+  } else {
+    x[0] = p[0];
+  }
+}
+
+// b_t = exp(G_C - G_t) for the chunk (warp 0), once per chunk
+__device__ __forceinline__ void chunk_decay(const float* sG, float* sB) {
+  if (threadIdx.x < kC) sB[threadIdx.x] = expf(sG[kC - 1] - sG[threadIdx.x]);
+}
+
+// fwd_chain: S entering each chunk -> ws S; Delta = U - W S -> ws D.  The
+// state slice lives in registers, thread (ty, tx) holding rows NK ty .. NK ty
+// + NK - 1 (consecutive, for vector loads of K^) and columns tx + 16 w.
 template <int DK, int DV>
 __global__ void __launch_bounds__(kNT, 2) bwd_fwd_chain_kernel(const BwdArgs a) {
   using L = ChainSmem<DK, DV>;
   using SL = Slice<DV>;
   constexpr int SW = SL::SW, NW = SL::NW, NK = DK / 16;
   extern __shared__ __align__(16) float smem[];
-  float *sW = smem + L::oW, *sK = smem + L::oK, *sS = smem + L::oS, *sD = smem + L::oD,
-        *sG = smem + L::oG;
+  float *sWt = smem + L::oW, *sK = smem + L::oK, *sS = smem + L::oS, *sD = smem + L::oD,
+        *sB = smem + L::oB, *sG = smem + L::oG;
   const int seq = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * SW;
   const int hq = h / (a.H_v / a.H_qk);
   const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
   const size_t st = ((size_t)seq * a.H_v + h) * DK * DV;
-  float sr[NK][NW];  // this thread's state elements: rows ty + 16u, columns j0 + tx + 16w
+  float sr[NK][NW];
 #pragma unroll
   for (int u = 0; u < NK; ++u)
 #pragma unroll
     for (int w = 0; w < NW; ++w)
       sr[u][w] = a.initial_state
-                     ? __ldg(a.initial_state + st + (size_t)(ty + 16 * u) * DV + j0 + tx + 16 * w)
+                     ? __ldg(a.initial_state + st + (size_t)(NK * ty + u) * DV + j0 + tx + 16 * w)
                      : 0.f;
   const int c_begin = a.seq_first[seq], c_end = a.seq_first[seq + 1];
   const ChunkEnt* ents = reinterpret_cast<const ChunkEnt*>(a.chunks);
@@ -404,65 +436,66 @@ __global__ void __launch_bounds__(kNT, 2) bwd_fwd_chain_kernel(const BwdArgs a) 
     const ChunkEnt e = ents[c];
     const size_t ch = (size_t)c * a.H_v + h;
     __syncthreads();  // the previous chunk is done with every buffer
-    cp_tile(sW, L::LK, a.W + ch * kC * DK, DK, kC, kC, DK);
+    cp_tile(sWt, L::LT, a.WT + ch * DK * kC, kC, DK, DK, kC);
     cp_tile(sK, L::LK, a.kh + ((size_t)e.t0 * a.H_qk + hq) * DK, (size_t)a.H_qk * DK, kC, e.n, DK);
     cp_tile(sG, kC, a.G + ch * kC, kC, 1, 1, kC);
     cp_async_commit();
     float* gS = a.S + ch * DK * DV + j0;
-    float acc[4][NW];
 #pragma unroll
     for (int u = 0; u < NK; ++u)
 #pragma unroll
       for (int w = 0; w < NW; ++w) {
-        const int i = ty + 16 * u, j = tx + 16 * w;
+        const int i = NK * ty + u, j = tx + 16 * w;
         sS[i * L::LS + j] = sr[u][w];
         gS[(size_t)i * DV + j] = sr[u][w];
       }
+    float acc[4][NW];  // Delta rows 4 ty + u
     const float* gU = a.UT + ch * kC * DV + j0;
 #pragma unroll
     for (int u = 0; u < 4; ++u)
 #pragma unroll
-      for (int w = 0; w < NW; ++w) acc[u][w] = __ldg(gU + (size_t)(ty + 16 * u) * DV + tx + 16 * w);
+      for (int w = 0; w < NW; ++w) acc[u][w] = __ldg(gU + (size_t)(4 * ty + u) * DV + tx + 16 * w);
     cp_async_wait_all();
     __syncthreads();
-    // Delta = U - W S
+    chunk_decay(sG, sB);
+    // Delta = U - W S   (W^T rows give each thread's 4 rows in one load)
     for (int i = 0; i < DK; ++i) {
-      float sv[NW];
+      float sv[NW], wv[4];
 #pragma unroll
       for (int w = 0; w < NW; ++w) sv[w] = sS[i * L::LS + tx + 16 * w];
+      lds_row<4>(sWt + i * L::LT + 4 * ty, wv);
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float wv = sW[(ty + 16 * u) * L::LK + i];
+      for (int u = 0; u < 4; ++u)
 #pragma unroll
-        for (int w = 0; w < NW; ++w) acc[u][w] -= wv * sv[w];
-      }
+        for (int w = 0; w < NW; ++w) acc[u][w] -= wv[u] * sv[w];
     }
     float* gD = a.D + ch * kC * DV + j0;
 #pragma unroll
     for (int u = 0; u < 4; ++u)
 #pragma unroll
       for (int w = 0; w < NW; ++w) {
-        const int t = ty + 16 * u, j = tx + 16 * w;
+        const int t = 4 * ty + u, j = tx + 16 * w;
         sD[t * L::LS + j] = acc[u][w];
         gD[(size_t)t * DV + j] = acc[u][w];
       }
     __syncthreads();
     // S <- gamma_C S + (diag(b) K)^T Delta
-    const float GC = sG[kC - 1], gC = expf(GC);
+    const float gC = expf(sG[kC - 1]);
 #pragma unroll
     for (int u = 0; u < NK; ++u)
 #pragma unroll
       for (int w = 0; w < NW; ++w) sr[u][w] *= gC;
     for (int t = 0; t < kC; ++t) {
-      const float bt = expf(GC - sG[t]);
-      float dv[NW];
+      const float bt = sB[t];
+      float dv[NW], kv[NK];
 #pragma unroll
       for (int w = 0; w < NW; ++w) dv[w] = sD[t * L::LS + tx + 16 * w];
+      lds_row<NK>(sK + t * L::LK + NK * ty, kv);
 #pragma unroll
       for (int u = 0; u < NK; ++u) {
-        const float kv = bt * sK[t * L::LK + ty + 16 * u];
+        const float kb = bt * kv[u];
 #pragma unroll
-        for (int w = 0; w < NW; ++w) sr[u][w] += kv * dv[w];
+        for (int w = 0; w < NW; ++w) sr[u][w] += kb * dv[w];
       }
     }
   }
@@ -659,7 +692,8 @@ __global__ void __launch_bounds__(kNT, EPI ? 1 : 2) bwd_dout_kernel(const BwdArg
 }
 
 // bwd_chain: chunks in reverse; dS1 of each chunk -> ws dS (after taking X2
-// from there); dDelta = X1 + diag(b) K dS1 -> ws dD (in place of X1).
+// from there); dDelta = X1 + diag(b) K dS1 -> ws dD (in place of X1).  The
+// dS slice lives in registers with the row mapping of fwd_chain.
 template <int DK, int DV>
 __global__ void __launch_bounds__(kNT, 2) bwd_bwd_chain_kernel(const BwdArgs a) {
   using L = ChainSmem<DK, DV>;
@@ -667,18 +701,18 @@ __global__ void __launch_bounds__(kNT, 2) bwd_bwd_chain_kernel(const BwdArgs a) 
   constexpr int SW = SL::SW, NW = SL::NW, NK = DK / 16;
   extern __shared__ __align__(16) float smem[];
   float *sW = smem + L::oW, *sK = smem + L::oK, *sdS = smem + L::oS, *sdD = smem + L::oD,
-        *sG = smem + L::oG;
+        *sB = smem + L::oB, *sG = smem + L::oG;
   const int seq = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * SW;
   const int hq = h / (a.H_v / a.H_qk);
   const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
   const size_t st = ((size_t)seq * a.H_v + h) * DK * DV;
-  float dr[NK][NW];  // this thread's dS elements: rows ty + 16u, columns j0 + tx + 16w
+  float dr[NK][NW];  // rows NK ty + u, columns j0 + tx + 16 w
 #pragma unroll
   for (int u = 0; u < NK; ++u)
 #pragma unroll
     for (int w = 0; w < NW; ++w)
       dr[u][w] = a.d_final_state
-                     ? __ldg(a.d_final_state + st + (size_t)(ty + 16 * u) * DV + j0 + tx + 16 * w)
+                     ? __ldg(a.d_final_state + st + (size_t)(NK * ty + u) * DV + j0 + tx + 16 * w)
                      : 0.f;
   const int c_begin = a.seq_first[seq], c_end = a.seq_first[seq + 1];
   const ChunkEnt* ents = reinterpret_cast<const ChunkEnt*>(a.chunks);
@@ -696,7 +730,7 @@ __global__ void __launch_bounds__(kNT, 2) bwd_bwd_chain_kernel(const BwdArgs a) 
     for (int u = 0; u < NK; ++u)
 #pragma unroll
       for (int w = 0; w < NW; ++w) {
-        const int i = ty + 16 * u, j = tx + 16 * w;
+        const int i = NK * ty + u, j = tx + 16 * w;
         x2[u][w] = gdS[(size_t)i * DV + j];  // X2, then the same element gets dS1
         gdS[(size_t)i * DV + j] = dr[u][w];
         sdS[i * L::LS + j] = dr[u][w];
@@ -709,7 +743,7 @@ __global__ void __launch_bounds__(kNT, 2) bwd_bwd_chain_kernel(const BwdArgs a) 
       for (int w = 0; w < NW; ++w) acc[u][w] = gdD[(size_t)(ty + 16 * u) * DV + tx + 16 * w];
     cp_async_wait_all();
     __syncthreads();
-    const float GC = sG[kC - 1];
+    chunk_decay(sG, sB);
     // dDelta = X1 + diag(b) K dS1  (zero on rows past the chunk's end)
     {
       float kacc[4][NW];
@@ -728,10 +762,11 @@ __global__ void __launch_bounds__(kNT, 2) bwd_bwd_chain_kernel(const BwdArgs a) 
           for (int w = 0; w < NW; ++w) kacc[u][w] += kv * sv[w];
         }
       }
+      __syncthreads();  // sB ready
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int t = ty + 16 * u;
-        const float bt = expf(GC - sG[t]);
+        const float bt = sB[t];
 #pragma unroll
         for (int w = 0; w < NW; ++w) {
           const int j = tx + 16 * w;
@@ -744,21 +779,20 @@ __global__ void __launch_bounds__(kNT, 2) bwd_bwd_chain_kernel(const BwdArgs a) 
     __syncthreads();
     // dS <- gamma_C dS + X2 - W^T dDelta
     {
-      const float gC = expf(GC);
+      const float gC = expf(sG[kC - 1]);
 #pragma unroll
       for (int u = 0; u < NK; ++u)
 #pragma unroll
         for (int w = 0; w < NW; ++w) dr[u][w] = gC * dr[u][w] + x2[u][w];
       for (int t = 0; t < kC; ++t) {
-        float dv[NW];
+        float dv[NW], wv[NK];
 #pragma unroll
         for (int w = 0; w < NW; ++w) dv[w] = sdD[t * L::LS + tx + 16 * w];
+        lds_row<NK>(sW + t * L::LK + NK * ty, wv);
 #pragma unroll
-        for (int u = 0; u < NK; ++u) {
-          const float wv = sW[t * L::LK + ty + 16 * u];
+        for (int u = 0; u < NK; ++u)
 #pragma unroll
-          for (int w = 0; w < NW; ++w) dr[u][w] -= wv * dv[w];
-        }
+          for (int w = 0; w < NW; ++w) dr[u][w] -= wv[u] * dv[w];
       }
     }
   }
@@ -767,7 +801,7 @@ __global__ void __launch_bounds__(kNT, 2) bwd_bwd_chain_kernel(const BwdArgs a) 
     for (int u = 0; u < NK; ++u)
 #pragma unroll
       for (int w = 0; w < NW; ++w)
-        a.d_initial_state[st + (size_t)(ty + 16 * u) * DV + j0 + tx + 16 * w] = dr[u][w];
+        a.d_initial_state[st + (size_t)(NK * ty + u) * DV + j0 + tx + 16 * w] = dr[u][w];
   }
 }
 
@@ -1352,7 +1386,7 @@ size_t chunk_bwd_workspace_bytes(int32_t n_seq, int64_t total_T, int32_t H_qk, i
   b += align256(maxc * sizeof(ChunkEnt));
   b += align256((size_t)(n_seq + 1) * sizeof(int32_t));
   b += 2 * align256(nch * d_k * d_v * f);            // S, dS
-  b += align256(nch * kC * d_k * f);                 // W
+  b += 2 * align256(nch * kC * d_k * f);             // W, W^T
   b += 3 * align256(nch * kC * d_v * f);             // U / TdD, Delta, dDelta
   b += 5 * align256(nch * kC * kC * f);              // T, KKE, P, dPE, B
   b += align256(nch * kC * f);                       // G
@@ -1379,6 +1413,7 @@ void chunk_bwd_workspace_layout(void* ws, BwdArgs* a) {
   a->S = reinterpret_cast<float*>(take(nch * a->d_k * a->d_v * f));
   a->dS = reinterpret_cast<float*>(take(nch * a->d_k * a->d_v * f));
   a->W = reinterpret_cast<float*>(take(nch * kC * a->d_k * f));
+  a->WT = reinterpret_cast<float*>(take(nch * kC * a->d_k * f));
   a->UT = reinterpret_cast<float*>(take(nch * kC * a->d_v * f));
   a->D = reinterpret_cast<float*>(take(nch * kC * a->d_v * f));
   a->dD = reinterpret_cast<float*>(take(nch * kC * a->d_v * f));

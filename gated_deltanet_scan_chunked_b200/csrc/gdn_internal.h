@@ -96,8 +96,8 @@ struct BwdArgs {
   // workspace parts, placed by chunk_bwd_workspace_layout
   void* chunks;
   int32_t* seq_first;
-  float *S, *dS, *W, *UT, *D, *dD, *T, *KKE, *P, *dPE, *Bm, *G, *row, *dw, *dO, *dqh, *dkh,
-      *qh, *kh;
+  float *S, *dS, *W, *WT, *UT, *D, *dD, *T, *KKE, *P, *dPE, *Bm, *G, *row, *dw, *dO, *dqh,
+      *dkh, *qh, *kh;
 };
 
 struct ConvArgs {
