@@ -147,3 +147,13 @@ def test_model_shape_one_group_sampled():
     ref, hv, hq = _oracle(w, dy, dsT, heads=[15, 16, 17])
     ref.pop("dnorm_w")  # needs every head
     _compare(got, ref, hv, hq, what="T=4096")
+
+
+def test_ungrouped_heads_fp32():
+    """H_qk = H_v (one value head per QK head) with a ragged packed batch."""
+    w = to_device(inputs.make_prefill([65, 3], 2, 2, 32, 16, dtype=torch.float32, seed=13,
+                                      epilogue=True, s0_std=0.1))
+    dy, dsT = inputs.make_cotangents(w, seed=13)
+    got = _gpu(w, dy, dsT)
+    ref, _, _ = _oracle(w, dy, dsT)
+    _compare(got, ref, what="H_qk = H_v")

@@ -183,3 +183,14 @@ def test_decode_conv_continues_prefill_conv():
     assert_close(y_a, y_all[:T].cpu().double().numpy(), torch.float32, "prefix y")
     assert_close(y_b[0], y_all[T:].cpu().double().numpy(), torch.float32, "decoded y")
     assert_close(state, fs_all.cpu().double().numpy(), torch.float32, "state")
+
+
+def test_conv_frontend_all_sequences_empty_carries_state():
+    w = to_device(inputs.make_prefill([0, 0, 0], 2, 4, 16, 32, dtype=torch.float32, seed=2,
+                                      epilogue=False))
+    cw, st = inputs.make_conv_params(3, 2, 4, 16, 32, seed=2)
+    qo, ko, vo, so = gdn_conv_frontend(w.q, w.k, w.v, cw.cuda(), st.cuda(),
+                                       cu_seqlens=w.cu_seqlens)
+    torch.cuda.synchronize()
+    assert gdn_check_device_error() == gdn.GDN_OK
+    torch.testing.assert_close(so, st.cuda(), rtol=0, atol=0)

@@ -26,7 +26,7 @@ def _cuda(g):
 
 
 @pytest.mark.parametrize("T,n_r,d,rank", [(300, 4, 256, 32), (128, 4, 2560, 320), (17, 1, 64, 8),
-                                          (64, 3, 128, 16)])
+                                          (64, 3, 128, 16), (40, 8, 96, 24)])
 def test_gr_read(T, n_r, d, rank):
     g = inputs.make_gr(T, n_r, d, rank, seed=T + d)
     c = _cuda(g)
@@ -39,7 +39,7 @@ def test_gr_read(T, n_r, d, rank):
     assert_close(s, sr, torch.bfloat16, "s")
 
 
-@pytest.mark.parametrize("T,n_r,d", [(300, 4, 256), (64, 4, 2560), (5, 2, 8)])
+@pytest.mark.parametrize("T,n_r,d", [(300, 4, 256), (64, 4, 2560), (5, 2, 8), (33, 8, 4096)])
 def test_gr_write_bit_exact(T, n_r, d):
     g = inputs.make_gr(T, n_r, d, 8, seed=7 * T + d)
     want_c, want_s = ogr.gr_write(_np(g["codes"]), _np(g["scales"]), _np(g["y"]), _np(g["s"]))
