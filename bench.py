@@ -611,7 +611,8 @@ def run_ours(args, world, rank, local):
             "roofline": {"bound": "hbm", "achieved": bb / (bms * 1e-3) / 1e9,
                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": bb / (bms * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                         "algorithmic_bytes": bb, "traffic": None},
+                         "algorithmic_bytes": bb, "traffic": kernel_traffic("bwd_chunk_b"),
+                         "traffic_kernel": "bwd_chunk_b (the largest share of the call)"},
             "tensor": {"achieved_tflops": bfl / (bms * 1e-3) / 1e12,
                        "peak_tflops": peaks["bf16_tflops"],
                        "frac": bfl / (bms * 1e-3) / 1e12 / (peaks["bf16_tflops"])},
