@@ -328,16 +328,16 @@ def _prefix(w, T):
                 s0=None if w.initial_state is None else w.initial_state[:1].to("cpu", torch.float32))
 
 
-def make_workload(name, rank):
+def make_workload(name, rank, device="cuda"):
     from gated_deltanet_scan_chunked_b200 import inputs
-    w = inputs.workload(name, device="cuda")
+    w = inputs.workload(name, device=device)
     if rank:
         # an independent batch per rank: same recipe, another seed
         seed = rank_seed(name, rank)
         lengths = w.meta["lengths"]
         w = inputs.make_prefill(lengths, H_QK, H_V, D, D, seed=seed,
                                 s0_std=0.01 if w.initial_state is not None else 0.0,
-                                device="cuda")
+                                device=device)
     return w
 
 
@@ -345,8 +345,12 @@ def run_reference(args, world, rank):
     """The oracle arm: rank 0 only, no process group, no GPU kernels of ours."""
     if rank != 0:
         return
-    torch.cuda.set_device(0)
-    w = make_workload(args.workload, 0)
+    # the same recipe; generated on the GPU when there is one (as the other
+    # arm does), else on the host (a different draw of the same distributions)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    if dev == "cuda":
+        torch.cuda.set_device(0)
+    w = make_workload(args.workload, 0, device=dev)
     times = []
     base = None
     per_step = min(args.ref_seconds, 150.0 / (args.steps + args.warmup))
