@@ -1,4 +1,6 @@
 // Backward of the chunked gated delta rule on CUDA cores, fp32 throughout.
+// Tiles move into shared memory with 16-byte asynchronous copies; the two
+// chains keep their state slice in registers and run two CTAs per SM.
 //
 // The forward is the recurrence of "Qwen3.8-Flash-Next: architecture,
 // efficiency and technical lineage", section 03 "Gated DeltaNet" (update
@@ -32,10 +34,13 @@
 // device-built table of (sequence, first token, length)):
 //   chunk_table  chunk list and each sequence's first chunk
 //   normalise    q^, k^ in fp32
-//   prep         per chunk: G, T, K K^T o E, P, W, U
+//   prep         per chunk: G, T, K K^T o E, P, W (and W^T), U
 //   fwd_chain    per (sequence, 32 state columns): S entering each chunk, Delta
-//   epilogue     per chunk: O, then dO from dy through the gate and RMS norm
-//   bwd_chain    per (sequence, 32 state columns): dS1 of each chunk, dDelta
+//   dout         per chunk: dO (with the epilogue: O recomputed, then dy taken
+//                back through the gate and the RMS norm), and the dO-only
+//                products X1 = P^T dO, X2 = (diag(gamma) Qs)^T dO
+//   bwd_chain    per (sequence, 32 state columns): dS1 of each chunk,
+//                dDelta = X1 + diag(b) K dS1
 //   chunk_a      per chunk: TdD, dV, R, dT, dA, dP and their row terms
 //   chunk_b      per chunk: L1..L3, dq^ and dk^ of this value head, dbeta, dlog alpha
 //   qk_final     sum over the value heads of a QK head, then the L2 norm
