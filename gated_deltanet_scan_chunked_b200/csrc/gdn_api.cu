@@ -48,13 +48,18 @@ gdn_status check_common(int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v, gdn
 
 using namespace gdn;
 
-extern "C" gdn_status gdn_chunk_fwd_ws(
+namespace {
+
+// gdn_chunk_fwd_ws, optionally with the front end fused into the portable
+// kernel (conv_w non-null: only the portable path takes it).
+gdn_status chunk_fwd_impl(
     const void* q, const void* k, const void* v, const float* log_alpha, const float* beta,
     const void* g, const float* norm_w, const float* initial_state, const int32_t* cu_seqlens,
     int32_t n_seq, int64_t total_T, int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v,
     gdn_dtype in_dtype, int32_t l2norm_qk, float eps_l2, float eps_norm, float scale, void* y,
     float* final_state, gdn_prefill_path path, void* workspace, size_t workspace_bytes,
-    gdn_stream_t stream) {
+    gdn_stream_t stream, const float* conv_w, const float* conv_state_in,
+    float* conv_state_out) {
   gdn_status st = check_common(H_qk, H_v, d_k, d_v, in_dtype, eps_l2, eps_norm);
   if (st != GDN_OK) return st;
   if (n_seq < 1 || total_T < 0) return GDN_ERR_INVALID_ARG;
@@ -104,8 +109,28 @@ extern "C" gdn_status gdn_chunk_fwd_ws(
   if (want_tc && !tc_ok) return GDN_ERR_UNSUPPORTED;
   a.err = error_word_ptr();
   if (a.err == nullptr) return GDN_ERR_CUDA;
+  if (conv_w != nullptr) {
+    if (path != GDN_PATH_SIMT) return GDN_ERR_UNSUPPORTED;
+    a.conv_w = conv_w; a.conv_state_in = conv_state_in; a.conv_state_out = conv_state_out;
+    return launch_prefill_simt(a, s);
+  }
   if (want_tc || (path == GDN_PATH_AUTO && tc_ok)) return launch_prefill_tc(a, s);
   return launch_prefill_simt(a, s);
+}
+
+}  // namespace
+
+extern "C" gdn_status gdn_chunk_fwd_ws(
+    const void* q, const void* k, const void* v, const float* log_alpha, const float* beta,
+    const void* g, const float* norm_w, const float* initial_state, const int32_t* cu_seqlens,
+    int32_t n_seq, int64_t total_T, int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v,
+    gdn_dtype in_dtype, int32_t l2norm_qk, float eps_l2, float eps_norm, float scale, void* y,
+    float* final_state, gdn_prefill_path path, void* workspace, size_t workspace_bytes,
+    gdn_stream_t stream) {
+  return chunk_fwd_impl(q, k, v, log_alpha, beta, g, norm_w, initial_state, cu_seqlens, n_seq,
+                        total_T, H_qk, H_v, d_k, d_v, in_dtype, l2norm_qk, eps_l2, eps_norm, scale,
+                        y, final_state, path, workspace, workspace_bytes, stream, nullptr,
+                        nullptr, nullptr);
 }
 
 extern "C" gdn_status gdn_chunk_fwd_path(
@@ -305,6 +330,20 @@ extern "C" gdn_status gdn_chunk_fwd_conv(
   if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
       workspace_bytes < need)
     return GDN_ERR_INVALID_ARG;
+  // the portable kernel takes the front end fused (no activation round trip)
+  const bool tc_shape = in_dtype == GDN_BF16 && d_k == 128 && d_v == 128;
+  if (path == GDN_PATH_SIMT || (path == GDN_PATH_AUTO && !tc_shape)) {
+    if (!conv_w || !aligned16(conv_w)) return GDN_ERR_INVALID_ARG;
+    if ((conv_state_in && !aligned16(conv_state_in)) ||
+        (conv_state_out && !aligned16(conv_state_out)))
+      return GDN_ERR_INVALID_ARG;
+    const size_t ns = (size_t)n_seq * H_v * 3 * (2 * d_k + d_v) * sizeof(float);
+    if (overlaps(conv_state_in, ns, conv_state_out, ns)) return GDN_ERR_INVALID_ARG;
+    return chunk_fwd_impl(q, k, v, log_alpha, beta, g, norm_w, initial_state, cu_seqlens, n_seq,
+                          total_T, H_qk, H_v, d_k, d_v, in_dtype, l2norm_qk, eps_l2, eps_norm,
+                          scale, y, final_state, GDN_PATH_SIMT, nullptr, 0, stream, conv_w,
+                          conv_state_in, conv_state_out);
+  }
   // the front end's outputs first in the workspace, the prefill's part after
   const size_t e = in_dtype == GDN_BF16 ? 2 : 4;
   auto a256 = [](size_t x) { return (x + 255) & ~(size_t)255; };

@@ -42,7 +42,8 @@ struct SimtSmem {
   static constexpr int oAP = oS + DK * LV;        // A (upper, transposed) + P (lower)
   static constexpr int oG = oAP + kC * LC;        // G_t
   static constexpr int oB = oG + kC;              // beta_t
-  static constexpr int total = oB + kC;
+  static constexpr int oCS = oB + kC;             // carried conv inputs [3][2 DK + DV]
+  static constexpr int total = oCS + 3 * (2 * DK + DV);
   static constexpr size_t bytes = sizeof(float) * total;
 };
 
@@ -58,6 +59,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_simt_kernel(const PrefillA
   float* sAP = smem + L::oAP;
   float* sG = smem + L::oG;
   float* sB = smem + L::oB;
+  float* sCS = smem + L::oCS;
 
   const int seq = blockIdx.x / a.H_v;
   const int h = blockIdx.x % a.H_v;
@@ -78,6 +80,28 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_simt_kernel(const PrefillA
   const Tin* Gg = static_cast<const Tin*>(a.g);
   Tin* Yg = static_cast<Tin*>(a.y);
   const int ty = tid / 16, tx = tid % 16;
+  // front end (optional): this value head's carried conv inputs
+  constexpr int SROW = 2 * DK + DV;
+  const bool conv = a.conv_w != nullptr;
+  const size_t cs_off = ((size_t)seq * a.H_v + h) * 3 * SROW;
+  if (conv)
+    for (int e = tid; e < 3 * SROW; e += kNT)
+      sCS[e] = a.conv_state_in ? __ldg(a.conv_state_in + cs_off + e) : 0.f;
+  // The input x (raw, before the front end) of channel column `col` of the
+  // carried-state row layout at token t, from the tensor (row stride `rs`,
+  // column `c`), or from the carried inputs before the sequence's start.
+  auto raw = [&](const Tin* X, size_t rs, int c, int col, int64_t t) -> float {
+    return t >= t_begin ? Elem<Tin>::load(X + (size_t)t * rs + c)
+                        : sCS[(3 - (int)(t_begin - t)) * SROW + col];
+  };
+  // conv of kernel 4 then SiLU: weights row `wrow` of conv_w
+  auto front = [&](const Tin* X, size_t rs, int c, int col, int wrow, int64_t t) -> float {
+    const float4 w = __ldg(reinterpret_cast<const float4*>(a.conv_w) + wrow);
+    const float u = w.w * raw(X, rs, c, col, t) + w.z * raw(X, rs, c, col, t - 1) +
+                    w.y * raw(X, rs, c, col, t - 2) + w.x * raw(X, rs, c, col, t - 3);
+    return u / (1.f + __expf(-u));
+  };
+  if (conv) __syncthreads();  // sCS loaded
 
   for (int64_t c0 = t_begin; c0 < t_end; c0 += kC) {
     const int n = (t_end - c0) < kC ? (int)(t_end - c0) : kC;
@@ -88,9 +112,15 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_simt_kernel(const PrefillA
       for (int d = lane; d < DK; d += 32) {
         float kv = 0.f, qv = 0.f;
         if (r < n) {
-          const size_t off = ((size_t)(c0 + r) * a.H_qk + hq) * DK + d;
-          kv = Elem<Tin>::load(Kg + off);
-          qv = Elem<Tin>::load(Qg + off);
+          if (conv) {
+            const size_t rs = (size_t)a.H_qk * DK;
+            kv = front(Kg, rs, hq * DK + d, DK + d, (a.H_qk + hq) * DK + d, c0 + r);
+            qv = front(Qg, rs, hq * DK + d, d, hq * DK + d, c0 + r);
+          } else {
+            const size_t off = ((size_t)(c0 + r) * a.H_qk + hq) * DK + d;
+            kv = Elem<Tin>::load(Kg + off);
+            qv = Elem<Tin>::load(Qg + off);
+          }
         }
         sK[r * L::LK + d] = kv;
         sQ[r * L::LK + d] = qv;
@@ -107,7 +137,10 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_simt_kernel(const PrefillA
       }
       for (int j = lane; j < DV; j += 32)
         sV[r * L::LV + j] =
-            r < n ? Elem<Tin>::load(Vg + ((size_t)(c0 + r) * a.H_v + h) * DV + j) : 0.f;
+            r >= n ? 0.f
+            : conv ? front(Vg, (size_t)a.H_v * DV, h * DV + j, 2 * DK + j,
+                           2 * a.H_qk * DK + h * DV + j, c0 + r)
+                   : Elem<Tin>::load(Vg + ((size_t)(c0 + r) * a.H_v + h) * DV + j);
     }
     if (warp == 0) {
       // inclusive cumsum of log alpha over the chunk (two 32-lane scans)
@@ -303,6 +336,26 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_simt_kernel(const PrefillA
     }
   }
   __syncthreads();
+  if (conv && a.conv_state_out) {
+    // the sequence's last three raw inputs, oldest first (from the carried
+    // ones for a sequence shorter than three)
+    const int64_t len = t_end - t_begin;
+    for (int e = tid; e < 3 * SROW; e += kNT) {
+      const int m = e / SROW, col = e % SROW;
+      const int64_t t = t_end - 3 + m;
+      float x;
+      if (t < t_begin) {
+        x = sCS[(m + (int)len) * SROW + col];
+      } else if (col < DK) {
+        x = Elem<Tin>::load(Qg + ((size_t)t * a.H_qk + hq) * DK + col);
+      } else if (col < 2 * DK) {
+        x = Elem<Tin>::load(Kg + ((size_t)t * a.H_qk + hq) * DK + col - DK);
+      } else {
+        x = Elem<Tin>::load(Vg + ((size_t)t * a.H_v + h) * DV + col - 2 * DK);
+      }
+      a.conv_state_out[cs_off + e] = x;
+    }
+  }
   if (a.final_state) {
     for (int e = tid; e < DK * DV; e += kNT) {
       const int i = e / DV, j = e % DV;

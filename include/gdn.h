@@ -298,10 +298,13 @@ size_t gdn_chunk_fwd_conv_workspace_size(int32_t n_seq, int64_t total_T, int32_t
                                          gdn_dtype in_dtype);
 
 /*
- * gdn_chunk_fwd_conv -- gdn_chunk_fwd_ws on pre-conv q, k, v: the front end
- * (gdn_conv_frontend, written into the workspace in the input dtype), then
- * the chunked prefill on its outputs (the L2 norm of q and k, when
- * l2norm_qk, follows the SiLU).  conv_state_in / conv_state_out as for
+ * gdn_chunk_fwd_conv -- gdn_chunk_fwd_ws on pre-conv q, k, v (the L2 norm of
+ * q and k, when l2norm_qk, follows the SiLU).  On the portable path
+ * (GDN_PATH_SIMT, or GDN_PATH_AUTO for shapes the tensor-core kernel does not
+ * serve) the front end is fused into the prefill kernel and the activations
+ * stay in fp32 on chip.  On the tensor-core paths the front end runs first
+ * (gdn_conv_frontend, its outputs written into the workspace in the input
+ * dtype), then the prefill.  conv_state_in / conv_state_out as for
  * gdn_conv_frontend; everything else as for gdn_chunk_fwd_ws.  The workspace
  * (256-byte aligned, at least gdn_chunk_fwd_conv_workspace_size bytes) is
  * required.

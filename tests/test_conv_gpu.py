@@ -5,10 +5,11 @@ the front end fused (gdn_decode_conv), including a decode that continues a
 prefill.  Carried conv states are compared bit for bit (they are copies of
 inputs); outputs within the library's tolerances.
 
-gdn_chunk_fwd_conv hands the front end's outputs to the scan in the input
-dtype, as the scan's q/k/v inputs are in that dtype; its oracle therefore
-rounds the oracle's own conv outputs to that dtype (on the host) before the
-recurrence.  The fused decode keeps them in fp32 and is compared with the
+On the tensor-core path gdn_chunk_fwd_conv hands the front end's outputs to
+the scan in the input dtype, as the scan's q/k/v inputs are in that dtype;
+its oracle then rounds the oracle's own conv outputs to that dtype (on the
+host) before the recurrence.  The portable prefill kernel and the decode take
+the front end fused, keep the activations in fp32, and are compared with the
 unrounded oracle.
 """
 import numpy as np
@@ -111,10 +112,14 @@ def test_chunk_fwd_conv(path, dtype, dims):
     torch.cuda.synchronize()
     assert gdn_check_device_error() == gdn.GDN_OK
     rq, rk, rv, rso = _oracle_conv(w.q, w.k, w.v, cw, st, w.cu_seqlens)
-    # the front end's outputs are the scan's q/k/v, held in the input dtype
-    # (bf16 activations in bf16 mode): the oracle rounds its own conv outputs
-    # to that dtype on the host before the recurrence
-    rnd = lambda x: torch.tensor(x).to(dtype).to(torch.float32).numpy()
+    # the tensor-core path hands the front end's outputs to the scan in the
+    # input dtype (bf16 activations in bf16 mode): there the oracle rounds its
+    # own conv outputs to that dtype on the host before the recurrence; the
+    # portable kernel takes the front end fused and keeps them in fp32
+    fused = path == "simt" or (path == "auto" and not (dtype == torch.bfloat16 and dk == 128
+                                                       and dv == 128))
+    act = torch.float32 if fused else dtype
+    rnd = lambda x: torch.tensor(x).to(act).to(torch.float32).numpy()
     y_ref, s_ref = oracle.recurrence(rnd(rq), rnd(rk), rnd(rv), w.log_alpha.cpu(), w.beta.cpu(),
                                      g=w.g.cpu().float(), norm_w=w.norm_w.cpu(),
                                      initial_state=w.initial_state.cpu(),
