@@ -157,3 +157,14 @@ def test_ungrouped_heads_fp32():
     got = _gpu(w, dy, dsT)
     ref, _, _ = _oracle(w, dy, dsT)
     _compare(got, ref, what="H_qk = H_v")
+
+
+def test_long_sequence_one_group_sampled():
+    """T = 16,384 (256 chunks per head) with an initial state: the whole launch
+    at the model's head counts, checked on the value heads of QK head 10."""
+    w = inputs.workload("prefill256k", T=16384, device="cuda")
+    dy, dsT = inputs.make_cotangents(w, seed=16384)
+    got = _gpu(w, dy, dsT)
+    ref, hv, hq = _oracle(w, dy, dsT, heads=[30, 31, 32])
+    ref.pop("dnorm_w")
+    _compare(got, ref, hv, hq, what="T=16384")
