@@ -5,9 +5,21 @@
 #include <mutex>
 
 #include "gdn_internal.h"
+#include "gdn_sm100.cuh"
 
 namespace gdn {
 namespace {
+
+// A hand-off flag that nothing ever sets, for the bounded-wait self-test.
+__device__ unsigned long long g_never_set = 0;
+
+// One CTA waits on g_never_set with the library's bounded wait (the one the
+// split prefill uses for its hand-off flags), gives up after `iters` polls,
+// records the timeout in the error word and returns.
+__global__ void selftest_wait_kernel(int* err, uint32_t iters) {
+  if (threadIdx.x != 0) return;
+  if (!sm100::wait_flag_ge(&g_never_set, 1ull, iters)) atomicOr(err, kErrTimeout);
+}
 
 // One error word per device.  Kernels OR bits into it (a bounded wait that
 // ran out, a malformed cu_seqlens); gdn_check_device_error reads and clears.
@@ -473,6 +485,15 @@ extern "C" gdn_status gdn_gr_write(uint8_t* codes, float* scales, const void* y,
   GrWriteArgs a;
   a.codes = codes; a.scales = scales; a.y = y; a.s = s; a.T = T; a.n_r = n_r; a.d = d;
   return launch_gr_write(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" gdn_status gdn_selftest_bounded_wait(int32_t iterations, gdn_stream_t stream) {
+  if (iterations < 1) return GDN_ERR_INVALID_ARG;
+  int* err = error_word_ptr();
+  if (err == nullptr) return GDN_ERR_CUDA;
+  selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      err, (uint32_t)iterations);
+  return cudaPeekAtLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
 extern "C" gdn_status gdn_check_device_error(gdn_stream_t stream) {

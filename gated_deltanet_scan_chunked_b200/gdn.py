@@ -108,6 +108,8 @@ def load(path: str = LIB_PATH):
     f = lib.gdn_gr_write
     f.restype = ctypes.c_int
     f.argtypes = [_vp] * 4 + [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, _vp]
+    lib.gdn_selftest_bounded_wait.restype = ctypes.c_int
+    lib.gdn_selftest_bounded_wait.argtypes = [ctypes.c_int32, _vp]
     lib.gdn_check_device_error.restype = ctypes.c_int
     lib.gdn_check_device_error.argtypes = [_vp]
     lib.gdn_status_string.restype = ctypes.c_char_p

@@ -457,6 +457,17 @@ gdn_status gdn_chunk_bwd(
  */
 gdn_status gdn_check_device_error(gdn_stream_t stream);
 
+/*
+ * gdn_selftest_bounded_wait -- exercises the failure path of the library's
+ * bounded waits without a fault: one thread waits on a device flag that
+ * nothing sets, with the same bounded poll the split prefill uses for its
+ * hand-off flags, gives up after `iterations` polls (each ~32 ns apart),
+ * records the timeout in the device error word and returns.  A following
+ * gdn_check_device_error reports GDN_ERR_TIMEOUT once, and the context stays
+ * usable.  (A test entry point; the pages have no counterpart.)
+ */
+gdn_status gdn_selftest_bounded_wait(int32_t iterations, gdn_stream_t stream);
+
 /* Static text for a status code. */
 const char* gdn_status_string(gdn_status status);
 

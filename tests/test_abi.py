@@ -286,3 +286,7 @@ def test_gr_entry_points_reject_on_host(lib):
     assert lib.gdn_gr_write(FAKE, FAKE, FAKE, FAKE, 64, 4, 12, None) == gdn.GDN_ERR_INVALID_ARG
     assert lib.gdn_gr_write(None, FAKE, FAKE, FAKE, 64, 4, 16, None) == gdn.GDN_ERR_INVALID_ARG
     assert lib.gdn_gr_write(None, None, None, None, 0, 4, 16, None) == gdn.GDN_OK
+
+
+def test_selftest_rejects_nonpositive_iterations(lib):
+    assert lib.gdn_selftest_bounded_wait(0, None) == gdn.GDN_ERR_INVALID_ARG

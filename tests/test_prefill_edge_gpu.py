@@ -13,7 +13,7 @@ import pytest
 import torch
 
 from gated_deltanet_scan_chunked_b200 import gdn, gdn_check_device_error, gdn_chunk_fwd, inputs
-from tests._parity import errors, oracle_prefill, to_device
+from tests._parity import assert_close, errors, oracle_prefill, to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -128,3 +128,19 @@ def test_deterministic():
     y1, s1 = _run(w, "auto")
     y2, s2 = _run(w, "auto")
     assert torch.equal(y1, y2) and torch.equal(s1, s2)
+
+
+def test_bounded_wait_times_out_and_context_stays_usable():
+    """A wait on a flag that nothing sets gives up, the host reads
+    GDN_ERR_TIMEOUT once, and the next prefill still runs and is correct."""
+    lib = gdn.load()
+    assert lib.gdn_selftest_bounded_wait(1 << 12, None) == gdn.GDN_OK
+    assert gdn_check_device_error() == gdn.GDN_ERR_TIMEOUT
+    assert gdn_check_device_error() == gdn.GDN_OK  # cleared
+    w = to_device(inputs.make_prefill([70], 2, 4, 16, 16, dtype=torch.float32, seed=3,
+                                      epilogue=False))
+    y, fs = gdn_chunk_fwd(w.q, w.k, w.v, w.log_alpha, w.beta, cu_seqlens=w.cu_seqlens)
+    torch.cuda.synchronize()
+    assert gdn_check_device_error() == gdn.GDN_OK
+    y_ref, s_ref, _ = oracle_prefill(w)
+    assert_close(y, y_ref, torch.float32, "after timeout y")
