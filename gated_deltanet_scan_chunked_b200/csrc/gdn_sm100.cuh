@@ -347,6 +347,10 @@ __device__ __forceinline__ void cp_async_commit() {
 __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_all;" ::: "memory");
 }
+// Wait until at most the most recently committed group is still in flight.
+__device__ __forceinline__ void cp_async_wait_group1() {
+  asm volatile("cp.async.wait_group 1;" ::: "memory");
+}
 
 // 2^x with the hardware approximation (relative error ~2^-22).
 __device__ __forceinline__ float ex2_approx(float x) {
