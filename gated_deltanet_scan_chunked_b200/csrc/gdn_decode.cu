@@ -35,6 +35,52 @@ struct DecodeGeom {
   static_assert(NT % TPR == 0 && DK % ROWG == 0 && RPT >= 1, "bad decode geometry");
 };
 
+// The per-row arithmetic both kernels share (so that T_s steps of the
+// multi-token kernel equal T_s single steps bit for bit), on column pairs
+// with the packed fp32 instructions.
+// a and b partial sums over one state row i: pa += S_i k^_i, pb += S_i q^_i.
+__device__ __forceinline__ void row_partials(const float4& s, float ki, float qi, uint64_t* pa,
+                                             uint64_t* pb) {
+  const uint64_t s0 = f2_pack(s.x, s.y), s1 = f2_pack(s.z, s.w);
+  const uint64_t k2 = f2_pack(ki, ki), q2 = f2_pack(qi, qi);
+  pa[0] = f2_fma(s0, k2, pa[0]);
+  pa[1] = f2_fma(s1, k2, pa[1]);
+  pb[0] = f2_fma(s0, q2, pb[0]);
+  pb[1] = f2_fma(s1, q2, pb[1]);
+}
+__device__ __forceinline__ float4 f2_to_float4(const uint64_t* p) {
+  float4 r;
+  f2_unpack(p[0], r.x, r.y);
+  f2_unpack(p[1], r.z, r.w);
+  return r;
+}
+// Sum over the row groups of their partial sums (in row-group order).
+template <int ROWG, int TPR>
+__device__ __forceinline__ void col_sums(const float4 (*red_a)[TPR], const float4 (*red_b)[TPR],
+                                         int c4, float4* ta, float4* tb) {
+  uint64_t sa[2] = {0ull, 0ull}, sb[2] = {0ull, 0ull};
+#pragma unroll
+  for (int g2 = 0; g2 < ROWG; ++g2) {
+    const float4 x = red_a[g2][c4], z = red_b[g2][c4];
+    sa[0] = f2_add(sa[0], f2_pack(x.x, x.y));
+    sa[1] = f2_add(sa[1], f2_pack(x.z, x.w));
+    sb[0] = f2_add(sb[0], f2_pack(z.x, z.y));
+    sb[1] = f2_add(sb[1], f2_pack(z.z, z.w));
+  }
+  *ta = f2_to_float4(sa);
+  *tb = f2_to_float4(sb);
+}
+// One state row after the step: alpha S_i + (beta k^_i) e, per column
+// fma(beta k^_i, e, alpha S_i) with the product alpha S_i rounded first.
+__device__ __forceinline__ float4 row_update(const float4& s, uint64_t alpha2, float bk,
+                                             const uint64_t* e2) {
+  const uint64_t b2 = f2_pack(bk, bk);
+  uint64_t o[2];
+  o[0] = f2_fma(b2, e2[0], f2_mul(alpha2, f2_pack(s.x, s.y)));
+  o[1] = f2_fma(b2, e2[1], f2_mul(alpha2, f2_pack(s.z, s.w)));
+  return f2_to_float4(o);
+}
+
 template <int DK, int DV, typename Tin>
 __global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT)
     gdn_decode_kernel(const DecodeArgs a) {
@@ -92,39 +138,32 @@ __global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT)
   const float rq = snorm[0], rk = snorm[1], kq = snorm[2];
 
   // a = S^T k^, b = S^T q^ over this thread's rows, then across row groups
-  float4 pa = make_float4(0.f, 0.f, 0.f, 0.f), pb = pa;
+  uint64_t pa[2] = {0ull, 0ull}, pb[2] = {0ull, 0ull};
   float kk[RPT];
 #pragma unroll
   for (int r = 0; r < RPT; ++r) {
     const int i = rg + ROWG * r;
     const float ki = sk[i] * rk, qi = sq[i] * rq;
     kk[r] = ki;
-    pa.x += s[r].x * ki; pa.y += s[r].y * ki; pa.z += s[r].z * ki; pa.w += s[r].w * ki;
-    pb.x += s[r].x * qi; pb.y += s[r].y * qi; pb.z += s[r].z * qi; pb.w += s[r].w * qi;
+    row_partials(s[r], ki, qi, pa, pb);
   }
-  red_a[rg][c4] = pa;
-  red_b[rg][c4] = pb;
+  red_a[rg][c4] = f2_to_float4(pa);
+  red_b[rg][c4] = f2_to_float4(pb);
   __syncthreads();
-  float4 ta = make_float4(0.f, 0.f, 0.f, 0.f), tb = ta;
-#pragma unroll
-  for (int g2 = 0; g2 < ROWG; ++g2) {
-    const float4 x = red_a[g2][c4], z = red_b[g2][c4];
-    ta.x += x.x; ta.y += x.y; ta.z += x.z; ta.w += x.w;
-    tb.x += z.x; tb.y += z.y; tb.z += z.z; tb.w += z.w;
-  }
+  float4 ta, tb;
+  col_sums<ROWG, TPR>(red_a, red_b, c4, &ta, &tb);
   float4 e;
   e.x = v4.x - alpha * ta.x; e.y = v4.y - alpha * ta.y;
   e.z = v4.z - alpha * ta.z; e.w = v4.w - alpha * ta.w;
 
   // S' = alpha S + beta k^ e^T, stored in place (each thread rewrites
   // exactly the elements it loaded)
+  const uint64_t alpha2 = f2_pack(alpha, alpha);
+  const uint64_t e2[2] = {f2_pack(e.x, e.y), f2_pack(e.z, e.w)};
 #pragma unroll
   for (int r = 0; r < RPT; ++r) {
     const int i = rg + ROWG * r;
-    const float bk = beta * kk[r];
-    float4 o;
-    o.x = alpha * s[r].x + bk * e.x; o.y = alpha * s[r].y + bk * e.y;
-    o.z = alpha * s[r].z + bk * e.z; o.w = alpha * s[r].w + bk * e.w;
+    const float4 o = row_update(s[r], alpha2, beta * kk[r], e2);
     __stcs(reinterpret_cast<float4*>(S + (size_t)i * DV) + c4, o);
   }
 
@@ -284,26 +323,20 @@ __global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT)
     kq = kq * rq * rk;  // the same association as the single-token kernel
 
     // a = S^T k^, b = S^T q^ over this thread's rows, then across row groups
-    float4 pa = make_float4(0.f, 0.f, 0.f, 0.f), pb = pa;
+    uint64_t pa[2] = {0ull, 0ull}, pb[2] = {0ull, 0ull};
     float kk[RPT];
 #pragma unroll
     for (int r = 0; r < RPT; ++r) {
       const int i = rg + ROWG * r;
       const float ki = sk[i] * rk, qi = sq[i] * rq;
       kk[r] = ki;
-      pa.x += s[r].x * ki; pa.y += s[r].y * ki; pa.z += s[r].z * ki; pa.w += s[r].w * ki;
-      pb.x += s[r].x * qi; pb.y += s[r].y * qi; pb.z += s[r].z * qi; pb.w += s[r].w * qi;
+      row_partials(s[r], ki, qi, pa, pb);
     }
-    red_a[par][rg][c4] = pa;
-    red_b[par][rg][c4] = pb;
+    red_a[par][rg][c4] = f2_to_float4(pa);
+    red_b[par][rg][c4] = f2_to_float4(pb);
     __syncthreads();  // (the other parity's buffers were read before this barrier)
-    float4 ta = make_float4(0.f, 0.f, 0.f, 0.f), tbv = ta;
-#pragma unroll
-    for (int g2 = 0; g2 < ROWG; ++g2) {
-      const float4 x = red_a[par][g2][c4], z = red_b[par][g2][c4];
-      ta.x += x.x; ta.y += x.y; ta.z += x.z; ta.w += x.w;
-      tbv.x += z.x; tbv.y += z.y; tbv.z += z.z; tbv.w += z.w;
-    }
+    float4 ta, tbv;
+    col_sums<ROWG, TPR>(red_a[par], red_b[par], c4, &ta, &tbv);
     const float4 v4 = *reinterpret_cast<const float4*>(tv + t * DV + 4 * c4);
     float4 e;
     e.x = v4.x - alpha * ta.x; e.y = v4.y - alpha * ta.y;
@@ -315,13 +348,12 @@ __global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT)
     float* snap = a.snapshots ? a.snapshots + ((size_t)t * a.N * a.H_v) * (size_t)(DK * DV) + so
                               : nullptr;
     float* sout = (t + 1 == T_s && a.state_out) ? a.state_out + so : nullptr;
+    const uint64_t alpha2 = f2_pack(alpha, alpha);
+    const uint64_t e2[2] = {f2_pack(e.x, e.y), f2_pack(e.z, e.w)};
 #pragma unroll
     for (int r = 0; r < RPT; ++r) {
       const int i = rg + ROWG * r;
-      const float bk = beta * kk[r];
-      float4 o;
-      o.x = alpha * s[r].x + bk * e.x; o.y = alpha * s[r].y + bk * e.y;
-      o.z = alpha * s[r].z + bk * e.z; o.w = alpha * s[r].w + bk * e.w;
+      const float4 o = row_update(s[r], alpha2, beta * kk[r], e2);
       s[r] = o;
       if (snap) __stcs(reinterpret_cast<float4*>(snap + (size_t)i * DV) + c4, o);
       if (sout) __stcs(reinterpret_cast<float4*>(sout + (size_t)i * DV) + c4, o);
