@@ -407,6 +407,15 @@ __device__ __forceinline__ void lds_row(const float* p, float* x) {
   }
 }
 
+// L2 prefetch of `rows` rows of `row_floats` floats (a multiple of 32: whole
+// 128-byte lines), `stride` floats apart, spread over the CTA's threads.
+__device__ __forceinline__ void prefetch_rows(const float* p, int rows, size_t stride,
+                                              int row_floats) {
+  const int lines = row_floats / 32;
+  for (int x = threadIdx.x; x < rows * lines; x += kNT)
+    sm100::prefetch_l2(p + (size_t)(x / lines) * stride + (x % lines) * 32);
+}
+
 // b_t = exp(G_C - G_t) for the chunk (warp 0), once per chunk
 __device__ __forceinline__ void chunk_decay(const float* sG, float* sB) {
   if (threadIdx.x < kC) sB[threadIdx.x] = expf(sG[kC - 1] - sG[threadIdx.x]);
@@ -463,6 +472,15 @@ __global__ void __launch_bounds__(kNT, 2) bwd_fwd_chain_kernel(const BwdArgs a) 
     cp_async_wait_all();
     __syncthreads();
     chunk_decay(sG, sB);
+    if (c + 1 < c_end) {
+      // the next chunk's inputs into L2 while this one is computed
+      const ChunkEnt e1 = ents[c + 1];
+      const size_t ch1 = (size_t)(c + 1) * a.H_v + h;
+      prefetch_rows(a.WT + ch1 * DK * kC, 1, 0, DK * kC);
+      prefetch_rows(a.kh + ((size_t)e1.t0 * a.H_qk + hq) * DK, e1.n, (size_t)a.H_qk * DK, DK);
+      prefetch_rows(a.UT + ch1 * kC * DV + j0, kC, DV, SW);
+      if (threadIdx.x == 0) sm100::prefetch_l2(a.G + ch1 * kC);
+    }
     // Delta = U - W S   (W^T rows give each thread's 4 rows in one load)
     for (int i = 0; i < DK; ++i) {
       float sv[NW], wv[4];
@@ -749,6 +767,16 @@ __global__ void __launch_bounds__(kNT, 2) bwd_bwd_chain_kernel(const BwdArgs a) 
     cp_async_wait_all();
     __syncthreads();
     chunk_decay(sG, sB);
+    if (c - 1 >= c_begin) {
+      // the next (earlier) chunk's inputs into L2 while this one is computed
+      const ChunkEnt e1 = ents[c - 1];
+      const size_t ch1 = (size_t)(c - 1) * a.H_v + h;
+      prefetch_rows(a.W + ch1 * kC * DK, 1, 0, kC * DK);
+      prefetch_rows(a.kh + ((size_t)e1.t0 * a.H_qk + hq) * DK, e1.n, (size_t)a.H_qk * DK, DK);
+      prefetch_rows(a.dS + ch1 * DK * DV + j0, DK, DV, SW);
+      prefetch_rows(a.dD + ch1 * kC * DV + j0, kC, DV, SW);
+      if (threadIdx.x == 0) sm100::prefetch_l2(a.G + ch1 * kC);
+    }
     // dDelta = X1 + diag(b) K dS1  (zero on rows past the chunk's end)
     {
       float kacc[4][NW];
