@@ -55,7 +55,7 @@ typedef struct CUstream_st* gdn_stream_t;
 typedef enum {
   GDN_OK = 0,
   GDN_ERR_INVALID_ARG = 1, /* null pointer, bad shape, bad cu_seqlens ...  */
-  GDN_ERR_UNSUPPORTED = 2, /* a head dim or dtype this build does not have */
+  GDN_ERR_UNSUPPORTED = 2, /* a head dim or dtype the library does not support */
   GDN_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed         */
   GDN_ERR_TIMEOUT = 4      /* a device-side wait hit its iteration limit   */
 } gdn_status;
