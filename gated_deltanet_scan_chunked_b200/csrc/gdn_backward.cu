@@ -482,6 +482,7 @@ __global__ void __launch_bounds__(kNT, 2) bwd_fwd_chain_kernel(const BwdArgs a) 
       if (threadIdx.x == 0) sm100::prefetch_l2(a.G + ch1 * kC);
     }
     // Delta = U - W S   (W^T rows give each thread's 4 rows in one load)
+#pragma unroll 8
     for (int i = 0; i < DK; ++i) {
       float sv[NW], wv[4];
 #pragma unroll
@@ -508,6 +509,7 @@ __global__ void __launch_bounds__(kNT, 2) bwd_fwd_chain_kernel(const BwdArgs a) 
     for (int u = 0; u < NK; ++u)
 #pragma unroll
       for (int w = 0; w < NW; ++w) sr[u][w] *= gC;
+#pragma unroll 8
     for (int t = 0; t < kC; ++t) {
       const float bt = sB[t];
       float dv[NW], kv[NK];
@@ -784,6 +786,7 @@ __global__ void __launch_bounds__(kNT, 2) bwd_bwd_chain_kernel(const BwdArgs a) 
       for (int u = 0; u < 4; ++u)
 #pragma unroll
         for (int w = 0; w < NW; ++w) kacc[u][w] = 0.f;
+#pragma unroll 8
       for (int i = 0; i < DK; ++i) {
         float sv[NW];
 #pragma unroll
@@ -817,6 +820,7 @@ __global__ void __launch_bounds__(kNT, 2) bwd_bwd_chain_kernel(const BwdArgs a) 
       for (int u = 0; u < NK; ++u)
 #pragma unroll
         for (int w = 0; w < NW; ++w) dr[u][w] = gC * dr[u][w] + x2[u][w];
+#pragma unroll 8
       for (int t = 0; t < kC; ++t) {
         float dv[NW], wv[NK];
 #pragma unroll
