@@ -62,9 +62,26 @@ __device__ __forceinline__ void bf16x8_store(__nv_bfloat16* p, const float* x) {
   *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+// Two E4M3 codes (low byte first) -> their values as an fp32 pair (exact).
+__device__ __forceinline__ uint64_t e4m3x2_to_f2(uint32_t c2) {
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((unsigned short)c2));
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+  return f2_pack(f.x, f.y);
+}
+// An fp32 pair -> two E4M3 codes (low byte = first), round to nearest even,
+// saturating to +-448.
+__device__ __forceinline__ uint32_t f2_to_e4m3x2(uint64_t v) {
+  float x0, x1;
+  f2_unpack(v, x0, x1);
+  unsigned short c;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(c) : "f"(x1), "f"(x0));
+  return c;
+}
+
 // gr_norm: one warp per (token, branch) row, the row's codes held in
 // registers (GPL groups of 8 per lane): R^ = dequant / sqrt(mean sq + eps) *
-// gamma, stored in bf16.
+// gamma, stored in bf16; the codes are decoded and scaled in pairs.
 template <int GPL>
 __global__ void __launch_bounds__(128) gr_norm_kernel(const GrArgs a) {
   const int64_t row = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
@@ -74,23 +91,26 @@ __global__ void __launch_bounds__(128) gr_norm_kernel(const GrArgs a) {
   const int g8 = a.d / 8;
   const uint8_t* codes = a.codes + (size_t)row * a.d;
   const float sc = __ldg(a.scales + row);
+  const uint64_t sc2 = f2_pack(sc, sc);
   uint2 raw[GPL];
 #pragma unroll
   for (int k = 0; k < GPL; ++k) {
     const int j = lane + 32 * k;
     raw[k] = j < g8 ? __ldg(reinterpret_cast<const uint2*>(codes) + j) : make_uint2(0u, 0u);
   }
-  float ss = 0.f;
+  uint64_t ss2 = 0ull;
 #pragma unroll
   for (int k = 0; k < GPL; ++k) {
-    const uint32_t w[2] = {raw[k].x, raw[k].y};
+    const uint32_t cw[2] = {raw[k].x, raw[k].y};
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float x = __fmul_rn(e4m3_to_float((w[i / 4] >> (8 * (i % 4))) & 0xFF), sc);
-      ss += x * x;
+    for (int p = 0; p < 4; ++p) {
+      const uint64_t x = f2_mul(e4m3x2_to_f2(cw[p / 2] >> (16 * (p % 2))), sc2);
+      ss2 = f2_fma(x, x, ss2);
     }
   }
-  ss = warp_sum(ss);
+  float s0, s1;
+  f2_unpack(ss2, s0, s1);
+  const float ss = warp_sum(s0 + s1);
   const float r = rsqrtf(ss / (float)a.d + a.eps);
   __nv_bfloat16* out = a.rhat + (size_t)row * a.d;
   const float* gam = a.gamma + (size_t)b * a.d;
@@ -98,14 +118,16 @@ __global__ void __launch_bounds__(128) gr_norm_kernel(const GrArgs a) {
   for (int k = 0; k < GPL; ++k) {
     const int j = lane + 32 * k;
     if (j < g8) {
-      const uint32_t w[2] = {raw[k].x, raw[k].y};
+      const uint32_t cw[2] = {raw[k].x, raw[k].y};
       const float4 g0 = __ldg(reinterpret_cast<const float4*>(gam + 8 * j));
       const float4 g1 = __ldg(reinterpret_cast<const float4*>(gam + 8 * j) + 1);
-      const float gm[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+      const uint64_t gm[4] = {f2_pack(g0.x * r, g0.y * r), f2_pack(g0.z * r, g0.w * r),
+                              f2_pack(g1.x * r, g1.y * r), f2_pack(g1.z * r, g1.w * r)};
       float x[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        x[i] = __fmul_rn(e4m3_to_float((w[i / 4] >> (8 * (i % 4))) & 0xFF), sc) * r * gm[i];
+      for (int p = 0; p < 4; ++p)
+        f2_unpack(f2_mul(f2_mul(e4m3x2_to_f2(cw[p / 2] >> (16 * (p % 2))), sc2), gm[p]),
+                  x[2 * p], x[2 * p + 1]);
       bf16x8_store(out + 8 * j, x);
     }
   }
@@ -137,7 +159,15 @@ __global__ void __launch_bounds__(kNT) gr_router_kernel(const GrArgs a, __nv_bfl
 }
 
 // gr_gate: x[t, c] = (1/n_r) sum_i sigmoid(L[t, i d + c]) R^[t, i d + c]; the
-// branches' loads are issued together
+// branches' loads are issued together.  sigmoid(l) = (1 + tanh(l / 2)) / 2
+// with the hardware tanh (relative error about 2^-11, below the bf16
+// rounding of L and R^), on channel pairs.
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+template <int NR>  // branches (n_r)
 __global__ void __launch_bounds__(kNT) gr_gate_kernel(const GrArgs a) {
   const int64_t idx = (int64_t)blockIdx.x * kNT + threadIdx.x;  // 8-channel group
   const int g8 = a.d / 8;
@@ -145,41 +175,47 @@ __global__ void __launch_bounds__(kNT) gr_gate_kernel(const GrArgs a) {
   const int64_t t = idx / g8;
   const int c = (int)(idx % g8) * 8;
   const size_t base = (size_t)t * a.n_r * a.d + c;
-  uint4 lr[kMaxGrBranches], rr[kMaxGrBranches];
+  uint4 lr[NR], rr[NR];
 #pragma unroll
-  for (int b = 0; b < kMaxGrBranches; ++b) {
-    if (b < a.n_r) {
-      lr[b] = __ldg(reinterpret_cast<const uint4*>(a.logits + base + (size_t)b * a.d));
-      rr[b] = __ldg(reinterpret_cast<const uint4*>(a.rhat + base + (size_t)b * a.d));
+  for (int b = 0; b < NR; ++b) {
+    lr[b] = __ldg(reinterpret_cast<const uint4*>(a.logits + base + (size_t)b * a.d));
+    rr[b] = __ldg(reinterpret_cast<const uint4*>(a.rhat + base + (size_t)b * a.d));
+  }
+  const uint64_t half2 = f2_pack(0.5f, 0.5f);
+  uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+  for (int b = 0; b < NR; ++b) {
+    const uint32_t lw[4] = {lr[b].x, lr[b].y, lr[b].z, lr[b].w};
+    const uint32_t rw[4] = {rr[b].x, rr[b].y, rr[b].z, rr[b].w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      // bf16 pairs: a bf16 is the high half of its fp32 value
+      const uint64_t l2 = f2_pack(__uint_as_float(lw[i] << 16), __uint_as_float(lw[i] & 0xffff0000u));
+      const uint64_t r2 = f2_pack(__uint_as_float(rw[i] << 16), __uint_as_float(rw[i] & 0xffff0000u));
+      float h0, h1;
+      f2_unpack(f2_mul(l2, half2), h0, h1);
+      const uint64_t g = f2_fma(f2_pack(tanh_approx(h0), tanh_approx(h1)), half2, half2);
+      acc[i] = f2_fma(g, r2, acc[i]);
     }
   }
-  float acc[8];
+  const float inv = 1.f / (float)NR;
+  float o[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-#pragma unroll
-  for (int b = 0; b < kMaxGrBranches; ++b) {
-    if (b < a.n_r) {
-      const uint32_t lw[4] = {lr[b].x, lr[b].y, lr[b].z, lr[b].w};
-      const uint32_t rw[4] = {rr[b].x, rr[b].y, rr[b].z, rr[b].w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 l = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&lw[i]));
-        const float2 r = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&rw[i]));
-        acc[2 * i] += __fdividef(r.x, 1.f + __expf(-l.x));
-        acc[2 * i + 1] += __fdividef(r.y, 1.f + __expf(-l.y));
-      }
-    }
+  for (int i = 0; i < 4; ++i) {
+    f2_unpack(acc[i], o[2 * i], o[2 * i + 1]);
+    o[2 * i] *= inv;
+    o[2 * i + 1] *= inv;
   }
-  const float inv = 1.f / (float)a.n_r;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i] *= inv;
-  bf16x8_store(static_cast<__nv_bfloat16*>(a.x) + (size_t)t * a.d + c, acc);
+  bf16x8_store(static_cast<__nv_bfloat16*>(a.x) + (size_t)t * a.d + c, o);
 }
 
 // gr_write: one warp per (token, branch) row, in place, the row's values
-// held in registers (GPL groups of 8 per lane).  r = deq + s y with one
-// rounding per operation; scale' = max|r| / 448 (1 if zero); inv = 1 /
-// scale'; code = E4M3(r * inv) with round to nearest even and saturation.
+// held in registers (GPL groups of 8 per lane, as fp32 pairs).  r = deq + s
+// y with one rounding per operation; scale' = max|r| / 448 (1 if zero); inv
+// = 1 / scale'; code = E4M3(r * inv) with round to nearest even and
+// saturation.  Decoding and encoding work on channel pairs (packed
+// conversions); the product and the sum stay scalar fp32 operations with
+// explicit rounding, so that they are never fused into one.
 template <int GPL>
 __global__ void __launch_bounds__(128) gr_write_kernel(const GrWriteArgs a) {
   const int64_t row = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
@@ -199,36 +235,37 @@ __global__ void __launch_bounds__(128) gr_write_kernel(const GrWriteArgs a) {
     raw[k] = j < g8 ? reinterpret_cast<const uint2*>(codes)[j] : make_uint2(0u, 0u);
     yr[k] = j < g8 ? __ldg(reinterpret_cast<const uint4*>(y) + j) : make_uint4(0u, 0u, 0u, 0u);
   }
-  float r[GPL][8];
+  uint64_t r[GPL][4];  // element pairs (2p, 2p + 1) of group k
   float amax = 0.f;
 #pragma unroll
   for (int k = 0; k < GPL; ++k) {
+    const uint32_t cw[2] = {raw[k].x, raw[k].y};
     const uint32_t yw[4] = {yr[k].x, yr[k].y, yr[k].z, yr[k].w};
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint32_t w = i < 4 ? raw[k].x : raw[k].y;
-      const float q = __fmul_rn(e4m3_to_float((w >> (8 * (i % 4))) & 0xFF), sc);
-      const float yv = __bfloat162float(__ushort_as_bfloat16(
-          (unsigned short)((i & 1) ? (yw[i / 2] >> 16) : (yw[i / 2] & 0xFFFFu))));
-      r[k][i] = __fadd_rn(q, __fmul_rn(sv, yv));
-      amax = fmaxf(amax, fabsf(r[k][i]));
+    for (int p = 0; p < 4; ++p) {
+      float d0, d1;
+      f2_unpack(e4m3x2_to_f2(cw[p / 2] >> (16 * (p % 2))), d0, d1);
+      const float r0 = __fadd_rn(__fmul_rn(d0, sc), __fmul_rn(sv, __uint_as_float(yw[p] << 16)));
+      const float r1 =
+          __fadd_rn(__fmul_rn(d1, sc), __fmul_rn(sv, __uint_as_float(yw[p] & 0xffff0000u)));
+      r[k][p] = f2_pack(r0, r1);
+      amax = fmaxf(amax, fmaxf(fabsf(r0), fabsf(r1)));
     }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   const float nsc = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
   const float inv = __fdiv_rn(1.f, nsc);
+  const uint64_t inv2 = f2_pack(inv, inv);
 #pragma unroll
   for (int k = 0; k < GPL; ++k) {
     const int j = lane + 32 * k;
     if (j < g8) {
-      uint32_t w[2] = {0u, 0u};
+      uint32_t w[2];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const uint32_t c =
-            __nv_cvt_float_to_fp8(__fmul_rn(r[k][i], inv), __NV_SATFINITE, __NV_E4M3);
-        w[i / 4] |= (c & 0xFFu) << (8 * (i % 4));
-      }
+      for (int h = 0; h < 2; ++h)
+        w[h] = f2_to_e4m3x2(f2_mul(r[k][2 * h], inv2)) |
+               (f2_to_e4m3x2(f2_mul(r[k][2 * h + 1], inv2)) << 16);
       reinterpret_cast<uint2*>(codes)[j] = make_uint2(w[0], w[1]);
     }
   }
@@ -364,7 +401,14 @@ gdn_status launch_gr_read(GrArgs a, void* ws, cudaStream_t stream) {
                kLtWorkspace, stream);
   if (st != GDN_OK) return st;
   const int64_t g2 = a.T * (a.d / 8);
-  gr_gate_kernel<<<(unsigned)((g2 + kNT - 1) / kNT), kNT, 0, stream>>>(a);
+  const unsigned gg = (unsigned)((g2 + kNT - 1) / kNT);
+  switch (a.n_r) {
+#define GDN_NR(n) \
+  case n: gr_gate_kernel<n><<<gg, kNT, 0, stream>>>(a); break;
+    GDN_NR(1) GDN_NR(2) GDN_NR(3) GDN_NR(4) GDN_NR(5) GDN_NR(6) GDN_NR(7) GDN_NR(8)
+#undef GDN_NR
+    default: return GDN_ERR_UNSUPPORTED;
+  }
   return cudaPeekAtLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
