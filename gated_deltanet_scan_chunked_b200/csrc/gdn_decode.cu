@@ -21,6 +21,7 @@
 // 128-bit load or store.
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
+#include "gdn_sm100.cuh"
 
 namespace gdn {
 namespace {
@@ -190,8 +191,12 @@ __global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT)
 
 // a.T_s tokens per sequence, the state in registers from token to token,
 // stored to state_out after the last token and optionally snapshotted after
-// every token.  All tokens' inputs (q, k, v, g, gates) are staged in shared
-// memory at the start, in flight together with the state loads; per token
+// every token.  The CTAs are persistent: each takes (sequence, value head)
+// items blockIdx.x, blockIdx.x + gridDim.x, ..., and while it runs the tokens
+// of one item the state of its next item is already on its way into shared
+// memory (16-byte asynchronous copies; every thread copies exactly the
+// elements it will read, so no barrier guards that buffer).  All tokens'
+// inputs (q, k, v, g, gates) are staged in shared memory per item; per token
 // there is then a single block barrier (the cross-warp reduction, double
 // buffered by token parity), the q/k norms being computed by every warp.
 template <int DK, int DV, typename Tin>
@@ -202,188 +207,204 @@ __global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT)
   extern __shared__ float4 dsm4[];
   __shared__ float4 red_a[2][ROWG][TPR], red_b[2][ROWG][TPR];
 
-  const int n = blockIdx.x / a.H_v;
-  const int h = blockIdx.x % a.H_v;
-  const int hq = h / (a.H_v / a.H_qk);
   const int tid = threadIdx.x, lane = tid & 31;
   const int rg = tid / TPR, c4 = tid % TPR;
   const bool has_g = a.g != nullptr;
   const int T_s = a.T_s;
+  // the next item's state [DK][DV] (16-byte aligned at the start), then the
   // staged inputs, fp32: q, k [T_s][DK]; v, g [T_s][DV]; log alpha, beta [T_s]
-  float* tq = reinterpret_cast<float*>(dsm4);
+  float4* sst = dsm4;
+  float* tq = reinterpret_cast<float*>(dsm4) + DK * DV;
   float* tk = tq + T_s * DK;
   float* tv = tk + T_s * DK;
   float* tg = tv + T_s * DV;
   float* tla = tg + (has_g ? T_s * DV : 0);
   float* tb = tla + T_s;
 
-  const size_t so = ((size_t)n * a.H_v + h) * (size_t)(DK * DV);
-  const float* Sin = a.state_in + so;
-  // issue every state load first: they are the bulk of the traffic
-  float4 s[RPT];
-#pragma unroll
-  for (int r = 0; r < RPT; ++r) {
-    const int i = rg + ROWG * r;
-    s[r] = __ldcs(reinterpret_cast<const float4*>(Sin + (size_t)i * DV) + c4);
-  }
-  // front end: this thread's channels' conv weights and carried inputs,
-  // fetched together with the state
-  constexpr int SROW = 2 * DK + DV;
-  constexpr int CPT = (SROW + NT - 1) / NT;  // channels per thread
-  float4 cwr[CPT];
-  float cxr[CPT][3];
-  float* cst = (a.conv_w && a.conv_state) ? a.conv_state + ((size_t)n * a.H_v + h) * 3 * SROW
-                                          : nullptr;
-  if (a.conv_w != nullptr) {
-#pragma unroll
-    for (int u = 0; u < CPT; ++u) {
-      const int c = tid + u * NT;
-      if (c < SROW) {
-        const int wrow = c < DK ? hq * DK + c
-                         : c < 2 * DK ? (a.H_qk + hq) * DK + (c - DK)
-                                      : 2 * a.H_qk * DK + h * DV + (c - 2 * DK);
-        cwr[u] = __ldg(reinterpret_cast<const float4*>(a.conv_w) + wrow);
-#pragma unroll
-        for (int r = 0; r < 3; ++r) cxr[u][r] = cst ? cst[r * SROW + c] : 0.f;
-      }
-    }
-  }
-  {
-    const Tin* Q = static_cast<const Tin*>(a.q);
-    const Tin* K = static_cast<const Tin*>(a.k);
-    const Tin* V = static_cast<const Tin*>(a.v);
-    const Tin* G = static_cast<const Tin*>(a.g);
-    for (int i = tid; i < T_s * DK; i += NT) {
-      const size_t tok = (size_t)n * T_s + i / DK;
-      tq[i] = Elem<Tin>::load(Q + (tok * a.H_qk + hq) * DK + i % DK);
-      tk[i] = Elem<Tin>::load(K + (tok * a.H_qk + hq) * DK + i % DK);
-    }
-    for (int i = tid; i < T_s * DV; i += NT) {
-      const size_t tok = (size_t)n * T_s + i / DV;
-      tv[i] = Elem<Tin>::load(V + (tok * a.H_v + h) * DV + i % DV);
-      if (has_g) tg[i] = Elem<Tin>::load(G + (tok * a.H_v + h) * DV + i % DV);
-    }
-    for (int i = tid; i < T_s; i += NT) {
-      const size_t tok = (size_t)n * T_s + i;
-      tla[i] = __ldg(a.log_alpha + tok * a.H_v + h);
-      tb[i] = __ldg(a.beta + tok * a.H_v + h);
-    }
-  }
-  float4 w4 = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (has_g && a.norm_w) w4 = __ldg(reinterpret_cast<const float4*>(a.norm_w + 4 * c4));
-  if (a.conv_w != nullptr) {
-    // front end: causal depthwise conv of kernel 4, then SiLU, over each
-    // q / k / v channel of this (sequence, value head), in place on the
-    // staged inputs; the three inputs before the first token come from this
-    // value head's conv state, which is then rewritten with the last three
-    __syncthreads();  // raw inputs staged
-#pragma unroll
-    for (int u = 0; u < CPT; ++u) {
-      const int c = tid + u * NT;
-      if (c >= SROW) break;
-      float* col = c < DK ? tq + c : c < 2 * DK ? tk + (c - DK) : tv + (c - 2 * DK);
-      const int stride = c < 2 * DK ? DK : DV;
-      const float4 cw = cwr[u];
-      float x3 = cxr[u][0], x2 = cxr[u][1], x1 = cxr[u][2];  // inputs 3, 2, 1 tokens back
-      for (int t = 0; t < T_s; ++t) {
-        const float x = col[t * stride];
-        const float uu = cw.w * x + cw.z * x1 + cw.y * x2 + cw.x * x3;
-        col[t * stride] = uu / (1.f + __expf(-uu));
-        x3 = x2;
-        x2 = x1;
-        x1 = x;
-      }
-      if (cst) {
-        cst[c] = x3;
-        cst[SROW + c] = x2;
-        cst[2 * SROW + c] = x1;
-      }
-    }
-  }
-  __syncthreads();
-
-  for (int t = 0; t < T_s; ++t) {
-    const int par = t & 1;
-    const float* sq = tq + t * DK;
-    const float* sk = tk + t * DK;
-    const float alpha = __expf(tla[t]);
-    const float beta = tb[t];
-    // norms and k.q, computed by every warp (no barrier)
-    float nq = 0.f, nk = 0.f, kq = 0.f;
-    for (int i = lane; i < DK; i += 32) {
-      nq += sq[i] * sq[i];
-      nk += sk[i] * sk[i];
-      kq += sk[i] * sq[i];
-    }
-    nq = warp_sum(nq);
-    nk = warp_sum(nk);
-    kq = warp_sum(kq);
-    const float rq = a.l2norm ? rsqrtf(nq + a.eps_l2) : 1.f;
-    const float rk = a.l2norm ? rsqrtf(nk + a.eps_l2) : 1.f;
-    kq = kq * rq * rk;  // the same association as the single-token kernel
-
-    // a = S^T k^, b = S^T q^ over this thread's rows, then across row groups
-    uint64_t pa[2] = {0ull, 0ull}, pb[2] = {0ull, 0ull};
-    float kk[RPT];
+  const int items = a.N * a.H_v;
+  // this thread's elements of an item's state into the buffer
+  auto prefetch_state = [&](int it) {
+    const float* Sin = a.state_in + (size_t)it * (DK * DV);
 #pragma unroll
     for (int r = 0; r < RPT; ++r) {
       const int i = rg + ROWG * r;
-      const float ki = sk[i] * rk, qi = sq[i] * rq;
-      kk[r] = ki;
-      row_partials(s[r], ki, qi, pa, pb);
+      sm100::cp_async16(sm100::smem_u32(sst + i * TPR + c4), Sin + (size_t)i * DV + 4 * c4, true);
     }
-    red_a[par][rg][c4] = f2_to_float4(pa);
-    red_b[par][rg][c4] = f2_to_float4(pb);
-    __syncthreads();  // (the other parity's buffers were read before this barrier)
-    float4 ta, tbv;
-    col_sums<ROWG, TPR>(red_a[par], red_b[par], c4, &ta, &tbv);
-    const float4 v4 = *reinterpret_cast<const float4*>(tv + t * DV + 4 * c4);
-    float4 e;
-    e.x = v4.x - alpha * ta.x; e.y = v4.y - alpha * ta.y;
-    e.z = v4.z - alpha * ta.z; e.w = v4.w - alpha * ta.w;
-
-    // S' = alpha S + beta k^ e^T (each thread updates exactly the elements it
-    // loaded), kept in registers, optionally snapshotted, stored to
-    // state_out after the last token
-    float* snap = a.snapshots ? a.snapshots + ((size_t)t * a.N * a.H_v) * (size_t)(DK * DV) + so
-                              : nullptr;
-    float* sout = (t + 1 == T_s && a.state_out) ? a.state_out + so : nullptr;
-    const uint64_t alpha2 = f2_pack(alpha, alpha);
-    const uint64_t e2[2] = {f2_pack(e.x, e.y), f2_pack(e.z, e.w)};
+    sm100::cp_async_commit();
+  };
+  if ((int)blockIdx.x < items) prefetch_state(blockIdx.x);
+  for (int item = blockIdx.x; item < items; item += gridDim.x) {
+    const int n = item / a.H_v;
+    const int h = item % a.H_v;
+    const int hq = h / (a.H_v / a.H_qk);
+    const size_t so = (size_t)item * (size_t)(DK * DV);
+    // front end: this thread's channels' conv weights and carried inputs,
+    // fetched together with the state
+    constexpr int SROW = 2 * DK + DV;
+    constexpr int CPT = (SROW + NT - 1) / NT;  // channels per thread
+    float4 cwr[CPT];
+    float cxr[CPT][3];
+    float* cst = (a.conv_w && a.conv_state) ? a.conv_state + ((size_t)n * a.H_v + h) * 3 * SROW
+                                            : nullptr;
+    if (a.conv_w != nullptr) {
 #pragma unroll
-    for (int r = 0; r < RPT; ++r) {
-      const int i = rg + ROWG * r;
-      const float4 o = row_update(s[r], alpha2, beta * kk[r], e2);
-      s[r] = o;
-      if (snap) __stcs(reinterpret_cast<float4*>(snap + (size_t)i * DV) + c4, o);
-      if (sout) __stcs(reinterpret_cast<float4*>(sout + (size_t)i * DV) + c4, o);
+      for (int u = 0; u < CPT; ++u) {
+        const int c = tid + u * NT;
+        if (c < SROW) {
+          const int wrow = c < DK ? hq * DK + c
+                           : c < 2 * DK ? (a.H_qk + hq) * DK + (c - DK)
+                                        : 2 * a.H_qk * DK + h * DV + (c - 2 * DK);
+          cwr[u] = __ldg(reinterpret_cast<const float4*>(a.conv_w) + wrow);
+#pragma unroll
+          for (int r = 0; r < 3; ++r) cxr[u][r] = cst ? cst[r * SROW + c] : 0.f;
+        }
+      }
     }
+    {
+      const Tin* Q = static_cast<const Tin*>(a.q);
+      const Tin* K = static_cast<const Tin*>(a.k);
+      const Tin* V = static_cast<const Tin*>(a.v);
+      const Tin* G = static_cast<const Tin*>(a.g);
+      for (int i = tid; i < T_s * DK; i += NT) {
+        const size_t tok = (size_t)n * T_s + i / DK;
+        tq[i] = Elem<Tin>::load(Q + (tok * a.H_qk + hq) * DK + i % DK);
+        tk[i] = Elem<Tin>::load(K + (tok * a.H_qk + hq) * DK + i % DK);
+      }
+      for (int i = tid; i < T_s * DV; i += NT) {
+        const size_t tok = (size_t)n * T_s + i / DV;
+        tv[i] = Elem<Tin>::load(V + (tok * a.H_v + h) * DV + i % DV);
+        if (has_g) tg[i] = Elem<Tin>::load(G + (tok * a.H_v + h) * DV + i % DV);
+      }
+      for (int i = tid; i < T_s; i += NT) {
+        const size_t tok = (size_t)n * T_s + i;
+        tla[i] = __ldg(a.log_alpha + tok * a.H_v + h);
+        tb[i] = __ldg(a.beta + tok * a.H_v + h);
+      }
+    }
+    float4 w4 = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (has_g && a.norm_w) w4 = __ldg(reinterpret_cast<const float4*>(a.norm_w + 4 * c4));
+    // this item's state (its copies have landed), then the next item's copies
+    // into the same slots
+    float4 s[RPT];
+    sm100::cp_async_wait_all();
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) s[r] = sst[(rg + ROWG * r) * TPR + c4];
+    if (item + (int)gridDim.x < items) prefetch_state(item + gridDim.x);
+    if (a.conv_w != nullptr) {
+      // front end: causal depthwise conv of kernel 4, then SiLU, over each
+      // q / k / v channel of this (sequence, value head), in place on the
+      // staged inputs; the three inputs before the first token come from this
+      // value head's conv state, which is then rewritten with the last three
+      __syncthreads();  // raw inputs staged
+#pragma unroll
+      for (int u = 0; u < CPT; ++u) {
+        const int c = tid + u * NT;
+        if (c >= SROW) break;
+        float* col = c < DK ? tq + c : c < 2 * DK ? tk + (c - DK) : tv + (c - 2 * DK);
+        const int stride = c < 2 * DK ? DK : DV;
+        const float4 cw = cwr[u];
+        float x3 = cxr[u][0], x2 = cxr[u][1], x1 = cxr[u][2];  // inputs 3, 2, 1 tokens back
+        for (int t = 0; t < T_s; ++t) {
+          const float x = col[t * stride];
+          const float uu = cw.w * x + cw.z * x1 + cw.y * x2 + cw.x * x3;
+          col[t * stride] = uu / (1.f + __expf(-uu));
+          x3 = x2;
+          x2 = x1;
+          x1 = x;
+        }
+        if (cst) {
+          cst[c] = x3;
+          cst[SROW + c] = x2;
+          cst[2 * SROW + c] = x1;
+        }
+      }
+    }
+    __syncthreads();
 
-    // y = scale (alpha b + beta (k^.q^) e), then the optional epilogue
-    const size_t tok = (size_t)n * T_s + t;
-    const float bkq = beta * kq;
-    float4 y;
-    y.x = a.scale * (alpha * tbv.x + bkq * e.x); y.y = a.scale * (alpha * tbv.y + bkq * e.y);
-    y.z = a.scale * (alpha * tbv.z + bkq * e.z); y.w = a.scale * (alpha * tbv.w + bkq * e.w);
-    const size_t yo = (tok * a.H_v + h) * DV + 4 * c4;
-    if (has_g) {
-      float ss = y.x * y.x + y.y * y.y + y.z * y.z + y.w * y.w;
-      ss = group_sum<TPR>(ss);  // every row group holds the same y
-      const float r = rsqrtf(ss / (float)DV + a.eps_norm);
-      const float4 g4 = *reinterpret_cast<const float4*>(tg + t * DV + 4 * c4);
-      y.x = y.x * r * (1.f + w4.x) * sigmoidf_(g4.x);
-      y.y = y.y * r * (1.f + w4.y) * sigmoidf_(g4.y);
-      y.z = y.z * r * (1.f + w4.z) * sigmoidf_(g4.z);
-      y.w = y.w * r * (1.f + w4.w) * sigmoidf_(g4.w);
-    }
-    if (rg == 0) Elem<Tin>::store4(static_cast<Tin*>(a.y) + yo, y);
-  }  // tokens
+    for (int t = 0; t < T_s; ++t) {
+      const int par = t & 1;
+      const float* sq = tq + t * DK;
+      const float* sk = tk + t * DK;
+      const float alpha = __expf(tla[t]);
+      const float beta = tb[t];
+      // norms and k.q, computed by every warp (no barrier)
+      float nq = 0.f, nk = 0.f, kq = 0.f;
+      for (int i = lane; i < DK; i += 32) {
+        nq += sq[i] * sq[i];
+        nk += sk[i] * sk[i];
+        kq += sk[i] * sq[i];
+      }
+      nq = warp_sum(nq);
+      nk = warp_sum(nk);
+      kq = warp_sum(kq);
+      const float rq = a.l2norm ? rsqrtf(nq + a.eps_l2) : 1.f;
+      const float rk = a.l2norm ? rsqrtf(nk + a.eps_l2) : 1.f;
+      kq = kq * rq * rk;  // the same association as the single-token kernel
+
+      // a = S^T k^, b = S^T q^ over this thread's rows, then across row groups
+      uint64_t pa[2] = {0ull, 0ull}, pb[2] = {0ull, 0ull};
+      float kk[RPT];
+#pragma unroll
+      for (int r = 0; r < RPT; ++r) {
+        const int i = rg + ROWG * r;
+        const float ki = sk[i] * rk, qi = sq[i] * rq;
+        kk[r] = ki;
+        row_partials(s[r], ki, qi, pa, pb);
+      }
+      red_a[par][rg][c4] = f2_to_float4(pa);
+      red_b[par][rg][c4] = f2_to_float4(pb);
+      __syncthreads();  // (the other parity's buffers were read before this barrier)
+      float4 ta, tbv;
+      col_sums<ROWG, TPR>(red_a[par], red_b[par], c4, &ta, &tbv);
+      const float4 v4 = *reinterpret_cast<const float4*>(tv + t * DV + 4 * c4);
+      float4 e;
+      e.x = v4.x - alpha * ta.x; e.y = v4.y - alpha * ta.y;
+      e.z = v4.z - alpha * ta.z; e.w = v4.w - alpha * ta.w;
+
+      // S' = alpha S + beta k^ e^T (each thread updates exactly the elements it
+      // loaded), kept in registers, optionally snapshotted, stored to
+      // state_out after the last token
+      float* snap = a.snapshots ? a.snapshots + ((size_t)t * a.N * a.H_v) * (size_t)(DK * DV) + so
+                                : nullptr;
+      float* sout = (t + 1 == T_s && a.state_out) ? a.state_out + so : nullptr;
+      const uint64_t alpha2 = f2_pack(alpha, alpha);
+      const uint64_t e2[2] = {f2_pack(e.x, e.y), f2_pack(e.z, e.w)};
+#pragma unroll
+      for (int r = 0; r < RPT; ++r) {
+        const int i = rg + ROWG * r;
+        const float4 o = row_update(s[r], alpha2, beta * kk[r], e2);
+        s[r] = o;
+        if (snap) __stcs(reinterpret_cast<float4*>(snap + (size_t)i * DV) + c4, o);
+        if (sout) __stcs(reinterpret_cast<float4*>(sout + (size_t)i * DV) + c4, o);
+      }
+
+      // y = scale (alpha b + beta (k^.q^) e), then the optional epilogue
+      const size_t tok = (size_t)n * T_s + t;
+      const float bkq = beta * kq;
+      float4 y;
+      y.x = a.scale * (alpha * tbv.x + bkq * e.x); y.y = a.scale * (alpha * tbv.y + bkq * e.y);
+      y.z = a.scale * (alpha * tbv.z + bkq * e.z); y.w = a.scale * (alpha * tbv.w + bkq * e.w);
+      const size_t yo = (tok * a.H_v + h) * DV + 4 * c4;
+      if (has_g) {
+        float ss = y.x * y.x + y.y * y.y + y.z * y.z + y.w * y.w;
+        ss = group_sum<TPR>(ss);  // every row group holds the same y
+        const float r = rsqrtf(ss / (float)DV + a.eps_norm);
+        const float4 g4 = *reinterpret_cast<const float4*>(tg + t * DV + 4 * c4);
+        y.x = y.x * r * (1.f + w4.x) * sigmoidf_(g4.x);
+        y.y = y.y * r * (1.f + w4.y) * sigmoidf_(g4.y);
+        y.z = y.z * r * (1.f + w4.z) * sigmoidf_(g4.z);
+        y.w = y.w * r * (1.f + w4.w) * sigmoidf_(g4.w);
+      }
+      if (rg == 0) Elem<Tin>::store4(static_cast<Tin*>(a.y) + yo, y);
+    }  // tokens
+    __syncthreads();  // the staged inputs and the reduction buffers are refilled for the next item
+  }  // items
 }
 
 // Dynamic shared memory of the multi-token kernel for T_s tokens.
 template <int DK, int DV>
 size_t multi_smem_bytes(int T_s, bool has_g) {
-  return sizeof(float) * (size_t)T_s * (2 * DK + (has_g ? 2 : 1) * DV + 2);
+  return sizeof(float) * ((size_t)DK * DV + (size_t)T_s * (2 * DK + (has_g ? 2 : 1) * DV + 2));
 }
 
 template <int DK, int DV, typename Tin>
@@ -409,7 +430,16 @@ gdn_status launch(const DecodeArgs& a, cudaStream_t stream) {
         if (dev >= 0 && dev < 64) opted[dev] = true;
       }
     }
-    gdn_decode_multi_kernel<DK, DV, Tin><<<grid, DecodeGeom<DK, DV>::NT, smem, stream>>>(a);
+    // persistent CTAs: as many as can be resident at once (at most one per item)
+    auto fn = gdn_decode_multi_kernel<DK, DV, Tin>;
+    int dev = 0, sms = 0, per_sm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, DecodeGeom<DK, DV>::NT, smem) !=
+            cudaSuccess)
+      return GDN_ERR_CUDA;
+    const unsigned cap = (unsigned)(per_sm > 0 ? per_sm : 1) * (unsigned)sms;
+    fn<<<grid < cap ? grid : cap, DecodeGeom<DK, DV>::NT, smem, stream>>>(a);
   }
   return cudaPeekAtLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
