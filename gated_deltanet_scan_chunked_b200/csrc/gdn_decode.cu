@@ -200,7 +200,7 @@ __global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT)
 // there is then a single block barrier (the cross-warp reduction, double
 // buffered by token parity), the q/k norms being computed by every warp.
 template <int DK, int DV, typename Tin>
-__global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT)
+__global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT, 2)
     gdn_decode_multi_kernel(const DecodeArgs a) {
   using Geo = DecodeGeom<DK, DV>;
   constexpr int TPR = Geo::TPR, ROWG = Geo::ROWG, RPT = Geo::RPT, NT = Geo::NT;
@@ -212,7 +212,8 @@ __global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT)
   const bool has_g = a.g != nullptr;
   const int T_s = a.T_s;
   // the next item's state [DK][DV] (16-byte aligned at the start), then the
-  // staged inputs, fp32: q, k [T_s][DK]; v, g [T_s][DV]; log alpha, beta [T_s]
+  // staged inputs, fp32: q, k [T_s][DK]; v, g [T_s][DV]; log alpha, beta,
+  // k^ . q^ [T_s]
   float4* sst = dsm4;
   float* tq = reinterpret_cast<float*>(dsm4) + DK * DV;
   float* tk = tq + T_s * DK;
@@ -220,6 +221,7 @@ __global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT)
   float* tg = tv + T_s * DV;
   float* tla = tg + (has_g ? T_s * DV : 0);
   float* tb = tla + T_s;
+  float* tkq = tb + T_s;  // k^ . q^ per token
 
   const int items = a.N * a.H_v;
   // this thread's elements of an item's state into the buffer
@@ -320,14 +322,12 @@ __global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT)
       }
     }
     __syncthreads();
-
-    for (int t = 0; t < T_s; ++t) {
-      const int par = t & 1;
-      const float* sq = tq + t * DK;
-      const float* sk = tk + t * DK;
-      const float alpha = __expf(tla[t]);
-      const float beta = tb[t];
-      // norms and k.q, computed by every warp (no barrier)
+    // once per token: the q/k norms and k^ . q^ (one warp per token, with the
+    // single-token kernel's lane partition and order), then q and k
+    // normalised in place
+    for (int t = tid >> 5; t < T_s; t += NT / 32) {
+      float* sq = tq + t * DK;
+      float* sk = tk + t * DK;
       float nq = 0.f, nk = 0.f, kq = 0.f;
       for (int i = lane; i < DK; i += 32) {
         nq += sq[i] * sq[i];
@@ -339,7 +339,22 @@ __global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT)
       kq = warp_sum(kq);
       const float rq = a.l2norm ? rsqrtf(nq + a.eps_l2) : 1.f;
       const float rk = a.l2norm ? rsqrtf(nk + a.eps_l2) : 1.f;
-      kq = kq * rq * rk;  // the same association as the single-token kernel
+      if (lane == 0) tkq[t] = kq * rq * rk;  // the same association as the single-token kernel
+      __syncwarp();
+      for (int i = lane; i < DK; i += 32) {
+        sq[i] *= rq;
+        sk[i] *= rk;
+      }
+    }
+    __syncthreads();
+
+    for (int t = 0; t < T_s; ++t) {
+      const int par = t & 1;
+      const float* sq = tq + t * DK;  // q^
+      const float* sk = tk + t * DK;  // k^
+      const float alpha = __expf(tla[t]);
+      const float beta = tb[t];
+      const float kq = tkq[t];
 
       // a = S^T k^, b = S^T q^ over this thread's rows, then across row groups
       uint64_t pa[2] = {0ull, 0ull}, pb[2] = {0ull, 0ull};
@@ -347,7 +362,7 @@ __global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT)
 #pragma unroll
       for (int r = 0; r < RPT; ++r) {
         const int i = rg + ROWG * r;
-        const float ki = sk[i] * rk, qi = sq[i] * rq;
+        const float ki = sk[i], qi = sq[i];
         kk[r] = ki;
         row_partials(s[r], ki, qi, pa, pb);
       }
@@ -404,7 +419,7 @@ __global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT)
 // Dynamic shared memory of the multi-token kernel for T_s tokens.
 template <int DK, int DV>
 size_t multi_smem_bytes(int T_s, bool has_g) {
-  return sizeof(float) * ((size_t)DK * DV + (size_t)T_s * (2 * DK + (has_g ? 2 : 1) * DV + 2));
+  return sizeof(float) * ((size_t)DK * DV + (size_t)T_s * (2 * DK + (has_g ? 2 : 1) * DV + 3));
 }
 
 template <int DK, int DV, typename Tin>
