@@ -40,6 +40,9 @@ struct PrefillArgs {
   // flags, laid out by prefill_tc_workspace_bytes.
   void* ring = nullptr;
   unsigned long long* ring_flags = nullptr;
+  // Larger batches with a workspace: the order in which the one-CTA layout
+  // takes the sequences, longest first (nullptr: in index order).
+  int32_t* seq_order = nullptr;
   // Front end fused into the portable kernel (nullptr: q, k, v are used as
   // given): conv weights [2 H_qk d_k + H_v d_v, 4] and the per-value-head conv
   // states [n_seq, H_v, 3, 2 d_k + d_v] before / after each sequence.

@@ -413,7 +413,9 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
   uint64_t* bar = reinterpret_cast<uint64_t*>(gb + OFF_BAR);
   uint32_t* tslot = reinterpret_cast<uint32_t*>(gb + OFF_BAR + 8);
 
-  const int seq = blockIdx.x / a.H_v;
+  // (sequence, value head) item: sequences longest first when the order is
+  // given, so that the long ones do not start in the last wave
+  const int seq = a.seq_order ? a.seq_order[blockIdx.x / a.H_v] : (int)(blockIdx.x / a.H_v);
   const int h = blockIdx.x % a.H_v;
   const int hq = h / (a.H_v / a.H_qk);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1924,6 +1926,30 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
   }
 }
 
+// Larger batches (more than kSplitMaxItems items, at most kMaxOrderSeqs
+// sequences) with a workspace: the one-CTA layout takes the sequences
+// longest first.
+constexpr int kMaxOrderSeqs = 1024;
+
+// order[r] = the sequence of rank r by decreasing length (ties: lower index
+// first); one CTA of kMaxOrderSeqs threads, one sequence each.  cu_seqlens
+// is only read: the prefill kernel validates it.
+__global__ void __launch_bounds__(kMaxOrderSeqs) order_by_length_kernel(const int32_t* cu,
+                                                                        int n_seq,
+                                                                        int64_t total_T,
+                                                                        int32_t* order) {
+  __shared__ int64_t len[kMaxOrderSeqs];
+  const int s = threadIdx.x;
+  if (s < n_seq) len[s] = cu ? (int64_t)cu[s + 1] - cu[s] : total_T;
+  __syncthreads();
+  if (s < n_seq) {
+    const int64_t ls = len[s];
+    int rank = 0;
+    for (int j = 0; j < n_seq; ++j) rank += (len[j] > ls || (len[j] == ls && j < s)) ? 1 : 0;
+    order[rank] = s;
+  }
+}
+
 }  // namespace
 
 bool prefill_tc_supports(const PrefillArgs& a) {
@@ -1933,6 +1959,8 @@ bool prefill_tc_supports(const PrefillArgs& a) {
 // Split-launch workspace: flags (ready[kRing], consumed[kRing] per item,
 // 64-bit), padded to 256 bytes, then the ring slots (kSlotBytes each, a
 // multiple of 256).  Only batches of at most kSplitMaxItems items can use it.
+// Larger batches of at most kMaxOrderSeqs sequences use the workspace for
+// the one-CTA layout's sequence order instead (n_seq int32, longest first).
 constexpr long long kSplitMaxItems = 64;
 
 static size_t split_flag_bytes(long long items) {
@@ -1942,13 +1970,18 @@ static size_t split_flag_bytes(long long items) {
 size_t prefill_tc_workspace_bytes(int32_t n_seq, int32_t H_v, int32_t d_k, int32_t d_v,
                                   gdn_dtype dtype) {
   const long long items = (long long)n_seq * H_v;
-  if (dtype != GDN_BF16 || d_k != kD || d_v != kD || items < 1 || items > kSplitMaxItems)
-    return 0;
+  if (dtype != GDN_BF16 || d_k != kD || d_v != kD || items < 1) return 0;
+  if (items > kSplitMaxItems)
+    return n_seq <= kMaxOrderSeqs ? (((size_t)n_seq * sizeof(int32_t) + 255) & ~(size_t)255) : 0;
   return split_flag_bytes(items) + (size_t)items * kRing * kSlotBytes;
 }
 
 void prefill_tc_workspace_layout(void* ws, int32_t n_seq, int32_t H_v, PrefillArgs* a) {
   const long long items = (long long)n_seq * H_v;
+  if (items > kSplitMaxItems) {
+    a->seq_order = static_cast<int32_t*>(ws);
+    return;
+  }
   a->ring_flags = static_cast<unsigned long long*>(ws);
   a->ring = static_cast<uint8_t*>(ws) + split_flag_bytes(items);
 }
@@ -2068,6 +2101,10 @@ gdn_status launch_prefill_tc(const PrefillArgs& a, cudaStream_t stream) {
                                  : cudaLaunchKernelEx(&cfg, gdn_prefill_tc_pair_kernel<1, false>, a);
     if (err != cudaSuccess) return GDN_ERR_CUDA;
   } else {
+    if (a.seq_order != nullptr) {
+      order_by_length_kernel<<<1, kMaxOrderSeqs, 0, stream>>>(a.cu_seqlens, a.n_seq, a.total_T,
+                                                              a.seq_order);
+    }
     gdn_prefill_tc_kernel<<<(unsigned)items, kNT, kSmemBytes, stream>>>(a);
   }
   return cudaPeekAtLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;

@@ -48,7 +48,8 @@ extern "C" gdn_status gdn_chunk_fwd_static_ws(
   if (n_seq < 1 || H_v < 1) return GDN_ERR_INVALID_ARG;
   const size_t need = gdn_chunk_fwd_workspace_size(n_seq, H_v, d_k, d_v, in_dtype);
   // a shape the split layout does not serve, or more items than the array holds
-  if (need == 0 || need > gdn::kStaticBytes) return GDN_ERR_UNSUPPORTED;
+  if ((long long)n_seq * H_v > gdn::kStaticItems || need == 0 || need > gdn::kStaticBytes)
+    return GDN_ERR_UNSUPPORTED;
   void* ws = gdn::static_ws_ptr();
   if (ws == nullptr) return GDN_ERR_CUDA;
   // the split launch clears the array's flags on `stream` before its kernel

@@ -125,18 +125,22 @@ gdn_status gdn_chunk_fwd_path(
 
 /*
  * gdn_chunk_fwd_workspace_size -- bytes of device workspace that
- * gdn_chunk_fwd_ws can use for a batch of n_seq sequences x H_v value heads
- * (the split layout: a ring of four 80.25 KB hand-off slots plus 64 bytes of
- * flags per item).  Returns 0 when that layout cannot apply to the shape:
- * not bf16 with d_k = d_v = 128, or more than 64 items.  Host only; no CUDA
- * call.
+ * gdn_chunk_fwd_ws can use for a batch of n_seq sequences x H_v value heads.
+ * Up to 64 items: the split layout (a ring of four 80.25 KB hand-off slots
+ * plus 64 bytes of flags per item).  More than 64 items and at most 1024
+ * sequences: n_seq int32 (rounded up to 256 bytes) for the order in which
+ * the one-CTA layout takes the sequences, longest first, so that long
+ * sequences do not start last.  Returns 0 when neither applies: not bf16
+ * with d_k = d_v = 128, or more than 64 items and more than 1024 sequences.
+ * Host only; no CUDA call.
  */
 size_t gdn_chunk_fwd_workspace_size(int32_t n_seq, int32_t H_v, int32_t d_k, int32_t d_v,
                                     gdn_dtype in_dtype);
 
 /*
  * gdn_chunk_fwd_ws -- gdn_chunk_fwd_path with a caller-owned device
- * workspace that enables the split layout for small batches.
+ * workspace that enables the split layout for small batches (and the
+ * longest-first sequence order of the one-CTA layout for larger ones).
  *
  *   workspace        DEVICE pointer, 256-byte aligned, or NULL (then this is
  *                    gdn_chunk_fwd_path)
@@ -149,8 +153,11 @@ size_t gdn_chunk_fwd_workspace_size(int32_t n_seq, int32_t H_v, int32_t d_k, int
  * workspace is not touched.  SPLIT without a workspace is
  * GDN_ERR_INVALID_ARG; SPLIT on a batch that does not fit is
  * GDN_ERR_UNSUPPORTED.  The library clears the workspace's flags on `stream`
- * at the start of every call (an asynchronous memset), so no initialisation
- * is needed; its contents are meaningless between calls.  Two calls that
+ * at the start of every call (an asynchronous memset) or rewrites the
+ * sequence order (a one-CTA kernel launched before the prefill), so no
+ * initialisation is needed; its contents are meaningless between calls.
+ * The order changes which CTA takes which item, not the arithmetic: the
+ * results equal those of a call without a workspace bit for bit.  Two calls that
  * may run at the same time (different streams) must not share a workspace.
  */
 gdn_status gdn_chunk_fwd_ws(

@@ -65,6 +65,28 @@ def test_packed_varlen_small(path, epilogue):
     np.testing.assert_array_equal(fs[0].cpu().numpy(), w.initial_state[0].cpu().numpy())
 
 
+@pytest.mark.parametrize("epilogue", [True, False])
+def test_one_cta_longest_first(epilogue):
+    """More than 64 items with a workspace: the one-CTA layout takes the
+    sequences longest first (the order is written into the workspace).  The
+    results equal those of the in-order launch bit for bit and meet the bar
+    against the oracle."""
+    lengths = [0, 5, 64, 130, 1, 77, 0, 128, 300, 33]
+    H_v = 8
+    w = to_device(inputs.make_prefill(lengths, 2, H_v, 128, 128, seed=9, epilogue=epilogue,
+                                      s0_std=0.01))
+    nbytes = gdn.workspace_size(len(lengths), H_v, 128, 128)
+    assert nbytes == 256
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    y1, fs1 = _run(w, "tensor_single", workspace=ws)
+    y0, fs0 = _run(w, "tensor_single", workspace=None)
+    torch.testing.assert_close(y1, y0, rtol=0, atol=0)
+    torch.testing.assert_close(fs1, fs0, rtol=0, atol=0)
+    order = ws[:4 * len(lengths)].view(torch.int32).cpu().tolist()
+    assert order == sorted(range(len(lengths)), key=lambda s: (-lengths[s], s))
+    _check_all(w, y1, fs1, torch.bfloat16, "longest first")
+
+
 @pytest.mark.parametrize("path", ["tensor_split", "tensor_pair"])
 @pytest.mark.parametrize("epilogue", [True, False])
 def test_packed_varlen_few_heads(path, epilogue):
