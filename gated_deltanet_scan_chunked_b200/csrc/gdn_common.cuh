@@ -91,6 +91,15 @@ __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
   return d;
 }
 
+// SiLU u sigmoid(u) = u / (1 + 2^(-u log2 e)) on the hardware 2^x and
+// reciprocal approximations, each step rounded in fp32.
+__device__ __forceinline__ float silu_approx(float u) {
+  float e, r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(__fmul_rn(u, -1.4426950408889634f)));
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(__fadd_rn(e, 1.f)));
+  return __fmul_rn(u, r);
+}
+
 __device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + __expf(-x)); }
 
 // Sequence bounds of sequence s; returns false (and flags the error word)

@@ -47,14 +47,10 @@ __device__ __forceinline__ float rcp_approx(float x) {
   return y;
 }
 
-// SiLU u sigmoid(u) = u / (1 + 2^(-u log2 e)), every step rounded in fp32
-// (hardware 2^x and reciprocal approximations).  silu2 takes a pair and
-// performs, per lane, the same operations as silu1.
+// SiLU on a channel pair: per lane the operations of silu_approx
+// (u / (1 + 2^(-u log2 e)), every step rounded in fp32, on the hardware 2^x
+// and reciprocal approximations), with the multiplies and the add packed.
 constexpr float kNegLog2e = -1.4426950408889634f;
-__device__ __forceinline__ float silu1(float u) {
-  const float e = sm100::ex2_approx(__fmul_rn(u, kNegLog2e));
-  return __fmul_rn(u, rcp_approx(__fadd_rn(e, 1.f)));
-}
 __device__ __forceinline__ uint64_t silu2(uint64_t u) {
   float z0, z1;
   f2_unpack(f2_mul(u, f2_pack(kNegLog2e, kNegLog2e)), z0, z1);
@@ -329,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtas) gdn_conv_kernel(const Conv
         }
         float y[kCh];
 #pragma unroll
-        for (int j = 0; j < kCh; ++j) y[j] = silu1(u[j]);
+        for (int j = 0; j < kCh; ++j) y[j] = silu_approx(u[j]);
         Vec4<Tin>::store(Y + (size_t)t * m.row_len + m.col, y);
         if (a.state_out != nullptr) {
           // the sequence's last three inputs, oldest first; for a sequence

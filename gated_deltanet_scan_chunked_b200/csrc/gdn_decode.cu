@@ -309,7 +309,7 @@ __global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT, 2)
         for (int t = 0; t < T_s; ++t) {
           const float x = col[t * stride];
           const float uu = cw.w * x + cw.z * x1 + cw.y * x2 + cw.x * x3;
-          col[t * stride] = uu / (1.f + __expf(-uu));
+          col[t * stride] = silu_approx(uu);
           x3 = x2;
           x2 = x1;
           x1 = x;
