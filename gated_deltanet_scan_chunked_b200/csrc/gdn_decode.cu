@@ -11,8 +11,10 @@
 //   y   = S'^T q^ = alpha b + beta (k^ . q^) e        (times `scale`)
 // so the state is loaded into registers, reduced once over d_k, updated and
 // stored back, with no second read.  Several tokens of one sequence (for
-// speculative verification) run in one launch: the state stays in registers
-// from token to token, is read once and written once, and may be
+// speculative verification) run in one launch of the multi-token kernel,
+// whose persistent CTAs loop over the (sequence, value head) items: the
+// state stays in registers from token to token, is read once (streamed into
+// shared memory while the previous item runs) and written once, and may be
 // snapshotted after every token.
 //
 // Thread layout (d_k = d_v = 128, 256 threads): thread (rg, c4) owns columns
