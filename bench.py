@@ -363,7 +363,10 @@ def run_reference(args, world, rank):
     v = statistics.median(vals)
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+            # a whole step of the workload at the sampled rate
+            "ms_per_step": 1e3 * w.total_T / v if v > 0 else None,
+            "ms_per_step_basis": "extrapolated from the bounded sample",
+            "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": args.workload, "global_batch": 1, "seq_len": w.total_T,
                        "heads": "16 QK / 48 value", "d": D},
