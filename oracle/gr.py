@@ -22,10 +22,14 @@ Readings where the pages are silent (listed in the design notes):
     before the block, which the read has at hand).
 
 Read: fp64 arithmetic from the exact fp32 dequantised state.  Write: the
-codes are integers decided by floating point, so the write takes them in the
-precision the kernel uses, fp32, one rounding per operation in this order:
-r = deq + s * y (product rounded, then the sum), amax, scale = amax / 448,
-inv = 1 / scale, code = E4M3(r * inv).
+new state R' = R + s y is an fp32 row (the state's own precision), formed with
+one rounding per operation: r = deq + s * y (product rounded, then the sum).
+The row's scale is amax / 448 rounded to fp32.  Each code is the E4M3 value
+nearest to the exact quotient r / scale (ties to the even code), i.e. one
+rounding from the definition of the format; the quotient is taken in fp64,
+which is exact enough: for fp32 r and scale, r / scale is either an E4M3
+rounding boundary itself or at least 2^-29 (relative) away from every
+boundary, so the fp64 quotient (relative error 2^-53) rounds the same way.
 """
 from __future__ import annotations
 
@@ -77,15 +81,15 @@ def dequant(codes, scales):
 
 
 def quantize_rows(r):
-    """fp32 rows [..., d] -> (codes uint8, scales fp32) with the row's own
-    scale amax / 448 (1 for an all-zero row): inv = 1 / scale, code =
-    E4M3(r * inv), each operation rounded in fp32."""
+    """fp32 rows [..., d] -> (codes uint8, scales fp32): the row's own scale
+    amax / 448 rounded to fp32 (1 for an all-zero row), and code = the E4M3
+    value nearest to the exact quotient r / scale (see the module notes on
+    why an fp64 quotient gives the same rounding)."""
     r = np.asarray(r, dtype=np.float32)
     amax = np.abs(r).max(axis=-1).astype(np.float32)
     scale = np.where(amax > 0, (amax / np.float32(E4M3_MAX)).astype(np.float32),
                      np.float32(1.0)).astype(np.float32)
-    inv = (np.float32(1.0) / scale).astype(np.float32)
-    q = (r * inv[..., None]).astype(np.float32)
+    q = r.astype(np.float64) / scale.astype(np.float64)[..., None]
     return e4m3_encode(q), scale
 
 

@@ -134,3 +134,62 @@ def test_identical_branches_read_as_one():
     np.testing.assert_allclose(x, x1, rtol=1e-13, atol=1e-14)
     np.testing.assert_allclose(s, np.repeat(s1, n, axis=1), rtol=1e-13, atol=1e-14)
     np.testing.assert_allclose(p["G"], np.repeat(p1["G"], n, axis=1), rtol=1e-13, atol=1e-14)
+
+
+def _nearest_code_exact(r, s):
+    """The E4M3 code nearest to the exact rational r / s (ties to the even
+    code, saturating at 448), by brute force over the code table with
+    fractions.Fraction: independent of the oracle's fp64 quotient."""
+    from fractions import Fraction
+    q = Fraction(float(r)) / Fraction(float(s))
+    a = abs(q)
+    pos = gr.e4m3_decode(np.arange(0x7F, dtype=np.uint8))
+    if a >= 448:
+        c = 0x7E
+    else:
+        best = None
+        for code in range(0x7F):
+            dist = abs(a - Fraction(float(pos[code])))
+            if best is None or dist < best[0] or (dist == best[0] and code % 2 == 0):
+                best = (dist, code)
+        c = best[1]
+    return c | (0x80 if q < 0 or (q == 0 and np.signbit(r)) else 0)
+
+
+# Rows (amax, r) found by search where the fp32 reciprocal form
+# E4M3(r * fl(1 / scale)) and the exact E4M3(r / scale) fall on opposite
+# sides of a rounding boundary, in both directions.  Bit patterns of the fp32
+# values, with the reciprocal form's code and the exact code.
+_TIE_ROWS = [
+    (1085189614, 1024425110, 68, 67),
+    (1067759192, 976641066, 40, 39),
+    (1066323723, 964625409, 28, 29),
+]
+
+
+def test_quantize_rounds_the_exact_quotient():
+    """The written code is the E4M3 rounding of the exact quotient r / scale
+    (the format's definition), not of an fp32 reciprocal product: pinned on
+    rows where the two differ, and on a random sample against brute force."""
+    for amax_bits, r_bits, recip_code, exact_code in _TIE_ROWS:
+        amax = np.array([amax_bits], np.uint32).view(np.float32)[0]
+        r = np.array([r_bits], np.uint32).view(np.float32)[0]
+        row = np.array([[amax, r, -r]], np.float32)
+        codes, scales = gr.quantize_rows(row)
+        s = scales[0]
+        assert s == np.float32(amax / np.float32(448.0))
+        inv = np.float32(np.float32(1.0) / s)
+        # the reciprocal form really does round the other way here
+        assert int(gr.e4m3_encode(np.array([np.float32(r * inv)], np.float64))[0]) == recip_code
+        assert _nearest_code_exact(r, s) == exact_code != recip_code
+        assert int(codes[0, 1]) == exact_code
+        assert int(codes[0, 2]) == exact_code | 0x80
+        assert int(codes[0, 0]) == 0x7E
+    rng = np.random.default_rng(21)
+    R = (rng.standard_normal((6, 40)) * rng.uniform(0.01, 50.0, (6, 1))).astype(np.float32)
+    R[0, :5] = 0.0
+    R[1, 3] = -0.0
+    codes, scales = gr.quantize_rows(R)
+    for i in range(R.shape[0]):
+        for j in range(R.shape[1]):
+            assert int(codes[i, j]) == _nearest_code_exact(R[i, j], scales[i]), (i, j)
