@@ -16,7 +16,10 @@ the workspace flags).  The JSON line also carries the decode step
 model-shape prefill (gdn_chunk_bwd, T=4096) and the conv + SiLU front end
 (alone, ahead of the prefill, and fused into a 4-token decode) and the
 Gated Residual read / write over an FP8 state as separate objects with their
-own timing, roofline and clocks.
+own timing, roofline and clocks; so are the T=262,144 prefill and the packed
+24-sequence prefill (``prefill_configs``).  The line ends with ``summary``:
+every headline figure (prefill fractions of the roofline time, decode state
+bandwidth fraction, ...) in one short object.
 
 Multi-GPU (torchrun, one process per GPU): every rank runs its own
 independent batch (weak scaling; sequences and heads are independent, so the
@@ -341,6 +344,58 @@ def make_workload(name, rank, device="cuda"):
     return w
 
 
+def config_of(args, world, n_seq, T):
+    """The workload's config object, printed the same way by both arms."""
+    return {"workload": args.workload, "global_batch": world * n_seq, "seq_len": T,
+            "heads": "16 QK / 48 value", "d": D,
+            "parallelism": "replicas%d" % world if world > 1 else "single",
+            "l2": "flushed between steps (256 MB write outside the events)"}
+
+
+def prefill_object(name, args, world, rank, local, peaks, steps, warmup):
+    """One prefill workload timed in a region of its own (the same call and
+    roofline as the headline), for the configs that are not the headline."""
+    from gated_deltanet_scan_chunked_b200 import gdn, gdn_chunk_fwd
+    w = make_workload(name, rank)
+    T, n_seq = w.total_T, w.n_seq
+    has_s0 = w.initial_state is not None
+    y = torch.empty_like(w.v)
+    fs = torch.empty((n_seq, H_V, D, D), dtype=torch.float32, device="cuda")
+    ws_bytes = gdn.workspace_size(n_seq, H_V, D, D)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda") if ws_bytes > 0 else None
+    flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
+    clk = clock_sampler(local)
+    clk.start()
+    times = timed_steps(lambda: gdn_chunk_fwd(w.q, w.k, w.v, w.log_alpha, w.beta, g=w.g,
+                                              norm_w=w.norm_w, initial_state=w.initial_state,
+                                              cu_seqlens=w.cu_seqlens, y=y, final_state=fs,
+                                              workspace=ws),
+                        steps, warmup, world, flush=lambda: flush_buf.zero_())
+    clk_r = clk.stop()
+    err = gdn.gdn_check_device_error()
+    if err != gdn.GDN_OK:
+        raise RuntimeError("device error in %s: %s" % (name, gdn.status_string(err)))
+    ms = max_over_ranks(statistics.mean(times), world)
+    nbytes = prefill_bytes(T, n_seq, epilogue=w.g is not None, init_state=has_s0)
+    nflops = flops_per_token() * T
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = nflops / (peaks["bf16_tflops"] * 1e12)
+    out = {"workload": "%s: %d sequence(s), %d tokens, 16 QK / 48 value heads, d=128, bf16, "
+                       "epilogue, fp32 initial states" % (name, n_seq, T),
+           "ms_per_step": ms, "steps": steps, "tokens_per_s": world * T / (ms * 1e-3),
+           "roofline": {"bound": "hbm" if t_hbm >= t_tc else "tensor",
+                        "achieved": nbytes / (ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
+                        "unit": "GB/s", "frac_of_roofline_time": max(t_hbm, t_tc) / (ms * 1e-3),
+                        "roofline_time_us": max(t_hbm, t_tc) * 1e6, "algorithmic_bytes": nbytes,
+                        "counted_flops": nflops,
+                        "tensor_frac": nflops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"]},
+           "clocks": clk_r,
+           "gpu_launches_per_step": 2 if (ws is not None and n_seq * H_V > 64) else 1}
+    del w, y, fs, ws, flush_buf
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_reference(args, world, rank):
     """The oracle arm: rank 0 only, no process group, no GPU kernels of ours."""
     if rank != 0:
@@ -368,8 +423,7 @@ def run_reference(args, world, rank):
             "ms_per_step_basis": "extrapolated from the bounded sample",
             "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": args.workload, "global_batch": 1, "seq_len": w.total_T,
-                       "heads": "16 QK / 48 value", "d": D},
+            "config": config_of(args, world, w.n_seq, w.total_T),
             "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": base["cores"],
                              "kind": "oracle", "sample": base["sample"]},
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -506,6 +560,18 @@ def run_ours(args, world, rank, local):
                "pipelining": "double-buffered: step i+1's host-to-device copy overlaps "
                              "step i's kernel and step i-1's device-to-host read"}
         del dev, host, yb, fsb
+
+    # the other prefill configs (T=262,144 and the 24-sequence packed batch),
+    # each in a region of its own, when the headline is the T=4096 workload
+    others = None
+    launches_others = 0
+    if args.workload == "prefill4k" and not args.no_configs:
+        del flush_buf
+        others = {}
+        for nm in ("prefill256k", "varlen"):
+            others[nm] = prefill_object(nm, args, world, rank, local, peaks, steps=5, warmup=3)
+            launches_others += 5 * others[nm]["gpu_launches_per_step"]
+        flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
 
     # the decode step, timed on its own (256 sequences x 64 steps, in place)
     decode = None
@@ -790,17 +856,34 @@ def run_ours(args, world, rank, local):
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16", "data": "synthetic",
-                "config": {"workload": args.workload, "global_batch": world * n_seq,
-                           "seq_len": T, "heads": "16 QK / 48 value", "d": D,
-                           "path": args.path, "workspace_bytes": ws_bytes,
-                           "parallelism": "replicas%d" % world if world > 1 else "single",
-                           "l2": "flushed between steps (256 MB write outside the events)"},
+                "config": config_of(args, world, n_seq, T),
+                "path": args.path, "workspace_bytes": ws_bytes,
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": args.steps, "clocks": clk, "decode": decode,
-                "gpu_launches_decode_region": launches_decode, "backward": backward,
-                "gpu_launches_backward_region": launches_bwd, "front_end": front,
-                "gpu_launches_front_end_region": launches_front, "gated_residual": grd,
-                "gpu_launches_gated_residual_region": launches_gr}
+                "gpu_launches": args.steps, "clocks": clk,
+                "backward": backward, "gpu_launches_backward_region": launches_bwd,
+                "front_end": front, "gpu_launches_front_end_region": launches_front,
+                "gated_residual": grd, "gpu_launches_gated_residual_region": launches_gr,
+                "prefill_configs": others, "gpu_launches_prefill_configs_region": launches_others,
+                "decode": decode, "gpu_launches_decode_region": launches_decode}
+        # last: a compact summary of every figure the targets name, so that a
+        # reader of the line's tail has them all
+        summ = {"prefill4k_ms": ms_max, "prefill4k_frac": roofline["frac_of_roofline_time"]}
+        for nm, o in (others or {}).items():
+            summ[nm + "_ms"] = o["ms_per_step"]
+            summ[nm + "_frac"] = o["roofline"]["frac_of_roofline_time"]
+        if backward:
+            summ["backward_ms"] = backward["ms_per_step"]
+        if front:
+            summ["front_end_prefill_ms"] = front["prefill_with_front_end_ms"]
+            summ["conv_frac"] = front["conv_roofline"]["frac"]
+        if grd:
+            summ["gr_read_us"] = grd["read_us"]
+            summ["gr_write_frac"] = grd["write_roofline"]["frac"]
+        if decode:
+            summ["decode_multi_frac"] = decode["multi_token"]["roofline"]["frac"]
+            summ["decode_us_per_step"] = decode["us_per_step"]
+            summ["decode_frac"] = decode["roofline"]["frac"]
+        line["summary"] = summ
         print(json.dumps(line), flush=True)
 
 
@@ -816,6 +899,8 @@ def main():
                     choices=["auto", "tensor", "simt", "tensor_pair", "tensor_single",
                              "tensor_split"])
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the T=262,144 and packed-batch prefill objects")
     ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--no-front-end", action="store_true")
     ap.add_argument("--no-gr", action="store_true")

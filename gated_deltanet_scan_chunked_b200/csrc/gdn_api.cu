@@ -45,6 +45,8 @@ bool dim_ok(int32_t d) { return d == 16 || d == 32 || d == 64 || d == 128; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+}  // namespace
+
 gdn_status check_common(int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v, gdn_dtype dt,
                         float eps_l2, float eps_norm) {
   if (H_qk <= 0 || H_v <= 0 || H_v % H_qk != 0) return GDN_ERR_INVALID_ARG;
@@ -55,7 +57,6 @@ gdn_status check_common(int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v, gdn
   return GDN_OK;
 }
 
-}  // namespace
 }  // namespace gdn
 
 using namespace gdn;

@@ -79,6 +79,40 @@ __device__ __forceinline__ uint32_t f2_to_e4m3x2(uint64_t v) {
   return c;
 }
 
+// The write's codes are the E4M3 rounding of the exact quotient r / scale.
+// The kernel forms q = r * fl(1 / scale), which is within 2 ulps of the exact
+// quotient, so q rounds the same way unless it lies within a few ulps of an
+// E4M3 rounding boundary.  In E4M3's normal range the boundaries are the
+// fp32 values whose 20 fraction bits below E4M3's three are 0x80000; below
+// 2^-6 (E4M3 subnormals) every nonzero q is checked.
+__device__ __forceinline__ bool e4m3_near_boundary(float q) {
+  const uint32_t b = __float_as_uint(q) & 0x7fffffffu;
+  if (b < 0x3C800000u) return b != 0u;
+  return ((b - 0x7FFF8u) & 0xFFFFFu) <= 16u;  // within 8 ulps of a boundary
+}
+
+// Exact code for such a q: the codes of q -+ 8 ulps bracket the exact
+// quotient's code; when they differ, the boundary m between them (exact in
+// fp32) is compared with r / scale through the sign of r - m scale, which one
+// fused multiply-add gives exactly (ties go to the even code).
+__device__ __noinline__ uint32_t e4m3_code_exact(float r, float scale, float q) {
+  const uint32_t b = __float_as_uint(q) & 0x7fffffffu;
+  const float lo = __uint_as_float(b > 8u ? b - 8u : 0u);
+  const float hi = __uint_as_float(b + 8u);
+  unsigned short c2;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(c2) : "f"(hi), "f"(lo));
+  const uint32_t clo = c2 & 0xffu, chi = (uint32_t)c2 >> 8;
+  uint32_t c = clo;
+  if (chi != clo) {
+    float vlo, vhi;
+    f2_unpack(e4m3x2_to_f2(c2), vlo, vhi);
+    const float m = 0.5f * (vlo + vhi);
+    const float t = __fmaf_rn(-m, scale, fabsf(r));
+    c = t > 0.f ? chi : (t < 0.f ? clo : ((clo & 1u) ? chi : clo));
+  }
+  return c | ((__float_as_uint(r) >> 24) & 0x80u);
+}
+
 // gr_norm: one warp per (token, branch) row, the row's codes held in
 // registers (GPL groups of 8 per lane): R^ = dequant / sqrt(mean sq + eps) *
 // gamma, stored in bf16; the codes are decoded and scaled in pairs.
@@ -262,10 +296,33 @@ __global__ void __launch_bounds__(128) gr_write_kernel(const GrWriteArgs a) {
     const int j = lane + 32 * k;
     if (j < g8) {
       uint32_t w[2];
+      uint64_t q[4];
+      bool near = false;
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        q[p] = f2_mul(r[k][p], inv2);
+        float q0, q1;
+        f2_unpack(q[p], q0, q1);
+        near |= e4m3_near_boundary(q0) | e4m3_near_boundary(q1);
+      }
 #pragma unroll
       for (int h = 0; h < 2; ++h)
-        w[h] = f2_to_e4m3x2(f2_mul(r[k][2 * h], inv2)) |
-               (f2_to_e4m3x2(f2_mul(r[k][2 * h + 1], inv2)) << 16);
+        w[h] = f2_to_e4m3x2(q[2 * h]) | (f2_to_e4m3x2(q[2 * h + 1]) << 16);
+      if (near) {
+        // rare: settle the codes next to a rounding boundary exactly
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          float q0, q1, r0, r1;
+          f2_unpack(q[p], q0, q1);
+          f2_unpack(r[k][p], r0, r1);
+          const int sh = 16 * (p & 1);
+          if (e4m3_near_boundary(q0))
+            w[p >> 1] = (w[p >> 1] & ~(0xffu << sh)) | (e4m3_code_exact(r0, nsc, q0) << sh);
+          if (e4m3_near_boundary(q1))
+            w[p >> 1] =
+                (w[p >> 1] & ~(0xffu << (sh + 8))) | (e4m3_code_exact(r1, nsc, q1) << (sh + 8));
+        }
+      }
       reinterpret_cast<uint2*>(codes)[j] = make_uint2(w[0], w[1]);
     }
   }

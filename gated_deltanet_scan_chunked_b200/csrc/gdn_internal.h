@@ -166,6 +166,12 @@ size_t chunk_bwd_workspace_bytes(int32_t n_seq, int64_t total_T, int32_t H_qk, i
 void chunk_bwd_workspace_layout(void* ws, BwdArgs* a);
 gdn_status launch_chunk_bwd(const BwdArgs& a, cudaStream_t stream);
 
+// Argument checks shared by the entry points: head counts and grouping, dims
+// and epsilons (GDN_ERR_INVALID_ARG), then dtype and compiled dims
+// (GDN_ERR_UNSUPPORTED).
+gdn_status check_common(int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v, gdn_dtype dt,
+                        float eps_l2, float eps_norm);
+
 // Each launcher returns GDN_OK, GDN_ERR_UNSUPPORTED (shape not compiled) or
 // GDN_ERR_CUDA (launch failed).
 gdn_status launch_decode(const DecodeArgs& a, cudaStream_t stream);
@@ -177,6 +183,20 @@ bool prefill_tc_supports(const PrefillArgs& a);
 // 256-byte aligned workspace.
 size_t prefill_tc_workspace_bytes(int32_t n_seq, int32_t H_v, int32_t d_k, int32_t d_v,
                                   gdn_dtype dtype);
+
+// Split-launch workspace of the tensor-core prefill for `items` (sequence,
+// value head) items: per item kSplitRing "ready" and kSplitRing "consumed"
+// flags (64-bit), the whole flag block padded to 256 bytes, then per item
+// kSplitRing hand-off slots of kSplitSlotBytes (a multiple of 256).
+constexpr int kSplitRing = 4;
+constexpr size_t kSplitSlotBytes = 82176;
+constexpr long long kSplitMaxItems = 64;
+constexpr size_t split_flag_bytes(long long items) {
+  return ((size_t)items * 2 * kSplitRing * sizeof(unsigned long long) + 255) & ~(size_t)255;
+}
+constexpr size_t split_ws_bytes(long long items) {
+  return split_flag_bytes(items) + (size_t)items * kSplitRing * kSplitSlotBytes;
+}
 void prefill_tc_workspace_layout(void* ws, int32_t n_seq, int32_t H_v, PrefillArgs* a);
 
 }  // namespace gdn

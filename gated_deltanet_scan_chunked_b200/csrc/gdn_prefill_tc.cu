@@ -1011,12 +1011,13 @@ constexpr uint32_t P_MAX = 227872;        // block-max scratch [16]
 constexpr uint32_t P_BAR = 227936;        // empty[2], mma, tmem slot, staging free[2]
 constexpr uint32_t kPairSmemBytes = 231072 + 1024;  // the chain CTA's map is the larger
 // split launch: global ring per item
-constexpr int kRing = 4;
+constexpr int kRing = kSplitRing;
 // slot: tiles (64 KB), gate factors (1 + w) sigmoid(g) fp16 [64][128] (16 KB),
 // scalars [4] fp32 (16 B), padding to a multiple of 256
 constexpr uint32_t kSlotGF = kShipBytes;
 constexpr uint32_t kSlotLoad = kShipBytes + 16384;  // bytes of tiles + gate factors
 constexpr size_t kSlotBytes = kSlotLoad + 256;
+static_assert(kSlotBytes == kSplitSlotBytes, "split workspace slot size");
 
 template <int NPREP, bool kGlobal>
 __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const PrefillArgs a) {
@@ -1961,19 +1962,13 @@ bool prefill_tc_supports(const PrefillArgs& a) {
 // multiple of 256).  Only batches of at most kSplitMaxItems items can use it.
 // Larger batches of at most kMaxOrderSeqs sequences use the workspace for
 // the one-CTA layout's sequence order instead (n_seq int32, longest first).
-constexpr long long kSplitMaxItems = 64;
-
-static size_t split_flag_bytes(long long items) {
-  return ((size_t)items * 2 * kRing * sizeof(unsigned long long) + 255) & ~(size_t)255;
-}
-
 size_t prefill_tc_workspace_bytes(int32_t n_seq, int32_t H_v, int32_t d_k, int32_t d_v,
                                   gdn_dtype dtype) {
   const long long items = (long long)n_seq * H_v;
   if (dtype != GDN_BF16 || d_k != kD || d_v != kD || items < 1) return 0;
   if (items > kSplitMaxItems)
     return n_seq <= kMaxOrderSeqs ? (((size_t)n_seq * sizeof(int32_t) + 255) & ~(size_t)255) : 0;
-  return split_flag_bytes(items) + (size_t)items * kRing * kSlotBytes;
+  return split_ws_bytes(items);
 }
 
 void prefill_tc_workspace_layout(void* ws, int32_t n_seq, int32_t H_v, PrefillArgs* a) {

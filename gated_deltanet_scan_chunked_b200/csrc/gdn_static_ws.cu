@@ -2,7 +2,8 @@
 // workspace in a fixed device array of this library, for callers that cannot
 // hand the library any memory.  Nothing here allocates: the array is part of
 // the module image, its address comes from cudaGetSymbolAddress (looked up
-// once per device), and the call forwards to gdn_chunk_fwd_ws.
+// once per device and kept; not valid across a device reset), and the call
+// forwards to gdn_chunk_fwd_ws.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -13,10 +14,10 @@ namespace gdn {
 namespace {
 
 // Capacity: 48 (sequence, value head) items -- one sequence of a 48-value-head
-// layer.  Per item the split layout needs 64 bytes of flags and four 80.25 KB
-// hand-off slots, 328,768 bytes; 48 items need 15,780,864 bytes.
+// layer -- sized from the split layout's own workspace formula.
 constexpr int kStaticItems = 48;
-constexpr size_t kStaticBytes = (size_t)kStaticItems * 64 + (size_t)kStaticItems * 4 * 82176;
+constexpr size_t kStaticBytes = split_ws_bytes(kStaticItems);
+static_assert(kStaticItems <= kSplitMaxItems, "static workspace holds a split-layout batch");
 
 static __device__ __align__(256) unsigned char g_static_ws[kStaticBytes];
 
@@ -45,7 +46,10 @@ extern "C" gdn_status gdn_chunk_fwd_static_ws(
     int32_t n_seq, int64_t total_T, int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v,
     gdn_dtype in_dtype, int32_t l2norm_qk, float eps_l2, float eps_norm, float scale, void* y,
     float* final_state, gdn_stream_t stream) {
-  if (n_seq < 1 || H_v < 1) return GDN_ERR_INVALID_ARG;
+  // the same argument errors as gdn_chunk_fwd_ws, before the capacity check
+  const gdn_status st = gdn::check_common(H_qk, H_v, d_k, d_v, in_dtype, eps_l2, eps_norm);
+  if (st != GDN_OK) return st;
+  if (n_seq < 1 || total_T < 0) return GDN_ERR_INVALID_ARG;
   const size_t need = gdn_chunk_fwd_workspace_size(n_seq, H_v, d_k, d_v, in_dtype);
   // a shape the split layout does not serve, or more items than the array holds
   if ((long long)n_seq * H_v > gdn::kStaticItems || need == 0 || need > gdn::kStaticBytes)

@@ -177,14 +177,17 @@ gdn_status gdn_chunk_fwd_ws(
  * description has no counterpart to this call; it is a deployment variant of
  * the split layout.  Nothing is allocated.
  *
- *   Arguments as for gdn_chunk_fwd.
+ *   Arguments as for gdn_chunk_fwd, with the same argument errors
+ *   (GDN_ERR_INVALID_ARG for bad head counts, dims or epsilons) checked first.
  *   Capacity: n_seq * H_v <= 48 items.  A larger batch, or a shape the split
  *   layout does not serve (not bf16 with d_k = d_v = 128), returns
  *   GDN_ERR_UNSUPPORTED before anything is enqueued; so does a batch whose
  *   3 x n_seq x H_v CTAs cannot all be resident on the device.
  *   The first call on each device looks the array's address up
- *   (cudaGetSymbolAddress, which may load the module); make that first call
- *   outside stream capture.  Each call clears the array's flags on `stream`
+ *   (cudaGetSymbolAddress, which may load the module) and keeps it; make that
+ *   first call outside stream capture.  The kept address is not valid across
+ *   a device reset (cudaDeviceReset or a destroyed primary context): do not
+ *   call this entry point after one.  Each call clears the array's flags on `stream`
  *   before its kernel runs, so nothing needs initialising.
  *   All calls on a device share the one array: calls that can overlap (other
  *   streams, other host threads) race on it and must be serialised by the

@@ -153,6 +153,17 @@ def test_static_workspace_call_rejects_on_host(lib):
     assert call(n_seq=1, cu=None, dk=64) == gdn.GDN_ERR_UNSUPPORTED
     assert call(n_seq=1, cu=None, dt=1) == gdn.GDN_ERR_UNSUPPORTED
     assert call(n_seq=0) == gdn.GDN_ERR_INVALID_ARG
+    # argument errors come first, with the codes gdn_chunk_fwd_ws gives
+    for kw in (dict(n_seq=1, cu=None, dk=0), dict(n_seq=1, cu=None, Hv=47),
+               dict(n_seq=1, cu=None, dt=7), dict(n_seq=1, cu=None, dk=-128)):
+        a = dict(cu=FAKE, n_seq=2, Hv=48, dk=128, dt=0)
+        a.update(kw)
+        ref = lib.gdn_chunk_fwd_ws(FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, a["cu"],
+                                   a["n_seq"], 64, 16, a["Hv"], a["dk"], 128, a["dt"], 1, 1e-6,
+                                   1e-6, 1.0, FAKE, None, 0, None, 0, None)
+        assert ref in (gdn.GDN_ERR_INVALID_ARG, gdn.GDN_ERR_UNSUPPORTED)
+        assert call(**kw) == ref, kw
+    assert call(n_seq=1, cu=None, dk=0) == gdn.GDN_ERR_INVALID_ARG
 
 
 def _multi(lib, **kw):

@@ -30,3 +30,8 @@ def test_reference_arm_json_line():
     assert e2e["value"] == line["value"] and e2e["unit"] == line["unit"]
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
     assert line["gpu_launches"] == 0
+    # the same config object the GPU arm prints for this workload
+    sys.path.insert(0, ROOT)
+    import argparse
+    import bench
+    assert line["config"] == bench.config_of(argparse.Namespace(workload="prefill4k"), 1, 1, 4096)

@@ -3,7 +3,8 @@
 Read: x and s within the bf16 bar (the router and the write scalars come
 from bf16 GEMMs with fp32 accumulation; R^, the router output and the logits
 are held in bf16).
-Write: the E4M3 codes and the scales are integers / floats decided by fp32
+Write: the E4M3 codes (the rounding of the exact quotient r / scale) and the
+scales are integers / floats decided by fp32
 arithmetic in a fixed order, so they must match the oracle bit for bit.
 """
 import numpy as np
@@ -84,3 +85,40 @@ def test_gr_read_then_write_layer_step():
         torch.cuda.synchronize()
         np.testing.assert_array_equal(codes.cpu().numpy(), oc)
         np.testing.assert_array_equal(scales.cpu().numpy(), osc)
+
+
+# (e, write scalar s as fp32 bits): with a zero state, y = (1, 3 2^(e-10), ...)
+# and this s, the row's second value r = fl(s y) has r / scale just above an
+# E4M3 rounding boundary while fp32 r * fl(1 / scale) falls on or below it.
+_TIE_WRITES = [(-3, 1075015380), (-2, 1069550077), (-1, 1060131433), (0, 1072414671),
+               (1, 1059623179), (2, 1059827673), (3, 1082118337), (4, 1080628333)]
+
+
+def test_gr_write_rounds_the_exact_quotient():
+    """Rows whose codes sit next to a rounding boundary: the kernel's codes
+    are the rounding of the exact quotient r / scale, bit for bit."""
+    T, n_r, d = len(_TIE_WRITES), 2, 32
+    rng = np.random.default_rng(4)
+    y = torch.tensor(rng.uniform(-0.9, 0.9, (T, d)), dtype=torch.float32).to(torch.bfloat16)
+    s = torch.tensor(rng.uniform(0.5, 1.5, (T, n_r)), dtype=torch.float32)
+    for t, (e, s_bits) in enumerate(_TIE_WRITES):
+        y[t, 0] = 1.0
+        y[t, 1] = 3 * 2.0 ** (e - 10)
+        y[t, 2] = -3 * 2.0 ** (e - 10)
+        s[t, 0] = float(np.array([s_bits], np.uint32).view(np.float32)[0])
+    codes = torch.zeros((T, n_r, d), dtype=torch.uint8)
+    scales = torch.ones((T, n_r), dtype=torch.float32)
+    want_c, want_s = ogr.gr_write(codes.numpy(), scales.numpy(), _np(y), s.numpy())
+    # the planted values do sit on the exact side of the boundary
+    for t, (e, s_bits) in enumerate(_TIE_WRITES):
+        sv = np.float32(s[t, 0].item())
+        r = np.float32(sv * np.float32(3 * 2.0 ** (e - 10)))
+        inv = np.float32(np.float32(1.0) / want_s[t, 0])
+        recip = int(ogr.e4m3_encode(np.array([np.float32(r * inv)], np.float64))[0])
+        assert int(want_c[t, 0, 1]) == recip + 1 and int(want_c[t, 0, 2]) == (recip + 1) | 0x80
+    cd, sd = codes.cuda(), scales.cuda()
+    gdn.gdn_gr_write(cd, sd, y.cuda(), s.cuda())
+    torch.cuda.synchronize()
+    assert gdn_check_device_error() == gdn.GDN_OK
+    np.testing.assert_array_equal(cd.cpu().numpy(), want_c)
+    np.testing.assert_array_equal(sd.cpu().numpy(), want_s)

@@ -24,11 +24,21 @@ def test_static_workspace_matches_caller_workspace_twice():
     w = to_device(inputs.make_prefill([333], 16, 48, 128, 128, seed=31, s0_std=0.01))
     ws = torch.empty(gdn.workspace_size(1, 48, 128, 128), dtype=torch.uint8, device="cuda")
     y_ref, s_ref = gdn.gdn_chunk_fwd(*_args(w), **_kw(w), path="tensor_split", workspace=ws)
+    # outputs allocated up front, so that the device's free memory can show
+    # that the calls themselves allocate nothing
+    y = torch.empty_like(y_ref)
+    fs = torch.empty_like(s_ref)
+    gdn.gdn_chunk_fwd_static_ws(*_args(w), **_kw(w), y=y, final_state=fs)  # first call: set-up
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
     for _ in range(2):
-        y, fs = gdn.gdn_chunk_fwd_static_ws(*_args(w), **_kw(w))
+        y.zero_()
+        fs.zero_()
+        gdn.gdn_chunk_fwd_static_ws(*_args(w), **_kw(w), y=y, final_state=fs)
         torch.cuda.synchronize()
         assert gdn.gdn_check_device_error() == gdn.GDN_OK
         assert torch.equal(y, y_ref) and torch.equal(fs, s_ref)
+    assert torch.cuda.mem_get_info()[0] == free0
     y_o, s_o, _ = oracle_prefill(w)
     assert_close(y, y_o, torch.bfloat16, "static-workspace y")
     assert_close(fs, s_o, torch.bfloat16, "static-workspace state")
@@ -43,6 +53,7 @@ def test_static_workspace_packed_batch_twice():
     for _ in range(2):
         out = gdn.gdn_chunk_fwd_static_ws(*_args(w), **_kw(w))
         torch.cuda.synchronize()
+        assert gdn.gdn_check_device_error() == gdn.GDN_OK
         assert torch.equal(out[0], ref[0]) and torch.equal(out[1], ref[1])
 
 
