@@ -80,37 +80,31 @@ __device__ __forceinline__ uint32_t f2_to_e4m3x2(uint64_t v) {
 }
 
 // The write's codes are the E4M3 rounding of the exact quotient r / scale.
-// The kernel forms q = r * fl(1 / scale), which is within 2 ulps of the exact
-// quotient, so q rounds the same way unless it lies within a few ulps of an
-// E4M3 rounding boundary.  In E4M3's normal range the boundaries are the
-// fp32 values whose 20 fraction bits below E4M3's three are 0x80000; below
-// 2^-6 (E4M3 subnormals) every nonzero q is checked.
-__device__ __forceinline__ bool e4m3_near_boundary(float q) {
-  const uint32_t b = __float_as_uint(q) & 0x7fffffffu;
-  if (b < 0x3C800000u) return b != 0u;
-  return ((b - 0x7FFF8u) & 0xFFFFFu) <= 16u;  // within 8 ulps of a boundary
-}
-
-// Exact code for such a q: the codes of q -+ 8 ulps bracket the exact
-// quotient's code; when they differ, the boundary m between them (exact in
-// fp32) is compared with r / scale through the sign of r - m scale, which one
-// fused multiply-add gives exactly (ties go to the even code).
-__device__ __noinline__ uint32_t e4m3_code_exact(float r, float scale, float q) {
-  const uint32_t b = __float_as_uint(q) & 0x7fffffffu;
-  const float lo = __uint_as_float(b > 8u ? b - 8u : 0u);
-  const float hi = __uint_as_float(b + 8u);
-  unsigned short c2;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(c2) : "f"(hi), "f"(lo));
-  const uint32_t clo = c2 & 0xffu, chi = (uint32_t)c2 >> 8;
-  uint32_t c = clo;
-  if (chi != clo) {
-    float vlo, vhi;
-    f2_unpack(e4m3x2_to_f2(c2), vlo, vhi);
-    const float m = 0.5f * (vlo + vhi);
-    const float t = __fmaf_rn(-m, scale, fabsf(r));
-    c = t > 0.f ? chi : (t < 0.f ? clo : ((clo & 1u) ? chi : clo));
+// With inv = fl(1 / scale), the kernel forms q- = r * fl(inv (1 - 2^-21)) and
+// q+ = r * fl(inv (1 + 2^-21)), which bracket the exact quotient (each
+// rounding moves the products by at most 2^-24 relative), and converts both
+// (packed conversions): where the two codes agree, that is the exact
+// quotient's code (rounding is monotone).  Where they differ -- the quotient
+// lies within ~2^-20 (relative) of a rounding boundary, which is rare -- the
+// boundary m between the two codes (exact in fp32) is compared with r / scale
+// through the sign of |r| - m scale, which one fused multiply-add gives
+// exactly; ties go to the even code.
+__device__ __forceinline__ uint32_t e4m3_settle(float r, float scale, uint32_t clo,
+                                                uint32_t chi) {
+  const uint32_t sign = (__float_as_uint(r) >> 24) & 0x80u;
+  clo &= 0x7fu;
+  chi &= 0x7fu;
+  if (clo > chi) {  // magnitudes in increasing order
+    const uint32_t t = clo;
+    clo = chi;
+    chi = t;
   }
-  return c | ((__float_as_uint(r) >> 24) & 0x80u);
+  float vlo, vhi;
+  f2_unpack(e4m3x2_to_f2(clo | (chi << 8)), vlo, vhi);
+  const float m = 0.5f * (vlo + vhi);
+  const float t = __fmaf_rn(-m, scale, fabsf(r));
+  const uint32_t c = t > 0.f ? chi : (t < 0.f ? clo : ((clo & 1u) ? chi : clo));
+  return c | sign;
 }
 
 // gr_norm: one warp per (token, branch) row, the row's codes held in
@@ -245,11 +239,12 @@ __global__ void __launch_bounds__(kNT) gr_gate_kernel(const GrArgs a) {
 
 // gr_write: one warp per (token, branch) row, in place, the row's values
 // held in registers (GPL groups of 8 per lane, as fp32 pairs).  r = deq + s
-// y with one rounding per operation; scale' = max|r| / 448 (1 if zero); inv
-// = 1 / scale'; code = E4M3(r * inv) with round to nearest even and
-// saturation.  Decoding and encoding work on channel pairs (packed
-// conversions); the product and the sum stay scalar fp32 operations with
-// explicit rounding, so that they are never fused into one.
+// y with one rounding per operation; scale' = max|r| / 448 (1 if zero); code
+// = the E4M3 rounding (nearest, ties to even, saturating) of the exact
+// quotient r / scale', from r * fl(1 / scale') and the settlement above.
+// Decoding and encoding work on channel pairs (packed conversions); the
+// product and the sum stay scalar fp32 operations with explicit rounding, so
+// that they are never fused into one.
 template <int GPL>
 __global__ void __launch_bounds__(128) gr_write_kernel(const GrWriteArgs a) {
   const int64_t row = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
@@ -279,6 +274,7 @@ __global__ void __launch_bounds__(128) gr_write_kernel(const GrWriteArgs a) {
     for (int p = 0; p < 4; ++p) {
       float d0, d1;
       f2_unpack(e4m3x2_to_f2(cw[p / 2] >> (16 * (p % 2))), d0, d1);
+      // product and sum rounded separately (never fused)
       const float r0 = __fadd_rn(__fmul_rn(d0, sc), __fmul_rn(sv, __uint_as_float(yw[p] << 16)));
       const float r1 =
           __fadd_rn(__fmul_rn(d1, sc), __fmul_rn(sv, __uint_as_float(yw[p] & 0xffff0000u)));
@@ -290,40 +286,34 @@ __global__ void __launch_bounds__(128) gr_write_kernel(const GrWriteArgs a) {
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   const float nsc = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
   const float inv = __fdiv_rn(1.f, nsc);
-  const uint64_t inv2 = f2_pack(inv, inv);
+  const float inv_lo = inv * (1.f - 0x1p-21f), inv_hi = inv * (1.f + 0x1p-21f);
+  const uint64_t inv2lo = f2_pack(inv_lo, inv_lo), inv2hi = f2_pack(inv_hi, inv_hi);
 #pragma unroll
   for (int k = 0; k < GPL; ++k) {
     const int j = lane + 32 * k;
     if (j < g8) {
-      uint32_t w[2];
-      uint64_t q[4];
-      bool near = false;
+      // codes of q- (wl) and q+ (wh), element pairs packed
+      uint32_t wl[2], wh[2];
 #pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        q[p] = f2_mul(r[k][p], inv2);
-        float q0, q1;
-        f2_unpack(q[p], q0, q1);
-        near |= e4m3_near_boundary(q0) | e4m3_near_boundary(q1);
+      for (int h = 0; h < 2; ++h) {
+        const uint64_t ra = r[k][2 * h], rb = r[k][2 * h + 1];
+        wl[h] = f2_to_e4m3x2(f2_mul(ra, inv2lo)) | (f2_to_e4m3x2(f2_mul(rb, inv2lo)) << 16);
+        wh[h] = f2_to_e4m3x2(f2_mul(ra, inv2hi)) | (f2_to_e4m3x2(f2_mul(rb, inv2hi)) << 16);
       }
+      if (((wl[0] ^ wh[0]) | (wl[1] ^ wh[1])) != 0u) {
+        // rare: a code next to a rounding boundary, settled exactly
 #pragma unroll
-      for (int h = 0; h < 2; ++h)
-        w[h] = f2_to_e4m3x2(q[2 * h]) | (f2_to_e4m3x2(q[2 * h + 1]) << 16);
-      if (near) {
-        // rare: settle the codes next to a rounding boundary exactly
-#pragma unroll
-        for (int p = 0; p < 4; ++p) {
-          float q0, q1, r0, r1;
-          f2_unpack(q[p], q0, q1);
-          f2_unpack(r[k][p], r0, r1);
-          const int sh = 16 * (p & 1);
-          if (e4m3_near_boundary(q0))
-            w[p >> 1] = (w[p >> 1] & ~(0xffu << sh)) | (e4m3_code_exact(r0, nsc, q0) << sh);
-          if (e4m3_near_boundary(q1))
-            w[p >> 1] =
-                (w[p >> 1] & ~(0xffu << (sh + 8))) | (e4m3_code_exact(r1, nsc, q1) << (sh + 8));
+        for (int e = 0; e < 8; ++e) {
+          const int h = e >> 2, sh = 8 * (e & 3);
+          const uint32_t cl = (wl[h] >> sh) & 0xffu, ch = (wh[h] >> sh) & 0xffu;
+          if (cl != ch) {
+            float r0, r1;
+            f2_unpack(r[k][e >> 1], r0, r1);
+            wl[h] = (wl[h] & ~(0xffu << sh)) | (e4m3_settle((e & 1) ? r1 : r0, nsc, cl, ch) << sh);
+          }
         }
       }
-      reinterpret_cast<uint2*>(codes)[j] = make_uint2(w[0], w[1]);
+      reinterpret_cast<uint2*>(codes)[j] = make_uint2(wl[0], wl[1]);
     }
   }
   if (lane == 0) a.scales[row] = nsc;
