@@ -184,19 +184,24 @@ bool prefill_tc_supports(const PrefillArgs& a);
 size_t prefill_tc_workspace_bytes(int32_t n_seq, int32_t H_v, int32_t d_k, int32_t d_v,
                                   gdn_dtype dtype);
 
-// Split-launch workspace of the tensor-core prefill for `items` (sequence,
-// value head) items: per item kSplitRing "ready" and kSplitRing "consumed"
-// flags (64-bit), the whole flag block padded to 256 bytes, then per item
-// kSplitRing hand-off slots of kSplitSlotBytes (a multiple of 256).
-constexpr int kSplitRing = 4;
-constexpr size_t kSplitSlotBytes = 82176;
-constexpr long long kSplitMaxItems = 64;
-constexpr size_t split_flag_bytes(long long items) {
-  return ((size_t)items * 2 * kSplitRing * sizeof(unsigned long long) + 255) & ~(size_t)255;
+// Workspace of the tensor-core prefill's scan layout (small batches) for
+// `items` (sequence, value head) items: per item kScanRing "ready" and
+// kScanRing "consumed" flags (64-bit), the whole flag block padded to 256
+// bytes, then per item kScanRing hand-off slots of kScanSlotBytes (a
+// multiple of 256).
+constexpr int kScanRing = 8;
+constexpr size_t kScanSlotBytes = 73984;
+constexpr long long kScanMaxItems = 64;
+constexpr size_t scan_flag_bytes(long long items) {
+  return ((size_t)items * 2 * kScanRing * sizeof(unsigned long long) + 255) & ~(size_t)255;
 }
-constexpr size_t split_ws_bytes(long long items) {
-  return split_flag_bytes(items) + (size_t)items * kSplitRing * kSplitSlotBytes;
+constexpr size_t scan_ws_bytes(long long items) {
+  return scan_flag_bytes(items) + (size_t)items * kScanRing * kScanSlotBytes;
 }
+// Co-resident items of the scan layout on this device (0: unavailable), and
+// its launch (needs the workspace placed in a.ring / a.ring_flags).
+int prefill_scan_capacity();
+gdn_status launch_prefill_scan(const PrefillArgs& a, cudaStream_t stream);
 void prefill_tc_workspace_layout(void* ws, int32_t n_seq, int32_t H_v, PrefillArgs* a);
 
 }  // namespace gdn

@@ -1011,13 +1011,12 @@ constexpr uint32_t P_MAX = 227872;        // block-max scratch [16]
 constexpr uint32_t P_BAR = 227936;        // empty[2], mma, tmem slot, staging free[2]
 constexpr uint32_t kPairSmemBytes = 231072 + 1024;  // the chain CTA's map is the larger
 // split launch: global ring per item
-constexpr int kRing = kSplitRing;
+constexpr int kRing = 4;
 // slot: tiles (64 KB), gate factors (1 + w) sigmoid(g) fp16 [64][128] (16 KB),
 // scalars [4] fp32 (16 B), padding to a multiple of 256
 constexpr uint32_t kSlotGF = kShipBytes;
 constexpr uint32_t kSlotLoad = kShipBytes + 16384;  // bytes of tiles + gate factors
 constexpr size_t kSlotBytes = kSlotLoad + 256;
-static_assert(kSlotBytes == kSplitSlotBytes, "split workspace slot size");
 
 template <int NPREP, bool kGlobal>
 __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const PrefillArgs a) {
@@ -1957,28 +1956,27 @@ bool prefill_tc_supports(const PrefillArgs& a) {
   return a.dtype == GDN_BF16 && a.d_k == kD && a.d_v == kD;
 }
 
-// Split-launch workspace: flags (ready[kRing], consumed[kRing] per item,
-// 64-bit), padded to 256 bytes, then the ring slots (kSlotBytes each, a
-// multiple of 256).  Only batches of at most kSplitMaxItems items can use it.
+// Workspace: batches of at most kScanMaxItems items take the scan layout
+// (gdn_prefill_scan.cu), whose hand-off ring lives in it (scan_ws_bytes).
 // Larger batches of at most kMaxOrderSeqs sequences use the workspace for
 // the one-CTA layout's sequence order instead (n_seq int32, longest first).
 size_t prefill_tc_workspace_bytes(int32_t n_seq, int32_t H_v, int32_t d_k, int32_t d_v,
                                   gdn_dtype dtype) {
   const long long items = (long long)n_seq * H_v;
   if (dtype != GDN_BF16 || d_k != kD || d_v != kD || items < 1) return 0;
-  if (items > kSplitMaxItems)
+  if (items > kScanMaxItems)
     return n_seq <= kMaxOrderSeqs ? (((size_t)n_seq * sizeof(int32_t) + 255) & ~(size_t)255) : 0;
-  return split_ws_bytes(items);
+  return scan_ws_bytes(items);
 }
 
 void prefill_tc_workspace_layout(void* ws, int32_t n_seq, int32_t H_v, PrefillArgs* a) {
   const long long items = (long long)n_seq * H_v;
-  if (items > kSplitMaxItems) {
+  if (items > kScanMaxItems) {
     a->seq_order = static_cast<int32_t*>(ws);
     return;
   }
   a->ring_flags = static_cast<unsigned long long*>(ws);
-  a->ring = static_cast<uint8_t*>(ws) + split_flag_bytes(items);
+  a->ring = static_cast<uint8_t*>(ws) + scan_flag_bytes(items);
 }
 
 gdn_status launch_prefill_tc(const PrefillArgs& a, cudaStream_t stream) {
@@ -1995,47 +1993,15 @@ gdn_status launch_prefill_tc(const PrefillArgs& a, cudaStream_t stream) {
   }
   static bool pair_attr_set[64][2] = {{false}};
   const long long items = (long long)a.n_seq * a.H_v;
-  // Split launch (needs the workspace): chain + two preparation CTAs per
-  // item as one cooperative grid, used when every CTA can be resident at
-  // once.  Capacity = co-resident CTAs of that kernel on this device.
-  static int split_capacity[64] = {0};
-  auto split_fits = [&]() -> bool {
-    if (a.ring == nullptr || a.ring_flags == nullptr || items > kSplitMaxItems) return false;
-    if (dev < 0 || dev >= 64) return false;
-    if (split_capacity[dev] == 0) {
-      int cap = -1;
-      const void* fn = (const void*)gdn_prefill_tc_pair_kernel<2, true>;
-      int coop = 0, sms = 0, per_sm = 0;
-      if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)kPairSmemBytes) == cudaSuccess &&
-          cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) == cudaSuccess &&
-          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
-          cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kNT, kPairSmemBytes) ==
-              cudaSuccess &&
-          coop)
-        cap = per_sm * sms;
-      split_capacity[dev] = cap;
-    }
-    return split_capacity[dev] >= 3 * items;
+  // Scan layout (needs the workspace): a chain CTA and two preparation CTAs
+  // per item in one cooperative launch, when every CTA can be resident.
+  auto scan_fits = [&]() -> bool {
+    return a.ring != nullptr && a.ring_flags != nullptr && items <= kScanMaxItems &&
+           items <= prefill_scan_capacity();
   };
-  if (a.tc_variant == 3 || (a.tc_variant == 0 && split_fits())) {
-    if (!split_fits()) return GDN_ERR_UNSUPPORTED;
-    // flags count chunks from zero in every call
-    if (cudaMemsetAsync(a.ring_flags, 0, split_flag_bytes(items), stream) != cudaSuccess)
-      return GDN_ERR_CUDA;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(3 * items), 1, 1);
-    cfg.blockDim = dim3(kNT, 1, 1);
-    cfg.dynamicSmemBytes = kPairSmemBytes;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, gdn_prefill_tc_pair_kernel<2, true>, a) != cudaSuccess)
-      return GDN_ERR_CUDA;
-    return cudaPeekAtLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+  if (a.tc_variant == 3 || (a.tc_variant == 0 && a.total_T >= kC && scan_fits())) {
+    if (!scan_fits()) return GDN_ERR_UNSUPPORTED;
+    return launch_prefill_scan(a, stream);
   }
   // While there are too few (sequence, head) items to fill the GPU, give each
   // a cluster: one chain CTA plus one or two preparation CTAs -- but only a

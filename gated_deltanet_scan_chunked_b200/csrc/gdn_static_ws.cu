@@ -16,8 +16,8 @@ namespace {
 // Capacity: 48 (sequence, value head) items -- one sequence of a 48-value-head
 // layer -- sized from the split layout's own workspace formula.
 constexpr int kStaticItems = 48;
-constexpr size_t kStaticBytes = split_ws_bytes(kStaticItems);
-static_assert(kStaticItems <= kSplitMaxItems, "static workspace holds a split-layout batch");
+constexpr size_t kStaticBytes = scan_ws_bytes(kStaticItems);
+static_assert(kStaticItems <= kScanMaxItems, "static workspace holds a scan-layout batch");
 
 static __device__ __align__(256) unsigned char g_static_ws[kStaticBytes];
 

@@ -171,7 +171,7 @@ gdn_status gdn_chunk_fwd_ws(
 
 /*
  * gdn_chunk_fwd_static_ws -- gdn_chunk_fwd_ws with GDN_PATH_TENSOR_SPLIT and
- * a workspace that is a fixed array inside the library (15,780,864 bytes of
+ * a workspace that is a fixed array inside the library (28,416,000 bytes of
  * device memory per device, part of the module image) instead of caller
  * memory: for callers that cannot give the library any memory.  The method's
  * description has no counterpart to this call; it is a deployment variant of

@@ -99,14 +99,14 @@ def _chunk_ws(lib, ws=None, ws_bytes=0, path=0, **kw):
 
 
 def test_workspace_size(lib):
-    """Split layout: 64 bytes of flags per item (padded to 256), then four
-    80 KB + 256 B slots per item; beyond 64 items, the one-CTA layout's
-    sequence order (n_seq int32, padded to 256) up to 1024 sequences;
-    nothing for shapes the tensor-core kernel cannot serve."""
-    one = 4 * (81920 + 256)
-    assert gdn.workspace_size(1, 48, 128, 128) == 48 * 64 + 48 * one
+    """Scan layout: 128 bytes of flags per item (padded to 256), then eight
+    90,368-byte hand-off slots per item; beyond 64 items, the one-CTA
+    layout's sequence order (n_seq int32, padded to 256) up to 1024
+    sequences; nothing for shapes the tensor-core kernel cannot serve."""
+    one = 8 * 73984
+    assert gdn.workspace_size(1, 48, 128, 128) == 48 * 128 + 48 * one
     assert gdn.workspace_size(1, 1, 128, 128) == 256 + one
-    assert gdn.workspace_size(2, 32, 128, 128) == 64 * 64 + 64 * one
+    assert gdn.workspace_size(2, 32, 128, 128) == 64 * 128 + 64 * one
     assert gdn.workspace_size(3, 32, 128, 128) == 256        # more than 64 items: the order
     assert gdn.workspace_size(24, 48, 128, 128) == 256
     assert gdn.workspace_size(100, 48, 128, 128) == 512
