@@ -93,8 +93,8 @@ constexpr uint32_t C_YS = 2 * kSlotStride;        // Y^T 2^-e stages: 2 x fp16 [
 constexpr uint32_t C_GS = C_YS + 32768;           // raw g of the staged chunks (TMA): 2 x
                                                   //   bf16 [64 t][128 j], SW128, 2 panels
 constexpr uint32_t C_WN = C_GS + 32768;           // 1 + norm_w [128] fp32
-constexpr uint32_t C_MISC = C_WN + 512;           // warp maxima [8], stage exponents [2]
-constexpr uint32_t C_BAR = C_MISC + 64;           // full[2] bar1 bar3 barY[2] ysfull[2]
+constexpr uint32_t C_MISC = C_WN + 512;           // warp maxima [2][8], stage exponents [2]
+constexpr uint32_t C_BAR = C_MISC + 128;           // full[2] bar1 bar3 barY[2] ysfull[2]
                                                   //   ysempty[2] sready dready gfull[2],
                                                   //   TMEM slot
 constexpr uint32_t kChainSmem = C_BAR + 128;
@@ -445,15 +445,20 @@ __device__ void prep_compute(const ScanParams& P, uint8_t* gb, uint32_t sb, uint
     fence_after_sync();
     GDN_SCAN_TRACE(1, 31);
     {
-      const int row = 32 * warp + lane;  // lanes 0-63: K rows (A), 64-127: Q rows (P)
+      // lanes 0-63: K rows, A_ti = beta_t rk_t rk_i 2^(G2_t - G2_i) (k.k)_ti, i < t;
+      // lanes 64-127: Q rows, P_ti = rq_t rk_i 2^(G2_t - G2_i) (q.k)_ti, i <= t
+      const int row = 32 * warp + lane;
       const int t = row & 63;
+      const bool is_a = row < 64;
       const float Gt = sG2[t];
-#pragma unroll
+      const float sc = is_a ? sBeta[t] * sRk[t] : sRq[t];
+      const int lim = is_a ? t : t + 1;  // columns i < lim are kept
+#pragma unroll 1
       for (int hh = 0; hh < 2; ++hh) {
         const int i0 = 32 * hh;
         float v[32];
         tmem_ld32(tb + lane_off + i0, v);
-        // the half's column factors rk_i and G2_i (loaded before any store)
+        // the half's column factors rk_i and G2_i
         float rkv[32], gv[32];
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
@@ -463,39 +468,26 @@ __device__ void prep_compute(const ScanParams& P, uint8_t* gb, uint32_t sb, uint
           gv[4 * q] = g4.x; gv[4 * q + 1] = g4.y; gv[4 * q + 2] = g4.z; gv[4 * q + 3] = g4.w;
         }
         tmem_wait_ld();
-        if (row < 64) {
-          // A_ti = beta_t rk_t rk_i 2^(G2_t - G2_i) (k.k)_ti, i < t
-          const float bt = sBeta[t] * sRk[t];
 #pragma unroll
-          for (int i = 0; i < 32; i += 4) {
-            float o[4];
+        for (int x = 0; x < 32; ++x) {
+          // masked entries take 2^-inf = 0 (no branch around the exponential)
+          const float d = i0 + x < lim ? Gt - gv[x] : -INFINITY;
+          v[x] = sc * rkv[x] * ex2_approx(d) * v[x];
+        }
+        if (is_a) {
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int ii = i0 + i + u;
-              // masked entries take 2^-inf = 0 (no branch around the exponential)
-              const float d = ii < t ? Gt - gv[i + u] : -INFINITY;
-              o[u] = bt * rkv[i + u] * ex2_approx(d) * v[i + u];
-            }
-            *reinterpret_cast<float4*>(sA + fidx(t, i0 + i)) = make_float4(o[0], o[1], o[2], o[3]);
-          }
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(sA + fidx(t, i0 + i)) =
+                make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
         } else {
-          // P_ti = rq_t rk_i 2^(G2_t - G2_i) (q.k)_ti, i <= t
-          const float qt = sRq[t];
-          const uint32_t dst = sb + P_SP + t * 128;
+          // P row t into its stage (the slot's layout)
+          uint8_t* dst = gb + P_SP + t * 128;
 #pragma unroll
-          for (int c8 = 0; c8 < 4; ++c8) {
-            uint32_t pk[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int ia = i0 + 8 * c8 + 2 * u, x = 8 * c8 + 2 * u;
-              const float d0 = ia <= t ? Gt - gv[x] : -INFINITY;
-              const float d1 = ia + 1 <= t ? Gt - gv[x + 1] : -INFINITY;
-              const float p0 = qt * rkv[x] * ex2_approx(d0) * v[x];
-              const float p1 = qt * rkv[x + 1] * ex2_approx(d1) * v[x + 1];
-              pk[u] = pack_h2(p0, p1);
-            }
-            st_shared_v4(dst + (((4 * hh + c8) ^ (t & 7)) << 4), pk[0], pk[1], pk[2], pk[3]);
-          }
+          for (int c8 = 0; c8 < 4; ++c8)
+            *reinterpret_cast<uint4*>(dst + (((4 * hh + c8) ^ (t & 7)) << 4)) =
+                make_uint4(pack_h2(v[8 * c8], v[8 * c8 + 1]), pack_h2(v[8 * c8 + 2], v[8 * c8 + 3]),
+                           pack_h2(v[8 * c8 + 4], v[8 * c8 + 5]),
+                           pack_h2(v[8 * c8 + 6], v[8 * c8 + 7]));
         }
       }
     }
@@ -795,23 +787,23 @@ __device__ void chain_compute(const ScanParams& P, uint8_t* gb, uint32_t sb, uin
   const int nch = bounds_ok ? (int)((t_end - t_begin + kC - 1) / kC) : 0;
   float* sMaxw = reinterpret_cast<float*>(gb + C_MISC);
   unsigned long long* consumed = a.ring_flags + (size_t)item * 2 * kRingS + kRingS;
-  int* sYExp = reinterpret_cast<int*>(gb + C_MISC + 32);  // exponent of each Y stage
+  int* sYExp = reinterpret_cast<int*>(gb + C_MISC + 64);  // exponent of each Y stage
   const size_t st_off = ((size_t)seq * a.H_v + h) * (size_t)(kD * kD);
   const uint32_t tSA = tbase + lane_off + 32 * cg;
   const uint32_t tDA = tbase + lane_off + 64 + 16 * cg;
   const uint32_t tDS = tbase + lane_off + 128 + 64 * cg;
   auto tD1 = [&](int b) -> uint32_t { return tbase + lane_off + 256 + 128 * b; };
 
+  // the initial state (zero without one); plain loads under a branch, so that
+  // no load from a null initial state can be speculated
   float S[64];
+  if (a.initial_state != nullptr) {
+    const float* s0 = a.initial_state + st_off + (size_t)(64 * cg) * kD + j;
 #pragma unroll
-  for (int x = 0; x < 64; ++x)
-    S[x] = a.initial_state ? __ldg(a.initial_state + st_off + (size_t)(64 * cg + x) * kD + j) : 0.f;
-  if (nch == 0) {
-    if (a.final_state && bounds_ok) {
+    for (int x = 0; x < 64; ++x) S[x] = s0[(size_t)x * kD];
+  } else {
 #pragma unroll
-      for (int x = 0; x < 64; ++x) a.final_state[st_off + (size_t)(64 * cg + x) * kD + j] = S[x];
-    }
-    return;
+    for (int x = 0; x < 64; ++x) S[x] = 0.f;
   }
 
   uint32_t ph_full = 0, ph1 = 0, ph3 = 0, phY = 0, phE = 0;  // parity bits per buffer
@@ -823,15 +815,18 @@ __device__ void chain_compute(const ScanParams& P, uint8_t* gb, uint32_t sb, uin
   auto state_operand = [&](int c, float smax, bool okin) -> int {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, o));
-    if (lane == 0) sMaxw[warp] = smax;
+    // per-warp maxima in the half of the scratch for chunk parity c % 2 (a warp
+    // still reading chunk c - 1's maxima is not overwritten)
+    float* mx = sMaxw + 8 * (c & 1);
+    if (lane == 0) mx[warp] = smax;
     bool okw = mbar_wait(&B.full[c & 1], par(ph_full, c & 1), kWait) && okin;
     ph_full ^= 1u << (c & 1);
     if (!named_sync_and(1, kChainT, okw)) return INT32_MIN;
     // slot c has landed in shared memory: its global image may be reused
     if (tid == 0) st_release_u64(&consumed[c % kRingS], (unsigned long long)c + 1);
-    float mS = sMaxw[0];
+    float mS = mx[0];
 #pragma unroll
-    for (int w = 1; w < 8; ++w) mS = fmaxf(mS, sMaxw[w]);
+    for (int w = 1; w < 8; ++w) mS = fmaxf(mS, mx[w]);
     const float mV = reinterpret_cast<const float*>(gb + (c & 1) * kSlotStride + SL_SCAL)[2];
     const int e = scale_exp(mV + 12.f * mS, 12);
     const float se = ldexpf(1.f, -e);
@@ -870,61 +865,69 @@ __device__ void chain_compute(const ScanParams& P, uint8_t* gb, uint32_t sb, uin
     return okw;
   };
 
-  {
-    float sm = 0.f;
+  float smax = 0.f, gC = 1.f;
 #pragma unroll
-    for (int x = 0; x < 64; ++x) sm = fmaxf(sm, fabsf(S[x]));
-    e_cur = state_operand(0, sm, true);
-    ok = e_cur != INT32_MIN;
-  }
-  for (int c = 0; ok && c < nch; ++c) {
+  for (int x = 0; x < 64; ++x) smax = fmaxf(smax, fabsf(S[x]));
+  bool okw = true;
+  // Iteration c: the state operand and Delta of chunk c, the Y stage of chunk
+  // c - 1 (while chunk c's state products run), the state update of chunk c;
+  // iteration nch only stages the last Y.
+  for (int c = 0; c <= nch && nch > 0; ++c) {
+    const bool live = c < nch;
     const int b = c & 1;
-    const uint8_t* slotp = gb + b * kSlotStride;
-    const float gC = reinterpret_cast<const float*>(slotp + SL_SCAL)[0];
-    const int eu = (int)reinterpret_cast<const float*>(slotp + SL_SCAL)[1];
-    GDN_SCAN_TRACE(0, 0);
+    if (live) {
+      e_cur = state_operand(c, smax, okw);
+      if (e_cur == INT32_MIN) { ok = false; break; }
+      // slot c's scalars: read before its products complete (buffer b then takes
+      // chunk c + 2)
+      const float* scal = reinterpret_cast<const float*>(gb + b * kSlotStride + SL_SCAL);
+      gC = scal[0];
+      const int eu = (int)scal[1];
+      GDN_SCAN_TRACE(0, 0);
 
-    // ---- Delta^T 2^-e = acc + U^T 2^(e_u - e) -> fp16 A operand ------------------
-    bool okw = mbar_wait(B.bar1, ph1, kWait);
-    ph1 ^= 1;
-    fence_after_sync();
-    GDN_SCAN_TRACE(0, 2);
-    {
-      float v[32];
-      tmem_ld32(tD1(b) + 32 * cg, v);
-      uint4 uq[4];
+      // ---- Delta^T 2^-e = acc + U^T 2^(e_u - e) -> fp16 A operand ------------------
+      okw = mbar_wait(B.bar1, ph1, kWait);
+      ph1 ^= 1;
+      fence_after_sync();
+      GDN_SCAN_TRACE(0, 2);
+      {
+        float v[32];
+        tmem_ld32(tD1(b) + 32 * cg, v);
+        uint4 uq[4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
-        uq[q] = ld_shared_v4(sb + b * kSlotStride + SL_U + j * 128 + (((4 * cg + q) ^ (j & 7)) << 4));
-      tmem_wait_ld();
-      const float su = ldexpf(1.f, eu - e_cur);
-      uint32_t pk[16];
+        for (int q = 0; q < 4; ++q)
+          uq[q] = ld_shared_v4(sb + b * kSlotStride + SL_U + j * 128 + (((4 * cg + q) ^ (j & 7)) << 4));
+        tmem_wait_ld();
+        const float su = ldexpf(1.f, eu - e_cur);
+        uint32_t pk[16];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint32_t uw[4] = {uq[q].x, uq[q].y, uq[q].z, uq[q].w};
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t uw[4] = {uq[q].x, uq[q].y, uq[q].z, uq[q].w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 uf = h2f(uw[e]);
-          const int x = 8 * q + 2 * e;
-          pk[4 * q + e] = pack_h2(v[x] + uf.x * su, v[x + 1] + uf.y * su);
+          for (int e = 0; e < 4; ++e) {
+            const float2 uf = h2f(uw[e]);
+            const int x = 8 * q + 2 * e;
+            pk[4 * q + e] = pack_h2(v[x] + uf.x * su, v[x + 1] + uf.y * su);
+          }
         }
+        tmem_st16(tDA, pk);
+        tmem_wait_st();
       }
-      tmem_st16(tDA, pk);
-      tmem_wait_st();
+      fence_before_sync();
+      mbar_arrive(B.dready);
+      GDN_SCAN_TRACE(0, 3);
     }
-    fence_before_sync();
-    mbar_arrive(B.dready);
-    GDN_SCAN_TRACE(0, 3);
     // the previous chunk's Y^T to the stage while the state products run
     if (c > 0) okw = export_y(c - 1, e_prev) && okw;
     GDN_SCAN_TRACE(0, 4);
+    if (!live) break;
 
-    // ---- S <- gamma_C S + 2^e increment; the next S^T operand ---------------------
+    // ---- S <- gamma_C S + 2^e increment --------------------------------------------
     okw = mbar_wait(B.bar3, ph3, kWait) && okw;
     ph3 ^= 1;
     fence_after_sync();
     GDN_SCAN_TRACE(0, 5);
-    float smax = 0.f;
+    smax = 0.f;
     {
       float v[64];
       tmem_ld32(tDS, v);
@@ -939,18 +942,13 @@ __device__ void chain_compute(const ScanParams& P, uint8_t* gb, uint32_t sb, uin
     }
     GDN_SCAN_TRACE(0, 6);
     e_prev = e_cur;
-    if (c + 1 < nch) {
-      e_cur = state_operand(c + 1, smax, okw);
-      ok = e_cur != INT32_MIN;
-    } else {
-      ok = okw;
-    }
     GDN_SCAN_TRACE(0, 7);
   }
-  if (ok) ok = export_y(nch - 1, e_prev);
-  if (ok && a.final_state) {
+  ok = ok && okw;
+  if (ok && a.final_state && bounds_ok) {
+    float* fs = a.final_state + st_off + (size_t)(64 * cg) * kD + j;
 #pragma unroll
-    for (int x = 0; x < 64; ++x) a.final_state[st_off + (size_t)(64 * cg + x) * kD + j] = S[x];
+    for (int x = 0; x < 64; ++x) fs[(size_t)x * kD] = S[x];
   }
   GDN_SCAN_TRACE(0, 8);
   if (!ok) {
@@ -1087,7 +1085,7 @@ __device__ void chain_epilogue(const ScanParams& P, uint8_t* gb, int item, const
   if (!seq_bounds(a.cu_seqlens, seq, a.total_T, &t_begin, &t_end, nullptr)) return;
   const int nch = (int)((t_end - t_begin + kC - 1) / kC);
   const float* sWn = reinterpret_cast<const float*>(gb + C_WN);
-  const int* sExp = reinterpret_cast<const int*>(gb + C_MISC + 32);
+  const int* sExp = reinterpret_cast<const int*>(gb + C_MISC + 64);
   const bool has_g = a.g != nullptr;
   uint32_t phF = 0, phG = 0;  // parity bits per stage
   bool ok = true;
@@ -1106,9 +1104,12 @@ __device__ void chain_epilogue(const ScanParams& P, uint8_t* gb, int item, const
     if (t < n) {
       uint8_t* dst = reinterpret_cast<uint8_t*>(static_cast<__nv_bfloat16*>(a.y) +
                                                 ((size_t)(c0 + t) * a.H_v + h) * kD);
+      // RMSNorm x gate when g is given (gate factor (1 + w_j) sigmoid(g_tj)),
+      // the plain scaled rows otherwise
+      float rr = ys;
       if (has_g) {
         float ss = 0.f;
-#pragma unroll
+#pragma unroll 4
         for (int ch = 0; ch < 16; ++ch) {
           const uint4 u = *reinterpret_cast<const uint4*>(yst + ((ch ^ (t & 15)) << 4));
           const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
@@ -1118,53 +1119,40 @@ __device__ void chain_epilogue(const ScanParams& P, uint8_t* gb, int item, const
             ss += f.x * f.x + f.y * f.y;
           }
         }
-        const float rr = ys * rsqrtf(ss * ys * ys / (float)kD + a.eps_norm);
-        // raw g row t: 16-byte chunk cc of panel p at cc ^ (t % 8) (TMA, SW128)
-        const uint8_t* gsrc = gb + C_GS + b * 16384 + t * 128;
-        // four 16-byte chunks at a time, their loads ahead of their stores
+        rr = ys * rsqrtf(ss * ys * ys / (float)kD + a.eps_norm);
+      }
+      // raw g row t: 16-byte chunk cc of panel p at cc ^ (t % 8) (TMA, SW128)
+      const uint8_t* gsrc = gb + C_GS + b * 16384 + t * 128;
+      // four 16-byte chunks at a time, their loads ahead of their stores
 #pragma unroll 1
-        for (int cb = 0; cb < 16; cb += 4) {
-          uint4 u[4], gq[4];
-          float4 w[8];
+      for (int cb = 0; cb < 16; cb += 4) {
+        uint4 u[4], gq[4];
+        float4 w[8];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int ch = cb + k;
-            u[k] = *reinterpret_cast<const uint4*>(yst + ((ch ^ (t & 15)) << 4));
-            gq[k] = *reinterpret_cast<const uint4*>(gsrc + (ch >> 3) * 8192 +
-                                                    (((ch & 7) ^ (t & 7)) << 4));
-            w[2 * k] = *reinterpret_cast<const float4*>(sWn + 8 * ch);
-            w[2 * k + 1] = *reinterpret_cast<const float4*>(sWn + 8 * ch + 4);
-          }
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const float wv[8] = {w[2 * k].x,     w[2 * k].y,     w[2 * k].z,     w[2 * k].w,
-                                 w[2 * k + 1].x, w[2 * k + 1].y, w[2 * k + 1].z, w[2 * k + 1].w};
-            const uint32_t w4[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
-            const uint32_t g4[4] = {gq[k].x, gq[k].y, gq[k].z, gq[k].w};
-            uint32_t o[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              // (1 + w_j) sigmoid(g_tj) y_tj / rms
-              const float2 f = h2f(w4[e]);
-              const float s0 = rcp_approx(1.f + ex2_approx(-kLog2e * bf_lo(g4[e])));
-              const float s1 = rcp_approx(1.f + ex2_approx(-kLog2e * bf_hi(g4[e])));
-              o[e] = pack_b2(f.x * rr * (wv[2 * e] * s0), f.y * rr * (wv[2 * e + 1] * s1));
-            }
-            st_global_v4(dst + 16 * (cb + k), o[0], o[1], o[2], o[3]);
-          }
+        for (int k = 0; k < 4; ++k) {
+          const int ch = cb + k;
+          u[k] = *reinterpret_cast<const uint4*>(yst + ((ch ^ (t & 15)) << 4));
+          gq[k] = *reinterpret_cast<const uint4*>(gsrc + (ch >> 3) * 8192 +
+                                                  (((ch & 7) ^ (t & 7)) << 4));
+          w[2 * k] = *reinterpret_cast<const float4*>(sWn + 8 * ch);
+          w[2 * k + 1] = *reinterpret_cast<const float4*>(sWn + 8 * ch + 4);
         }
-      } else {
-#pragma unroll 4
-        for (int ch = 0; ch < 16; ++ch) {
-          const uint4 u = *reinterpret_cast<const uint4*>(yst + ((ch ^ (t & 15)) << 4));
-          const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float wv[8] = {w[2 * k].x,     w[2 * k].y,     w[2 * k].z,     w[2 * k].w,
+                               w[2 * k + 1].x, w[2 * k + 1].y, w[2 * k + 1].z, w[2 * k + 1].w};
+          const uint32_t w4[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
+          const uint32_t g4[4] = {gq[k].x, gq[k].y, gq[k].z, gq[k].w};
           uint32_t o[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
+            // (1 + w_j) sigmoid(g_tj) y_tj / rms (w = 0 and no gate without g)
             const float2 f = h2f(w4[e]);
-            o[e] = pack_b2(f.x * ys, f.y * ys);
+            const float s0 = has_g ? rcp_approx(1.f + ex2_approx(-kLog2e * bf_lo(g4[e]))) : 1.f;
+            const float s1 = has_g ? rcp_approx(1.f + ex2_approx(-kLog2e * bf_hi(g4[e]))) : 1.f;
+            o[e] = pack_b2(f.x * rr * (wv[2 * e] * s0), f.y * rr * (wv[2 * e + 1] * s1));
           }
-          st_global_v4(dst + 16 * ch, o[0], o[1], o[2], o[3]);
+          st_global_v4(dst + 16 * (cb + k), o[0], o[1], o[2], o[3]);
         }
       }
     }
