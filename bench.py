@@ -478,7 +478,15 @@ def run_ours(args, world, rank, local):
         achieved, peak, unit = nbytes / (ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s"
     else:
         achieved, peak, unit = nflops / (ms * 1e-3) / 1e12, peaks["bf16_tflops"], "TFLOP/s"
-    kernel_key = "prefill_simt" if args.path == "simt" else "prefill_tc"
+    # the kernel that runs: the scan layout for at most 64 (sequence, head)
+    # items of at least one chunk, the one-CTA layout otherwise
+    items = n_seq * H_V
+    if args.path == "simt":
+        kernel_key = "prefill_simt"
+    elif args.path in ("auto", "tensor", "tensor_split") and items <= 64 and T >= 64:
+        kernel_key = "prefill_scan"
+    else:
+        kernel_key = "prefill_tc"
     roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                 "frac": achieved / peak, "traffic": kernel_traffic(kernel_key),
                 "peak_source": peaks["source"], "roofline_time_us": max(t_hbm, t_tc) * 1e6,
