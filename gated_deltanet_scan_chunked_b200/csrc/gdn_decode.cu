@@ -57,6 +57,18 @@ __device__ __forceinline__ float4 f2_to_float4(const uint64_t* p) {
   f2_unpack(p[1], r.z, r.w);
   return r;
 }
+// Sum over the row groups of one array of partial sums (in row-group order).
+template <int ROWG, int TPR>
+__device__ __forceinline__ float4 col_sum(const float4 (*red)[TPR], int c4) {
+  uint64_t sa[2] = {0ull, 0ull};
+#pragma unroll
+  for (int g2 = 0; g2 < ROWG; ++g2) {
+    const float4 x = red[g2][c4];
+    sa[0] = f2_add(sa[0], f2_pack(x.x, x.y));
+    sa[1] = f2_add(sa[1], f2_pack(x.z, x.w));
+  }
+  return f2_to_float4(sa);
+}
 // Sum over the row groups of their partial sums (in row-group order).
 template <int ROWG, int TPR>
 __device__ __forceinline__ void col_sums(const float4 (*red_a)[TPR], const float4 (*red_b)[TPR],
@@ -82,6 +94,25 @@ __device__ __forceinline__ float4 row_update(const float4& s, uint64_t alpha2, f
   o[0] = f2_fma(b2, e2[0], f2_mul(alpha2, f2_pack(s.x, s.y)));
   o[1] = f2_fma(b2, e2[1], f2_mul(alpha2, f2_pack(s.z, s.w)));
   return f2_to_float4(o);
+}
+
+// e = v - alpha a, and y = scale (alpha b + (beta k^.q^) e), with every
+// rounding written out, so that both kernels compute them alike wherever the
+// code stands.
+__device__ __forceinline__ float4 err4(const float4& v, float alpha, const float4& ta) {
+  return make_float4(__fmaf_rn(-alpha, ta.x, v.x), __fmaf_rn(-alpha, ta.y, v.y),
+                     __fmaf_rn(-alpha, ta.z, v.z), __fmaf_rn(-alpha, ta.w, v.w));
+}
+__device__ __forceinline__ float4 out4(float scale, float alpha, const float4& tb, float bkq,
+                                       const float4& e) {
+  return make_float4(__fmul_rn(scale, __fmaf_rn(alpha, tb.x, __fmul_rn(bkq, e.x))),
+                     __fmul_rn(scale, __fmaf_rn(alpha, tb.y, __fmul_rn(bkq, e.y))),
+                     __fmul_rn(scale, __fmaf_rn(alpha, tb.z, __fmul_rn(bkq, e.z))),
+                     __fmul_rn(scale, __fmaf_rn(alpha, tb.w, __fmul_rn(bkq, e.w))));
+}
+// This thread's share of sum(y^2) over a row.
+__device__ __forceinline__ float sq4(const float4& y) {
+  return __fmaf_rn(y.w, y.w, __fmaf_rn(y.z, y.z, __fmaf_rn(y.y, y.y, __fmul_rn(y.x, y.x))));
 }
 
 template <int DK, int DV, typename Tin>
@@ -155,9 +186,7 @@ __global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT)
   __syncthreads();
   float4 ta, tb;
   col_sums<ROWG, TPR>(red_a, red_b, c4, &ta, &tb);
-  float4 e;
-  e.x = v4.x - alpha * ta.x; e.y = v4.y - alpha * ta.y;
-  e.z = v4.z - alpha * ta.z; e.w = v4.w - alpha * ta.w;
+  const float4 e = err4(v4, alpha, ta);
 
   // S' = alpha S + beta k^ e^T, stored in place (each thread rewrites
   // exactly the elements it loaded)
@@ -171,15 +200,13 @@ __global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT)
   }
 
   // y = scale (alpha b + beta (k^.q^) e), then the optional epilogue
-  const float bkq = beta * kq;
-  float4 y;
-  y.x = a.scale * (alpha * tb.x + bkq * e.x); y.y = a.scale * (alpha * tb.y + bkq * e.y);
-  y.z = a.scale * (alpha * tb.z + bkq * e.z); y.w = a.scale * (alpha * tb.w + bkq * e.w);
+  const float bkq = __fmul_rn(beta, kq);
+  float4 y = out4(a.scale, alpha, tb, bkq, e);
   const size_t yo = ((size_t)n * a.H_v + h) * DV + 4 * c4;
   if (a.g != nullptr) {
-    float ss = y.x * y.x + y.y * y.y + y.z * y.z + y.w * y.w;
+    float ss = sq4(y);
     ss = group_sum<TPR>(ss);  // every row group holds the same y
-    const float r = rsqrtf(ss / (float)DV + a.eps_norm);
+    const float r = rsqrtf(__fadd_rn(__fmul_rn(ss, 1.f / (float)DV), a.eps_norm));
     const float4 g4 = Elem<Tin>::load4(static_cast<const Tin*>(a.g) + yo);
     float4 w4 = make_float4(0.f, 0.f, 0.f, 0.f);
     if (a.norm_w) w4 = __ldg(reinterpret_cast<const float4*>(a.norm_w + 4 * c4));
@@ -224,6 +251,16 @@ __global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT, 2)
   float* tla = tg + (has_g ? T_s * DV : 0);
   float* tb = tla + T_s;
   float* tkq = tb + T_s;  // k^ . q^ per token
+  // the next item's raw inputs as they are in memory (copied while the
+  // current item runs): q, k [T_s][DK]; v, g [T_s][DV]; log alpha, beta [T_s]
+  constexpr int VE = 16 / (int)sizeof(Tin);  // elements per 16-byte copy
+  Tin* rq = reinterpret_cast<Tin*>(
+      reinterpret_cast<uintptr_t>(tkq + T_s + 3) & ~(uintptr_t)15);  // 16-byte aligned
+  Tin* rk = rq + T_s * DK;
+  Tin* rv = rk + T_s * DK;
+  Tin* rgt = rv + T_s * DV;
+  float* rla = reinterpret_cast<float*>(rgt + (has_g ? T_s * DV : 0));
+  float* rbe = rla + T_s;
 
   const int items = a.N * a.H_v;
   // this thread's elements of an item's state into the buffer
@@ -236,7 +273,44 @@ __global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT, 2)
     }
     sm100::cp_async_commit();
   };
-  if ((int)blockIdx.x < items) prefetch_state(blockIdx.x);
+  auto prefetch_inputs = [&](int it) {
+    const int n = it / a.H_v, h = it % a.H_v, hq = h / (a.H_v / a.H_qk);
+    const Tin* Q = static_cast<const Tin*>(a.q);
+    const Tin* K = static_cast<const Tin*>(a.k);
+    const Tin* V = static_cast<const Tin*>(a.v);
+    const Tin* G = static_cast<const Tin*>(a.g);
+    for (int i = tid; i < T_s * (DK / VE); i += NT) {
+      const int t = i / (DK / VE), col = (i % (DK / VE)) * VE;
+      const size_t tok = (size_t)n * T_s + t;
+      sm100::cp_async16(sm100::smem_u32(rq + t * DK + col), Q + (tok * a.H_qk + hq) * DK + col, true);
+      sm100::cp_async16(sm100::smem_u32(rk + t * DK + col), K + (tok * a.H_qk + hq) * DK + col, true);
+    }
+    for (int i = tid; i < T_s * (DV / VE); i += NT) {
+      const int t = i / (DV / VE), col = (i % (DV / VE)) * VE;
+      const size_t tok = (size_t)n * T_s + t;
+      sm100::cp_async16(sm100::smem_u32(rv + t * DV + col), V + (tok * a.H_v + h) * DV + col, true);
+      if (has_g)
+        sm100::cp_async16(sm100::smem_u32(rgt + t * DV + col), G + (tok * a.H_v + h) * DV + col,
+                          true);
+    }
+    for (int i = tid; i < T_s; i += NT) {
+      const size_t tok = (size_t)n * T_s + i;
+      sm100::cp_async4(sm100::smem_u32(rla + i), a.log_alpha + tok * a.H_v + h, true);
+      sm100::cp_async4(sm100::smem_u32(rbe + i), a.beta + tok * a.H_v + h, true);
+    }
+    sm100::cp_async_commit();
+  };
+  auto to_f = [](Tin x) -> float {
+    if constexpr (sizeof(Tin) == 4) {
+      return (float)x;
+    } else {
+      return __bfloat162float(x);
+    }
+  };
+  if ((int)blockIdx.x < items) {
+    prefetch_state(blockIdx.x);
+    prefetch_inputs(blockIdx.x);
+  }
   for (int item = blockIdx.x; item < items; item += gridDim.x) {
     const int n = item / a.H_v;
     const int h = item % a.H_v;
@@ -264,36 +338,33 @@ __global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT, 2)
         }
       }
     }
-    {
-      const Tin* Q = static_cast<const Tin*>(a.q);
-      const Tin* K = static_cast<const Tin*>(a.k);
-      const Tin* V = static_cast<const Tin*>(a.v);
-      const Tin* G = static_cast<const Tin*>(a.g);
-      for (int i = tid; i < T_s * DK; i += NT) {
-        const size_t tok = (size_t)n * T_s + i / DK;
-        tq[i] = Elem<Tin>::load(Q + (tok * a.H_qk + hq) * DK + i % DK);
-        tk[i] = Elem<Tin>::load(K + (tok * a.H_qk + hq) * DK + i % DK);
-      }
-      for (int i = tid; i < T_s * DV; i += NT) {
-        const size_t tok = (size_t)n * T_s + i / DV;
-        tv[i] = Elem<Tin>::load(V + (tok * a.H_v + h) * DV + i % DV);
-        if (has_g) tg[i] = Elem<Tin>::load(G + (tok * a.H_v + h) * DV + i % DV);
-      }
-      for (int i = tid; i < T_s; i += NT) {
-        const size_t tok = (size_t)n * T_s + i;
-        tla[i] = __ldg(a.log_alpha + tok * a.H_v + h);
-        tb[i] = __ldg(a.beta + tok * a.H_v + h);
-      }
-    }
     float4 w4 = make_float4(0.f, 0.f, 0.f, 0.f);
     if (has_g && a.norm_w) w4 = __ldg(reinterpret_cast<const float4*>(a.norm_w + 4 * c4));
-    // this item's state (its copies have landed), then the next item's copies
-    // into the same slots
-    float4 s[RPT];
+    // this item's state and raw inputs (their copies have landed): the state
+    // into registers, the inputs to fp32, then the next item's copies into
+    // the same buffers
     sm100::cp_async_wait_all();
+    __syncthreads();  // every thread's copies of the raw inputs have landed
+    for (int i = tid; i < T_s * DK; i += NT) {
+      tq[i] = to_f(rq[i]);
+      tk[i] = to_f(rk[i]);
+    }
+    for (int i = tid; i < T_s * DV; i += NT) {
+      tv[i] = to_f(rv[i]);
+      if (has_g) tg[i] = to_f(rgt[i]);
+    }
+    for (int i = tid; i < T_s; i += NT) {
+      tla[i] = rla[i];
+      tb[i] = rbe[i];
+    }
+    __syncthreads();  // the raw buffers are read before the next item's copies
+    float4 s[RPT];
 #pragma unroll
     for (int r = 0; r < RPT; ++r) s[r] = sst[(rg + ROWG * r) * TPR + c4];
-    if (item + (int)gridDim.x < items) prefetch_state(item + gridDim.x);
+    if (item + (int)gridDim.x < items) {
+      prefetch_state(item + gridDim.x);
+      prefetch_inputs(item + gridDim.x);
+    }
     if (a.conv_w != nullptr) {
       // front end: causal depthwise conv of kernel 4, then SiLU, over each
       // q / k / v channel of this (sequence, value head), in place on the
@@ -360,23 +431,18 @@ __global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT, 2)
 
       // a = S^T k^, b = S^T q^ over this thread's rows, then across row groups
       uint64_t pa[2] = {0ull, 0ull}, pb[2] = {0ull, 0ull};
-      float kk[RPT];
 #pragma unroll
       for (int r = 0; r < RPT; ++r) {
         const int i = rg + ROWG * r;
-        const float ki = sk[i], qi = sq[i];
-        kk[r] = ki;
-        row_partials(s[r], ki, qi, pa, pb);
+        row_partials(s[r], sk[i], sq[i], pa, pb);
       }
       red_a[par][rg][c4] = f2_to_float4(pa);
       red_b[par][rg][c4] = f2_to_float4(pb);
       __syncthreads();  // (the other parity's buffers were read before this barrier)
-      float4 ta, tbv;
-      col_sums<ROWG, TPR>(red_a[par], red_b[par], c4, &ta, &tbv);
+      // a for every thread (its rows' update); b only for warp 0, which forms y
+      const float4 ta = col_sum<ROWG, TPR>(red_a[par], c4);
       const float4 v4 = *reinterpret_cast<const float4*>(tv + t * DV + 4 * c4);
-      float4 e;
-      e.x = v4.x - alpha * ta.x; e.y = v4.y - alpha * ta.y;
-      e.z = v4.z - alpha * ta.z; e.w = v4.w - alpha * ta.w;
+      const float4 e = err4(v4, alpha, ta);
 
       // S' = alpha S + beta k^ e^T (each thread updates exactly the elements it
       // loaded), kept in registers, optionally snapshotted, stored to
@@ -389,30 +455,34 @@ __global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT, 2)
 #pragma unroll
       for (int r = 0; r < RPT; ++r) {
         const int i = rg + ROWG * r;
-        const float4 o = row_update(s[r], alpha2, beta * kk[r], e2);
+        // k^_i again (not held across the reduction)
+        const float4 o = row_update(s[r], alpha2, beta * sk[i], e2);
         s[r] = o;
         if (snap) __stcs(reinterpret_cast<float4*>(snap + (size_t)i * DV) + c4, o);
         if (sout) __stcs(reinterpret_cast<float4*>(sout + (size_t)i * DV) + c4, o);
       }
 
-      // y = scale (alpha b + beta (k^.q^) e), then the optional epilogue
-      const size_t tok = (size_t)n * T_s + t;
-      const float bkq = beta * kq;
-      float4 y;
-      y.x = a.scale * (alpha * tbv.x + bkq * e.x); y.y = a.scale * (alpha * tbv.y + bkq * e.y);
-      y.z = a.scale * (alpha * tbv.z + bkq * e.z); y.w = a.scale * (alpha * tbv.w + bkq * e.w);
-      const size_t yo = (tok * a.H_v + h) * DV + 4 * c4;
-      if (has_g) {
-        float ss = y.x * y.x + y.y * y.y + y.z * y.z + y.w * y.w;
-        ss = group_sum<TPR>(ss);  // every row group holds the same y
-        const float r = rsqrtf(ss / (float)DV + a.eps_norm);
-        const float4 g4 = *reinterpret_cast<const float4*>(tg + t * DV + 4 * c4);
-        y.x = y.x * r * (1.f + w4.x) * sigmoidf_(g4.x);
-        y.y = y.y * r * (1.f + w4.y) * sigmoidf_(g4.y);
-        y.z = y.z * r * (1.f + w4.z) * sigmoidf_(g4.z);
-        y.w = y.w * r * (1.f + w4.w) * sigmoidf_(g4.w);
+      // y = scale (alpha b + beta (k^.q^) e), then the optional epilogue: every
+      // row group holds the same column sums, so warp 0 alone forms y (its row
+      // groups in full, for the lane-group sum) and row group 0 stores it
+      if (tid < 32) {
+        const float4 tbv = col_sum<ROWG, TPR>(red_b[par], c4);
+        const size_t tok = (size_t)n * T_s + t;
+        const float bkq = __fmul_rn(beta, kq);
+        float4 y = out4(a.scale, alpha, tbv, bkq, e);
+        const size_t yo = (tok * a.H_v + h) * DV + 4 * c4;
+        if (has_g) {
+          float ss = sq4(y);
+          ss = group_sum<TPR>(ss);
+          const float r = rsqrtf(__fadd_rn(__fmul_rn(ss, 1.f / (float)DV), a.eps_norm));
+          const float4 g4 = *reinterpret_cast<const float4*>(tg + t * DV + 4 * c4);
+          y.x = y.x * r * (1.f + w4.x) * sigmoidf_(g4.x);
+          y.y = y.y * r * (1.f + w4.y) * sigmoidf_(g4.y);
+          y.z = y.z * r * (1.f + w4.z) * sigmoidf_(g4.z);
+          y.w = y.w * r * (1.f + w4.w) * sigmoidf_(g4.w);
+        }
+        if (rg == 0) Elem<Tin>::store4(static_cast<Tin*>(a.y) + yo, y);
       }
-      if (rg == 0) Elem<Tin>::store4(static_cast<Tin*>(a.y) + yo, y);
     }  // tokens
     __syncthreads();  // the staged inputs and the reduction buffers are refilled for the next item
   }  // items
@@ -421,7 +491,10 @@ __global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT, 2)
 // Dynamic shared memory of the multi-token kernel for T_s tokens.
 template <int DK, int DV>
 size_t multi_smem_bytes(int T_s, bool has_g) {
-  return sizeof(float) * ((size_t)DK * DV + (size_t)T_s * (2 * DK + (has_g ? 2 : 1) * DV + 3));
+  // state, fp32 inputs and scalars, then the raw next-item inputs (16-byte
+  // aligned, at most 4 B of input per element) and their scalars
+  return sizeof(float) * ((size_t)DK * DV + (size_t)T_s * (2 * DK + (has_g ? 2 : 1) * DV + 3) + 4) +
+         (size_t)T_s * (2 * DK + (has_g ? 2 : 1) * DV) * 4 + (size_t)T_s * 8 + 16;
 }
 
 template <int DK, int DV, typename Tin>
