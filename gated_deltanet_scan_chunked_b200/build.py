@@ -67,7 +67,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
                 sys.stdout.write(log)
     if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < _newest(objs):
         tmp = LIB + ".tmp%d" % os.getpid()
-        cmd = [NVCC, *ARCH, "-shared", "-Xcompiler", "-fPIC", *objs, "-o", tmp, "-lcudart_static", "-lcublasLt"]
+        cmd = [NVCC, *ARCH, "-shared", "-Xcompiler", "-fPIC", *objs, "-o", tmp, "-lcudart_static"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError("link failed:\n%s%s" % (r.stdout, r.stderr))

@@ -13,8 +13,8 @@
 // The state is E4M3 with one fp32 scale per (token, branch) row; a written
 // row is requantised with scale max|R'| / 448 (1 for an all-zero row).
 //
-// Read = three kernels of this file around two bf16 GEMMs (cuBLASLt, fp32
-// accumulation) for the low-rank router:
+// Read = three kernels of this file around two bf16 GEMMs (gdn_gemm.cu:
+// tcgen05 MMAs, fp32 accumulation) for the low-rank router:
 //   gr_norm    codes -> R^ (bf16, group RMSNorm with gains), a warp per row
 //   GEMM       H' = (1/n_r) R^ [W_d; W_w; 0]^T            [T, rank + 8]
 //   gr_router  H = SiLU(H'[:, :rank]) in place; s = 2 sigmoid(H'[:, rank:rank+n_r])
@@ -22,11 +22,8 @@
 //   gr_gate    x = (1/n_r) sum_i sigmoid(L_i) o R^_i      [T, d] bf16
 // Write = one kernel, one warp per (token, branch) row held in registers, in
 // place.
-#include <cublasLt.h>
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
-
-#include <mutex>
 
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
@@ -319,73 +316,15 @@ __global__ void __launch_bounds__(128) gr_write_kernel(const GrWriteArgs a) {
   if (lane == 0) a.scales[row] = nsc;
 }
 
-// ---- cuBLASLt, one handle per device --------------------------------------
-
-constexpr int kMaxDevices = 64;
-std::mutex g_lt_mu;
-cublasLtHandle_t g_lt[kMaxDevices] = {nullptr};
-
-cublasLtHandle_t lt_handle() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lk(g_lt_mu);
-  if (g_lt[dev] == nullptr && cublasLtCreate(&g_lt[dev]) != CUBLAS_STATUS_SUCCESS)
-    g_lt[dev] = nullptr;
-  return g_lt[dev];
-}
-
-// Column-major D[m x n] = alpha op(A) op(B), bf16 operands and result, fp32
-// accumulation; A is stored k x m (ld lda) and transposed, B is k x n (ldb).
-gdn_status lt_gemm(int m, int n, int k, float alpha, const void* A, int lda, const void* B,
-                   int ldb, void* D, int ldd, void* ws, size_t ws_bytes, cudaStream_t stream) {
-  cublasLtHandle_t h = lt_handle();
-  if (h == nullptr) return GDN_ERR_CUDA;
-  cublasLtMatmulDesc_t op = nullptr;
-  cublasLtMatrixLayout_t Ad = nullptr, Bd = nullptr, Dd = nullptr;
-  cublasLtMatmulPreference_t pref = nullptr;
-  gdn_status st = GDN_ERR_CUDA;
-  const cublasOperation_t ta = CUBLAS_OP_T, tb = CUBLAS_OP_N;
-  const float beta = 0.f;
-  cublasLtMatmulHeuristicResult_t res;
-  int nres = 0;
-  if (cublasLtMatmulDescCreate(&op, CUBLAS_COMPUTE_32F, CUDA_R_32F) != CUBLAS_STATUS_SUCCESS)
-    goto done;
-  cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_TRANSA, &ta, sizeof(ta));
-  cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_TRANSB, &tb, sizeof(tb));
-  if (cublasLtMatrixLayoutCreate(&Ad, CUDA_R_16BF, k, m, lda) != CUBLAS_STATUS_SUCCESS ||
-      cublasLtMatrixLayoutCreate(&Bd, CUDA_R_16BF, k, n, ldb) != CUBLAS_STATUS_SUCCESS ||
-      cublasLtMatrixLayoutCreate(&Dd, CUDA_R_16BF, m, n, ldd) != CUBLAS_STATUS_SUCCESS)
-    goto done;
-  if (cublasLtMatmulPreferenceCreate(&pref) != CUBLAS_STATUS_SUCCESS) goto done;
-  cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES, &ws_bytes,
-                                       sizeof(ws_bytes));
-  if (cublasLtMatmulAlgoGetHeuristic(h, op, Ad, Bd, Dd, Dd, pref, 1, &res, &nres) !=
-          CUBLAS_STATUS_SUCCESS ||
-      nres == 0) {
-    st = GDN_ERR_UNSUPPORTED;
-    goto done;
-  }
-  if (cublasLtMatmul(h, op, &alpha, A, Ad, B, Bd, &beta, D, Dd, D, Dd, &res.algo, ws, ws_bytes,
-                     stream) == CUBLAS_STATUS_SUCCESS)
-    st = GDN_OK;
-done:
-  if (pref) cublasLtMatmulPreferenceDestroy(pref);
-  if (Dd) cublasLtMatrixLayoutDestroy(Dd);
-  if (Bd) cublasLtMatrixLayoutDestroy(Bd);
-  if (Ad) cublasLtMatrixLayoutDestroy(Ad);
-  if (op) cublasLtMatmulDescDestroy(op);
-  return st;
-}
-
 size_t a256(size_t x) { return (x + 255) & ~(size_t)255; }
-constexpr size_t kLtWorkspace = 32u << 20;
 
 }  // namespace
 
 size_t gr_read_workspace_bytes(int64_t T, int32_t n_r, int32_t d, int32_t rank) {
   const size_t nd = (size_t)n_r * d;
   return 2 * a256((size_t)T * nd * 2) + a256((size_t)T * (rank + 8) * 2) +
-         a256((size_t)(rank + 8) * nd * 2) + kLtWorkspace;
+         a256((size_t)(rank + 8) * nd * 2) +
+         a256(gemm_tn_workspace_bytes((int)T, rank + 8, (int)nd));
 }
 
 template <template <int> class K, typename Args>
@@ -424,7 +363,8 @@ gdn_status launch_gr_read(GrArgs a, void* ws, cudaStream_t stream) {
   a.logits = reinterpret_cast<__nv_bfloat16*>(p + a256((size_t)a.T * nd * 2));
   __nv_bfloat16* H = reinterpret_cast<__nv_bfloat16*>(p + 2 * a256((size_t)a.T * nd * 2));
   char* Wdw = p + 2 * a256((size_t)a.T * nd * 2) + a256((size_t)a.T * ldh * 2);
-  void* lt_ws = Wdw + a256((size_t)ldh * nd * 2);
+  char* gws = Wdw + a256((size_t)ldh * nd * 2);  // the router GEMM's split-K partials
+  const size_t gws_bytes = gemm_tn_workspace_bytes((int)a.T, ldh, (int)nd);
   if (a.T == 0) return GDN_OK;
   // [W_d; W_w; 0] in one operand, so that one GEMM gives the router and the
   // write scalars
@@ -437,15 +377,15 @@ gdn_status launch_gr_read(GrArgs a, void* ws, cudaStream_t stream) {
     return GDN_ERR_CUDA;
   gdn_status st = launch_rows<NormK>(a, a.T * a.n_r, a.d, stream);
   if (st != GDN_OK) return st;
-  // H'^T (col-major ldh x T) = [W_d; W_w; 0] R^^T, alpha = 1/n_r
-  st = lt_gemm(ldh, (int)a.T, (int)nd, 1.f / (float)a.n_r, Wdw, (int)nd, a.rhat, (int)nd, H, ldh,
-               lt_ws, kLtWorkspace, stream);
+  // H' [T][ldh] = (1/n_r) R^ [T][nd] [W_d; W_w; 0]^T
+  st = gemm_tn_bf16((int)a.T, ldh, (int)nd, 1.f / (float)a.n_r, a.rhat, (int64_t)nd, Wdw,
+                    (int64_t)nd, H, ldh, gws, gws_bytes, stream);
   if (st != GDN_OK) return st;
   const int64_t groups = a.T * (ldh / 8);
   gr_router_kernel<<<(unsigned)((groups + kNT - 1) / kNT), kNT, 0, stream>>>(a, H, ldh);
-  // L^T (col-major nd x T) = W_u (nd x rank) SiLU(H)^T
-  st = lt_gemm((int)nd, (int)a.T, a.rank, 1.f, a.W_u, a.rank, H, ldh, a.logits, (int)nd, lt_ws,
-               kLtWorkspace, stream);
+  // L [T][nd] = SiLU(H) [T][rank] W_u^T (W_u [nd][rank])
+  st = gemm_tn_bf16((int)a.T, (int)nd, a.rank, 1.f, H, ldh, a.W_u, a.rank, a.logits,
+                    (int64_t)nd, nullptr, 0, stream);
   if (st != GDN_OK) return st;
   const int64_t g2 = a.T * (a.d / 8);
   const unsigned gg = (unsigned)((g2 + kNT - 1) / kNT);

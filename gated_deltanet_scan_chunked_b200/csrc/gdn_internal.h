@@ -158,6 +158,20 @@ struct GrWriteArgs {
 };
 
 size_t gr_read_workspace_bytes(int64_t T, int32_t n_r, int32_t d, int32_t rank);
+
+// The library's device error word on the current device (nullptr on failure).
+int* device_error_word();
+
+// D[M][N] = alpha A[M][K] B[N][K]^T: bf16 row-major operands with leading
+// dimensions in elements, fp32 accumulation on the tensor cores
+// (gdn_gemm.cu).  K, N and the leading dimensions multiples of 8, pointers
+// 16-byte aligned, else GDN_ERR_UNSUPPORTED.  Products with few output tiles
+// split K over several CTAs; their fp32 partials need `ws` (16-byte aligned,
+// gemm_tn_workspace_bytes), without which K is not split.
+size_t gemm_tn_workspace_bytes(int M, int N, int K);
+gdn_status gemm_tn_bf16(int M, int N, int K, float alpha, const void* A, int64_t lda,
+                        const void* B, int64_t ldb, void* D, int64_t ldd, void* ws,
+                        size_t ws_bytes, cudaStream_t stream);
 gdn_status launch_gr_read(GrArgs a, void* ws, cudaStream_t stream);
 gdn_status launch_gr_write(const GrWriteArgs& a, cudaStream_t stream);
 
