@@ -852,7 +852,7 @@ def run_ours(args, world, rank, local):
                                "frac": wbytes / (wms_ * 1e-3) / 1e9 / peaks["hbm_gbs"],
                                "algorithmic_bytes": wbytes},
             "clocks": gclk_r}
-        launches_gr = gsteps * (3 + 1)  # our kernels: norm, silu, gate; write (plus 2 cuBLASLt GEMMs)
+        launches_gr = gsteps * (6 + 1)  # read: norm, GEMM, split-K sum, router, GEMM, gate; write
         del gws, gflush, rgraph, wgraph
 
     cpu = None

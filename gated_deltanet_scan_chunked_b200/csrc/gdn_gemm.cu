@@ -261,7 +261,7 @@ bool make_tmap_2d(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, 
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int gemm_bn(int N) { return N <= 1024 ? 64 : 128; }
+int gemm_bn(int N) { return N <= 64 ? 64 : 128; }
 
 // K splits: enough CTAs for two per SM on a 148-SM part when the tile grid
 // alone gives fewer, each split keeping at least eight 64-wide K steps.
@@ -295,8 +295,7 @@ gdn_status launch_bn(const GemmParams& prm, int splits, cudaStream_t stream) {
 // D[M][N] = alpha A[M][K] B[N][K]^T, bf16 row-major with leading dimensions
 // lda / ldb / ldd (elements).  Requirements (else GDN_ERR_UNSUPPORTED): K and
 // N multiples of 8, leading dimensions multiples of 8, 16-byte aligned
-// pointers.  Narrow products (N <= 1024) take 64-column tiles, so that more
-// CTAs share the K loop.
+// pointers.  Products with at most 64 columns take 64-column tiles.
 size_t gemm_tn_workspace_bytes(int M, int N, int K) {
   return (size_t)gemm_splits(M, N, K) * (size_t)M * (size_t)N * sizeof(float);
 }
@@ -329,8 +328,9 @@ gdn_status gemm_tn_bf16(int M, int N, int K, float alpha, const void* A, int64_t
   prm.alpha = alpha;
   prm.err = device_error_word();
   if (prm.err == nullptr) return GDN_ERR_CUDA;
-  // short K loops (a few stages suffice) leave room for more CTAs per SM
-  const bool short_k = prm.kc <= 4 * kBK;
+  // short K loops (two stages suffice) leave room for more CTAs per SM, whose
+  // epilogues then overlap each other's loads
+  const bool short_k = prm.kc <= 8 * kBK;
   gdn_status st = bn == 64 ? (short_k ? launch_bn<64, 2>(prm, splits, stream)
                                       : launch_bn<64, 4>(prm, splits, stream))
                            : (short_k ? launch_bn<128, 2>(prm, splits, stream)
