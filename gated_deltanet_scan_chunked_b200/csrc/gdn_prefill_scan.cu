@@ -685,7 +685,7 @@ __device__ void prep_control(const ScanParams& P, uint32_t sb, uint32_t tb, int 
   auto load_tiles = [&](int c) {
     const int z = (int)(t_begin + (int64_t)c * kC);
     mbar_arrive_expect_tx(B.tma, 49152);
-#pragma unroll
+#pragma unroll 1
     for (int pp = 0; pp < 2; ++pp) {
       tma_load_3d(sb + P_KQ + pp * 16384, &P.tk, 64 * pp, hq, z, B.tma);
       tma_load_3d(sb + P_KQ + pp * 16384 + 8192, &P.tq, 64 * pp, hq, z, B.tma);
@@ -706,7 +706,7 @@ __device__ void prep_control(const ScanParams& P, uint32_t sb, uint32_t tb, int 
     ok = mbar_wait(B.tma, ph_tma, kWait);
     ph_tma ^= 1;
     if (!ok) break;
-#pragma unroll
+#pragma unroll 1
     for (int kk = 0; kk < 8; ++kk) {
       const uint64_t d = sdesc(sb + P_KQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
       mma_f16(tb, d, d, ID_KQ, kk > 0);
@@ -718,11 +718,11 @@ __device__ void prep_control(const ScanParams& P, uint32_t sb, uint32_t tb, int 
     ph_sp ^= 1;
     if (!ok) break;
     fence_after_sync();
-#pragma unroll
+#pragma unroll 1
     for (int part = 0; part < 2; ++part) {
       const uint32_t aw = sb + (part ? P_TWL : P_TWH);
       const uint32_t bu = sb + (part ? P_TBL : P_TBH);
-#pragma unroll
+#pragma unroll 1
       for (int kk = 0; kk < 4; ++kk) {
         mma_f16(tb + 64, sdesc(aw + kk * 32, 16, 1024), sdesc(sb + P_KQ + kk * 2048, 16384, 1024),
                 ID_W, part | (kk > 0));
@@ -982,12 +982,12 @@ __device__ void chain_mma(const ScanParams& P, uint32_t sb, uint32_t tbase, int 
     GDN_SCAN_TRACE(2, 50);
     // Delta^T part first (its own commit: the state step waits only for it),
     // then the gamma Q^ part of Y^T
-#pragma unroll
+#pragma unroll 1
     for (int kk = 0; kk < 8; ++kk)
       mma_f16_ta(tbase + 256 + 128 * b, tbase + 8 * kk,
                  sdesc(slot + SL_WQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024), ID_Y, kk > 0);
     mma_commit(B.bar1);
-#pragma unroll
+#pragma unroll 1
     for (int kk = 0; kk < 8; ++kk)
       mma_f16_ta(tbase + 256 + 128 * b + 64, tbase + 8 * kk,
                  sdesc(slot + SL_WQ + (kk >> 2) * 16384 + 8192 + (kk & 3) * 32, 16, 1024), ID_Y,
@@ -998,12 +998,12 @@ __device__ void chain_mma(const ScanParams& P, uint32_t sb, uint32_t tbase, int 
     if (!ok) break;
     fence_after_sync();
     GDN_SCAN_TRACE(2, 52);
-#pragma unroll
+#pragma unroll 1
     for (int kk = 0; kk < 4; ++kk)
       mma_f16_ta(tbase + 128, tbase + 64 + 8 * kk, sdesc(slot + SL_K + kk * 2048, 8192, 1024),
                  ID_S, kk > 0);
     mma_commit(B.bar3);
-#pragma unroll
+#pragma unroll 1
     for (int kk = 0; kk < 4; ++kk)
       mma_f16_ta(tbase + 256 + 128 * b + 64, tbase + 64 + 8 * kk,
                  sdesc(slot + SL_P + kk * 32, 16, 1024), ID_Y, 1);
@@ -1043,7 +1043,7 @@ __device__ void chain_loader(const ScanParams& P, uint32_t sb, int item, const C
       const uint8_t* src = ring + (size_t)(c % kRingS) * kScanSlotBytes;
       const uint32_t dst = sb + b * kSlotStride;
       mbar_arrive_expect_tx(&B.full[b], kSlotLoadBytes);
-#pragma unroll
+#pragma unroll 1
       for (int k = 0; k < 3; ++k) bulk_load_g2s(dst + 16384 * k, src + 16384 * k, 16384, &B.full[b]);
       bulk_load_g2s(dst + SL_P, src + SL_P, kSlotLoadBytes - SL_P, &B.full[b]);
       nfull = c + 1;
@@ -1123,13 +1123,13 @@ __device__ void chain_epilogue(const ScanParams& P, uint8_t* gb, int item, const
       }
       // raw g row t: 16-byte chunk cc of panel p at cc ^ (t % 8) (TMA, SW128)
       const uint8_t* gsrc = gb + C_GS + b * 16384 + t * 128;
-      // four 16-byte chunks at a time, their loads ahead of their stores
+      // two 16-byte chunks at a time, their loads ahead of their stores
 #pragma unroll 1
-      for (int cb = 0; cb < 16; cb += 4) {
-        uint4 u[4], gq[4];
-        float4 w[8];
+      for (int cb = 0; cb < 16; cb += 2) {
+        uint4 u[2], gq[2];
+        float4 w[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
+        for (int k = 0; k < 2; ++k) {
           const int ch = cb + k;
           u[k] = *reinterpret_cast<const uint4*>(yst + ((ch ^ (t & 15)) << 4));
           gq[k] = *reinterpret_cast<const uint4*>(gsrc + (ch >> 3) * 8192 +
@@ -1138,7 +1138,7 @@ __device__ void chain_epilogue(const ScanParams& P, uint8_t* gb, int item, const
           w[2 * k + 1] = *reinterpret_cast<const float4*>(sWn + 8 * ch + 4);
         }
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
+        for (int k = 0; k < 2; ++k) {
           const float wv[8] = {w[2 * k].x,     w[2 * k].y,     w[2 * k].z,     w[2 * k].w,
                                w[2 * k + 1].x, w[2 * k + 1].y, w[2 * k + 1].z, w[2 * k + 1].w};
           const uint32_t w4[4] = {u[k].x, u[k].y, u[k].z, u[k].w};

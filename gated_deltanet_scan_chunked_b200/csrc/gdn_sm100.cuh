@@ -184,6 +184,8 @@ __device__ __forceinline__ void fence_mbar_init() {
 // `max_iter` polls.  Returns false on timeout.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t max_iter) {
   const uint32_t a = smem_u32(bar);
+  // a rolled loop: every wait site stays a few instructions long
+#pragma unroll 1
   for (uint32_t it = 0; it < max_iter; ++it) {
     uint32_t done;
     asm volatile(
@@ -254,6 +256,7 @@ __device__ __forceinline__ void bulk_wait_all() {
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
                                                   uint32_t max_iter) {
   const uint32_t a = smem_u32(bar);
+#pragma unroll 1
   for (uint32_t it = 0; it < max_iter; ++it) {
     uint32_t done;
     asm volatile(
@@ -305,6 +308,7 @@ __device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned l
 // Spin (bounded) until *p >= target; returns false on timeout.
 __device__ __forceinline__ bool wait_flag_ge(const unsigned long long* p, unsigned long long target,
                                              uint32_t max_iter) {
+#pragma unroll 1
   for (uint32_t it = 0; it < max_iter; ++it) {
     if (ld_acquire_u64(p) >= target) return true;
     __nanosleep(32);
