@@ -94,10 +94,11 @@ constexpr uint32_t C_GS = C_YS + 32768;           // raw g of the staged chunks 
                                                   //   bf16 [64 t][128 j], SW128, 2 panels
 constexpr uint32_t C_WN = C_GS + 32768;           // 1 + norm_w [128] fp32
 constexpr uint32_t C_MISC = C_WN + 512;           // warp maxima [2][8], stage exponents [2]
-constexpr uint32_t C_BAR = C_MISC + 128;           // full[2] bar1 bar3 barY[2] ysfull[2]
-                                                  //   ysempty[2] sready dready gfull[2],
+constexpr uint32_t C_BAR = C_MISC + 128;           // fullA[2] bar1 bar3 barY[2] ysfull[2]
+                                                  //   ysempty[2] sready dready gfull[2]
+                                                  //   fullB[2] fullC[2] bar1b[2] ufree[2],
                                                   //   TMEM slot
-constexpr uint32_t kChainSmem = C_BAR + 128;
+constexpr uint32_t kChainSmem = C_BAR + 256;
 
 // ---- preparation sub-pipeline shared memory (two per CTA) -------------------------
 constexpr uint32_t P_KQ = 0;           // [K; Q] raw bf16 [128][128], SW128, 2 panels x 16 KB
@@ -682,6 +683,17 @@ __device__ void prep_control(const ScanParams& P, uint32_t sb, uint32_t tb, int 
   const int nch = (int)((t_end - t_begin + kC - 1) / kC);
   unsigned long long* ready = a.ring_flags + (size_t)item * 2 * kRingS;
   unsigned long long* consumed = ready + kRingS;
+  // chunk c's q / k / v tiles into L2 ahead of their loads (the loads land
+  // only a few thousand cycles before the compute threads need them)
+  auto prefetch_tiles = [&](int c) {
+    const int z = (int)(t_begin + (int64_t)c * kC);
+#pragma unroll 1
+    for (int pp = 0; pp < 2; ++pp) {
+      tma_prefetch_3d(&P.tk, 64 * pp, hq, z);
+      tma_prefetch_3d(&P.tq, 64 * pp, hq, z);
+      tma_prefetch_3d(&P.tv, 64 * pp, h, z);
+    }
+  };
   auto load_tiles = [&](int c) {
     const int z = (int)(t_begin + (int64_t)c * kC);
     mbar_arrive_expect_tx(B.tma, 49152);
@@ -694,14 +706,22 @@ __device__ void prep_control(const ScanParams& P, uint32_t sb, uint32_t tb, int 
   };
   uint32_t ph_tma = 0, ph_wu = 0, ph_sp = 0, ph_st = 0;
   bool ok = true;
-  if (lane_id < nch) load_tiles(lane_id);
-  for (int c = lane_id; ok && c < nch; c += kLanes) {
-    // the output slot of chunk c held chunk c - ring: the chain side must be
-    // done with it
-    if (c >= kRingS)
-      ok = wait_flag_ge(&consumed[c % kRingS], (unsigned long long)(c - kRingS) + 1, kWait);
-    if (!ok) break;
+  // The compute threads may start chunk c once its output slot (which held
+  // chunk c - ring: the chain side must be done with it) is free.  The next
+  // chunk's slot is handed over before this chunk is published, so that they
+  // do not wait for the publication.
+  auto open_slot = [&](int c) -> bool {
+    if (c >= kRingS &&
+        !wait_flag_ge(&consumed[c % kRingS], (unsigned long long)(c - kRingS) + 1, kWait))
+      return false;
     mbar_arrive(B.slot);
+    return true;
+  };
+  if (lane_id < nch) {
+    load_tiles(lane_id);
+    ok = open_slot(lane_id);
+  }
+  for (int c = lane_id; ok && c < nch; c += kLanes) {
     // [K; Q] K^T once the tiles have landed
     ok = mbar_wait(B.tma, ph_tma, kWait);
     ph_tma ^= 1;
@@ -712,6 +732,8 @@ __device__ void prep_control(const ScanParams& P, uint32_t sb, uint32_t tb, int 
       mma_f16(tb, d, d, ID_KQ, kk > 0);
     }
     mma_commit(B.mma0);
+    // the next chunk's tiles into L2 while this one is prepared
+    if (c + kLanes < nch) prefetch_tiles(c + kLanes);
     // W = T diag(beta gamma rk) K_raw (M = 64, N = 128) and U^T = V^T (T
     // diag(beta))^T (M = 128, N = 64), hi then lo parts, once the splits are in
     ok = mbar_wait(B.splits, ph_sp, kWait);
@@ -738,6 +760,8 @@ __device__ void prep_control(const ScanParams& P, uint32_t sb, uint32_t tb, int 
     if (c + kLanes < nch) {
       fence_proxy_async();  // the generic reads of the raw tiles precede the TMA writes
       load_tiles(c + kLanes);
+      ok = open_slot(c + kLanes);
+      if (!ok) break;
     }
     // the compute threads have stored the slot: publish it
     ok = mbar_wait(B.stored, ph_st, kWait);
@@ -762,7 +786,7 @@ __device__ void prep_control(const ScanParams& P, uint32_t sb, uint32_t tb, int 
 // hand off through mbarriers, all of whose waits are bounded.
 // ============================================================================
 struct ChainBars {
-  uint64_t* full;     // [2] slot bytes landed (buffer c % 2)
+  uint64_t* fullA;    // [2] [-W; gamma Q^] of the slot in buffer c % 2 landed
   uint64_t* bar1;     // [Delta^T | Y^T] = S^T [-W; gamma Q^]^T done
   uint64_t* bar3;     // S^T increment done
   uint64_t* barY;     // [2] Y^T of chunk c complete (accumulator c % 2)
@@ -771,6 +795,10 @@ struct ChainBars {
   uint64_t* sready;   // S^T operand of the next chunk in TMEM (compute warps)
   uint64_t* dready;   // Delta^T operand in TMEM (compute warps)
   uint64_t* gfull;    // [2] raw g of the chunk in stage c % 2 landed (TMA)
+  uint64_t* fullB;    // [2] the scalars and U^T landed
+  uint64_t* fullC;    // [2] dec K^ and P landed
+  uint64_t* bar1b;    // [2] both S^T [-W; gamma Q^]^T products done ([-W; gamma Q^] free)
+  uint64_t* ufree;    // [2] the scalars and U^T read (arrived by the MMA thread after dready)
 };
 
 __device__ void chain_compute(const ScanParams& P, uint8_t* gb, uint32_t sb, uint32_t tbase,
@@ -786,7 +814,6 @@ __device__ void chain_compute(const ScanParams& P, uint8_t* gb, uint32_t sb, uin
       seq_bounds(a.cu_seqlens, seq, a.total_T, &t_begin, &t_end, tid == 0 ? a.err : nullptr);
   const int nch = bounds_ok ? (int)((t_end - t_begin + kC - 1) / kC) : 0;
   float* sMaxw = reinterpret_cast<float*>(gb + C_MISC);
-  unsigned long long* consumed = a.ring_flags + (size_t)item * 2 * kRingS + kRingS;
   int* sYExp = reinterpret_cast<int*>(gb + C_MISC + 64);  // exponent of each Y stage
   const size_t st_off = ((size_t)seq * a.H_v + h) * (size_t)(kD * kD);
   const uint32_t tSA = tbase + lane_off + 32 * cg;
@@ -819,11 +846,10 @@ __device__ void chain_compute(const ScanParams& P, uint8_t* gb, uint32_t sb, uin
     // still reading chunk c - 1's maxima is not overwritten)
     float* mx = sMaxw + 8 * (c & 1);
     if (lane == 0) mx[warp] = smax;
-    bool okw = mbar_wait(&B.full[c & 1], par(ph_full, c & 1), kWait) && okin;
+    // the slot's scalars (and U^T) have landed
+    bool okw = mbar_wait(&B.fullB[c & 1], par(ph_full, c & 1), kWait) && okin;
     ph_full ^= 1u << (c & 1);
     if (!named_sync_and(1, kChainT, okw)) return INT32_MIN;
-    // slot c has landed in shared memory: its global image may be reused
-    if (tid == 0) st_release_u64(&consumed[c % kRingS], (unsigned long long)c + 1);
     float mS = mx[0];
 #pragma unroll
     for (int w = 1; w < 8; ++w) mS = fmaxf(mS, mx[w]);
@@ -969,14 +995,18 @@ __device__ void chain_mma(const ScanParams& P, uint32_t sb, uint32_t tbase, int 
   int64_t t_begin, t_end;
   if (!seq_bounds(a.cu_seqlens, seq, a.total_T, &t_begin, &t_end, nullptr)) return;
   const int nch = (int)((t_end - t_begin + kC - 1) / kC);
-  uint32_t ph_s = 0, ph_d = 0;
+  unsigned long long* consumed = a.ring_flags + (size_t)item * 2 * kRingS + kRingS;
+  uint32_t ph_s = 0, ph_d = 0, phA = 0, phC = 0;  // phA, phC: parity bits per buffer
   bool ok = true;
   for (int c = 0; ok && c < nch; ++c) {
     const int b = c & 1;
     const uint32_t slot = sb + b * kSlotStride;
-    // S^T of chunk c is in TMEM (the compute warps saw slot c land)
+    // S^T of chunk c is in TMEM (the compute warps saw slot c's scalars land)
+    // and [-W; gamma Q^] of chunk c has landed
     ok = mbar_wait(B.sready, ph_s, kWait);
     ph_s ^= 1;
+    ok = ok && mbar_wait(&B.fullA[b], par(phA, b), kWait);
+    phA ^= 1u << b;
     if (!ok) break;
     fence_after_sync();
     GDN_SCAN_TRACE(2, 50);
@@ -992,9 +1022,17 @@ __device__ void chain_mma(const ScanParams& P, uint32_t sb, uint32_t tbase, int 
       mma_f16_ta(tbase + 256 + 128 * b + 64, tbase + 8 * kk,
                  sdesc(slot + SL_WQ + (kk >> 2) * 16384 + 8192 + (kk & 3) * 32, 16, 1024), ID_Y,
                  kk > 0);
+    mma_commit(&B.bar1b[b]);  // buffer b's [-W; gamma Q^] may take chunk c + 2's
     GDN_SCAN_TRACE(2, 51);
     ok = mbar_wait(B.dready, ph_d, kWait);  // Delta^T of chunk c is in TMEM
     ph_d ^= 1;
+    if (!ok) break;
+    // the compute warps have read the scalars and U^T: buffer b may take
+    // chunk c + 2's
+    mbar_arrive(&B.ufree[b]);
+    // dec K^ and P of chunk c have landed
+    ok = mbar_wait(&B.fullC[b], par(phC, b), kWait);
+    phC ^= 1u << b;
     if (!ok) break;
     fence_after_sync();
     GDN_SCAN_TRACE(2, 52);
@@ -1008,6 +1046,10 @@ __device__ void chain_mma(const ScanParams& P, uint32_t sb, uint32_t tbase, int 
       mma_f16_ta(tbase + 256 + 128 * b + 64, tbase + 64 + 8 * kk,
                  sdesc(slot + SL_P + kk * 32, 16, 1024), ID_Y, 1);
     mma_commit(&B.barY[b]);
+    // every part of slot c is in shared memory: its global image may be
+    // reused (a release store waits for this thread's earlier stores, so it
+    // comes after the products are issued)
+    st_release_u64(&consumed[c % kRingS], (unsigned long long)c + 1);
     GDN_SCAN_TRACE(2, 53);
   }
   if (!ok) atomicOr(a.err, kErrTimeout);
@@ -1025,29 +1067,49 @@ __device__ void chain_loader(const ScanParams& P, uint32_t sb, int item, const C
   const uint8_t* ring =
       static_cast<const uint8_t*>(a.ring) + (size_t)item * kRingS * kScanSlotBytes;
   unsigned long long* ready = a.ring_flags + (size_t)item * 2 * kRingS;
-  uint32_t phY = 0, phE = 0;  // parity bits per buffer
-  int nfull = 0, ngs = 0;     // chunks whose slot / g copies were issued (for the drain)
+  // parity bits per buffer of the barriers that free each part of it
+  uint32_t ph1b = 0, phU = 0, phY = 0, phE = 0;
+  // chunks whose copies were issued, per part (for the drain)
+  int nA = 0, nB = 0, nC = 0, ngs = 0;
   bool ok = true;
+  // Chunk c into buffer c % 2 in three parts, each as soon as chunk c - 2 is
+  // done with that part of the buffer: [-W; gamma Q^] after both products
+  // that read it, the scalars and U^T after the Delta step, dec K^ and P
+  // after the last products of chunk c - 2.
   for (int c = 0; ok && c < nch; ++c) {
     const int b = c & 1;
+    const uint8_t* src = ring + (size_t)(c % kRingS) * kScanSlotBytes;
+    const uint32_t dst = sb + b * kSlotStride;
+    ok = wait_flag_ge(&ready[c % kRingS], (unsigned long long)c + 1, kWait);
+    if (!ok) break;
+    fence_proxy_async_global();
+    if (c >= 2) {
+      ok = mbar_wait(&B.bar1b[b], par(ph1b, b), kWait);
+      ph1b ^= 1u << b;
+      if (!ok) break;
+    }
+    mbar_arrive_expect_tx(&B.fullA[b], 32768);
+    bulk_load_g2s(dst + SL_WQ, src + SL_WQ, 16384, &B.fullA[b]);
+    bulk_load_g2s(dst + SL_WQ + 16384, src + SL_WQ + 16384, 16384, &B.fullA[b]);
+    nA = c + 1;
+    if (c >= 2) {
+      ok = mbar_wait(&B.ufree[b], par(phU, b), kWait);
+      phU ^= 1u << b;
+      if (!ok) break;
+    }
+    fence_proxy_async();  // the compute warps' reads of the old scalars / U^T precede the copy
+    mbar_arrive_expect_tx(&B.fullB[b], (SL_U - SL_SCAL) + 16384);
+    bulk_load_g2s(dst + SL_SCAL, src + SL_SCAL, SL_U - SL_SCAL, &B.fullB[b]);
+    bulk_load_g2s(dst + SL_U, src + SL_U, 16384, &B.fullB[b]);
+    nB = c + 1;
     if (c >= 2) {
       ok = mbar_wait(&B.barY[b], par(phY, b), kWait);
       phY ^= 1u << b;
       if (!ok) break;
     }
-    ok = wait_flag_ge(&ready[c % kRingS], (unsigned long long)c + 1, kWait);
-    if (!ok) break;
-    fence_proxy_async_global();
-    fence_proxy_async();  // this buffer's earlier generic reads precede the copy
-    {
-      const uint8_t* src = ring + (size_t)(c % kRingS) * kScanSlotBytes;
-      const uint32_t dst = sb + b * kSlotStride;
-      mbar_arrive_expect_tx(&B.full[b], kSlotLoadBytes);
-#pragma unroll 1
-      for (int k = 0; k < 3; ++k) bulk_load_g2s(dst + 16384 * k, src + 16384 * k, 16384, &B.full[b]);
-      bulk_load_g2s(dst + SL_P, src + SL_P, kSlotLoadBytes - SL_P, &B.full[b]);
-      nfull = c + 1;
-    }
+    mbar_arrive_expect_tx(&B.fullC[b], SL_SCAL - SL_K);
+    bulk_load_g2s(dst + SL_K, src + SL_K, SL_SCAL - SL_K, &B.fullC[b]);
+    nC = c + 1;
     if (c >= 2) {
       ok = mbar_wait(&B.ysempty[b], par(phE, b), kWait);
       phE ^= 1u << b;
@@ -1068,8 +1130,12 @@ __device__ void chain_loader(const ScanParams& P, uint32_t sb, int item, const C
     // copies still landing get a short bounded chance before the CTA may exit:
     // the last chunk issued into each buffer completes that buffer's phase
     // (chunk index / 2) % 2
-    for (int c = nfull - 2 < 0 ? 0 : nfull - 2; c < nfull; ++c)
-      mbar_wait(&B.full[c & 1], (uint32_t)(c >> 1) & 1u, kDrain);
+    for (int c = nA - 2 < 0 ? 0 : nA - 2; c < nA; ++c)
+      mbar_wait(&B.fullA[c & 1], (uint32_t)(c >> 1) & 1u, kDrain);
+    for (int c = nB - 2 < 0 ? 0 : nB - 2; c < nB; ++c)
+      mbar_wait(&B.fullB[c & 1], (uint32_t)(c >> 1) & 1u, kDrain);
+    for (int c = nC - 2 < 0 ? 0 : nC - 2; c < nC; ++c)
+      mbar_wait(&B.fullC[c & 1], (uint32_t)(c >> 1) & 1u, kDrain);
     for (int c = ngs - 2 < 0 ? 0 : ngs - 2; c < ngs; ++c)
       mbar_wait(&B.gfull[c & 1], (uint32_t)(c >> 1) & 1u, kDrain);
   }
@@ -1173,14 +1239,14 @@ __global__ void __launch_bounds__(kCta, 1)
   if (bx < p.items) {
     // ---- chain CTA ----
     uint64_t* bars = reinterpret_cast<uint64_t*>(gb + C_BAR);
-    ChainBars B{bars, bars + 2, bars + 3, bars + 4, bars + 6, bars + 8, bars + 10, bars + 11,
-                bars + 12};
+    ChainBars B{bars,      bars + 2,  bars + 3,  bars + 4,  bars + 6,  bars + 8, bars + 10,
+                bars + 11, bars + 12, bars + 14, bars + 16, bars + 18, bars + 20};
     if (tid < kD) reinterpret_cast<float*>(gb + C_WN)[tid] = 1.f + a_norm_w_or_zero(p.a, tid);
     if (tid == 32 * kLoadWarp && p.has_tiles && p.a.g != nullptr) prefetch_tmap(&p.tg);
-    uint32_t* tslot = reinterpret_cast<uint32_t*>(gb + C_BAR + 112);
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(gb + C_BAR + 176);
     if (warp == 0) tmem_alloc(tslot, 512);
     if (tid == 0) {
-      for (int k = 0; k < 14; ++k) {
+      for (int k = 0; k < 22; ++k) {
         // ysfull, sready, dready count the compute threads, ysempty the
         // epilogue threads, the others one arrival (commit, copy, control)
         const uint32_t cnt = (k == 6 || k == 7 || k == 10 || k == 11)
