@@ -126,8 +126,9 @@ gdn_status gdn_chunk_fwd_path(
 /*
  * gdn_chunk_fwd_workspace_size -- bytes of device workspace that
  * gdn_chunk_fwd_ws can use for a batch of n_seq sequences x H_v value heads.
- * Up to 64 items: the split layout (a ring of four 80.25 KB hand-off slots
- * plus 64 bytes of flags per item).  More than 64 items and at most 1024
+ * Up to 64 items: the split layout (per item a ring of eight 73,984-byte
+ * hand-off slots and 128 bytes of flags, the flag block rounded up to 256
+ * bytes; 28,416,000 bytes for 48 items).  More than 64 items and at most 1024
  * sequences: n_seq int32 (rounded up to 256 bytes) for the order in which
  * the one-CTA layout takes the sequences, longest first, so that long
  * sequences do not start last.  Returns 0 when neither applies: not bf16
