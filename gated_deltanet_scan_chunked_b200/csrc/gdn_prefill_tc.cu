@@ -963,26 +963,15 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
 // TMEM (MMA A operands), and runs [Delta | Y] = S^T [-W; gamma Q^]^T,
 // Delta += U, the state update, Y += Delta P^T and the epilogue.
 //
-// Cluster launch (kGlobal = false): one 2- or 3-CTA cluster per item; the
-// tiles go over distributed shared memory with bulk copies (shared::cta ->
-// shared::cluster, no multicast), double-buffered.  "full" barriers in the
-// chain CTA (arrive + expected bytes, completed by the copies), "empty"
-// barriers in the preparation CTA (arrived by the chain CTA once its MMAs
-// have read a buffer), "staging free" barriers in the preparation CTA
-// (arrived once a copy has landed, so its source may be overwritten).
-//
-// Split launch (kGlobal = true, needs a caller workspace): the same roles
-// without a cluster, in one cooperative launch of items chain CTAs followed
-// by NPREP preparation CTAs per item, placed anywhere (clusters of 3 cannot
-// all be placed at once on 148 SMs; single CTAs can).  Per item a ring of
-// kRing slots in the workspace (L2-resident) carries the tiles plus the
-// chunk's gate factors (1 + w) sigmoid(g), 80 KB: the preparation CTA
-// bulk-stores them (shared::cta -> global) and, once the stores are
-// complete, publishes the slot with a release flag; a non-MMA thread of the
-// chain CTA acquires the flag and bulk-loads the slot into shared memory a
-// chunk ahead, then returns the slot with a relaxed flag store once its bytes
-// have landed.  Flags hold chunk index + 1 and start at zero.  Every wait is
-// bounded.
+// One 2- or 3-CTA cluster per item; the tiles go over distributed shared
+// memory with bulk copies (shared::cta -> shared::cluster, no multicast),
+// double-buffered.  "full" barriers in the chain CTA (arrive + expected
+// bytes, completed by the copies), "empty" barriers in the preparation CTA
+// (arrived by the chain CTA once its MMAs have read a buffer), "staging
+// free" barriers in the preparation CTA (arrived once a copy has landed, so
+// its source may be overwritten).  Every wait is bounded.  (The workspace
+// form of these roles, without a cluster, is the scan layout in
+// gdn_prefill_scan.cu.)
 // ============================================================================
 
 // chain CTA (rank 0) shared memory
@@ -990,8 +979,8 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_kernel(const PrefillArg
 // -W, rows 64-127 gamma Q^: one N = 128 MMA gives [Delta^T | Y^T]); P; T diag(b)
 constexpr uint32_t SH_KT = 0, SH_WQ = 16384, SH_P = 49152, SH_TB = 57344;
 constexpr uint32_t kShipBytes = 65536;
-constexpr uint32_t C_SHIP = 0;            // 2 ship buffers; then V raw -> fp16, S^T fp16,
-                                          // Delta^T fp16, g (cluster launch): see the kernel
+constexpr uint32_t C_SHIP = 0;            // 2 ship buffers; then V raw -> fp16, the output
+                                          // staging tile and g: see the kernel
 constexpr uint32_t C_SCAL = 229376;       // shipped scalars [2][4]
 constexpr uint32_t C_RED = 229632;        // red[4][64], rr[64], max[16]
 constexpr uint32_t C_BAR = 231040;        // full[2], mma, tmem slot
@@ -1010,45 +999,25 @@ constexpr uint32_t P_SCAL = 227840;       // scalar staging [2][4]
 constexpr uint32_t P_MAX = 227872;        // block-max scratch [16]
 constexpr uint32_t P_BAR = 227936;        // empty[2], mma, tmem slot, staging free[2]
 constexpr uint32_t kPairSmemBytes = 231072 + 1024;  // the chain CTA's map is the larger
-// split launch: global ring per item
-constexpr int kRing = 4;
-// slot: tiles (64 KB), gate factors (1 + w) sigmoid(g) fp16 [64][128] (16 KB),
-// scalars [4] fp32 (16 B), padding to a multiple of 256
-constexpr uint32_t kSlotGF = kShipBytes;
-constexpr uint32_t kSlotLoad = kShipBytes + 16384;  // bytes of tiles + gate factors
-constexpr size_t kSlotBytes = kSlotLoad + 256;
 
-template <int NPREP, bool kGlobal>
+template <int NPREP>
 __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const PrefillArgs a) {
   // chain CTA map: 2 ship buffers (64 KB of tiles each), V, the output
-  // staging tile, and gate-factor buffers (cluster launch: 2 for g,
-  // converted in place; split launch: a ring of 3 that the slot loads fill
-  // directly); then C_SCAL / C_RED / C_BAR at fixed offsets.
-  // TMEM (512 columns): S^T fp32 0-127, [Delta^T | Y^T] 128-255, the fp16 MMA
-  // A operands S^T 2^-e (256-319) and Delta^T 2^-e (320-351), and (split
-  // launch) a second [Delta^T | Y^T] 384-511 for odd chunks: the split launch
-  // runs chunk c's epilogue during chunk c+1's MMAs.
+  // staging tile, and 2 buffers for g (converted in place to the gate
+  // factors); then C_SCAL / C_RED / C_BAR at fixed offsets.
+  // TMEM (512 columns): S^T fp32 0-127, [Delta^T | Y^T] 128-255, and the fp16
+  // MMA A operands S^T 2^-e (256-319) and Delta^T 2^-e (320-351).
   constexpr uint32_t kShipStride = kShipBytes;
   constexpr uint32_t X_VT = C_SHIP + 2 * kShipStride;
   constexpr uint32_t X_DT = X_VT + 16384;  // output staging (16 KB)
   constexpr uint32_t X_GS = X_DT + 16384;
-  static_assert(X_GS + 3 * 16384 <= C_SCAL, "chain shared-memory map overlaps");
+  static_assert(X_GS + 2 * 16384 <= C_SCAL, "chain shared-memory map overlaps");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sb = (raw + 1023u) & ~1023u;
   uint8_t* gb = smem_raw + (sb - raw);
-  uint32_t rank;
-  int item;
-  if constexpr (kGlobal) {
-    // [0, items): chain CTAs; then NPREP preparation CTAs per item
-    const int items = a.n_seq * a.H_v;
-    const int bx = (int)blockIdx.x;
-    rank = bx < items ? 0u : 1u + (uint32_t)((bx - items) % NPREP);
-    item = bx < items ? bx : (bx - items) / NPREP;
-  } else {
-    rank = cluster_ctarank();
-    item = blockIdx.x / (1 + NPREP);
-  }
+  const uint32_t rank = cluster_ctarank();
+  const int item = blockIdx.x / (1 + NPREP);
   const int seq = item / a.H_v;
   const int h = item % a.H_v;
   const int hq = h / (a.H_v / a.H_qk);
@@ -1080,15 +1049,6 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
   const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
   uint32_t phase = 0;
   bool ok = true;
-  // this item's ring of slots and its flags (split launch only)
-  uint8_t* ring = nullptr;
-  unsigned long long* ready = nullptr;
-  unsigned long long* consumed = nullptr;
-  if constexpr (kGlobal) {
-    ring = static_cast<uint8_t*>(a.ring) + (size_t)item * kRing * kSlotBytes;
-    ready = a.ring_flags + (size_t)item * 2 * kRing;
-    consumed = ready + kRing;
-  }
 
   if (rank == 0) {
     // =========================== chain CTA ===========================
@@ -1106,7 +1066,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
     if (t_begin < t_end) {
       const int n0 = (t_end - t_begin) < kC ? (int)(t_end - t_begin) : kC;
       ld.v(t_begin, n0);
-      if (!kGlobal && has_g) ld.g(t_begin, n0, 0);
+      if (has_g) ld.g(t_begin, n0, 0);
     }
     cp_async_commit();
     if (warp == 0) tmem_alloc(tslot, 512);
@@ -1118,45 +1078,13 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
     }
     fence_before_sync();
     __syncthreads();
-    if constexpr (!kGlobal) cluster_sync();
+    cluster_sync();
     fence_after_sync();
     const uint32_t tbase = *tslot;
     const uint32_t tS = tbase + lane_off;
     const uint32_t tSA = tbase + lane_off + 256, tDA = tbase + lane_off + 320;
-    // TMEM column of chunk c's [Delta^T | Y^T]
-    auto dy_col = [](int c) -> uint32_t { return (kGlobal && (c & 1)) ? 384u : 128u; };
-    // Split launch, thread kFetcher only (not the MMA issuer: its proxy
-    // fence would wait for the MMAs in flight): issue the bulk load of chunk
-    // c from its slot into buffer c & 1 (free: it held chunk c - 2, whose
-    // MMAs are complete).  `block` waits (bounded) for the slot's flag;
-    // otherwise a slot not yet published is left for a later call.  Loads
-    // are issued in chunk order; `fetched` counts them.
-    constexpr int kFetcher = 32;
-    int fetched = 0;
-    auto fetch = [&](int c, bool block) -> bool {
-      if (fetched > c) return true;
-      const int s = c % kRing;
-      const unsigned long long want = (unsigned long long)c + 1;
-      if (block) {
-        if (!wait_flag_ge(&ready[s], want, kWaitLimit)) return false;
-      } else if (ld_acquire_u64(&ready[s]) < want) {
-        return true;
-      }
-      fence_proxy_async_global();
-      const int bb = c & 1;
-      const uint8_t* src = ring + (size_t)s * kSlotBytes;
-      mbar_arrive_expect_tx(&full[bb], kSlotLoad + 16);
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        bulk_load_g2s(sb + C_SHIP + bb * kShipStride + 16384 * k, src + 16384 * k, 16384,
-                      &full[bb]);
-      // gate factors into ring entry c % 3 (last read by the epilogue of
-      // chunk c - 3, which ran during chunk c - 2)
-      bulk_load_g2s(sb + X_GS + (c % 3) * 16384, src + kSlotGF, 16384, &full[bb]);
-      bulk_load_g2s(sb + C_SCAL + 16 * bb, src + kSlotLoad, 16, &full[bb]);
-      ++fetched;
-      return true;
-    };
+    // TMEM column of [Delta^T | Y^T]
+    constexpr uint32_t kDY = 128;
     {
       float v[32];
 #pragma unroll
@@ -1243,11 +1171,6 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
         }
       }
     };
-    // split launch: the previous chunk, whose epilogue runs in this chunk's
-    // MMA windows
-    int64_t p_c0 = 0;
-    int p_n = 0, p_e = 0;
-
     int ci = 0;
     for (int64_t c0 = t_begin; c0 < t_end; c0 += kC, ++ci) {
       const int n = (t_end - c0) < kC ? (int)(t_end - c0) : kC;
@@ -1255,37 +1178,21 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
       const int nn = has_next ? ((t_end - c0 - kC) < kC ? (int)(t_end - c0 - kC) : kC) : 0;
       const int b = ci & 1;
       const uint32_t ship = sb + C_SHIP + b * kShipStride;
-      // this chunk's gate factors: shipped (split launch: ring entry ci % 3)
-      // or computed here from g in place (cluster launch: buffer b)
-      const uint32_t gsb = kGlobal ? sb + X_GS + (ci % 3) * 16384 : sb + X_GS + b * 16384;
+      // this chunk's gate factors, computed here from g in place (buffer b)
+      const uint32_t gsb = sb + X_GS + b * 16384;
       cp_async_wait_all();
       // the other g buffer was last read by the previous chunk's epilogue
-      if (!kGlobal && has_next && has_g) ld.g(c0 + kC, nn, b ^ 1);
+      if (has_next && has_g) ld.g(c0 + kC, nn, b ^ 1);
       cp_async_commit();
       bool okw = true;
-      if constexpr (kGlobal) {
-        if (tid == kFetcher) okw = fetch(ci, true);
-        if (!__syncthreads_and(okw)) { ok = false; break; }
-      } else {
-        __syncthreads();
-      }
+      __syncthreads();
       GDN_TRACE_POINT(0);
-      if constexpr (kGlobal) okw = mbar_wait(&full[b], (ci >> 1) & 1, kWaitLimit);
-      else okw = mbar_wait_cluster(&full[b], (ci >> 1) & 1, kWaitLimit);
+      okw = mbar_wait_cluster(&full[b], (ci >> 1) & 1, kWaitLimit);
       if (!__syncthreads_and(okw)) { ok = false; break; }
-      if constexpr (kGlobal) {
-        // Chunk ci's bytes are in shared memory: hand its slot back.  The
-        // bulk reads of the slot are complete (the barrier phase above), so
-        // a relaxed store suffices: nothing this thread did afterwards needs
-        // to be visible to the preparation CTA, and a release here would
-        // first drain this thread's outstanding y stores.
-        if (tid == 0) st_relaxed_u64(&consumed[ci % kRing], (unsigned long long)ci + 1);
-      } else {
-        // the copy has landed: its source staging buffer may be reused
-        if (tid == 0)
-          mbar_remote_arrive(
-              mapa_shared(sb + P_BAR + 32 + 8 * ((ci / NPREP) & 1), 1 + ci % NPREP));
-      }
+      // the copy has landed: its source staging buffer may be reused
+      if (tid == 0)
+        mbar_remote_arrive(
+            mapa_shared(sb + P_BAR + 32 + 8 * ((ci / NPREP) & 1), 1 + ci % NPREP));
       GDN_TRACE_POINT(1);
       const float gC = sScal[b * 4 + 0];
       const int f = (int)sScal[b * 4 + 1];
@@ -1346,23 +1253,17 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t db = sdesc(ship + SH_WQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-          mma_f16_ta(tbase + dy_col(ci), tbase + 256 + kk * 8, db, ID_KK128, kk > 0);
+          mma_f16_ta(tbase + kDY, tbase + 256 + kk * 8, db, ID_KK128, kk > 0);
         }
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint64_t da = sdesc(sb + X_VT + kk * 2048, 8192, 1024);
           const uint64_t db = sdesc(ship + SH_TB + kk * 32, 16, 1024);
-          mma_f16(tbase + dy_col(ci), da, db, ID_MK, 1);
+          mma_f16(tbase + kDY, da, db, ID_MK, 1);
         }
         mma_commit(mbar);
       }
-      if constexpr (kGlobal) {
-        // the next chunk's tiles, while the MMAs run
-        if (tid == kFetcher && has_next) fetch(ci + 1, false);
-        // and part (A) of the previous chunk's epilogue
-        if (ci > 0) epi_a(tbase + lane_off + dy_col(ci - 1) + 64, p_e);
-      }
-      if (!kGlobal && has_g && tid >= 64) {
+      if (has_g && tid >= 64) {
         // Also while the MMAs run: this chunk's gate factors (1 + w)
         // sigmoid(g), in place as fp16 (g landed before the loop-top
         // barrier).  Warps 2-7 only: warp 0 issues the MMAs, warp 1 fetches.
@@ -1391,7 +1292,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
       // Delta^T 2^-e -> fp16 A operand in TMEM (token pairs per column)
       {
         float v[32];
-        tmem_ld32(tbase + lane_off + dy_col(ci) + half * 32, v);
+        tmem_ld32(tbase + lane_off + kDY + half * 32, v);
         tmem_wait_ld();
         const float sf = ldexpf(1.f, f);
         uint32_t pk[16];
@@ -1415,49 +1316,27 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint64_t db = sdesc(ship + SH_P + kk * 32, 16, 1024);
-          mma_f16_ta(tbase + dy_col(ci) + 64, tbase + 320 + kk * 8, db, ID_KK, 1);
+          mma_f16_ta(tbase + kDY + 64, tbase + 320 + kk * 8, db, ID_KK, 1);
         }
         mma_commit(mbar);
-      }
-      if constexpr (kGlobal) {
-        // part (B) of the previous chunk's epilogue, while the MMAs run
-        if (ci > 0) epi_b(p_c0, p_n, sb + X_GS + ((ci - 1) % 3) * 16384);
       }
       okw = mbar_wait(mbar, phase, kWaitLimit);
       phase ^= 1;
       if (!__syncthreads_and(okw)) { ok = false; break; }
       fence_after_sync();
       // this chunk's shipped tiles are no longer read: hand the buffer back
-      if constexpr (kGlobal) {
-        if (tid == kFetcher && has_next) fetch(ci + 1, false);
-      } else {
-        if (tid == 0) mbar_remote_arrive(mapa_shared(sb + P_BAR + 8 * b, 1 + ci % NPREP));
-      }
+      if (tid == 0) mbar_remote_arrive(mapa_shared(sb + P_BAR + 8 * b, 1 + ci % NPREP));
       GDN_TRACE_POINT(5);
 
-      if constexpr (kGlobal) {
-        p_c0 = c0;
-        p_n = n;
-        p_e = e;
-      } else {
-        // epilogue now (its gate factors were converted in place, buffer b)
-        epi_a(tbase + lane_off + 128 + 64, e);
-        __syncthreads();
-        epi_b(c0, n, gsb);
-        __syncthreads();  // staging reads done: g buffer and staging tile reusable
-      }
+      // epilogue now (its gate factors were converted in place, buffer b)
+      epi_a(tbase + lane_off + kDY + 64, e);
+      __syncthreads();
+      epi_b(c0, n, gsb);
+      __syncthreads();  // staging reads done: g buffer and staging tile reusable
       fence_before_sync();
       GDN_TRACE_POINT(6);
     }
     cp_async_wait_all();
-    if constexpr (kGlobal) {
-      // the last chunk's epilogue
-      if (ok && ci > 0) {
-        epi_a(tbase + lane_off + dy_col(ci - 1) + 64, p_e);
-        __syncthreads();
-        epi_b(p_c0, p_n, sb + X_GS + ((ci - 1) % 3) * 16384);
-      }
-    }
     if (ok) {
       if (a.final_state) {
         const float sc = ldexpf(1.f, s_exp);
@@ -1475,18 +1354,13 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
     } else {
       if (tid == 0) atomicOr(a.err, kErrTimeout);
       mbar_wait(mbar, phase ^ 1, kWaitLimit);
-      // copies into this CTA's buffers that may still be landing
-      if constexpr (kGlobal) {
-        if (tid == 0)
-          for (int c = ci; c < fetched; ++c) mbar_wait(&full[c & 1], (c >> 1) & 1, kWaitLimit);
-      } else {
-        if (t_begin + (int64_t)(ci + 1) * kC < t_end)
-          mbar_wait_cluster(&full[(ci + 1) & 1], ((ci + 1) >> 1) & 1, kWaitLimit >> 6);
-      }
+      // a copy into this CTA's buffers that may still be landing
+      if (t_begin + (int64_t)(ci + 1) * kC < t_end)
+        mbar_wait_cluster(&full[(ci + 1) & 1], ((ci + 1) >> 1) & 1, kWaitLimit >> 6);
     }
     fence_before_sync();
     __syncthreads();
-    if constexpr (!kGlobal) cluster_sync();
+    cluster_sync();
     if (warp == 0) tmem_dealloc(tbase, 512);
   } else {
     // =========================== prep CTA ============================
@@ -1526,65 +1400,14 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
     }
     fence_before_sync();
     __syncthreads();
-    if constexpr (!kGlobal) cluster_sync();
+    cluster_sync();
     fence_after_sync();
     const uint32_t tbase = *tslot;
     const uint32_t tKQ = tbase + lane_off, tW = tbase + lane_off;
-    uint32_t full_cl0 = 0, ship_cl0 = 0, scal_cl0 = 0;
-    if constexpr (!kGlobal) {
-      full_cl0 = mapa_shared(sb + C_BAR, 0);
-      ship_cl0 = mapa_shared(sb + C_SHIP, 0);
-      scal_cl0 = mapa_shared(sb + C_SCAL, 0);
-    }
+    const uint32_t full_cl0 = mapa_shared(sb + C_BAR, 0);
+    const uint32_t ship_cl0 = mapa_shared(sb + C_SHIP, 0);
+    const uint32_t scal_cl0 = mapa_shared(sb + C_SCAL, 0);
 
-    // Split launch: this CTA also computes the chunk's gate factors
-    // (1 + w) sigmoid(g) and stores them into the slot; thread (r, c) of
-    // piece index tid + 256 k handles token row (tid / 16) + 16 k, columns
-    // 8 (tid % 16) .. + 7.
-    float wv[8];
-#pragma unroll
-    for (int j2 = 0; j2 < 8; ++j2)
-      wv[j2] = 1.f + ((has_g && a.norm_w) ? __ldg(a.norm_w + (tid & 15) * 8 + j2) : 0.f);
-    const __nv_bfloat16* Gh = static_cast<const __nv_bfloat16*>(a.g);
-    uint4 graw[4];  // this thread's g pieces of the chunk (bf16 x 8)
-    // Split launch: thread kShip (warp 2: it issues no MMAs -- a release or
-    // proxy fence on the MMA issuer waits for its MMAs -- and is idle in the
-    // windows used) does all the slot traffic: it issues the bulk stores,
-    // waits for them and publishes the slot.
-    constexpr int kShip = 64;
-    // Split launch, thread kShip: the slot whose bulk stores are in flight and
-    // not yet published (published once complete, during the next chunk).
-    int pend_slot = -1;
-    unsigned long long pend_val = 0;
-    auto publish = [&]() {
-      if (pend_slot >= 0) {
-        bulk_wait_all();
-        // the stores are complete; publish them to the chain CTA
-        fence_proxy_async_global();
-        st_release_u64(&ready[pend_slot], pend_val);
-        pend_slot = -1;
-      }
-    };
-    // Split launch, thread kShip: a slot whose bulk stores are staged but not
-    // yet issued.  They are issued right after the next loop-top barrier:
-    // issued earlier, the loop-top proxy fence would wait for their reads.
-    int iss_slot = -1, iss_lb = 0;
-    unsigned long long iss_val = 0;
-    auto issue = [&]() {
-      if (iss_slot >= 0) {
-        uint8_t* dst = ring + (size_t)iss_slot * kSlotBytes;
-        const uint32_t src = sb + P_STG + iss_lb * kShipBytes;
-        fence_proxy_async_global();
-#pragma unroll
-        for (int k = 0; k < 4; ++k) bulk_store_s2g(dst + 16384 * k, src + 16384 * k, 16384);
-        if (has_g) bulk_store_s2g(dst + kSlotGF, sb + P_A, 16384);
-        bulk_store_s2g(dst + kSlotLoad, sb + P_SCAL + 16 * iss_lb, 16);
-        bulk_commit();
-        pend_slot = iss_slot;
-        pend_val = iss_val;
-        iss_slot = -1;
-      }
-    };
     int ci = first, lc = 0;  // chunk index, local count
     for (int64_t c0 = c_first; c0 < t_end; c0 += (int64_t)kC * NPREP, ci += NPREP, ++lc) {
       const int n = (t_end - c0) < kC ? (int)(t_end - c0) : kC;
@@ -1597,29 +1420,12 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
       cp_async_wait_all();
       fence_proxy_async();  // the raw [K; Q] tile is read by MMA0 below
       bool okw = true;
-      if constexpr (!kGlobal) {
-        // staging buffer lb was the source of the copy two local chunks ago;
-        // the chain CTA reports when that copy has landed.  (The split
-        // launch waits for its stores to complete when it issues them.)
-        if (tid == 0 && lc >= 2)
-          okw = mbar_wait_cluster(&stg_free[lb], ((lc - 2) >> 1) & 1, kWaitLimit);
-      }
+      // staging buffer lb was the source of the copy two local chunks ago;
+      // the chain CTA reports when that copy has landed
+      if (tid == 0 && lc >= 2)
+        okw = mbar_wait_cluster(&stg_free[lb], ((lc - 2) >> 1) & 1, kWaitLimit);
       if (!__syncthreads_and(okw)) { ok = false; break; }
-      if constexpr (kGlobal) {
-        if (tid == kShip) issue();  // the previous chunk's slot
-      }
       GDN_TRACE_POINT(20);
-
-      if constexpr (kGlobal) {
-        // g of this chunk into L2 now; it is read after the W product
-        if (has_g) {
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int rr = (tid >> 4) + 16 * k;
-            if (rr < n) prefetch_l2(Gh + ((size_t)(c0 + rr) * a.H_v + h) * kD + (tid & 15) * 8);
-          }
-        }
-      }
 
       // [K; Q] K^T on the raw inputs, overlapped with the gates and norms
       if (tid == 0) {
@@ -1699,11 +1505,6 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
       }
       fence_proxy_async();
       fence_before_sync();
-      // split launch: the last bulk store has finished reading its sources
-      // before the A scratch (its gate-factor staging) is rewritten below
-      if constexpr (kGlobal) {
-        if (tid == kShip) bulk_wait_read_all();
-      }
       okw = mbar_wait(mbar, phase, kWaitLimit);
       phase ^= 1;
       if (!__syncthreads_and(okw)) { ok = false; break; }
@@ -1811,22 +1612,6 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
         }
         mma_commit(mbar);
       }
-      if constexpr (kGlobal) {
-        // the previous chunk's slot (its stores are long complete), while
-        // the MMAs run; a first chunk is published as soon as it is stored
-        if (tid == kShip) publish();
-      }
-      if constexpr (kGlobal) {
-        // this chunk's g rows (from L2) while the MMAs run
-        if (has_g) {
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int rr = (tid >> 4) + 16 * k;
-            graw[k] = rr < n ? ld_nc_v4(Gh + ((size_t)(c0 + rr) * a.H_v + h) * kD + (tid & 15) * 8)
-                             : make_uint4(0u, 0u, 0u, 0u);
-          }
-        }
-      }
       okw = mbar_wait(mbar, phase, kWaitLimit);
       phase ^= 1;
       if (!__syncthreads_and(okw)) { ok = false; break; }
@@ -1853,44 +1638,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
 
       // ship this chunk's tiles once the chain CTA has released buffer b
       okw = true;
-      if constexpr (kGlobal) {
-        // slot ci % kRing last held chunk ci - kRing: the chain CTA must
-        // have loaded it
-        const int s = ci % kRing;
-        if (tid == 0 && ci >= kRing)
-          okw = wait_flag_ge(&consumed[s], (unsigned long long)(ci - kRing) + 1, kWaitLimit);
-        if (has_g) {
-          // meanwhile (the other threads), the gate factors (1 + w) sigmoid(g),
-          // token-major [64][128] fp16, staged in the A scratch (dead since
-          // the W product) and shipped with the tiles
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int rr = (tid >> 4) + 16 * k;
-            float gf[8];
-            unpack_bf16x8(graw[k], gf);
-            uint32_t o[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              o[q] = pack_f16(__fdividef(wv[2 * q], 1.f + __expf(-gf[2 * q])),
-                              __fdividef(wv[2 * q + 1], 1.f + __expf(-gf[2 * q + 1])));
-            st_shared_v4(sb + P_A + rr * 256 + (tid & 15) * 16, o[0], o[1], o[2], o[3]);
-          }
-          fence_proxy_async();
-        }
-        if (!__syncthreads_and(okw)) { ok = false; break; }
-        GDN_TRACE_POINT(30);
-        if (tid == kShip) {
-          iss_slot = s;
-          iss_lb = lb;
-          iss_val = (unsigned long long)ci + 1;
-          if (lc == 0) {
-            // the first chunk is shipped and published at once
-            issue();
-            publish();
-          }
-        }
-        GDN_TRACE_POINT(31);
-      } else if (tid == 0) {
+      if (tid == 0) {
         okw = mbar_wait_cluster(&empty[b], ((ci >> 1) & 1) ^ 1, kWaitLimit);
         if (okw) {
           // the cluster window keeps the peer's layout: offsets carry over
@@ -1907,26 +1655,18 @@ __global__ void __launch_bounds__(kNT, 1) gdn_prefill_tc_pair_kernel(const Prefi
       GDN_TRACE_POINT(27);
     }
     cp_async_wait_all();
-    if constexpr (kGlobal) {
-      if (tid == kShip && ok) {
-        publish();
-        issue();
-        publish();
-      }
-      if (tid == kShip) bulk_wait_all();
-    }
     if (!ok) {
       if (tid == 0) atomicOr(a.err, kErrTimeout);
       mbar_wait(mbar, phase ^ 1, kWaitLimit);
     }
     fence_before_sync();
     __syncthreads();
-    if constexpr (!kGlobal) cluster_sync();
+    cluster_sync();
     if (warp == 0) tmem_dealloc(tbase, 128);
   }
 }
 
-// Larger batches (more than kSplitMaxItems items, at most kMaxOrderSeqs
+// Larger batches (more than kScanMaxItems items, at most kMaxOrderSeqs
 // sequences) with a workspace: the one-CTA layout takes the sequences
 // longest first.
 constexpr int kMaxOrderSeqs = 1024;
@@ -2011,8 +1751,8 @@ gdn_status launch_prefill_tc(const PrefillArgs& a, cudaStream_t stream) {
   auto fits = [&](int np) -> bool {
     if (dev < 0 || dev >= 64) return false;
     if (max_clusters[dev][np - 1] == 0) {
-      const void* fn = np == 2 ? (const void*)gdn_prefill_tc_pair_kernel<2, false>
-                               : (const void*)gdn_prefill_tc_pair_kernel<1, false>;
+      const void* fn = np == 2 ? (const void*)gdn_prefill_tc_pair_kernel<2>
+                               : (const void*)gdn_prefill_tc_pair_kernel<1>;
       if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)kPairSmemBytes) != cudaSuccess)
         return false;
@@ -2038,8 +1778,8 @@ gdn_status launch_prefill_tc(const PrefillArgs& a, cudaStream_t stream) {
   if (a.tc_variant == 1) nprep = fits(2) ? 2 : 1;
   else if (a.tc_variant == 0) nprep = fits(2) ? 2 : (fits(1) ? 1 : 0);
   if (nprep > 0) {
-    const void* fn = nprep == 2 ? (const void*)gdn_prefill_tc_pair_kernel<2, false>
-                                : (const void*)gdn_prefill_tc_pair_kernel<1, false>;
+    const void* fn = nprep == 2 ? (const void*)gdn_prefill_tc_pair_kernel<2>
+                                : (const void*)gdn_prefill_tc_pair_kernel<1>;
     if (dev < 0 || dev >= 64 || !pair_attr_set[dev][nprep - 1]) {
       if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)kPairSmemBytes) != cudaSuccess)
@@ -2058,8 +1798,8 @@ gdn_status launch_prefill_tc(const PrefillArgs& a, cudaStream_t stream) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t err = nprep == 2 ? cudaLaunchKernelEx(&cfg, gdn_prefill_tc_pair_kernel<2, false>, a)
-                                 : cudaLaunchKernelEx(&cfg, gdn_prefill_tc_pair_kernel<1, false>, a);
+    cudaError_t err = nprep == 2 ? cudaLaunchKernelEx(&cfg, gdn_prefill_tc_pair_kernel<2>, a)
+                                 : cudaLaunchKernelEx(&cfg, gdn_prefill_tc_pair_kernel<1>, a);
     if (err != cudaSuccess) return GDN_ERR_CUDA;
   } else {
     if (a.seq_order != nullptr) {
