@@ -14,7 +14,7 @@ namespace {
 __device__ unsigned long long g_never_set = 0;
 
 // One CTA waits on g_never_set with the library's bounded wait (the one the
-// split prefill uses for its hand-off flags), gives up after `iters` polls,
+// scan-layout prefill uses for its hand-off flags), gives up after `iters` polls,
 // records the timeout in the error word and returns.
 __global__ void selftest_wait_kernel(int* err, uint32_t iters) {
   if (threadIdx.x != 0) return;

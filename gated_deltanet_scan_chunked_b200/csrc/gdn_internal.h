@@ -35,9 +35,9 @@ struct PrefillArgs {
   int32_t l2norm;
   float eps_l2, eps_norm, scale;
   int* err;                // device error word
-  int tc_variant;          // tensor kernel: 0 auto, 1 CTA pairs, 2 one CTA per head, 3 split
-  // Split-launch workspace (nullptr: none): hand-off ring slots and their
-  // flags, laid out by prefill_tc_workspace_bytes.
+  int tc_variant;          // tensor kernel: 0 auto, 1 CTA pairs, 2 one CTA per head, 3 scan layout
+  // Scan-layout workspace (nullptr: none): hand-off ring slots and their
+  // flags, placed by prefill_tc_workspace_layout (sizes: scan_ws_bytes).
   void* ring = nullptr;
   unsigned long long* ring_flags = nullptr;
   // Larger batches with a workspace: the order in which the one-CTA layout
@@ -192,9 +192,10 @@ gdn_status launch_decode(const DecodeArgs& a, cudaStream_t stream);
 gdn_status launch_prefill_simt(const PrefillArgs& a, cudaStream_t stream);
 gdn_status launch_prefill_tc(const PrefillArgs& a, cudaStream_t stream);
 bool prefill_tc_supports(const PrefillArgs& a);
-// Workspace bytes the split launch of the tensor kernel needs for n_seq x H_v
-// items (0 when it can never apply), and the placement of its parts within a
-// 256-byte aligned workspace.
+// Workspace bytes the tensor kernel can use for n_seq x H_v items (the scan
+// layout's ring for small batches, the one-CTA layout's sequence order for
+// larger ones; 0 when neither applies), and the placement of its parts
+// within a 256-byte aligned workspace.
 size_t prefill_tc_workspace_bytes(int32_t n_seq, int32_t H_v, int32_t d_k, int32_t d_v,
                                   gdn_dtype dtype);
 

@@ -1,4 +1,5 @@
-// gdn_chunk_fwd_static_ws: the split-layout prefill with its hand-off
+// gdn_chunk_fwd_static_ws: the split-layout prefill (GDN_PATH_TENSOR_SPLIT:
+// the scan layout of gdn_prefill_scan.cu) with its hand-off
 // workspace in a fixed device array of this library, for callers that cannot
 // hand the library any memory.  Nothing here allocates: the array is part of
 // the module image, its address comes from cudaGetSymbolAddress (looked up
@@ -14,7 +15,7 @@ namespace gdn {
 namespace {
 
 // Capacity: 48 (sequence, value head) items -- one sequence of a 48-value-head
-// layer -- sized from the split layout's own workspace formula.
+// layer -- sized from the scan layout's own workspace formula.
 constexpr int kStaticItems = 48;
 constexpr size_t kStaticBytes = scan_ws_bytes(kStaticItems);
 static_assert(kStaticItems <= kScanMaxItems, "static workspace holds a scan-layout batch");
@@ -56,7 +57,7 @@ extern "C" gdn_status gdn_chunk_fwd_static_ws(
     return GDN_ERR_UNSUPPORTED;
   void* ws = gdn::static_ws_ptr();
   if (ws == nullptr) return GDN_ERR_CUDA;
-  // the split launch clears the array's flags on `stream` before its kernel
+  // the scan launch clears the array's flags on `stream` before its kernel
   return gdn_chunk_fwd_ws(q, k, v, log_alpha, beta, g, norm_w, initial_state, cu_seqlens, n_seq,
                           total_T, H_qk, H_v, d_k, d_v, in_dtype, l2norm_qk, eps_l2, eps_norm,
                           scale, y, final_state, GDN_PATH_TENSOR_SPLIT, ws, gdn::kStaticBytes,
