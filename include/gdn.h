@@ -383,9 +383,15 @@ size_t gdn_gr_read_workspace_size(int64_t T, int32_t n_r, int32_t d, int32_t ran
  *   x               [T, d] bf16, written
  *   s               [T, n_r] fp32, written (pass to gdn_gr_write)
  *   workspace       256-byte aligned, gdn_gr_read_workspace_size bytes
- * The two router products run as bf16 GEMMs with fp32 accumulation through
- * cuBLASLt; the normalisation and the gated branch mean are this library's
- * kernels.
+ * The two router products run on this library's tcgen05 GEMM (bf16
+ * operands, fp32 accumulation in tensor memory, bf16 results; when its
+ * tile grid is small and K long, the first is split along K into fp32
+ * partials in the workspace that are summed in a fixed order, so results
+ * stay deterministic); the normalisation, the router
+ * activations and the gated branch mean are kernels of their own.  Five or
+ * six kernel launches (six when the first GEMM splits K), after two
+ * device-to-device copies and a memset that stack [W_d; W_w; 0] into the
+ * workspace, all on `stream`.
  */
 gdn_status gdn_gr_read(const uint8_t* codes, const float* scales, const float* gamma,
                        const void* W_d, const void* W_u, const void* W_w, int64_t T,
