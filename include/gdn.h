@@ -23,9 +23,10 @@
  * Conventions shared by every entry point:
  *   - All pointers are DEVICE pointers unless stated otherwise, dense and
  *     row-major, 16-byte aligned.  The caller owns every buffer; the library
- *     allocates no memory and never synchronises.  Work is enqueued on
- *     `stream` and runs asynchronously; a CUDA error raised by the kernel
- *     surfaces on the caller's next synchronisation.
+ *     allocates no memory and, apart from gdn_check_device_error, never
+ *     synchronises.  Work is enqueued on `stream` and runs asynchronously;
+ *     a CUDA error raised by the kernel surfaces on the caller's next
+ *     synchronisation.
  *   - Value head h reads QK head h / (H_v / H_qk) (contiguous groups);
  *     H_v % H_qk != 0 is GDN_ERR_INVALID_ARG.
  *   - The recurrent state of one head is S[i][j], i over d_k, j over d_v,
@@ -477,8 +478,9 @@ gdn_status gdn_check_device_error(gdn_stream_t stream);
 /*
  * gdn_selftest_bounded_wait -- exercises the failure path of the library's
  * bounded waits without a fault: one thread waits on a device flag that
- * nothing sets, with the same bounded poll the split prefill uses for its
- * hand-off flags, gives up after `iterations` polls (each ~32 ns apart),
+ * nothing sets, with the same bounded poll the split-layout prefill
+ * (GDN_PATH_TENSOR_SPLIT) uses for its hand-off flags, gives up after
+ * `iterations` polls (each ~32 ns apart),
  * records the timeout in the device error word and returns.  A following
  * gdn_check_device_error reports GDN_ERR_TIMEOUT once, and the context stays
  * usable.  (A test entry point; the pages have no counterpart.)
