@@ -103,9 +103,44 @@ def load_peaks():
                 source="fallback")
 
 
+def code_text(src):
+    """The code of a C/C++/CUDA source with its comments removed (string and
+    character literals kept as written), trailing blanks stripped and empty
+    lines dropped: two sources with the same code text differ only in
+    comments and blank lines."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        elif c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        else:
+            out.append(c)
+            i += 1
+    lines = (ln.rstrip() for ln in "".join(out).split("\n"))
+    return "\n".join(ln for ln in lines if ln)
+
+
+def code_sha(path):
+    """sha256[:16] of a source file's code text (comments do not count)."""
+    with open(path, encoding="utf-8") as f:
+        return hashlib.sha256(code_text(f.read()).encode()).hexdigest()[:16]
+
+
 def kernel_traffic(kernel_key):
-    """DRAM bytes per launch from the committed ncu summary, if the kernel
-    source it was taken on is unchanged; else None."""
+    """DRAM bytes per launch from the committed ncu summary, if the code of
+    the kernel source it was taken on is unchanged (comments may differ);
+    else None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
@@ -114,8 +149,11 @@ def kernel_traffic(kernel_key):
         if not d:
             return None
         src = os.path.join(ROOT, d["source"])
-        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-        return float(d["bytes_per_launch"]) if sha == d["source_sha"] else None
+        if "code_sha" in d:
+            same = code_sha(src) == d["code_sha"]
+        else:
+            same = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] == d["source_sha"]
+        return float(d["bytes_per_launch"]) if same else None
     except Exception:
         return None
 

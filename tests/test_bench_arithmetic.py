@@ -1,6 +1,7 @@
 """bench.py's roofline arithmetic (CPU): the counted FLOPs and algorithmic
 bytes per workload against the figures the workload definitions fix, written
-out here term by term, and the traffic registry's source-hash gate."""
+out here term by term, and the traffic registry's gate (a DRAM figure is
+reported only while the code it was captured on is unchanged)."""
 import hashlib
 import json
 
@@ -75,6 +76,28 @@ def test_traffic_registry_gate(tmp_path, monkeypatch):
     assert bench.kernel_traffic("k") == 1234.0
     assert bench.kernel_traffic("missing") is None
     src.write_text("kernel source, edited\n")   # changed since the capture: no figure
+    assert bench.kernel_traffic("k") is None
+
+
+def test_code_gate_ignores_comments_only(tmp_path, monkeypatch):
+    src = tmp_path / "k.cu"
+    src.write_text('// header\nint f(int x) { return x + 1; }  // tail\n'
+                   'const char* s = "// kept";\n/* block\n comment */ int g;\n')
+    (tmp_path / "profiles").mkdir()
+    reg = {"k": {"source": "k.cu", "source_sha": "0" * 16, "code_sha": bench.code_sha(str(src)),
+                 "bytes_per_launch": 99}}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(reg))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.kernel_traffic("k") == 99.0
+    # reworded and reflowed comments, blank lines: the same code
+    src.write_text('// a new header,\n// two lines long\n\nint f(int x) { return x + 1; }\n'
+                   'const char* s = "// kept";\n/* other */ int g;\n')
+    assert bench.kernel_traffic("k") == 99.0
+    # a string literal is code, even when it looks like a comment
+    src.write_text('int f(int x) { return x + 1; }\nconst char* s = "// edited";\nint g;\n')
+    assert bench.kernel_traffic("k") is None
+    # so is any other change
+    src.write_text('int f(int x) { return x + 2; }\nconst char* s = "// kept";\nint g;\n')
     assert bench.kernel_traffic("k") is None
 
 
