@@ -15,25 +15,31 @@
 // Only S depends on the previous chunk.  Per (sequence, value head) item the
 // work is split accordingly:
 //
-//   * four preparation sub-pipelines (two CTAs of two independent 8-warp
-//     halves) take the chunks in turn and do everything that does not need S:
-//     q, k, v arrive by TMA (3-D tiles, 128-byte swizzle, straight into the
-//     MMA operand layout); [K; Q] K^T on the raw bf16 inputs (exact
+//   * four preparation sub-pipelines (two CTAs, each with two sub-pipelines
+//     of four compute warps and one control thread) take the chunks in turn
+//     (chunk c goes to sub-pipeline c % 4) and do everything that does not
+//     need S: q, k, v arrive by TMA (3-D tiles, 128-byte swizzle, straight
+//     into the MMA operand layout); [K; Q] K^T on the raw bf16 inputs (exact
 //     products, norms applied in fp32); A and P; T by recursive doubling
 //     (fp32); W and U^T as bf16 MMAs on the raw k and v tiles with T diag(.)
-//     split into bf16 hi + lo parts (about 16 significant bits); and store
-//     fp16 -W, dec K^, gamma Q^, U^T 2^-e_u and P (72 KB) straight from
-//     registers into a slot of a per-item ring in the workspace (L2), then
-//     publish the slot with a release flag;
-//   * one chain CTA (16 warps) keeps S in registers (fp32, 32 values per
-//     thread) and per chunk runs two dependent MMA batches from shared
-//     memory: Delta^T = S^T (-W)^T (+ U^T in fp32), then S^T += Delta^T K~
-//     (K~ = dec K^), with Y = gamma Q^ S + P Delta queued behind them; the
-//     RMSNorm x sigmoid(g) epilogue of chunk c runs during chunk c + 1's MMA
-//     windows.  The fp16 copies of S and Delta carry a per-chunk power-of-two
-//     exponent e from max|V| + 12 max|S| (|Delta| <= |v| + |S| ||k^||_1).
+//     split into bf16 hi + lo parts (about 16 significant bits).  fp16 -W,
+//     dec K^, gamma Q^, U^T 2^-e_u and P (72 KB) are staged in shared memory
+//     in the slot's layout and bulk-copied into a slot of a per-item ring in
+//     the workspace (L2); the control thread then publishes the slot with a
+//     release flag;
+//   * one chain CTA keeps S in the registers of its eight compute warps
+//     (fp32, 64 values per thread) and writes fp16 S^T 2^-e and Delta^T 2^-e
+//     into tensor memory as the A operands of the per-chunk products, whose
+//     B operands come from the slot in shared memory: [Delta^T | Y^T] =
+//     S^T [-W; gamma Q^]^T (Delta^T then gains U^T in fp32), S^T += Delta^T K~
+//     (K~ = dec K^) and Y^T += Delta^T P^T.  One thread issues the products,
+//     one thread loads the slot (in three parts, each as soon as its buffer
+//     is free) and the raw g by TMA, and two epilogue warps apply RMSNorm x
+//     (1 + w) sigmoid(g) to chunk c - 1's staged Y while chunk c runs.  The
+//     fp16 copies of S and Delta carry a per-chunk power-of-two exponent e
+//     from max|V| + 12 max|S| (|Delta| <= |v| + |S| ||k^||_1).
 //
-// All CTAs (chain + two preparation CTAs per item, 512 threads each) are one
+// All CTAs (chain + two preparation CTAs per item, 384 threads each) are one
 // cooperative launch, so they are co-resident.  Every wait is bounded; a
 // wait that runs out sets the device error word and the CTA winds down
 // without faulting.
@@ -74,8 +80,8 @@ constexpr uint32_t kDrain = 1u << 16;
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ---- a ring slot (global image) ---------------------------------------------------
-// The chain CTA bulk-loads the whole slot (MMA operands, scalars and U^T) into
-// shared memory.
+// The chain CTA bulk-loads the slot (MMA operands, scalars and U^T) into
+// shared memory, in three parts.
 constexpr uint32_t SL_WQ = 0;       // [-W; gamma Q^] fp16 [128 rows][128 d_k], SW128, 2 panels
                                     //   x 16 KB: rows 0-63 -W (token t), rows 64-127 gamma Q^
 constexpr uint32_t SL_K = 32768;    // dec K^ fp16 [64 t][128 d_k], SW128, 2 panels x 8 KB
@@ -776,9 +782,9 @@ __device__ void prep_control(const ScanParams& P, uint32_t sb, uint32_t tb, int 
 // ============================================================================
 // Chain CTA.  Compute warps 0-7: thread (warp w, lane l) owns d_v index
 // j = 32 (w % 4) + l (its TMEM lane) and the state entries S[i][j],
-// i in [64 cg, 64 cg + 64), cg = w / 4, in registers.  Control warp 8 (lane 0)
-// loads the slots and issues the MMAs.  Epilogue warps 9-10 apply RMSNorm x
-// gate to staged Y rows and store y.
+// i in [64 cg, 64 cg + 64), cg = w / 4, in registers.  MMA warp 8 (lane 0)
+// issues the products; loader warp 11 (lane 0) loads the slots and the raw g.
+// Epilogue warps 9-10 apply RMSNorm x gate to staged Y rows and store y.
 // TMEM columns: S^T 2^-e A operand 0-63 (two fp16 K elements per column),
 // Delta^T 2^-e A operand 64-95, S^T increment 128-255, and two
 // [Delta^T | Y^T] accumulators 256-383 / 384-511 (chunk c in c & 1).
@@ -1142,7 +1148,7 @@ __device__ void chain_loader(const ScanParams& P, uint32_t sb, int item, const C
 }
 
 // The chain CTA's epilogue warps: token t = thread index; per chunk, the staged
-// Y row, the gate factors from the slot, RMSNorm x gate, bf16 out.
+// Y row and the raw g row (TMA), RMSNorm x (1 + w) sigmoid(g), bf16 out.
 __device__ void chain_epilogue(const ScanParams& P, uint8_t* gb, int item, const ChainBars& B) {
   const PrefillArgs& a = P.a;
   const int seq = item / a.H_v, h = item % a.H_v;
