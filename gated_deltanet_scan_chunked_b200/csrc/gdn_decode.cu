@@ -222,12 +222,15 @@ __global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT)
 // stored to state_out after the last token and optionally snapshotted after
 // every token.  The CTAs are persistent: each takes (sequence, value head)
 // items blockIdx.x, blockIdx.x + gridDim.x, ..., and while it runs the tokens
-// of one item the state of its next item is already on its way into shared
-// memory (16-byte asynchronous copies; every thread copies exactly the
-// elements it will read, so no barrier guards that buffer).  All tokens'
-// inputs (q, k, v, g, gates) are staged in shared memory per item; per token
-// there is then a single block barrier (the cross-warp reduction, double
-// buffered by token parity), the q/k norms being computed by every warp.
+// of one item the state and the raw inputs of its next item are already on
+// their way into shared memory (16-byte asynchronous copies; every thread
+// copies exactly the state elements it will read, so no barrier guards that
+// buffer).  All tokens' inputs (q, k, v, g, gates) are staged in shared
+// memory per item, and the q/k norms and k^ . q^ of every token are taken
+// once per item (one warp per token).  Per token there is then a single
+// block barrier (the cross-warp reduction, double buffered by token parity);
+// every thread sums the partials of a = S^T k^ (its update needs them),
+// warp 0 alone those of b = S^T q^, from which it forms y and the epilogue.
 template <int DK, int DV, typename Tin>
 __global__ void __launch_bounds__(DecodeGeom<DK, DV>::NT, 2)
     gdn_decode_multi_kernel(const DecodeArgs a) {
