@@ -40,8 +40,10 @@
 // undone in the fp32 epilogue and in the final state.
 //
 // Layouts: one CTA (8 warps) per (sequence, value head) for large batches
-// (gdn_prefill_tc_kernel); for small batches a chain CTA plus preparation
-// CTAs per item (gdn_prefill_tc_pair_kernel, below).  Warps 0-3 and 4-7 reach
+// (gdn_prefill_tc_kernel); for small batches without a workspace a chain CTA
+// plus preparation CTAs per item in a cluster (gdn_prefill_tc_pair_kernel,
+// below; with a workspace the scan layout of gdn_prefill_scan.cu runs
+// instead).  Warps 0-3 and 4-7 reach
 // the same TMEM lanes (lane quarter = warp % 4) and split the columns.  One
 // thread issues the MMAs; completion is tracked with mbarriers whose waits are
 // bounded: a wait that runs out flags the device error word and the CTA
