@@ -23,7 +23,11 @@ stated at the top of ``gdn_oracle.c``:
 * the backward of all of the above (the adjoint of the error-form recurrence,
   differentiated by hand token by token in reverse order), for training.
 
-Parity pins for every function here are in ``tests/test_oracle_pins.py``.
+The pins that tie each function to the pages and to mathematics other than
+itself are in ``tests/test_oracle_pins.py`` (the recurrence, both forms, the
+epilogue), ``tests/test_oracle_conv_pins.py`` (the front end) and
+``tests/test_oracle_backward_pins.py`` (the backward); the Gated Residual
+oracle (``oracle/gr.py``) is pinned in ``tests/test_oracle_gr_pins.py``.
 """
 from __future__ import annotations
 
